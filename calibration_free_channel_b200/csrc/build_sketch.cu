@@ -1,0 +1,141 @@
+// build_sketch.cu -- offline: the rotated ternary sketch of every gate/up row.
+//
+// "KAIST: MoE Decoding Needs No Calibration Data", section "A reader that
+// needs no data at all": each expert keeps a rotated ternary sketch of its
+// gate and up weights, resident on the GPU, made from the weights alone.
+// Per row: w' = H (s . w) (unnormalised Sylvester Walsh-Hadamard, fp32, stages
+// h = 1, 2, 4, ...); Delta = 0.7 mean|w'| and alpha = mean |w'| over the kept
+// entries, both fp64 in index order (TWN, Li & Liu 2016); 2-bit codes.  The
+// index-order sums are done by one thread per row so the result equals the
+// serial definition bit for bit.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRowsPerCta = 8;
+
+// s_j = +1 if the top bit of SplitMix64 output j is 0, else -1 (Steele, Lea &
+// Flood 2014: output j = mix(seed + (j+1) * 0x9E3779B97F4A7C15)).
+__global__ void rot_sign_kernel(int d, uint64_t seed, int8_t* s) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= d) return;
+  uint64_t z = seed + (uint64_t)(j + 1) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  z ^= z >> 31;
+  s[j] = (z >> 63) ? (int8_t)-1 : (int8_t)1;
+}
+
+__global__ void __launch_bounds__(256) sketch_kernel(int E, int I, int d, const uint16_t* __restrict__ wg,
+                                                     const uint16_t* __restrict__ wu,
+                                                     const int8_t* __restrict__ sign, uint32_t* skg,
+                                                     uint32_t* sku, float* ag, float* au) {
+  extern __shared__ float v[];  // [kRowsPerCta][d]
+  __shared__ double delta[kRowsPerCta];
+  const long rows_per_mat = (long)E * I;
+  const long row0 = (long)blockIdx.x * kRowsPerCta;
+  const int nr = (int)min((long)kRowsPerCta, 2 * rows_per_mat - row0);
+  for (int idx = threadIdx.x; idx < nr * d; idx += blockDim.x) {
+    const int rr = idx / d, j = idx % d;
+    const long g = row0 + rr;
+    const uint16_t* w = g < rows_per_mat ? wg + g * d : wu + (g - rows_per_mat) * d;
+    v[rr * d + j] = (float)sign[j] * bf16f(w[j]);
+  }
+  __syncthreads();
+  for (int h = 1, lh = 0; h < d; h <<= 1, lh++) {
+    for (int p = threadIdx.x; p < nr * (d / 2); p += blockDim.x) {
+      const int rr = p / (d / 2), pp = p % (d / 2);
+      const int j = ((pp >> lh) << (lh + 1)) | (pp & (h - 1));
+      float* x = v + rr * d;
+      const float x0 = x[j], x1 = x[j + h];
+      x[j] = __fadd_rn(x0, x1);
+      x[j + h] = __fsub_rn(x0, x1);
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x < nr) {
+    const int rr = threadIdx.x;
+    const float* x = v + rr * d;
+    double sabs = 0.0;
+    for (int j = 0; j < d; j++) sabs += fabs((double)x[j]);
+    const double dl = 0.7 * (sabs / (double)d);
+    double snz = 0.0;
+    int nnz = 0;
+    for (int j = 0; j < d; j++) {
+      const double a = fabs((double)x[j]);
+      if (a > dl) {
+        snz += a;
+        nnz++;
+      }
+    }
+    delta[rr] = dl;
+    const long g = row0 + rr;
+    const float alpha = nnz ? (float)(snz / (double)nnz) : 0.0f;
+    if (g < rows_per_mat) ag[g] = alpha;
+    else au[g - rows_per_mat] = alpha;
+  }
+  __syncthreads();
+  const int words = d / 16;
+  for (int idx = threadIdx.x; idx < nr * words; idx += blockDim.x) {
+    const int rr = idx / words, m = idx % words;
+    const float* x = v + rr * d + 16 * m;
+    const double dl = delta[rr];
+    uint32_t word = 0;
+#pragma unroll
+    for (int p = 0; p < 16; p++) {
+      const float xv = x[p];
+      uint32_t code = 0;
+      if (fabs((double)xv) > dl) code = xv > 0.0f ? 1u : 3u;
+      const int sh = p < 8 ? 4 * p : 4 * (p - 8) + 2;
+      word |= code << sh;
+    }
+    const long g = row0 + rr;
+    if (g < rows_per_mat) skg[g * words + m] = word;
+    else sku[(g - rows_per_mat) * words + m] = word;
+  }
+}
+
+__global__ void rmsnorm_kernel(int d, float eps, const uint16_t* __restrict__ x, uint16_t* __restrict__ h) {
+  __shared__ float red[32];
+  const uint16_t* xb = x + (size_t)blockIdx.x * d;
+  float ss = 0.0f;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    const float t = bf16f(xb[j]);
+    ss = fmaf(t, t, ss);
+  }
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.0f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); w++) tot += red[w];
+  const float inv = 1.0f / sqrtf(tot / (float)d + eps);
+  for (int j = threadIdx.x; j < d; j += blockDim.x) h[(size_t)blockIdx.x * d + j] = f2bf16(bf16f(xb[j]) * inv);
+}
+
+}  // namespace
+
+cudaError_t launch_build_sketch(int E, int I, int d, const uint16_t* w_gate, const uint16_t* w_up,
+                                uint64_t seed, int8_t* rot_sign, uint32_t* sk_gate, uint32_t* sk_up,
+                                float* alpha_gate, float* alpha_up, cudaStream_t s) {
+  rot_sign_kernel<<<(d + 255) / 256, 256, 0, s>>>(d, seed, rot_sign);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const size_t smem = sizeof(float) * kRowsPerCta * d;
+  err = cudaFuncSetAttribute(sketch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  const long rows = 2L * E * I;
+  const long grid = (rows + kRowsPerCta - 1) / kRowsPerCta;
+  sketch_kernel<<<(unsigned)grid, 256, smem, s>>>(E, I, d, w_gate, w_up, rot_sign, sk_gate, sk_up, alpha_gate,
+                                                   alpha_up);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(int B, int d, float eps, const uint16_t* x, uint16_t* h, cudaStream_t s) {
+  rmsnorm_kernel<<<B, 256, 0, s>>>(d, eps, x, h);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,165 @@
+// common.cuh -- device helpers shared by the reader's kernels (sm_100a).
+#pragma once
+#include <cooperative_groups.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+namespace cg = cooperative_groups;
+
+constexpr int kThreads = 256;          // threads per CTA of the expert kernels
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxSlots = 16;          // row slots per warp in the copy rings
+constexpr int kMaxGroup = 8;           // tokens per work item (tokens sharing an expert)
+constexpr int kMaxRank = 128;
+constexpr int kMaxCluster = 16;
+
+// Error word bits (workspace), set by bounded waits that ran out.
+constexpr uint32_t kErrCopyTimeout = 1u;
+constexpr uint32_t kErrBadWorkItem = 2u;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+// ------------------------------------------------------------------ bf16
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float bf16f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+// fp32 -> bf16, round to nearest even (finite inputs).
+__device__ __forceinline__ uint16_t f2bf16(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7f800000u) == 0x7f800000u) return (uint16_t)((u >> 16) | ((u & 0xffff) ? 0x40 : 0));
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+// ------------------------------------------------------------ exp / SiLU
+// exp_r: Cody & Waite reduction t = n ln2 + r (ln 2 split into a
+// 16-significant-bit head and an fp32 tail), degree-7 Taylor polynomial of
+// exp(r) in Horner form with correctly rounded FMAs, exact scale by 2^n.
+// Input clamped to [-87, 88] so the result is a normal float.  Every step is
+// a single correctly rounded operation, so the host reference computes the
+// same bits.
+__device__ __forceinline__ float exp_r(float t) {
+  const float kLog2e = 0x1.715476p+0f;
+  const float kLn2Hi = 0x1.62e4p-1f;
+  const float kLn2Lo = 0x1.7f7d1cp-20f;
+  t = fminf(fmaxf(t, -87.0f), 88.0f);
+  const float n = rintf(__fmul_rn(t, kLog2e));
+  float r = __fmaf_rn(-n, kLn2Hi, t);
+  r = __fmaf_rn(-n, kLn2Lo, r);
+  float p = 0x1.a01a02p-13f;             // 1/7!
+  p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);  // 1/6!
+  p = __fmaf_rn(p, r, 0x1.111112p-7f);   // 1/5!
+  p = __fmaf_rn(p, r, 0x1.555556p-5f);   // 1/4!
+  p = __fmaf_rn(p, r, 0x1.555556p-3f);   // 1/3!
+  p = __fmaf_rn(p, r, 0.5f);
+  p = __fmaf_rn(p, r, 1.0f);
+  p = __fmaf_rn(p, r, 1.0f);
+  const float two_n = __uint_as_float((uint32_t)((int)n + 127) << 23);
+  return __fmul_rn(p, two_n);
+}
+
+__device__ __forceinline__ float silu_r(float t) {
+  return __fdiv_rn(t, __fadd_rn(1.0f, exp_r(-t)));
+}
+
+// ------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait on an mbarrier phase.  Returns false (and sets *err) if the
+// phase did not complete within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      atomicOr(err, kErrCopyTimeout);
+      return false;
+    }
+  }
+}
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------- reductions
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Ternary-sketch dot of one packed row word with 16 int8 activations.
+// Word layout: position n (< 8) at bits [4n, 4n+1], position 8+n at bits
+// [4n+2, 4n+3]; codes 00 = 0, 01 = +1, 11 = -1.  A nibble's code selects a
+// byte of kTritLut = {0x00, 0x01, 0x00, 0xff} (byte_perm), giving the trits
+// as signed bytes; dp4a multiplies them with the activations exactly.
+__device__ __forceinline__ int trit_dot16(uint32_t w, uint4 q, int acc) {
+  const uint32_t kTritLut = 0xff000100u;
+  const uint32_t lo = w & 0x33333333u;
+  const uint32_t hi = (w >> 2) & 0x33333333u;
+  acc = __dp4a((int)__byte_perm(kTritLut, 0, lo & 0xffffu), (int)q.x, acc);
+  acc = __dp4a((int)__byte_perm(kTritLut, 0, lo >> 16), (int)q.y, acc);
+  acc = __dp4a((int)__byte_perm(kTritLut, 0, hi & 0xffffu), (int)q.z, acc);
+  acc = __dp4a((int)__byte_perm(kTritLut, 0, hi >> 16), (int)q.w, acc);
+  return acc;
+}
+
+// 8 bf16 (one uint4) times 8 bf16, accumulated in fp32.
+__device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
+  acc = fmaf(bf16lo(a.x), bf16lo(b.x), acc);
+  acc = fmaf(bf16hi(a.x), bf16hi(b.x), acc);
+  acc = fmaf(bf16lo(a.y), bf16lo(b.y), acc);
+  acc = fmaf(bf16hi(a.y), bf16hi(b.y), acc);
+  acc = fmaf(bf16lo(a.z), bf16lo(b.z), acc);
+  acc = fmaf(bf16hi(a.z), bf16hi(b.z), acc);
+  acc = fmaf(bf16lo(a.w), bf16lo(b.w), acc);
+  acc = fmaf(bf16hi(a.w), bf16hi(b.w), acc);
+  return acc;
+}
+
+}  // namespace moe

@@ -1,0 +1,83 @@
+// kernels.h -- argument blocks and launchers of the reader's kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Workspace carved out of the caller's buffer (see workspace_layout).
+struct Workspace {
+  uint32_t* err;        // [1] device error word
+  int* n_items;         // [1] number of work items this step
+  double* logits;       // [B, E]
+  int* ids;             // [B, top_e]
+  float* wts;           // [B, top_e]
+  int8_t* q;            // [B, d] int8 rotated activations
+  float* cx;            // [B] dequantisation scale
+  int* item_e;          // [max_items]
+  int* item_n;          // [max_items]
+  int* item_tok;        // [max_items, kMaxGroup]
+  int* item_slot;       // [max_items, kMaxGroup]
+  float* ye;            // [B, top_e, d] per-expert outputs (fp32)
+  unsigned* counters;   // [B, kMaxCluster] arrival counters of the combine
+  int max_items;
+};
+
+size_t workspace_layout(int B, int E, int top_e, int d, void* base, Workspace* ws);
+int max_work_items(int B, int E, int top_e, int group);
+
+struct RouteArgs {
+  int B, E, d, top_e, cs;
+  const uint16_t* x;
+  const uint16_t* w_router;
+  const float* bias;
+  const int8_t* rot_sign;
+  Workspace ws;
+  int32_t* dbg_ids;
+  float* dbg_w;
+  bool quantize;  // also rotate + quantize the tokens (sparse path)
+};
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+
+struct ExpertArgs {
+  int B, E, top_e, I, d, k, c, r;
+  int cs;            // CTAs per cluster (one cluster per work item)
+  int nmax;          // max tokens per work item this launch
+  int ring_rows;     // copy-ring row slots per warp (sparse) / rows (dense)
+  const uint16_t* x;
+  const uint16_t* w_gate;
+  const uint16_t* w_up;
+  const uint16_t* w_down;
+  const uint32_t* sk_gate;
+  const uint32_t* sk_up;
+  const float* alpha_gate;
+  const float* alpha_up;
+  const uint16_t* u_sigma;
+  const uint16_t* v;
+  const uint16_t* residual;
+  uint16_t* y;
+  Workspace ws;
+  // debug outputs (may be null)
+  int32_t* dbg_G;
+  int32_t* dbg_U;
+  float* dbg_sigma;
+  int32_t* dbg_cand;
+  int32_t* dbg_kept;
+  float* dbg_a_kept;
+  float* dbg_y_expert;
+};
+size_t reader_smem_bytes(const ExpertArgs& a, int ring_rows);
+size_t dense_smem_bytes(const ExpertArgs& a, int ring_rows);
+cudaError_t launch_reader(const ExpertArgs& a, cudaStream_t s);
+cudaError_t launch_dense(const ExpertArgs& a, cudaStream_t s);
+
+cudaError_t launch_build_sketch(int E, int I, int d, const uint16_t* w_gate, const uint16_t* w_up,
+                                uint64_t seed, int8_t* rot_sign, uint32_t* sk_gate, uint32_t* sk_up,
+                                float* alpha_gate, float* alpha_up, cudaStream_t s);
+size_t lowrank_ws_bytes(int E, int I, int d, int r);
+cudaError_t launch_build_lowrank(int E, int I, int d, int r, const uint16_t* w_down, uint16_t* u_sigma,
+                                 uint16_t* v, void* ws, cudaStream_t s);
+cudaError_t launch_rmsnorm(int B, int d, float eps, const uint16_t* x, uint16_t* h, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,243 @@
+"""Python binding of the C ABI in include/moe_reader.h.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  torch provides device memory and streams.  If the library is not
+built, importing the functions raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe_reader.so")
+
+MOE_OK, MOE_EINVAL, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT = range(5)
+_STATUS = {0: "MOE_OK", 1: "MOE_EINVAL", 2: "MOE_EUNSUPPORTED", 3: "MOE_ECUDA", 4: "MOE_ETIMEOUT"}
+
+EXPORTS = ["moe_reader_workspace_bytes", "moe_reader_build_sketch", "moe_reader_lowrank_workspace_bytes",
+           "moe_reader_build_lowrank", "moe_reader_forward", "moe_reader_forward_dense",
+           "moe_reader_forward_host", "moe_reader_rmsnorm", "moe_reader_set_expert_events",
+           "moe_reader_check_error", "moe_reader_last_error"]
+
+
+class MoeReaderLayer(C.Structure):
+    _fields_ = [("E", C.c_int32), ("I", C.c_int32), ("d", C.c_int32), ("top_e", C.c_int32), ("r", C.c_int32),
+                ("w_router", C.c_void_p), ("router_bias", C.c_void_p), ("w_gate", C.c_void_p),
+                ("w_up", C.c_void_p), ("w_down", C.c_void_p), ("rot_sign", C.c_void_p),
+                ("sk_gate", C.c_void_p), ("sk_up", C.c_void_p), ("alpha_gate", C.c_void_p),
+                ("alpha_up", C.c_void_p), ("u_sigma", C.c_void_p), ("v", C.c_void_p)]
+
+
+class MoeReaderDebug(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("ids", "weights", "dot_gate", "dot_up", "score", "cand", "kept",
+                                          "a_kept", "y_expert")]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with calibration_free_channel_b200.build.build()")
+        L = C.CDLL(LIB_PATH)
+        P, i32, sz = C.c_void_p, C.c_int, C.c_size_t
+        L.moe_reader_workspace_bytes.restype = sz
+        L.moe_reader_workspace_bytes.argtypes = [i32] * 8
+        L.moe_reader_build_sketch.argtypes = [i32, i32, i32, P, P, C.c_uint64, P, P, P, P, P, P]
+        L.moe_reader_lowrank_workspace_bytes.restype = sz
+        L.moe_reader_lowrank_workspace_bytes.argtypes = [i32] * 4
+        L.moe_reader_build_lowrank.argtypes = [i32, i32, i32, i32, P, P, P, P, sz, P]
+        L.moe_reader_forward.argtypes = [C.POINTER(MoeReaderLayer), i32, i32, i32, P, P, P,
+                                         C.POINTER(MoeReaderDebug), P, sz, P]
+        L.moe_reader_forward_dense.argtypes = [C.POINTER(MoeReaderLayer), i32, P, P, P, P, sz, P]
+        L.moe_reader_forward_host.argtypes = [C.POINTER(MoeReaderLayer), i32, i32, i32, P, P, P, P, P, sz, P]
+        L.moe_reader_rmsnorm.argtypes = [i32, i32, C.c_float, P, P, P]
+        L.moe_reader_set_expert_events.argtypes = [P, P]
+        L.moe_reader_check_error.argtypes = [P, P]
+        L.moe_reader_last_error.restype = C.c_char_p
+        L.moe_reader_last_error.argtypes = []
+        for f in EXPORTS:
+            if f != "moe_reader_workspace_bytes" and f != "moe_reader_lowrank_workspace_bytes" \
+                    and f != "moe_reader_last_error":
+                getattr(L, f).restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != MOE_OK:
+        raise MoeError(status, lib().moe_reader_last_error().decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+# ------------------------------------------------------ the C ABI, by name
+def moe_reader_workspace_bytes(B, E, top_e, I, d, k, c, r) -> int:
+    return int(lib().moe_reader_workspace_bytes(B, E, top_e, I, d, k, c, r))
+
+
+def moe_reader_lowrank_workspace_bytes(E, I, d, r) -> int:
+    return int(lib().moe_reader_lowrank_workspace_bytes(E, I, d, r))
+
+
+def moe_reader_build_sketch(E, I, d, w_gate, w_up, rot_seed, rot_sign, sk_gate, sk_up, alpha_gate, alpha_up,
+                            stream=None):
+    _check(lib().moe_reader_build_sketch(E, I, d, _ptr(w_gate), _ptr(w_up), rot_seed & ((1 << 64) - 1),
+                                         _ptr(rot_sign), _ptr(sk_gate), _ptr(sk_up), _ptr(alpha_gate),
+                                         _ptr(alpha_up), _stream(stream)))
+
+
+def moe_reader_build_lowrank(E, I, d, r, w_down, u_sigma, v, workspace, ws_bytes, stream=None):
+    _check(lib().moe_reader_build_lowrank(E, I, d, r, _ptr(w_down), _ptr(u_sigma), _ptr(v), _ptr(workspace),
+                                          ws_bytes, _stream(stream)))
+
+
+def moe_reader_forward(layer: MoeReaderLayer, B, k, c, x, residual, y, dbg, workspace, ws_bytes, stream=None):
+    _check(lib().moe_reader_forward(C.byref(layer), B, k, c, _ptr(x), _ptr(residual), _ptr(y),
+                                    C.byref(dbg) if dbg is not None else None, _ptr(workspace), ws_bytes,
+                                    _stream(stream)))
+
+
+def moe_reader_forward_dense(layer: MoeReaderLayer, B, x, residual, y, workspace, ws_bytes, stream=None):
+    _check(lib().moe_reader_forward_dense(C.byref(layer), B, _ptr(x), _ptr(residual), _ptr(y), _ptr(workspace),
+                                          ws_bytes, _stream(stream)))
+
+
+def moe_reader_forward_host(layer: MoeReaderLayer, B, k, c, x_host, x_dev, y_dev, y_host, workspace, ws_bytes,
+                            stream=None):
+    _check(lib().moe_reader_forward_host(C.byref(layer), B, k, c, _ptr(x_host), _ptr(x_dev), _ptr(y_dev),
+                                         _ptr(y_host), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def moe_reader_rmsnorm(B, d, eps, x, h, stream=None):
+    _check(lib().moe_reader_rmsnorm(B, d, eps, _ptr(x), _ptr(h), _stream(stream)))
+
+
+def moe_reader_set_expert_events(ev_before, ev_after):
+    h = lambda ev: None if ev is None else ev.cuda_event  # noqa: E731
+    _check(lib().moe_reader_set_expert_events(h(ev_before), h(ev_after)))
+
+
+def moe_reader_check_error(workspace, stream=None):
+    _check(lib().moe_reader_check_error(_ptr(workspace), _stream(stream)))
+
+
+# ----------------------------------------------------------- convenience
+class Layer:
+    """A resident MoE layer on the GPU: bf16 weights, the sketch and the
+    low-rank map, with the C struct that describes them."""
+
+    def __init__(self, weights: dict, top_e: int, device="cuda"):
+        dev = torch.device(device)
+        self.w = {k: (v.to(dev).contiguous() if v is not None else None) for k, v in weights.items()}
+        E, I, d = self.w["w_gate"].shape
+        self.E, self.I, self.d, self.top_e, self.r = E, I, d, top_e, 0
+        self.rot_sign = torch.empty(d, dtype=torch.int8, device=dev)
+        self.sk_gate = torch.empty((E, I, d // 16), dtype=torch.int32, device=dev)
+        self.sk_up = torch.empty_like(self.sk_gate)
+        self.alpha_gate = torch.empty((E, I), dtype=torch.float32, device=dev)
+        self.alpha_up = torch.empty_like(self.alpha_gate)
+        self.u_sigma = None
+        self.v = None
+        self._ws = None
+
+    def build_sketch(self, rot_seed: int, stream=None):
+        moe_reader_build_sketch(self.E, self.I, self.d, self.w["w_gate"], self.w["w_up"], rot_seed,
+                                self.rot_sign, self.sk_gate, self.sk_up, self.alpha_gate, self.alpha_up, stream)
+        return self
+
+    def build_lowrank(self, r: int, stream=None):
+        dev = self.w["w_down"].device
+        self.u_sigma = torch.empty((self.E, self.I, r), dtype=torch.bfloat16, device=dev)
+        self.v = torch.empty((self.E, self.d, r), dtype=torch.bfloat16, device=dev)
+        nb = moe_reader_lowrank_workspace_bytes(self.E, self.I, self.d, r)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        moe_reader_build_lowrank(self.E, self.I, self.d, r, self.w["w_down"], self.u_sigma, self.v, ws, nb, stream)
+        torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+        del ws
+        self.r = r
+        return self
+
+    def set_lowrank(self, u_sigma, v):
+        """Use given factors ([E, I, r], [E, d, r] bf16) or none (None)."""
+        if u_sigma is None:
+            self.u_sigma = self.v = None
+            self.r = 0
+        else:
+            dev = self.w["w_down"].device
+            self.u_sigma = u_sigma.to(dev).contiguous()
+            self.v = v.to(dev).contiguous()
+            self.r = int(u_sigma.shape[-1])
+        return self
+
+    def struct(self, r: int | None = None) -> MoeReaderLayer:
+        rr = self.r if r is None else r
+        return MoeReaderLayer(self.E, self.I, self.d, self.top_e, rr, _ptr(self.w["w_router"]),
+                              _ptr(self.w.get("router_bias")), _ptr(self.w["w_gate"]), _ptr(self.w["w_up"]),
+                              _ptr(self.w["w_down"]), _ptr(self.rot_sign), _ptr(self.sk_gate), _ptr(self.sk_up),
+                              _ptr(self.alpha_gate), _ptr(self.alpha_up),
+                              _ptr(self.u_sigma) if rr else None, _ptr(self.v) if rr else None)
+
+    def workspace(self, B: int):
+        nb = moe_reader_workspace_bytes(B, self.E, self.top_e, self.I, self.d, 1, 1, self.r)
+        if self._ws is None or self._ws.numel() < nb:
+            self._ws = torch.zeros(nb, dtype=torch.uint8, device=self.w["w_gate"].device)
+        return self._ws
+
+    def forward(self, x, k: int, c: int, residual=None, debug: bool = False, r: int | None = None, stream=None,
+                out=None):
+        B = x.shape[0]
+        ws = self.workspace(B)
+        y = out if out is not None else torch.empty_like(x)
+        dbg = None
+        dbg_t = None
+        if debug:
+            dev = x.device
+            P = (B, self.top_e)
+            dbg_t = dict(ids=torch.empty(P, dtype=torch.int32, device=dev),
+                         weights=torch.empty(P, dtype=torch.float32, device=dev),
+                         dot_gate=torch.empty(P + (self.I,), dtype=torch.int32, device=dev),
+                         dot_up=torch.empty(P + (self.I,), dtype=torch.int32, device=dev),
+                         score=torch.empty(P + (self.I,), dtype=torch.float32, device=dev),
+                         cand=torch.empty(P + (c,), dtype=torch.int32, device=dev),
+                         kept=torch.empty(P + (k,), dtype=torch.int32, device=dev),
+                         a_kept=torch.empty(P + (k,), dtype=torch.float32, device=dev),
+                         y_expert=torch.empty(P + (self.d,), dtype=torch.float32, device=dev))
+            dbg = MoeReaderDebug(*[_ptr(dbg_t[n]) for n, _ in MoeReaderDebug._fields_])
+        moe_reader_forward(self.struct(r), B, k, c, x, residual, y, dbg, ws, ws.numel(), stream)
+        return (y, dbg_t) if debug else y
+
+    def forward_dense(self, x, residual=None, stream=None, out=None):
+        B = x.shape[0]
+        ws = self.workspace(B)
+        y = out if out is not None else torch.empty_like(x)
+        moe_reader_forward_dense(self.struct(0), B, x, residual, y, ws, ws.numel(), stream)
+        return y
+
+    def check(self, stream=None):
+        if self._ws is not None:
+            moe_reader_check_error(self._ws, stream)

@@ -1,0 +1,185 @@
+/*
+ * moe_reader.h -- C ABI of the calibration-free sparse routed-expert reader
+ * for MoE decoding at small batch, on NVIDIA B200 (sm_100a).
+ *
+ * The method ("Channel Selection for Mixture-of-Experts Decoding Needs No
+ * Calibration Data", arXiv:2610.37386, abstract; "KAIST: MoE Decoding Needs
+ * No Calibration Data", section "A reader that needs no data at all"): for
+ * every (token, routed expert) pair the reader
+ *   1. screens the expert's gate/up channels with a resident ternary sketch
+ *      of the rotated gate/up weights, built from the weights alone;
+ *   2. computes the surviving candidates exactly from the native BF16
+ *      gate/up rows;
+ *   3. keeps the token's top-k channels by |silu(g) * u| (no calibrated
+ *      threshold: abstract, "top-k keeps each token's k highest-scoring
+ *      channels");
+ *   4. reads only those k rows of the down projection;
+ *   5. adds back the skipped channels through a low-rank map of the down
+ *      projection.
+ *
+ * Conventions for every entry point.
+ *  - Tensors are dense row-major.  bf16 values are passed as uint16_t bit
+ *    patterns.  Every pointer is a DEVICE pointer unless its name ends in
+ *    _host, and must be 16-byte aligned.  The caller owns all memory; the
+ *    library never allocates or frees device memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls only enqueue work; they never synchronize, except
+ *    moe_reader_check_error.
+ *  - Arguments are validated on the host before anything is enqueued.  On
+ *    MOE_EINVAL / MOE_EUNSUPPORTED nothing was launched.  MOE_ECUDA means a
+ *    launch failed.  moe_reader_last_error() describes the last non-OK
+ *    status of the calling thread.
+ *  - Device-side waits are bounded; a wait that runs out records an error
+ *    word in the workspace (read with moe_reader_check_error) instead of
+ *    hanging the GPU.
+ *
+ * Limits of this build: 128 <= d <= 4096 and d a power of two;
+ * 16 <= I <= 2048; 1 <= k <= c <= I; r in {0, 8, 16, ..., 128} and r <= I;
+ * 1 <= top_e <= min(E, 16); E <= 1024; 1 <= B <= 256.
+ */
+#ifndef MOE_READER_H
+#define MOE_READER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_EINVAL = 1,       /* bad argument (null, misaligned, out of range)      */
+  MOE_EUNSUPPORTED = 2, /* valid shape outside this build's compiled limits   */
+  MOE_ECUDA = 3,        /* a CUDA launch or query failed                      */
+  MOE_ETIMEOUT = 4      /* a bounded device wait ran out (moe_reader_check_error) */
+} moe_status;
+
+/* One resident MoE layer: the weights and what the offline builders made
+ * from them.  Per expert e, W_gate[e] and W_up[e] are [I, d] (row i =
+ * channel i) and W_down[e] is stored channel-major, [I, d] (row i = the
+ * output weights of channel i), so "read only the kept rows" reads whole
+ * rows. */
+typedef struct {
+  int32_t E, I, d, top_e, r;
+  const uint16_t* w_router;    /* [E, d] bf16                                    */
+  const float* router_bias;    /* [E] fp32, or NULL (added to the logits)        */
+  const uint16_t* w_gate;      /* [E, I, d] bf16                                 */
+  const uint16_t* w_up;        /* [E, I, d] bf16                                 */
+  const uint16_t* w_down;      /* [E, I, d] bf16, channel-major                  */
+  const int8_t* rot_sign;      /* [d] +-1: the random signs of the rotation      */
+  const uint32_t* sk_gate;     /* [E, I, d/16] 2-bit ternary sketch of W_gate     */
+  const uint32_t* sk_up;       /* [E, I, d/16] 2-bit ternary sketch of W_up       */
+  const float* alpha_gate;     /* [E, I] per-row sketch scale                    */
+  const float* alpha_up;       /* [E, I]                                         */
+  const uint16_t* u_sigma;     /* [E, I, r] bf16 = U_r Sigma_r of W_down, or NULL */
+  const uint16_t* v;           /* [E, d, r] bf16 = V_r of W_down, or NULL         */
+} moe_reader_layer;
+
+/* Optional per-stage outputs of moe_reader_forward (each pointer may be
+ * NULL; (b, s) = token b, routing slot s, slot 0 the highest logit). */
+typedef struct {
+  int32_t* ids;      /* [B, top_e] routed expert ids                             */
+  float* weights;    /* [B, top_e] routing weights                               */
+  int32_t* dot_gate; /* [B, top_e, I] exact integer sketch dots T^g . q          */
+  int32_t* dot_up;   /* [B, top_e, I]                                            */
+  float* score;      /* [B, top_e, I] screening score sigma                      */
+  int32_t* cand;     /* [B, top_e, c] candidate channels, ascending              */
+  int32_t* kept;     /* [B, top_e, k] kept channels, ascending                   */
+  float* a_kept;     /* [B, top_e, k] exact silu(g)*u of the kept channels        */
+  float* y_expert;   /* [B, top_e, d] fp32 expert output before the combine      */
+} moe_reader_debug;
+
+/* Bytes of device workspace moe_reader_forward / moe_reader_forward_dense
+ * need for this shape (16-byte aligned base).  Contents need no
+ * initialisation; a workspace must not be shared by calls that may run
+ * concurrently. */
+size_t moe_reader_workspace_bytes(int B, int E, int top_e, int I, int d, int k, int c, int r);
+
+/* Offline: the rotated ternary sketch of every gate and up row ("A reader
+ * that needs no data at all": a rotated ternary sketch of the gate/up
+ * weights, resident on the GPU, built from the weights alone).
+ *   rot_sign[j] = +1 if the top bit of output j of SplitMix64(rot_seed) is 0,
+ *                 else -1 (Steele, Lea & Flood 2014);
+ *   w' = H (rot_sign . w), H the unnormalised Sylvester Walsh-Hadamard
+ *        transform (fp32, stages h = 1, 2, 4, ...);
+ *   Delta = 0.7 * mean |w'| (fp64, index order); T_j = sign(w'_j) if
+ *   |w'_j| > Delta else 0; alpha = mean |w'_j| over T_j != 0 (fp64, index
+ *   order; 0 if none), stored fp32 (TWN, Li & Liu 2016).
+ * Packing: 16 trits per uint32; word m holds positions 16m..16m+15;
+ * position 16m+n (n < 8) at bits [4n, 4n+1], position 16m+8+n at bits
+ * [4n+2, 4n+3]; codes 00 = 0, 01 = +1, 11 = -1.
+ * Outputs are bit-identical to the reference definition above. */
+moe_status moe_reader_build_sketch(int E, int I, int d, const uint16_t* w_gate, const uint16_t* w_up,
+                                   uint64_t rot_seed, int8_t* rot_sign, uint32_t* sk_gate,
+                                   uint32_t* sk_up, float* alpha_gate, float* alpha_up, void* stream);
+
+/* Offline: the low-rank map of the down projections ("A reader that needs
+ * no data at all": skipped channels are recovered through a low-rank map of
+ * the down projections).  Per expert, the rank-r truncated SVD
+ * W_down[e] = U S V^T gives u_sigma = U[:, :r] S[:r] ([I, r]) and
+ * v = V[:, :r] ([d, r]); in each column the entry of v with the largest
+ * magnitude is positive.  Computed by subspace iteration on W W^T with a
+ * Rayleigh-Ritz step; factors are rounded to bf16.
+ * Needs moe_reader_lowrank_workspace_bytes(E, I, d, r) bytes of workspace. */
+size_t moe_reader_lowrank_workspace_bytes(int E, int I, int d, int r);
+moe_status moe_reader_build_lowrank(int E, int I, int d, int r, const uint16_t* w_down,
+                                    uint16_t* u_sigma, uint16_t* v, void* workspace,
+                                    size_t ws_bytes, void* stream);
+
+/* One MoE block step over B tokens x [B, d] (bf16) -> y [B, d] (bf16).
+ *   routing: logit_e = W_router[e] . x (+ bias_e), products exact, fp64 sums;
+ *     top-`top_e` experts (ties: lower id), weights = softmax over the chosen
+ *     logits (the abstract's "routed experts");
+ *   per (token, expert): the reader steps 1-5 above with c candidates and
+ *     k kept channels; the screening score of channel i is
+ *     |silu(ghat_i) uhat_i| with ghat_i = ((float)G_i alpha_i) c_x,
+ *     G_i = T_i . q exact, q = int8 quantisation of H (rot_sign . x),
+ *     c_x = max|H (rot_sign . x)| / (127 d); candidates and kept sets break
+ *     ties toward the lower channel;
+ *   recovery (r > 0): + V z with z = sum over skipped channels of
+ *     silu(ghat_i) uhat_i u_sigma[i, :];
+ *   combine: y_b = sum over slots of w * y_e in fp32, rounded once to bf16;
+ *     with `residual` (may be NULL) y_b += residual_b before the rounding.
+ * Tokens routed to the same expert share its reads (one sketch read, the
+ * union of their candidate and kept rows).  dbg may be NULL. */
+moe_status moe_reader_forward(const moe_reader_layer* layer, int B, int k, int c,
+                              const uint16_t* x, const uint16_t* residual, uint16_t* y,
+                              const moe_reader_debug* dbg, void* workspace, size_t ws_bytes,
+                              void* stream);
+
+/* The dense all-channel MoE block on the same layer (same routing and
+ * combine; every channel of every routed expert is read): the baseline the
+ * reader is measured against. */
+moe_status moe_reader_forward_dense(const moe_reader_layer* layer, int B, const uint16_t* x,
+                                    const uint16_t* residual, uint16_t* y, void* workspace,
+                                    size_t ws_bytes, void* stream);
+
+/* moe_reader_forward with HOST input and output: copies x_host (pinned,
+ * [B, d] bf16) into x_dev, runs the step, copies y_dev back into y_host
+ * (pinned), all enqueued on `stream`.  The caller synchronizes. */
+moe_status moe_reader_forward_host(const moe_reader_layer* layer, int B, int k, int c,
+                                   const uint16_t* x_host, uint16_t* x_dev, uint16_t* y_dev,
+                                   uint16_t* y_host, void* workspace, size_t ws_bytes, void* stream);
+
+/* Between stacked layers: h = bf16(x / sqrt(mean(x^2) + eps)) per token,
+ * no learned gain (fp32). */
+moe_status moe_reader_rmsnorm(int B, int d, float eps, const uint16_t* x, uint16_t* h, void* stream);
+
+/* Optional timing hooks: when set (non-NULL cudaEvent_t handles), the
+ * forward calls of this thread record events[0] before the expert kernel and
+ * events[1] after it on `stream`.  Pass NULL to clear. */
+moe_status moe_reader_set_expert_events(void* ev_before, void* ev_after);
+
+/* Synchronizes `stream`, reads and clears the workspace's device error word.
+ * Returns MOE_OK, or MOE_ETIMEOUT if a bounded wait ran out since the last
+ * check. */
+moe_status moe_reader_check_error(void* workspace, void* stream);
+
+/* Message for the last non-OK status returned on this thread. */
+const char* moe_reader_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_READER_H */

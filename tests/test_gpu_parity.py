@@ -1,0 +1,210 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on
+the same seeded inputs, on the tiny block, the Qwen3-30B-A3B-shaped layer at
+batch 1, the budget and batch sweeps, and edge cases."""
+import numpy as np
+import pytest
+import torch
+
+from calibration_free_channel_b200 import moe_reader as M
+from calibration_free_channel_b200 import synth
+from oracle import oracle as O
+from tests.gpu_helpers import MAX_ABS, REL_L2, OracleCache, check_pair
+
+pytestmark = pytest.mark.gpu
+
+QWEN = synth.QWEN3_30B_A3B
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    W = synth.layer_weights(synth.TINY, seed=0)
+    seed = synth.rot_seed(0)
+    layer = M.Layer(W, top_e=2).build_sketch(seed)
+    return W, layer, OracleCache(W, seed, 8)
+
+
+@pytest.fixture(scope="module")
+def qwen():
+    W = synth.layer_weights(QWEN, seed=0)
+    seed = synth.rot_seed(0)
+    layer = M.Layer(W, top_e=8).build_sketch(seed)
+    return W, layer, OracleCache(W, seed, 32)
+
+
+@pytest.fixture(scope="module")
+def qwen_skewed():
+    W = synth.layer_weights(QWEN, seed=1, bias=True)
+    seed = synth.rot_seed(1)
+    layer = M.Layer(W, top_e=8).build_sketch(seed)
+    return W, layer, OracleCache(W, seed, 32)
+
+
+# ------------------------------------------------------------------ sketch
+def _check_sketch(layer, oc):
+    s, skg, sku, ag, au = oc.sk
+    assert np.array_equal(layer.rot_sign.cpu().numpy(), s)
+    assert np.array_equal(layer.sk_gate.cpu().numpy().view(np.uint32), skg)
+    assert np.array_equal(layer.sk_up.cpu().numpy().view(np.uint32), sku)
+    assert np.array_equal(layer.alpha_gate.cpu().numpy().view(np.uint32), ag.view(np.uint32))
+    assert np.array_equal(layer.alpha_up.cpu().numpy().view(np.uint32), au.view(np.uint32))
+
+
+def test_build_sketch_bit_exact_tiny(tiny):
+    _, layer, oc = tiny
+    _check_sketch(layer, oc)
+
+
+def test_build_sketch_bit_exact_qwen_layer(qwen):
+    _, layer, oc = qwen
+    _check_sketch(layer, oc)
+
+
+# ---------------------------------------------------------------- forward
+@pytest.mark.parametrize("B", [1, 2, 5])
+def test_forward_tiny(tiny, B):
+    W, layer, oc = tiny
+    for seed in range(3):
+        x = synth.tokens(256, B, seed=seed)
+        check_pair(layer, oc, x, k=24, c=48, top_e=2)
+
+
+@pytest.mark.parametrize("k,c,r", [(1, 1, 8), (24, 24, 8), (24, 128, 8), (128, 128, 0), (5, 17, 0), (64, 100, 8)])
+def test_forward_tiny_budgets(tiny, k, c, r):
+    W, layer, _ = tiny
+    oc = OracleCache(W, synth.rot_seed(0), r)
+    x = synth.tokens(256, 3, seed=11)
+    if r == 0:
+        layer.set_lowrank(None, None)
+    check_pair(layer, oc, x, k=k, c=c, top_e=2)
+
+
+def test_forward_qwen_layer_batch1_steps(qwen):
+    """The Qwen3-30B-A3B-shaped layer at batch 1 over decode steps with
+    tokens from seeds 0..7 (k = 136, c = 272, r = 32)."""
+    W, layer, oc = qwen
+    for s in range(8):
+        x = synth.tokens(2048, 1, seed=s)
+        check_pair(layer, oc, x, k=136, c=272, top_e=8)
+
+
+@pytest.mark.parametrize("B,k", [(4, 100), (16, 136), (8, 100)])
+def test_forward_qwen_budget_sweep(qwen, B, k):
+    W, layer, oc = qwen
+    x = synth.tokens(2048, B, seed=100 + B)
+    check_pair(layer, oc, x, k=k, c=2 * k, top_e=8)
+
+
+@pytest.mark.parametrize("B", [32, 64])
+def test_forward_qwen_skewed_batch(qwen_skewed, B):
+    """Skewed router prior: many tokens share experts, so one expert's
+    tokens span several work items of up to 8 tokens."""
+    W, layer, oc = qwen_skewed
+    x = synth.tokens(2048, B, seed=200 + B)
+    _, ids, _ = O.route(x, W["w_router"], W["router_bias"], 8)
+    assert np.bincount(ids.ravel()).max() > 8
+    check_pair(layer, oc, x, k=136, c=272, top_e=8)
+
+
+def test_forward_with_own_lowrank_build(qwen):
+    """End to end with the GPU's own sketch and low-rank map against the
+    oracle's own (both built from the weights alone)."""
+    W, layer, oc = qwen
+    layer.build_lowrank(32)
+    x = synth.tokens(2048, 2, seed=300)
+    check_pair(layer, oc, x, k=136, c=272, top_e=8, use_oracle_factors=False)
+
+
+def test_identical_tokens_share_work_items(tiny):
+    W, layer, oc = tiny
+    x1 = synth.tokens(256, 1, seed=5)
+    x = x1.repeat(11, 1)  # 11 tokens on the same 2 experts: items of 8 + 3
+    check_pair(layer, oc, x, k=24, c=48, top_e=2)
+
+
+def test_forward_host_matches_forward(qwen):
+    W, layer, oc = qwen
+    x = synth.tokens(2048, 1, seed=7)
+    y_dev = layer.forward(x.cuda(), k=136, c=272)
+    xh = x.pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    xd = torch.empty_like(x, device="cuda")
+    yd = torch.empty_like(x, device="cuda")
+    ws = layer.workspace(1)
+    M.moe_reader_forward_host(layer.struct(), 1, 136, 272, xh, xd, yd, yh, ws, ws.numel())
+    torch.cuda.synchronize()
+    assert torch.equal(yh, y_dev.cpu())
+
+
+# ------------------------------------------------------------------ dense
+@pytest.mark.parametrize("B", [1, 9])
+def test_dense_tiny(tiny, B):
+    W, layer, _ = tiny
+    x = synth.tokens(256, B, seed=20 + B)
+    y = layer.forward_dense(x.cuda())
+    _, y64 = O.forward_dense(x, W, top_e=2)
+    yg = y.float().cpu().numpy()
+    assert np.abs(yg - y64).max() <= MAX_ABS
+    assert np.linalg.norm(yg - y64) / np.linalg.norm(y64) <= REL_L2
+
+
+def test_dense_qwen_layer(qwen):
+    W, layer, _ = qwen
+    x = synth.tokens(2048, 2, seed=21)
+    y = layer.forward_dense(x.cuda())
+    _, y64 = O.forward_dense(x, W, top_e=8)
+    yg = y.float().cpu().numpy()
+    assert np.abs(yg - y64).max() <= MAX_ABS
+    assert np.linalg.norm(yg - y64) / np.linalg.norm(y64) <= REL_L2
+
+
+def test_all_channels_kept_equals_dense_on_gpu(qwen):
+    """k = c = I with recovery off is the dense block (property, any size)."""
+    W, layer, _ = qwen
+    x = synth.tokens(2048, 3, seed=22).cuda()
+    ys = layer.forward(x, k=768, c=768, r=0).float()
+    yd = layer.forward_dense(x).float()
+    assert (ys - yd).abs().max().item() <= 2e-2
+    assert ((ys - yd).norm() / yd.norm()).item() <= 1e-2
+
+
+# ---------------------------------------------------------------- lowrank
+def _lowrank_check(W, layer, r, experts):
+    us = layer.u_sigma.float().cpu().numpy()
+    vv = layer.v.float().cpu().numpy()
+    wd = synth.bf16_bits(W["w_down"])
+    for e in experts:
+        ubar, V, S = O.lowrank_f64(wd[e], r)
+        want = ubar @ V.T
+        got = us[e].astype(np.float64) @ vv[e].astype(np.float64).T
+        assert np.linalg.norm(got - want) <= 1e-2 * np.linalg.norm(want)
+        for p in range(r):
+            j = np.argmax(np.abs(vv[e][:, p]))
+            assert vv[e][j, p] > 0
+        # residual close to the optimum (Eckart-Young)
+        Wf = O.bf16_to_f64(wd[e])
+        best = np.sqrt(max(np.sum(S[r:] ** 2), 0))
+        assert np.linalg.norm(Wf - got) <= best * 1.01 + 1e-6 * np.linalg.norm(Wf)
+
+
+def test_build_lowrank_tiny(tiny):
+    W, layer, _ = tiny
+    layer.build_lowrank(8)
+    _lowrank_check(W, layer, 8, range(8))
+
+
+def test_build_lowrank_qwen_layer(qwen):
+    W, layer, _ = qwen
+    layer.build_lowrank(32)
+    _lowrank_check(W, layer, 32, [0, 17, 64, 127])
+
+
+# ---------------------------------------------------------------- rmsnorm
+def test_rmsnorm_matches_oracle():
+    x = synth.tokens(2048, 5, seed=3)
+    x = (x.float() * 3.7).to(torch.bfloat16)
+    h = torch.empty_like(x, device="cuda")
+    M.moe_reader_rmsnorm(5, 2048, 1e-6, x.cuda(), h)
+    torch.cuda.synchronize()
+    ho = O.rmsnorm(x)
+    diff = np.abs(O.bf16_to_f64(h.cpu()) - O.bf16_to_f64(ho))
+    assert diff.max() <= 2 ** -7 * np.abs(O.bf16_to_f64(ho)).max()
