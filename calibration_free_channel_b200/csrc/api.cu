@@ -273,6 +273,32 @@ moe_status moe_reader_check_error(void* workspace, void* stream) {
   return fail(MOE_ETIMEOUT, "device error word 0x%x (1: a bounded copy wait ran out; 2: bad work item)", word);
 }
 
+moe_status moe_reader_set_cluster_size(int cs) {
+  REQUIRE(cs == 0 || cs == 4 || cs == 8 || cs == 16, "cluster size %d: use 0 (automatic), 4, 8 or 16", cs);
+  moe::set_forced_cluster_size(cs);
+  return MOE_OK;
+}
+
+moe_status moe_reader_launch_plan(int dense, int B, int E, int top_e, int I, int d, int r, int32_t* out4) {
+  moe_status st = check_shape(B, E, top_e, I, d);
+  if (st != MOE_OK) return st;
+  REQUIRE(out4 != nullptr, "out4 is NULL");
+  moe::ExpertArgs a = {};
+  a.B = B;
+  a.E = E;
+  a.top_e = top_e;
+  a.I = I;
+  a.d = d;
+  a.r = dense ? 0 : r;
+  a.nmax = B < moe::kMaxGroup ? B : moe::kMaxGroup;
+  a.ws.max_items = moe::max_work_items(B, E, top_e, moe::kMaxGroup);
+  int o[4];
+  cudaError_t e = moe::query_plan(a, dense != 0, o);
+  if (e != cudaSuccess) return cuda_fail(e, "launch plan");
+  for (int i = 0; i < 4; i++) out4[i] = o[i];
+  return MOE_OK;
+}
+
 const char* moe_reader_last_error(void) { return g_err.c_str(); }
 
 }  // extern "C"

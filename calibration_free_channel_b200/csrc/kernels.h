@@ -71,6 +71,8 @@ size_t reader_smem_bytes(const ExpertArgs& a, int ring_rows);
 size_t dense_smem_bytes(const ExpertArgs& a, int ring_rows);
 cudaError_t launch_reader(const ExpertArgs& a, cudaStream_t s);
 cudaError_t launch_dense(const ExpertArgs& a, cudaStream_t s);
+void set_forced_cluster_size(int cs);
+cudaError_t query_plan(const ExpertArgs& a, bool dense, int out[4]);
 
 cudaError_t launch_build_sketch(int E, int I, int d, const uint16_t* w_gate, const uint16_t* w_up,
                                 uint64_t seed, int8_t* rot_sign, uint32_t* sk_gate, uint32_t* sk_up,

@@ -936,21 +936,27 @@ int pick_ring_rows(const ExpertArgs& a, bool dense, int smem_max) {
 }
 
 struct LaunchPlan {
-  int dev, dense, nmax, I, d, r;
-  int cs, ring_rows, smem;
+  int dev, dense, nmax, I, d, r, items, forced;
+  int cs, ring_rows, smem, max_clusters;
 };
 
-// Picks the cluster size (16 when a GPC can hold such a cluster with this
-// shared-memory footprint, else 8) and the ring depth; cached per shape.
+int g_forced_cs = 0;  // 0: automatic
+
+// Cluster size: among 16, 8, 4 (those that fit this shape), the one that
+// keeps the most SMs busy on this launch, min(items, co-resident clusters)
+// * cs, ties to the larger cluster.  Ring depth: the deepest that fits.
+// Cached per shape and device.
 cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
-  thread_local LaunchPlan cache[8];
-  thread_local int ncache = 0;
+  thread_local LaunchPlan cache[16];
+  thread_local int ncache = 0, next = 0;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
+  const int items = a.ws.max_items;
   for (int i = 0; i < ncache; i++) {
     const LaunchPlan& c = cache[i];
-    if (c.dev == dev && c.dense == (int)dense && c.nmax == a.nmax && c.I == a.I && c.d == a.d && c.r == a.r) {
+    if (c.dev == dev && c.dense == (int)dense && c.nmax == a.nmax && c.I == a.I && c.d == a.d && c.r == a.r &&
+        c.items == items && c.forced == g_forced_cs) {
       *out = c;
       return cudaSuccess;
     }
@@ -961,8 +967,10 @@ cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
   auto fn = dense ? dense_kernel : reader_kernel;
   err = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (err != cudaSuccess) return err;
-  LaunchPlan p = {dev, (int)dense, a.nmax, a.I, a.d, a.r, 0, 0, 0};
-  for (int cs = 16; cs >= 8; cs /= 2) {
+  LaunchPlan p = {dev, (int)dense, a.nmax, a.I, a.d, a.r, items, g_forced_cs, 0, 0, 0, 0};
+  long best_busy = -1;
+  for (int cs = 16; cs >= 4; cs /= 2) {
+    if (g_forced_cs && cs != g_forced_cs) continue;
     if (a.d / cs > 256 || a.d / cs < 8 || a.I < cs) continue;
     ExpertArgs t = a;
     t.cs = cs;
@@ -988,16 +996,19 @@ cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
       cudaGetLastError();
       continue;
     }
-    if (nclusters >= 1) {
+    if (nclusters < 1) continue;
+    const long busy = (long)(items < nclusters ? items : nclusters) * cs;
+    if (busy > best_busy) {
+      best_busy = busy;
       p.cs = cs;
       p.ring_rows = rr;
       p.smem = smem;
-      break;
+      p.max_clusters = nclusters;
     }
   }
   if (p.cs == 0) return cudaErrorInvalidConfiguration;
-  if (ncache < 8) cache[ncache++] = p;
-  else cache[0] = p;
+  if (ncache < 16) cache[ncache++] = p;
+  else cache[next++ % 16] = p;
   *out = p;
   return cudaSuccess;
 }
@@ -1040,6 +1051,17 @@ size_t dense_smem_bytes(const ExpertArgs& a, int ring_rows) {
   return make_layout(a.nmax, a.I, a.d, a.r, a.cs, ring_rows, true).total;
 }
 cudaError_t launch_reader(const ExpertArgs& a, cudaStream_t s) { return launch_expert(a, s, false); }
+void set_forced_cluster_size(int cs) { g_forced_cs = cs; }
+cudaError_t query_plan(const ExpertArgs& a, bool dense, int out[4]) {
+  LaunchPlan p;
+  cudaError_t e = plan_launch(a, dense, &p);
+  if (e != cudaSuccess) return e;
+  out[0] = p.cs;
+  out[1] = p.ring_rows;
+  out[2] = p.smem;
+  out[3] = p.max_clusters;
+  return cudaSuccess;
+}
 cudaError_t launch_dense(const ExpertArgs& a, cudaStream_t s) { return launch_expert(a, s, true); }
 
 }  // namespace moe

@@ -20,7 +20,8 @@ _STATUS = {0: "MOE_OK", 1: "MOE_EINVAL", 2: "MOE_EUNSUPPORTED", 3: "MOE_ECUDA", 
 EXPORTS = ["moe_reader_workspace_bytes", "moe_reader_build_sketch", "moe_reader_lowrank_workspace_bytes",
            "moe_reader_build_lowrank", "moe_reader_forward", "moe_reader_forward_dense",
            "moe_reader_forward_host", "moe_reader_rmsnorm", "moe_reader_set_expert_events",
-           "moe_reader_check_error", "moe_reader_last_error"]
+           "moe_reader_check_error", "moe_reader_set_cluster_size", "moe_reader_launch_plan",
+           "moe_reader_last_error"]
 
 
 class MoeReaderLayer(C.Structure):
@@ -66,6 +67,8 @@ def lib():
         L.moe_reader_rmsnorm.argtypes = [i32, i32, C.c_float, P, P, P]
         L.moe_reader_set_expert_events.argtypes = [P, P]
         L.moe_reader_check_error.argtypes = [P, P]
+        L.moe_reader_set_cluster_size.argtypes = [i32]
+        L.moe_reader_launch_plan.argtypes = [i32] * 7 + [P]
         L.moe_reader_last_error.restype = C.c_char_p
         L.moe_reader_last_error.argtypes = []
         for f in EXPORTS:
@@ -144,6 +147,16 @@ def moe_reader_set_expert_events(ev_before, ev_after):
 
 def moe_reader_check_error(workspace, stream=None):
     _check(lib().moe_reader_check_error(_ptr(workspace), _stream(stream)))
+
+
+def moe_reader_set_cluster_size(cs: int):
+    _check(lib().moe_reader_set_cluster_size(cs))
+
+
+def moe_reader_launch_plan(dense: bool, B, E, top_e, I, d, r) -> dict:
+    out = (C.c_int32 * 4)()
+    _check(lib().moe_reader_launch_plan(int(dense), B, E, top_e, I, d, r, C.cast(out, C.c_void_p)))
+    return dict(cluster_size=out[0], ring_rows=out[1], smem_bytes=out[2], max_active_clusters=out[3])
 
 
 # ----------------------------------------------------------- convenience

@@ -91,9 +91,10 @@ typedef struct {
 } moe_reader_debug;
 
 /* Bytes of device workspace moe_reader_forward / moe_reader_forward_dense
- * need for this shape (16-byte aligned base).  Contents need no
- * initialisation; a workspace must not be shared by calls that may run
- * concurrently. */
+ * need for this shape (16-byte aligned base).  Zero-fill a workspace once
+ * before its first use (it holds the device error word); the library keeps
+ * the rest consistent from call to call.  A workspace must not be shared by
+ * calls that may run concurrently. */
 size_t moe_reader_workspace_bytes(int B, int E, int top_e, int I, int d, int k, int c, int r);
 
 /* Offline: the rotated ternary sketch of every gate and up row ("A reader
@@ -119,7 +120,7 @@ moe_status moe_reader_build_sketch(int E, int I, int d, const uint16_t* w_gate, 
  * the down projections).  Per expert, the rank-r truncated SVD
  * W_down[e] = U S V^T gives u_sigma = U[:, :r] S[:r] ([I, r]) and
  * v = V[:, :r] ([d, r]); in each column the entry of v with the largest
- * magnitude is positive.  Computed by subspace iteration on W W^T with a
+ * magnitude is positive (decided before the bf16 rounding).  Computed by subspace iteration on W W^T with a
  * Rayleigh-Ritz step; factors are rounded to bf16.
  * Needs moe_reader_lowrank_workspace_bytes(E, I, d, r) bytes of workspace. */
 size_t moe_reader_lowrank_workspace_bytes(int E, int I, int d, int r);
@@ -170,6 +171,16 @@ moe_status moe_reader_rmsnorm(int B, int d, float eps, const uint16_t* x, uint16
  * forward calls of this thread record events[0] before the expert kernel and
  * events[1] after it on `stream`.  Pass NULL to clear. */
 moe_status moe_reader_set_expert_events(void* ev_before, void* ev_after);
+
+/* Tuning: force the thread-block cluster size of the expert kernels (one
+ * cluster per (expert, token group)): 4, 8 or 16 CTAs, or 0 to choose
+ * automatically (the size that keeps the most SMs busy for the launch). */
+moe_status moe_reader_set_cluster_size(int cs);
+
+/* The launch the expert kernel would use for this shape on the current
+ * device (dense != 0: the dense block): out4 = {cluster size, copy-ring rows
+ * per warp, dynamic shared memory bytes per CTA, co-resident clusters}. */
+moe_status moe_reader_launch_plan(int dense, int B, int E, int top_e, int I, int d, int r, int32_t* out4);
 
 /* Synchronizes `stream`, reads and clears the workspace's device error word.
  * Returns MOE_OK, or MOE_ETIMEOUT if a bounded wait ran out since the last

@@ -87,12 +87,32 @@ def compare_step(W, x, gpu_y, gdbg, ora_y64, odbg, k, ora_logits=None, check_kep
             for i in G ^ Ok:
                 assert k1 * (1 - 1e-6) <= amap[i] <= kth * (1 + 1e-6), f"channel {i} outside the tie band"
             swaps += 1
+    # fp32 per-expert outputs (before the bf16 rounding) where the kept sets agree
+    ye_err = 0.0
+    if "y_expert" in odbg and odbg["y_expert"] is not None:
+        for b in tok:
+            for s in range(top):
+                if set(g["kept"][b, s].tolist()) == set(odbg["kept"][b, s].tolist()):
+                    d = np.abs(g["y_expert"][b, s].astype(np.float64) - odbg["y_expert"][b, s])
+                    ye_err = max(ye_err, float(d.max()))
+        assert ye_err <= MAX_ABS, f"fp32 expert output error {ye_err}"
     yg = gpu_y.float().cpu().numpy().astype(np.float64)[tok]
     yo = ora_y64[tok]
-    err = float(np.abs(yg - yo).max())
+    diff = np.abs(yg - yo)
+    err = float(diff.max())
     rel = float(np.linalg.norm(yg - yo) / max(np.linalg.norm(yo), 1e-30))
-    assert err <= MAX_ABS and rel <= REL_L2, (err, rel)
-    return dict(max_abs=err, rel_l2=rel, swaps=swaps)
+    # bf16 output: 2e-2 beyond one bf16 ulp of the exact value
+    ulp = bf16_ulp(yo)
+    excess = float((diff - ulp).max())
+    assert excess <= MAX_ABS and rel <= REL_L2, dict(max_abs=err, excess=excess, rel=rel, ye_err=ye_err,
+                                                     swaps=swaps, ymax=float(np.abs(yo).max()))
+    return dict(max_abs=err, excess_over_ulp=excess, rel_l2=rel, y_expert_max_abs=ye_err, swaps=swaps)
+
+
+def bf16_ulp(v):
+    """One bf16 ulp at the magnitude of v (8 significant bits)."""
+    a = np.maximum(np.abs(np.asarray(v, np.float64)), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(a)) - 7)
 
 
 def run_pair(layer: M.Layer, oc: OracleCache, x, k, c, top_e, use_oracle_factors=True):
