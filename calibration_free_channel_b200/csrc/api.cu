@@ -112,8 +112,11 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   ra.dbg_ids = dbg ? dbg->ids : nullptr;
   ra.dbg_w = dbg ? dbg->weights : nullptr;
   ra.quantize = !dense;
-  cudaError_t e = moe::launch_route(ra, s);
-  if (e != cudaSuccess) return cuda_fail(e, "route launch");
+  cudaError_t e = cudaSuccess;
+  if (!moe::fused_routing(B)) {
+    e = moe::launch_route(ra, s);
+    if (e != cudaSuccess) return cuda_fail(e, "route launch");
+  }
 
   moe::ExpertArgs a = {};
   a.B = B;
@@ -127,6 +130,9 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   a.cs = 0;  // chosen at launch (16 when schedulable, else 8)
   a.nmax = B < moe::kMaxGroup ? B : moe::kMaxGroup;
   a.x = x;
+  a.w_router = L->w_router;
+  a.bias = L->router_bias;
+  a.rot_sign = L->rot_sign;
   a.w_gate = L->w_gate;
   a.w_up = L->w_up;
   a.w_down = L->w_down;
@@ -140,6 +146,8 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   a.y = y;
   a.ws = ws;
   if (dbg) {
+    a.dbg_ids = dbg->ids;
+    a.dbg_w = dbg->weights;
     a.dbg_G = dbg->dot_gate;
     a.dbg_U = dbg->dot_up;
     a.dbg_sigma = dbg->score;

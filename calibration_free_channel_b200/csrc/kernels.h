@@ -46,6 +46,9 @@ struct ExpertArgs {
   int nmax;          // max tokens per work item this launch
   int ring_rows;     // copy-ring row slots per warp (sparse) / rows (dense)
   const uint16_t* x;
+  const uint16_t* w_router;  // routing inside the expert kernel (small B)
+  const float* bias;
+  const int8_t* rot_sign;
   const uint16_t* w_gate;
   const uint16_t* w_up;
   const uint16_t* w_down;
@@ -59,6 +62,8 @@ struct ExpertArgs {
   uint16_t* y;
   Workspace ws;
   // debug outputs (may be null)
+  int32_t* dbg_ids;
+  float* dbg_w;
   int32_t* dbg_G;
   int32_t* dbg_U;
   float* dbg_sigma;
@@ -67,8 +72,9 @@ struct ExpertArgs {
   float* dbg_a_kept;
   float* dbg_y_expert;
 };
-size_t reader_smem_bytes(const ExpertArgs& a, int ring_rows);
-size_t dense_smem_bytes(const ExpertArgs& a, int ring_rows);
+// Steps of at most this many tokens route inside the expert kernel (one
+// launch per step); larger steps use the route and select kernels first.
+bool fused_routing(int B);
 cudaError_t launch_reader(const ExpertArgs& a, cudaStream_t s);
 cudaError_t launch_dense(const ExpertArgs& a, cudaStream_t s);
 void set_forced_cluster_size(int cs);

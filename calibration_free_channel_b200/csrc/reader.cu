@@ -1,27 +1,34 @@
 // reader.cu -- the sparse routed-expert reader and the dense baseline block.
 //
-// One thread-block cluster (cs CTAs, cs = 16 or 8) runs one work item: an
-// expert e and the (up to kMaxGroup) tokens routed to it, so tokens that share
-// an expert share its reads.  The steps ("Channel Selection for
+// One thread-block cluster (cs CTAs, 8 <= cs <= 16) runs one work item: an
+// expert e and the tokens routed to it (up to NT), so tokens that share an
+// expert share its reads.  The reader's steps ("Channel Selection for
 // Mixture-of-Experts Decoding Needs No Calibration Data", abstract; "KAIST:
 // MoE Decoding Needs No Calibration Data", section "A reader that needs no
 // data at all"):
+//   R  (B <= 4) routing inside the cluster: every CTA computes the logits of
+//      its slice of experts and pushes them to all CTAs; every CTA then takes
+//      the same top-e and finds its cluster's work item;
 //   S  screen: every CTA reads the ternary sketch rows of its slice of the I
-//      channels, computes exact integer dots with the int8 rotated token and
-//      the screening score sigma = |silu(ghat) uhat|;          cluster barrier
-//   c  every CTA gathers all sigma over distributed shared memory and selects
-//      the same top-c candidates per token (ties: lower channel);
+//      channels, forms exact integer dots with the int8 rotated token and the
+//      screening score sigma = |silu(ghat) uhat|, and pushes sigma (and the
+//      estimate ahat) to every CTA of the cluster;           cluster barrier
+//   c  every CTA selects the same top-c candidates per token (ties: lower
+//      channel);
 //   C  exact: the CTAs split the union of the candidates, read the BF16 gate
-//      and up rows and compute a = silu(g) u;                    cluster barrier
-//   k  every CTA gathers a and selects the same top-k per token (the
-//      top-k keep rule: no calibrated threshold);
+//      and up rows, compute a = silu(g) u and push it to every CTA;
+//                                                           cluster barrier
+//   k  every CTA selects the same top-k per token by |a|: the top-k keep rule,
+//      no calibrated threshold;
 //   D  down + recovery: every CTA reads its column slice of the kept down
-//      rows (and the kept rows of the low-rank factor U_r S_r) and forms
+//      rows (with the kept rows of the factor Ubar = U_r S_r) and forms
 //      y_e = sum_K a_i W_down[i,:] + V z, z = sum_{i not in K} ahat_i Ubar_i;
-//   combine: the last of a token's top_e experts to finish a column slice
-//      sums w_s y_e,s in slot order and writes bf16 y.
-// All rows move with 1-D bulk copies (cp.async.bulk) into per-warp rings in
-// the CTA's own shared memory; every wait on them is bounded.
+//   combine: the last of a token's top_e experts to finish a column slice sums
+//      w_s y_e,s in slot order, writes bf16 y and resets the slice's counter.
+// Rows move with 1-D bulk copies (cp.async.bulk) into per-warp rings in the
+// CTA's own shared memory; every wait on them is bounded.  Every exchange
+// between the CTAs of a cluster is a store into the receivers' shared memory
+// followed by a cluster barrier: no CTA reads another CTA's shared memory.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -29,62 +36,122 @@ namespace moe {
 
 namespace {
 
+constexpr int NTHR = 512;
+constexpr int NWARP = NTHR / 32;
+constexpr int kMaxCols = 256;  // output columns per CTA (8 per lane)
+
 __host__ __device__ inline int rup(int x, int a) { return (x + a - 1) / a * a; }
 __host__ __device__ inline int cdiv(int x, int a) { return (x + a - 1) / a; }
 
-// Shared-memory carve-up, identical on host and device.
+// ------------------------------------------------------------ smem layout
 struct Layout {
-  int mbar, misc, hist, x, q, sig_own, ahat_own, zpart, ubar, vown, sig_all, ahat_all, z_all, candm,
-      keptm, ulist, upos, dlist, keys, kidx, a_own, ring, total;
-  int own, cols, words, ring_bytes;  // per CTA: channels, output columns; mask words; ring bytes per warp
+  int mbar, misc, hist, wtot, pmask, x, q, logit, sig, ahat, zparts, z, apos, candm, keptm, ulist, upos, dlist,
+      keys, kidx, ubar, vown, ring, total;
+  int ntok;        // tokens held in smem (fused routing: B; otherwise NT)
+  int own_max;     // max channels per CTA
+  int cols_max;    // max output columns per CTA
+  int words;       // mask words over I
+  int ring_bytes;  // per warp
 };
 
-__host__ __device__ inline Layout make_layout(int nmax, int I, int d, int r, int cs, int ring_rows,
-                                              bool dense) {
+__host__ __device__ inline Layout make_layout(int NT, int ntok, bool fused, int E, int I, int d, int r, int cs,
+                                              int ring_rows, bool dense) {
   Layout L;
-  L.own = cdiv(I, cs);
-  L.cols = d / cs;
+  L.ntok = ntok;
+  L.own_max = cdiv(I, cs);
+  L.cols_max = 8 * cdiv(d / 8, cs);
   L.words = cdiv(I, 32);
   L.ring_bytes = ring_rows * d * 2;
+  const int rr = r > 0 ? r : 1;
   int o = 0;
   auto take = [&](int bytes) {
     int at = o;
     o = rup(o + bytes, 128);
     return at;
   };
-  L.mbar = take((kWarps * kMaxSlots + 2) * 8);
-  L.misc = take(1024);
-  L.hist = take(260 * 4);
-  L.x = take(nmax * d * 2);
-  L.q = dense ? 0 : take(nmax * d);
-  L.sig_own = take(nmax * L.own * 4);  // dense: h of the own channels
-  L.ahat_own = dense ? 0 : take(nmax * L.own * 4);
-  L.zpart = dense ? 0 : take(nmax * (r > 0 ? r : 1) * 4);
-  L.ubar = dense ? 0 : take(L.own * (r > 0 ? r : 1) * 2);
-  L.vown = dense ? 0 : take(L.cols * (r > 0 ? r : 1) * 2);
-  L.sig_all = take(nmax * I * 4);  // sparse: sigma then a (by U position); dense: h of all channels
-  L.ahat_all = dense ? 0 : take(nmax * I * 4);
-  L.z_all = dense ? 0 : take(nmax * (r > 0 ? r : 1) * 4);
-  L.candm = dense ? 0 : take(nmax * L.words * 4);
-  L.keptm = dense ? 0 : take(nmax * L.words * 4);
+  L.mbar = take((NWARP * kMaxSlots + 4) * 8);
+  L.misc = take(256 * 4);
+  L.hist = take(2 * 2048 * 4);
+  L.wtot = take(64 * 4);
+  L.pmask = take(L.words * 4);
+  L.x = take(ntok * d * 2);
+  L.q = take(ntok * d);
+  L.logit = fused ? take(ntok * E * 8) : 0;
+  L.sig = take(NT * I * 4);  // sparse: sigma by channel; dense: h by channel
+  L.ahat = dense ? 0 : take(NT * I * 4);
+  L.zparts = dense ? 0 : take(cs * NT * rr * 4);
+  L.z = dense ? 0 : take(NT * rr * 4);
+  L.apos = dense ? 0 : take(NT * I * 4);  // a by union position
+  L.candm = dense ? 0 : take(NT * L.words * 4);
+  L.keptm = dense ? 0 : take(NT * L.words * 4);
   L.ulist = dense ? 0 : take(I * 4);
   L.upos = dense ? 0 : take(I * 4);
   L.dlist = dense ? 0 : take(I * 4);
   L.keys = dense ? 0 : take(I * 4);
   L.kidx = dense ? 0 : take(I * 4);
-  L.a_own = dense ? 0 : take(nmax * L.own * 4);
-  L.ring = take(kWarps * L.ring_bytes);
+  L.ubar = dense ? 0 : take(L.own_max * rr * 2);
+  L.vown = dense ? 0 : take(L.cols_max * rr * 2);
+  L.ring = take(NWARP * L.ring_bytes);
   L.total = o;
   return L;
 }
 
 // misc ints
-enum { MI_E = 0, MI_N, MI_NU, MI_ND, MI_ERR, MI_PREFIX, MI_REM, MI_TOK = 8, MI_SLOT = 16, MI_LAST = 24, MI_CX = 32,
-       MI_SCAN = 48 };
+enum {
+  MI_E = 0, MI_N, MI_NU, MI_ND, MI_NC, MI_DIG, MI_REM, MI_CNT, MI_DONE,
+  MI_TOK = 16, MI_SLOT = 32, MI_LAST = 48, MI_TIX = 64, MI_CX = 80, MI_SCAN = 96,
+  MI_RIDS = 128,  // fused routing: ids [B <= 4][top_e <= 16]
+  MI_RW = 192     // fused routing: weights
+};
+
+// ---------------------------------------------------------- cluster helpers
+__device__ __forceinline__ uint32_t cluster_addr(const void* local, int rank) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
+  return ra;
+}
+__device__ __forceinline__ void st_cluster(const void* local, int rank, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr(local, rank)), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster(const void* local, int rank, double v) {
+  asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(cluster_addr(local, rank)), "d"(v) : "memory");
+}
+
+// -------------------------------------------------------- mixed-precision dot
+// 8 bf16 x 8 bf16 accumulated in fp32: fma.rn.f32.bf16 multiplies the bf16
+// operands exactly and rounds once into the fp32 accumulator (two chains).
+__device__ __forceinline__ void dot8_mixed(uint4 a, uint4 b, float& acc0, float& acc1) {
+  asm("{\n\t.reg .b16 a0, a1, a2, a3, a4, a5, a6, a7, b0, b1, b2, b3, b4, b5, b6, b7;\n\t"
+      "mov.b32 {a0, a1}, %2;\n\tmov.b32 {a2, a3}, %3;\n\tmov.b32 {a4, a5}, %4;\n\tmov.b32 {a6, a7}, %5;\n\t"
+      "mov.b32 {b0, b1}, %6;\n\tmov.b32 {b2, b3}, %7;\n\tmov.b32 {b4, b5}, %8;\n\tmov.b32 {b6, b7}, %9;\n\t"
+      "fma.rn.f32.bf16 %0, a0, b0, %0;\n\tfma.rn.f32.bf16 %1, a1, b1, %1;\n\t"
+      "fma.rn.f32.bf16 %0, a2, b2, %0;\n\tfma.rn.f32.bf16 %1, a3, b3, %1;\n\t"
+      "fma.rn.f32.bf16 %0, a4, b4, %0;\n\tfma.rn.f32.bf16 %1, a5, b5, %1;\n\t"
+      "fma.rn.f32.bf16 %0, a6, b6, %0;\n\tfma.rn.f32.bf16 %1, a7, b7, %1;\n\t}"
+      : "+f"(acc0), "+f"(acc1)
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w));
+}
+
+// Trits of one packed sketch word as four words of signed bytes.  Layout:
+// position n (< 8) at bits [4n, 4n+1], position 8+n at bits [4n+2, 4n+3];
+// codes 00 = 0, 01 = +1, 11 = -1.  A nibble's code selects a byte of
+// kTritLut = {0x00, 0x01, 0x00, 0xff} through byte_perm.
+__device__ __forceinline__ uint4 decode_trits(uint32_t w) {
+  const uint32_t kTritLut = 0xff000100u;
+  const uint32_t lo = w & 0x33333333u;
+  const uint32_t hi = (w >> 2) & 0x33333333u;
+  return make_uint4(__byte_perm(kTritLut, 0, lo), __byte_perm(kTritLut, 0, lo >> 16),
+                    __byte_perm(kTritLut, 0, hi), __byte_perm(kTritLut, 0, hi >> 16));
+}
+__device__ __forceinline__ int dot16_i8(uint4 t, uint4 q, int acc) {
+  acc = __dp4a((int)t.x, (int)q.x, acc);
+  acc = __dp4a((int)t.y, (int)q.y, acc);
+  acc = __dp4a((int)t.z, (int)q.z, acc);
+  acc = __dp4a((int)t.w, (int)q.w, acc);
+  return acc;
+}
 
 // ----------------------------------------------------------- block helpers
-// Exclusive scan of one int per thread over the CTA; returns the prefix and
-// writes the total to *total (every thread).
 __device__ int block_excl_scan(int v, int* scratch, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int inc = v;
@@ -96,122 +163,132 @@ __device__ int block_excl_scan(int v, int* scratch, int* total) {
   if (lane == 31) scratch[warp] = inc;
   __syncthreads();
   int off = 0, tot = 0;
-  for (int w = 0; w < kWarps; w++) {
-    if (w < warp) off += scratch[w];
-    tot += scratch[w];
+#pragma unroll
+  for (int w = 0; w < NWARP; w++) {
+    const int s = scratch[w];
+    off += w < warp ? s : 0;
+    tot += s;
   }
   __syncthreads();
   *total = tot;
   return off + inc - v;
 }
 
-// Top-n of N keys (uint32, larger = better, ties to the lower position):
-// radix select on 8-bit digits, then an ordered pass over the keys equal to
-// the threshold.  Sets bit p of out_mask for each chosen position p.
-__device__ void block_select_top(const uint32_t* keys, int N, int n_sel, int* hist, int* misc,
+// Top-n_sel of N keys (uint32, larger first, ties to the lower position):
+// radix select with digits of 11, 11 and 10 bits from the top, stopping as
+// soon as the boundary bin is taken whole; keys equal to a fully resolved
+// threshold are taken in position order.  Sets bit p of out_mask for each
+// chosen position p.  hist holds 2 x 2048 ints, wtot 16 ints.
+__device__ void block_select_top(const uint32_t* keys, int N, int n_sel, int* hist, int* wtot, int* misc,
                                  uint32_t* out_mask) {
-  const int tid = threadIdx.x;
-  for (int w = tid; w < cdiv(N, 32); w += kThreads) out_mask[w] = 0u;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = cdiv(N, 32);
+  for (int w = tid; w < nw; w += NTHR) out_mask[w] = 0u;
   if (n_sel >= N) {
     __syncthreads();
-    for (int p = tid; p < N; p += kThreads) atomicOr(&out_mask[p >> 5], 1u << (p & 31));
+    for (int p = tid; p < N; p += NTHR) atomicOr(&out_mask[p >> 5], 1u << (p & 31));
     __syncthreads();
     return;
   }
-  if (tid == 0) {
-    misc[MI_PREFIX] = 0;
-    misc[MI_REM] = n_sel;
-  }
-  uint32_t mask = 0u;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = tid; b < 256; b += kThreads) hist[b] = 0;
-    __syncthreads();
-    const uint32_t prefix = (uint32_t)misc[MI_PREFIX];
-    for (int p = tid; p < N; p += kThreads) {
+  for (int b = tid; b < 2048; b += NTHR) hist[b] = 0;
+  uint32_t prefix = 0u, mask = 0u;
+  int rem = n_sel;
+  bool done = false;
+  for (int pass = 0; pass < 3 && !done; pass++) {
+    const int shift = pass == 0 ? 21 : pass == 1 ? 10 : 0;
+    const int nb = pass == 2 ? 1024 : 2048;
+    int* h = hist + (pass & 1) * 2048;
+    int* hn = hist + ((pass + 1) & 1) * 2048;
+    __syncthreads();  // h is zero and the previous pass is done with hn
+    for (int p = tid; p < N; p += NTHR) {
       const uint32_t k = keys[p];
-      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
+      if ((k & mask) == prefix) atomicAdd(&h[(k >> shift) & (nb - 1)], 1);
     }
+    for (int b = tid; b < 2048; b += NTHR) hn[b] = 0;
     __syncthreads();
-    if (tid < 32) {
-      // suffix sums over digits 255..0, 8 digits per lane (lane 0 = top digits)
-      int loc[8], s = 0;
+    // warp w covers bins [nb - (w+1) bpw, nb - w bpw), top-down; lane l a run
+    const int bpw = nb / NWARP, bpl = bpw / 32;
+    const int top = nb - warp * bpw - lane * bpl;  // bins top-1 .. top-bpl
+    int s = 0;
+    for (int j = 1; j <= bpl; j++) s += h[top - j];
+    int inc = s;
 #pragma unroll
-      for (int t = 0; t < 8; t++) {
-        loc[t] = hist[255 - (tid * 8 + t)];
-        s += loc[t];
-      }
-      int inc = s;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, inc, o);
-        if (tid >= o) inc += n;
-      }
-      const int rem = misc[MI_REM];
-      int before = inc - s;  // keys with a larger digit than this lane's first
-      int found = -1, take_before = 0;
-#pragma unroll
-      for (int t = 0; t < 8; t++) {
-        if (found < 0 && before < rem && before + loc[t] >= rem) {
-          found = 255 - (tid * 8 + t);
-          take_before = before;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += n;
+    }
+    if (lane == 31) wtot[warp] = inc;
+    __syncthreads();
+    int before = inc - s;  // keys in bins above this lane's run
+    for (int w = 0; w < warp; w++) before += wtot[w];
+    if (before < rem && before + s >= rem) {
+      for (int j = 1; j <= bpl; j++) {
+        const int c = h[top - j];
+        if (before + c >= rem) {
+          misc[MI_DIG] = top - j;
+          misc[MI_REM] = rem - before;
+          misc[MI_CNT] = c;
+          break;
         }
-        before += loc[t];
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, found >= 0);
-      const int src = __ffs(bal) - 1;
-      const int dig = __shfl_sync(0xffffffffu, found, src);
-      const int tb = __shfl_sync(0xffffffffu, take_before, src);
-      if (tid == 0) {
-        misc[MI_PREFIX] = (int)(prefix | ((uint32_t)dig << shift));
-        misc[MI_REM] = rem - tb;
+        before += c;
       }
     }
-    mask |= 255u << shift;
     __syncthreads();
+    prefix |= (uint32_t)misc[MI_DIG] << shift;
+    mask |= (uint32_t)(nb - 1) << shift;
+    rem = misc[MI_REM];
+    done = rem == misc[MI_CNT];
   }
-  const uint32_t T = (uint32_t)misc[MI_PREFIX];
-  const int rem = misc[MI_REM];  // keys equal to T to take, lowest positions first
-  // contiguous chunk per thread for the ordered equal-key pass
-  const int chunk = cdiv(N, kThreads);
+  if (done) {
+    // the boundary bin is taken whole: keep every key whose decided bits are
+    // at least the boundary prefix
+    for (int p = tid; p < N; p += NTHR)
+      if ((keys[p] & mask) >= prefix) atomicOr(&out_mask[p >> 5], 1u << (p & 31));
+    __syncthreads();
+    return;
+  }
+  // fully resolved threshold T = prefix with more equal keys than needed:
+  // keys > T, and the first `rem` keys == T by position
+  const int chunk = cdiv(N, NTHR);
   const int p0 = min(N, tid * chunk), p1 = min(N, p0 + chunk);
   int eq = 0;
-  for (int p = p0; p < p1; p++) eq += keys[p] == T;
+  for (int p = p0; p < p1; p++) eq += keys[p] == prefix;
   int tot;
   int before = block_excl_scan(eq, misc + MI_SCAN, &tot);
   for (int p = p0; p < p1; p++) {
     const uint32_t k = keys[p];
-    bool take = k > T;
-    if (k == T) {
-      take = before < rem;
-      before++;
-    }
+    bool take = k > prefix;
+    if (k == prefix) take = before++ < rem;
     if (take) atomicOr(&out_mask[p >> 5], 1u << (p & 31));
   }
   __syncthreads();
 }
 
-// Warp 0: ascending list of the set bits of mask over [0, N); returns count
-// through misc[slot_idx] (after a __syncthreads by the caller).
-__device__ void warp_mask_to_list(const uint32_t* mask, int N, int* list, int* pos_of, int* count_out) {
-  const int lane = threadIdx.x & 31;
-  int base = 0;
-  for (int w0 = 0; w0 < N; w0 += 32) {
-    const int p = w0 + lane;
-    const bool on = p < N && ((mask[w0 >> 5] >> lane) & 1u);
+// Ascending list of the set bits of mask over [0, N), all warps; the count
+// lands in *count_out; pos_of (if given) gets each bit's list position or -1.
+__device__ void block_mask_to_list(const uint32_t* mask, int N, int* list, int* pos_of, int* count_out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = cdiv(N, 32);
+  for (int w = warp; w < nw; w += NWARP) {
+    int off = 0;
+    for (int v = lane; v < w; v += 32) off += __popc(mask[v]);
+    off = warp_sum(off);
+    const int p = w * 32 + lane;
+    const bool on = p < N && ((mask[w] >> lane) & 1u);
     const unsigned bal = __ballot_sync(0xffffffffu, on);
-    const int at = base + __popc(bal & ((1u << lane) - 1u));
+    const int at = off + __popc(bal & ((1u << lane) - 1u));
     if (on) list[at] = p;
     if (pos_of && p < N) pos_of[p] = on ? at : -1;
-    base += __popc(bal);
+    if (w == nw - 1 && lane == 0) *count_out = off + __popc(bal);
   }
-  if (lane == 0) *count_out = base;
+  __syncthreads();
 }
 
 // --------------------------------------------------------- per-warp rings
 // A warp streams `cnt` elements through P slots of its ring.  Lane 0 issues
 // element j into slot j % P (issue(j, slot, bar)); all lanes consume it after
 // a bounded wait.  `par` holds the parity bit of each slot barrier and
-// persists across pipelines.  Returns false if a wait ran out (the warp then
+// persists across stages.  Returns false if a wait ran out (the warp then
 // stops issuing and drains what is in flight).
 template <class Issue, class Consume>
 __device__ bool warp_stream(int cnt, int P, uint64_t* bars, uint32_t& par, uint32_t* err, Issue issue,
@@ -220,15 +297,14 @@ __device__ bool warp_stream(int cnt, int P, uint64_t* bars, uint32_t& par, uint3
   if (cnt <= 0) return true;
   P = min(P, cnt);
   uint32_t pend = 0;
-  // the ring may have been read by generic loads in an earlier stage
-  if (lane == 0) fence_proxy_async();
+  if (lane == 0) fence_proxy_async();  // the ring may have been read by generic loads
   for (int j = 0; j < P; j++) {
     if (lane == 0) issue(j, j, &bars[j]);
     pend |= 1u << j;
   }
   __syncwarp();
   bool ok = true;
-  for (int j = 0; j < cnt && ok; j++) {
+  for (int j = 0; j < cnt; j++) {
     const int s = j % P;
     ok = mbar_wait_bounded(&bars[s], (par >> s) & 1u, err);
     if (!ok) break;
@@ -247,22 +323,30 @@ __device__ bool warp_stream(int cnt, int P, uint64_t* bars, uint32_t& par, uint3
   }
   if (!ok) {
     for (int s = 0; s < P; s++)
-      if ((pend >> s) & 1u) {
+      if ((pend >> s) & 1u)
         if (mbar_wait_bounded(&bars[s], (par >> s) & 1u, err)) par ^= 1u << s;
-      }
   }
   return ok;
 }
 
-// Loads the work item of this cluster; returns false if the cluster is idle.
-__device__ bool load_item(const ExpertArgs& a, int cid, int* misc) {
+// Column slice of a CTA in 8-column units (16-byte aligned slices).
+__device__ __forceinline__ void col_slice(int d, int cs, int rank, int& j0, int& ncols) {
+  const int u = d / 8;
+  const int u0 = cdiv(rank * u, cs), u1 = cdiv((rank + 1) * u, cs);
+  j0 = u0 * 8;
+  ncols = (u1 - u0) * 8;
+}
+
+// ------------------------------------------------------- work item set-up
+// The item comes from the work table the select kernel wrote.
+__device__ bool load_item_table(const ExpertArgs& a, int cid, int* misc, int NT) {
   if (threadIdx.x == 0) {
     const int n_items = *a.ws.n_items;
     int e = -1, n = 0;
     if (cid < n_items && cid < a.ws.max_items) {
       e = a.ws.item_e[cid];
       n = a.ws.item_n[cid];
-      if (e < 0 || e >= a.E || n < 1 || n > kMaxGroup || n > a.nmax) {
+      if (e < 0 || e >= a.E || n < 1 || n > NT) {
         atomicOr(a.ws.err, kErrBadWorkItem);
         e = -1;
       }
@@ -278,21 +362,217 @@ __device__ bool load_item(const ExpertArgs& a, int cid, int* misc) {
       }
       misc[MI_TOK + t] = tok;
       misc[MI_SLOT + t] = sl;
-      reinterpret_cast<float*>(misc)[MI_CX + t] = a.ws.cx ? a.ws.cx[tok] : 0.0f;
+      misc[MI_TIX + t] = t;  // tokens are loaded in item order
     }
   }
   __syncthreads();
   return misc[MI_E] >= 0;
 }
 
+// Loads tokens into smem: toks[t] -> smem token t.
+__device__ void load_x(const ExpertArgs& a, const Layout& L, char* smem, const int* toks, int n) {
+  const int vx = a.d / 8;
+  uint4* xs = reinterpret_cast<uint4*>(smem + L.x);
+  for (int idx = threadIdx.x; idx < n * vx; idx += NTHR) {
+    const int t = idx / vx, j = idx - t * vx;
+    xs[idx] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)toks[t] * a.d) + j);
+  }
+}
+__device__ void load_q(const ExpertArgs& a, const Layout& L, char* smem, const int* toks, int n) {
+  const int vq = a.d / 16;
+  uint4* qs = reinterpret_cast<uint4*>(smem + L.q);
+  for (int idx = threadIdx.x; idx < n * vq; idx += NTHR) {
+    const int t = idx / vq, j = idx - t * vq;
+    qs[idx] = __ldcg(reinterpret_cast<const uint4*>(a.ws.q + (size_t)toks[t] * a.d) + j);
+  }
+}
+
+// Rotation + int8 quantisation of smem token t: v = FWHT(s . x) in the fp32
+// scratch (d floats), q = rint(127 v / amax), c_x = amax / (127 d).  The
+// butterflies follow the reference order (stages h = 1, 2, 4, ...), so the
+// bits equal the reference transform's.
+__device__ void rotate_quantize_smem(const ExpertArgs& a, const Layout& L, char* smem, int t, float* v,
+                                     float* cx_out, float* red) {
+  const int d = a.d;
+  const uint16_t* xs = reinterpret_cast<const uint16_t*>(smem + L.x) + (size_t)t * d;
+  for (int j = threadIdx.x; j < d; j += NTHR) v[j] = (float)a.rot_sign[j] * bf16f(xs[j]);
+  __syncthreads();
+  for (int h = 1, lh = 0; h < d; h <<= 1, lh++) {
+    for (int p = threadIdx.x; p < d / 2; p += NTHR) {
+      const int j = ((p >> lh) << (lh + 1)) | (p & (h - 1));
+      const float x0 = v[j], x1 = v[j + h];
+      v[j] = __fadd_rn(x0, x1);
+      v[j + h] = __fsub_rn(x0, x1);
+    }
+    __syncthreads();
+  }
+  float m = 0.0f;
+  for (int j = threadIdx.x; j < d; j += NTHR) m = fmaxf(m, fabsf(v[j]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float amax = 0.0f;
+  for (int w = 0; w < NWARP; w++) amax = fmaxf(amax, red[w]);
+  int8_t* q = reinterpret_cast<int8_t*>(smem + L.q) + (size_t)t * d;
+  for (int j = threadIdx.x; j < d; j += NTHR) {
+    int n = 0;
+    if (amax > 0.0f) n = max(-127, min(127, __float2int_rn(__fdiv_rn(__fmul_rn(v[j], 127.0f), amax))));
+    q[j] = (int8_t)n;
+  }
+  if (threadIdx.x == 0) *cx_out = amax > 0.0f ? __fdiv_rn(amax, __fmul_rn(127.0f, (float)d)) : 0.0f;
+  __syncthreads();
+}
+
+// Fused routing (B <= NT <= 4): every CTA loads all tokens, rotates and
+// quantises them, computes the logits of its slice of experts and pushes
+// them to all CTAs; after the cluster barrier every CTA runs the same top-e
+// and builds the same work table (one item per routed expert, experts
+// ascending).  Returns false if this cluster has no item.
+template <int NT>
+__device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, int* misc, int cs, int rank,
+                            int cid, uint64_t* wrbar, cg::cluster_group& cluster) {
+  const int B = a.B, E = a.E, d = a.d, top = a.top_e;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int e0 = cdiv(rank * E, cs), e1 = cdiv((rank + 1) * E, cs), ne = e1 - e0;
+  char* wr = smem + L.ring;  // router rows of this CTA's experts
+  if (threadIdx.x == 0 && ne > 0) {
+    mbar_expect_tx(wrbar, ne * d * 2);
+    bulk_g2s(wr, a.w_router + (size_t)e0 * d, ne * d * 2, wrbar);
+  }
+  {
+    int toks[NT];
+#pragma unroll
+    for (int t = 0; t < NT; t++) toks[t] = t;
+    load_x(a, L, smem, toks, B);
+  }
+  __syncthreads();
+  // rotate + quantise every token (the ring tail is the fp32 scratch)
+  float* scratch = reinterpret_cast<float*>(smem + L.ring + NWARP * L.ring_bytes - d * 4);
+  float* cxs = reinterpret_cast<float*>(misc + MI_CX);
+  for (int t = 0; t < B; t++)
+    rotate_quantize_smem(a, L, smem, t, scratch, &cxs[t], reinterpret_cast<float*>(misc + MI_SCAN));
+  // logits of the own experts, one warp per expert, pushed to every CTA
+  if (ne > 0 && !mbar_wait_bounded(wrbar, 0, a.ws.err)) misc[MI_DONE] = 1;
+  double* lg = reinterpret_cast<double*>(smem + L.logit);
+  for (int el = warp; el < ne; el += NWARP) {
+    const uint4* wrow = reinterpret_cast<const uint4*>(wr + (size_t)el * d * 2);
+    double acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; t++) acc[t] = 0.0;
+    for (int j = lane; j < d / 8; j += 32) {
+      const uint4 w = wrow[j];
+#pragma unroll
+      for (int t = 0; t < NT; t++) {
+        if (t < B) {
+          const uint4 x = reinterpret_cast<const uint4*>(smem + L.x + (size_t)t * d * 2)[j];
+          acc[t] = fma((double)bf16lo(w.x), (double)bf16lo(x.x), acc[t]);
+          acc[t] = fma((double)bf16hi(w.x), (double)bf16hi(x.x), acc[t]);
+          acc[t] = fma((double)bf16lo(w.y), (double)bf16lo(x.y), acc[t]);
+          acc[t] = fma((double)bf16hi(w.y), (double)bf16hi(x.y), acc[t]);
+          acc[t] = fma((double)bf16lo(w.z), (double)bf16lo(x.z), acc[t]);
+          acc[t] = fma((double)bf16hi(w.z), (double)bf16hi(x.z), acc[t]);
+          acc[t] = fma((double)bf16lo(w.w), (double)bf16lo(x.w), acc[t]);
+          acc[t] = fma((double)bf16hi(w.w), (double)bf16hi(x.w), acc[t]);
+        }
+      }
+    }
+    const int e = e0 + el;
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+      if (t < B) {
+        const double s = warp_sum(acc[t]) + (a.bias ? (double)a.bias[e] : 0.0);
+        if (lane < cs) st_cluster(&lg[t * E + e], lane, s);
+      }
+    }
+  }
+  cluster.sync();
+  // top-e per token (warp b), ties to the lower id; softmax over the chosen
+  int* rids = misc + MI_RIDS;
+  float* rw = reinterpret_cast<float*>(misc + MI_RW);
+  if (warp < B) {
+    const int b = warp;
+    uint32_t taken = 0;
+    double cv[16];
+    for (int s = 0; s < top; s++) {
+      double bv = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int m = 0; lane + 32 * m < E; m++) {
+        const int e = lane + 32 * m;
+        if (taken & (1u << m)) continue;
+        const double lv = lg[b * E + e];
+        if (bi == 0x7fffffff || lv > bv) {
+          bv = lv;
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      cv[s] = bv;
+      if (lane == 0) rids[b * top + s] = bi;
+    }
+    if (lane == 0) {
+      double den = 0.0;
+      for (int s = 0; s < top; s++) den += exp(cv[s] - cv[0]);
+      for (int s = 0; s < top; s++) {
+        const float w = (float)(exp(cv[s] - cv[0]) / den);
+        rw[b * top + s] = w;
+        if (cid == 0 && rank == 0) {
+          a.ws.ids[b * top + s] = rids[b * top + s];
+          a.ws.wts[b * top + s] = w;
+          if (a.dbg_ids) a.dbg_ids[b * top + s] = rids[b * top + s];
+          if (a.dbg_w) a.dbg_w[b * top + s] = w;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // work table: distinct experts ascending; item cid = the cid-th of them
+  if (threadIdx.x == 0) {
+    int chosen = -1, count = 0, prev = -1;
+    while (true) {
+      int nxt = 0x7fffffff;
+      for (int i = 0; i < B * top; i++)
+        if (rids[i] > prev && rids[i] < nxt) nxt = rids[i];
+      if (nxt == 0x7fffffff) break;
+      if (count == cid) chosen = nxt;
+      count++;
+      prev = nxt;
+    }
+    misc[MI_E] = chosen;
+    int n = 0;
+    if (chosen >= 0)
+      for (int b = 0; b < B; b++)
+        for (int s = 0; s < top; s++)
+          if (rids[b * top + s] == chosen) {
+            misc[MI_TOK + n] = b;
+            misc[MI_SLOT + n] = s;
+            misc[MI_TIX + n] = b;
+            n++;
+          }
+    misc[MI_N] = n;
+  }
+  __syncthreads();
+  return misc[MI_E] >= 0;
+}
+
 // Epilogue shared by both kernels: write y_e for this CTA's columns, then the
-// last expert of each token to finish this column slice combines.
-__device__ void write_and_combine(const ExpertArgs& a, const Layout& L, int rank, const float* yfin,
-                                  int* misc) {
+// last expert of each token to finish this column slice combines and resets
+// the slice's counter (so the counters are zero again after every call).
+// wts: routing weights [B, top_e] (global or this CTA's shared copy).
+__device__ void write_and_combine(const ExpertArgs& a, int rank, int j0, int ncols, const float* yfin, int* misc,
+                                  const float* wts) {
   const int n = misc[MI_N];
-  const int j0 = rank * L.cols;
-  for (int idx = threadIdx.x; idx < n * L.cols; idx += kThreads) {
-    const int t = idx / L.cols, col = idx % L.cols;
+  for (int idx = threadIdx.x; idx < n * ncols; idx += NTHR) {
+    const int t = idx / ncols, col = idx - t * ncols;
     const int tok = misc[MI_TOK + t], sl = misc[MI_SLOT + t];
     const size_t off = ((size_t)tok * a.top_e + sl) * a.d + j0 + col;
     a.ws.ye[off] = yfin[idx];
@@ -300,137 +580,151 @@ __device__ void write_and_combine(const ExpertArgs& a, const Layout& L, int rank
   }
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int t = 0; t < n; t++) {
-      const unsigned old = atomicAdd(&a.ws.counters[misc[MI_TOK + t] * kMaxCluster + rank], 1u);
-      misc[MI_LAST + t] = old == (unsigned)(a.top_e - 1);
-    }
+  if (threadIdx.x < n) {
+    const int t = threadIdx.x;
+    const unsigned old = atomicAdd(&a.ws.counters[misc[MI_TOK + t] * kMaxCluster + rank], 1u);
+    misc[MI_LAST + t] = old == (unsigned)(a.top_e - 1);
   }
   __syncthreads();
   for (int t = 0; t < n; t++) {
     if (!misc[MI_LAST + t]) continue;
     __threadfence();
     const int tok = misc[MI_TOK + t];
-    for (int col = threadIdx.x; col < L.cols; col += kThreads) {
+    for (int col = threadIdx.x; col < ncols; col += NTHR) {
       const int j = j0 + col;
       float acc = 0.0f;
       for (int s = 0; s < a.top_e; s++)
-        acc = fmaf(__ldcg(&a.ws.wts[tok * a.top_e + s]), __ldcg(&a.ws.ye[((size_t)tok * a.top_e + s) * a.d + j]),
-                   acc);
+        acc = fmaf(wts[tok * a.top_e + s], __ldcg(&a.ws.ye[((size_t)tok * a.top_e + s) * a.d + j]), acc);
       if (a.residual) acc += bf16f(a.residual[(size_t)tok * a.d + j]);
       a.y[(size_t)tok * a.d + j] = f2bf16(acc);
     }
-  }
-}
-
-// Loads x (and q) of the item's tokens into shared memory.
-__device__ void load_tokens(const ExpertArgs& a, const Layout& L, char* smem, const int* misc, bool with_q) {
-  const int n = misc[MI_N];
-  const int vx = a.d / 8, vq = a.d / 16;
-  uint4* xs = reinterpret_cast<uint4*>(smem + L.x);
-  for (int idx = threadIdx.x; idx < n * vx; idx += kThreads) {
-    const int t = idx / vx, j = idx % vx;
-    xs[idx] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)misc[MI_TOK + t] * a.d) + j);
-  }
-  if (with_q) {
-    uint4* qs = reinterpret_cast<uint4*>(smem + L.q);
-    for (int idx = threadIdx.x; idx < n * vq; idx += kThreads) {
-      const int t = idx / vq, j = idx % vq;
-      qs[idx] = __ldcg(reinterpret_cast<const uint4*>(a.ws.q + (size_t)misc[MI_TOK + t] * a.d) + j);
-    }
+    if (threadIdx.x == 0) a.ws.counters[tok * kMaxCluster + rank] = 0u;
   }
 }
 
 // ================================================================ sparse
-__global__ void __launch_bounds__(kThreads, 1) reader_kernel(ExpertArgs a) {
+template <int NT, bool FUSED>
+__global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L) {
   extern __shared__ __align__(128) char smem[];
   cg::cluster_group cluster = cg::this_cluster();
-  const int cs = a.cs;
+  const int cs = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
   const int cid = blockIdx.x / cs;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const Layout L = make_layout(a.nmax, a.I, a.d, a.r, cs, a.ring_rows, false);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.mbar);
   uint64_t* wbars = bars + warp * kMaxSlots;
-  uint64_t* uvbar = bars + kWarps * kMaxSlots;
+  uint64_t* uvbar = bars + NWARP * kMaxSlots;
+  uint64_t* wrbar = uvbar + 1;
   int* misc = reinterpret_cast<int*>(smem + L.misc);
   int* hist = reinterpret_cast<int*>(smem + L.hist);
-  if (tid < kWarps * kMaxSlots + 1) mbar_init(&bars[tid], 1);
+  int* wtot = reinterpret_cast<int*>(smem + L.wtot);
+  if (tid < NWARP * kMaxSlots + 2) mbar_init(&bars[tid], 1);
+  if (tid == 0) misc[MI_DONE] = 0;
   fence_mbar_init();
   __syncthreads();
 
-  pdl_wait();
-  if (!load_item(a, cid, misc)) return;  // uniform across the cluster
+  if (FUSED) {
+    if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, wrbar, cluster)) return;  // uniform per cluster
+  } else {
+    pdl_wait();
+    if (!load_item_table(a, cid, misc, NT)) return;
+  }
   const int e = misc[MI_E], n = misc[MI_N];
   const int I = a.I, d = a.d, r = a.r;
   const int i0 = cdiv(rank * I, cs), i1 = cdiv((rank + 1) * I, cs), nown = i1 - i0;
-  const int j0 = rank * L.cols;
+  int j0, ncols;
+  col_slice(d, cs, rank, j0, ncols);
   uint32_t* err = a.ws.err;
   uint32_t par = 0;
   char* ring = smem + L.ring + warp * L.ring_bytes;
+  int tix[NT];
+#pragma unroll
+  for (int t = 0; t < NT; t++) tix[t] = misc[MI_TIX + (t < n ? t : 0)];
 
-  // low-rank factor rows of the own channels and V rows of the own columns
+  // factor rows of the own channels and V rows of the own columns
   if (tid == 0 && r > 0) {
-    const uint32_t bu = nown * r * 2, bv = L.cols * r * 2;
+    const uint32_t bu = nown * r * 2, bv = ncols * r * 2;
     mbar_expect_tx(uvbar, bu + bv);
     bulk_g2s(smem + L.ubar, a.u_sigma + ((size_t)e * I + i0) * r, bu, uvbar);
     bulk_g2s(smem + L.vown, a.v + ((size_t)e * d + j0) * r, bv, uvbar);
   }
-  load_tokens(a, L, smem, misc, true);
-  __syncthreads();
+  if (!FUSED) {
+    int toks[NT];
+#pragma unroll
+    for (int t = 0; t < NT; t++) toks[t] = misc[MI_TOK + (t < n ? t : 0)];
+    load_x(a, L, smem, toks, n);
+    load_q(a, L, smem, toks, n);
+    if (tid < n) reinterpret_cast<float*>(misc + MI_CX)[tid] = __ldcg(&a.ws.cx[toks[tid]]);
+    __syncthreads();
+  }
+
+  float* sig = reinterpret_cast<float*>(smem + L.sig);        // [NT, I] pushed by the owners
+  float* ahat = reinterpret_cast<float*>(smem + L.ahat);      // [NT, I]
+  float* zparts = reinterpret_cast<float*>(smem + L.zparts);  // [cs, NT, r]
+  float* z = reinterpret_cast<float*>(smem + L.z);            // [NT, r]
+  float* apos = reinterpret_cast<float*>(smem + L.apos);      // [NT, I] by union position
+  uint32_t* candm = reinterpret_cast<uint32_t*>(smem + L.candm);
+  uint32_t* keptm = reinterpret_cast<uint32_t*>(smem + L.keptm);
+  uint32_t* pmask = reinterpret_cast<uint32_t*>(smem + L.pmask);
+  int* ulist = reinterpret_cast<int*>(smem + L.ulist);
+  int* upos = reinterpret_cast<int*>(smem + L.upos);
+  int* dlist = reinterpret_cast<int*>(smem + L.dlist);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.keys);
+  int* kidx = reinterpret_cast<int*>(smem + L.kidx);
+  const float* cxs = reinterpret_cast<const float*>(misc + MI_CX);
 
   // ---------------------------------------------------------- S: screen
   {
-    float* sig_own = reinterpret_cast<float*>(smem + L.sig_own);
-    float* ahat_own = reinterpret_cast<float*>(smem + L.ahat_own);
-    const float* cxs = reinterpret_cast<const float*>(misc) + MI_CX;
-    const int c0 = i0 + (warp * nown) / kWarps, c1 = i0 + ((warp + 1) * nown) / kWarps;
-    const int skrow = d / 4;                           // bytes per sketch row
-    const int per = max(1, (L.ring_bytes / 2) / (2 * skrow));  // channels per slot
-    const int nch = cdiv(c1 - c0, per);
+    const int c0 = i0 + (warp * nown) / NWARP, c1 = i0 + ((warp + 1) * nown) / NWARP;
+    const int skrow = d / 4;
+    const int half = L.ring_bytes / 2;
+    const int per = max(1, half / (2 * skrow));
     const int words = d / 16;
     const uint4* qs = reinterpret_cast<const uint4*>(smem + L.q);
+    const float* ag_row = a.alpha_gate + (size_t)e * I;
+    const float* au_row = a.alpha_up + (size_t)e * I;
     warp_stream(
-        nch, 2, wbars, par, err,
+        cdiv(c1 - c0, per), 2, wbars, par, err,
         [&](int j, int s, uint64_t* bar) {
           const int a0 = c0 + j * per, cnt = min(per, c1 - a0);
-          char* dst = ring + s * (L.ring_bytes / 2);
+          char* dst = ring + s * half;
           mbar_expect_tx(bar, 2 * cnt * skrow);
           bulk_g2s(dst, a.sk_gate + ((size_t)e * I + a0) * words, cnt * skrow, bar);
           bulk_g2s(dst + cnt * skrow, a.sk_up + ((size_t)e * I + a0) * words, cnt * skrow, bar);
         },
         [&](int j, int s) {
           const int a0 = c0 + j * per, cnt = min(per, c1 - a0);
-          const uint32_t* gw = reinterpret_cast<const uint32_t*>(ring + s * (L.ring_bytes / 2));
+          const uint32_t* gw = reinterpret_cast<const uint32_t*>(ring + s * half);
           const uint32_t* uw = gw + cnt * words;
           for (int ci = 0; ci < cnt; ci++) {
             const int i = a0 + ci;
-            int G[kMaxGroup], U[kMaxGroup];
+            int G[NT], U[NT];
 #pragma unroll
-            for (int t = 0; t < kMaxGroup; t++) G[t] = U[t] = 0;
+            for (int t = 0; t < NT; t++) G[t] = U[t] = 0;
             for (int w = lane; w < words; w += 32) {
-              const uint32_t g = gw[ci * words + w], u = uw[ci * words + w];
+              const uint4 tg = decode_trits(gw[ci * words + w]);
+              const uint4 tu = decode_trits(uw[ci * words + w]);
 #pragma unroll
-              for (int t = 0; t < kMaxGroup; t++) {
-                if (t < n) {
-                  const uint4 qv = qs[t * words + w];
-                  G[t] = trit_dot16(g, qv, G[t]);
-                  U[t] = trit_dot16(u, qv, U[t]);
-                }
+              for (int t = 0; t < NT; t++) {
+                const uint4 qv = qs[tix[t] * words + w];
+                G[t] = dot16_i8(tg, qv, G[t]);
+                U[t] = dot16_i8(tu, qv, U[t]);
               }
             }
-            const float ag = __ldg(&a.alpha_gate[(size_t)e * I + i]);
-            const float au = __ldg(&a.alpha_up[(size_t)e * I + i]);
+            const float ag = __ldg(ag_row + i), au = __ldg(au_row + i);
 #pragma unroll
-            for (int t = 0; t < kMaxGroup; t++) {
+            for (int t = 0; t < NT; t++) {
               if (t < n) {
                 const int gs = warp_sum(G[t]), us = warp_sum(U[t]);
-                if (lane == t) {
-                  const float gh = __fmul_rn(__fmul_rn((float)gs, ag), cxs[t]);
-                  const float uh = __fmul_rn(__fmul_rn((float)us, au), cxs[t]);
-                  const float ah = __fmul_rn(silu_r(gh), uh);
-                  sig_own[t * L.own + (i - i0)] = fabsf(ah);
-                  ahat_own[t * L.own + (i - i0)] = ah;
+                const float cx = cxs[tix[t]];
+                const float gh = __fmul_rn(__fmul_rn((float)gs, ag), cx);
+                const float uh = __fmul_rn(__fmul_rn((float)us, au), cx);
+                const float ah = __fmul_rn(silu_r(gh), uh);
+                if (lane < cs) {
+                  st_cluster(&sig[t * I + i], lane, fabsf(ah));
+                  st_cluster(&ahat[t * I + i], lane, ah);
+                }
+                if (lane == 31) {
                   const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * I + i;
                   if (a.dbg_G) a.dbg_G[off] = gs;
                   if (a.dbg_U) a.dbg_U[off] = us;
@@ -440,87 +734,59 @@ __global__ void __launch_bounds__(kThreads, 1) reader_kernel(ExpertArgs a) {
             }
           }
         });
+    // partial recovery input over the own channels, pushed to every CTA:
+    // zparts[rank][t] = sum_{own i} ahat_i Ubar_i.  The local ahat of the own
+    // channels was written by this CTA's own stores above.
     __syncthreads();
-    // partial recovery input over the own channels: zpart[t] = sum ahat_i Ubar_i
     if (r > 0) {
-      if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_ERR] = 1;
+      if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
       const uint16_t* ub = reinterpret_cast<const uint16_t*>(smem + L.ubar);
-      float* zpart = reinterpret_cast<float*>(smem + L.zpart);
-      for (int idx = tid; idx < n * r; idx += kThreads) {
-        const int t = idx / r, p = idx % r;
-        float z = 0.0f;
-        for (int li = 0; li < nown; li++) z = fmaf(ahat_own[t * L.own + li], bf16f(ub[li * r + p]), z);
-        zpart[idx] = z;
+      for (int idx = tid; idx < n * r; idx += NTHR) {
+        const int t = idx / r, p = idx - t * r;
+        float zz = 0.0f;
+        for (int li = 0; li < nown; li++) zz = fmaf(ahat[t * I + i0 + li], bf16f(ub[li * r + p]), zz);
+        for (int o = 0; o < cs; o++) st_cluster(&zparts[(rank * NT + t) * r + p], o, zz);
       }
     }
   }
   cluster.sync();
 
-  // ---------------------------------------------- c: gather sigma, top-c
-  float* sig_all = reinterpret_cast<float*>(smem + L.sig_all);  // later: a by U position
-  float* ahat_all = reinterpret_cast<float*>(smem + L.ahat_all);
-  float* z_all = reinterpret_cast<float*>(smem + L.z_all);
-  uint32_t* candm = reinterpret_cast<uint32_t*>(smem + L.candm);
-  uint32_t* keptm = reinterpret_cast<uint32_t*>(smem + L.keptm);
-  int* ulist = reinterpret_cast<int*>(smem + L.ulist);
-  int* upos = reinterpret_cast<int*>(smem + L.upos);
-  int* dlist = reinterpret_cast<int*>(smem + L.dlist);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.keys);
-  int* kidx = reinterpret_cast<int*>(smem + L.kidx);
-  float* a_own = reinterpret_cast<float*>(smem + L.a_own);
-  {
-    const float* so = reinterpret_cast<const float*>(smem + L.sig_own);
-    const float* ao = reinterpret_cast<const float*>(smem + L.ahat_own);
-    for (int idx = tid; idx < n * I; idx += kThreads) {
-      const int t = idx / I, i = idx % I;
-      const int o = (i * cs) / I, li = i - cdiv(o * I, cs);
-      sig_all[idx] = cluster.map_shared_rank(so, o)[t * L.own + li];
-      ahat_all[idx] = cluster.map_shared_rank(ao, o)[t * L.own + li];
-    }
-    if (r > 0) {
-      const float* zp = reinterpret_cast<const float*>(smem + L.zpart);
-      for (int idx = tid; idx < n * r; idx += kThreads) {
-        float z = 0.0f;
-        for (int o = 0; o < cs; o++) z += cluster.map_shared_rank(zp, o)[idx];
-        z_all[idx] = z;
-      }
-    }
-  }
-  __syncthreads();
+  // ---------------------------------------------------------- c: top-c
   for (int t = 0; t < n; t++)
-    block_select_top(reinterpret_cast<const uint32_t*>(sig_all + t * I), I, a.c, hist, misc,
+    block_select_top(reinterpret_cast<const uint32_t*>(sig + t * I), I, a.c, hist, wtot, misc,
                      candm + t * L.words);
+  for (int idx = tid; idx < n * r; idx += NTHR) {
+    const int t = idx / r, p = idx - t * r;
+    float zz = 0.0f;
+    for (int o = 0; o < cs; o++) zz += zparts[(o * NT + t) * r + p];
+    z[idx] = zz;
+  }
   // union of the candidates, ascending
-  if (warp == 0) {
-    uint32_t* um = keys;  // scratch mask
-    for (int w = lane; w < L.words; w += 32) {
-      uint32_t m = 0;
-      for (int t = 0; t < n; t++) m |= candm[t * L.words + w];
-      um[w] = m;
-    }
-    __syncwarp();
-    warp_mask_to_list(um, I, ulist, upos, &misc[MI_NU]);
-    if (a.dbg_cand && rank == 0) {
-      for (int t = 0; t < n; t++) {
-        int base = 0;
-        int* out = a.dbg_cand + ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.c;
-        for (int w0 = 0; w0 < I; w0 += 32) {
-          const int p = w0 + lane;
-          const bool on = p < I && ((candm[t * L.words + (w0 >> 5)] >> lane) & 1u);
-          const unsigned bal = __ballot_sync(0xffffffffu, on);
-          if (on) out[base + __popc(bal & ((1u << lane) - 1u))] = p;
-          base += __popc(bal);
-        }
-      }
-    }
+  for (int w = tid; w < L.words; w += NTHR) {
+    uint32_t m = 0;
+    for (int t = 0; t < n; t++) m |= candm[t * L.words + w];
+    pmask[w] = m;
   }
   __syncthreads();
+  block_mask_to_list(pmask, I, ulist, upos, &misc[MI_NU]);
+  if (a.dbg_cand && rank == 0 && warp < n) {
+    const int t = warp;
+    int base = 0;
+    int* out = a.dbg_cand + ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.c;
+    for (int w0 = 0; w0 < I; w0 += 32) {
+      const int p = w0 + lane;
+      const bool on = p < I && ((candm[t * L.words + (w0 >> 5)] >> lane) & 1u);
+      const unsigned bal = __ballot_sync(0xffffffffu, on);
+      if (on) out[base + __popc(bal & ((1u << lane) - 1u))] = p;
+      base += __popc(bal);
+    }
+  }
   const int nU = misc[MI_NU];
 
   // -------------------------------------------- C: exact candidate stage
   {
     const int u0 = cdiv(rank * nU, cs), u1 = cdiv((rank + 1) * nU, cs), nsl = u1 - u0;
-    const int m0 = (warp * nsl) / kWarps, m1 = ((warp + 1) * nsl) / kWarps;
+    const int m0 = (warp * nsl) / NWARP, m1 = ((warp + 1) * nsl) / NWARP;
     const int rowb = d * 2;
     const int P = max(1, min(kMaxSlots, L.ring_bytes / (2 * rowb)));
     const uint4* xs = reinterpret_cast<const uint4*>(smem + L.x);
@@ -535,50 +801,41 @@ __global__ void __launch_bounds__(kThreads, 1) reader_kernel(ExpertArgs a) {
           bulk_g2s(dst + rowb, a.w_up + ((size_t)e * I + i) * d, rowb, bar);
         },
         [&](int j, int s) {
-          const int m = m0 + j, i = ulist[u0 + m];
+          const int u = u0 + m0 + j, i = ulist[u];
           const uint4* gr = reinterpret_cast<const uint4*>(ring + s * 2 * rowb);
           const uint4* ur = gr + vx;
-          float g[kMaxGroup], u[kMaxGroup];
+          float g0[NT], g1[NT], v0[NT], v1[NT];
 #pragma unroll
-          for (int t = 0; t < kMaxGroup; t++) g[t] = u[t] = 0.0f;
-          for (int v = lane; v < vx; v += 32) {
-            const uint4 gv = gr[v], uv = ur[v];
+          for (int t = 0; t < NT; t++) g0[t] = g1[t] = v0[t] = v1[t] = 0.0f;
+          for (int vv = lane; vv < vx; vv += 32) {
+            const uint4 gv = gr[vv], uv = ur[vv];
 #pragma unroll
-            for (int t = 0; t < kMaxGroup; t++)
-              if (t < n) {
-                const uint4 xv = xs[t * vx + v];
-                g[t] = dot8_bf16(gv, xv, g[t]);
-                u[t] = dot8_bf16(uv, xv, u[t]);
-              }
+            for (int t = 0; t < NT; t++) {
+              const uint4 xv = xs[tix[t] * vx + vv];
+              dot8_mixed(gv, xv, g0[t], g1[t]);
+              dot8_mixed(uv, xv, v0[t], v1[t]);
+            }
           }
 #pragma unroll
-          for (int t = 0; t < kMaxGroup; t++)
+          for (int t = 0; t < NT; t++) {
             if (t < n) {
-              const float gs = warp_sum(g[t]), us = warp_sum(u[t]);
-              if (lane == t) {
-                const bool is_c = (candm[t * L.words + (i >> 5)] >> (i & 31)) & 1u;
-                a_own[t * L.own + m] = is_c ? __fmul_rn(silu_r(gs), us) : 0.0f;
-              }
+              const float gs = warp_sum(g0[t] + g1[t]), us = warp_sum(v0[t] + v1[t]);
+              const bool is_c = (candm[t * L.words + (i >> 5)] >> (i & 31)) & 1u;
+              const float av = is_c ? __fmul_rn(silu_r(gs), us) : 0.0f;
+              if (lane < cs) st_cluster(&apos[t * I + u], lane, av);
             }
+          }
         });
   }
-  cluster.sync();
+  cluster.sync();  // the last exchange: no CTA touches another's smem after this
 
-  // ------------------------------------------------ k: gather a, top-k
-  float* a_all = sig_all;  // [n, nU] by U position
-  for (int idx = tid; idx < n * nU; idx += kThreads) {
-    const int t = idx / nU, u = idx % nU;
-    const int o = (u * cs) / nU, lu = u - cdiv(o * nU, cs);
-    a_all[t * nU + u] = cluster.map_shared_rank(a_own, o)[t * L.own + lu];
-  }
-  cluster_arrive();  // no remote reads past this point
-  __syncthreads();
+  // ------------------------------------------------------------ k: top-k
   for (int t = 0; t < n; t++) {
     // the token's candidates in ascending channel order, key |a|
     if (warp == 0) {
       int base = 0;
-      for (int u0 = 0; u0 < nU; u0 += 32) {
-        const int u = u0 + lane;
+      for (int w0 = 0; w0 < nU; w0 += 32) {
+        const int u = w0 + lane;
         bool on = false;
         int i = 0;
         if (u < nU) {
@@ -588,88 +845,76 @@ __global__ void __launch_bounds__(kThreads, 1) reader_kernel(ExpertArgs a) {
         const unsigned bal = __ballot_sync(0xffffffffu, on);
         if (on) {
           const int at = base + __popc(bal & ((1u << lane) - 1u));
-          keys[at] = __float_as_uint(fabsf(a_all[t * nU + u]));
+          keys[at] = __float_as_uint(fabsf(apos[t * I + u]));
           kidx[at] = i;
         }
         base += __popc(bal);
       }
-      if (lane == 0) misc[MI_ND] = base;  // = c
+      if (lane == 0) misc[MI_NC] = base;  // = c
     }
     __syncthreads();
-    // select k of the c candidates: a mask over the compact positions,
-    // remapped to channel bits below
-    block_select_top(keys, misc[MI_ND], a.k, hist, misc, keptm + t * L.words);
-    // remap compact positions -> channel bits (in place through a scratch pass)
-    if (warp == 0) {
-      const int c = misc[MI_ND];
-      int* tmp = dlist;  // scratch list of kept channels
+    const int c = misc[MI_NC];
+    uint32_t* km = keptm + t * L.words;
+    block_select_top(keys, c, a.k, hist, wtot, misc, pmask);  // over compact positions
+    for (int w = tid; w < L.words; w += NTHR) km[w] = 0u;
+    __syncthreads();
+    for (int p = tid; p < c; p += NTHR)
+      if ((pmask[p >> 5] >> (p & 31)) & 1u) atomicOr(&km[kidx[p] >> 5], 1u << (kidx[p] & 31));
+    __syncthreads();
+    if (a.dbg_kept && rank == 0 && warp == 0) {
+      const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.k;
       int base = 0;
-      for (int p0 = 0; p0 < c; p0 += 32) {
-        const int p = p0 + lane;
-        const bool on = p < c && ((keptm[t * L.words + (p0 >> 5)] >> lane) & 1u);
+      for (int w0 = 0; w0 < I; w0 += 32) {
+        const int i = w0 + lane;
+        const bool on = i < I && ((km[w0 >> 5] >> lane) & 1u);
         const unsigned bal = __ballot_sync(0xffffffffu, on);
-        if (on) tmp[base + __popc(bal & ((1u << lane) - 1u))] = kidx[p];
+        const int at = base + __popc(bal & ((1u << lane) - 1u));
+        if (on && at < a.k) {
+          a.dbg_kept[off + at] = i;
+          if (a.dbg_a_kept) a.dbg_a_kept[off + at] = apos[t * I + upos[i]];
+        }
         base += __popc(bal);
       }
-      __syncwarp();
-      for (int w = lane; w < L.words; w += 32) keptm[t * L.words + w] = 0u;
-      __syncwarp();
-      for (int q = lane; q < base; q += 32) atomicOr(&keptm[t * L.words + (tmp[q] >> 5)], 1u << (tmp[q] & 31));
-      __syncwarp();
-      if (a.dbg_kept && rank == 0) {
-        const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.k;
-        for (int q = lane; q < base && q < a.k; q += 32) {
-          a.dbg_kept[off + q] = tmp[q];
-          if (a.dbg_a_kept) a.dbg_a_kept[off + q] = a_all[t * nU + upos[tmp[q]]];
-        }
-      }
     }
-    __syncthreads();
   }
   // union of the kept channels
-  if (warp == 0) {
-    uint32_t* um = keys;
-    for (int w = lane; w < L.words; w += 32) {
-      uint32_t m = 0;
-      for (int t = 0; t < n; t++) m |= keptm[t * L.words + w];
-      um[w] = m;
-    }
-    __syncwarp();
-    warp_mask_to_list(um, I, dlist, nullptr, &misc[MI_ND]);
+  for (int w = tid; w < L.words; w += NTHR) {
+    uint32_t m = 0;
+    for (int t = 0; t < n; t++) m |= keptm[t * L.words + w];
+    pmask[w] = m;
   }
   __syncthreads();
+  block_mask_to_list(pmask, I, dlist, nullptr, &misc[MI_ND]);
   const int nD = misc[MI_ND];
 
   // ---------------------------------------------- D: down rows + recovery
   {
-    const int colb = L.cols * 2, ub = r * 2;
-    const int eb = rup(colb + ub, 16);
-    const int m0 = (warp * nD) / kWarps, m1 = ((warp + 1) * nD) / kWarps, cnt = m1 - m0;
-    const int cap = max(1, L.ring_bytes / eb);  // elements resident per warp
+    const int colb = ncols * 2, ubb = r * 2;
+    const int eb = rup(colb + ubb, 16);
+    const int m0 = (warp * nD) / NWARP, m1 = ((warp + 1) * nD) / NWARP, cnt = m1 - m0;
+    const int cap = max(1, L.ring_bytes / eb);
     int P = min(kMaxSlots, max(1, cnt));
     int per = max(1, min(cdiv(cnt, P), cap / P));
     if (per * P > cap) P = max(1, cap / per);
-    const int ngroups = cdiv(cnt, per);
-    const int ncl = cdiv(L.cols, 128);  // column groups of 4 per lane
-    float acc[kMaxGroup][8];
-    float cor[kMaxGroup][4];
+    float acc[NT][8];
+    float cor[NT][4];
 #pragma unroll
-    for (int t = 0; t < kMaxGroup; t++) {
+    for (int t = 0; t < NT; t++) {
 #pragma unroll
       for (int q = 0; q < 8; q++) acc[t][q] = 0.0f;
 #pragma unroll
       for (int q = 0; q < 4; q++) cor[t][q] = 0.0f;
     }
     warp_stream(
-        ngroups, P, wbars, par, err,
+        cdiv(cnt, per), P, wbars, par, err,
         [&](int j, int s, uint64_t* bar) {
           const int g0 = m0 + j * per, gc = min(per, m1 - g0);
           char* dst = ring + s * per * eb;
-          mbar_expect_tx(bar, gc * (colb + ub));
+          mbar_expect_tx(bar, gc * (colb + ubb));
           for (int q = 0; q < gc; q++) {
             const int i = dlist[g0 + q];
             bulk_g2s(dst + q * eb, a.w_down + ((size_t)e * I + i) * d + j0, colb, bar);
-            if (r > 0) bulk_g2s(dst + q * eb + colb, a.u_sigma + ((size_t)e * I + i) * r, ub, bar);
+            if (r > 0) bulk_g2s(dst + q * eb + colb, a.u_sigma + ((size_t)e * I + i) * r, ubb, bar);
           }
         },
         [&](int j, int s) {
@@ -677,30 +922,27 @@ __global__ void __launch_bounds__(kThreads, 1) reader_kernel(ExpertArgs a) {
           const char* src = ring + s * per * eb;
           for (int q = 0; q < gc; q++) {
             const int i = dlist[g0 + q];
-            float co[kMaxGroup], ch[kMaxGroup];
+            float co[NT], ch[NT];
 #pragma unroll
-            for (int t = 0; t < kMaxGroup; t++) {
-              co[t] = ch[t] = 0.0f;
-              if (t < n && ((keptm[t * L.words + (i >> 5)] >> (i & 31)) & 1u)) {
-                co[t] = a_all[t * nU + upos[i]];
-                ch[t] = ahat_all[t * I + i];
-              }
+            for (int t = 0; t < NT; t++) {
+              const bool kept = t < n && ((keptm[t * L.words + (i >> 5)] >> (i & 31)) & 1u);
+              co[t] = kept ? apos[t * I + upos[i]] : 0.0f;
+              ch[t] = kept ? ahat[t * I + i] : 0.0f;
             }
             const uint16_t* wd = reinterpret_cast<const uint16_t*>(src + q * eb);
 #pragma unroll
             for (int cg4 = 0; cg4 < 2; cg4++) {
               const int c4 = 4 * lane + 128 * cg4;
-              if (cg4 < ncl && c4 < L.cols) {
+              if (c4 < ncols) {
                 const uint2 wv = *reinterpret_cast<const uint2*>(wd + c4);
                 const float w0 = bf16lo(wv.x), w1 = bf16hi(wv.x), w2 = bf16lo(wv.y), w3 = bf16hi(wv.y);
 #pragma unroll
-                for (int t = 0; t < kMaxGroup; t++)
-                  if (t < n) {
-                    acc[t][4 * cg4 + 0] = fmaf(co[t], w0, acc[t][4 * cg4 + 0]);
-                    acc[t][4 * cg4 + 1] = fmaf(co[t], w1, acc[t][4 * cg4 + 1]);
-                    acc[t][4 * cg4 + 2] = fmaf(co[t], w2, acc[t][4 * cg4 + 2]);
-                    acc[t][4 * cg4 + 3] = fmaf(co[t], w3, acc[t][4 * cg4 + 3]);
-                  }
+                for (int t = 0; t < NT; t++) {
+                  acc[t][4 * cg4 + 0] = fmaf(co[t], w0, acc[t][4 * cg4 + 0]);
+                  acc[t][4 * cg4 + 1] = fmaf(co[t], w1, acc[t][4 * cg4 + 1]);
+                  acc[t][4 * cg4 + 2] = fmaf(co[t], w2, acc[t][4 * cg4 + 2]);
+                  acc[t][4 * cg4 + 3] = fmaf(co[t], w3, acc[t][4 * cg4 + 3]);
+                }
               }
             }
             if (r > 0) {
@@ -711,92 +953,101 @@ __global__ void __launch_bounds__(kThreads, 1) reader_kernel(ExpertArgs a) {
                 if (p < r) {
                   const float uv = bf16f(ur[p]);
 #pragma unroll
-                  for (int t = 0; t < kMaxGroup; t++)
-                    if (t < n) cor[t][kk] = fmaf(ch[t], uv, cor[t][kk]);
+                  for (int t = 0; t < NT; t++) cor[t][kk] = fmaf(ch[t], uv, cor[t][kk]);
                 }
               }
             }
           }
         });
-    // per-warp partials into the warp's own ring area (its copies are done)
     __syncwarp();
-    float* part = reinterpret_cast<float*>(ring);            // [n, cols]
-    float* cpart = part + n * L.cols;                        // [n, r]
+    float* part = reinterpret_cast<float*>(ring);  // [NT, cols_max] then [NT, r]
+    float* cpart = part + NT * L.cols_max;
 #pragma unroll
-    for (int t = 0; t < kMaxGroup; t++)
-      if (t < n) {
+    for (int t = 0; t < NT; t++) {
 #pragma unroll
-        for (int cg4 = 0; cg4 < 2; cg4++) {
-          const int c4 = 4 * lane + 128 * cg4;
-          if (cg4 < ncl && c4 < L.cols) {
+      for (int cg4 = 0; cg4 < 2; cg4++) {
+        const int c4 = 4 * lane + 128 * cg4;
+        if (c4 < ncols) {
 #pragma unroll
-            for (int q = 0; q < 4; q++) part[t * L.cols + c4 + q] = acc[t][4 * cg4 + q];
-          }
-        }
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++) {
-          const int p = lane + 32 * kk;
-          if (p < r) cpart[t * r + p] = cor[t][kk];
+          for (int q = 0; q < 4; q++) part[t * L.cols_max + c4 + q] = acc[t][4 * cg4 + q];
         }
       }
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) {
+        const int p = lane + 32 * kk;
+        if (p < r) cpart[t * r + p] = cor[t][kk];
+      }
+    }
   }
   __syncthreads();
-  float* yfin = reinterpret_cast<float*>(smem + L.x);  // [n, cols]; x is no longer needed
+  float* yfin = reinterpret_cast<float*>(smem + L.x);  // [n, ncols]; x is no longer needed
+  for (int idx = tid; idx < n * r; idx += NTHR) {
+    const int t = idx / r, p = idx - t * r;
+    float cc = 0.0f;
+    for (int w = 0; w < NWARP; w++)
+      cc += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[NT * L.cols_max + t * r + p];
+    z[idx] -= cc;
+  }
+  __syncthreads();
   {
-    for (int idx = tid; idx < n * r; idx += kThreads) {
-      const int t = idx / r, p = idx % r;
-      float c = 0.0f;
-      for (int w = 0; w < kWarps; w++) {
-        const float* part = reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes);
-        c += part[n * L.cols + t * r + p];
-      }
-      z_all[idx] -= c;
-    }
-    __syncthreads();
     const uint16_t* vo = reinterpret_cast<const uint16_t*>(smem + L.vown);
-    for (int idx = tid; idx < n * L.cols; idx += kThreads) {
-      const int t = idx / L.cols, col = idx % L.cols;
+    for (int idx = tid; idx < n * ncols; idx += NTHR) {
+      const int t = idx / ncols, col = idx - t * ncols;
       float y = 0.0f;
-      for (int w = 0; w < kWarps; w++) y += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[idx];
+      for (int w = 0; w < NWARP; w++)
+        y += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[t * L.cols_max + col];
       float rec = 0.0f;
-      for (int p = 0; p < r; p++) rec = fmaf(bf16f(vo[col * r + p]), z_all[t * r + p], rec);
+      for (int p = 0; p < r; p++) rec = fmaf(bf16f(vo[col * r + p]), z[t * r + p], rec);
       yfin[idx] = y + rec;
     }
   }
   __syncthreads();
-  write_and_combine(a, L, rank, yfin, misc);
-  cluster_wait();
+  write_and_combine(a, rank, j0, ncols, yfin, misc,
+                    FUSED ? reinterpret_cast<const float*>(misc + MI_RW) : a.ws.wts);
 }
 
 // ================================================================= dense
-__global__ void __launch_bounds__(kThreads, 1) dense_kernel(ExpertArgs a) {
+template <int NT, bool FUSED>
+__global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) {
   extern __shared__ __align__(128) char smem[];
   cg::cluster_group cluster = cg::this_cluster();
-  const int cs = a.cs;
+  const int cs = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
   const int cid = blockIdx.x / cs;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const Layout L = make_layout(a.nmax, a.I, a.d, a.r, cs, a.ring_rows, true);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.mbar);
   uint64_t* wbars = bars + warp * kMaxSlots;
+  uint64_t* wrbar = bars + NWARP * kMaxSlots + 1;
   int* misc = reinterpret_cast<int*>(smem + L.misc);
-  if (tid < kWarps * kMaxSlots) mbar_init(&bars[tid], 1);
+  if (tid < NWARP * kMaxSlots + 2) mbar_init(&bars[tid], 1);
+  if (tid == 0) misc[MI_DONE] = 0;
   fence_mbar_init();
   __syncthreads();
-  pdl_wait();
-  if (!load_item(a, cid, misc)) return;
+  if (FUSED) {
+    if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, wrbar, cluster)) return;
+  } else {
+    pdl_wait();
+    if (!load_item_table(a, cid, misc, NT)) return;
+    int toks[NT];
+#pragma unroll
+    for (int t = 0; t < NT; t++) toks[t] = misc[MI_TOK + (t < misc[MI_N] ? t : 0)];
+    load_x(a, L, smem, toks, misc[MI_N]);
+    __syncthreads();
+  }
   const int e = misc[MI_E], n = misc[MI_N];
   const int I = a.I, d = a.d;
   const int i0 = cdiv(rank * I, cs), i1 = cdiv((rank + 1) * I, cs), nown = i1 - i0;
-  const int j0 = rank * L.cols;
+  int j0, ncols;
+  col_slice(d, cs, rank, j0, ncols);
   uint32_t* err = a.ws.err;
   uint32_t par = 0;
   char* ring = smem + L.ring + warp * L.ring_bytes;
-  load_tokens(a, L, smem, misc, false);
-  __syncthreads();
-  float* h_own = reinterpret_cast<float*>(smem + L.sig_own);
+  int tix[NT];
+#pragma unroll
+  for (int t = 0; t < NT; t++) tix[t] = misc[MI_TIX + (t < n ? t : 0)];
+  float* h = reinterpret_cast<float*>(smem + L.sig);  // [NT, I] pushed by the owners
   {
-    const int m0 = (warp * nown) / kWarps, m1 = ((warp + 1) * nown) / kWarps;
+    const int m0 = (warp * nown) / NWARP, m1 = ((warp + 1) * nown) / NWARP;
     const int rowb = d * 2, vx = d / 8;
     const int P = max(1, min(kMaxSlots, L.ring_bytes / (2 * rowb)));
     const uint4* xs = reinterpret_cast<const uint4*>(smem + L.x);
@@ -810,56 +1061,46 @@ __global__ void __launch_bounds__(kThreads, 1) dense_kernel(ExpertArgs a) {
           bulk_g2s(dst + rowb, a.w_up + ((size_t)e * I + i) * d, rowb, bar);
         },
         [&](int j, int s) {
-          const int m = m0 + j;
+          const int i = i0 + m0 + j;
           const uint4* gr = reinterpret_cast<const uint4*>(ring + s * 2 * rowb);
           const uint4* ur = gr + vx;
-          float g[kMaxGroup], u[kMaxGroup];
+          float g0[NT], g1[NT], v0[NT], v1[NT];
 #pragma unroll
-          for (int t = 0; t < kMaxGroup; t++) g[t] = u[t] = 0.0f;
-          for (int v = lane; v < vx; v += 32) {
-            const uint4 gv = gr[v], uv = ur[v];
+          for (int t = 0; t < NT; t++) g0[t] = g1[t] = v0[t] = v1[t] = 0.0f;
+          for (int vv = lane; vv < vx; vv += 32) {
+            const uint4 gv = gr[vv], uv = ur[vv];
 #pragma unroll
-            for (int t = 0; t < kMaxGroup; t++)
-              if (t < n) {
-                const uint4 xv = xs[t * vx + v];
-                g[t] = dot8_bf16(gv, xv, g[t]);
-                u[t] = dot8_bf16(uv, xv, u[t]);
-              }
+            for (int t = 0; t < NT; t++) {
+              const uint4 xv = xs[tix[t] * vx + vv];
+              dot8_mixed(gv, xv, g0[t], g1[t]);
+              dot8_mixed(uv, xv, v0[t], v1[t]);
+            }
           }
 #pragma unroll
-          for (int t = 0; t < kMaxGroup; t++)
+          for (int t = 0; t < NT; t++) {
             if (t < n) {
-              const float gs = warp_sum(g[t]), us = warp_sum(u[t]);
-              if (lane == t) h_own[t * L.own + m] = __fmul_rn(silu_r(gs), us);
+              const float gs = warp_sum(g0[t] + g1[t]), us = warp_sum(v0[t] + v1[t]);
+              if (lane < cs) st_cluster(&h[t * I + i], lane, __fmul_rn(silu_r(gs), us));
             }
+          }
         });
   }
-  cluster.sync();
-  float* h_all = reinterpret_cast<float*>(smem + L.sig_all);
-  for (int idx = tid; idx < n * I; idx += kThreads) {
-    const int t = idx / I, i = idx % I;
-    const int o = (i * cs) / I, li = i - cdiv(o * I, cs);
-    h_all[idx] = cluster.map_shared_rank(h_own, o)[t * L.own + li];
-  }
-  cluster_arrive();
-  __syncthreads();
+  cluster.sync();  // the only exchange: no CTA touches another's smem after this
   {
-    const int colb = L.cols * 2;
+    const int colb = ncols * 2;
     const int eb = rup(colb, 16);
-    const int m0 = (warp * I) / kWarps, m1 = ((warp + 1) * I) / kWarps, cnt = m1 - m0;
+    const int m0 = (warp * I) / NWARP, m1 = ((warp + 1) * I) / NWARP, cnt = m1 - m0;
     const int cap = max(1, L.ring_bytes / eb);
     int P = min(kMaxSlots, max(1, cnt));
     int per = max(1, min(cdiv(cnt, P), cap / P));
     if (per * P > cap) P = max(1, cap / per);
-    const int ngroups = cdiv(cnt, per);
-    const int ncl = cdiv(L.cols, 128);
-    float acc[kMaxGroup][8];
+    float acc[NT][8];
 #pragma unroll
-    for (int t = 0; t < kMaxGroup; t++)
+    for (int t = 0; t < NT; t++)
 #pragma unroll
       for (int q = 0; q < 8; q++) acc[t][q] = 0.0f;
     warp_stream(
-        ngroups, P, wbars, par, err,
+        cdiv(cnt, per), P, wbars, par, err,
         [&](int j, int s, uint64_t* bar) {
           const int g0 = m0 + j * per, gc = min(per, m1 - g0);
           char* dst = ring + s * per * eb;
@@ -872,24 +1113,23 @@ __global__ void __launch_bounds__(kThreads, 1) dense_kernel(ExpertArgs a) {
           const char* src = ring + s * per * eb;
           for (int q = 0; q < gc; q++) {
             const int i = g0 + q;
-            float co[kMaxGroup];
+            float co[NT];
 #pragma unroll
-            for (int t = 0; t < kMaxGroup; t++) co[t] = t < n ? h_all[t * I + i] : 0.0f;
+            for (int t = 0; t < NT; t++) co[t] = t < n ? h[t * I + i] : 0.0f;
             const uint16_t* wd = reinterpret_cast<const uint16_t*>(src + q * eb);
 #pragma unroll
             for (int cg4 = 0; cg4 < 2; cg4++) {
               const int c4 = 4 * lane + 128 * cg4;
-              if (cg4 < ncl && c4 < L.cols) {
+              if (c4 < ncols) {
                 const uint2 wv = *reinterpret_cast<const uint2*>(wd + c4);
                 const float w0 = bf16lo(wv.x), w1 = bf16hi(wv.x), w2 = bf16lo(wv.y), w3 = bf16hi(wv.y);
 #pragma unroll
-                for (int t = 0; t < kMaxGroup; t++)
-                  if (t < n) {
-                    acc[t][4 * cg4 + 0] = fmaf(co[t], w0, acc[t][4 * cg4 + 0]);
-                    acc[t][4 * cg4 + 1] = fmaf(co[t], w1, acc[t][4 * cg4 + 1]);
-                    acc[t][4 * cg4 + 2] = fmaf(co[t], w2, acc[t][4 * cg4 + 2]);
-                    acc[t][4 * cg4 + 3] = fmaf(co[t], w3, acc[t][4 * cg4 + 3]);
-                  }
+                for (int t = 0; t < NT; t++) {
+                  acc[t][4 * cg4 + 0] = fmaf(co[t], w0, acc[t][4 * cg4 + 0]);
+                  acc[t][4 * cg4 + 1] = fmaf(co[t], w1, acc[t][4 * cg4 + 1]);
+                  acc[t][4 * cg4 + 2] = fmaf(co[t], w2, acc[t][4 * cg4 + 2]);
+                  acc[t][4 * cg4 + 3] = fmaf(co[t], w3, acc[t][4 * cg4 + 3]);
+                }
               }
             }
           }
@@ -897,66 +1137,71 @@ __global__ void __launch_bounds__(kThreads, 1) dense_kernel(ExpertArgs a) {
     __syncwarp();
     float* part = reinterpret_cast<float*>(ring);
 #pragma unroll
-    for (int t = 0; t < kMaxGroup; t++)
-      if (t < n) {
+    for (int t = 0; t < NT; t++) {
 #pragma unroll
-        for (int cg4 = 0; cg4 < 2; cg4++) {
-          const int c4 = 4 * lane + 128 * cg4;
-          if (cg4 < ncl && c4 < L.cols) {
+      for (int cg4 = 0; cg4 < 2; cg4++) {
+        const int c4 = 4 * lane + 128 * cg4;
+        if (c4 < ncols) {
 #pragma unroll
-            for (int q = 0; q < 4; q++) part[t * L.cols + c4 + q] = acc[t][4 * cg4 + q];
-          }
+          for (int q = 0; q < 4; q++) part[t * L.cols_max + c4 + q] = acc[t][4 * cg4 + q];
         }
       }
+    }
   }
   __syncthreads();
-  float* out = reinterpret_cast<float*>(smem + L.x);  // [n, cols]; x is no longer needed
-  for (int idx = tid; idx < n * L.cols; idx += kThreads) {
+  float* out = reinterpret_cast<float*>(smem + L.x);
+  for (int idx = tid; idx < n * ncols; idx += NTHR) {
+    const int t = idx / ncols, col = idx - t * ncols;
     float y = 0.0f;
-    for (int w = 0; w < kWarps; w++) y += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[idx];
+    for (int w = 0; w < NWARP; w++)
+      y += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[t * L.cols_max + col];
     out[idx] = y;
   }
   __syncthreads();
-  write_and_combine(a, L, rank, out, misc);
-  cluster_wait();
+  write_and_combine(a, rank, j0, ncols, out, misc, FUSED ? reinterpret_cast<const float*>(misc + MI_RW) : a.ws.wts);
 }
 
-// Largest ring that fits; at least two rows per warp, and room for the
-// per-warp partial sums [n, cols + r] fp32 that the down stage leaves there.
-int pick_ring_rows(const ExpertArgs& a, bool dense, int smem_max) {
-  const int need = a.nmax * (a.d / a.cs + a.r) * 4;
-  const int min_rows = max(2, cdiv(need, 2 * a.d));
-  int best = 0;
-  for (int rr = min_rows; rr <= 64; rr++) {
-    const Layout L = make_layout(a.nmax, a.I, a.d, a.r, a.cs, rr, dense);
-    if (L.total <= smem_max) best = rr;
-    else break;
-  }
-  return best;
-}
-
+// ---------------------------------------------------------- launch plans
 struct LaunchPlan {
-  int dev, dense, nmax, I, d, r, items, forced;
+  int dev, dense, NT, fused, B, E, I, d, r, items, forced;
   int cs, ring_rows, smem, max_clusters;
+  Layout L;
 };
 
 int g_forced_cs = 0;  // 0: automatic
 
-// Cluster size: among 16, 8, 4 (those that fit this shape), the one that
-// keeps the most SMs busy on this launch, min(items, co-resident clusters)
-// * cs, ties to the larger cluster.  Ring depth: the deepest that fits.
-// Cached per shape and device.
+template <int NT, bool FUSED>
+const void* kernel_ptr(bool dense) {
+  return dense ? reinterpret_cast<const void*>(&dense_kernel<NT, FUSED>)
+               : reinterpret_cast<const void*>(&reader_kernel<NT, FUSED>);
+}
+const void* pick_kernel(bool dense, int NT, bool fused) {
+  switch (NT) {
+    case 1: return fused ? kernel_ptr<1, true>(dense) : kernel_ptr<1, false>(dense);
+    case 2: return fused ? kernel_ptr<2, true>(dense) : kernel_ptr<2, false>(dense);
+    case 4: return fused ? kernel_ptr<4, true>(dense) : kernel_ptr<4, false>(dense);
+    default: return kernel_ptr<8, false>(dense);
+  }
+}
+
+// Cluster size: among 8..16 (those that fit this shape), the one with the
+// fewest waves per CTA of width, ceil(items / co-resident clusters) / cs,
+// ties to the larger cluster.  Ring: the deepest that fits, with room for the
+// per-warp partial sums [NT, cols + r] fp32 of the down stage (and, with the
+// fused router, for the CTA's router rows and an fp32 transform scratch).
 cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
   thread_local LaunchPlan cache[16];
   thread_local int ncache = 0, next = 0;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  const int items = a.ws.max_items;
+  const int NT = a.nmax <= 1 ? 1 : a.nmax <= 2 ? 2 : a.nmax <= 4 ? 4 : 8;
+  const bool fused = fused_routing(a.B);
+  const int items = fused ? (a.B * a.top_e < a.E ? a.B * a.top_e : a.E) : a.ws.max_items;
   for (int i = 0; i < ncache; i++) {
     const LaunchPlan& c = cache[i];
-    if (c.dev == dev && c.dense == (int)dense && c.nmax == a.nmax && c.I == a.I && c.d == a.d && c.r == a.r &&
-        c.items == items && c.forced == g_forced_cs) {
+    if (c.dev == dev && c.dense == (int)dense && c.NT == NT && c.fused == (int)fused && c.B == a.B && c.E == a.E &&
+        c.I == a.I && c.d == a.d && c.r == a.r && c.items == items && c.forced == g_forced_cs) {
       *out = c;
       return cudaSuccess;
     }
@@ -964,25 +1209,32 @@ cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
   int smem_max = 0;
   err = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (err != cudaSuccess) return err;
-  auto fn = dense ? dense_kernel : reader_kernel;
+  const void* fn = pick_kernel(dense, NT, fused);
   err = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (err != cudaSuccess) return err;
-  LaunchPlan p = {dev, (int)dense, a.nmax, a.I, a.d, a.r, items, g_forced_cs, 0, 0, 0, 0};
-  long best_busy = -1;
-  for (int cs = 16; cs >= 4; cs /= 2) {
+  LaunchPlan p = {dev, (int)dense, NT, (int)fused, a.B, a.E, a.I, a.d, a.r, items, g_forced_cs, 0, 0, 0, 0, {}};
+  double best = 1e30;
+  const int ntok = fused ? a.B : NT;
+  for (int cs = 16; cs >= 8; cs--) {
     if (g_forced_cs && cs != g_forced_cs) continue;
-    if (a.d / cs > 256 || a.d / cs < 8 || a.I < cs) continue;
-    ExpertArgs t = a;
-    t.cs = cs;
-    const int rr = pick_ring_rows(t, dense, smem_max);
+    const int cols_max = 8 * cdiv(a.d / 8, cs);
+    if (cols_max > kMaxCols || a.I < cs || (fused && a.E < cs)) continue;
+    const int need = NT * (cols_max + a.r) * 4;
+    const int wr_need = fused ? cdiv(a.E, cs) * a.d * 2 + a.d * 4 : 0;
+    int rr = 0;
+    for (int t = 2; t <= 64; t++) {
+      const Layout L = make_layout(NT, ntok, fused, a.E, a.I, a.d, a.r, cs, t, dense);
+      if (L.total > smem_max) break;
+      if (L.ring_bytes >= need && NWARP * L.ring_bytes >= wr_need) rr = t;
+    }
     if (rr < 2) continue;
-    const int smem = make_layout(a.nmax, a.I, a.d, a.r, cs, rr, dense).total;
-    err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const Layout L = make_layout(NT, ntok, fused, a.E, a.I, a.d, a.r, cs, rr, dense);
+    err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cs);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.blockDim = dim3(NTHR);
+    cfg.dynamicSmemBytes = L.total;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = cs;
@@ -997,13 +1249,14 @@ cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
       continue;
     }
     if (nclusters < 1) continue;
-    const long busy = (long)(items < nclusters ? items : nclusters) * cs;
-    if (busy > best_busy) {
-      best_busy = busy;
+    const double cost = (double)cdiv(items, nclusters) / cs;
+    if (cost < best - 1e-12) {
+      best = cost;
       p.cs = cs;
       p.ring_rows = rr;
-      p.smem = smem;
+      p.smem = L.total;
       p.max_clusters = nclusters;
+      p.L = L;
     }
   }
   if (p.cs == 0) return cudaErrorInvalidConfiguration;
@@ -1020,15 +1273,13 @@ cudaError_t launch_expert(const ExpertArgs& a0, cudaStream_t s, bool dense) {
   if (err != cudaSuccess) return err;
   a.cs = plan.cs;
   a.ring_rows = plan.ring_rows;
-  const Layout L = make_layout(a.nmax, a.I, a.d, a.r, a.cs, a.ring_rows, dense);
-  auto fn = dense ? dense_kernel : reader_kernel;
-  err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+  const void* fn = pick_kernel(dense, plan.NT, plan.fused);
+  err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem);
   if (err != cudaSuccess) return err;
-  const int items = a.ws.max_items;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(items * a.cs);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = L.total;
+  cfg.gridDim = dim3(plan.items * a.cs);
+  cfg.blockDim = dim3(NTHR);
+  cfg.dynamicSmemBytes = plan.smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1038,19 +1289,16 @@ cudaError_t launch_expert(const ExpertArgs& a0, cudaStream_t s, bool dense) {
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, fn, a);
+  cfg.numAttrs = plan.fused ? 1 : 2;  // the fused kernel is the step's first
+  void* args[] = {&a, &plan.L};
+  return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
 }  // namespace
 
-size_t reader_smem_bytes(const ExpertArgs& a, int ring_rows) {
-  return make_layout(a.nmax, a.I, a.d, a.r, a.cs, ring_rows, false).total;
-}
-size_t dense_smem_bytes(const ExpertArgs& a, int ring_rows) {
-  return make_layout(a.nmax, a.I, a.d, a.r, a.cs, ring_rows, true).total;
-}
+bool fused_routing(int B) { return B <= 4; }
 cudaError_t launch_reader(const ExpertArgs& a, cudaStream_t s) { return launch_expert(a, s, false); }
+cudaError_t launch_dense(const ExpertArgs& a, cudaStream_t s) { return launch_expert(a, s, true); }
 void set_forced_cluster_size(int cs) { g_forced_cs = cs; }
 cudaError_t query_plan(const ExpertArgs& a, bool dense, int out[4]) {
   LaunchPlan p;
@@ -1062,6 +1310,5 @@ cudaError_t query_plan(const ExpertArgs& a, bool dense, int out[4]) {
   out[3] = p.max_clusters;
   return cudaSuccess;
 }
-cudaError_t launch_dense(const ExpertArgs& a, cudaStream_t s) { return launch_expert(a, s, true); }
 
 }  // namespace moe

@@ -113,15 +113,18 @@ __global__ void __launch_bounds__(512) select_kernel(RouteArgs a) {
     uint32_t taken = 0;
     double chosen[16];
     int chosen_id[16];
+    double lv[32];  // this lane's logits (E <= 1024), read once
+#pragma unroll
+    for (int m = 0; m < 32; m++) lv[m] = lane + 32 * m < E ? L[lane + 32 * m] : -INFINITY;
     for (int s = 0; s < top; s++) {
       double bv = -INFINITY;
       int bi = 0x7fffffff;
-      for (int m = 0; lane + 32 * m < E; m++) {
+#pragma unroll
+      for (int m = 0; m < 32; m++) {
         const int e = lane + 32 * m;
-        if (taken & (1u << m)) continue;
-        const double lv = L[e];
-        if (lv > bv || (lv == bv && e < bi) || bi == 0x7fffffff) {
-          bv = lv;
+        if (e >= E || (taken & (1u << m))) continue;
+        if (bi == 0x7fffffff || lv[m] > bv) {
+          bv = lv[m];
           bi = e;
         }
       }
