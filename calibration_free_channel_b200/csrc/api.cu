@@ -155,6 +155,7 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
     a.dbg_kept = dbg->kept;
     a.dbg_a_kept = dbg->a_kept;
     a.dbg_y_expert = dbg->y_expert;
+    a.dbg_phase = reinterpret_cast<unsigned long long*>(dbg->phase_ns);
   }
   if (g_ev_before) cudaEventRecord(g_ev_before, s);
   e = dense ? moe::launch_dense(a, s) : moe::launch_reader(a, s);

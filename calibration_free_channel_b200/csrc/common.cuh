@@ -11,9 +11,10 @@ namespace cg = cooperative_groups;
 constexpr int kThreads = 256;          // threads per CTA of the expert kernels
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxSlots = 16;          // row slots per warp in the copy rings
-constexpr int kMaxGroup = 8;           // tokens per work item (tokens sharing an expert)
+constexpr int kMaxGroup = 2;           // tokens per work item (tokens sharing an expert)
 constexpr int kMaxRank = 128;
 constexpr int kMaxCluster = 16;
+constexpr int kMaxTokens = 256;        // tokens per step (B)
 
 // Error word bits (workspace), set by bounded waits that ran out.
 constexpr uint32_t kErrCopyTimeout = 1u;
@@ -85,12 +86,14 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
+// try_wait with a suspend-time hint: the warp sleeps until the phase
+// completes (or the hint elapses) instead of spinning.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }

@@ -71,6 +71,7 @@ struct ExpertArgs {
   int32_t* dbg_kept;
   float* dbg_a_kept;
   float* dbg_y_expert;
+  unsigned long long* dbg_phase;
 };
 // Steps of at most this many tokens route inside the expert kernel (one
 // launch per step); larger steps use the route and select kernels first.

@@ -388,17 +388,40 @@ __device__ void load_q(const ExpertArgs& a, const Layout& L, char* smem, const i
 }
 
 // Rotation + int8 quantisation of smem token t: v = FWHT(s . x) in the fp32
-// scratch (d floats), q = rint(127 v / amax), c_x = amax / (127 d).  The
-// butterflies follow the reference order (stages h = 1, 2, 4, ...), so the
+// scratch (d floats), q = rint(127 v / amax), c_x = amax / (127 d).  Thread T
+// (< d/4) holds elements 4T..4T+3: stages h = 1, 2 run in registers, h = 4..64
+// across the lanes of a warp (a warp holds 128 consecutive elements), h >= 128
+// in shared memory.  Every stage applies the reference butterflies
+// (a + b, a - b), lower index first, in the reference stage order, so the
 // bits equal the reference transform's.
 __device__ void rotate_quantize_smem(const ExpertArgs& a, const Layout& L, char* smem, int t, float* v,
                                      float* cx_out, float* red) {
   const int d = a.d;
-  const uint16_t* xs = reinterpret_cast<const uint16_t*>(smem + L.x) + (size_t)t * d;
-  for (int j = threadIdx.x; j < d; j += NTHR) v[j] = (float)a.rot_sign[j] * bf16f(xs[j]);
+  const int T = threadIdx.x, lane = T & 31;
+  if (T < d / 4) {
+    const uint2 xv = reinterpret_cast<const uint2*>(smem + L.x + (size_t)t * d * 2)[T];
+    const char4 sv = reinterpret_cast<const char4*>(a.rot_sign)[T];
+    float r0 = (float)sv.x * bf16lo(xv.x), r1 = (float)sv.y * bf16hi(xv.x);
+    float r2 = (float)sv.z * bf16lo(xv.y), r3 = (float)sv.w * bf16hi(xv.y);
+    float b0 = __fadd_rn(r0, r1), b1 = __fsub_rn(r0, r1), b2 = __fadd_rn(r2, r3), b3 = __fsub_rn(r2, r3);  // h = 1
+    r0 = __fadd_rn(b0, b2);  // h = 2
+    r2 = __fsub_rn(b0, b2);
+    r1 = __fadd_rn(b1, b3);
+    r3 = __fsub_rn(b1, b3);
+    for (int m = 1; m < 32 && 4 * m < d; m <<= 1) {  // h = 4m: partner lane ^ m
+      const bool up = lane & m;
+      const float p0 = __shfl_xor_sync(0xffffffffu, r0, m), p1 = __shfl_xor_sync(0xffffffffu, r1, m);
+      const float p2 = __shfl_xor_sync(0xffffffffu, r2, m), p3 = __shfl_xor_sync(0xffffffffu, r3, m);
+      r0 = up ? __fsub_rn(p0, r0) : __fadd_rn(r0, p0);
+      r1 = up ? __fsub_rn(p1, r1) : __fadd_rn(r1, p1);
+      r2 = up ? __fsub_rn(p2, r2) : __fadd_rn(r2, p2);
+      r3 = up ? __fsub_rn(p3, r3) : __fadd_rn(r3, p3);
+    }
+    reinterpret_cast<float4*>(v)[T] = make_float4(r0, r1, r2, r3);
+  }
   __syncthreads();
-  for (int h = 1, lh = 0; h < d; h <<= 1, lh++) {
-    for (int p = threadIdx.x; p < d / 2; p += NTHR) {
+  for (int h = 128, lh = 7; h < d; h <<= 1, lh++) {
+    for (int p = threadIdx.x; p < d / 2; p += blockDim.x) {
       const int j = ((p >> lh) << (lh + 1)) | (p & (h - 1));
       const float x0 = v[j], x1 = v[j + h];
       v[j] = __fadd_rn(x0, x1);
@@ -407,15 +430,15 @@ __device__ void rotate_quantize_smem(const ExpertArgs& a, const Layout& L, char*
     __syncthreads();
   }
   float m = 0.0f;
-  for (int j = threadIdx.x; j < d; j += NTHR) m = fmaxf(m, fabsf(v[j]));
+  for (int j = threadIdx.x; j < d; j += blockDim.x) m = fmaxf(m, fabsf(v[j]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  if (lane == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
   float amax = 0.0f;
-  for (int w = 0; w < NWARP; w++) amax = fmaxf(amax, red[w]);
+  for (int w = 0; w < (int)(blockDim.x >> 5); w++) amax = fmaxf(amax, red[w]);
   int8_t* q = reinterpret_cast<int8_t*>(smem + L.q) + (size_t)t * d;
-  for (int j = threadIdx.x; j < d; j += NTHR) {
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
     int n = 0;
     if (amax > 0.0f) n = max(-127, min(127, __float2int_rn(__fdiv_rn(__fmul_rn(v[j], 127.0f), amax))));
     q[j] = (int8_t)n;
@@ -487,78 +510,80 @@ __device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, in
     }
   }
   cluster.sync();
-  // top-e per token (warp b), ties to the lower id; softmax over the chosen
+  // top-e per token by rank: 4 threads per (token, expert) count the logits
+  // that beat it (larger, or equal with a lower id); rank < top_e is chosen
   int* rids = misc + MI_RIDS;
   float* rw = reinterpret_cast<float*>(misc + MI_RW);
-  if (warp < B) {
-    const int b = warp;
-    uint32_t taken = 0;
-    double cv[16];
-    for (int s = 0; s < top; s++) {
-      double bv = -INFINITY;
-      int bi = 0x7fffffff;
-      for (int m = 0; lane + 32 * m < E; m++) {
-        const int e = lane + 32 * m;
-        if (taken & (1u << m)) continue;
-        const double lv = lg[b * E + e];
-        if (bi == 0x7fffffff || lv > bv) {
-          bv = lv;
-          bi = e;
+  double* ex = reinterpret_cast<double*>(smem + L.hist);  // [B, top] scratch
+  {
+    const int ntask = B * E * 4;
+    for (int task = threadIdx.x; task < rup(ntask, 32); task += blockDim.x) {
+      int cnt = 0, b = 0, e = 0;
+      const int qtr = task & 3;
+      if (task < ntask) {
+        b = task / (E * 4);
+        e = (task >> 2) - b * E;
+        const double l = lg[b * E + e];
+        for (int e2 = qtr; e2 < E; e2 += 4) {
+          const double l2 = lg[b * E + e2];
+          cnt += (l2 > l) || (l2 == l && e2 < e);
         }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      cv[s] = bv;
-      if (lane == 0) rids[b * top + s] = bi;
-    }
-    if (lane == 0) {
-      double den = 0.0;
-      for (int s = 0; s < top; s++) den += exp(cv[s] - cv[0]);
-      for (int s = 0; s < top; s++) {
-        const float w = (float)(exp(cv[s] - cv[0]) / den);
-        rw[b * top + s] = w;
-        if (cid == 0 && rank == 0) {
-          a.ws.ids[b * top + s] = rids[b * top + s];
-          a.ws.wts[b * top + s] = w;
-          if (a.dbg_ids) a.dbg_ids[b * top + s] = rids[b * top + s];
-          if (a.dbg_w) a.dbg_w[b * top + s] = w;
-        }
-      }
+      cnt += __shfl_xor_sync(0xffffffffu, cnt, 1);
+      cnt += __shfl_xor_sync(0xffffffffu, cnt, 2);
+      if (task < ntask && qtr == 0 && cnt < top) rids[b * top + cnt] = e;
     }
   }
   __syncthreads();
-  // work table: distinct experts ascending; item cid = the cid-th of them
-  if (threadIdx.x == 0) {
-    int chosen = -1, count = 0, prev = -1;
-    while (true) {
-      int nxt = 0x7fffffff;
-      for (int i = 0; i < B * top; i++)
-        if (rids[i] > prev && rids[i] < nxt) nxt = rids[i];
-      if (nxt == 0x7fffffff) break;
-      if (count == cid) chosen = nxt;
-      count++;
-      prev = nxt;
+  // softmax over the chosen logits (fp64), summed in slot order
+  if (threadIdx.x < B * top) {
+    const int b = threadIdx.x / top;
+    ex[threadIdx.x] = exp(lg[b * E + rids[threadIdx.x]] - lg[b * E + rids[b * top]]);
+  }
+  __syncthreads();
+  if (threadIdx.x < B * top) {
+    const int b = threadIdx.x / top, s = threadIdx.x - b * top;
+    double den = 0.0;
+    for (int s2 = 0; s2 < top; s2++) den += ex[b * top + s2];
+    const float w = (float)(ex[threadIdx.x] / den);
+    rw[threadIdx.x] = w;
+    if (cid == 0 && rank == 0) {
+      a.ws.ids[threadIdx.x] = rids[threadIdx.x];
+      a.ws.wts[threadIdx.x] = w;
+      if (a.dbg_ids) a.dbg_ids[threadIdx.x] = rids[threadIdx.x];
+      if (a.dbg_w) a.dbg_w[threadIdx.x] = w;
     }
-    misc[MI_E] = chosen;
-    int n = 0;
-    if (chosen >= 0)
-      for (int b = 0; b < B; b++)
-        for (int s = 0; s < top; s++)
-          if (rids[b * top + s] == chosen) {
-            misc[MI_TOK + n] = b;
-            misc[MI_SLOT + n] = s;
-            misc[MI_TIX + n] = b;
-            n++;
-          }
-    misc[MI_N] = n;
+    (void)s;
+  }
+  // work table: distinct experts ascending; item cid = the cid-th of them
+  int* first = reinterpret_cast<int*>(ex + 64);
+  const int nent = B * top;
+  if (threadIdx.x < nent) {
+    const int id = rids[threadIdx.x];
+    int f = 1;
+    for (int j = 0; j < threadIdx.x; j++) f &= rids[j] != id;
+    first[threadIdx.x] = f;
+  }
+  if (threadIdx.x == 0) misc[MI_E] = -1;
+  __syncthreads();
+  if (threadIdx.x < nent && first[threadIdx.x]) {
+    const int id = rids[threadIdx.x];
+    int rk = 0;
+    for (int j = 0; j < nent; j++) rk += first[j] && rids[j] < id;
+    if (rk == cid) misc[MI_E] = id;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int e = misc[MI_E];
+    const bool on = e >= 0 && lane < nent && rids[lane] == e;
+    const unsigned bal = __ballot_sync(0xffffffffu, on);
+    if (on) {
+      const int at = __popc(bal & ((1u << lane) - 1u));
+      misc[MI_TOK + at] = lane / top;
+      misc[MI_SLOT + at] = lane % top;
+      misc[MI_TIX + at] = lane / top;
+    }
+    if (lane == 0) misc[MI_N] = __popc(bal);
   }
   __syncthreads();
   return misc[MI_E] >= 0;
@@ -602,6 +627,11 @@ __device__ void write_and_combine(const ExpertArgs& a, int rank, int j0, int nco
   }
 }
 
+// Stage time stamps (globaltimer, ns) of the first CTA of each cluster.
+__device__ __forceinline__ void stamp(const ExpertArgs& a, int cid, int rank, int k) {
+  if (a.dbg_phase && rank == 0 && threadIdx.x == 0) a.dbg_phase[cid * 8 + k] = global_ns();
+}
+
 // ================================================================ sparse
 template <int NT, bool FUSED>
 __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L) {
@@ -622,6 +652,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
   if (tid == 0) misc[MI_DONE] = 0;
   fence_mbar_init();
   __syncthreads();
+  stamp(a, cid, rank, 0);
 
   if (FUSED) {
     if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, wrbar, cluster)) return;  // uniform per cluster
@@ -629,6 +660,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
     pdl_wait();
     if (!load_item_table(a, cid, misc, NT)) return;
   }
+  stamp(a, cid, rank, 1);
   const int e = misc[MI_E], n = misc[MI_N];
   const int I = a.I, d = a.d, r = a.r;
   const int i0 = cdiv(rank * I, cs), i1 = cdiv((rank + 1) * I, cs), nown = i1 - i0;
@@ -749,6 +781,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
       }
     }
   }
+  stamp(a, cid, rank, 2);
   cluster.sync();
 
   // ---------------------------------------------------------- c: top-c
@@ -782,6 +815,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
     }
   }
   const int nU = misc[MI_NU];
+  stamp(a, cid, rank, 3);
 
   // -------------------------------------------- C: exact candidate stage
   {
@@ -827,6 +861,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
           }
         });
   }
+  stamp(a, cid, rank, 4);
   cluster.sync();  // the last exchange: no CTA touches another's smem after this
 
   // ------------------------------------------------------------ k: top-k
@@ -886,6 +921,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
   __syncthreads();
   block_mask_to_list(pmask, I, dlist, nullptr, &misc[MI_ND]);
   const int nD = misc[MI_ND];
+  stamp(a, cid, rank, 5);
 
   // ---------------------------------------------- D: down rows + recovery
   {
@@ -980,6 +1016,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
     }
   }
   __syncthreads();
+  stamp(a, cid, rank, 6);
   float* yfin = reinterpret_cast<float*>(smem + L.x);  // [n, ncols]; x is no longer needed
   for (int idx = tid; idx < n * r; idx += NTHR) {
     const int t = idx / r, p = idx - t * r;
@@ -1004,6 +1041,8 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
   __syncthreads();
   write_and_combine(a, rank, j0, ncols, yfin, misc,
                     FUSED ? reinterpret_cast<const float*>(misc + MI_RW) : a.ws.wts);
+  __syncthreads();
+  stamp(a, cid, rank, 7);
 }
 
 // ================================================================= dense
@@ -1175,13 +1214,10 @@ const void* kernel_ptr(bool dense) {
   return dense ? reinterpret_cast<const void*>(&dense_kernel<NT, FUSED>)
                : reinterpret_cast<const void*>(&reader_kernel<NT, FUSED>);
 }
+static_assert(kMaxGroup == 2, "kernels are instantiated for 1 and 2 tokens per item");
 const void* pick_kernel(bool dense, int NT, bool fused) {
-  switch (NT) {
-    case 1: return fused ? kernel_ptr<1, true>(dense) : kernel_ptr<1, false>(dense);
-    case 2: return fused ? kernel_ptr<2, true>(dense) : kernel_ptr<2, false>(dense);
-    case 4: return fused ? kernel_ptr<4, true>(dense) : kernel_ptr<4, false>(dense);
-    default: return kernel_ptr<8, false>(dense);
-  }
+  if (NT == 1) return fused ? kernel_ptr<1, true>(dense) : kernel_ptr<1, false>(dense);
+  return fused ? kernel_ptr<2, true>(dense) : kernel_ptr<2, false>(dense);
 }
 
 // Cluster size: among 8..16 (those that fit this shape), the one with the
@@ -1195,7 +1231,7 @@ cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  const int NT = a.nmax <= 1 ? 1 : a.nmax <= 2 ? 2 : a.nmax <= 4 ? 4 : 8;
+  const int NT = a.nmax <= 1 ? 1 : 2;
   const bool fused = fused_routing(a.B);
   const int items = fused ? (a.B * a.top_e < a.E ? a.B * a.top_e : a.E) : a.ws.max_items;
   for (int i = 0; i < ncache; i++) {
@@ -1296,7 +1332,7 @@ cudaError_t launch_expert(const ExpertArgs& a0, cudaStream_t s, bool dense) {
 
 }  // namespace
 
-bool fused_routing(int B) { return B <= 4; }
+bool fused_routing(int B) { return B <= kMaxGroup; }
 cudaError_t launch_reader(const ExpertArgs& a, cudaStream_t s) { return launch_expert(a, s, false); }
 cudaError_t launch_dense(const ExpertArgs& a, cudaStream_t s) { return launch_expert(a, s, true); }
 void set_forced_cluster_size(int cs) { g_forced_cs = cs; }

@@ -207,14 +207,15 @@ size_t workspace_layout(int B, int E, int top_e, int d, void* base, Workspace* w
     off = align256(off + bytes);
     return o;
   };
-  const size_t o_err = take(16), o_ni = take(16);
+  // error word and combine counters sit at fixed offsets for every shape, so
+  // a workspace stays valid when it is reused for a different batch size
+  const size_t o_err = take(16), o_ct = take(sizeof(unsigned) * kMaxTokens * kMaxCluster), o_ni = take(16);
   const size_t o_log = take(sizeof(double) * B * E);
   const size_t o_ids = take(sizeof(int) * B * top_e), o_w = take(sizeof(float) * B * top_e);
   const size_t o_q = take((size_t)B * d), o_cx = take(sizeof(float) * B);
   const size_t o_ie = take(sizeof(int) * mi), o_in = take(sizeof(int) * mi);
   const size_t o_it = take(sizeof(int) * mi * kMaxGroup), o_is = take(sizeof(int) * mi * kMaxGroup);
   const size_t o_ye = take(sizeof(float) * B * top_e * (size_t)d);
-  const size_t o_ct = take(sizeof(unsigned) * B * kMaxCluster);
   if (ws && base) {
     char* p = static_cast<char*>(base);
     ws->err = reinterpret_cast<uint32_t*>(p + o_err);

@@ -34,7 +34,7 @@ class MoeReaderLayer(C.Structure):
 
 class MoeReaderDebug(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("ids", "weights", "dot_gate", "dot_up", "score", "cand", "kept",
-                                          "a_kept", "y_expert")]
+                                          "a_kept", "y_expert", "phase_ns")]
 
 
 class MoeError(RuntimeError):
@@ -239,7 +239,8 @@ class Layer:
                          cand=torch.empty(P + (c,), dtype=torch.int32, device=dev),
                          kept=torch.empty(P + (k,), dtype=torch.int32, device=dev),
                          a_kept=torch.empty(P + (k,), dtype=torch.float32, device=dev),
-                         y_expert=torch.empty(P + (self.d,), dtype=torch.float32, device=dev))
+                         y_expert=torch.empty(P + (self.d,), dtype=torch.float32, device=dev),
+                         phase_ns=torch.zeros((B * self.top_e, 8), dtype=torch.int64, device=dev))
             dbg = MoeReaderDebug(*[_ptr(dbg_t[n]) for n, _ in MoeReaderDebug._fields_])
         moe_reader_forward(self.struct(r), B, k, c, x, residual, y, dbg, ws, ws.numel(), stream)
         return (y, dbg_t) if debug else y

@@ -88,6 +88,10 @@ typedef struct {
   int32_t* kept;     /* [B, top_e, k] kept channels, ascending                   */
   float* a_kept;     /* [B, top_e, k] exact silu(g)*u of the kept channels        */
   float* y_expert;   /* [B, top_e, d] fp32 expert output before the combine      */
+  uint64_t* phase_ns; /* [B * top_e, 8] device clock (ns) at the stage boundaries of
+                         the sparse expert kernel, one row per work item: start,
+                         item known, screen done, candidates chosen, exact stage
+                         done, kept chosen, down done, combined              */
 } moe_reader_debug;
 
 /* Bytes of device workspace moe_reader_forward / moe_reader_forward_dense
