@@ -6,7 +6,7 @@
 // Mixture-of-Experts Decoding Needs No Calibration Data", abstract; "KAIST:
 // MoE Decoding Needs No Calibration Data", section "A reader that needs no
 // data at all"):
-//   R  (B <= 4) routing inside the cluster: every CTA computes the logits of
+//   R  (B <= 2) routing inside the cluster: every CTA computes the logits of
 //      its slice of experts and pushes them to all CTAs; every CTA then takes
 //      the same top-e and finds its cluster's work item;
 //   S  screen: every CTA reads the ternary sketch rows of its slice of the I
@@ -29,6 +29,11 @@
 // CTA's own shared memory; every wait on them is bounded.  Every exchange
 // between the CTAs of a cluster is a store into the receivers' shared memory
 // followed by a cluster barrier: no CTA reads another CTA's shared memory.
+//
+// At batch 1 the step is a chain of short dependent stages whose code runs
+// once per launch, so instruction fetch is a first-order cost: the kernels
+// keep their static code small (host-computed geometry instead of runtime
+// divisions, short loops kept rolled, one shared copy of the selection).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -43,7 +48,11 @@ constexpr int kMaxCols = 256;  // output columns per CTA (8 per lane)
 __host__ __device__ inline int rup(int x, int a) { return (x + a - 1) / a * a; }
 __host__ __device__ inline int cdiv(int x, int a) { return (x + a - 1) / a; }
 
-// ------------------------------------------------------------ smem layout
+// One shared copy of a runtime integer division (kernel code stays small).
+__device__ __noinline__ int idiv(int a, int b) { return a / b; }
+
+// ------------------------------------------------------- launch geometry
+// Shared-memory offsets and the partitions of a launch, computed on the host.
 struct Layout {
   int mbar, misc, hist, wtot, pmask, x, q, logit, sig, ahat, zparts, z, apos, candm, keptm, ulist, upos, dlist,
       keys, kidx, ubar, vown, ring, total;
@@ -52,16 +61,32 @@ struct Layout {
   int cols_max;    // max output columns per CTA
   int words;       // mask words over I
   int ring_bytes;  // per warp
+  int d8, d16;     // d / 8, d / 16
+  int s_per;       // channels per screen slot (half a ring)
+  int c_slots;     // candidate-pair slots per warp
+  int ch0[17];     // channel partition over the CTAs of a cluster
+  int col0[17];    // output-column partition (multiples of 8)
+  int ex0[17];     // expert partition (in-kernel routing)
 };
 
-__host__ __device__ inline Layout make_layout(int NT, int ntok, bool fused, int E, int I, int d, int r, int cs,
-                                              int ring_rows, bool dense) {
-  Layout L;
+__host__ inline Layout make_layout(int NT, int ntok, bool fused, int E, int I, int d, int r, int cs,
+                                   int ring_rows, bool dense) {
+  Layout L = {};
   L.ntok = ntok;
   L.own_max = cdiv(I, cs);
   L.cols_max = 8 * cdiv(d / 8, cs);
   L.words = cdiv(I, 32);
   L.ring_bytes = ring_rows * d * 2;
+  L.d8 = d / 8;
+  L.d16 = d / 16;
+  L.s_per = (L.ring_bytes / 2) / (2 * (d / 4));
+  if (L.s_per > 32) L.s_per = 32;  // one alpha per lane
+  L.c_slots = L.ring_bytes / (4 * d);
+  for (int o = 0; o <= cs && o < 17; o++) {
+    L.ch0[o] = cdiv(o * I, cs);
+    L.col0[o] = 8 * cdiv(o * (d / 8), cs);
+    L.ex0[o] = cdiv(o * E, cs);
+  }
   const int rr = r > 0 ? r : 1;
   int o = 0;
   auto take = [&](int bytes) {
@@ -100,11 +125,16 @@ __host__ __device__ inline Layout make_layout(int NT, int ntok, bool fused, int 
 enum {
   MI_E = 0, MI_N, MI_NU, MI_ND, MI_NC, MI_DIG, MI_REM, MI_CNT, MI_DONE,
   MI_TOK = 16, MI_SLOT = 32, MI_LAST = 48, MI_TIX = 64, MI_CX = 80, MI_SCAN = 96,
-  MI_RIDS = 128,  // fused routing: ids [B <= 4][top_e <= 16]
-  MI_RW = 192     // fused routing: weights
+  MI_RIDS = 128,  // in-kernel routing: ids [B <= 2][top_e <= 16]
+  MI_RW = 192     // in-kernel routing: weights
 };
 
 // ---------------------------------------------------------- cluster helpers
+__device__ __forceinline__ int cluster_id() {
+  int c;
+  asm("mov.u32 %0, %%clusterid.x;" : "=r"(c));
+  return c;
+}
 __device__ __forceinline__ uint32_t cluster_addr(const void* local, int rank) {
   uint32_t ra;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
@@ -152,7 +182,7 @@ __device__ __forceinline__ int dot16_i8(uint4 t, uint4 q, int acc) {
 }
 
 // ----------------------------------------------------------- block helpers
-__device__ int block_excl_scan(int v, int* scratch, int* total) {
+__device__ __noinline__ int block_excl_scan(int v, int* scratch, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int inc = v;
 #pragma unroll
@@ -163,7 +193,7 @@ __device__ int block_excl_scan(int v, int* scratch, int* total) {
   if (lane == 31) scratch[warp] = inc;
   __syncthreads();
   int off = 0, tot = 0;
-#pragma unroll
+#pragma unroll 1
   for (int w = 0; w < NWARP; w++) {
     const int s = scratch[w];
     off += w < warp ? s : 0;
@@ -179,10 +209,10 @@ __device__ int block_excl_scan(int v, int* scratch, int* total) {
 // soon as the boundary bin is taken whole; keys equal to a fully resolved
 // threshold are taken in position order.  Sets bit p of out_mask for each
 // chosen position p.  hist holds 2 x 2048 ints, wtot 16 ints.
-__device__ void block_select_top(const uint32_t* keys, int N, int n_sel, int* hist, int* wtot, int* misc,
-                                 uint32_t* out_mask) {
+__device__ __noinline__ void block_select_top(const uint32_t* keys, int N, int n_sel, int* hist, int* wtot,
+                                              int* misc, uint32_t* out_mask) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nw = cdiv(N, 32);
+  const int nw = (N + 31) >> 5;
   for (int w = tid; w < nw; w += NTHR) out_mask[w] = 0u;
   if (n_sel >= N) {
     __syncthreads();
@@ -194,9 +224,11 @@ __device__ void block_select_top(const uint32_t* keys, int N, int n_sel, int* hi
   uint32_t prefix = 0u, mask = 0u;
   int rem = n_sel;
   bool done = false;
+#pragma unroll 1
   for (int pass = 0; pass < 3 && !done; pass++) {
     const int shift = pass == 0 ? 21 : pass == 1 ? 10 : 0;
-    const int nb = pass == 2 ? 1024 : 2048;
+    const int lnb = pass == 2 ? 10 : 11;
+    const int nb = 1 << lnb;
     int* h = hist + (pass & 1) * 2048;
     int* hn = hist + ((pass + 1) & 1) * 2048;
     __syncthreads();  // h is zero and the previous pass is done with hn
@@ -207,9 +239,10 @@ __device__ void block_select_top(const uint32_t* keys, int N, int n_sel, int* hi
     for (int b = tid; b < 2048; b += NTHR) hn[b] = 0;
     __syncthreads();
     // warp w covers bins [nb - (w+1) bpw, nb - w bpw), top-down; lane l a run
-    const int bpw = nb / NWARP, bpl = bpw / 32;
-    const int top = nb - warp * bpw - lane * bpl;  // bins top-1 .. top-bpl
+    const int bpl = nb >> 9;                            // bins per lane (4 or 2)
+    const int top = nb - (warp * 32 + lane) * bpl;      // bins top-1 .. top-bpl
     int s = 0;
+#pragma unroll 1
     for (int j = 1; j <= bpl; j++) s += h[top - j];
     int inc = s;
 #pragma unroll
@@ -220,8 +253,10 @@ __device__ void block_select_top(const uint32_t* keys, int N, int n_sel, int* hi
     if (lane == 31) wtot[warp] = inc;
     __syncthreads();
     int before = inc - s;  // keys in bins above this lane's run
+#pragma unroll 1
     for (int w = 0; w < warp; w++) before += wtot[w];
     if (before < rem && before + s >= rem) {
+#pragma unroll 1
       for (int j = 1; j <= bpl; j++) {
         const int c = h[top - j];
         if (before + c >= rem) {
@@ -249,7 +284,7 @@ __device__ void block_select_top(const uint32_t* keys, int N, int n_sel, int* hi
   }
   // fully resolved threshold T = prefix with more equal keys than needed:
   // keys > T, and the first `rem` keys == T by position
-  const int chunk = cdiv(N, NTHR);
+  const int chunk = (N + NTHR - 1) / NTHR;
   const int p0 = min(N, tid * chunk), p1 = min(N, p0 + chunk);
   int eq = 0;
   for (int p = p0; p < p1; p++) eq += keys[p] == prefix;
@@ -266,9 +301,10 @@ __device__ void block_select_top(const uint32_t* keys, int N, int n_sel, int* hi
 
 // Ascending list of the set bits of mask over [0, N), all warps; the count
 // lands in *count_out; pos_of (if given) gets each bit's list position or -1.
-__device__ void block_mask_to_list(const uint32_t* mask, int N, int* list, int* pos_of, int* count_out) {
+__device__ __noinline__ void block_mask_to_list(const uint32_t* mask, int N, int* list, int* pos_of,
+                                                int* count_out) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nw = cdiv(N, 32);
+  const int nw = (N + 31) >> 5;
   for (int w = warp; w < nw; w += NWARP) {
     int off = 0;
     for (int v = lane; v < w; v += 32) off += __popc(mask[v]);
@@ -291,21 +327,23 @@ __device__ void block_mask_to_list(const uint32_t* mask, int N, int* list, int* 
 // persists across stages.  Returns false if a wait ran out (the warp then
 // stops issuing and drains what is in flight).
 template <class Issue, class Consume>
-__device__ bool warp_stream(int cnt, int P, uint64_t* bars, uint32_t& par, uint32_t* err, Issue issue,
-                            Consume consume) {
+__device__ __forceinline__ bool warp_stream(int cnt, int P, uint64_t* bars, uint32_t& par, uint32_t* err,
+                                            Issue issue, Consume consume) {
   const int lane = threadIdx.x & 31;
   if (cnt <= 0) return true;
   P = min(P, cnt);
   uint32_t pend = 0;
   if (lane == 0) fence_proxy_async();  // the ring may have been read by generic loads
+#pragma unroll 1
   for (int j = 0; j < P; j++) {
     if (lane == 0) issue(j, j, &bars[j]);
     pend |= 1u << j;
   }
   __syncwarp();
   bool ok = true;
+  int s = 0;
+#pragma unroll 1
   for (int j = 0; j < cnt; j++) {
-    const int s = j % P;
     ok = mbar_wait_bounded(&bars[s], (par >> s) & 1u, err);
     if (!ok) break;
     par ^= 1u << s;
@@ -320,21 +358,15 @@ __device__ bool warp_stream(int cnt, int P, uint64_t* bars, uint32_t& par, uint3
       pend |= 1u << s;
       __syncwarp();
     }
+    s = s + 1 == P ? 0 : s + 1;
   }
   if (!ok) {
-    for (int s = 0; s < P; s++)
-      if ((pend >> s) & 1u)
-        if (mbar_wait_bounded(&bars[s], (par >> s) & 1u, err)) par ^= 1u << s;
+#pragma unroll 1
+    for (int q = 0; q < P; q++)
+      if ((pend >> q) & 1u)
+        if (mbar_wait_bounded(&bars[q], (par >> q) & 1u, err)) par ^= 1u << q;
   }
   return ok;
-}
-
-// Column slice of a CTA in 8-column units (16-byte aligned slices).
-__device__ __forceinline__ void col_slice(int d, int cs, int rank, int& j0, int& ncols) {
-  const int u = d / 8;
-  const int u0 = cdiv(rank * u, cs), u1 = cdiv((rank + 1) * u, cs);
-  j0 = u0 * 8;
-  ncols = (u1 - u0) * 8;
 }
 
 // ------------------------------------------------------- work item set-up
@@ -363,27 +395,26 @@ __device__ bool load_item_table(const ExpertArgs& a, int cid, int* misc, int NT)
       misc[MI_TOK + t] = tok;
       misc[MI_SLOT + t] = sl;
       misc[MI_TIX + t] = t;  // tokens are loaded in item order
+      reinterpret_cast<float*>(misc + MI_CX)[t] = a.ws.cx[tok];
     }
   }
   __syncthreads();
   return misc[MI_E] >= 0;
 }
 
-// Loads tokens into smem: toks[t] -> smem token t.
-__device__ void load_x(const ExpertArgs& a, const Layout& L, char* smem, const int* toks, int n) {
-  const int vx = a.d / 8;
+// Loads the item's tokens (misc[MI_TOK + t] -> smem token t): x and, for the
+// sparse reader, q.
+__device__ void load_tokens(const ExpertArgs& a, const Layout& L, char* smem, const int* misc, int n, bool with_q) {
   uint4* xs = reinterpret_cast<uint4*>(smem + L.x);
-  for (int idx = threadIdx.x; idx < n * vx; idx += NTHR) {
-    const int t = idx / vx, j = idx - t * vx;
-    xs[idx] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)toks[t] * a.d) + j);
-  }
-}
-__device__ void load_q(const ExpertArgs& a, const Layout& L, char* smem, const int* toks, int n) {
-  const int vq = a.d / 16;
   uint4* qs = reinterpret_cast<uint4*>(smem + L.q);
-  for (int idx = threadIdx.x; idx < n * vq; idx += NTHR) {
-    const int t = idx / vq, j = idx - t * vq;
-    qs[idx] = __ldcg(reinterpret_cast<const uint4*>(a.ws.q + (size_t)toks[t] * a.d) + j);
+#pragma unroll 1
+  for (int t = 0; t < n; t++) {
+    const int tok = misc[MI_TOK + t];
+    for (int j = threadIdx.x; j < L.d8; j += NTHR)
+      xs[t * L.d8 + j] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)tok * a.d) + j);
+    if (with_q)
+      for (int j = threadIdx.x; j < L.d16; j += NTHR)
+        qs[t * L.d16 + j] = __ldcg(reinterpret_cast<const uint4*>(a.ws.q + (size_t)tok * a.d) + j);
   }
 }
 
@@ -398,7 +429,7 @@ __device__ void rotate_quantize_smem(const ExpertArgs& a, const Layout& L, char*
                                      float* cx_out, float* red) {
   const int d = a.d;
   const int T = threadIdx.x, lane = T & 31;
-  if (T < d / 4) {
+  if (T < 2 * L.d8) {
     const uint2 xv = reinterpret_cast<const uint2*>(smem + L.x + (size_t)t * d * 2)[T];
     const char4 sv = reinterpret_cast<const char4*>(a.rot_sign)[T];
     float r0 = (float)sv.x * bf16lo(xv.x), r1 = (float)sv.y * bf16hi(xv.x);
@@ -408,6 +439,7 @@ __device__ void rotate_quantize_smem(const ExpertArgs& a, const Layout& L, char*
     r2 = __fsub_rn(b0, b2);
     r1 = __fadd_rn(b1, b3);
     r3 = __fsub_rn(b1, b3);
+#pragma unroll 1
     for (int m = 1; m < 32 && 4 * m < d; m <<= 1) {  // h = 4m: partner lane ^ m
       const bool up = lane & m;
       const float p0 = __shfl_xor_sync(0xffffffffu, r0, m), p1 = __shfl_xor_sync(0xffffffffu, r1, m);
@@ -420,8 +452,9 @@ __device__ void rotate_quantize_smem(const ExpertArgs& a, const Layout& L, char*
     reinterpret_cast<float4*>(v)[T] = make_float4(r0, r1, r2, r3);
   }
   __syncthreads();
+#pragma unroll 1
   for (int h = 128, lh = 7; h < d; h <<= 1, lh++) {
-    for (int p = threadIdx.x; p < d / 2; p += blockDim.x) {
+    for (int p = threadIdx.x; p < 4 * L.d8; p += NTHR) {
       const int j = ((p >> lh) << (lh + 1)) | (p & (h - 1));
       const float x0 = v[j], x1 = v[j + h];
       v[j] = __fadd_rn(x0, x1);
@@ -430,15 +463,16 @@ __device__ void rotate_quantize_smem(const ExpertArgs& a, const Layout& L, char*
     __syncthreads();
   }
   float m = 0.0f;
-  for (int j = threadIdx.x; j < d; j += blockDim.x) m = fmaxf(m, fabsf(v[j]));
+  for (int j = threadIdx.x; j < d; j += NTHR) m = fmaxf(m, fabsf(v[j]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
   float amax = 0.0f;
-  for (int w = 0; w < (int)(blockDim.x >> 5); w++) amax = fmaxf(amax, red[w]);
+#pragma unroll 1
+  for (int w = 0; w < NWARP; w++) amax = fmaxf(amax, red[w]);
   int8_t* q = reinterpret_cast<int8_t*>(smem + L.q) + (size_t)t * d;
-  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+  for (int j = threadIdx.x; j < d; j += NTHR) {
     int n = 0;
     if (amax > 0.0f) n = max(-127, min(127, __float2int_rn(__fdiv_rn(__fmul_rn(v[j], 127.0f), amax))));
     q[j] = (int8_t)n;
@@ -447,9 +481,14 @@ __device__ void rotate_quantize_smem(const ExpertArgs& a, const Layout& L, char*
   __syncthreads();
 }
 
-// Fused routing (B <= NT <= 4): every CTA loads all tokens, rotates and
+// Stage time stamps (globaltimer, ns) of the first CTA of each cluster.
+__device__ __forceinline__ void stamp(const ExpertArgs& a, int cid, int rank, int k) {
+  if (a.dbg_phase && rank == 0 && threadIdx.x == 0) a.dbg_phase[cid * 16 + k] = global_ns();
+}
+
+// In-kernel routing (B <= NT <= 2): every CTA loads all tokens, rotates and
 // quantises them, computes the logits of its slice of experts and pushes
-// them to all CTAs; after the cluster barrier every CTA runs the same top-e
+// them to all CTAs; after the cluster barrier every CTA takes the same top-e
 // and builds the same work table (one item per routed expert, experts
 // ascending).  Returns false if this cluster has no item.
 template <int NT>
@@ -457,24 +496,25 @@ __device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, in
                             int cid, uint64_t* wrbar, cg::cluster_group& cluster) {
   const int B = a.B, E = a.E, d = a.d, top = a.top_e;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int e0 = cdiv(rank * E, cs), e1 = cdiv((rank + 1) * E, cs), ne = e1 - e0;
+  const int e0 = L.ex0[rank], ne = L.ex0[rank + 1] - e0;
   char* wr = smem + L.ring;  // router rows of this CTA's experts
   if (threadIdx.x == 0 && ne > 0) {
     mbar_expect_tx(wrbar, ne * d * 2);
     bulk_g2s(wr, a.w_router + (size_t)e0 * d, ne * d * 2, wrbar);
   }
-  {
-    int toks[NT];
-#pragma unroll
-    for (int t = 0; t < NT; t++) toks[t] = t;
-    load_x(a, L, smem, toks, B);
+  if (threadIdx.x < B) {
+    misc[MI_TOK + threadIdx.x] = threadIdx.x;
   }
+  __syncthreads();
+  load_tokens(a, L, smem, misc, B, false);
   __syncthreads();
   // rotate + quantise every token (the ring tail is the fp32 scratch)
   float* scratch = reinterpret_cast<float*>(smem + L.ring + NWARP * L.ring_bytes - d * 4);
   float* cxs = reinterpret_cast<float*>(misc + MI_CX);
+#pragma unroll 1
   for (int t = 0; t < B; t++)
     rotate_quantize_smem(a, L, smem, t, scratch, &cxs[t], reinterpret_cast<float*>(misc + MI_SCAN));
+  stamp(a, cid, rank, 1);
   // logits of the own experts, one warp per expert, pushed to every CTA
   if (ne > 0 && !mbar_wait_bounded(wrbar, 0, a.ws.err)) misc[MI_DONE] = 1;
   double* lg = reinterpret_cast<double*>(smem + L.logit);
@@ -483,66 +523,73 @@ __device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, in
     double acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; t++) acc[t] = 0.0;
-    for (int j = lane; j < d / 8; j += 32) {
+#pragma unroll 1
+    for (int j = lane; j < L.d8; j += 32) {
       const uint4 w = wrow[j];
 #pragma unroll
       for (int t = 0; t < NT; t++) {
-        if (t < B) {
-          const uint4 x = reinterpret_cast<const uint4*>(smem + L.x + (size_t)t * d * 2)[j];
-          acc[t] = fma((double)bf16lo(w.x), (double)bf16lo(x.x), acc[t]);
-          acc[t] = fma((double)bf16hi(w.x), (double)bf16hi(x.x), acc[t]);
-          acc[t] = fma((double)bf16lo(w.y), (double)bf16lo(x.y), acc[t]);
-          acc[t] = fma((double)bf16hi(w.y), (double)bf16hi(x.y), acc[t]);
-          acc[t] = fma((double)bf16lo(w.z), (double)bf16lo(x.z), acc[t]);
-          acc[t] = fma((double)bf16hi(w.z), (double)bf16hi(x.z), acc[t]);
-          acc[t] = fma((double)bf16lo(w.w), (double)bf16lo(x.w), acc[t]);
-          acc[t] = fma((double)bf16hi(w.w), (double)bf16hi(x.w), acc[t]);
-        }
+        const uint4 x = reinterpret_cast<const uint4*>(smem + L.x)[(t < B ? t : 0) * L.d8 + j];
+        acc[t] = fma((double)bf16lo(w.x), (double)bf16lo(x.x), acc[t]);
+        acc[t] = fma((double)bf16hi(w.x), (double)bf16hi(x.x), acc[t]);
+        acc[t] = fma((double)bf16lo(w.y), (double)bf16lo(x.y), acc[t]);
+        acc[t] = fma((double)bf16hi(w.y), (double)bf16hi(x.y), acc[t]);
+        acc[t] = fma((double)bf16lo(w.z), (double)bf16lo(x.z), acc[t]);
+        acc[t] = fma((double)bf16hi(w.z), (double)bf16hi(x.z), acc[t]);
+        acc[t] = fma((double)bf16lo(w.w), (double)bf16lo(x.w), acc[t]);
+        acc[t] = fma((double)bf16hi(w.w), (double)bf16hi(x.w), acc[t]);
       }
     }
     const int e = e0 + el;
+    const double bias = a.bias ? (double)a.bias[e] : 0.0;
 #pragma unroll
     for (int t = 0; t < NT; t++) {
-      if (t < B) {
-        const double s = warp_sum(acc[t]) + (a.bias ? (double)a.bias[e] : 0.0);
-        if (lane < cs) st_cluster(&lg[t * E + e], lane, s);
-      }
+      const double s = warp_sum(acc[t]) + bias;
+      if (t < B && lane < cs) st_cluster(&lg[t * E + e], lane, s);
     }
   }
+  stamp(a, cid, rank, 2);
   cluster.sync();
-  // top-e per token by rank: 4 threads per (token, expert) count the logits
-  // that beat it (larger, or equal with a lower id); rank < top_e is chosen
+  stamp(a, cid, rank, 3);
+  // top-e per token by rank: 4 threads per expert count the logits that beat
+  // it (larger, or equal with a lower id); rank < top_e is chosen
   int* rids = misc + MI_RIDS;
   float* rw = reinterpret_cast<float*>(misc + MI_RW);
   double* ex = reinterpret_cast<double*>(smem + L.hist);  // [B, top] scratch
-  {
-    const int ntask = B * E * 4;
-    for (int task = threadIdx.x; task < rup(ntask, 32); task += blockDim.x) {
-      int cnt = 0, b = 0, e = 0;
-      const int qtr = task & 3;
-      if (task < ntask) {
-        b = task / (E * 4);
-        e = (task >> 2) - b * E;
-        const double l = lg[b * E + e];
+  int* first = reinterpret_cast<int*>(ex + 64);
+#pragma unroll 1
+  for (int b = 0; b < B; b++) {
+    const double* lb = lg + b * E;
+    for (int task = threadIdx.x; task < rup(4 * E, 32); task += NTHR) {
+      int cnt = 0;
+      const int e = task >> 2, qtr = task & 3;
+      if (e < E) {
+        const double l = lb[e];
         for (int e2 = qtr; e2 < E; e2 += 4) {
-          const double l2 = lg[b * E + e2];
+          const double l2 = lb[e2];
           cnt += (l2 > l) || (l2 == l && e2 < e);
         }
       }
       cnt += __shfl_xor_sync(0xffffffffu, cnt, 1);
       cnt += __shfl_xor_sync(0xffffffffu, cnt, 2);
-      if (task < ntask && qtr == 0 && cnt < top) rids[b * top + cnt] = e;
+      if (e < E && qtr == 0 && cnt < top) rids[b * top + cnt] = e;
     }
   }
   __syncthreads();
-  // softmax over the chosen logits (fp64), summed in slot order
-  if (threadIdx.x < B * top) {
-    const int b = threadIdx.x / top;
-    ex[threadIdx.x] = exp(lg[b * E + rids[threadIdx.x]] - lg[b * E + rids[b * top]]);
+  // softmax over the chosen logits, summed in slot order (fp32 exponentials
+  // of the fp64 logit differences; the weights only scale outputs)
+  const int nent = B * top;
+  if (threadIdx.x < nent) {
+    const int b = threadIdx.x >= top;  // B <= 2
+    ex[threadIdx.x] = (double)__expf((float)(lg[b * E + rids[threadIdx.x]] - lg[b * E + rids[b * top]]));
+    const int id = rids[threadIdx.x];
+    int f = 1;
+    for (int j = 0; j < threadIdx.x; j++) f &= rids[j] != id;
+    first[threadIdx.x] = f;
   }
+  if (threadIdx.x == 0) misc[MI_E] = -1;
   __syncthreads();
-  if (threadIdx.x < B * top) {
-    const int b = threadIdx.x / top, s = threadIdx.x - b * top;
+  if (threadIdx.x < nent) {
+    const int b = threadIdx.x >= top;
     double den = 0.0;
     for (int s2 = 0; s2 < top; s2++) den += ex[b * top + s2];
     const float w = (float)(ex[threadIdx.x] / den);
@@ -553,24 +600,13 @@ __device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, in
       if (a.dbg_ids) a.dbg_ids[threadIdx.x] = rids[threadIdx.x];
       if (a.dbg_w) a.dbg_w[threadIdx.x] = w;
     }
-    (void)s;
-  }
-  // work table: distinct experts ascending; item cid = the cid-th of them
-  int* first = reinterpret_cast<int*>(ex + 64);
-  const int nent = B * top;
-  if (threadIdx.x < nent) {
-    const int id = rids[threadIdx.x];
-    int f = 1;
-    for (int j = 0; j < threadIdx.x; j++) f &= rids[j] != id;
-    first[threadIdx.x] = f;
-  }
-  if (threadIdx.x == 0) misc[MI_E] = -1;
-  __syncthreads();
-  if (threadIdx.x < nent && first[threadIdx.x]) {
-    const int id = rids[threadIdx.x];
-    int rk = 0;
-    for (int j = 0; j < nent; j++) rk += first[j] && rids[j] < id;
-    if (rk == cid) misc[MI_E] = id;
+    // work table: distinct experts ascending; item cid = the cid-th of them
+    if (first[threadIdx.x]) {
+      const int id = rids[threadIdx.x];
+      int rk = 0;
+      for (int j = 0; j < nent; j++) rk += first[j] && rids[j] < id;
+      if (rk == cid) misc[MI_E] = id;
+    }
   }
   __syncthreads();
   if (threadIdx.x < 32) {
@@ -579,9 +615,10 @@ __device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, in
     const unsigned bal = __ballot_sync(0xffffffffu, on);
     if (on) {
       const int at = __popc(bal & ((1u << lane) - 1u));
-      misc[MI_TOK + at] = lane / top;
-      misc[MI_SLOT + at] = lane % top;
-      misc[MI_TIX + at] = lane / top;
+      const int b = lane >= top;
+      misc[MI_TOK + at] = b;
+      misc[MI_SLOT + at] = lane - b * top;
+      misc[MI_TIX + at] = b;
     }
     if (lane == 0) misc[MI_N] = __popc(bal);
   }
@@ -593,15 +630,17 @@ __device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, in
 // last expert of each token to finish this column slice combines and resets
 // the slice's counter (so the counters are zero again after every call).
 // wts: routing weights [B, top_e] (global or this CTA's shared copy).
-__device__ void write_and_combine(const ExpertArgs& a, int rank, int j0, int ncols, const float* yfin, int* misc,
-                                  const float* wts) {
+__device__ void write_and_combine(const ExpertArgs& a, int rank, int j0, int ncols, int ldy, const float* yfin,
+                                  int* misc, const float* wts) {
   const int n = misc[MI_N];
-  for (int idx = threadIdx.x; idx < n * ncols; idx += NTHR) {
-    const int t = idx / ncols, col = idx - t * ncols;
+#pragma unroll 1
+  for (int t = 0; t < n; t++) {
     const int tok = misc[MI_TOK + t], sl = misc[MI_SLOT + t];
-    const size_t off = ((size_t)tok * a.top_e + sl) * a.d + j0 + col;
-    a.ws.ye[off] = yfin[idx];
-    if (a.dbg_y_expert) a.dbg_y_expert[off] = yfin[idx];
+    float* dst = a.ws.ye + ((size_t)tok * a.top_e + sl) * a.d + j0;
+    for (int col = threadIdx.x; col < ncols; col += NTHR) {
+      dst[col] = yfin[t * ldy + col];
+      if (a.dbg_y_expert) a.dbg_y_expert[((size_t)tok * a.top_e + sl) * a.d + j0 + col] = yfin[t * ldy + col];
+    }
   }
   __threadfence();
   __syncthreads();
@@ -611,6 +650,7 @@ __device__ void write_and_combine(const ExpertArgs& a, int rank, int j0, int nco
     misc[MI_LAST + t] = old == (unsigned)(a.top_e - 1);
   }
   __syncthreads();
+#pragma unroll 1
   for (int t = 0; t < n; t++) {
     if (!misc[MI_LAST + t]) continue;
     __threadfence();
@@ -618,6 +658,7 @@ __device__ void write_and_combine(const ExpertArgs& a, int rank, int j0, int nco
     for (int col = threadIdx.x; col < ncols; col += NTHR) {
       const int j = j0 + col;
       float acc = 0.0f;
+#pragma unroll 1
       for (int s = 0; s < a.top_e; s++)
         acc = fmaf(wts[tok * a.top_e + s], __ldcg(&a.ws.ye[((size_t)tok * a.top_e + s) * a.d + j]), acc);
       if (a.residual) acc += bf16f(a.residual[(size_t)tok * a.d + j]);
@@ -627,19 +668,14 @@ __device__ void write_and_combine(const ExpertArgs& a, int rank, int j0, int nco
   }
 }
 
-// Stage time stamps (globaltimer, ns) of the first CTA of each cluster.
-__device__ __forceinline__ void stamp(const ExpertArgs& a, int cid, int rank, int k) {
-  if (a.dbg_phase && rank == 0 && threadIdx.x == 0) a.dbg_phase[cid * 8 + k] = global_ns();
-}
-
 // ================================================================ sparse
-template <int NT, bool FUSED>
+template <int NT, bool FUSED, bool DBG>
 __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L) {
   extern __shared__ __align__(128) char smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int cs = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
-  const int cid = blockIdx.x / cs;
+  const int cid = cluster_id();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.mbar);
   uint64_t* wbars = bars + warp * kMaxSlots;
@@ -652,7 +688,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
   if (tid == 0) misc[MI_DONE] = 0;
   fence_mbar_init();
   __syncthreads();
-  stamp(a, cid, rank, 0);
+  if (DBG) stamp(a, cid, rank, 0);
 
   if (FUSED) {
     if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, wrbar, cluster)) return;  // uniform per cluster
@@ -660,12 +696,11 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
     pdl_wait();
     if (!load_item_table(a, cid, misc, NT)) return;
   }
-  stamp(a, cid, rank, 1);
+  if (DBG) stamp(a, cid, rank, 4);
   const int e = misc[MI_E], n = misc[MI_N];
   const int I = a.I, d = a.d, r = a.r;
-  const int i0 = cdiv(rank * I, cs), i1 = cdiv((rank + 1) * I, cs), nown = i1 - i0;
-  int j0, ncols;
-  col_slice(d, cs, rank, j0, ncols);
+  const int i0 = L.ch0[rank], nown = L.ch0[rank + 1] - i0;
+  const int j0 = L.col0[rank], ncols = L.col0[rank + 1] - j0;
   uint32_t* err = a.ws.err;
   uint32_t par = 0;
   char* ring = smem + L.ring + warp * L.ring_bytes;
@@ -681,12 +716,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
     bulk_g2s(smem + L.vown, a.v + ((size_t)e * d + j0) * r, bv, uvbar);
   }
   if (!FUSED) {
-    int toks[NT];
-#pragma unroll
-    for (int t = 0; t < NT; t++) toks[t] = misc[MI_TOK + (t < n ? t : 0)];
-    load_x(a, L, smem, toks, n);
-    load_q(a, L, smem, toks, n);
-    if (tid < n) reinterpret_cast<float*>(misc + MI_CX)[tid] = __ldcg(&a.ws.cx[toks[tid]]);
+    load_tokens(a, L, smem, misc, n, true);
     __syncthreads();
   }
 
@@ -708,15 +738,16 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
   // ---------------------------------------------------------- S: screen
   {
     const int c0 = i0 + (warp * nown) / NWARP, c1 = i0 + ((warp + 1) * nown) / NWARP;
-    const int skrow = d / 4;
+    const int skrow = 4 * L.d16;  // bytes per sketch row
     const int half = L.ring_bytes / 2;
-    const int per = max(1, half / (2 * skrow));
-    const int words = d / 16;
+    const int per = L.s_per;
+    const int words = L.d16;
     const uint4* qs = reinterpret_cast<const uint4*>(smem + L.q);
     const float* ag_row = a.alpha_gate + (size_t)e * I;
     const float* au_row = a.alpha_up + (size_t)e * I;
+    const int nchunk = c1 > c0 ? idiv(c1 - c0 + per - 1, per) : 0;
     warp_stream(
-        cdiv(c1 - c0, per), 2, wbars, par, err,
+        nchunk, 2, wbars, par, err,
         [&](int j, int s, uint64_t* bar) {
           const int a0 = c0 + j * per, cnt = min(per, c1 - a0);
           char* dst = ring + s * half;
@@ -728,11 +759,16 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
           const int a0 = c0 + j * per, cnt = min(per, c1 - a0);
           const uint32_t* gw = reinterpret_cast<const uint32_t*>(ring + s * half);
           const uint32_t* uw = gw + cnt * words;
+          // the scales of this chunk, one per lane, loaded ahead of the dots
+          const float agl = lane < cnt ? __ldg(ag_row + a0 + lane) : 0.0f;
+          const float aul = lane < cnt ? __ldg(au_row + a0 + lane) : 0.0f;
+#pragma unroll 1
           for (int ci = 0; ci < cnt; ci++) {
             const int i = a0 + ci;
             int G[NT], U[NT];
 #pragma unroll
             for (int t = 0; t < NT; t++) G[t] = U[t] = 0;
+#pragma unroll 1
             for (int w = lane; w < words; w += 32) {
               const uint4 tg = decode_trits(gw[ci * words + w]);
               const uint4 tu = decode_trits(uw[ci * words + w]);
@@ -743,7 +779,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
                 U[t] = dot16_i8(tu, qv, U[t]);
               }
             }
-            const float ag = __ldg(ag_row + i), au = __ldg(au_row + i);
+            const float ag = __shfl_sync(0xffffffffu, agl, ci), au = __shfl_sync(0xffffffffu, aul, ci);
 #pragma unroll
             for (int t = 0; t < NT; t++) {
               if (t < n) {
@@ -756,7 +792,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
                   st_cluster(&sig[t * I + i], lane, fabsf(ah));
                   st_cluster(&ahat[t * I + i], lane, ah);
                 }
-                if (lane == 31) {
+                if (DBG && lane == 31) {
                   const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * I + i;
                   if (a.dbg_G) a.dbg_G[off] = gs;
                   if (a.dbg_U) a.dbg_U[off] = us;
@@ -766,6 +802,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
             }
           }
         });
+    if (DBG) stamp(a, cid, rank, 5);
     // partial recovery input over the own channels, pushed to every CTA:
     // zparts[rank][t] = sum_{own i} ahat_i Ubar_i.  The local ahat of the own
     // channels was written by this CTA's own stores above.
@@ -773,36 +810,45 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
     if (r > 0) {
       if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
       const uint16_t* ub = reinterpret_cast<const uint16_t*>(smem + L.ubar);
-      for (int idx = tid; idx < n * r; idx += NTHR) {
-        const int t = idx / r, p = idx - t * r;
-        float zz = 0.0f;
-        for (int li = 0; li < nown; li++) zz = fmaf(ahat[t * I + i0 + li], bf16f(ub[li * r + p]), zz);
-        for (int o = 0; o < cs; o++) st_cluster(&zparts[(rank * NT + t) * r + p], o, zz);
-      }
+#pragma unroll 1
+      for (int t = 0; t < n; t++)
+        for (int p = tid; p < r; p += NTHR) {
+          float zz = 0.0f;
+#pragma unroll 4
+          for (int li = 0; li < nown; li++) zz = fmaf(ahat[t * I + i0 + li], bf16f(ub[li * r + p]), zz);
+#pragma unroll 1
+          for (int o = 0; o < cs; o++) st_cluster(&zparts[(rank * NT + t) * r + p], o, zz);
+        }
     }
   }
-  stamp(a, cid, rank, 2);
+  if (DBG) stamp(a, cid, rank, 6);
   cluster.sync();
+  if (DBG) stamp(a, cid, rank, 7);
 
   // ---------------------------------------------------------- c: top-c
+#pragma unroll 1
   for (int t = 0; t < n; t++)
     block_select_top(reinterpret_cast<const uint32_t*>(sig + t * I), I, a.c, hist, wtot, misc,
                      candm + t * L.words);
-  for (int idx = tid; idx < n * r; idx += NTHR) {
-    const int t = idx / r, p = idx - t * r;
-    float zz = 0.0f;
-    for (int o = 0; o < cs; o++) zz += zparts[(o * NT + t) * r + p];
-    z[idx] = zz;
-  }
+  if (DBG) stamp(a, cid, rank, 8);
+#pragma unroll 1
+  for (int t = 0; t < n; t++)
+    for (int p = tid; p < r; p += NTHR) {
+      float zz = 0.0f;
+#pragma unroll 1
+      for (int o = 0; o < cs; o++) zz += zparts[(o * NT + t) * r + p];
+      z[t * r + p] = zz;
+    }
   // union of the candidates, ascending
   for (int w = tid; w < L.words; w += NTHR) {
     uint32_t m = 0;
-    for (int t = 0; t < n; t++) m |= candm[t * L.words + w];
+#pragma unroll
+    for (int t = 0; t < NT; t++) m |= t < n ? candm[t * L.words + w] : 0u;
     pmask[w] = m;
   }
   __syncthreads();
   block_mask_to_list(pmask, I, ulist, upos, &misc[MI_NU]);
-  if (a.dbg_cand && rank == 0 && warp < n) {
+  if (DBG && a.dbg_cand && rank == 0 && warp < n) {
     const int t = warp;
     int base = 0;
     int* out = a.dbg_cand + ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.c;
@@ -815,16 +861,16 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
     }
   }
   const int nU = misc[MI_NU];
-  stamp(a, cid, rank, 3);
+  if (DBG) stamp(a, cid, rank, 9);
 
   // -------------------------------------------- C: exact candidate stage
   {
-    const int u0 = cdiv(rank * nU, cs), u1 = cdiv((rank + 1) * nU, cs), nsl = u1 - u0;
+    const int u0 = idiv(rank * nU + cs - 1, cs), u1 = idiv((rank + 1) * nU + cs - 1, cs), nsl = u1 - u0;
     const int m0 = (warp * nsl) / NWARP, m1 = ((warp + 1) * nsl) / NWARP;
     const int rowb = d * 2;
-    const int P = max(1, min(kMaxSlots, L.ring_bytes / (2 * rowb)));
+    const int P = max(1, min(kMaxSlots, L.c_slots));
     const uint4* xs = reinterpret_cast<const uint4*>(smem + L.x);
-    const int vx = d / 8;
+    const int vx = L.d8;
     warp_stream(
         m1 - m0, P, wbars, par, err,
         [&](int j, int s, uint64_t* bar) {
@@ -841,6 +887,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
           float g0[NT], g1[NT], v0[NT], v1[NT];
 #pragma unroll
           for (int t = 0; t < NT; t++) g0[t] = g1[t] = v0[t] = v1[t] = 0.0f;
+#pragma unroll 2
           for (int vv = lane; vv < vx; vv += 32) {
             const uint4 gv = gr[vv], uv = ur[vv];
 #pragma unroll
@@ -861,10 +908,12 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
           }
         });
   }
-  stamp(a, cid, rank, 4);
+  if (DBG) stamp(a, cid, rank, 10);
   cluster.sync();  // the last exchange: no CTA touches another's smem after this
+  if (DBG) stamp(a, cid, rank, 11);
 
   // ------------------------------------------------------------ k: top-k
+#pragma unroll 1
   for (int t = 0; t < n; t++) {
     // the token's candidates in ascending channel order, key |a|
     if (warp == 0) {
@@ -896,7 +945,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
     for (int p = tid; p < c; p += NTHR)
       if ((pmask[p >> 5] >> (p & 31)) & 1u) atomicOr(&km[kidx[p] >> 5], 1u << (kidx[p] & 31));
     __syncthreads();
-    if (a.dbg_kept && rank == 0 && warp == 0) {
+    if (DBG && a.dbg_kept && rank == 0 && warp == 0) {
       const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.k;
       int base = 0;
       for (int w0 = 0; w0 < I; w0 += 32) {
@@ -912,26 +961,28 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
       }
     }
   }
+  if (DBG) stamp(a, cid, rank, 12);
   // union of the kept channels
   for (int w = tid; w < L.words; w += NTHR) {
     uint32_t m = 0;
-    for (int t = 0; t < n; t++) m |= keptm[t * L.words + w];
+#pragma unroll
+    for (int t = 0; t < NT; t++) m |= t < n ? keptm[t * L.words + w] : 0u;
     pmask[w] = m;
   }
   __syncthreads();
   block_mask_to_list(pmask, I, dlist, nullptr, &misc[MI_ND]);
   const int nD = misc[MI_ND];
-  stamp(a, cid, rank, 5);
+  if (DBG) stamp(a, cid, rank, 13);
 
   // ---------------------------------------------- D: down rows + recovery
   {
     const int colb = ncols * 2, ubb = r * 2;
     const int eb = rup(colb + ubb, 16);
     const int m0 = (warp * nD) / NWARP, m1 = ((warp + 1) * nD) / NWARP, cnt = m1 - m0;
-    const int cap = max(1, L.ring_bytes / eb);
+    const int cap = max(1, idiv(L.ring_bytes, eb));
     int P = min(kMaxSlots, max(1, cnt));
-    int per = max(1, min(cdiv(cnt, P), cap / P));
-    if (per * P > cap) P = max(1, cap / per);
+    int per = max(1, min(idiv(cnt + P - 1, P), idiv(cap, P)));
+    if (per * P > cap) P = max(1, idiv(cap, per));
     float acc[NT][8];
     float cor[NT][4];
 #pragma unroll
@@ -942,11 +993,12 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
       for (int q = 0; q < 4; q++) cor[t][q] = 0.0f;
     }
     warp_stream(
-        cdiv(cnt, per), P, wbars, par, err,
+        cnt > 0 ? idiv(cnt + per - 1, per) : 0, P, wbars, par, err,
         [&](int j, int s, uint64_t* bar) {
           const int g0 = m0 + j * per, gc = min(per, m1 - g0);
           char* dst = ring + s * per * eb;
           mbar_expect_tx(bar, gc * (colb + ubb));
+#pragma unroll 1
           for (int q = 0; q < gc; q++) {
             const int i = dlist[g0 + q];
             bulk_g2s(dst + q * eb, a.w_down + ((size_t)e * I + i) * d + j0, colb, bar);
@@ -956,6 +1008,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
         [&](int j, int s) {
           const int g0 = m0 + j * per, gc = min(per, m1 - g0);
           const char* src = ring + s * per * eb;
+#pragma unroll 1
           for (int q = 0; q < gc; q++) {
             const int i = dlist[g0 + q];
             float co[NT], ch[NT];
@@ -1016,33 +1069,40 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
     }
   }
   __syncthreads();
-  stamp(a, cid, rank, 6);
-  float* yfin = reinterpret_cast<float*>(smem + L.x);  // [n, ncols]; x is no longer needed
-  for (int idx = tid; idx < n * r; idx += NTHR) {
-    const int t = idx / r, p = idx - t * r;
-    float cc = 0.0f;
-    for (int w = 0; w < NWARP; w++)
-      cc += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[NT * L.cols_max + t * r + p];
-    z[idx] -= cc;
-  }
+  float* yfin = reinterpret_cast<float*>(smem + L.x);  // [n, cols_max]; x is no longer needed
+#pragma unroll 1
+  for (int t = 0; t < n; t++)
+    for (int p = tid; p < r; p += NTHR) {
+      float cc = 0.0f;
+#pragma unroll 1
+      for (int w = 0; w < NWARP; w++)
+        cc += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[NT * L.cols_max + t * r + p];
+      z[t * r + p] -= cc;
+    }
   __syncthreads();
   {
     const uint16_t* vo = reinterpret_cast<const uint16_t*>(smem + L.vown);
-    for (int idx = tid; idx < n * ncols; idx += NTHR) {
-      const int t = idx / ncols, col = idx - t * ncols;
-      float y = 0.0f;
-      for (int w = 0; w < NWARP; w++)
-        y += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[t * L.cols_max + col];
-      float rec = 0.0f;
-      for (int p = 0; p < r; p++) rec = fmaf(bf16f(vo[col * r + p]), z[t * r + p], rec);
-      yfin[idx] = y + rec;
-    }
+#pragma unroll 1
+    for (int t = 0; t < n; t++)
+      for (int col = tid; col < ncols; col += NTHR) {
+        float y = 0.0f;
+#pragma unroll 1
+        for (int w = 0; w < NWARP; w++)
+          y += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[t * L.cols_max + col];
+        float rec = 0.0f;
+#pragma unroll 4
+        for (int p = 0; p < r; p++) rec = fmaf(bf16f(vo[col * r + p]), z[t * r + p], rec);
+        yfin[t * L.cols_max + col] = y + rec;
+      }
   }
   __syncthreads();
-  write_and_combine(a, rank, j0, ncols, yfin, misc,
+  if (DBG) stamp(a, cid, rank, 14);
+  write_and_combine(a, rank, j0, ncols, L.cols_max, yfin, misc,
                     FUSED ? reinterpret_cast<const float*>(misc + MI_RW) : a.ws.wts);
-  __syncthreads();
-  stamp(a, cid, rank, 7);
+  if (DBG) {
+    __syncthreads();
+    stamp(a, cid, rank, 15);
+  }
 }
 
 // ================================================================= dense
@@ -1052,7 +1112,7 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
   cg::cluster_group cluster = cg::this_cluster();
   const int cs = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
-  const int cid = blockIdx.x / cs;
+  const int cid = cluster_id();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.mbar);
   uint64_t* wbars = bars + warp * kMaxSlots;
@@ -1067,17 +1127,13 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
   } else {
     pdl_wait();
     if (!load_item_table(a, cid, misc, NT)) return;
-    int toks[NT];
-#pragma unroll
-    for (int t = 0; t < NT; t++) toks[t] = misc[MI_TOK + (t < misc[MI_N] ? t : 0)];
-    load_x(a, L, smem, toks, misc[MI_N]);
+    load_tokens(a, L, smem, misc, misc[MI_N], false);
     __syncthreads();
   }
   const int e = misc[MI_E], n = misc[MI_N];
   const int I = a.I, d = a.d;
-  const int i0 = cdiv(rank * I, cs), i1 = cdiv((rank + 1) * I, cs), nown = i1 - i0;
-  int j0, ncols;
-  col_slice(d, cs, rank, j0, ncols);
+  const int i0 = L.ch0[rank], nown = L.ch0[rank + 1] - i0;
+  const int j0 = L.col0[rank], ncols = L.col0[rank + 1] - j0;
   uint32_t* err = a.ws.err;
   uint32_t par = 0;
   char* ring = smem + L.ring + warp * L.ring_bytes;
@@ -1087,8 +1143,8 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
   float* h = reinterpret_cast<float*>(smem + L.sig);  // [NT, I] pushed by the owners
   {
     const int m0 = (warp * nown) / NWARP, m1 = ((warp + 1) * nown) / NWARP;
-    const int rowb = d * 2, vx = d / 8;
-    const int P = max(1, min(kMaxSlots, L.ring_bytes / (2 * rowb)));
+    const int rowb = d * 2, vx = L.d8;
+    const int P = max(1, min(kMaxSlots, L.c_slots));
     const uint4* xs = reinterpret_cast<const uint4*>(smem + L.x);
     warp_stream(
         m1 - m0, P, wbars, par, err,
@@ -1106,6 +1162,7 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
           float g0[NT], g1[NT], v0[NT], v1[NT];
 #pragma unroll
           for (int t = 0; t < NT; t++) g0[t] = g1[t] = v0[t] = v1[t] = 0.0f;
+#pragma unroll 2
           for (int vv = lane; vv < vx; vv += 32) {
             const uint4 gv = gr[vv], uv = ur[vv];
 #pragma unroll
@@ -1129,27 +1186,29 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
     const int colb = ncols * 2;
     const int eb = rup(colb, 16);
     const int m0 = (warp * I) / NWARP, m1 = ((warp + 1) * I) / NWARP, cnt = m1 - m0;
-    const int cap = max(1, L.ring_bytes / eb);
+    const int cap = max(1, idiv(L.ring_bytes, eb));
     int P = min(kMaxSlots, max(1, cnt));
-    int per = max(1, min(cdiv(cnt, P), cap / P));
-    if (per * P > cap) P = max(1, cap / per);
+    int per = max(1, min(idiv(cnt + P - 1, P), idiv(cap, P)));
+    if (per * P > cap) P = max(1, idiv(cap, per));
     float acc[NT][8];
 #pragma unroll
     for (int t = 0; t < NT; t++)
 #pragma unroll
       for (int q = 0; q < 8; q++) acc[t][q] = 0.0f;
     warp_stream(
-        cdiv(cnt, per), P, wbars, par, err,
+        cnt > 0 ? idiv(cnt + per - 1, per) : 0, P, wbars, par, err,
         [&](int j, int s, uint64_t* bar) {
           const int g0 = m0 + j * per, gc = min(per, m1 - g0);
           char* dst = ring + s * per * eb;
           mbar_expect_tx(bar, gc * colb);
+#pragma unroll 1
           for (int q = 0; q < gc; q++)
             bulk_g2s(dst + q * eb, a.w_down + ((size_t)e * I + g0 + q) * d + j0, colb, bar);
         },
         [&](int j, int s) {
           const int g0 = m0 + j * per, gc = min(per, m1 - g0);
           const char* src = ring + s * per * eb;
+#pragma unroll 1
           for (int q = 0; q < gc; q++) {
             const int i = g0 + q;
             float co[NT];
@@ -1189,15 +1248,18 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
   }
   __syncthreads();
   float* out = reinterpret_cast<float*>(smem + L.x);
-  for (int idx = tid; idx < n * ncols; idx += NTHR) {
-    const int t = idx / ncols, col = idx - t * ncols;
-    float y = 0.0f;
-    for (int w = 0; w < NWARP; w++)
-      y += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[t * L.cols_max + col];
-    out[idx] = y;
-  }
+#pragma unroll 1
+  for (int t = 0; t < n; t++)
+    for (int col = tid; col < ncols; col += NTHR) {
+      float y = 0.0f;
+#pragma unroll 1
+      for (int w = 0; w < NWARP; w++)
+        y += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[t * L.cols_max + col];
+      out[t * L.cols_max + col] = y;
+    }
   __syncthreads();
-  write_and_combine(a, rank, j0, ncols, out, misc, FUSED ? reinterpret_cast<const float*>(misc + MI_RW) : a.ws.wts);
+  write_and_combine(a, rank, j0, ncols, L.cols_max, out, misc,
+                    FUSED ? reinterpret_cast<const float*>(misc + MI_RW) : a.ws.wts);
 }
 
 // ---------------------------------------------------------- launch plans
@@ -1210,21 +1272,23 @@ struct LaunchPlan {
 int g_forced_cs = 0;  // 0: automatic
 
 template <int NT, bool FUSED>
-const void* kernel_ptr(bool dense) {
-  return dense ? reinterpret_cast<const void*>(&dense_kernel<NT, FUSED>)
-               : reinterpret_cast<const void*>(&reader_kernel<NT, FUSED>);
+const void* kernel_ptr(bool dense, bool dbg) {
+  if (dense) return reinterpret_cast<const void*>(&dense_kernel<NT, FUSED>);
+  return dbg ? reinterpret_cast<const void*>(&reader_kernel<NT, FUSED, true>)
+             : reinterpret_cast<const void*>(&reader_kernel<NT, FUSED, false>);
 }
 static_assert(kMaxGroup == 2, "kernels are instantiated for 1 and 2 tokens per item");
-const void* pick_kernel(bool dense, int NT, bool fused) {
-  if (NT == 1) return fused ? kernel_ptr<1, true>(dense) : kernel_ptr<1, false>(dense);
-  return fused ? kernel_ptr<2, true>(dense) : kernel_ptr<2, false>(dense);
+const void* pick_kernel(bool dense, int NT, bool fused, bool dbg) {
+  if (NT == 1) return fused ? kernel_ptr<1, true>(dense, dbg) : kernel_ptr<1, false>(dense, dbg);
+  return fused ? kernel_ptr<2, true>(dense, dbg) : kernel_ptr<2, false>(dense, dbg);
 }
 
 // Cluster size: among 8..16 (those that fit this shape), the one with the
-// fewest waves per CTA of width, ceil(items / co-resident clusters) / cs,
-// ties to the larger cluster.  Ring: the deepest that fits, with room for the
+// least estimated time, waves * (1 + 8 / cs) with waves = ceil(items /
+// co-resident clusters): a wave costs a fixed latency plus work that shrinks
+// with the cluster's width.  Ring: the deepest that fits, with room for the
 // per-warp partial sums [NT, cols + r] fp32 of the down stage (and, with the
-// fused router, for the CTA's router rows and an fp32 transform scratch).
+// in-kernel router, for the CTA's router rows and an fp32 transform scratch).
 cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
   thread_local LaunchPlan cache[16];
   thread_local int ncache = 0, next = 0;
@@ -1245,9 +1309,11 @@ cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
   int smem_max = 0;
   err = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (err != cudaSuccess) return err;
-  const void* fn = pick_kernel(dense, NT, fused);
-  err = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (err != cudaSuccess) return err;
+  const void* fns[2] = {pick_kernel(dense, NT, fused, false), pick_kernel(dense, NT, fused, true)};
+  for (const void* f : fns) {
+    err = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (err != cudaSuccess) return err;
+  }
   LaunchPlan p = {dev, (int)dense, NT, (int)fused, a.B, a.E, a.I, a.d, a.r, items, g_forced_cs, 0, 0, 0, 0, {}};
   double best = 1e30;
   const int ntok = fused ? a.B : NT;
@@ -1265,27 +1331,31 @@ cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
     }
     if (rr < 2) continue;
     const Layout L = make_layout(NT, ntok, fused, a.E, a.I, a.d, a.r, cs, rr, dense);
-    err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
-    if (err != cudaSuccess) return err;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cs);
-    cfg.blockDim = dim3(NTHR);
-    cfg.dynamicSmemBytes = L.total;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int nclusters = 0;
-    err = cudaOccupancyMaxActiveClusters(&nclusters, fn, &cfg);
-    if (err != cudaSuccess) {
-      cudaGetLastError();
-      continue;
+    int nclusters = 1 << 30;
+    for (const void* f : fns) {
+      err = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+      if (err != cudaSuccess) return err;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(cs);
+      cfg.blockDim = dim3(NTHR);
+      cfg.dynamicSmemBytes = L.total;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = cs;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int nc = 0;
+      err = cudaOccupancyMaxActiveClusters(&nc, f, &cfg);
+      if (err != cudaSuccess) {
+        cudaGetLastError();
+        nc = 0;
+      }
+      nclusters = nc < nclusters ? nc : nclusters;
     }
     if (nclusters < 1) continue;
-    const double cost = (double)cdiv(items, nclusters) / cs;
+    const double cost = (double)cdiv(items, nclusters) * (1.0 + 8.0 / cs);
     if (cost < best - 1e-12) {
       best = cost;
       p.cs = cs;
@@ -1309,7 +1379,9 @@ cudaError_t launch_expert(const ExpertArgs& a0, cudaStream_t s, bool dense) {
   if (err != cudaSuccess) return err;
   a.cs = plan.cs;
   a.ring_rows = plan.ring_rows;
-  const void* fn = pick_kernel(dense, plan.NT, plan.fused);
+  const bool dbg = a.dbg_ids || a.dbg_w || a.dbg_G || a.dbg_U || a.dbg_sigma || a.dbg_cand || a.dbg_kept ||
+                   a.dbg_a_kept || a.dbg_y_expert || a.dbg_phase;
+  const void* fn = pick_kernel(dense, plan.NT, plan.fused, dbg);
   err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -1325,7 +1397,7 @@ cudaError_t launch_expert(const ExpertArgs& a0, cudaStream_t s, bool dense) {
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = plan.fused ? 1 : 2;  // the fused kernel is the step's first
+  cfg.numAttrs = plan.fused ? 1 : 2;  // the in-kernel router makes it the step's first kernel
   void* args[] = {&a, &plan.L};
   return cudaLaunchKernelExC(&cfg, fn, args);
 }

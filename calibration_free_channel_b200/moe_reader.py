@@ -240,7 +240,7 @@ class Layer:
                          kept=torch.empty(P + (k,), dtype=torch.int32, device=dev),
                          a_kept=torch.empty(P + (k,), dtype=torch.float32, device=dev),
                          y_expert=torch.empty(P + (self.d,), dtype=torch.float32, device=dev),
-                         phase_ns=torch.zeros((B * self.top_e, 8), dtype=torch.int64, device=dev))
+                         phase_ns=torch.zeros((B * self.top_e, 16), dtype=torch.int64, device=dev))
             dbg = MoeReaderDebug(*[_ptr(dbg_t[n]) for n, _ in MoeReaderDebug._fields_])
         moe_reader_forward(self.struct(r), B, k, c, x, residual, y, dbg, ws, ws.numel(), stream)
         return (y, dbg_t) if debug else y

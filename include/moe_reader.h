@@ -88,10 +88,15 @@ typedef struct {
   int32_t* kept;     /* [B, top_e, k] kept channels, ascending                   */
   float* a_kept;     /* [B, top_e, k] exact silu(g)*u of the kept channels        */
   float* y_expert;   /* [B, top_e, d] fp32 expert output before the combine      */
-  uint64_t* phase_ns; /* [B * top_e, 8] device clock (ns) at the stage boundaries of
-                         the sparse expert kernel, one row per work item: start,
-                         item known, screen done, candidates chosen, exact stage
-                         done, kept chosen, down done, combined              */
+  uint64_t* phase_ns; /* [B * top_e, 16] device clock (ns) at the stage
+                         boundaries of the sparse expert kernel, one row per work
+                         item (its first CTA): 0 start, 1 token rotated, 2 router
+                         logits done, 3 logits exchanged, 4 item known, 5 screen
+                         dots done, 6 screen pushed, 7 screen exchanged,
+                         8 candidates chosen, 9 union listed, 10 exact stage done,
+                         11 exact exchanged, 12 kept chosen, 13 kept listed,
+                         14 down + recovery done, 15 combined; 0 where a stage
+                         does not run (routing stamps need B <= 2)            */
 } moe_reader_debug;
 
 /* Bytes of device workspace moe_reader_forward / moe_reader_forward_dense
