@@ -269,7 +269,7 @@ def run_native(args, rank, world, local_rank):
         "step_roofline_frac": round(value / world / peak, 4),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": B * shape.d * 2,
                 "d2h_bytes_per_step": B * shape.d * 2, "us_per_step": float(t[0]) * 1e3},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": (1 if B <= 2 else 3) * args.steps,  # in-kernel routing at B <= 2
         "clocks": clocks,
         "dense": dense,
     }
