@@ -166,6 +166,11 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
 
 }  // namespace
 
+moe_status moe::set_last_error(moe_status st, const char* msg) {
+  g_err = msg;
+  return st;
+}
+
 extern "C" {
 
 size_t moe_reader_workspace_bytes(int B, int E, int top_e, int I, int d, int k, int c, int r) {

@@ -4,7 +4,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/moe_reader.h"
+
 namespace moe {
+
+// Records the message returned by moe_reader_last_error and returns st.
+moe_status set_last_error(moe_status st, const char* msg);
 
 // Workspace carved out of the caller's buffer (see workspace_layout).
 struct Workspace {

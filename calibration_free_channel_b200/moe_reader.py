@@ -21,7 +21,7 @@ EXPORTS = ["moe_reader_workspace_bytes", "moe_reader_build_sketch", "moe_reader_
            "moe_reader_build_lowrank", "moe_reader_forward", "moe_reader_forward_dense",
            "moe_reader_forward_host", "moe_reader_rmsnorm", "moe_reader_set_expert_events",
            "moe_reader_check_error", "moe_reader_set_cluster_size", "moe_reader_launch_plan",
-           "moe_reader_last_error"]
+           "moe_reader_forward_noalloc", "moe_reader_last_error"]
 
 
 class MoeReaderLayer(C.Structure):
@@ -69,6 +69,7 @@ def lib():
         L.moe_reader_check_error.argtypes = [P, P]
         L.moe_reader_set_cluster_size.argtypes = [i32]
         L.moe_reader_launch_plan.argtypes = [i32] * 7 + [P]
+        L.moe_reader_forward_noalloc.argtypes = [C.POINTER(MoeReaderLayer), i32, i32, i32, P, P, P, P]
         L.moe_reader_last_error.restype = C.c_char_p
         L.moe_reader_last_error.argtypes = []
         for f in EXPORTS:
@@ -128,6 +129,13 @@ def moe_reader_forward(layer: MoeReaderLayer, B, k, c, x, residual, y, dbg, work
 def moe_reader_forward_dense(layer: MoeReaderLayer, B, x, residual, y, workspace, ws_bytes, stream=None):
     _check(lib().moe_reader_forward_dense(C.byref(layer), B, _ptr(x), _ptr(residual), _ptr(y), _ptr(workspace),
                                           ws_bytes, _stream(stream)))
+
+
+def moe_reader_forward_noalloc(layer: MoeReaderLayer, B, k, c, x, residual, y, stream=None):
+    """The step with the library's fixed device scratch (no workspace
+    argument): for callers that cannot allocate device memory."""
+    _check(lib().moe_reader_forward_noalloc(C.byref(layer), B, k, c, _ptr(x), _ptr(residual), _ptr(y),
+                                            _stream(stream)))
 
 
 def moe_reader_forward_host(layer: MoeReaderLayer, B, k, c, x_host, x_dev, y_dev, y_host, workspace, ws_bytes,

@@ -172,6 +172,25 @@ moe_status moe_reader_forward_host(const moe_reader_layer* layer, int B, int k, 
                                    const uint16_t* x_host, uint16_t* x_dev, uint16_t* y_dev,
                                    uint16_t* y_host, void* workspace, size_t ws_bytes, void* stream);
 
+/* moe_reader_forward with no caller-provided workspace, for callers that
+ * cannot allocate device memory: code that runs while a stream is captured
+ * into a CUDA graph, serving loops that forbid allocation after start-up,
+ * hosts whose device allocator belongs to another runtime.  (The paper has no
+ * counterpart; this is an interface convenience.)
+ *  - The scratch is a fixed 8 MiB __device__ array inside the library; every
+ *    GPU that loads the library holds it until the process exits.  Shapes
+ *    whose workspace (moe_reader_workspace_bytes) exceeds 8 MiB return
+ *    MOE_EINVAL ("workspace has ... bytes, needs ...") and launch nothing.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Every call shares the one array per device: calls that may overlap on
+ *    the GPU (different streams, no ordering) race and must not be issued.
+ *    Each call first clears the array's combine counters (cudaMemsetAsync on
+ *    `stream`); nothing is allocated or freed.
+ *  - No debug outputs; errors as for moe_reader_forward. */
+moe_status moe_reader_forward_noalloc(const moe_reader_layer* layer, int B, int k, int c,
+                                      const uint16_t* x, const uint16_t* residual, uint16_t* y, void* stream);
+
 /* Between stacked layers: h = bf16(x / sqrt(mean(x^2) + eps)) per token,
  * no learned gain (fp32). */
 moe_status moe_reader_rmsnorm(int B, int d, float eps, const uint16_t* x, uint16_t* h, void* stream);
