@@ -51,7 +51,7 @@ moe_status check_shape(int B, int E, int top_e, int I, int d) {
   REQUIRE(E >= 1 && E <= 1024, "E = %d outside [1, 1024]", E);
   REQUIRE(top_e >= 1 && top_e <= 16 && top_e <= E, "top_e = %d outside [1, min(E, 16)]", top_e);
   REQUIRE(I >= 16 && I <= 2048, "I = %d outside [16, 2048]", I);
-  REQUIRE(pow2(d) && d >= 128 && d <= 4096, "d = %d is not a power of two in [128, 4096]", d);
+  REQUIRE(pow2(d) && d >= 256 && d <= 4096, "d = %d is not a power of two in [256, 4096]", d);
   return MOE_OK;
 }
 

@@ -5,7 +5,8 @@
 // gate and up weights, resident on the GPU, made from the weights alone.
 // Per row: w' = H (s . w) (unnormalised Sylvester Walsh-Hadamard, fp32, stages
 // h = 1, 2, 4, ...); Delta = 0.7 mean|w'| and alpha = mean |w'| over the kept
-// entries, both fp64 in index order (TWN, Li & Liu 2016); 2-bit codes.  The
+// entries, both fp64 in index order (TWN, Li & Liu 2016); 2-bit codes T + 1,
+// position 4p + b of a 16-position word at bits 8b + 2p.  The
 // index-order sums are done by one thread per row so the result equals the
 // serial definition bit for bit.
 #include "common.cuh"
@@ -87,10 +88,9 @@ __global__ void __launch_bounds__(256) sketch_kernel(int E, int I, int d, const 
 #pragma unroll
     for (int p = 0; p < 16; p++) {
       const float xv = x[p];
-      uint32_t code = 0;
-      if (fabs((double)xv) > dl) code = xv > 0.0f ? 1u : 3u;
-      const int sh = p < 8 ? 4 * p : 4 * (p - 8) + 2;
-      word |= code << sh;
+      uint32_t code = 1u;  // T + 1
+      if (fabs((double)xv) > dl) code = xv > 0.0f ? 2u : 0u;
+      word |= code << (8 * (p & 3) + 2 * (p >> 2));
     }
     const long g = row0 + rr;
     if (g < rows_per_mat) skg[g * words + m] = word;

@@ -8,11 +8,10 @@ namespace moe {
 
 namespace cg = cooperative_groups;
 
-constexpr int kThreads = 256;          // threads per CTA of the expert kernels
+constexpr int kThreads = 256;          // threads per CTA of the route kernel
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxSlots = 16;          // row slots per warp in the copy rings
 constexpr int kMaxGroup = 2;           // tokens per work item (tokens sharing an expert)
-constexpr int kMaxRank = 128;
 constexpr int kMaxCluster = 16;
 constexpr int kMaxTokens = 256;        // tokens per step (B)
 
@@ -110,6 +109,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
   }
 }
+// Raises the transaction count of the current phase without arriving.
+__device__ __forceinline__ void mbar_expect_tx_only(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+// L2 prefetch of the line holding p.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -137,32 +144,26 @@ __device__ __forceinline__ T warp_sum(T v) {
 }
 
 // Ternary-sketch dot of one packed row word with 16 int8 activations.
-// Word layout: position n (< 8) at bits [4n, 4n+1], position 8+n at bits
-// [4n+2, 4n+3]; codes 00 = 0, 01 = +1, 11 = -1.  A nibble's code selects a
-// byte of kTritLut = {0x00, 0x01, 0x00, 0xff} (byte_perm), giving the trits
-// as signed bytes; dp4a multiplies them with the activations exactly.
-__device__ __forceinline__ int trit_dot16(uint32_t w, uint4 q, int acc) {
-  const uint32_t kTritLut = 0xff000100u;
-  const uint32_t lo = w & 0x33333333u;
-  const uint32_t hi = (w >> 2) & 0x33333333u;
-  acc = __dp4a((int)__byte_perm(kTritLut, 0, lo & 0xffffu), (int)q.x, acc);
-  acc = __dp4a((int)__byte_perm(kTritLut, 0, lo >> 16), (int)q.y, acc);
-  acc = __dp4a((int)__byte_perm(kTritLut, 0, hi & 0xffffu), (int)q.z, acc);
-  acc = __dp4a((int)__byte_perm(kTritLut, 0, hi >> 16), (int)q.w, acc);
-  return acc;
+// Word layout: position 4p + b (p, b in 0..3) at bits [8b + 2p, 8b + 2p + 1]
+// as the code T + 1 (0, 1 or 2).  Masking the word with 0x03030303 << 2p
+// leaves the codes of positions 4p .. 4p+3 in four bytes, scaled by 4^p;
+// dp4a multiplies them with the activation bytes exactly.  The four partial
+// sums are kept apart (acc[p] is a multiple of 4^p) and combined by
+// code_dot_total; the row's code offset is removed by subtracting the sum of
+// the activations once per row.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
-
-// 8 bf16 (one uint4) times 8 bf16, accumulated in fp32.
-__device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
-  acc = fmaf(bf16lo(a.x), bf16lo(b.x), acc);
-  acc = fmaf(bf16hi(a.x), bf16hi(b.x), acc);
-  acc = fmaf(bf16lo(a.y), bf16lo(b.y), acc);
-  acc = fmaf(bf16hi(a.y), bf16hi(b.y), acc);
-  acc = fmaf(bf16lo(a.z), bf16lo(b.z), acc);
-  acc = fmaf(bf16hi(a.z), bf16hi(b.z), acc);
-  acc = fmaf(bf16lo(a.w), bf16lo(b.w), acc);
-  acc = fmaf(bf16hi(a.w), bf16hi(b.w), acc);
-  return acc;
+__device__ __forceinline__ void code_dot16(uint32_t w, uint4 q, int (&acc)[4]) {
+  acc[0] = dp4a_us(w & 0x03030303u, q.x, acc[0]);
+  acc[1] = dp4a_us(w & 0x0c0c0c0cu, q.y, acc[1]);
+  acc[2] = dp4a_us(w & 0x30303030u, q.z, acc[2]);
+  acc[3] = dp4a_us(w & 0xc0c0c0c0u, q.w, acc[3]);
+}
+__device__ __forceinline__ int code_dot_total(const int (&acc)[4]) {
+  return acc[0] + (acc[1] >> 2) + (acc[2] >> 4) + (acc[3] >> 6);
 }
 
 }  // namespace moe

@@ -25,15 +25,20 @@
 //      y_e = sum_K a_i W_down[i,:] + V z, z = sum_{i not in K} ahat_i Ubar_i;
 //   combine: the last of a token's top_e experts to finish a column slice sums
 //      w_s y_e,s in slot order, writes bf16 y and resets the slice's counter.
-// Rows move with 1-D bulk copies (cp.async.bulk) into per-warp rings in the
-// CTA's own shared memory; every wait on them is bounded.  Every exchange
-// between the CTAs of a cluster is a store into the receivers' shared memory
-// followed by a cluster barrier: no CTA reads another CTA's shared memory.
 //
-// At batch 1 the step is a chain of short dependent stages whose code runs
-// once per launch, so instruction fetch is a first-order cost: the kernels
-// keep their static code small (host-computed geometry instead of runtime
-// divisions, short loops kept rolled, one shared copy of the selection).
+// Large contiguous rows (sketch chunks of 16 channels, BF16 gate/up rows)
+// move with 1-D bulk copies (cp.async.bulk) into shared memory, waited on
+// through mbarriers with bounded waits.  The many short row slices of the
+// down stage are plain 16-byte loads spread over all threads: a bulk copy
+// costs the SM's copy engine a fixed issue time per copy, which dominates
+// for slices of a few hundred bytes.  Every exchange between the CTAs of a
+// cluster is a store into the receivers' shared memory followed by a cluster
+// barrier: no CTA reads another CTA's shared memory.
+//
+// At batch 1 the step is a chain of short dependent stages, so the kernels
+// are written for latency: few block barriers per stage, no serial loops over
+// warps, the rotation placed under the sketch's DRAM latency, the screen's
+// byte-wise dots on pre-masked code words.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -43,7 +48,9 @@ namespace {
 
 constexpr int NTHR = 512;
 constexpr int NWARP = NTHR / 32;
-constexpr int kMaxCols = 256;  // output columns per CTA (8 per lane)
+constexpr int kMaxCols = 256;  // output columns per CTA
+constexpr int kSkBars = 16;    // sketch chunk barriers (a chunk is 16 channels)
+constexpr unsigned kFull = 0xffffffffu;
 
 __host__ __device__ inline int rup(int x, int a) { return (x + a - 1) / a * a; }
 __host__ __device__ inline int cdiv(int x, int a) { return (x + a - 1) / a; }
@@ -54,17 +61,18 @@ __device__ __noinline__ int idiv(int a, int b) { return a / b; }
 // ------------------------------------------------------- launch geometry
 // Shared-memory offsets and the partitions of a launch, computed on the host.
 struct Layout {
-  int mbar, misc, hist, wtot, pmask, x, q, logit, sig, ahat, zparts, z, apos, candm, keptm, ulist, upos, dlist,
-      keys, kidx, ubar, vown, ring, total;
+  int mbar, misc, hist, x, q, logit, alpha, sig, sa, zred, zparts, z, cor, apos, candm, keptm, ulist, dlist, keys,
+      ubar, vown, ring, total;
   int ntok;        // tokens held in smem (fused routing: B; otherwise NT)
   int own_max;     // max channels per CTA
   int cols_max;    // max output columns per CTA
   int words;       // mask words over I
   int ring_bytes;  // per warp
-  int d8, d16;     // d / 8, d / 16
-  int s_per;       // channels per screen slot (half a ring)
-  int c_slots;     // candidate-pair slots per warp
-  int ch0[17];     // channel partition over the CTAs of a cluster
+  int d8, d64;     // d / 8, d / 64
+  int c_slots;     // candidate row slots (gate + up) per warp
+  int skc;         // bytes of 16 sketch rows of one matrix
+  int sk_round;    // sketch chunks resident at once
+  int ch0[17];     // channel partition over the CTAs of a cluster (multiples of 4)
   int col0[17];    // output-column partition (multiples of 8)
   int ex0[17];     // expert partition (in-kernel routing)
 };
@@ -73,17 +81,21 @@ __host__ inline Layout make_layout(int NT, int ntok, bool fused, int E, int I, i
                                    int ring_rows, bool dense) {
   Layout L = {};
   L.ntok = ntok;
-  L.own_max = cdiv(I, cs);
+  for (int o = 0; o <= cs && o < 17; o++) {
+    const int c4 = 4 * cdiv(o * cdiv(I, 4), cs);
+    L.ch0[o] = c4 < I ? c4 : I;
+  }
+  L.own_max = 0;
+  for (int o = 0; o < cs && o < 16; o++)
+    if (L.ch0[o + 1] - L.ch0[o] > L.own_max) L.own_max = L.ch0[o + 1] - L.ch0[o];
   L.cols_max = 8 * cdiv(d / 8, cs);
   L.words = cdiv(I, 32);
   L.ring_bytes = ring_rows * d * 2;
   L.d8 = d / 8;
-  L.d16 = d / 16;
-  L.s_per = (L.ring_bytes / 2) / (2 * (d / 4));
-  if (L.s_per > 32) L.s_per = 32;  // one alpha per lane
+  L.d64 = d / 64;
   L.c_slots = L.ring_bytes / (4 * d);
+  L.skc = 16 * (d / 4);
   for (int o = 0; o <= cs && o < 17; o++) {
-    L.ch0[o] = cdiv(o * I, cs);
     L.col0[o] = 8 * cdiv(o * (d / 8), cs);
     L.ex0[o] = cdiv(o * E, cs);
   }
@@ -94,39 +106,44 @@ __host__ inline Layout make_layout(int NT, int ntok, bool fused, int E, int I, i
     o = rup(o + bytes, 128);
     return at;
   };
-  L.mbar = take((NWARP * kMaxSlots + 4) * 8);
+  L.mbar = take((NWARP * kMaxSlots + kSkBars + 2) * 8);
   L.misc = take(256 * 4);
   L.hist = take(2 * 2048 * 4);
-  L.wtot = take(64 * 4);
-  L.pmask = take(L.words * 4);
   L.x = take(ntok * d * 2);
-  L.q = take(ntok * d);
+  L.q = dense ? 0 : take(ntok * d);
   L.logit = fused ? take(ntok * E * 8) : 0;
-  L.sig = take(NT * I * 4);  // sparse: sigma by channel; dense: h by channel
-  L.ahat = dense ? 0 : take(NT * I * 4);
+  L.alpha = dense ? 0 : take(2 * L.own_max * 4);
+  L.sig = dense ? take(NT * I * 4) : 0;           // dense: h by channel
+  L.sa = dense ? 0 : take(rup(I, 4) * NT * 8);    // sparse: (sigma, ahat) by channel, token
+  L.zred = dense ? 0 : take(NWARP * NT * rr * 4);
   L.zparts = dense ? 0 : take(cs * NT * rr * 4);
   L.z = dense ? 0 : take(NT * rr * 4);
+  L.cor = dense ? 0 : take(NT * rr * 4);
   L.apos = dense ? 0 : take(NT * I * 4);  // a by union position
   L.candm = dense ? 0 : take(NT * L.words * 4);
   L.keptm = dense ? 0 : take(NT * L.words * 4);
   L.ulist = dense ? 0 : take(I * 4);
-  L.upos = dense ? 0 : take(I * 4);
   L.dlist = dense ? 0 : take(I * 4);
   L.keys = dense ? 0 : take(I * 4);
-  L.kidx = dense ? 0 : take(I * 4);
   L.ubar = dense ? 0 : take(L.own_max * rr * 2);
   L.vown = dense ? 0 : take(L.cols_max * rr * 2);
   L.ring = take(NWARP * L.ring_bytes);
   L.total = o;
+  const int region = NWARP * L.ring_bytes;
+  int rounds = (region - 4 * d) / (2 * L.skc);
+  if (rounds > kSkBars) rounds = kSkBars;
+  if (rounds > cdiv(L.own_max, 16)) rounds = cdiv(L.own_max, 16);
+  L.sk_round = dense ? 0 : (rounds > 0 ? rounds : 0);
   return L;
 }
 
 // misc ints
 enum {
-  MI_E = 0, MI_N, MI_NU, MI_ND, MI_NC, MI_DIG, MI_REM, MI_CNT, MI_DONE,
-  MI_TOK = 16, MI_SLOT = 32, MI_LAST = 48, MI_TIX = 64, MI_CX = 80, MI_SCAN = 96,
+  MI_E = 0, MI_N, MI_NU, MI_ND, MI_DIG, MI_REM, MI_CNT, MI_DONE,
+  MI_TOK = 16, MI_SLOT = 32, MI_LAST = 48, MI_TIX = 64, MI_CX = 80, MI_RED = 96, MI_WT = 112,
   MI_RIDS = 128,  // in-kernel routing: ids [B <= 2][top_e <= 16]
-  MI_RW = 192     // in-kernel routing: weights
+  MI_RW = 192,    // in-kernel routing: weights
+  MI_FID = 224    // in-kernel routing: first-occurrence ids
 };
 
 // ---------------------------------------------------------- cluster helpers
@@ -142,6 +159,11 @@ __device__ __forceinline__ uint32_t cluster_addr(const void* local, int rank) {
 }
 __device__ __forceinline__ void st_cluster(const void* local, int rank, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr(local, rank)), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster(const void* local, int rank, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr(local, rank)), "f"(v.x),
+               "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
 }
 __device__ __forceinline__ void st_cluster(const void* local, int rank, double v) {
   asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(cluster_addr(local, rank)), "d"(v) : "memory");
@@ -162,110 +184,89 @@ __device__ __forceinline__ void dot8_mixed(uint4 a, uint4 b, float& acc0, float&
       : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w));
 }
 
-// Trits of one packed sketch word as four words of signed bytes.  Layout:
-// position n (< 8) at bits [4n, 4n+1], position 8+n at bits [4n+2, 4n+3];
-// codes 00 = 0, 01 = +1, 11 = -1.  A nibble's code selects a byte of
-// kTritLut = {0x00, 0x01, 0x00, 0xff} through byte_perm.
-__device__ __forceinline__ uint4 decode_trits(uint32_t w) {
-  const uint32_t kTritLut = 0xff000100u;
-  const uint32_t lo = w & 0x33333333u;
-  const uint32_t hi = (w >> 2) & 0x33333333u;
-  return make_uint4(__byte_perm(kTritLut, 0, lo), __byte_perm(kTritLut, 0, lo >> 16),
-                    __byte_perm(kTritLut, 0, hi), __byte_perm(kTritLut, 0, hi >> 16));
-}
-__device__ __forceinline__ int dot16_i8(uint4 t, uint4 q, int acc) {
-  acc = __dp4a((int)t.x, (int)q.x, acc);
-  acc = __dp4a((int)t.y, (int)q.y, acc);
-  acc = __dp4a((int)t.z, (int)q.z, acc);
-  acc = __dp4a((int)t.w, (int)q.w, acc);
-  return acc;
-}
-
 // ----------------------------------------------------------- block helpers
-__device__ __noinline__ int block_excl_scan(int v, int* scratch, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int inc = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += n;
-  }
-  if (lane == 31) scratch[warp] = inc;
-  __syncthreads();
-  int off = 0, tot = 0;
-#pragma unroll 1
-  for (int w = 0; w < NWARP; w++) {
-    const int s = scratch[w];
-    off += w < warp ? s : 0;
-    tot += s;
-  }
-  __syncthreads();
-  *total = tot;
-  return off + inc - v;
-}
-
-// Top-n_sel of N keys (uint32, larger first, ties to the lower position):
-// radix select with digits of 11, 11 and 10 bits from the top, stopping as
-// soon as the boundary bin is taken whole; keys equal to a fully resolved
-// threshold are taken in position order.  Sets bit p of out_mask for each
-// chosen position p.  hist holds 2 x 2048 ints, wtot 16 ints.
-__device__ __noinline__ void block_select_top(const uint32_t* keys, int N, int n_sel, int* hist, int* wtot,
+// Top-n_sel of N <= 2048 keys (uint32, larger first, ties to the lower
+// position): radix select with digits of 11, 11 and 10 bits from the top.
+// A pass counts the keys that share the decided prefix into the bins of the
+// next digit (shared-memory atomics), scans the bins from the top (each warp
+// a run of bins, warp totals through shared memory) and finds the boundary
+// digit.  The selection stops as soon as the boundary bin is taken whole;
+// after the last digit the threshold T is fully resolved and the first keys
+// equal to T by position fill the rest.  Bit p of out_mask (p < N, words
+// [0, ceil(N / 32))) is set for each chosen position p.  Key p sits at
+// keys[p * kstride].  hist holds 2 x 2048 ints; misc[MI_WT ..] 16 ints of
+// warp totals.
+__device__ __noinline__ void block_select_top(const uint32_t* keys, int kstride, int N, int n_sel, int* hist,
                                               int* misc, uint32_t* out_mask) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nw = (N + 31) >> 5;
-  for (int w = tid; w < nw; w += NTHR) out_mask[w] = 0u;
-  if (n_sel >= N) {
-    __syncthreads();
-    for (int p = tid; p < N; p += NTHR) atomicOr(&out_mask[p >> 5], 1u << (p & 31));
+  if (n_sel >= N || n_sel <= 0) {
+    for (int w = tid; w < nw; w += NTHR) {
+      const int left = N - 32 * w;
+      out_mask[w] = n_sel <= 0 ? 0u : left >= 32 ? kFull : (1u << left) - 1u;
+    }
     __syncthreads();
     return;
   }
-  for (int b = tid; b < 2048; b += NTHR) hist[b] = 0;
+  reinterpret_cast<int4*>(hist)[tid] = make_int4(0, 0, 0, 0);  // bins 0 .. 2047 (NTHR * 4 = 2048)
+  int* wt = misc + MI_WT;
+  __syncthreads();
   uint32_t prefix = 0u, mask = 0u;
   int rem = n_sel;
   bool done = false;
 #pragma unroll 1
-  for (int pass = 0; pass < 3 && !done; pass++) {
+  for (int pass = 0; pass < 3; pass++) {
     const int shift = pass == 0 ? 21 : pass == 1 ? 10 : 0;
-    const int lnb = pass == 2 ? 10 : 11;
-    const int nb = 1 << lnb;
+    const int nb = pass == 2 ? 1024 : 2048;
     int* h = hist + (pass & 1) * 2048;
-    int* hn = hist + ((pass + 1) & 1) * 2048;
-    __syncthreads();  // h is zero and the previous pass is done with hn
-    for (int p = tid; p < N; p += NTHR) {
-      const uint32_t k = keys[p];
-      if ((k & mask) == prefix) atomicAdd(&h[(k >> shift) & (nb - 1)], 1);
-    }
-    for (int b = tid; b < 2048; b += NTHR) hn[b] = 0;
-    __syncthreads();
-    // warp w covers bins [nb - (w+1) bpw, nb - w bpw), top-down; lane l a run
-    const int bpl = nb >> 9;                            // bins per lane (4 or 2)
-    const int top = nb - (warp * 32 + lane) * bpl;      // bins top-1 .. top-bpl
-    int s = 0;
 #pragma unroll 1
-    for (int j = 1; j <= bpl; j++) s += h[top - j];
+    for (int base = 0; base < N; base += NTHR) {
+      const int p = base + tid;
+      if (p < N) {
+        const uint32_t k = keys[p * kstride];
+        if ((k & mask) == prefix) atomicAdd(&h[(k >> shift) & (nb - 1)], 1);
+      }
+    }
+    // the other half is zeroed for the next pass (its counts were read before the last barrier)
+    if (pass < 2) reinterpret_cast<int4*>(hist + ((pass + 1) & 1) * 2048)[tid] = make_int4(0, 0, 0, 0);
+    __syncthreads();
+    // thread (warp, lane) scans bins top - 1 .. top - bpl, top = nb - (32 warp + lane) bpl
+    const int bpl = nb >> 9;
+    const int top = nb - (warp * 32 + lane) * bpl;
+    int c[4];
+    if (bpl == 4) {
+      const int4 v = reinterpret_cast<const int4*>(h)[(top >> 2) - 1];
+      c[0] = v.w; c[1] = v.z; c[2] = v.y; c[3] = v.x;
+    } else {
+      const int2 v = reinterpret_cast<const int2*>(h)[(top >> 1) - 1];
+      c[0] = v.y; c[1] = v.x; c[2] = 0; c[3] = 0;
+    }
+    const int s = c[0] + c[1] + c[2] + c[3];
     int inc = s;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += n;
+      const int nb2 = __shfl_up_sync(kFull, inc, o);
+      if (lane >= o) inc += nb2;
     }
-    if (lane == 31) wtot[warp] = inc;
+    if (lane == 31) wt[warp] = inc;
     __syncthreads();
-    int before = inc - s;  // keys in bins above this lane's run
-#pragma unroll 1
-    for (int w = 0; w < warp; w++) before += wtot[w];
+    int before = inc - s;
+#pragma unroll
+    for (int w4 = 0; w4 < NWARP; w4 += 4) {
+      const int4 t4 = reinterpret_cast<const int4*>(wt)[w4 >> 2];
+      before += (w4 < warp ? t4.x : 0) + (w4 + 1 < warp ? t4.y : 0) + (w4 + 2 < warp ? t4.z : 0) +
+                (w4 + 3 < warp ? t4.w : 0);
+    }
     if (before < rem && before + s >= rem) {
-#pragma unroll 1
-      for (int j = 1; j <= bpl; j++) {
-        const int c = h[top - j];
-        if (before + c >= rem) {
-          misc[MI_DIG] = top - j;
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        if (before + c[j] >= rem) {
+          misc[MI_DIG] = top - 1 - j;
           misc[MI_REM] = rem - before;
-          misc[MI_CNT] = c;
+          misc[MI_CNT] = c[j];
           break;
         }
-        before += c;
+        before += c[j];
       }
     }
     __syncthreads();
@@ -273,49 +274,82 @@ __device__ __noinline__ void block_select_top(const uint32_t* keys, int N, int n
     mask |= (uint32_t)(nb - 1) << shift;
     rem = misc[MI_REM];
     done = rem == misc[MI_CNT];
+    if (done) break;
   }
   if (done) {
-    // the boundary bin is taken whole: keep every key whose decided bits are
-    // at least the boundary prefix
-    for (int p = tid; p < N; p += NTHR)
-      if ((keys[p] & mask) >= prefix) atomicOr(&out_mask[p >> 5], 1u << (p & 31));
+    // the boundary bin is taken whole: every key whose decided bits are at
+    // least the boundary prefix
+#pragma unroll 1
+    for (int base = 0; base < N; base += NTHR) {
+      const int p = base + tid;
+      const unsigned bal = __ballot_sync(kFull, p < N && (keys[p * kstride] & mask) >= prefix);
+      const int w = (base >> 5) + warp;
+      if (lane == 0 && w < nw) out_mask[w] = bal;
+    }
     __syncthreads();
     return;
   }
   // fully resolved threshold T = prefix with more equal keys than needed:
   // keys > T, and the first `rem` keys == T by position
-  const int chunk = (N + NTHR - 1) / NTHR;
-  const int p0 = min(N, tid * chunk), p1 = min(N, p0 + chunk);
-  int eq = 0;
-  for (int p = p0; p < p1; p++) eq += keys[p] == prefix;
-  int tot;
-  int before = block_excl_scan(eq, misc + MI_SCAN, &tot);
-  for (int p = p0; p < p1; p++) {
-    const uint32_t k = keys[p];
-    bool take = k > prefix;
-    if (k == prefix) take = before++ < rem;
-    if (take) atomicOr(&out_mask[p >> 5], 1u << (p & 31));
+  int* wc = hist;  // equal keys per word
+#pragma unroll 1
+  for (int base = 0; base < N; base += NTHR) {
+    const int p = base + tid;
+    const unsigned bal = __ballot_sync(kFull, p < N && keys[p * kstride] == prefix);
+    const int w = (base >> 5) + warp;
+    if (lane == 0 && w < nw) wc[w] = __popc(bal);
+  }
+  __syncthreads();
+#pragma unroll 1
+  for (int base = 0; base < N; base += NTHR) {
+    const int p = base + tid;
+    const int w = (base >> 5) + warp;
+    int before = 0;
+    for (int v = lane; v < w && v < nw; v += 32) before += wc[v];
+    before = warp_sum(before);
+    const uint32_t k = p < N ? keys[p * kstride] : 0u;
+    const unsigned eq = __ballot_sync(kFull, p < N && k == prefix);
+    const int rank = before + __popc(eq & ((1u << lane) - 1u));
+    const unsigned bal = __ballot_sync(kFull, p < N && (k > prefix || (k == prefix && rank < rem)));
+    if (lane == 0 && w < nw) out_mask[w] = bal;
   }
   __syncthreads();
 }
 
-// Ascending list of the set bits of mask over [0, N), all warps; the count
-// lands in *count_out; pos_of (if given) gets each bit's list position or -1.
-__device__ __noinline__ void block_mask_to_list(const uint32_t* mask, int N, int* list, int* pos_of,
-                                                int* count_out) {
+// Ascending list of the set bits of (m0 | m1) over [0, N), N <= 2048 (m1
+// may be null); the count lands in *count_out.  Warp 0 forms the union words
+// and their exclusive prefix counts (scratch, 64 ints each), then every warp
+// writes the positions of its words.
+__device__ __noinline__ void block_mask_to_list(const uint32_t* m0, const uint32_t* m1, int N, int* list,
+                                                int* count_out, int* scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nw = (N + 31) >> 5;
+  uint32_t* uw = reinterpret_cast<uint32_t*>(scratch + 64);
+  if (warp == 0) {
+    uint32_t a0 = 0u, a1 = 0u;
+    if (lane < nw) a0 = m0[lane] | (m1 ? m1[lane] : 0u);
+    if (lane + 32 < nw) a1 = m0[lane + 32] | (m1 ? m1[lane + 32] : 0u);
+    const int c0 = __popc(a0), c1 = __popc(a1);
+    int i0 = c0, i1 = c1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n0 = __shfl_up_sync(kFull, i0, o), n1 = __shfl_up_sync(kFull, i1, o);
+      if (lane >= o) {
+        i0 += n0;
+        i1 += n1;
+      }
+    }
+    const int t0 = __shfl_sync(kFull, i0, 31), t1 = __shfl_sync(kFull, i1, 31);
+    scratch[lane] = i0 - c0;
+    scratch[lane + 32] = t0 + i1 - c1;
+    uw[lane] = a0;
+    uw[lane + 32] = a1;
+    if (lane == 0) *count_out = t0 + t1;
+  }
+  __syncthreads();
   for (int w = warp; w < nw; w += NWARP) {
-    int off = 0;
-    for (int v = lane; v < w; v += 32) off += __popc(mask[v]);
-    off = warp_sum(off);
-    const int p = w * 32 + lane;
-    const bool on = p < N && ((mask[w] >> lane) & 1u);
-    const unsigned bal = __ballot_sync(0xffffffffu, on);
-    const int at = off + __popc(bal & ((1u << lane) - 1u));
-    if (on) list[at] = p;
-    if (pos_of && p < N) pos_of[p] = on ? at : -1;
-    if (w == nw - 1 && lane == 0) *count_out = off + __popc(bal);
+    const uint32_t m = uw[w];
+    if ((m >> lane) & 1u) list[scratch[w] + __popc(m & ((1u << lane) - 1u))] = 32 * w + lane;
   }
   __syncthreads();
 }
@@ -370,23 +404,31 @@ __device__ __forceinline__ bool warp_stream(int cnt, int P, uint64_t* bars, uint
 }
 
 // ------------------------------------------------------- work item set-up
-// The item comes from the work table the select kernel wrote.
+// The item comes from the work table the select kernel wrote (warp 0 reads
+// its fields in parallel).
 __device__ bool load_item_table(const ExpertArgs& a, int cid, int* misc, int NT) {
-  if (threadIdx.x == 0) {
-    const int n_items = *a.ws.n_items;
-    int e = -1, n = 0;
-    if (cid < n_items && cid < a.ws.max_items) {
-      e = a.ws.item_e[cid];
-      n = a.ws.item_n[cid];
-      if (e < 0 || e >= a.E || n < 1 || n > NT) {
-        atomicOr(a.ws.err, kErrBadWorkItem);
-        e = -1;
-      }
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const bool ok_cid = cid < a.ws.max_items;
+    int v = 0;
+    if (lane == 0) v = *a.ws.n_items;
+    else if (lane == 1 && ok_cid) v = a.ws.item_e[cid];
+    else if (lane == 2 && ok_cid) v = a.ws.item_n[cid];
+    else if (lane >= 4 && lane < 4 + kMaxGroup && ok_cid) v = a.ws.item_tok[cid * kMaxGroup + lane - 4];
+    else if (lane >= 8 && lane < 8 + kMaxGroup && ok_cid) v = a.ws.item_slot[cid * kMaxGroup + lane - 8];
+    const int n_items = __shfl_sync(kFull, v, 0);
+    int e = __shfl_sync(kFull, v, 1), n = __shfl_sync(kFull, v, 2);
+    if (!(cid < n_items && ok_cid)) {
+      e = -1;
+      n = 0;
+    } else if (e < 0 || e >= a.E || n < 1 || n > NT) {
+      if (lane == 0) atomicOr(a.ws.err, kErrBadWorkItem);
+      e = -1;
+      n = 0;
     }
-    misc[MI_E] = e;
-    misc[MI_N] = n;
-    for (int t = 0; t < n; t++) {
-      int tok = a.ws.item_tok[cid * kMaxGroup + t], sl = a.ws.item_slot[cid * kMaxGroup + t];
+    const int t = lane;
+    int tok = __shfl_sync(kFull, v, 4 + (t & 3)), sl = __shfl_sync(kFull, v, 8 + (t & 3));
+    if (t < n) {
       if (tok < 0 || tok >= a.B || sl < 0 || sl >= a.top_e) {
         atomicOr(a.ws.err, kErrBadWorkItem);
         tok = 0;
@@ -396,6 +438,10 @@ __device__ bool load_item_table(const ExpertArgs& a, int cid, int* misc, int NT)
       misc[MI_SLOT + t] = sl;
       misc[MI_TIX + t] = t;  // tokens are loaded in item order
       reinterpret_cast<float*>(misc + MI_CX)[t] = a.ws.cx[tok];
+    }
+    if (lane == 0) {
+      misc[MI_E] = e;
+      misc[MI_N] = n;
     }
   }
   __syncthreads();
@@ -413,25 +459,28 @@ __device__ void load_tokens(const ExpertArgs& a, const Layout& L, char* smem, co
     for (int j = threadIdx.x; j < L.d8; j += NTHR)
       xs[t * L.d8 + j] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)tok * a.d) + j);
     if (with_q)
-      for (int j = threadIdx.x; j < L.d16; j += NTHR)
-        qs[t * L.d16 + j] = __ldcg(reinterpret_cast<const uint4*>(a.ws.q + (size_t)tok * a.d) + j);
+      for (int j = threadIdx.x; j < L.d8 / 2; j += NTHR)
+        qs[t * (L.d8 / 2) + j] = __ldcg(reinterpret_cast<const uint4*>(a.ws.q + (size_t)tok * a.d) + j);
   }
 }
 
 // Rotation + int8 quantisation of smem token t: v = FWHT(s . x) in the fp32
-// scratch (d floats), q = rint(127 v / amax), c_x = amax / (127 d).  Thread T
-// (< d/4) holds elements 4T..4T+3: stages h = 1, 2 run in registers, h = 4..64
-// across the lanes of a warp (a warp holds 128 consecutive elements), h >= 128
-// in shared memory.  Every stage applies the reference butterflies
-// (a + b, a - b), lower index first, in the reference stage order, so the
-// bits equal the reference transform's.
-__device__ void rotate_quantize_smem(const ExpertArgs& a, const Layout& L, char* smem, int t, float* v,
-                                     float* cx_out, float* red) {
+// scratch (d floats), q = rint(127 v / amax), c_x = amax / (127 d).  Stages
+// h = 1, 2 run in registers (thread c holds elements 4c .. 4c+3) and
+// h = 4 .. 64 across the lanes of a warp (a warp holds 128 consecutive
+// elements); from h = 128 on, each pass over shared memory applies two stages
+// (h and 2h) to four elements held in registers, and a last single stage
+// runs alone when the count is odd.  Every element sees the reference
+// butterflies (a + b, a - b) of every stage in the reference stage order, so
+// the bits equal the reference transform's.  d >= 256.  sv_pre holds the
+// signs of elements 4T .. 4T+3, loaded early by the caller.
+__device__ void rotate_quantize(const ExpertArgs& a, const Layout& L, char* smem, int t, float* v, float* cx_out,
+                                float* red, char4 sv_pre) {
   const int d = a.d;
-  const int T = threadIdx.x, lane = T & 31;
-  if (T < 2 * L.d8) {
-    const uint2 xv = reinterpret_cast<const uint2*>(smem + L.x + (size_t)t * d * 2)[T];
-    const char4 sv = reinterpret_cast<const char4*>(a.rot_sign)[T];
+  const int T = threadIdx.x, lane = T & 31, warp = T >> 5;
+  for (int c = T; c < 2 * L.d8; c += NTHR) {  // d / 4 is a multiple of 32: whole warps
+    const uint2 xv = reinterpret_cast<const uint2*>(smem + L.x + (size_t)t * d * 2)[c];
+    const char4 sv = c == T ? sv_pre : reinterpret_cast<const char4*>(a.rot_sign)[c];
     float r0 = (float)sv.x * bf16lo(xv.x), r1 = (float)sv.y * bf16hi(xv.x);
     float r2 = (float)sv.z * bf16lo(xv.y), r3 = (float)sv.w * bf16hi(xv.y);
     float b0 = __fadd_rn(r0, r1), b1 = __fsub_rn(r0, r1), b2 = __fadd_rn(r2, r3), b3 = __fsub_rn(r2, r3);  // h = 1
@@ -440,44 +489,67 @@ __device__ void rotate_quantize_smem(const ExpertArgs& a, const Layout& L, char*
     r1 = __fadd_rn(b1, b3);
     r3 = __fsub_rn(b1, b3);
 #pragma unroll 1
-    for (int m = 1; m < 32 && 4 * m < d; m <<= 1) {  // h = 4m: partner lane ^ m
+    for (int m = 1; m < 32; m <<= 1) {  // h = 4m: partner lane ^ m
       const bool up = lane & m;
-      const float p0 = __shfl_xor_sync(0xffffffffu, r0, m), p1 = __shfl_xor_sync(0xffffffffu, r1, m);
-      const float p2 = __shfl_xor_sync(0xffffffffu, r2, m), p3 = __shfl_xor_sync(0xffffffffu, r3, m);
+      const float p0 = __shfl_xor_sync(kFull, r0, m), p1 = __shfl_xor_sync(kFull, r1, m);
+      const float p2 = __shfl_xor_sync(kFull, r2, m), p3 = __shfl_xor_sync(kFull, r3, m);
       r0 = up ? __fsub_rn(p0, r0) : __fadd_rn(r0, p0);
       r1 = up ? __fsub_rn(p1, r1) : __fadd_rn(r1, p1);
       r2 = up ? __fsub_rn(p2, r2) : __fadd_rn(r2, p2);
       r3 = up ? __fsub_rn(p3, r3) : __fadd_rn(r3, p3);
     }
-    reinterpret_cast<float4*>(v)[T] = make_float4(r0, r1, r2, r3);
+    reinterpret_cast<float4*>(v)[c] = make_float4(r0, r1, r2, r3);
   }
-  __syncthreads();
+  float m = 0.0f;  // max |v| over this thread's outputs of the last pass
 #pragma unroll 1
-  for (int h = 128, lh = 7; h < d; h <<= 1, lh++) {
-    for (int p = threadIdx.x; p < 4 * L.d8; p += NTHR) {
-      const int j = ((p >> lh) << (lh + 1)) | (p & (h - 1));
-      const float x0 = v[j], x1 = v[j + h];
-      v[j] = __fadd_rn(x0, x1);
-      v[j + h] = __fsub_rn(x0, x1);
-    }
+  for (int h = 128, lh = 7; h < d;) {
     __syncthreads();
+    m = 0.0f;
+    if (2 * h < d) {
+      for (int p = T; p < 2 * L.d8; p += NTHR) {
+        const int b = ((p >> lh) << (lh + 2)) | (p & (h - 1));
+        const float a0 = v[b], a1 = v[b + h], a2 = v[b + 2 * h], a3 = v[b + 3 * h];
+        const float s0 = __fadd_rn(a0, a1), s1 = __fsub_rn(a0, a1);  // stage h
+        const float s2 = __fadd_rn(a2, a3), s3 = __fsub_rn(a2, a3);
+        const float o0 = __fadd_rn(s0, s2), o2 = __fsub_rn(s0, s2);  // stage 2h
+        const float o1 = __fadd_rn(s1, s3), o3 = __fsub_rn(s1, s3);
+        v[b] = o0;
+        v[b + h] = o1;
+        v[b + 2 * h] = o2;
+        v[b + 3 * h] = o3;
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(o0), fabsf(o1)), fmaxf(fabsf(o2), fabsf(o3))));
+      }
+      h <<= 2;
+      lh += 2;
+    } else {  // the last stage, h = d / 2
+      for (int p = T; p < 4 * L.d8; p += NTHR) {
+        const float x0 = v[p], x1 = v[p + h];
+        const float o0 = __fadd_rn(x0, x1), o1 = __fsub_rn(x0, x1);
+        v[p] = o0;
+        v[p + h] = o1;
+        m = fmaxf(m, fmaxf(fabsf(o0), fabsf(o1)));
+      }
+      h <<= 1;
+      lh += 1;
+    }
   }
-  float m = 0.0f;
-  for (int j = threadIdx.x; j < d; j += NTHR) m = fmaxf(m, fabsf(v[j]));
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) red[threadIdx.x >> 5] = m;
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+  if (lane == 0) red[warp] = m;
   __syncthreads();
   float amax = 0.0f;
-#pragma unroll 1
-  for (int w = 0; w < NWARP; w++) amax = fmaxf(amax, red[w]);
+#pragma unroll
+  for (int w = 0; w < NWARP; w += 4) {
+    const float4 r4 = reinterpret_cast<const float4*>(red)[w >> 2];
+    amax = fmaxf(amax, fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w)));
+  }
   int8_t* q = reinterpret_cast<int8_t*>(smem + L.q) + (size_t)t * d;
-  for (int j = threadIdx.x; j < d; j += NTHR) {
+  for (int j = T; j < d; j += NTHR) {
     int n = 0;
     if (amax > 0.0f) n = max(-127, min(127, __float2int_rn(__fdiv_rn(__fmul_rn(v[j], 127.0f), amax))));
     q[j] = (int8_t)n;
   }
-  if (threadIdx.x == 0) *cx_out = amax > 0.0f ? __fdiv_rn(amax, __fmul_rn(127.0f, (float)d)) : 0.0f;
+  if (T == 0) *cx_out = amax > 0.0f ? __fdiv_rn(amax, __fmul_rn(127.0f, (float)d)) : 0.0f;
   __syncthreads();
 }
 
@@ -486,76 +558,86 @@ __device__ __forceinline__ void stamp(const ExpertArgs& a, int cid, int rank, in
   if (a.dbg_phase && rank == 0 && threadIdx.x == 0) a.dbg_phase[cid * 16 + k] = global_ns();
 }
 
-// In-kernel routing (B <= NT <= 2): every CTA loads all tokens, rotates and
-// quantises them, computes the logits of its slice of experts and pushes
-// them to all CTAs; after the cluster barrier every CTA takes the same top-e
-// and builds the same work table (one item per routed expert, experts
-// ascending).  Returns false if this cluster has no item.
+// 8 consecutive 16-byte vectors per lane (j = j0 + 32u + lane), zero past d8.
+__device__ __forceinline__ void load_row8(const uint4* row, int j0, int d8, int lane, uint4 (&w)[8]) {
+#pragma unroll
+  for (int u = 0; u < 8; u++) {
+    const int j = j0 + 32 * u + lane;
+    w[u] = j < d8 ? __ldg(row + j) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// In-kernel routing (B <= NT <= 2): every CTA loads all tokens and computes
+// the logits of its slice of experts (one warp per expert; the router row is
+// read straight into registers, overlapping the token loads) and pushes them
+// to all CTAs; after the cluster barrier every CTA takes the same top-e and
+// one warp derives the softmax weights and this cluster's work item (one
+// item per routed expert, experts ascending).  Returns false if this cluster
+// has no item.
 template <int NT>
 __device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, int* misc, int cs, int rank,
-                            int cid, uint64_t* wrbar, cg::cluster_group& cluster) {
-  const int B = a.B, E = a.E, d = a.d, top = a.top_e;
+                            int cid, cg::cluster_group& cluster) {
+  const int B = a.B, E = a.E, top = a.top_e;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int e0 = L.ex0[rank], ne = L.ex0[rank + 1] - e0;
-  char* wr = smem + L.ring;  // router rows of this CTA's experts
-  if (threadIdx.x == 0 && ne > 0) {
-    mbar_expect_tx(wrbar, ne * d * 2);
-    bulk_g2s(wr, a.w_router + (size_t)e0 * d, ne * d * 2, wrbar);
+  uint4* xs = reinterpret_cast<uint4*>(smem + L.x);
+  uint4 w[8];
+  double bias_w = 0.0;
+  if (warp < ne) {
+    load_row8(reinterpret_cast<const uint4*>(a.w_router + (size_t)(e0 + warp) * a.d), 0, L.d8, lane, w);
+    if (a.bias) bias_w = (double)__ldg(a.bias + e0 + warp);
   }
-  if (threadIdx.x < B) {
-    misc[MI_TOK + threadIdx.x] = threadIdx.x;
-  }
-  __syncthreads();
-  load_tokens(a, L, smem, misc, B, false);
-  __syncthreads();
-  // rotate + quantise every token (the ring tail is the fp32 scratch)
-  float* scratch = reinterpret_cast<float*>(smem + L.ring + NWARP * L.ring_bytes - d * 4);
-  float* cxs = reinterpret_cast<float*>(misc + MI_CX);
-#pragma unroll 1
   for (int t = 0; t < B; t++)
-    rotate_quantize_smem(a, L, smem, t, scratch, &cxs[t], reinterpret_cast<float*>(misc + MI_SCAN));
-  stamp(a, cid, rank, 1);
-  // logits of the own experts, one warp per expert, pushed to every CTA
-  if (ne > 0 && !mbar_wait_bounded(wrbar, 0, a.ws.err)) misc[MI_DONE] = 1;
+    for (int j = threadIdx.x; j < L.d8; j += NTHR)
+      xs[t * L.d8 + j] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d) + j);
+  if (threadIdx.x < B) misc[MI_TOK + threadIdx.x] = threadIdx.x;
+  __syncthreads();
+  // logit_e = sum_j W_r[e, j] x_j (+ b_e): bf16 products are exact in fp32
+  // (8-bit significands; products below 2^-126 in magnitude excepted) and are
+  // summed in fp64
   double* lg = reinterpret_cast<double*>(smem + L.logit);
-  for (int el = warp; el < ne; el += NWARP) {
-    const uint4* wrow = reinterpret_cast<const uint4*>(wr + (size_t)el * d * 2);
-    double acc[NT];
-#pragma unroll
-    for (int t = 0; t < NT; t++) acc[t] = 0.0;
 #pragma unroll 1
-    for (int j = lane; j < L.d8; j += 32) {
-      const uint4 w = wrow[j];
+  for (int el = warp; el < ne; el += NWARP) {
+    const uint4* row = reinterpret_cast<const uint4*>(a.w_router + (size_t)(e0 + el) * a.d);
+    double acc0[NT], acc1[NT];
 #pragma unroll
-      for (int t = 0; t < NT; t++) {
-        const uint4 x = reinterpret_cast<const uint4*>(smem + L.x)[(t < B ? t : 0) * L.d8 + j];
-        acc[t] = fma((double)bf16lo(w.x), (double)bf16lo(x.x), acc[t]);
-        acc[t] = fma((double)bf16hi(w.x), (double)bf16hi(x.x), acc[t]);
-        acc[t] = fma((double)bf16lo(w.y), (double)bf16lo(x.y), acc[t]);
-        acc[t] = fma((double)bf16hi(w.y), (double)bf16hi(x.y), acc[t]);
-        acc[t] = fma((double)bf16lo(w.z), (double)bf16lo(x.z), acc[t]);
-        acc[t] = fma((double)bf16hi(w.z), (double)bf16hi(x.z), acc[t]);
-        acc[t] = fma((double)bf16lo(w.w), (double)bf16lo(x.w), acc[t]);
-        acc[t] = fma((double)bf16hi(w.w), (double)bf16hi(x.w), acc[t]);
+    for (int t = 0; t < NT; t++) acc0[t] = acc1[t] = 0.0;
+#pragma unroll 1
+    for (int j0 = 0; j0 < L.d8; j0 += 256) {
+      if (el != warp || j0 != 0) load_row8(row, j0, L.d8, lane, w);
+#pragma unroll
+      for (int u = 0; u < 8; u++) {
+        const int j = j0 + 32 * u + lane;
+        if (j < L.d8) {
+#pragma unroll
+          for (int t = 0; t < NT; t++) {
+            const uint4 xv = xs[(t < B ? t : 0) * L.d8 + j];
+            acc0[t] += (double)__fmul_rn(bf16lo(w[u].x), bf16lo(xv.x));
+            acc1[t] += (double)__fmul_rn(bf16hi(w[u].x), bf16hi(xv.x));
+            acc0[t] += (double)__fmul_rn(bf16lo(w[u].y), bf16lo(xv.y));
+            acc1[t] += (double)__fmul_rn(bf16hi(w[u].y), bf16hi(xv.y));
+            acc0[t] += (double)__fmul_rn(bf16lo(w[u].z), bf16lo(xv.z));
+            acc1[t] += (double)__fmul_rn(bf16hi(w[u].z), bf16hi(xv.z));
+            acc0[t] += (double)__fmul_rn(bf16lo(w[u].w), bf16lo(xv.w));
+            acc1[t] += (double)__fmul_rn(bf16hi(w[u].w), bf16hi(xv.w));
+          }
+        }
       }
     }
     const int e = e0 + el;
-    const double bias = a.bias ? (double)a.bias[e] : 0.0;
+    const double bias = el == warp ? bias_w : a.bias ? (double)a.bias[e] : 0.0;
 #pragma unroll
     for (int t = 0; t < NT; t++) {
-      const double s = warp_sum(acc[t]) + bias;
+      const double s = warp_sum(acc0[t] + acc1[t]) + bias;
       if (t < B && lane < cs) st_cluster(&lg[t * E + e], lane, s);
     }
   }
-  stamp(a, cid, rank, 2);
+  stamp(a, cid, rank, 1);
   cluster.sync();
-  stamp(a, cid, rank, 3);
+  stamp(a, cid, rank, 2);
   // top-e per token by rank: 4 threads per expert count the logits that beat
   // it (larger, or equal with a lower id); rank < top_e is chosen
   int* rids = misc + MI_RIDS;
-  float* rw = reinterpret_cast<float*>(misc + MI_RW);
-  double* ex = reinterpret_cast<double*>(smem + L.hist);  // [B, top] scratch
-  int* first = reinterpret_cast<int*>(ex + 64);
 #pragma unroll 1
   for (int b = 0; b < B; b++) {
     const double* lb = lg + b * E;
@@ -569,61 +651,77 @@ __device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, in
           cnt += (l2 > l) || (l2 == l && e2 < e);
         }
       }
-      cnt += __shfl_xor_sync(0xffffffffu, cnt, 1);
-      cnt += __shfl_xor_sync(0xffffffffu, cnt, 2);
+      cnt += __shfl_xor_sync(kFull, cnt, 1);
+      cnt += __shfl_xor_sync(kFull, cnt, 2);
       if (e < E && qtr == 0 && cnt < top) rids[b * top + cnt] = e;
     }
   }
   __syncthreads();
-  // softmax over the chosen logits, summed in slot order (fp32 exponentials
-  // of the fp64 logit differences; the weights only scale outputs)
-  const int nent = B * top;
-  if (threadIdx.x < nent) {
-    const int b = threadIdx.x >= top;  // B <= 2
-    ex[threadIdx.x] = (double)__expf((float)(lg[b * E + rids[threadIdx.x]] - lg[b * E + rids[b * top]]));
-    const int id = rids[threadIdx.x];
-    int f = 1;
-    for (int j = 0; j < threadIdx.x; j++) f &= rids[j] != id;
-    first[threadIdx.x] = f;
-  }
-  if (threadIdx.x == 0) misc[MI_E] = -1;
-  __syncthreads();
-  if (threadIdx.x < nent) {
-    const int b = threadIdx.x >= top;
-    double den = 0.0;
-    for (int s2 = 0; s2 < top; s2++) den += ex[b * top + s2];
-    const float w = (float)(ex[threadIdx.x] / den);
-    rw[threadIdx.x] = w;
-    if (cid == 0 && rank == 0) {
-      a.ws.ids[threadIdx.x] = rids[threadIdx.x];
-      a.ws.wts[threadIdx.x] = w;
-      if (a.dbg_ids) a.dbg_ids[threadIdx.x] = rids[threadIdx.x];
-      if (a.dbg_w) a.dbg_w[threadIdx.x] = w;
-    }
+  if (warp == 0) {
     // work table: distinct experts ascending; item cid = the cid-th of them
-    if (first[threadIdx.x]) {
-      const int id = rids[threadIdx.x];
-      int rk = 0;
-      for (int j = 0; j < nent; j++) rk += first[j] && rids[j] < id;
-      if (rk == cid) misc[MI_E] = id;
+    const int nent = B * top;  // <= 32
+    const bool act = lane < nent;
+    const int b = act && lane >= top ? 1 : 0;
+    const int id = act ? rids[lane] : 0x7fffffff;
+    bool first = act;
+    if (B > 1) {
+      const unsigned same = __match_any_sync(kFull, id);
+      first = act && __ffs(same) - 1 == lane;
     }
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    const int e = misc[MI_E];
-    const bool on = e >= 0 && lane < nent && rids[lane] == e;
-    const unsigned bal = __ballot_sync(0xffffffffu, on);
+    int* fid = misc + MI_FID;
+    fid[lane] = first ? id : 0x7fffffff;
+    __syncwarp();
+    int rk = 0;
+#pragma unroll 1
+    for (int j4 = 0; j4 < nent; j4 += 4) {
+      const int4 f = reinterpret_cast<const int4*>(fid)[j4 >> 2];
+      rk += (f.x < id) + (f.y < id) + (f.z < id) + (f.w < id);
+    }
+    const unsigned mine = __ballot_sync(kFull, first && rk == cid);
+    const int e_item = mine ? __shfl_sync(kFull, id, __ffs(mine) - 1) : -1;
+    const bool on = act && e_item >= 0 && id == e_item;
+    const unsigned bal = __ballot_sync(kFull, on);
     if (on) {
       const int at = __popc(bal & ((1u << lane) - 1u));
-      const int b = lane >= top;
       misc[MI_TOK + at] = b;
       misc[MI_SLOT + at] = lane - b * top;
       misc[MI_TIX + at] = b;
     }
-    if (lane == 0) misc[MI_N] = __popc(bal);
+    if (lane == 0) {
+      misc[MI_E] = e_item;
+      misc[MI_N] = __popc(bal);
+    }
   }
   __syncthreads();
   return misc[MI_E] >= 0;
+}
+
+// Routing weights of the in-kernel router (one warp, off the critical path):
+// softmax over the chosen logits, summed in slot order (fp32 exponentials of
+// the fp64 logit differences; the weights only scale outputs).
+__device__ void route_weights(const ExpertArgs& a, const Layout& L, char* smem, int* misc, int cid, int rank) {
+  const int lane = threadIdx.x & 31;
+  const int top = a.top_e, nent = a.B * top;
+  const double* lg = reinterpret_cast<const double*>(smem + L.logit);
+  const bool act = lane < nent;
+  const int b = act && lane >= top ? 1 : 0;
+  const int id = act ? misc[MI_RIDS + lane] : 0;
+  const double l = act ? lg[b * a.E + id] : 0.0;
+  const double l0 = __shfl_sync(kFull, l, b * top);
+  const double ex = act ? (double)__expf((float)(l - l0)) : 0.0;
+  double den = 0.0;
+#pragma unroll 1
+  for (int s2 = 0; s2 < top; s2++) den += __shfl_sync(kFull, ex, b * top + s2);
+  const float wt = act ? (float)(ex / den) : 0.0f;
+  if (act) {
+    reinterpret_cast<float*>(misc + MI_RW)[lane] = wt;
+    if (cid == 0 && rank == 0) {
+      a.ws.ids[lane] = id;
+      a.ws.wts[lane] = wt;
+      if (a.dbg_ids) a.dbg_ids[lane] = id;
+      if (a.dbg_w) a.dbg_w[lane] = wt;
+    }
+  }
 }
 
 // Epilogue shared by both kernels: write y_e for this CTA's columns, then the
@@ -642,30 +740,145 @@ __device__ void write_and_combine(const ExpertArgs& a, int rank, int j0, int nco
       if (a.dbg_y_expert) a.dbg_y_expert[((size_t)tok * a.top_e + sl) * a.d + j0 + col] = yfin[t * ldy + col];
     }
   }
-  __threadfence();
+  // the CTA's stores are ordered before one gpu-scope release by the
+  // counting thread (barrier, then fence + atomic)
   __syncthreads();
   if (threadIdx.x < n) {
     const int t = threadIdx.x;
-    const unsigned old = atomicAdd(&a.ws.counters[misc[MI_TOK + t] * kMaxCluster + rank], 1u);
+    unsigned old;
+    asm volatile("fence.acq_rel.gpu;\n\tatom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                 : "=r"(old)
+                 : "l"(&a.ws.counters[misc[MI_TOK + t] * kMaxCluster + rank])
+                 : "memory");
     misc[MI_LAST + t] = old == (unsigned)(a.top_e - 1);
   }
   __syncthreads();
 #pragma unroll 1
   for (int t = 0; t < n; t++) {
     if (!misc[MI_LAST + t]) continue;
-    __threadfence();
     const int tok = misc[MI_TOK + t];
     for (int col = threadIdx.x; col < ncols; col += NTHR) {
       const int j = j0 + col;
+      float v[16];
+#pragma unroll
+      for (int s = 0; s < 16; s++)
+        v[s] = s < a.top_e ? __ldcg(&a.ws.ye[((size_t)tok * a.top_e + s) * a.d + j]) : 0.0f;
       float acc = 0.0f;
-#pragma unroll 1
-      for (int s = 0; s < a.top_e; s++)
-        acc = fmaf(wts[tok * a.top_e + s], __ldcg(&a.ws.ye[((size_t)tok * a.top_e + s) * a.d + j]), acc);
+#pragma unroll
+      for (int s = 0; s < 16; s++)
+        if (s < a.top_e) acc = fmaf(wts[tok * a.top_e + s], v[s], acc);
       if (a.residual) acc += bf16f(a.residual[(size_t)tok * a.d + j]);
       a.y[(size_t)tok * a.d + j] = f2bf16(acc);
     }
     if (threadIdx.x == 0) a.ws.counters[tok * kMaxCluster + rank] = 0u;
   }
+}
+
+// Down rows: thread (g, q) takes 16-byte chunk q of rows g, g + rg, ... (rg
+// row groups); chunks q < ncq are 8 W_down columns of this CTA's slice, the
+// rest 8 entries of the Ubar row (recovery).  Rows are loaded 8 at a time
+// per thread, all in flight together.  coef(m, i, is_w, co[NT]) gives each
+// token's coefficient of row m (channel i).  Per-group partial sums land in
+// red[g][t][q * 8 + c]; returns rg.
+template <int NT, class Chan, class Coef>
+__device__ int down_rows(const ExpertArgs& a, int e, int j0, int ncq, int nr8, int nrows, int rr, Chan chan,
+                         Coef coef, float* red) {
+  const int nch = ncq + nr8;
+  const int g = idiv(threadIdx.x, nch);
+  const int q = threadIdx.x - g * nch;
+  const int rg = idiv(NTHR, nch);
+  float acc[NT][8];
+#pragma unroll
+  for (int t = 0; t < NT; t++)
+#pragma unroll
+    for (int c = 0; c < 8; c++) acc[t][c] = 0.0f;
+  if (g < rg) {
+    const bool is_w = q < ncq;
+    const uint16_t* base = is_w ? a.w_down + (size_t)e * a.I * a.d + j0 + 8 * q
+                                : a.u_sigma + (size_t)e * a.I * rr + 8 * (q - ncq);
+    const size_t stride = is_w ? (size_t)a.d : (size_t)rr;
+#pragma unroll 1
+    for (int m0 = g; m0 < nrows; m0 += 8 * rg) {
+      uint4 w[8];
+      float co[8][NT];
+#pragma unroll
+      for (int u = 0; u < 8; u++) {
+        const int m = m0 + u * rg;
+        w[u] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int t = 0; t < NT; t++) co[u][t] = 0.0f;
+        if (m < nrows) {
+          const int i = chan(m);
+          w[u] = __ldg(reinterpret_cast<const uint4*>(base + (size_t)i * stride));
+          coef(m, i, is_w, co[u]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; u++) {
+        const float f[8] = {bf16lo(w[u].x), bf16hi(w[u].x), bf16lo(w[u].y), bf16hi(w[u].y),
+                            bf16lo(w[u].z), bf16hi(w[u].z), bf16lo(w[u].w), bf16hi(w[u].w)};
+#pragma unroll
+        for (int t = 0; t < NT; t++)
+#pragma unroll
+          for (int c = 0; c < 8; c++) acc[t][c] = fmaf(co[u][t], f[c], acc[t][c]);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+      float4* dst = reinterpret_cast<float4*>(red + ((size_t)(g * NT + t) * nch + q) * 8);
+      dst[0] = make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
+      dst[1] = make_float4(acc[t][4], acc[t][5], acc[t][6], acc[t][7]);
+    }
+  }
+  __syncthreads();
+  return rg;
+}
+
+// Warp totals of the sketch dots of 4 channels, spread over the lanes: every
+// lane holds partial sums pg[c][t] (gate) and pu[c][t] (up) of channel c and
+// token t; a reduce-scatter leaves lane L (L < 16) with the totals (g, u) of
+// channel (L >> 2) & 3 and token (L >> 1) & 1 (token 0 when NT = 1).
+template <int NT>
+__device__ __forceinline__ void reduce_scatter4(const int (&pg)[4][NT], const int (&pu)[4][NT], int& g, int& u) {
+  const int lane = threadIdx.x & 31;
+  const bool lo = lane < 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+  int v1[4][NT];
+#pragma unroll
+  for (int c = 0; c < 4; c++)
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+      v1[c][t] = (lo ? pg[c][t] : pu[c][t]) + __shfl_xor_sync(kFull, lo ? pu[c][t] : pg[c][t], 16);
+  int v2[2][NT];
+#pragma unroll
+  for (int c = 0; c < 2; c++)
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+      v2[c][t] = (b3 ? v1[2 + c][t] : v1[c][t]) + __shfl_xor_sync(kFull, b3 ? v1[c][t] : v1[2 + c][t], 8);
+  int v3[NT];
+#pragma unroll
+  for (int t = 0; t < NT; t++) v3[t] = (b2 ? v2[1][t] : v2[0][t]) + __shfl_xor_sync(kFull, b2 ? v2[0][t] : v2[1][t], 4);
+  int v;
+  if (NT == 1) {
+    v = v3[0] + __shfl_xor_sync(kFull, v3[0], 2);
+  } else {
+    v = (b1 ? v3[NT - 1] : v3[0]) + __shfl_xor_sync(kFull, b1 ? v3[0] : v3[NT - 1], 2);
+  }
+  v += __shfl_xor_sync(kFull, v, 1);
+  const int o = __shfl_xor_sync(kFull, v, 16);
+  g = lo ? v : o;
+  u = lo ? o : v;
+}
+
+// Bulk copies of sketch chunk ch (rows i0 + 16 ch .. of both matrices) into
+// buffer slot `slot`, completing on bars[slot].
+__device__ __forceinline__ void issue_sketch(const ExpertArgs& a, const Layout& L, char* buf, uint64_t* bars, int e,
+                                             int i0, int i1, int ch, int slot) {
+  const int c0 = i0 + 16 * ch, cnt = min(16, i1 - c0);
+  const uint32_t bytes = cnt * (a.d / 4);
+  char* dst = buf + (size_t)slot * 2 * L.skc;
+  mbar_expect_tx(&bars[slot], 2 * bytes);
+  bulk_g2s(dst, a.sk_gate + ((size_t)e * a.I + c0) * (a.d / 16), bytes, &bars[slot]);
+  bulk_g2s(dst + L.skc, a.sk_up + ((size_t)e * a.I + c0) * (a.d / 16), bytes, &bars[slot]);
 }
 
 // ================================================================ sparse
@@ -679,146 +892,266 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.mbar);
   uint64_t* wbars = bars + warp * kMaxSlots;
-  uint64_t* uvbar = bars + NWARP * kMaxSlots;
-  uint64_t* wrbar = uvbar + 1;
+  uint64_t* skbars = bars + NWARP * kMaxSlots;
+  uint64_t* uvbar = skbars + kSkBars;
   int* misc = reinterpret_cast<int*>(smem + L.misc);
   int* hist = reinterpret_cast<int*>(smem + L.hist);
-  int* wtot = reinterpret_cast<int*>(smem + L.wtot);
-  if (tid < NWARP * kMaxSlots + 2) mbar_init(&bars[tid], 1);
+  if (tid < NWARP * kMaxSlots + kSkBars + 2) mbar_init(&bars[tid], 1);
   if (tid == 0) misc[MI_DONE] = 0;
   fence_mbar_init();
   __syncthreads();
   if (DBG) stamp(a, cid, rank, 0);
 
+  char4 sv_pre = make_char4(0, 0, 0, 0);  // rotation signs of elements 4 tid .. 4 tid + 3 (in-kernel routing)
   if (FUSED) {
-    if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, wrbar, cluster)) return;  // uniform per cluster
+    if (tid < a.d / 4) sv_pre = __ldg(reinterpret_cast<const char4*>(a.rot_sign) + tid);
+    if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, cluster)) return;  // uniform per cluster
   } else {
     pdl_wait();
     if (!load_item_table(a, cid, misc, NT)) return;
   }
-  if (DBG) stamp(a, cid, rank, 4);
+  if (DBG) stamp(a, cid, rank, 3);
   const int e = misc[MI_E], n = misc[MI_N];
   const int I = a.I, d = a.d, r = a.r;
-  const int i0 = L.ch0[rank], nown = L.ch0[rank + 1] - i0;
+  const int i0 = L.ch0[rank], i1 = L.ch0[rank + 1], nown = i1 - i0;
   const int j0 = L.col0[rank], ncols = L.col0[rank + 1] - j0;
   uint32_t* err = a.ws.err;
-  uint32_t par = 0;
-  char* ring = smem + L.ring + warp * L.ring_bytes;
-  int tix[NT];
-#pragma unroll
-  for (int t = 0; t < NT; t++) tix[t] = misc[MI_TIX + (t < n ? t : 0)];
+  char* skbuf = smem + L.ring;
+  const int nchunk = cdiv(nown, 16);
 
-  // factor rows of the own channels and V rows of the own columns
-  if (tid == 0 && r > 0) {
-    const uint32_t bu = nown * r * 2, bv = ncols * r * 2;
-    mbar_expect_tx(uvbar, bu + bv);
-    bulk_g2s(smem + L.ubar, a.u_sigma + ((size_t)e * I + i0) * r, bu, uvbar);
-    bulk_g2s(smem + L.vown, a.v + ((size_t)e * d + j0) * r, bv, uvbar);
+  // factor rows of the own channels, V rows of the own columns, and the
+  // first round of sketch chunks: all in flight before the token work
+  if (tid == 0) {
+    if (r > 0) {
+      const uint32_t bu = nown * r * 2, bv = ncols * r * 2;
+      mbar_expect_tx(uvbar, bu + bv);
+      bulk_g2s(smem + L.ubar, a.u_sigma + ((size_t)e * I + i0) * r, bu, uvbar);
+      bulk_g2s(smem + L.vown, a.v + ((size_t)e * d + j0) * r, bv, uvbar);
+    }
+    // the sketch scales of the own channels complete on chunk 0's barrier
+    // (every warp waits for chunk 0 before its first channel)
+    if (I % 4 == 0 && nown > 0) {
+      mbar_expect_tx_only(&skbars[0], 2 * nown * 4);  // chunk 0's copies arrive on it below
+      bulk_g2s(smem + L.alpha, a.alpha_gate + (size_t)e * I + i0, nown * 4, &skbars[0]);
+      bulk_g2s(smem + L.alpha + L.own_max * 4, a.alpha_up + (size_t)e * I + i0, nown * 4, &skbars[0]);
+    }
+    const int c1 = min(nchunk, L.sk_round);
+    for (int ch = 0; ch < c1; ch++) issue_sketch(a, L, skbuf, skbars, e, i0, i1, ch, ch);
   }
-  if (!FUSED) {
+  float* alg = reinterpret_cast<float*>(smem + L.alpha);
+  float* alu = alg + L.own_max;
+  if (I % 4 != 0) {  // unaligned scale slices: plain loads, made visible by the barrier below
+    for (int li = tid; li < nown; li += NTHR) {
+      alg[li] = __ldg(a.alpha_gate + (size_t)e * I + i0 + li);
+      alu[li] = __ldg(a.alpha_up + (size_t)e * I + i0 + li);
+    }
+  }
+  int tix[NT];
+  if (FUSED) {
+    // rotate + quantise every token while the sketch is in flight (the fp32
+    // scratch sits past the sketch buffers); its barriers also publish the
+    // scales loaded above
+    float* scratch = reinterpret_cast<float*>(smem + L.ring + NWARP * L.ring_bytes - d * 4);
+#pragma unroll 1
+    for (int t = 0; t < a.B; t++)
+      rotate_quantize(a, L, smem, t, scratch, reinterpret_cast<float*>(misc + MI_CX) + t,
+                      reinterpret_cast<float*>(misc + MI_RED), sv_pre);
+  } else {
     load_tokens(a, L, smem, misc, n, true);
     __syncthreads();
   }
+#pragma unroll
+  for (int t = 0; t < NT; t++) tix[t] = misc[MI_TIX + (t < n ? t : 0)];
+  if (DBG) stamp(a, cid, rank, 4);
 
-  float* sig = reinterpret_cast<float*>(smem + L.sig);        // [NT, I] pushed by the owners
-  float* ahat = reinterpret_cast<float*>(smem + L.ahat);      // [NT, I]
+  float* sa = reinterpret_cast<float*>(smem + L.sa);          // [I, NT] (sigma, ahat) pairs, slices from the owners
   float* zparts = reinterpret_cast<float*>(smem + L.zparts);  // [cs, NT, r]
   float* z = reinterpret_cast<float*>(smem + L.z);            // [NT, r]
+  float* cor = reinterpret_cast<float*>(smem + L.cor);        // [NT, r]
   float* apos = reinterpret_cast<float*>(smem + L.apos);      // [NT, I] by union position
   uint32_t* candm = reinterpret_cast<uint32_t*>(smem + L.candm);
-  uint32_t* keptm = reinterpret_cast<uint32_t*>(smem + L.keptm);
-  uint32_t* pmask = reinterpret_cast<uint32_t*>(smem + L.pmask);
+  uint32_t* keptm = reinterpret_cast<uint32_t*>(smem + L.keptm);  // over union positions
   int* ulist = reinterpret_cast<int*>(smem + L.ulist);
-  int* upos = reinterpret_cast<int*>(smem + L.upos);
   int* dlist = reinterpret_cast<int*>(smem + L.dlist);
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.keys);
-  int* kidx = reinterpret_cast<int*>(smem + L.kidx);
   const float* cxs = reinterpret_cast<const float*>(misc + MI_CX);
 
   // ---------------------------------------------------------- S: screen
   {
-    const int c0 = i0 + (warp * nown) / NWARP, c1 = i0 + ((warp + 1) * nown) / NWARP;
-    const int skrow = 4 * L.d16;  // bytes per sketch row
-    const int half = L.ring_bytes / 2;
-    const int per = L.s_per;
-    const int words = L.d16;
-    const uint4* qs = reinterpret_cast<const uint4*>(smem + L.q);
-    const float* ag_row = a.alpha_gate + (size_t)e * I;
-    const float* au_row = a.alpha_up + (size_t)e * I;
-    const int nchunk = c1 > c0 ? idiv(c1 - c0 + per - 1, per) : 0;
-    warp_stream(
-        nchunk, 2, wbars, par, err,
-        [&](int j, int s, uint64_t* bar) {
-          const int a0 = c0 + j * per, cnt = min(per, c1 - a0);
-          char* dst = ring + s * half;
-          mbar_expect_tx(bar, 2 * cnt * skrow);
-          bulk_g2s(dst, a.sk_gate + ((size_t)e * I + a0) * words, cnt * skrow, bar);
-          bulk_g2s(dst + cnt * skrow, a.sk_up + ((size_t)e * I + a0) * words, cnt * skrow, bar);
-        },
-        [&](int j, int s) {
-          const int a0 = c0 + j * per, cnt = min(per, c1 - a0);
-          const uint32_t* gw = reinterpret_cast<const uint32_t*>(ring + s * half);
-          const uint32_t* uw = gw + cnt * words;
-          // the scales of this chunk, one per lane, loaded ahead of the dots
-          const float agl = lane < cnt ? __ldg(ag_row + a0 + lane) : 0.0f;
-          const float aul = lane < cnt ? __ldg(au_row + a0 + lane) : 0.0f;
-#pragma unroll 1
-          for (int ci = 0; ci < cnt; ci++) {
-            const int i = a0 + ci;
-            int G[NT], U[NT];
+    const int nv = L.d64;  // 16-byte sketch vectors per row
+    int sq[NT];
 #pragma unroll
-            for (int t = 0; t < NT; t++) G[t] = U[t] = 0;
-#pragma unroll 1
-            for (int w = lane; w < words; w += 32) {
-              const uint4 tg = decode_trits(gw[ci * words + w]);
-              const uint4 tu = decode_trits(uw[ci * words + w]);
+    for (int t = 0; t < NT; t++) {
+      const uint4* qv = reinterpret_cast<const uint4*>(smem + L.q + (size_t)tix[t] * d);
+      int s = 0;
+      for (int j = lane; j < L.d8 / 2; j += 32) {
+        const uint4 q4 = qv[j];
+        s = __dp4a((int)q4.x, 0x01010101, s);
+        s = __dp4a((int)q4.y, 0x01010101, s);
+        s = __dp4a((int)q4.z, 0x01010101, s);
+        s = __dp4a((int)q4.w, 0x01010101, s);
+      }
+      sq[t] = warp_sum(s);  // sum of the token's activations: the code offset
+    }
+    const uint16_t* ub = reinterpret_cast<const uint16_t*>(smem + L.ubar);
+    float zacc[NT][4];
 #pragma unroll
-              for (int t = 0; t < NT; t++) {
-                const uint4 qv = qs[tix[t] * words + w];
-                G[t] = dot16_i8(tg, qv, G[t]);
-                U[t] = dot16_i8(tu, qv, U[t]);
-              }
-            }
-            const float ag = __shfl_sync(0xffffffffu, agl, ci), au = __shfl_sync(0xffffffffu, aul, ci);
+    for (int t = 0; t < NT; t++)
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) zacc[t][kk] = 0.0f;
+    bool uv_ready = r == 0;
+    // this lane's activations for sketch vector lane (the row's first 32
+    // vectors), kept in registers across the channels
+    uint4 qr[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+      const uint4* qv = reinterpret_cast<const uint4*>(smem + L.q + (size_t)tix[t] * d);
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) qr[t][kk] = lane < nv ? qv[4 * lane + kk] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // warp w takes channel 16 j + w of every sketch chunk j (one channel per
+    // warp and chunk); the dots of 4 chunks are reduced together
+    const int tt = NT == 2 ? (lane >> 1) & 1 : 0;  // token of lanes 0..15 after reduce_scatter4
+    const int cl = (lane >> 2) & 3;                 // channel (of the 4) of lanes 0..15
+    const bool writer = lane < 16 && (lane & (NT == 2 ? 1 : 3)) == 0;
+    const int sqt = NT == 2 && tt ? sq[NT - 1] : sq[0];
+    const float cxt = cxs[tix[NT == 2 && tt ? NT - 1 : 0]];
+    int rb = 0, par = 0;  // first chunk of the resident round, parity of its barriers
+#pragma unroll 1
+    for (int jb = 0; jb < nchunk; jb += 4) {
+      int pg[4][NT], pu[4][NT];
+#pragma unroll
+      for (int c = 0; c < 4; c++) {
+        const int j = jb + c, li = 16 * j + warp;
+#pragma unroll
+        for (int t = 0; t < NT; t++) pg[c][t] = pu[c][t] = 0;
+        if (j < nchunk && j == rb + L.sk_round) {
+          // the next round of chunks reuses the buffers: every warp is done with them
+          __syncthreads();
+          rb = j;
+          par ^= 1;
+          if (tid == 0) {
+            fence_proxy_async();
+            const int c1 = min(nchunk, j + L.sk_round);
+            for (int ch = j; ch < c1; ch++) issue_sketch(a, L, skbuf, skbars, e, i0, i1, ch, ch - j);
+          }
+        }
+        if (j < nchunk && li < nown) {
+          const int slot = j - rb;
+          if (!mbar_wait_bounded(&skbars[slot], par, err)) misc[MI_DONE] = 1;
+          const uint4* gw = reinterpret_cast<const uint4*>(skbuf + (size_t)slot * 2 * L.skc + warp * (d / 4));
+          const uint4* uw = reinterpret_cast<const uint4*>(skbuf + (size_t)slot * 2 * L.skc + L.skc + warp * (d / 4));
+          int ga[NT][4], ua[NT][4];
+#pragma unroll
+          for (int t = 0; t < NT; t++)
+#pragma unroll
+            for (int kk = 0; kk < 4; kk++) ga[t][kk] = ua[t][kk] = 0;
+#pragma unroll 1
+          for (int vv = lane; vv < nv; vv += 32) {
+            const uint4 g4 = gw[vv], u4 = uw[vv];
 #pragma unroll
             for (int t = 0; t < NT; t++) {
-              if (t < n) {
-                const int gs = warp_sum(G[t]), us = warp_sum(U[t]);
-                const float cx = cxs[tix[t]];
-                const float gh = __fmul_rn(__fmul_rn((float)gs, ag), cx);
-                const float uh = __fmul_rn(__fmul_rn((float)us, au), cx);
-                const float ah = __fmul_rn(silu_r(gh), uh);
-                if (lane < cs) {
-                  st_cluster(&sig[t * I + i], lane, fabsf(ah));
-                  st_cluster(&ahat[t * I + i], lane, ah);
-                }
-                if (DBG && lane == 31) {
-                  const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * I + i;
-                  if (a.dbg_G) a.dbg_G[off] = gs;
-                  if (a.dbg_U) a.dbg_U[off] = us;
-                  if (a.dbg_sigma) a.dbg_sigma[off] = fabsf(ah);
-                }
+              uint4 q0 = qr[t][0], q1 = qr[t][1], q2 = qr[t][2], q3 = qr[t][3];
+              if (vv != lane) {
+                const uint4* qv = reinterpret_cast<const uint4*>(smem + L.q + (size_t)tix[t] * d) + 4 * vv;
+                q0 = qv[0];
+                q1 = qv[1];
+                q2 = qv[2];
+                q3 = qv[3];
+              }
+              code_dot16(g4.x, q0, ga[t]);
+              code_dot16(g4.y, q1, ga[t]);
+              code_dot16(g4.z, q2, ga[t]);
+              code_dot16(g4.w, q3, ga[t]);
+              code_dot16(u4.x, q0, ua[t]);
+              code_dot16(u4.y, q1, ua[t]);
+              code_dot16(u4.z, q2, ua[t]);
+              code_dot16(u4.w, q3, ua[t]);
+            }
+          }
+#pragma unroll
+          for (int t = 0; t < NT; t++) {
+            pg[c][t] = code_dot_total(ga[t]);
+            pu[c][t] = code_dot_total(ua[t]);
+          }
+        }
+      }
+      int gs, us;
+      reduce_scatter4<NT>(pg, pu, gs, us);
+      gs -= sqt;
+      us -= sqt;
+      const int li = 16 * (jb + cl) + warp;
+      const bool valid = lane < 16 && jb + cl < nchunk && li < nown && tt < n;
+      const int i = i0 + li;
+      const float gh = __fmul_rn(__fmul_rn((float)gs, valid ? alg[li] : 0.0f), cxt);
+      const float uh = __fmul_rn(__fmul_rn((float)us, valid ? alu[li] : 0.0f), cxt);
+      const float ah = __fmul_rn(silu_r(gh), uh);
+      if (valid && writer) {
+        reinterpret_cast<float2*>(sa)[i * NT + tt] = make_float2(fabsf(ah), ah);
+        if (DBG) {
+          const size_t off = ((size_t)misc[MI_TOK + tt] * a.top_e + misc[MI_SLOT + tt]) * I + i;
+          if (a.dbg_G) a.dbg_G[off] = gs;
+          if (a.dbg_U) a.dbg_U[off] = us;
+          if (a.dbg_sigma) a.dbg_sigma[off] = fabsf(ah);
+        }
+      }
+      // partial recovery input z_w = sum over this warp's channels of ahat_i Ubar_i
+      if (r > 0) {
+        if (!uv_ready) {
+          if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
+          uv_ready = true;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; c++) {
+          const int lc = 16 * (jb + c) + warp;
+          if (jb + c < nchunk && lc < nown) {
+#pragma unroll
+            for (int t = 0; t < NT; t++) {
+              const float aht = __shfl_sync(kFull, ah, 4 * c + 2 * t);
+#pragma unroll
+              for (int kk = 0; kk < 4; kk++) {
+                const int p = lane + 32 * kk;
+                if (p < r && t < n) zacc[t][kk] = fmaf(aht, bf16f(ub[lc * r + p]), zacc[t][kk]);
               }
             }
           }
-        });
-    if (DBG) stamp(a, cid, rank, 5);
-    // partial recovery input over the own channels, pushed to every CTA:
-    // zparts[rank][t] = sum_{own i} ahat_i Ubar_i.  The local ahat of the own
-    // channels was written by this CTA's own stores above.
-    __syncthreads();
-    if (r > 0) {
-      if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
-      const uint16_t* ub = reinterpret_cast<const uint16_t*>(smem + L.ubar);
-#pragma unroll 1
-      for (int t = 0; t < n; t++)
-        for (int p = tid; p < r; p += NTHR) {
-          float zz = 0.0f;
-#pragma unroll 4
-          for (int li = 0; li < nown; li++) zz = fmaf(ahat[t * I + i0 + li], bf16f(ub[li * r + p]), zz);
-#pragma unroll 1
-          for (int o = 0; o < cs; o++) st_cluster(&zparts[(rank * NT + t) * r + p], o, zz);
         }
+      }
+    }
+    if (FUSED && warp == NWARP - 1) route_weights(a, L, smem, misc, cid, rank);
+    if (DBG) stamp(a, cid, rank, 5);
+    // z partials of the CTA, pushed to every CTA: zparts[rank][t]
+    if (r > 0) {
+      float* zr = reinterpret_cast<float*>(smem + L.zred);  // [NWARP, NT, r]
+#pragma unroll
+      for (int t = 0; t < NT; t++)
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++) {
+          const int p = lane + 32 * kk;
+          if (p < r) zr[(warp * NT + t) * r + p] = zacc[t][kk];
+        }
+      __syncthreads();
+      for (int tp = tid; tp < NT * r; tp += NTHR) {
+        float zz = 0.0f;
+#pragma unroll
+        for (int w = 0; w < NWARP; w++) zz += zr[w * NT * r + tp];
+        zparts[rank * NT * r + tp] = zz;
+      }
+    }
+    __syncthreads();
+    // push the own (sigma, ahat) slice and z partial to every other CTA: one
+    // 16-byte store per thread and peer, all in flight together
+    {
+      const int nsa4 = cdiv((i1 - i0) * NT * 2, 4), nz4 = r > 0 ? NT * r / 4 : 0, per = nsa4 + nz4;
+      const float4* sa4 = reinterpret_cast<const float4*>(sa + i0 * NT * 2);
+      const float4* z4 = reinterpret_cast<const float4*>(zparts + rank * NT * r);
+#pragma unroll 1
+      for (int w = tid; w < (cs - 1) * per; w += NTHR) {
+        const int pi = idiv(w, per), j = w - pi * per;
+        const int o = pi + (pi >= rank);
+        if (j < nsa4) st_cluster(&sa4[j], o, sa4[j]);
+        else st_cluster(&z4[j - nsa4], o, z4[j - nsa4]);
+      }
     }
   }
   if (DBG) stamp(a, cid, rank, 6);
@@ -828,26 +1161,10 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
   // ---------------------------------------------------------- c: top-c
 #pragma unroll 1
   for (int t = 0; t < n; t++)
-    block_select_top(reinterpret_cast<const uint32_t*>(sig + t * I), I, a.c, hist, wtot, misc,
-                     candm + t * L.words);
-  if (DBG) stamp(a, cid, rank, 8);
-#pragma unroll 1
-  for (int t = 0; t < n; t++)
-    for (int p = tid; p < r; p += NTHR) {
-      float zz = 0.0f;
-#pragma unroll 1
-      for (int o = 0; o < cs; o++) zz += zparts[(o * NT + t) * r + p];
-      z[t * r + p] = zz;
-    }
+    block_select_top(reinterpret_cast<const uint32_t*>(sa) + 2 * t, 2 * NT, I, a.c, hist, misc, candm + t * L.words);
   // union of the candidates, ascending
-  for (int w = tid; w < L.words; w += NTHR) {
-    uint32_t m = 0;
-#pragma unroll
-    for (int t = 0; t < NT; t++) m |= t < n ? candm[t * L.words + w] : 0u;
-    pmask[w] = m;
-  }
-  __syncthreads();
-  block_mask_to_list(pmask, I, ulist, upos, &misc[MI_NU]);
+  block_mask_to_list(candm, n > 1 ? candm + L.words : nullptr, I, ulist, &misc[MI_NU], hist);
+  const int nU = misc[MI_NU];
   if (DBG && a.dbg_cand && rank == 0 && warp < n) {
     const int t = warp;
     int base = 0;
@@ -855,13 +1172,12 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
     for (int w0 = 0; w0 < I; w0 += 32) {
       const int p = w0 + lane;
       const bool on = p < I && ((candm[t * L.words + (w0 >> 5)] >> lane) & 1u);
-      const unsigned bal = __ballot_sync(0xffffffffu, on);
+      const unsigned bal = __ballot_sync(kFull, on);
       if (on) out[base + __popc(bal & ((1u << lane) - 1u))] = p;
       base += __popc(bal);
     }
   }
-  const int nU = misc[MI_NU];
-  if (DBG) stamp(a, cid, rank, 9);
+  if (DBG) stamp(a, cid, rank, 8);
 
   // -------------------------------------------- C: exact candidate stage
   {
@@ -871,6 +1187,8 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
     const int P = max(1, min(kMaxSlots, L.c_slots));
     const uint4* xs = reinterpret_cast<const uint4*>(smem + L.x);
     const int vx = L.d8;
+    char* ring = smem + L.ring + warp * L.ring_bytes;
+    uint32_t par = 0;
     warp_stream(
         m1 - m0, P, wbars, par, err,
         [&](int j, int s, uint64_t* bar) {
@@ -903,205 +1221,134 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
               const float gs = warp_sum(g0[t] + g1[t]), us = warp_sum(v0[t] + v1[t]);
               const bool is_c = (candm[t * L.words + (i >> 5)] >> (i & 31)) & 1u;
               const float av = is_c ? __fmul_rn(silu_r(gs), us) : 0.0f;
-              if (lane < cs) st_cluster(&apos[t * I + u], lane, av);
+              if (lane == 0) apos[t * I + u] = av;
             }
           }
         });
+    // push the own a values to every other CTA, one store per thread and peer
+    __syncthreads();
+    const int per = n * nsl;
+#pragma unroll 1
+    for (int w = tid; w < (cs - 1) * per; w += NTHR) {
+      const int pi = idiv(w, per), j = w - pi * per;
+      const int o = pi + (pi >= rank);
+      const int t = j >= nsl ? 1 : 0, u = u0 + j - t * nsl;
+      st_cluster(&apos[t * I + u], o, apos[t * I + u]);
+    }
   }
-  if (DBG) stamp(a, cid, rank, 10);
+  if (DBG) stamp(a, cid, rank, 9);
   cluster.sync();  // the last exchange: no CTA touches another's smem after this
-  if (DBG) stamp(a, cid, rank, 11);
+  if (DBG) stamp(a, cid, rank, 10);
 
   // ------------------------------------------------------------ k: top-k
+  // over union positions; a token's non-candidates get key 0, its candidates
+  // |a| + 1 (same order, ties still to the lower channel)
 #pragma unroll 1
   for (int t = 0; t < n; t++) {
-    // the token's candidates in ascending channel order, key |a|
-    if (warp == 0) {
-      int base = 0;
-      for (int w0 = 0; w0 < nU; w0 += 32) {
-        const int u = w0 + lane;
-        bool on = false;
-        int i = 0;
-        if (u < nU) {
-          i = ulist[u];
-          on = (candm[t * L.words + (i >> 5)] >> (i & 31)) & 1u;
-        }
-        const unsigned bal = __ballot_sync(0xffffffffu, on);
-        if (on) {
-          const int at = base + __popc(bal & ((1u << lane) - 1u));
-          keys[at] = __float_as_uint(fabsf(apos[t * I + u]));
-          kidx[at] = i;
-        }
-        base += __popc(bal);
-      }
-      if (lane == 0) misc[MI_NC] = base;  // = c
+    for (int u = tid; u < nU; u += NTHR) {
+      const int i = ulist[u];
+      const bool c = (candm[t * L.words + (i >> 5)] >> (i & 31)) & 1u;
+      keys[u] = c ? __float_as_uint(fabsf(apos[t * I + u])) + 1u : 0u;
     }
     __syncthreads();
-    const int c = misc[MI_NC];
-    uint32_t* km = keptm + t * L.words;
-    block_select_top(keys, c, a.k, hist, wtot, misc, pmask);  // over compact positions
-    for (int w = tid; w < L.words; w += NTHR) km[w] = 0u;
-    __syncthreads();
-    for (int p = tid; p < c; p += NTHR)
-      if ((pmask[p >> 5] >> (p & 31)) & 1u) atomicOr(&km[kidx[p] >> 5], 1u << (kidx[p] & 31));
-    __syncthreads();
+    block_select_top(keys, 1, nU, a.k, hist, misc, keptm + t * L.words);
     if (DBG && a.dbg_kept && rank == 0 && warp == 0) {
       const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.k;
       int base = 0;
-      for (int w0 = 0; w0 < I; w0 += 32) {
-        const int i = w0 + lane;
-        const bool on = i < I && ((km[w0 >> 5] >> lane) & 1u);
-        const unsigned bal = __ballot_sync(0xffffffffu, on);
+      for (int w0 = 0; w0 < nU; w0 += 32) {
+        const int u = w0 + lane;
+        const bool on = u < nU && ((keptm[t * L.words + (w0 >> 5)] >> lane) & 1u);
+        const unsigned bal = __ballot_sync(kFull, on);
         const int at = base + __popc(bal & ((1u << lane) - 1u));
         if (on && at < a.k) {
-          a.dbg_kept[off + at] = i;
-          if (a.dbg_a_kept) a.dbg_a_kept[off + at] = apos[t * I + upos[i]];
+          a.dbg_kept[off + at] = ulist[u];
+          if (a.dbg_a_kept) a.dbg_a_kept[off + at] = apos[t * I + u];
         }
         base += __popc(bal);
       }
     }
   }
-  if (DBG) stamp(a, cid, rank, 12);
-  // union of the kept channels
-  for (int w = tid; w < L.words; w += NTHR) {
-    uint32_t m = 0;
-#pragma unroll
-    for (int t = 0; t < NT; t++) m |= t < n ? keptm[t * L.words + w] : 0u;
-    pmask[w] = m;
-  }
-  __syncthreads();
-  block_mask_to_list(pmask, I, dlist, nullptr, &misc[MI_ND]);
+  // rows of the down stage: union positions kept by any token
+  block_mask_to_list(keptm, n > 1 ? keptm + L.words : nullptr, nU, dlist, &misc[MI_ND], hist);
   const int nD = misc[MI_ND];
-  if (DBG) stamp(a, cid, rank, 13);
+  if (DBG) stamp(a, cid, rank, 11);
 
   // ---------------------------------------------- D: down rows + recovery
-  {
-    const int colb = ncols * 2, ubb = r * 2;
-    const int eb = rup(colb + ubb, 16);
-    const int m0 = (warp * nD) / NWARP, m1 = ((warp + 1) * nD) / NWARP, cnt = m1 - m0;
-    const int cap = max(1, idiv(L.ring_bytes, eb));
-    int P = min(kMaxSlots, max(1, cnt));
-    int per = max(1, min(idiv(cnt + P - 1, P), idiv(cap, P)));
-    if (per * P > cap) P = max(1, idiv(cap, per));
-    float acc[NT][8];
-    float cor[NT][4];
+  float* red = reinterpret_cast<float*>(smem + L.ring);
+  const int ncq = ncols >> 3, nr8 = r >> 3, nch = ncq + nr8;
+  const int rg = down_rows<NT>(
+      a, e, j0, ncq, nr8, nD, r, [&](int m) { return ulist[dlist[m]]; },
+      [&](int m, int i, bool is_w, float (&co)[NT]) {
+        const int u = dlist[m];
 #pragma unroll
-    for (int t = 0; t < NT; t++) {
-#pragma unroll
-      for (int q = 0; q < 8; q++) acc[t][q] = 0.0f;
-#pragma unroll
-      for (int q = 0; q < 4; q++) cor[t][q] = 0.0f;
-    }
-    warp_stream(
-        cnt > 0 ? idiv(cnt + per - 1, per) : 0, P, wbars, par, err,
-        [&](int j, int s, uint64_t* bar) {
-          const int g0 = m0 + j * per, gc = min(per, m1 - g0);
-          char* dst = ring + s * per * eb;
-          mbar_expect_tx(bar, gc * (colb + ubb));
-#pragma unroll 1
-          for (int q = 0; q < gc; q++) {
-            const int i = dlist[g0 + q];
-            bulk_g2s(dst + q * eb, a.w_down + ((size_t)e * I + i) * d + j0, colb, bar);
-            if (r > 0) bulk_g2s(dst + q * eb + colb, a.u_sigma + ((size_t)e * I + i) * r, ubb, bar);
-          }
-        },
-        [&](int j, int s) {
-          const int g0 = m0 + j * per, gc = min(per, m1 - g0);
-          const char* src = ring + s * per * eb;
-#pragma unroll 1
-          for (int q = 0; q < gc; q++) {
-            const int i = dlist[g0 + q];
-            float co[NT], ch[NT];
-#pragma unroll
-            for (int t = 0; t < NT; t++) {
-              const bool kept = t < n && ((keptm[t * L.words + (i >> 5)] >> (i & 31)) & 1u);
-              co[t] = kept ? apos[t * I + upos[i]] : 0.0f;
-              ch[t] = kept ? ahat[t * I + i] : 0.0f;
-            }
-            const uint16_t* wd = reinterpret_cast<const uint16_t*>(src + q * eb);
-#pragma unroll
-            for (int cg4 = 0; cg4 < 2; cg4++) {
-              const int c4 = 4 * lane + 128 * cg4;
-              if (c4 < ncols) {
-                const uint2 wv = *reinterpret_cast<const uint2*>(wd + c4);
-                const float w0 = bf16lo(wv.x), w1 = bf16hi(wv.x), w2 = bf16lo(wv.y), w3 = bf16hi(wv.y);
-#pragma unroll
-                for (int t = 0; t < NT; t++) {
-                  acc[t][4 * cg4 + 0] = fmaf(co[t], w0, acc[t][4 * cg4 + 0]);
-                  acc[t][4 * cg4 + 1] = fmaf(co[t], w1, acc[t][4 * cg4 + 1]);
-                  acc[t][4 * cg4 + 2] = fmaf(co[t], w2, acc[t][4 * cg4 + 2]);
-                  acc[t][4 * cg4 + 3] = fmaf(co[t], w3, acc[t][4 * cg4 + 3]);
-                }
-              }
-            }
-            if (r > 0) {
-              const uint16_t* ur = reinterpret_cast<const uint16_t*>(src + q * eb + colb);
-#pragma unroll
-              for (int kk = 0; kk < 4; kk++) {
-                const int p = lane + 32 * kk;
-                if (p < r) {
-                  const float uv = bf16f(ur[p]);
-#pragma unroll
-                  for (int t = 0; t < NT; t++) cor[t][kk] = fmaf(ch[t], uv, cor[t][kk]);
-                }
-              }
-            }
-          }
-        });
-    __syncwarp();
-    float* part = reinterpret_cast<float*>(ring);  // [NT, cols_max] then [NT, r]
-    float* cpart = part + NT * L.cols_max;
-#pragma unroll
-    for (int t = 0; t < NT; t++) {
-#pragma unroll
-      for (int cg4 = 0; cg4 < 2; cg4++) {
-        const int c4 = 4 * lane + 128 * cg4;
-        if (c4 < ncols) {
-#pragma unroll
-          for (int q = 0; q < 4; q++) part[t * L.cols_max + c4 + q] = acc[t][4 * cg4 + q];
+        for (int t = 0; t < NT; t++) {
+          const bool kept = t < n && ((keptm[t * L.words + (u >> 5)] >> (u & 31)) & 1u);
+          co[t] = kept ? (is_w ? apos[t * I + u] : sa[(i * NT + t) * 2 + 1]) : 0.0f;
         }
-      }
-#pragma unroll
-      for (int kk = 0; kk < 4; kk++) {
-        const int p = lane + 32 * kk;
-        if (p < r) cpart[t * r + p] = cor[t][kk];
-      }
-    }
-  }
-  __syncthreads();
+      },
+      red);
   float* yfin = reinterpret_cast<float*>(smem + L.x);  // [n, cols_max]; x is no longer needed
 #pragma unroll 1
-  for (int t = 0; t < n; t++)
-    for (int p = tid; p < r; p += NTHR) {
-      float cc = 0.0f;
+  for (int o = tid; o < n * nch * 8; o += NTHR) {
+    const int t = o >= nch * 8 ? 1 : 0;
+    const int oc = o - t * nch * 8;
+    const float* rp = red + (size_t)t * nch * 8 + oc;
+    const int gstride = NT * nch * 8;
+    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+    int gg = 0;
 #pragma unroll 1
-      for (int w = 0; w < NWARP; w++)
-        cc += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[NT * L.cols_max + t * r + p];
-      z[t * r + p] -= cc;
+    for (; gg + 4 <= rg; gg += 4) {
+      s0 += rp[(gg + 0) * gstride];
+      s1 += rp[(gg + 1) * gstride];
+      s2 += rp[(gg + 2) * gstride];
+      s3 += rp[(gg + 3) * gstride];
     }
+    for (; gg < rg; gg++) s0 += rp[gg * gstride];
+    const float s = (s0 + s1) + (s2 + s3);
+    if (oc < ncols) yfin[t * L.cols_max + oc] = s;
+    else cor[t * r + (oc - ncols)] = s;
+  }
   __syncthreads();
-  {
+  if (r > 0) {
+#pragma unroll 1
+    for (int t = 0; t < n; t++)
+      for (int p = tid; p < r; p += NTHR) {
+        float zz = 0.0f;
+#pragma unroll 1
+        for (int o = 0; o < cs; o++) zz += zparts[(o * NT + t) * r + p];
+        z[t * r + p] = zz - cor[t * r + p];
+      }
+    if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
+    __syncthreads();
     const uint16_t* vo = reinterpret_cast<const uint16_t*>(smem + L.vown);
 #pragma unroll 1
     for (int t = 0; t < n; t++)
       for (int col = tid; col < ncols; col += NTHR) {
-        float y = 0.0f;
-#pragma unroll 1
-        for (int w = 0; w < NWARP; w++)
-          y += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[t * L.cols_max + col];
-        float rec = 0.0f;
+        float rec0 = 0.0f, rec1 = 0.0f;
 #pragma unroll 4
-        for (int p = 0; p < r; p++) rec = fmaf(bf16f(vo[col * r + p]), z[t * r + p], rec);
-        yfin[t * L.cols_max + col] = y + rec;
+        for (int p = 0; p < r; p += 8) {
+          const uint4 v8 = *reinterpret_cast<const uint4*>(vo + col * r + p);
+          const float4 za = *reinterpret_cast<const float4*>(z + t * r + p);
+          const float4 zb = *reinterpret_cast<const float4*>(z + t * r + p + 4);
+          rec0 = fmaf(bf16lo(v8.x), za.x, rec0);
+          rec1 = fmaf(bf16hi(v8.x), za.y, rec1);
+          rec0 = fmaf(bf16lo(v8.y), za.z, rec0);
+          rec1 = fmaf(bf16hi(v8.y), za.w, rec1);
+          rec0 = fmaf(bf16lo(v8.z), zb.x, rec0);
+          rec1 = fmaf(bf16hi(v8.z), zb.y, rec1);
+          rec0 = fmaf(bf16lo(v8.w), zb.z, rec0);
+          rec1 = fmaf(bf16hi(v8.w), zb.w, rec1);
+        }
+        yfin[t * L.cols_max + col] += rec0 + rec1;
       }
+    __syncthreads();
   }
-  __syncthreads();
-  if (DBG) stamp(a, cid, rank, 14);
+  if (DBG) stamp(a, cid, rank, 12);
   write_and_combine(a, rank, j0, ncols, L.cols_max, yfin, misc,
                     FUSED ? reinterpret_cast<const float*>(misc + MI_RW) : a.ws.wts);
   if (DBG) {
     __syncthreads();
-    stamp(a, cid, rank, 15);
+    stamp(a, cid, rank, 13);
   }
 }
 
@@ -1116,14 +1363,14 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.mbar);
   uint64_t* wbars = bars + warp * kMaxSlots;
-  uint64_t* wrbar = bars + NWARP * kMaxSlots + 1;
   int* misc = reinterpret_cast<int*>(smem + L.misc);
-  if (tid < NWARP * kMaxSlots + 2) mbar_init(&bars[tid], 1);
+  if (tid < NWARP * kMaxSlots + kSkBars + 2) mbar_init(&bars[tid], 1);
   if (tid == 0) misc[MI_DONE] = 0;
   fence_mbar_init();
   __syncthreads();
   if (FUSED) {
-    if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, wrbar, cluster)) return;
+    if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, cluster)) return;
+    if (warp == NWARP - 1) route_weights(a, L, smem, misc, cid, rank);
   } else {
     pdl_wait();
     if (!load_item_table(a, cid, misc, NT)) return;
@@ -1182,81 +1429,34 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
         });
   }
   cluster.sync();  // the only exchange: no CTA touches another's smem after this
-  {
-    const int colb = ncols * 2;
-    const int eb = rup(colb, 16);
-    const int m0 = (warp * I) / NWARP, m1 = ((warp + 1) * I) / NWARP, cnt = m1 - m0;
-    const int cap = max(1, idiv(L.ring_bytes, eb));
-    int P = min(kMaxSlots, max(1, cnt));
-    int per = max(1, min(idiv(cnt + P - 1, P), idiv(cap, P)));
-    if (per * P > cap) P = max(1, idiv(cap, per));
-    float acc[NT][8];
+  float* red = reinterpret_cast<float*>(smem + L.ring);
+  const int ncq = ncols >> 3;
+  const int rg = down_rows<NT>(
+      a, e, j0, ncq, 0, I, 0, [](int m) { return m; },
+      [&](int m, int, bool, float (&co)[NT]) {
 #pragma unroll
-    for (int t = 0; t < NT; t++)
-#pragma unroll
-      for (int q = 0; q < 8; q++) acc[t][q] = 0.0f;
-    warp_stream(
-        cnt > 0 ? idiv(cnt + per - 1, per) : 0, P, wbars, par, err,
-        [&](int j, int s, uint64_t* bar) {
-          const int g0 = m0 + j * per, gc = min(per, m1 - g0);
-          char* dst = ring + s * per * eb;
-          mbar_expect_tx(bar, gc * colb);
-#pragma unroll 1
-          for (int q = 0; q < gc; q++)
-            bulk_g2s(dst + q * eb, a.w_down + ((size_t)e * I + g0 + q) * d + j0, colb, bar);
-        },
-        [&](int j, int s) {
-          const int g0 = m0 + j * per, gc = min(per, m1 - g0);
-          const char* src = ring + s * per * eb;
-#pragma unroll 1
-          for (int q = 0; q < gc; q++) {
-            const int i = g0 + q;
-            float co[NT];
-#pragma unroll
-            for (int t = 0; t < NT; t++) co[t] = t < n ? h[t * I + i] : 0.0f;
-            const uint16_t* wd = reinterpret_cast<const uint16_t*>(src + q * eb);
-#pragma unroll
-            for (int cg4 = 0; cg4 < 2; cg4++) {
-              const int c4 = 4 * lane + 128 * cg4;
-              if (c4 < ncols) {
-                const uint2 wv = *reinterpret_cast<const uint2*>(wd + c4);
-                const float w0 = bf16lo(wv.x), w1 = bf16hi(wv.x), w2 = bf16lo(wv.y), w3 = bf16hi(wv.y);
-#pragma unroll
-                for (int t = 0; t < NT; t++) {
-                  acc[t][4 * cg4 + 0] = fmaf(co[t], w0, acc[t][4 * cg4 + 0]);
-                  acc[t][4 * cg4 + 1] = fmaf(co[t], w1, acc[t][4 * cg4 + 1]);
-                  acc[t][4 * cg4 + 2] = fmaf(co[t], w2, acc[t][4 * cg4 + 2]);
-                  acc[t][4 * cg4 + 3] = fmaf(co[t], w3, acc[t][4 * cg4 + 3]);
-                }
-              }
-            }
-          }
-        });
-    __syncwarp();
-    float* part = reinterpret_cast<float*>(ring);
-#pragma unroll
-    for (int t = 0; t < NT; t++) {
-#pragma unroll
-      for (int cg4 = 0; cg4 < 2; cg4++) {
-        const int c4 = 4 * lane + 128 * cg4;
-        if (c4 < ncols) {
-#pragma unroll
-          for (int q = 0; q < 4; q++) part[t * L.cols_max + c4 + q] = acc[t][4 * cg4 + q];
-        }
-      }
-    }
-  }
-  __syncthreads();
+        for (int t = 0; t < NT; t++) co[t] = t < n ? h[t * I + m] : 0.0f;
+      },
+      red);
   float* out = reinterpret_cast<float*>(smem + L.x);
 #pragma unroll 1
-  for (int t = 0; t < n; t++)
-    for (int col = tid; col < ncols; col += NTHR) {
-      float y = 0.0f;
+  for (int o = tid; o < n * ncq * 8; o += NTHR) {
+    const int t = o >= ncq * 8 ? 1 : 0;
+    const int oc = o - t * ncq * 8;
+    const float* rp = red + (size_t)t * ncq * 8 + oc;
+    const int gstride = NT * ncq * 8;
+    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+    int gg = 0;
 #pragma unroll 1
-      for (int w = 0; w < NWARP; w++)
-        y += reinterpret_cast<const float*>(smem + L.ring + w * L.ring_bytes)[t * L.cols_max + col];
-      out[t * L.cols_max + col] = y;
+    for (; gg + 4 <= rg; gg += 4) {
+      s0 += rp[(gg + 0) * gstride];
+      s1 += rp[(gg + 1) * gstride];
+      s2 += rp[(gg + 2) * gstride];
+      s3 += rp[(gg + 3) * gstride];
     }
+    for (; gg < rg; gg++) s0 += rp[gg * gstride];
+    out[t * L.cols_max + oc] = (s0 + s1) + (s2 + s3);
+  }
   __syncthreads();
   write_and_combine(a, rank, j0, ncols, L.cols_max, out, misc,
                     FUSED ? reinterpret_cast<const float*>(misc + MI_RW) : a.ws.wts);
@@ -1287,8 +1487,8 @@ const void* pick_kernel(bool dense, int NT, bool fused, bool dbg) {
 // least estimated time, waves * (1 + 8 / cs) with waves = ceil(items /
 // co-resident clusters): a wave costs a fixed latency plus work that shrinks
 // with the cluster's width.  Ring: the deepest that fits, with room for the
-// per-warp partial sums [NT, cols + r] fp32 of the down stage (and, with the
-// in-kernel router, for the CTA's router rows and an fp32 transform scratch).
+// down stage's partial sums (NT x 16 KB), the rotation scratch and at least
+// one sketch chunk.
 cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
   thread_local LaunchPlan cache[16];
   thread_local int ncache = 0, next = 0;
@@ -1321,13 +1521,13 @@ cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
     if (g_forced_cs && cs != g_forced_cs) continue;
     const int cols_max = 8 * cdiv(a.d / 8, cs);
     if (cols_max > kMaxCols || a.I < cs || (fused && a.E < cs)) continue;
-    const int need = NT * (cols_max + a.r) * 4;
-    const int wr_need = fused ? cdiv(a.E, cs) * a.d * 2 + a.d * 4 : 0;
+    const int red_need = NT * NTHR * 8 * 4;
     int rr = 0;
     for (int t = 2; t <= 64; t++) {
       const Layout L = make_layout(NT, ntok, fused, a.E, a.I, a.d, a.r, cs, t, dense);
       if (L.total > smem_max) break;
-      if (L.ring_bytes >= need && NWARP * L.ring_bytes >= wr_need) rr = t;
+      const int region = NWARP * L.ring_bytes;
+      if (L.c_slots >= 1 && region >= red_need && (dense || L.sk_round >= 1)) rr = t;
     }
     if (rr < 2) continue;
     const Layout L = make_layout(NT, ntok, fused, a.E, a.I, a.d, a.r, cs, rr, dense);

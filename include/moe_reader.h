@@ -33,7 +33,7 @@
  *    word in the workspace (read with moe_reader_check_error) instead of
  *    hanging the GPU.
  *
- * Limits of this build: 128 <= d <= 4096 and d a power of two;
+ * Limits of this build: 256 <= d <= 4096 and d a power of two;
  * 16 <= I <= 2048; 1 <= k <= c <= I; r in {0, 8, 16, ..., 128} and r <= I;
  * 1 <= top_e <= min(E, 16); E <= 1024; 1 <= B <= 256.
  */
@@ -116,9 +116,9 @@ size_t moe_reader_workspace_bytes(int B, int E, int top_e, int I, int d, int k, 
  *   Delta = 0.7 * mean |w'| (fp64, index order); T_j = sign(w'_j) if
  *   |w'_j| > Delta else 0; alpha = mean |w'_j| over T_j != 0 (fp64, index
  *   order; 0 if none), stored fp32 (TWN, Li & Liu 2016).
- * Packing: 16 trits per uint32; word m holds positions 16m..16m+15;
- * position 16m+n (n < 8) at bits [4n, 4n+1], position 16m+8+n at bits
- * [4n+2, 4n+3]; codes 00 = 0, 01 = +1, 11 = -1.
+ * Packing: 16 trits per uint32; word m of a row holds positions
+ * 16m..16m+15; position 16m + 4p + b (p, b in 0..3) sits at bits
+ * [8b + 2p, 8b + 2p + 1] as the code T + 1 (00 = -1, 01 = 0, 10 = +1).
  * Outputs are bit-identical to the reference definition above. */
 moe_status moe_reader_build_sketch(int E, int I, int d, const uint16_t* w_gate, const uint16_t* w_up,
                                    uint64_t rot_seed, int8_t* rot_sign, uint32_t* sk_gate,

@@ -189,24 +189,27 @@ void orc_twn_row(int d, const uint16_t* w, const int8_t* s, int8_t* trit,
     *alpha = nnz ? (float)(snz / (double)nnz) : 0.0f;
 }
 
-/* 2-bit packing, 16 trits per uint32 word; word k holds positions
- * 16k .. 16k+15.  Position 16k+n (n < 8) sits at bits [4n, 4n+1] and
- * position 16k+8+n at bits [4n+2, 4n+3].  Codes: 00 = 0, 01 = +1, 11 = -1
- * (10 is never written).  Reading: the pages fix no layout; this one lets a
- * decoder turn each nibble into a byte selector. */
-static int trit_shift(int p /* 0..15 */) { return p < 8 ? 4 * p : 4 * (p - 8) + 2; }
+/* 2-bit packing, 16 trits per uint32 word; word m of a row holds positions
+ * 16m .. 16m+15.  Position 16m + 4p + b (p, b in 0..3) sits at bits
+ * [8b + 2p, 8b + 2p + 1] as the unsigned code T + 1 (00 = -1, 01 = 0,
+ * 10 = +1; 11 is never written).  Reading: the pages fix no layout.  In this
+ * one, masking a word with 0x03030303 << 2p leaves four byte lanes that a
+ * byte-wise dot product multiplies with the int8 activations of positions
+ * 16m + 4p .. 16m + 4p + 3; the code offset is removed once per row by
+ * subtracting the sum of the activations. */
+static int trit_shift(int n /* 0..15 */) { return 8 * (n % 4) + 2 * (n / 4); }
 
 void orc_pack_trits(int d, const int8_t* trit, uint32_t* packed) {
     for (int k = 0; k < d / 16; k++) packed[k] = 0;
     for (int j = 0; j < d; j++) {
-        uint32_t code = trit[j] == 1 ? 1u : trit[j] == -1 ? 3u : 0u;
+        uint32_t code = (uint32_t)(trit[j] + 1);
         packed[j / 16] |= code << trit_shift(j % 16);
     }
 }
 
 int orc_unpack_trit(const uint32_t* packed, int j) {
     uint32_t code = (packed[j / 16] >> trit_shift(j % 16)) & 3u;
-    return code == 1u ? 1 : code == 3u ? -1 : 0;
+    return (int)code - 1;
 }
 
 /* Sketch of every gate and up row of E experts: sk[E, I, d/16], alpha[E, I]. */

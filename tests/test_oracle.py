@@ -169,15 +169,16 @@ def test_quantize_error_bound_and_range():
 
 # ---------------------------------------------------------------- packing
 def _independent_unpack(words, d):
-    """Decoder written from the documented layout, vectorised differently."""
+    """Decoder written from the documented layout, vectorised differently:
+    for each byte b and pair p, the 2-bit field at bits 8b + 2p is the code
+    of position 4p + b."""
     w = np.asarray(words, np.uint64)
     out = np.zeros((w.size, 16), np.int64)
-    for n in range(8):
-        lo = (w >> np.uint64(4 * n)) & np.uint64(3)
-        hi = (w >> np.uint64(4 * n + 2)) & np.uint64(3)
-        out[:, n] = np.where(lo == 1, 1, np.where(lo == 3, -1, 0))
-        out[:, 8 + n] = np.where(hi == 1, 1, np.where(hi == 3, -1, 0))
-        assert not np.any(lo == 2) and not np.any(hi == 2)
+    for b in range(4):
+        for p in range(4):
+            code = (w >> np.uint64(8 * b + 2 * p)) & np.uint64(3)
+            assert not np.any(code == 3)
+            out[:, 4 * p + b] = code.astype(np.int64) - 1
     return out.reshape(-1)[:d]
 
 
@@ -186,12 +187,22 @@ def test_pack_roundtrip_and_layout():
     t = rng.integers(-1, 2, 256).astype(np.int8)
     p = O.pack_trits(t)
     assert np.array_equal(_independent_unpack(p, 256), t)
-    one = np.zeros(16, np.int8)
-    one[9] = -1  # position 8+1 -> bits [6,7] = 11
-    assert O.pack_trits(one)[0] == 0b11 << 6
-    one[:] = 0
-    one[3] = 1  # position 3 -> bits [12,13] = 01
-    assert O.pack_trits(one)[0] == 1 << 12
+    zero = np.zeros(16, np.int8)
+    assert O.pack_trits(zero)[0] == 0x55555555  # every code 01 (T = 0)
+    one = zero.copy()
+    one[9] = -1  # position 9 = 4*2 + 1: byte 1, pair 2 -> bits [12, 13] = 00
+    assert O.pack_trits(one)[0] == 0x55555555 & ~(3 << 12)
+    one = zero.copy()
+    one[3] = 1  # position 3 = 4*0 + 3: byte 3, pair 0 -> bits [24, 25] = 10
+    assert O.pack_trits(one)[0] == (0x55555555 & ~(3 << 24)) | (2 << 24)
+    # a masked word times four int8 activations, minus their sum, is the dot
+    q = rng.integers(-127, 128, 16)
+    w = int(O.pack_trits(t[:16])[0])
+    acc = 0
+    for pp in range(4):
+        m = (w >> (2 * pp)) & 0x03030303
+        acc += sum(((m >> (8 * b)) & 0xFF) * q[4 * pp + b] for b in range(4))
+    assert acc - q.sum() == int(np.dot(t[:16].astype(np.int64), q))
 
 
 # ---------------------------------------------------------------- sketch
