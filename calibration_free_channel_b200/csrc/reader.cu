@@ -61,7 +61,7 @@ __device__ __noinline__ int idiv(int a, int b) { return a / b; }
 // ------------------------------------------------------- launch geometry
 // Shared-memory offsets and the partitions of a launch, computed on the host.
 struct Layout {
-  int mbar, misc, hist, x, q, logit, alpha, sig, sa, zred, zparts, z, cor, apos, candm, keptm, ulist, dlist, keys,
+  int mbar, misc, hist, x, q, logit, alpha, sig, sa, zred, zparts, z, apos, candm, keptm, ulist, dlist, keys,
       ubar, vown, ring, total;
   int ntok;        // tokens held in smem (fused routing: B; otherwise NT)
   int own_max;     // max channels per CTA
@@ -118,7 +118,6 @@ __host__ inline Layout make_layout(int NT, int ntok, bool fused, int E, int I, i
   L.zred = dense ? 0 : take(NWARP * NT * rr * 4);
   L.zparts = dense ? 0 : take(cs * NT * rr * 4);
   L.z = dense ? 0 : take(NT * rr * 4);
-  L.cor = dense ? 0 : take(NT * rr * 4);
   L.apos = dense ? 0 : take(NT * I * 4);  // a by union position
   L.candm = dense ? 0 : take(NT * L.words * 4);
   L.keptm = dense ? 0 : take(NT * L.words * 4);
@@ -834,35 +833,25 @@ __device__ int down_rows(const ExpertArgs& a, int e, int j0, int ncq, int nr8, i
   return rg;
 }
 
-// Warp totals of the sketch dots of 4 channels, spread over the lanes: every
-// lane holds partial sums pg[c][t] (gate) and pu[c][t] (up) of channel c and
-// token t; a reduce-scatter leaves lane L (L < 16) with the totals (g, u) of
-// channel (L >> 2) & 3 and token (L >> 1) & 1 (token 0 when NT = 1).
+// Warp totals of one channel's sketch dots: G (gate) and U (up) of each
+// token, reduced two values at a time.  On return lanes 0..15 hold (g, u) of
+// token (lane >> 3) & 1 when NT = 2, of token 0 when NT = 1.
 template <int NT>
-__device__ __forceinline__ void reduce_scatter4(const int (&pg)[4][NT], const int (&pu)[4][NT], int& g, int& u) {
+__device__ __forceinline__ void reduce_gu(const int (&G)[NT], const int (&U)[NT], int& g, int& u) {
   const int lane = threadIdx.x & 31;
-  const bool lo = lane < 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
-  int v1[4][NT];
-#pragma unroll
-  for (int c = 0; c < 4; c++)
-#pragma unroll
-    for (int t = 0; t < NT; t++)
-      v1[c][t] = (lo ? pg[c][t] : pu[c][t]) + __shfl_xor_sync(kFull, lo ? pu[c][t] : pg[c][t], 16);
-  int v2[2][NT];
-#pragma unroll
-  for (int c = 0; c < 2; c++)
-#pragma unroll
-    for (int t = 0; t < NT; t++)
-      v2[c][t] = (b3 ? v1[2 + c][t] : v1[c][t]) + __shfl_xor_sync(kFull, b3 ? v1[c][t] : v1[2 + c][t], 8);
-  int v3[NT];
-#pragma unroll
-  for (int t = 0; t < NT; t++) v3[t] = (b2 ? v2[1][t] : v2[0][t]) + __shfl_xor_sync(kFull, b2 ? v2[0][t] : v2[1][t], 4);
+  const bool lo = lane < 16;
   int v;
   if (NT == 1) {
-    v = v3[0] + __shfl_xor_sync(kFull, v3[0], 2);
+    v = (lo ? G[0] : U[0]) + __shfl_xor_sync(kFull, lo ? U[0] : G[0], 16);
+    v += __shfl_xor_sync(kFull, v, 8);
   } else {
-    v = (b1 ? v3[NT - 1] : v3[0]) + __shfl_xor_sync(kFull, b1 ? v3[0] : v3[NT - 1], 2);
+    const int k0 = (lo ? G[0] : U[0]) + __shfl_xor_sync(kFull, lo ? U[0] : G[0], 16);
+    const int k1 = (lo ? G[NT - 1] : U[NT - 1]) + __shfl_xor_sync(kFull, lo ? U[NT - 1] : G[NT - 1], 16);
+    const bool hi8 = lane & 8;
+    v = (hi8 ? k1 : k0) + __shfl_xor_sync(kFull, hi8 ? k0 : k1, 8);
   }
+  v += __shfl_xor_sync(kFull, v, 4);
+  v += __shfl_xor_sync(kFull, v, 2);
   v += __shfl_xor_sync(kFull, v, 1);
   const int o = __shfl_xor_sync(kFull, v, 16);
   g = lo ? v : o;
@@ -902,12 +891,16 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
   __syncthreads();
   if (DBG) stamp(a, cid, rank, 0);
 
+  // Programmatic dependent launch: the next kernel in the stream may be
+  // scheduled now (onto free SMs); this one reads nothing in global memory
+  // before the previous kernel has completed and its writes are visible.
+  pdl_trigger();
+  pdl_wait();
   char4 sv_pre = make_char4(0, 0, 0, 0);  // rotation signs of elements 4 tid .. 4 tid + 3 (in-kernel routing)
   if (FUSED) {
     if (tid < a.d / 4) sv_pre = __ldg(reinterpret_cast<const char4*>(a.rot_sign) + tid);
     if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, cluster)) return;  // uniform per cluster
   } else {
-    pdl_wait();
     if (!load_item_table(a, cid, misc, NT)) return;
   }
   if (DBG) stamp(a, cid, rank, 3);
@@ -967,7 +960,6 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
   float* sa = reinterpret_cast<float*>(smem + L.sa);          // [I, NT] (sigma, ahat) pairs, slices from the owners
   float* zparts = reinterpret_cast<float*>(smem + L.zparts);  // [cs, NT, r]
   float* z = reinterpret_cast<float*>(smem + L.z);            // [NT, r]
-  float* cor = reinterpret_cast<float*>(smem + L.cor);        // [NT, r]
   float* apos = reinterpret_cast<float*>(smem + L.apos);      // [NT, I] by union position
   uint32_t* candm = reinterpret_cast<uint32_t*>(smem + L.candm);
   uint32_t* keptm = reinterpret_cast<uint32_t*>(smem + L.keptm);  // over union positions
@@ -1010,112 +1002,122 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
       for (int kk = 0; kk < 4; kk++) qr[t][kk] = lane < nv ? qv[4 * lane + kk] : make_uint4(0u, 0u, 0u, 0u);
     }
     // warp w takes channel 16 j + w of every sketch chunk j (one channel per
-    // warp and chunk); the dots of 4 chunks are reduced together
-    const int tt = NT == 2 ? (lane >> 1) & 1 : 0;  // token of lanes 0..15 after reduce_scatter4
-    const int cl = (lane >> 2) & 3;                 // channel (of the 4) of lanes 0..15
-    const bool writer = lane < 16 && (lane & (NT == 2 ? 1 : 3)) == 0;
-    const int sqt = NT == 2 && tt ? sq[NT - 1] : sq[0];
-    const float cxt = cxs[tix[NT == 2 && tt ? NT - 1 : 0]];
+    // warp and chunk).  Each channel's dots are reduced over the warp and
+    // parked in the warp's slot of gu; every 4 chunks (and at the end) one
+    // pass over the lanes turns the parked sums into sigma and ahat.
+    int* gu = hist + warp * 4 * NT * 2;  // [4 channels][NT tokens][g, u]; hist is free during the screen
     int rb = 0, par = 0;  // first chunk of the resident round, parity of its barriers
 #pragma unroll 1
-    for (int jb = 0; jb < nchunk; jb += 4) {
-      int pg[4][NT], pu[4][NT];
-#pragma unroll
-      for (int c = 0; c < 4; c++) {
-        const int j = jb + c, li = 16 * j + warp;
-#pragma unroll
-        for (int t = 0; t < NT; t++) pg[c][t] = pu[c][t] = 0;
-        if (j < nchunk && j == rb + L.sk_round) {
-          // the next round of chunks reuses the buffers: every warp is done with them
-          __syncthreads();
-          rb = j;
-          par ^= 1;
-          if (tid == 0) {
-            fence_proxy_async();
-            const int c1 = min(nchunk, j + L.sk_round);
-            for (int ch = j; ch < c1; ch++) issue_sketch(a, L, skbuf, skbars, e, i0, i1, ch, ch - j);
-          }
+    for (int j = 0; j < nchunk; j++) {
+      const int li = 16 * j + warp;
+      if (j == rb + L.sk_round) {
+        // the next round of chunks reuses the buffers: every warp is done with them
+        __syncthreads();
+        rb = j;
+        par ^= 1;
+        if (tid == 0) {
+          fence_proxy_async();
+          const int c1 = min(nchunk, j + L.sk_round);
+          for (int ch = j; ch < c1; ch++) issue_sketch(a, L, skbuf, skbars, e, i0, i1, ch, ch - j);
         }
-        if (j < nchunk && li < nown) {
-          const int slot = j - rb;
-          if (!mbar_wait_bounded(&skbars[slot], par, err)) misc[MI_DONE] = 1;
-          const uint4* gw = reinterpret_cast<const uint4*>(skbuf + (size_t)slot * 2 * L.skc + warp * (d / 4));
-          const uint4* uw = reinterpret_cast<const uint4*>(skbuf + (size_t)slot * 2 * L.skc + L.skc + warp * (d / 4));
-          int ga[NT][4], ua[NT][4];
+      }
+      int G[NT], U[NT];
 #pragma unroll
-          for (int t = 0; t < NT; t++)
+      for (int t = 0; t < NT; t++) G[t] = U[t] = 0;
+      if (li < nown) {
+        const int slot = j - rb;
+        if (!mbar_wait_bounded(&skbars[slot], par, err)) misc[MI_DONE] = 1;
+        const uint4* gw = reinterpret_cast<const uint4*>(skbuf + (size_t)slot * 2 * L.skc + warp * (d / 4));
+        const uint4* uw = reinterpret_cast<const uint4*>(skbuf + (size_t)slot * 2 * L.skc + L.skc + warp * (d / 4));
+        int ga[NT][4], ua[NT][4];
 #pragma unroll
-            for (int kk = 0; kk < 4; kk++) ga[t][kk] = ua[t][kk] = 0;
+        for (int t = 0; t < NT; t++)
+#pragma unroll
+          for (int kk = 0; kk < 4; kk++) ga[t][kk] = ua[t][kk] = 0;
 #pragma unroll 1
-          for (int vv = lane; vv < nv; vv += 32) {
-            const uint4 g4 = gw[vv], u4 = uw[vv];
-#pragma unroll
-            for (int t = 0; t < NT; t++) {
-              uint4 q0 = qr[t][0], q1 = qr[t][1], q2 = qr[t][2], q3 = qr[t][3];
-              if (vv != lane) {
-                const uint4* qv = reinterpret_cast<const uint4*>(smem + L.q + (size_t)tix[t] * d) + 4 * vv;
-                q0 = qv[0];
-                q1 = qv[1];
-                q2 = qv[2];
-                q3 = qv[3];
-              }
-              code_dot16(g4.x, q0, ga[t]);
-              code_dot16(g4.y, q1, ga[t]);
-              code_dot16(g4.z, q2, ga[t]);
-              code_dot16(g4.w, q3, ga[t]);
-              code_dot16(u4.x, q0, ua[t]);
-              code_dot16(u4.y, q1, ua[t]);
-              code_dot16(u4.z, q2, ua[t]);
-              code_dot16(u4.w, q3, ua[t]);
-            }
-          }
+        for (int vv = lane; vv < nv; vv += 32) {
+          const uint4 g4 = gw[vv], u4 = uw[vv];
 #pragma unroll
           for (int t = 0; t < NT; t++) {
-            pg[c][t] = code_dot_total(ga[t]);
-            pu[c][t] = code_dot_total(ua[t]);
+            uint4 q0 = qr[t][0], q1 = qr[t][1], q2 = qr[t][2], q3 = qr[t][3];
+            if (vv != lane) {
+              const uint4* qv = reinterpret_cast<const uint4*>(smem + L.q + (size_t)tix[t] * d) + 4 * vv;
+              q0 = qv[0];
+              q1 = qv[1];
+              q2 = qv[2];
+              q3 = qv[3];
+            }
+            code_dot16(g4.x, q0, ga[t]);
+            code_dot16(g4.y, q1, ga[t]);
+            code_dot16(g4.z, q2, ga[t]);
+            code_dot16(g4.w, q3, ga[t]);
+            code_dot16(u4.x, q0, ua[t]);
+            code_dot16(u4.y, q1, ua[t]);
+            code_dot16(u4.z, q2, ua[t]);
+            code_dot16(u4.w, q3, ua[t]);
           }
+        }
+#pragma unroll
+        for (int t = 0; t < NT; t++) {
+          G[t] = code_dot_total(ga[t]);
+          U[t] = code_dot_total(ua[t]);
         }
       }
       int gs, us;
-      reduce_scatter4<NT>(pg, pu, gs, us);
-      gs -= sqt;
-      us -= sqt;
-      const int li = 16 * (jb + cl) + warp;
-      const bool valid = lane < 16 && jb + cl < nchunk && li < nown && tt < n;
-      const int i = i0 + li;
-      const float gh = __fmul_rn(__fmul_rn((float)gs, valid ? alg[li] : 0.0f), cxt);
-      const float uh = __fmul_rn(__fmul_rn((float)us, valid ? alu[li] : 0.0f), cxt);
-      const float ah = __fmul_rn(silu_r(gh), uh);
-      if (valid && writer) {
-        reinterpret_cast<float2*>(sa)[i * NT + tt] = make_float2(fabsf(ah), ah);
-        if (DBG) {
-          const size_t off = ((size_t)misc[MI_TOK + tt] * a.top_e + misc[MI_SLOT + tt]) * I + i;
-          if (a.dbg_G) a.dbg_G[off] = gs;
-          if (a.dbg_U) a.dbg_U[off] = us;
-          if (a.dbg_sigma) a.dbg_sigma[off] = fabsf(ah);
-        }
+      reduce_gu<NT>(G, U, gs, us);
+      if (lane < 16 && (lane & 7) == 0) {
+        const int t = NT == 2 ? lane >> 3 : 0;
+        gu[((j & 3) * NT + t) * 2] = gs;
+        gu[((j & 3) * NT + t) * 2 + 1] = us;
       }
-      // partial recovery input z_w = sum over this warp's channels of ahat_i Ubar_i
-      if (r > 0) {
-        if (!uv_ready) {
-          if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
-          uv_ready = true;
+      if ((j & 3) == 3 || j == nchunk - 1) {
+        // the batch's epilogue: lane (channel c, token t), c < 4, t < NT
+        __syncwarp();
+        const int jb = j & ~3;
+        const int c = lane / NT, t = lane - c * NT;
+        const int lc = 16 * (jb + c) + warp;
+        const bool valid = lane < 4 * NT && jb + c <= j && lc < nown && t < n;
+        int g2 = 0, u2 = 0;
+        if (lane < 4 * NT) {
+          g2 = gu[lane * 2] - (NT == 2 && t ? sq[NT - 1] : sq[0]);
+          u2 = gu[lane * 2 + 1] - (NT == 2 && t ? sq[NT - 1] : sq[0]);
         }
+        const float cx = cxs[tix[NT == 2 && t ? NT - 1 : 0]];
+        const float gh = __fmul_rn(__fmul_rn((float)g2, valid ? alg[lc] : 0.0f), cx);
+        const float uh = __fmul_rn(__fmul_rn((float)u2, valid ? alu[lc] : 0.0f), cx);
+        const float ah = __fmul_rn(silu_r(gh), uh);
+        if (valid) {
+          reinterpret_cast<float2*>(sa)[(i0 + lc) * NT + t] = make_float2(fabsf(ah), ah);
+          if (DBG) {
+            const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * I + i0 + lc;
+            if (a.dbg_G) a.dbg_G[off] = g2;
+            if (a.dbg_U) a.dbg_U[off] = u2;
+            if (a.dbg_sigma) a.dbg_sigma[off] = fabsf(ah);
+          }
+        }
+        // partial recovery input z_w = sum over this warp's channels of ahat_i Ubar_i
+        if (r > 0) {
+          if (!uv_ready) {
+            if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
+            uv_ready = true;
+          }
 #pragma unroll
-        for (int c = 0; c < 4; c++) {
-          const int lc = 16 * (jb + c) + warp;
-          if (jb + c < nchunk && lc < nown) {
+          for (int cc = 0; cc < 4; cc++) {
+            const int lcc = 16 * (jb + cc) + warp;
+            if (jb + cc <= j && lcc < nown) {
 #pragma unroll
-            for (int t = 0; t < NT; t++) {
-              const float aht = __shfl_sync(kFull, ah, 4 * c + 2 * t);
+              for (int tt = 0; tt < NT; tt++) {
+                const float aht = __shfl_sync(kFull, ah, cc * NT + tt);
 #pragma unroll
-              for (int kk = 0; kk < 4; kk++) {
-                const int p = lane + 32 * kk;
-                if (p < r && t < n) zacc[t][kk] = fmaf(aht, bf16f(ub[lc * r + p]), zacc[t][kk]);
+                for (int kk = 0; kk < 4; kk++) {
+                  const int p = lane + 32 * kk;
+                  if (p < r && tt < n) zacc[tt][kk] = fmaf(aht, bf16f(ub[lcc * r + p]), zacc[tt][kk]);
+                }
               }
             }
           }
         }
+        __syncwarp();
       }
     }
     if (FUSED && warp == NWARP - 1) route_weights(a, L, smem, misc, cid, rank);
@@ -1197,6 +1199,12 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
           mbar_expect_tx(bar, 2 * rowb);
           bulk_g2s(dst, a.w_gate + ((size_t)e * I + i) * d, rowb, bar);
           bulk_g2s(dst + rowb, a.w_up + ((size_t)e * I + i) * d, rowb, bar);
+          if (j + P < m1 - m0) {
+            // the row this slot takes next starts moving into L2 now
+            const int i2 = ulist[u0 + m0 + j + P];
+            bulk_prefetch_l2(a.w_gate + ((size_t)e * I + i2) * d, rowb);
+            bulk_prefetch_l2(a.w_up + ((size_t)e * I + i2) * d, rowb);
+          }
         },
         [&](int j, int s) {
           const int u = u0 + m0 + j, i = ulist[u];
@@ -1305,19 +1313,23 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
     }
     for (; gg < rg; gg++) s0 += rp[gg * gstride];
     const float s = (s0 + s1) + (s2 + s3);
-    if (oc < ncols) yfin[t * L.cols_max + oc] = s;
-    else cor[t * r + (oc - ncols)] = s;
-  }
-  __syncthreads();
-  if (r > 0) {
+    if (oc < ncols) {
+      yfin[t * L.cols_max + oc] = s;
+    } else {
+      // z = (sum over the CTAs' partials of all channels) - (the kept part)
+      const int p = oc - ncols;
+      float z0 = 0.0f, z1 = 0.0f;
+      int o = 0;
 #pragma unroll 1
-    for (int t = 0; t < n; t++)
-      for (int p = tid; p < r; p += NTHR) {
-        float zz = 0.0f;
-#pragma unroll 1
-        for (int o = 0; o < cs; o++) zz += zparts[(o * NT + t) * r + p];
-        z[t * r + p] = zz - cor[t * r + p];
+      for (; o + 2 <= cs; o += 2) {
+        z0 += zparts[(o * NT + t) * r + p];
+        z1 += zparts[((o + 1) * NT + t) * r + p];
       }
+      if (o < cs) z0 += zparts[(o * NT + t) * r + p];
+      z[t * r + p] = (z0 + z1) - s;
+    }
+  }
+  if (r > 0) {
     if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
     __syncthreads();
     const uint16_t* vo = reinterpret_cast<const uint16_t*>(smem + L.vown);
@@ -1341,8 +1353,8 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
         }
         yfin[t * L.cols_max + col] += rec0 + rec1;
       }
-    __syncthreads();
   }
+  __syncthreads();
   if (DBG) stamp(a, cid, rank, 12);
   write_and_combine(a, rank, j0, ncols, L.cols_max, yfin, misc,
                     FUSED ? reinterpret_cast<const float*>(misc + MI_RW) : a.ws.wts);
@@ -1368,11 +1380,12 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
   if (tid == 0) misc[MI_DONE] = 0;
   fence_mbar_init();
   __syncthreads();
+  pdl_trigger();
+  pdl_wait();
   if (FUSED) {
     if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, cluster)) return;
     if (warp == NWARP - 1) route_weights(a, L, smem, misc, cid, rank);
   } else {
-    pdl_wait();
     if (!load_item_table(a, cid, misc, NT)) return;
     load_tokens(a, L, smem, misc, misc[MI_N], false);
     __syncthreads();
@@ -1401,6 +1414,11 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
           mbar_expect_tx(bar, 2 * rowb);
           bulk_g2s(dst, a.w_gate + ((size_t)e * I + i) * d, rowb, bar);
           bulk_g2s(dst + rowb, a.w_up + ((size_t)e * I + i) * d, rowb, bar);
+          if (j + P < m1 - m0) {
+            // the row this slot takes next starts moving into L2 now
+            bulk_prefetch_l2(a.w_gate + ((size_t)e * I + i + P) * d, rowb);
+            bulk_prefetch_l2(a.w_up + ((size_t)e * I + i + P) * d, rowb);
+          }
         },
         [&](int j, int s) {
           const int i = i0 + m0 + j;
@@ -1597,7 +1615,7 @@ cudaError_t launch_expert(const ExpertArgs& a0, cudaStream_t s, bool dense) {
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = plan.fused ? 1 : 2;  // the in-kernel router makes it the step's first kernel
+  cfg.numAttrs = 2;  // programmatic dependent launch: overlaps this launch with the previous kernel's tail
   void* args[] = {&a, &plan.L};
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
