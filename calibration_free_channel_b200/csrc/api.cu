@@ -68,6 +68,7 @@ moe_status check_layer(const moe_reader_layer* L, bool sparse) {
     REQUIRE_PTR(L->sk_up);
     REQUIRE_PTR(L->alpha_gate);
     REQUIRE_PTR(L->alpha_up);
+    REQUIRE(L->recovery_input == 0 || L->recovery_input == 1, "recovery_input = %d: use 0 or 1", L->recovery_input);
     REQUIRE(L->r >= 0 && L->r <= 128 && L->r % 8 == 0 && L->r <= L->I, "r = %d: need r in {0, 8, ..., 128}, r <= I",
             L->r);
     if (L->r > 0) {
@@ -127,6 +128,7 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   a.k = k;
   a.c = c;
   a.r = dense ? 0 : L->r;
+  a.recovery_input = dense ? 0 : L->recovery_input;
   a.cs = 0;  // chosen at launch (16 when schedulable, else 8)
   a.nmax = B < moe::kMaxGroup ? B : moe::kMaxGroup;
   a.x = x;

@@ -50,6 +50,7 @@ struct ExpertArgs {
   int cs;            // CTAs per cluster (one cluster per work item)
   int nmax;          // max tokens per work item this launch
   int ring_rows;     // copy-ring row slots per warp (sparse) / rows (dense)
+  int recovery_input;  // 0: ahat of every skipped channel; 1: exact a of dropped candidates
   const uint16_t* x;
   const uint16_t* w_router;  // routing inside the expert kernel (small B)
   const float* bias;

@@ -777,8 +777,9 @@ __device__ void write_and_combine(const ExpertArgs& a, int rank, int j0, int nco
 // row groups); chunks q < ncq are 8 W_down columns of this CTA's slice, the
 // rest 8 entries of the Ubar row (recovery).  Rows are loaded 8 at a time
 // per thread, all in flight together.  coef(m, i, is_w, co[NT]) gives each
-// token's coefficient of row m (channel i).  Per-group partial sums land in
-// red[g][t][q * 8 + c]; returns rg.
+// token's coefficient of row m (channel i) and returns whether the chunk is
+// needed at all (a chunk whose coefficients are all zero is not read).
+// Per-group partial sums land in red[g][t][q * 8 + c]; returns rg.
 template <int NT, class Chan, class Coef>
 __device__ int down_rows(const ExpertArgs& a, int e, int j0, int ncq, int nr8, int nrows, int rr, Chan chan,
                          Coef coef, float* red) {
@@ -808,8 +809,7 @@ __device__ int down_rows(const ExpertArgs& a, int e, int j0, int ncq, int nr8, i
         for (int t = 0; t < NT; t++) co[u][t] = 0.0f;
         if (m < nrows) {
           const int i = chan(m);
-          w[u] = __ldg(reinterpret_cast<const uint4*>(base + (size_t)i * stride));
-          coef(m, i, is_w, co[u]);
+          if (coef(m, i, is_w, co[u])) w[u] = __ldg(reinterpret_cast<const uint4*>(base + (size_t)i * stride));
         }
       }
 #pragma unroll
@@ -1284,15 +1284,28 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
   // ---------------------------------------------- D: down rows + recovery
   float* red = reinterpret_cast<float*>(smem + L.ring);
   const int ncq = ncols >> 3, nr8 = r >> 3, nch = ncq + nr8;
+  // Rows: the kept union (recovery from the sketch estimates of every skipped
+  // channel: the factor rows of the kept channels enter with -ahat), or, with
+  // the exact recovery input, the whole candidate union (factor rows of the
+  // candidates enter with -(ahat - a) when dropped, -ahat when kept; down
+  // rows are read for the kept ones only).
+  const bool rec_exact = a.recovery_input == 1;
   const int rg = down_rows<NT>(
-      a, e, j0, ncq, nr8, nD, r, [&](int m) { return ulist[dlist[m]]; },
+      a, e, j0, ncq, nr8, rec_exact ? nU : nD, r, [&](int m) { return ulist[rec_exact ? m : dlist[m]]; },
       [&](int m, int i, bool is_w, float (&co)[NT]) {
-        const int u = dlist[m];
+        const int u = rec_exact ? m : dlist[m];
+        bool need = false;
 #pragma unroll
         for (int t = 0; t < NT; t++) {
           const bool kept = t < n && ((keptm[t * L.words + (u >> 5)] >> (u & 31)) & 1u);
-          co[t] = kept ? (is_w ? apos[t * I + u] : sa[(i * NT + t) * 2 + 1]) : 0.0f;
+          const bool cand = t < n && ((candm[t * L.words + (i >> 5)] >> (i & 31)) & 1u);
+          const float ah = sa[(i * NT + t) * 2 + 1];
+          if (is_w) co[t] = kept ? apos[t * I + u] : 0.0f;
+          else if (kept) co[t] = ah;
+          else co[t] = rec_exact && cand ? __fsub_rn(ah, apos[t * I + u]) : 0.0f;
+          need |= kept || (!is_w && rec_exact && cand);
         }
+        return need;
       },
       red);
   float* yfin = reinterpret_cast<float*>(smem + L.x);  // [n, cols_max]; x is no longer needed
@@ -1454,6 +1467,7 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
       [&](int m, int, bool, float (&co)[NT]) {
 #pragma unroll
         for (int t = 0; t < NT; t++) co[t] = t < n ? h[t * I + m] : 0.0f;
+        return true;
       },
       red);
   float* out = reinterpret_cast<float*>(smem + L.x);

@@ -29,7 +29,8 @@ class MoeReaderLayer(C.Structure):
                 ("w_router", C.c_void_p), ("router_bias", C.c_void_p), ("w_gate", C.c_void_p),
                 ("w_up", C.c_void_p), ("w_down", C.c_void_p), ("rot_sign", C.c_void_p),
                 ("sk_gate", C.c_void_p), ("sk_up", C.c_void_p), ("alpha_gate", C.c_void_p),
-                ("alpha_up", C.c_void_p), ("u_sigma", C.c_void_p), ("v", C.c_void_p)]
+                ("alpha_up", C.c_void_p), ("u_sigma", C.c_void_p), ("v", C.c_void_p),
+                ("recovery_input", C.c_int32)]
 
 
 class MoeReaderDebug(C.Structure):
@@ -215,13 +216,13 @@ class Layer:
             self.r = int(u_sigma.shape[-1])
         return self
 
-    def struct(self, r: int | None = None) -> MoeReaderLayer:
+    def struct(self, r: int | None = None, recovery_input: int = 0) -> MoeReaderLayer:
         rr = self.r if r is None else r
         return MoeReaderLayer(self.E, self.I, self.d, self.top_e, rr, _ptr(self.w["w_router"]),
                               _ptr(self.w.get("router_bias")), _ptr(self.w["w_gate"]), _ptr(self.w["w_up"]),
                               _ptr(self.w["w_down"]), _ptr(self.rot_sign), _ptr(self.sk_gate), _ptr(self.sk_up),
                               _ptr(self.alpha_gate), _ptr(self.alpha_up),
-                              _ptr(self.u_sigma) if rr else None, _ptr(self.v) if rr else None)
+                              _ptr(self.u_sigma) if rr else None, _ptr(self.v) if rr else None, recovery_input)
 
     def workspace(self, B: int):
         nb = moe_reader_workspace_bytes(B, self.E, self.top_e, self.I, self.d, 1, 1, self.r)
@@ -230,7 +231,7 @@ class Layer:
         return self._ws
 
     def forward(self, x, k: int, c: int, residual=None, debug: bool = False, r: int | None = None, stream=None,
-                out=None):
+                out=None, recovery_input: int = 0):
         B = x.shape[0]
         ws = self.workspace(B)
         y = out if out is not None else torch.empty_like(x)
@@ -250,7 +251,7 @@ class Layer:
                          y_expert=torch.empty(P + (self.d,), dtype=torch.float32, device=dev),
                          phase_ns=torch.zeros((B * self.top_e, 16), dtype=torch.int64, device=dev))
             dbg = MoeReaderDebug(*[_ptr(dbg_t[n]) for n, _ in MoeReaderDebug._fields_])
-        moe_reader_forward(self.struct(r), B, k, c, x, residual, y, dbg, ws, ws.numel(), stream)
+        moe_reader_forward(self.struct(r, recovery_input), B, k, c, x, residual, y, dbg, ws, ws.numel(), stream)
         return (y, dbg_t) if debug else y
 
     def forward_dense(self, x, residual=None, stream=None, out=None):

@@ -74,6 +74,13 @@ typedef struct {
   const float* alpha_up;       /* [E, I]                                         */
   const uint16_t* u_sigma;     /* [E, I, r] bf16 = U_r Sigma_r of W_down, or NULL */
   const uint16_t* v;           /* [E, d, r] bf16 = V_r of W_down, or NULL         */
+  /* What the low-rank map recovers from ("A reader that needs no data at
+   * all": skipped channels come back through the map).  0: the sketch
+   * estimates ahat_i of every skipped channel, z = sum_{i not kept} ahat_i
+   * Ubar_i.  1: the exact a_i of the candidates the top-k dropped (the exact
+   * stage computed them) and ahat_i only outside the candidate set; it reads
+   * no extra weight rows.  Any other value is MOE_EINVAL. */
+  int32_t recovery_input;
 } moe_reader_layer;
 
 /* Optional per-stage outputs of moe_reader_forward (each pointer may be

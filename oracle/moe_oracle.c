@@ -328,10 +328,14 @@ static float exact_dot(const uint16_t* row, const uint16_t* x, int d) {
  *        z   = sum_{i not in K} ahat_i Ubar[i,:].
  *     Reading: the map is applied to the sketch estimates of every skipped
  *     channel.  Accumulation is fp64.
+ *     recovery_input == 1 is the variant that feeds the map the exact a_i
+ *     of the candidates step 4 dropped (computed in step 3 anyway) and the
+ *     sketch estimates only outside the candidate set:
+ *        z = sum_{i in C, i not in K} a_i Ubar[i,:] + sum_{i not in C} ahat_i Ubar[i,:].
  * exact_mode != 0 replaces the sketch estimates by the exact g, u (a test
  * mode for the invariant "exact sketch + full-rank map = dense expert").
  * r == 0 or ubar == NULL disables recovery. */
-void orc_expert_reader(int I, int d, int k, int c, int r, int exact_mode,
+void orc_expert_reader(int I, int d, int k, int c, int r, int exact_mode, int recovery_input,
                        const uint16_t* x, const int8_t* q, float cx,
                        const uint32_t* skg, const uint32_t* sku,
                        const float* ag, const float* au,
@@ -381,6 +385,8 @@ void orc_expert_reader(int I, int d, int k, int c, int r, int exact_mode,
     }
     orc_top_n(c, cand, absa, k, kept);
     for (int t = 0; t < k; t++) is_kept[kept[t]] = 1;
+    char* is_cand = (char*)calloc((size_t)I, 1);
+    for (int t = 0; t < c; t++) is_cand[cand[t]] = 1;
     if (dbg_cand) memcpy(dbg_cand, cand, sizeof(int32_t) * (size_t)c);
     if (dbg_kept) memcpy(dbg_kept, kept, sizeof(int32_t) * (size_t)k);
     if (dbg_a_kept)
@@ -396,8 +402,9 @@ void orc_expert_reader(int I, int d, int k, int c, int r, int exact_mode,
         double* z = (double*)calloc((size_t)r, sizeof(double));
         for (int i = 0; i < I; i++) {
             if (is_kept[i]) continue;
+            const double zi = (recovery_input == 1 && is_cand[i]) ? (double)a[i] : (double)ahat[i];
             for (int p = 0; p < r; p++)
-                z[p] += (double)ahat[i] * (double)bf16_to_f32(ubar[(long)i * r + p]);
+                z[p] += zi * (double)bf16_to_f32(ubar[(long)i * r + p]);
         }
         for (int j = 0; j < d; j++) {
             double acc = 0.0;
@@ -408,7 +415,7 @@ void orc_expert_reader(int I, int d, int k, int c, int r, int exact_mode,
         free(z);
     }
     free(ahat); free(sigma); free(a); free(absa); free(all);
-    free(cand); free(kept); free(is_kept);
+    free(cand); free(kept); free(is_kept); free(is_cand);
 }
 
 /* ------------------------------------------------------------ whole forward
@@ -416,7 +423,7 @@ void orc_expert_reader(int I, int d, int k, int c, int r, int exact_mode,
  * slot), then y_b = sum over slots (routing order) of w * y_e, fp64, rounded
  * once to bf16.  If `residual` is given, it is added before the rounding.
  * Debug arrays (any may be NULL) are laid out [B, top_e, ...]. */
-void orc_forward(int B, int E, int top_e, int I, int d, int k, int c, int r, int exact_mode,
+void orc_forward(int B, int E, int top_e, int I, int d, int k, int c, int r, int exact_mode, int recovery_input,
                  const uint16_t* x, const uint16_t* w_router, const float* bias,
                  const uint16_t* w_gate, const uint16_t* w_up, const uint16_t* w_down,
                  const int8_t* rot_sign, const uint32_t* sk_gate, const uint32_t* sk_up,
@@ -442,7 +449,7 @@ void orc_forward(int B, int E, int top_e, int I, int d, int k, int c, int r, int
         for (int s = 0; s < top_e; s++) {
             int e = ids[b * top_e + s];
             long ps = (long)b * top_e + s;
-            orc_expert_reader(I, d, k, c, r, exact_mode, x + (long)b * d, q, cx,
+            orc_expert_reader(I, d, k, c, r, exact_mode, recovery_input, x + (long)b * d, q, cx,
                               sk_gate + e * skrow, sk_up + e * skrow,
                               alpha_gate + (long)e * I, alpha_up + (long)e * I,
                               w_gate + e * rowsz, w_up + e * rowsz, w_down + e * rowsz,

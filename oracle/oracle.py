@@ -61,9 +61,9 @@ def lib():
         L.orc_build_sketch.argtypes = [i32, i32, i32, P, P, u64, P, P, P, P, P]
         L.orc_route.argtypes = [i32, i32, i32, i32, P, P, P, P, P, P]
         L.orc_top_n.argtypes = [i32, P, P, i32, P]
-        L.orc_expert_reader.argtypes = [i32, i32, i32, i32, i32, i32, P, P, f32, P, P, P, P,
+        L.orc_expert_reader.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, f32, P, P, P, P,
                                         P, P, P, P, P, P, P, P, P, P, P, P]
-        L.orc_forward.argtypes = [i32] * 9 + [P] * 25
+        L.orc_forward.argtypes = [i32] * 10 + [P] * 25
         L.orc_forward_dense.argtypes = [i32] * 5 + [P] * 9
         L.orc_rmsnorm.argtypes = [i32, i32, f64, P, P]
         _lib = L
@@ -218,9 +218,12 @@ def build_lowrank(w_down, r: int, experts=None):
 
 # ---------------------------------------------------------------- forward
 def forward(x, W: dict, sketch, lowrank, k: int, c: int, r: int, top_e: int,
-            exact_mode: bool = False, residual=None, debug: bool = False):
+            exact_mode: bool = False, residual=None, debug: bool = False, recovery_input: int = 0):
     """The sparse reader over B tokens.  Returns y (uint16 bf16 [B,d]), the
-    fp64 output before rounding and (if debug) the per-stage values."""
+    fp64 output before rounding and (if debug) the per-stage values.
+    recovery_input 1 feeds the low-rank map the exact a of dropped candidates
+    (sketch estimates outside the candidate set); 0 sketch estimates for every
+    skipped channel."""
     x = _u16(x)
     B, d = x.shape
     wr, wg, wu, wd = (_u16(W[n]) for n in ("w_router", "w_gate", "w_up", "w_down"))
@@ -241,7 +244,7 @@ def forward(x, W: dict, sketch, lowrank, k: int, c: int, r: int, top_e: int,
                y_expert=np.empty((B, top_e, d), np.float64)) if debug else None
     g = (lambda n: _p(dbg[n])) if debug else (lambda n: None)
     assert P >= 1
-    lib().orc_forward(B, E, top_e, I, d, k, c, r if us is not None else 0, int(exact_mode),
+    lib().orc_forward(B, E, top_e, I, d, k, c, r if us is not None else 0, int(exact_mode), int(recovery_input),
                       _p(x), _p(wr), _p(bias), _p(wg), _p(wu), _p(wd), _p(s), _p(skg), _p(sku),
                       _p(ag), _p(au), _p(us), _p(vv), _p(res), _p(y), _p(y64),
                       g("ids"), g("weights"), g("dot_gate"), g("dot_up"), g("score"), g("cand"),

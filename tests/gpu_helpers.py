@@ -115,7 +115,7 @@ def bf16_ulp(v):
     return np.exp2(np.floor(np.log2(a)) - 7)
 
 
-def run_pair(layer: M.Layer, oc: OracleCache, x, k, c, top_e, use_oracle_factors=True):
+def run_pair(layer: M.Layer, oc: OracleCache, x, k, c, top_e, use_oracle_factors=True, recovery_input=0):
     """One step on both sides.  With use_oracle_factors the GPU reads the
     oracle's low-rank factors (so both sides read identical inputs);
     otherwise it reads its own build."""
@@ -125,12 +125,13 @@ def run_pair(layer: M.Layer, oc: OracleCache, x, k, c, top_e, use_oracle_factors
     if use_oracle_factors and lr is not None:
         layer.set_lowrank(torch.from_numpy(lr[0].view(np.int16)).view(torch.bfloat16),
                           torch.from_numpy(lr[1].view(np.int16)).view(torch.bfloat16))
-    y, dbg = layer.forward(x.cuda(), k=k, c=c, debug=True)
+    y, dbg = layer.forward(x.cuda(), k=k, c=c, debug=True, recovery_input=recovery_input)
     layer.check()
-    _, y64, odbg = O.forward(x, W, oc.sk, lr, k=k, c=c, r=oc.r, top_e=top_e, debug=True)
+    _, y64, odbg = O.forward(x, W, oc.sk, lr, k=k, c=c, r=oc.r, top_e=top_e, debug=True,
+                             recovery_input=recovery_input)
     return y, dbg, y64, odbg, logits
 
 
-def check_pair(layer, oc, x, k, c, top_e, use_oracle_factors=True, check_kept=True):
-    y, dbg, y64, odbg, logits = run_pair(layer, oc, x, k, c, top_e, use_oracle_factors)
+def check_pair(layer, oc, x, k, c, top_e, use_oracle_factors=True, check_kept=True, recovery_input=0):
+    y, dbg, y64, odbg, logits = run_pair(layer, oc, x, k, c, top_e, use_oracle_factors, recovery_input)
     return compare_step(oc.W, x, y, dbg, y64, odbg, k, ora_logits=logits, check_kept=check_kept)

@@ -170,6 +170,47 @@ def test_all_channels_kept_equals_dense_on_gpu(qwen):
     assert ((ys - yd).norm() / yd.norm()).item() <= REL_L2
 
 
+# ------------------------------------------ recovery from the exact a of dropped candidates
+@pytest.mark.parametrize("B", [1, 2, 5])
+def test_forward_recovery_exact_input_tiny(tiny, B):
+    W, layer, oc = tiny
+    for seed in range(2):
+        x = synth.tokens(256, B, seed=40 + seed)
+        check_pair(layer, oc, x, k=24, c=48, top_e=2, recovery_input=1)
+
+
+@pytest.mark.parametrize("B", [1, 4])
+def test_forward_recovery_exact_input_qwen(qwen, B):
+    W, layer, oc = qwen
+    x = synth.tokens(2048, B, seed=50 + B)
+    check_pair(layer, oc, x, k=136, c=272, top_e=8, recovery_input=1)
+
+
+@pytest.mark.parametrize("k", [1, 24, 77])
+def test_recovery_exact_input_all_candidates_exact_map_equals_dense_on_gpu(tiny, k):
+    """c = I, exact full-rank map (Ubar = I, V = W_down^T): with the exact
+    recovery input every skipped channel comes back exactly, so the reader
+    equals the dense block for every k (a property that holds at any size)."""
+    W, layer, oc = tiny
+    E, I = 8, 128
+    eye = torch.zeros((E, I, I), dtype=torch.float32)
+    eye[:, torch.arange(I), torch.arange(I)] = 1.0
+    vt = W["w_down"].transpose(1, 2).contiguous()
+    layer.set_lowrank(eye.to(torch.bfloat16), vt)
+    try:
+        x = synth.tokens(256, 3, seed=60).cuda()
+        ys = layer.forward(x, k=k, c=I, recovery_input=1).float()
+        yd = layer.forward_dense(x).float()
+        ulp = torch.from_numpy(bf16_ulp(yd.cpu().numpy())).cuda()
+        assert ((ys - yd).abs() - 2 * ulp).max().item() <= MAX_ABS
+        assert ((ys - yd).norm() / yd.norm()).item() <= REL_L2
+        # the default recovery input (sketch estimates) does not come back exactly
+        y0 = layer.forward(x, k=k, c=I, recovery_input=0).float()
+        assert ((y0 - yd).norm() / yd.norm()).item() > 5 * REL_L2
+    finally:
+        layer.set_lowrank(None, None)
+
+
 # ---------------------------------------------------------------- lowrank
 def _lowrank_check(W, layer, r, experts):
     us = layer.u_sigma.float().cpu().numpy()

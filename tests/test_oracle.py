@@ -381,6 +381,35 @@ def test_invariant_exact_sketch_full_rank_map_equals_dense(tiny, k):
         assert np.abs(y0 - yd).max() > 1e-3 * np.abs(yd).max()
 
 
+@pytest.mark.parametrize("k", [1, 24, 77])
+def test_recovery_variant_all_candidates_exact_map_equals_dense(tiny, k):
+    """Recovery variant with every channel a candidate (c = I): each skipped
+    channel enters the map with its exact a, so with the exact full-rank map
+    (Ubar = I, V = W_down^T) the block equals the dense one for every k,
+    without the exact-sketch test mode.  The default input (sketch estimates
+    for the skipped channels) does not."""
+    W, sk, _ = tiny
+    E, I, d = 8, 128, 256
+    x = synth.tokens(d, 2, seed=8)
+    eye = O.f64_to_bf16(np.broadcast_to(np.eye(I), (E, I, I)).copy())
+    wdT = np.ascontiguousarray(np.transpose(synth.bf16_bits(W["w_down"]), (0, 2, 1)))
+    yd = O.forward_dense(x, W, top_e=2)[1]
+    _, yv, _ = O.forward(x, W, sk, (eye, wdT), k=k, c=I, r=I, top_e=2, recovery_input=1)
+    assert np.abs(yv - yd).max() <= 1e-5 * np.abs(yd).max()
+    _, y0, _ = O.forward(x, W, sk, (eye, wdT), k=k, c=I, r=I, top_e=2, recovery_input=0)
+    assert not np.allclose(y0, yd, rtol=0, atol=1e-3 * np.abs(yd).max())
+
+
+def test_recovery_variant_equals_default_in_exact_sketch_mode(tiny):
+    """With exact screening estimates (ahat = a for every channel) the two
+    recovery inputs are the same numbers."""
+    W, sk, lr = tiny
+    x = synth.tokens(256, 2, seed=9)
+    _, ya, _ = O.forward(x, W, sk, lr, k=24, c=48, r=8, top_e=2, exact_mode=True, recovery_input=0)
+    _, yb, _ = O.forward(x, W, sk, lr, k=24, c=48, r=8, top_e=2, exact_mode=True, recovery_input=1)
+    assert np.array_equal(ya, yb)
+
+
 def test_invariant_svd_full_rank_map_equals_dense(tiny):
     """(ii) with the SVD map at full rank r = I (factors rounded to bf16)."""
     W, sk, _ = tiny
