@@ -290,6 +290,14 @@ def run_native(args, rank, world, local_rank):
             shape.top_e * B * accounting.dense_expert_bytes(shape.I, shape.d) if B == 1 else None
         dense = {"us_per_step": dms * 1e3, "speedup_of_sparse": dms / ms,
                  "achieved_gbs": (dbytes / (dms * 1e-3) / 1e9) if dbytes else None}
+    # the exact-input recovery (dropped candidates enter V z with their exact
+    # a): same bytes, the down stage walks every candidate
+    variant = None
+    if r > 0:
+        def variant_step(j):
+            layers[j % nlay].forward(xs[j % ntok], k=k, c=c, out=y, recovery_input=1)
+        vper, _, _ = chunk_loop(variant_step, max(64, args.steps // 4), args.warmup)
+        variant = {"us_per_step": statistics.mean(vper) * 1e3}
     layer.check()
 
     peak, peak_kind = measured_peaks()
@@ -333,6 +341,7 @@ def run_native(args, rank, world, local_rank):
         "gpu_launches": (1 if B <= 2 else 3) * nsteps,  # in-kernel routing at B <= 2
         "clocks": clocks,
         "dense": dense,
+        "recovery_exact_input": variant,
         "l2_flush": {"us_per_step": statistics.mean(fper) * 1e3, "kernel_us": statistics.mean(fkper) * 1e3,
                      "note": "one layer, L2 flushed before every step (also evicts the kernel code)"},
     }
