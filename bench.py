@@ -35,7 +35,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-block µs/step & achieved HBM GB/s (vs ~8 TB/s) at k/I≈18%, batch 1–16"
-WORKLOAD = "qwen3_30b_a3b_layer_b1"
+
+
+def workload_name(B: int) -> str:
+    return f"qwen3_30b_a3b_layer_b{B}"
 
 
 def parse():
@@ -49,6 +52,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--layers", type=int, default=32, help="distinct device copies of the layer the steps cycle through")
+    p.add_argument("--path", type=int, default=0, choices=[0, 1, 2],
+                   help="sparse reader: 0 automatic, 1 one cluster per expert, 2 streamed kernels")
     return p.parse_args()
 
 
@@ -139,6 +144,7 @@ def run_native(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    M.moe_reader_set_path(args.path)
     shape = synth.QWEN3_30B_A3B
     B, k, c, r = args.batch, args.k, 2 * args.k, 32
     W = synth.layer_weights(shape, seed=0, device=str(dev))
@@ -306,7 +312,7 @@ def run_native(args, rank, world, local_rank):
     # its average duration in the back-to-back chunks is the step time.  At
     # larger B the route/select kernels run first; the expert kernel's share
     # is timed with events right around its launch.
-    fused = B <= 2
+    fused = B <= 2 and args.path != 2
     launch_bytes = mean_bytes if fused else mean_ebytes
     launch_ms = ms_max if fused else kms_max
     achieved = launch_bytes / (launch_ms * 1e-3) / 1e9
@@ -324,17 +330,18 @@ def run_native(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16 (int8 x 2-bit sketch dots, fp32 accumulate)",
         "data": "synthetic (seeded; Qwen3-30B-A3B layer shape, lognormal channel scales, Student-t tokens)",
-        "config": {"workload": WORKLOAD, "d": shape.d, "I": shape.I, "E": shape.E, "top_e": shape.top_e,
+        "config": {"workload": workload_name(B), "d": shape.d, "I": shape.I, "E": shape.E, "top_e": shape.top_e,
                    "batch": B, "k": k, "c": c, "r": r, "decode_steps_cycled": ntok,
                    "l2": f"inputs larger than L2: steps cycle through {nlay} distinct device copies of the layer "
                          f"({nlay * layer_bytes(layer) / 1e9:.1f} GB)",
                    "parallelism": f"replicas x{world}", "algorithmic_bytes_per_step": mean_bytes},
-        "roofline": {"bound": "hbm", "kernel": "reader_kernel", "achieved": round(achieved, 1),
+        "roofline": {"bound": "hbm", "kernel": "reader_kernel" if fused else "streamed kernels (screen .. down)",
+                     "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
                      "bytes_per_launch": launch_bytes, "launch_us": launch_ms * 1e3,
                      "isolated_launch_us": kms_max * 1e3,
-                     "traffic": profiled_traffic("reader_kernel", WORKLOAD)},
+                     "traffic": profiled_traffic("reader_kernel", workload_name(B)) if fused else None},
         "step_roofline_frac": round(value / world / peak, 4),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": B * shape.d * 2,
                 "d2h_bytes_per_step": B * shape.d * 2, "us_per_step": float(t[0]) * 1e3},
@@ -435,7 +442,7 @@ def run_reference(args, rank, world):
     return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / tot_n * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64/f32 (oracle)",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "batch": B, "k": k, "c": c, "r": r},
+            "data": "synthetic", "config": {"workload": workload_name(B), "batch": B, "k": k, "c": c, "r": r},
             "cpu_baseline": cb,
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 

@@ -94,11 +94,12 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   REQUIRE_PTR(y);
   OPT_PTR(residual);
   REQUIRE_PTR(workspace);
-  const size_t need = moe::workspace_layout(B, L->E, L->top_e, L->d, nullptr, nullptr);
+  const int sI = dense ? 0 : L->I, sr = dense ? 0 : L->r;
+  const size_t need = moe::workspace_layout(B, L->E, L->top_e, L->d, sI, sr, nullptr, nullptr);
   REQUIRE(ws_bytes >= need, "workspace has %zu bytes, needs %zu", ws_bytes, need);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   moe::Workspace ws;
-  moe::workspace_layout(B, L->E, L->top_e, L->d, workspace, &ws);
+  moe::workspace_layout(B, L->E, L->top_e, L->d, sI, sr, workspace, &ws);
 
   moe::RouteArgs ra = {};
   ra.B = B;
@@ -114,7 +115,8 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   ra.dbg_w = dbg ? dbg->weights : nullptr;
   ra.quantize = !dense;
   cudaError_t e = cudaSuccess;
-  if (!moe::fused_routing(B)) {
+  const bool streamed = !dense && moe::use_streamed(B);
+  if (!moe::fused_routing(B) || streamed) {
     e = moe::launch_route(ra, s);
     if (e != cudaSuccess) return cuda_fail(e, "route launch");
   }
@@ -160,7 +162,7 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
     a.dbg_phase = reinterpret_cast<unsigned long long*>(dbg->phase_ns);
   }
   if (g_ev_before) cudaEventRecord(g_ev_before, s);
-  e = dense ? moe::launch_dense(a, s) : moe::launch_reader(a, s);
+  e = dense ? moe::launch_dense(a, s) : streamed ? moe::launch_stream(a, s) : moe::launch_reader(a, s);
   if (e != cudaSuccess) return cuda_fail(e, dense ? "dense expert launch" : "reader launch");
   if (g_ev_after) cudaEventRecord(g_ev_after, s);
   return MOE_OK;
@@ -176,12 +178,10 @@ moe_status moe::set_last_error(moe_status st, const char* msg) {
 extern "C" {
 
 size_t moe_reader_workspace_bytes(int B, int E, int top_e, int I, int d, int k, int c, int r) {
-  (void)I;
   (void)k;
   (void)c;
-  (void)r;
-  if (B < 1 || E < 1 || top_e < 1 || d < 1) return 0;
-  return moe::workspace_layout(B, E, top_e, d, nullptr, nullptr);
+  if (B < 1 || E < 1 || top_e < 1 || d < 1 || I < 0 || r < 0) return 0;
+  return moe::workspace_layout(B, E, top_e, d, I, r, nullptr, nullptr);
 }
 
 moe_status moe_reader_build_sketch(int E, int I, int d, const uint16_t* w_gate, const uint16_t* w_up,
@@ -279,7 +279,7 @@ moe_status moe_reader_check_error(void* workspace, void* stream) {
   cudaError_t e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
   moe::Workspace ws;
-  moe::workspace_layout(1, 1, 1, 16, workspace, &ws);  // err sits at offset 0 for every shape
+  moe::workspace_layout(1, 1, 1, 16, 0, 0, workspace, &ws);  // err sits at offset 0 for every shape
   uint32_t word = 0;
   e = cudaMemcpy(&word, ws.err, sizeof word, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "error word read");
@@ -292,6 +292,12 @@ moe_status moe_reader_check_error(void* workspace, void* stream) {
 moe_status moe_reader_set_cluster_size(int cs) {
   REQUIRE(cs == 0 || cs == 4 || cs == 8 || cs == 16, "cluster size %d: use 0 (automatic), 4, 8 or 16", cs);
   moe::set_forced_cluster_size(cs);
+  return MOE_OK;
+}
+
+moe_status moe_reader_set_path(int path) {
+  REQUIRE(path >= 0 && path <= 2, "path %d: use 0 (automatic), 1 (one cluster per expert) or 2 (streamed)", path);
+  moe::set_path(path);
   return MOE_OK;
 }
 

@@ -27,9 +27,31 @@ struct Workspace {
   float* ye;            // [B, top_e, d] per-expert outputs (fp32)
   unsigned* counters;   // [B, kMaxCluster] arrival counters of the combine
   int max_items;
+  // The streamed path (stream.cu).  Pairs (token, slot) are numbered in
+  // expert order, tokens ascending within an expert; W = ceil(I / 32).
+  int* qsum;            // [B] sum of each token's int8 activations (the code offset)
+  int* n_act;           // [1] experts chosen by at least one token this step
+  int* act_e;           // [E] those experts, ascending
+  int* act_off;         // [E + 1] first pair of each (act_off[n_act] = B * top_e)
+  int* pair_tok;        // [P] token of each pair
+  int* pair_slot;       // [P] routing slot of each pair
+  int* pair_ea;         // [P] active-expert index of each pair
+  unsigned* arrive;     // [2, E] arrival counters of the two selection kernels
+  float2* sa;           // [P, I] (sigma, ahat) of every channel
+  float* zpart;         // [P, ceil(I / 16), r] recovery-input partials of the screen blocks
+  uint32_t* candm;      // [P, W] candidate bit masks
+  float* apos;          // [P, I] exact a of each pair's candidates (by channel)
+  uint32_t* keptm;      // [P, W] kept bit masks
+  float* z;             // [P, r] recovery input of each pair
+  int* ulist;           // [E, I] candidate union of each active expert, ascending
+  int* n_u;             // [E]
+  int* dlist;           // [E, I] kept union of each active expert, ascending
+  int* n_d;             // [E]
+  float* coef;          // [P, I] each pair's coefficient of its expert's kept-union rows
 };
 
-size_t workspace_layout(int B, int E, int top_e, int d, void* base, Workspace* ws);
+// I and r size the streamed path's buffers (pass 0 for none).
+size_t workspace_layout(int B, int E, int top_e, int d, int I, int r, void* base, Workspace* ws);
 int max_work_items(int B, int E, int top_e, int group);
 
 struct RouteArgs {
@@ -83,6 +105,14 @@ struct ExpertArgs {
 // launch per step); larger steps use the route and select kernels first.
 bool fused_routing(int B);
 cudaError_t launch_reader(const ExpertArgs& a, cudaStream_t s);
+// The streamed reader: screen, top-c, exact candidates, top-k, down rows +
+// combine, each one kernel over every pair of the step (after launch_route).
+cudaError_t launch_stream(const ExpertArgs& a, cudaStream_t s);
+// Which reader runs a sparse step of B tokens: the one-cluster-per-expert
+// kernel (false) or the streamed kernels (true).  set_path forces one (1:
+// cluster, 2: streamed; 0: automatic, streamed above two tokens).
+bool use_streamed(int B);
+void set_path(int path);
 cudaError_t launch_dense(const ExpertArgs& a, cudaStream_t s);
 void set_forced_cluster_size(int cs);
 cudaError_t query_plan(const ExpertArgs& a, bool dense, int out[4]);

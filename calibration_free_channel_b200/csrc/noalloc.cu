@@ -66,7 +66,7 @@ extern "C" moe_status moe_reader_forward_noalloc(const moe_reader_layer* layer, 
     // step begins.  The kernels leave them zero, but the array keeps whatever
     // an earlier (possibly interrupted) call left, so clear them here.
     moe::Workspace ws;
-    moe::workspace_layout(1, 1, 1, 16, scratch, &ws);
+    moe::workspace_layout(1, 1, 1, 16, 0, 0, scratch, &ws);
     err = cudaMemsetAsync(ws.counters, 0, sizeof(unsigned) * moe::kMaxTokens * moe::kMaxCluster,
                           static_cast<cudaStream_t>(stream));
     if (err != cudaSuccess) return moe::set_last_error(MOE_ECUDA, "clearing the scratch counters failed");

@@ -42,11 +42,29 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a, int n_logit_blo
 #pragma unroll
     for (int t = 0; t < kRouteTokensPerCta; t++) acc[t] = 0.0;
     const uint4* wrow = reinterpret_cast<const uint4*>(a.w_router + (size_t)e * a.d);
-    for (int j = lane; j < a.d / 8; j += 32) {
-      const uint4 w = __ldg(wrow + j);
+    const int d8 = a.d / 8;
+    // the lane's router chunks 8 at a time, all loads in flight together
+#pragma unroll 1
+    for (int j0 = 0; j0 < d8; j0 += 256) {
+      uint4 w[8];
 #pragma unroll
-      for (int t = 0; t < kRouteTokensPerCta; t++)
-        if (t < nt) dfma8(w, __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)(t0 + t) * a.d) + j), acc[t]);
+      for (int u = 0; u < 8; u++) {
+        const int j = j0 + 32 * u + lane;
+        w[u] = j < d8 ? __ldg(wrow + j) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int t = 0; t < kRouteTokensPerCta; t++) {
+        if (t >= nt) break;
+        const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)(t0 + t) * a.d);
+        uint4 xv[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+          const int j = j0 + 32 * u + lane;
+          xv[u] = j < d8 ? __ldg(xr + j) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; u++) dfma8(w[u], xv[u], acc[t]);
+      }
     }
 #pragma unroll
     for (int t = 0; t < kRouteTokensPerCta; t++) {
@@ -85,6 +103,7 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a, int n_logit_blo
   float amax = 0.0f;
   for (int w = 0; w < (int)(blockDim.x >> 5); w++) amax = fmaxf(amax, red[w]);
   int8_t* q = a.ws.q + (size_t)b * d;
+  int qs = 0;
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
     int n = 0;
     if (amax > 0.0f) {
@@ -92,30 +111,45 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a, int n_logit_blo
       n = max(-127, min(127, n));
     }
     q[j] = (int8_t)n;
+    qs += n;
   }
-  if (threadIdx.x == 0) a.ws.cx[b] = amax > 0.0f ? __fdiv_rn(amax, __fmul_rn(127.0f, (float)d)) : 0.0f;
+  // the sum of the activations: the sketch dots' code offset (codes are T + 1)
+  __shared__ int redq[kWarps];
+  qs = warp_sum(qs);
+  if (lane == 0) redq[warp] = qs;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); w++) tot += redq[w];
+    a.ws.qsum[b] = tot;
+    a.ws.cx[b] = amax > 0.0f ? __fdiv_rn(amax, __fmul_rn(127.0f, (float)d)) : 0.0f;
+  }
 }
 
-// One CTA: top-e per token (ties to the lower id), softmax weights, the work
-// table (one item per (expert, group of <= kMaxGroup tokens)), and the
-// combine counters reset.
+// One CTA: top-e per token (ties to the lower id) and softmax weights, one
+// warp per token; then, one warp per expert, the token-ordered tables of the
+// step from ballots over the tokens: the work items of up to kMaxGroup tokens
+// (one-cluster and dense kernels), the active experts and the pairs in expert
+// order (streamed kernels).  Also zeroes the step's counters.
 __global__ void __launch_bounds__(512) select_kernel(RouteArgs a) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ int sm[];
-  int* cnt = sm;             // [E]
-  int* base = sm + a.E;      // [E]
-  int* cursor = base + a.E;  // [E]
+  const int E = a.E, top = a.top_e, B = a.B;
+  int* sids = sm;              // [B * top] chosen experts
+  int* cnt = sids + B * top;   // [E] tokens per expert
+  int* pbase = cnt + E;        // [E] first pair of each expert
+  int* ibase = pbase + E;      // [E] first work item of each expert
+  int* aidx = ibase + E;       // [E] active index (experts with tokens)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
-  const int E = a.E, top = a.top_e;
-  for (int b = warp; b < a.B; b += nwarp) {
+  for (int b = warp; b < B; b += nwarp) {
     const double* L = a.ws.logits + (size_t)b * E;
     uint32_t taken = 0;
-    double chosen[16];
-    int chosen_id[16];
     double lv[32];  // this lane's logits (E <= 1024), read once
 #pragma unroll
     for (int m = 0; m < 32; m++) lv[m] = lane + 32 * m < E ? L[lane + 32 * m] : -INFINITY;
+    double l0 = 0.0, my_l = 0.0;
+    int my_id = 0;
     for (int s = 0; s < top; s++) {
       double bv = -INFINITY;
       int bi = 0x7fffffff;
@@ -138,54 +172,109 @@ __global__ void __launch_bounds__(512) select_kernel(RouteArgs a) {
         }
       }
       if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      chosen[s] = bv;
-      chosen_id[s] = bi;
-    }
-    if (lane == 0) {
-      double den = 0.0;
-      for (int s = 0; s < top; s++) den += exp(chosen[s] - chosen[0]);
-      for (int s = 0; s < top; s++) {
-        const float w = (float)(exp(chosen[s] - chosen[0]) / den);
-        a.ws.ids[b * top + s] = chosen_id[s];
-        a.ws.wts[b * top + s] = w;
-        if (a.dbg_ids) a.dbg_ids[b * top + s] = chosen_id[s];
-        if (a.dbg_w) a.dbg_w[b * top + s] = w;
+      if (s == 0) l0 = bv;
+      if (lane == s) {
+        my_l = bv;
+        my_id = bi;
       }
     }
-  }
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    cnt[e] = 0;
-    cursor[e] = 0;
-  }
-  for (int i = threadIdx.x; i < a.B * kMaxCluster; i += blockDim.x) a.ws.counters[i] = 0u;
-  __syncthreads();
-  for (int i = threadIdx.x; i < a.B * top; i += blockDim.x) atomicAdd(&cnt[a.ws.ids[i]], 1);
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int e = 0; e < E; e++) {
-      base[e] = run;
-      run += (cnt[e] + kMaxGroup - 1) / kMaxGroup;
+    // softmax over the chosen logits: fp32 exponentials of the fp64
+    // differences to the largest (the weights only scale outputs)
+    const float ex = lane < top ? __expf((float)(my_l - l0)) : 0.0f;
+    double den = (double)ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (lane < top) {
+      const float w = (float)((double)ex / den);
+      a.ws.ids[b * top + lane] = my_id;
+      a.ws.wts[b * top + lane] = w;
+      sids[b * top + lane] = my_id;
+      if (a.dbg_ids) a.dbg_ids[b * top + lane] = my_id;
+      if (a.dbg_w) a.dbg_w[b * top + lane] = w;
     }
-    *a.ws.n_items = run;
+  }
+  for (int i = threadIdx.x; i < B * kMaxCluster; i += blockDim.x) a.ws.counters[i] = 0u;
+  for (int i = threadIdx.x; i < 2 * E; i += blockDim.x) a.ws.arrive[i] = 0u;
+  __syncthreads();
+  // tokens per expert
+  for (int e = warp; e < E; e += nwarp) {
+    int c = 0;
+    for (int t0 = 0; t0 < B; t0 += 32) {
+      const int t = t0 + lane;
+      bool on = false;
+      if (t < B)
+        for (int s = 0; s < top; s++) on |= sids[t * top + s] == e;
+      c += __popc(__ballot_sync(0xffffffffu, on));
+    }
+    if (lane == 0) cnt[e] = c;
   }
   __syncthreads();
-  // Tokens enter their expert's items in increasing token order.
-  for (int t = 0; t < a.B; t++) {
-    if (threadIdx.x < top) {
-      const int e = a.ws.ids[t * top + threadIdx.x];
-      const int pos = cursor[e]++;
-      const int item = base[e] + pos / kMaxGroup, g = pos % kMaxGroup;
-      if (item < a.ws.max_items) {
-        a.ws.item_tok[item * kMaxGroup + g] = t;
-        a.ws.item_slot[item * kMaxGroup + g] = threadIdx.x;
-        if (g == 0) {
-          a.ws.item_e[item] = e;
-          a.ws.item_n[item] = min(kMaxGroup, cnt[e] - pos);
+  // exclusive prefixes over the experts: pairs, work items, active experts
+  if (warp == 0) {
+    int rp = 0, ri = 0, ra = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int c = e < E ? cnt[e] : 0, it = (c + kMaxGroup - 1) / kMaxGroup, ac = c > 0;
+      int ip = c, ii = it, ia = ac;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int vp = __shfl_up_sync(0xffffffffu, ip, o), vi = __shfl_up_sync(0xffffffffu, ii, o),
+                  va = __shfl_up_sync(0xffffffffu, ia, o);
+        if (lane >= o) {
+          ip += vp;
+          ii += vi;
+          ia += va;
         }
       }
+      if (e < E) {
+        pbase[e] = rp + ip - c;
+        ibase[e] = ri + ii - it;
+        aidx[e] = ra + ia - ac;
+        if (ac) {
+          a.ws.act_e[ra + ia - 1] = e;
+          a.ws.act_off[ra + ia - 1] = rp + ip - c;
+        }
+      }
+      rp += __shfl_sync(0xffffffffu, ip, 31);
+      ri += __shfl_sync(0xffffffffu, ii, 31);
+      ra += __shfl_sync(0xffffffffu, ia, 31);
     }
-    __syncthreads();
+    if (lane == 0) {
+      *a.ws.n_items = ri;
+      *a.ws.n_act = ra;
+      a.ws.act_off[ra] = rp;
+    }
+  }
+  __syncthreads();
+  // each expert's pairs and work items, tokens ascending
+  for (int e = warp; e < E; e += nwarp) {
+    if (cnt[e] == 0) continue;
+    int run = 0;
+    for (int t0 = 0; t0 < B; t0 += 32) {
+      const int t = t0 + lane;
+      int slot = -1;
+      if (t < B)
+        for (int s = 0; s < top; s++)
+          if (sids[t * top + s] == e) slot = s;
+      const unsigned bal = __ballot_sync(0xffffffffu, slot >= 0);
+      if (slot >= 0) {
+        const int pos = run + __popc(bal & ((1u << lane) - 1u));
+        const int pr = pbase[e] + pos;
+        a.ws.pair_tok[pr] = t;
+        a.ws.pair_slot[pr] = slot;
+        a.ws.pair_ea[pr] = aidx[e];
+        const int item = ibase[e] + pos / kMaxGroup, g = pos % kMaxGroup;
+        if (item < a.ws.max_items) {
+          a.ws.item_tok[item * kMaxGroup + g] = t;
+          a.ws.item_slot[item * kMaxGroup + g] = slot;
+          if (g == 0) {
+            a.ws.item_e[item] = e;
+            a.ws.item_n[item] = min(kMaxGroup, cnt[e] - pos);
+          }
+        }
+      }
+      run += __popc(bal);
+    }
   }
 }
 
@@ -199,7 +288,7 @@ int max_work_items(int B, int E, int top_e, int group) {
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-size_t workspace_layout(int B, int E, int top_e, int d, void* base, Workspace* ws) {
+size_t workspace_layout(int B, int E, int top_e, int d, int I, int r, void* base, Workspace* ws) {
   const int mi = max_work_items(B, E, top_e, kMaxGroup);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -216,6 +305,18 @@ size_t workspace_layout(int B, int E, int top_e, int d, void* base, Workspace* w
   const size_t o_ie = take(sizeof(int) * mi), o_in = take(sizeof(int) * mi);
   const size_t o_it = take(sizeof(int) * mi * kMaxGroup), o_is = take(sizeof(int) * mi * kMaxGroup);
   const size_t o_ye = take(sizeof(float) * B * top_e * (size_t)d);
+  // the streamed path
+  const size_t P = (size_t)B * top_e, W = (size_t)(I + 31) / 32, nbs = (size_t)(I + 15) / 16;
+  const bool st = I > 0;
+  const size_t o_qs = take(sizeof(int) * B), o_na = take(16), o_ae = take(sizeof(int) * E),
+               o_ao = take(sizeof(int) * (E + 1)), o_pt = take(sizeof(int) * P), o_ps = take(sizeof(int) * P),
+               o_pe = take(sizeof(int) * P), o_ar = take(sizeof(unsigned) * 2 * E);
+  const size_t o_sa = st ? take(sizeof(float2) * P * I) : 0, o_zp = st ? take(sizeof(float) * P * nbs * r) : 0,
+               o_cm = st ? take(sizeof(uint32_t) * P * W) : 0, o_ap = st ? take(sizeof(float) * P * I) : 0,
+               o_km = st ? take(sizeof(uint32_t) * P * W) : 0, o_z = st ? take(sizeof(float) * P * r) : 0,
+               o_ul = st ? take(sizeof(int) * E * (size_t)I) : 0, o_nu = st ? take(sizeof(int) * E) : 0,
+               o_dl = st ? take(sizeof(int) * E * (size_t)I) : 0, o_nd = st ? take(sizeof(int) * E) : 0,
+               o_co = st ? take(sizeof(float) * P * I) : 0;
   if (ws && base) {
     char* p = static_cast<char*>(base);
     ws->err = reinterpret_cast<uint32_t*>(p + o_err);
@@ -232,6 +333,25 @@ size_t workspace_layout(int B, int E, int top_e, int d, void* base, Workspace* w
     ws->ye = reinterpret_cast<float*>(p + o_ye);
     ws->counters = reinterpret_cast<unsigned*>(p + o_ct);
     ws->max_items = mi;
+    ws->qsum = reinterpret_cast<int*>(p + o_qs);
+    ws->n_act = reinterpret_cast<int*>(p + o_na);
+    ws->act_e = reinterpret_cast<int*>(p + o_ae);
+    ws->act_off = reinterpret_cast<int*>(p + o_ao);
+    ws->pair_tok = reinterpret_cast<int*>(p + o_pt);
+    ws->pair_slot = reinterpret_cast<int*>(p + o_ps);
+    ws->pair_ea = reinterpret_cast<int*>(p + o_pe);
+    ws->arrive = reinterpret_cast<unsigned*>(p + o_ar);
+    ws->sa = st ? reinterpret_cast<float2*>(p + o_sa) : nullptr;
+    ws->zpart = st ? reinterpret_cast<float*>(p + o_zp) : nullptr;
+    ws->candm = st ? reinterpret_cast<uint32_t*>(p + o_cm) : nullptr;
+    ws->apos = st ? reinterpret_cast<float*>(p + o_ap) : nullptr;
+    ws->keptm = st ? reinterpret_cast<uint32_t*>(p + o_km) : nullptr;
+    ws->z = st ? reinterpret_cast<float*>(p + o_z) : nullptr;
+    ws->ulist = st ? reinterpret_cast<int*>(p + o_ul) : nullptr;
+    ws->n_u = st ? reinterpret_cast<int*>(p + o_nu) : nullptr;
+    ws->dlist = st ? reinterpret_cast<int*>(p + o_dl) : nullptr;
+    ws->n_d = st ? reinterpret_cast<int*>(p + o_nd) : nullptr;
+    ws->coef = st ? reinterpret_cast<float*>(p + o_co) : nullptr;
   }
   return off;
 }
@@ -249,7 +369,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1);
   cfg.blockDim = dim3(512);
-  cfg.dynamicSmemBytes = sizeof(int) * 3 * a.E;
+  cfg.dynamicSmemBytes = sizeof(int) * (4 * a.E + a.B * a.top_e);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -1,0 +1,872 @@
+// stream.cu -- the streamed reader: the steps of the sparse reader of
+// "KAIST: MoE Decoding Needs No Calibration Data" (section "A reader that
+// needs no data at all": screen with the rotated ternary sketch, top-c
+// candidates, exact BF16 gate/up of the candidates, top-k by |a|, the kept
+// down rows plus the low-rank recovery of the skipped ones), each one kernel
+// over every (token, expert) pair of the step, on all SMs.
+//
+// Stage kernels, after the route and select kernels (route.cu):
+//   screen_kernel     sketch dots of every (pair, channel): sigma, ahat, and
+//                     the recovery-input partial of each 32-channel block
+//   select_c_kernel   one pair per CTA: top-c by sigma; the expert's last pair
+//                     forms the candidate union (rows of the next stage)
+//   exact_kernel      16 union rows of one expert per unit: g, u of every
+//                     token of the expert, a = silu(g) u for its candidates
+//   select_k_kernel   one pair per CTA: top-k by |a| over its candidates, the
+//                     recovery input z; the expert's last pair forms the kept
+//                     union and the per-pair row coefficients
+//   down_kernel       one (expert, column slice) per unit: kept down rows,
+//                     V z, and the combine over the top-e slots by the last
+//                     arriving slot of each (token, slice)
+// Each kernel is launched with programmatic dependent launch and waits on
+// its predecessor before reading its outputs; weights are read with
+// non-allocating loads, data written by earlier kernels of the chain through
+// L2 (ld.global.cg).  Sets and rounding points are those of the one-cluster
+// reader (reader.cu), so both paths give the same candidate and kept sets.
+#include "common.cuh"
+#include "kernels.h"
+#include "select.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr unsigned kFullMask = 0xffffffffu;
+
+constexpr int kSThreads = 256;  // screen: 8 warps, 4 / NVL channels per warp
+constexpr int kSTG = 2;         // screen: tokens per register group
+constexpr int kSelT = sel::kSelThreads;
+constexpr int kDThreads = 256;  // down rows
+constexpr int kDTG = 4;         // down: tokens per register group
+constexpr int kDRows = 256;     // down: kept-union rows staged per chunk
+constexpr int kMaxI = 2048;
+constexpr int kMaxAct = 1024;   // active experts (E <= 1024)
+
+int g_path = 0;
+
+// 16-byte load of weights that are read once per step: no L1 allocation.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint4 ld_cg4(const void* p) { return __ldcg(reinterpret_cast<const uint4*>(p)); }
+
+// Counts one arrival at ctr (release of everything this thread ordered
+// before, acquire of the earlier arrivals); true for the last of `total`.
+__device__ __forceinline__ bool arrive_last(unsigned* ctr, unsigned total) {
+  unsigned old;
+  asm volatile("fence.acq_rel.gpu;\n\tatom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+               : "=r"(old)
+               : "l"(ctr)
+               : "memory");
+  return old == total - 1u;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(uint4 w, float (&f)[8]) {
+  f[0] = bf16lo(w.x);
+  f[1] = bf16hi(w.x);
+  f[2] = bf16lo(w.y);
+  f[3] = bf16hi(w.y);
+  f[4] = bf16lo(w.z);
+  f[5] = bf16hi(w.z);
+  f[6] = bf16lo(w.w);
+  f[7] = bf16hi(w.w);
+}
+
+// Screen-block geometry: channels per warp and per block for NVL 16-byte
+// sketch vectors per lane and row (NVL = 1 for d <= 2048, 2 for d = 4096);
+// a block's sketch rows are 16 KB per matrix either way.
+template <int NVL>
+struct ScreenGeom {
+  static constexpr int kPerWarp = 4 / NVL;
+  static constexpr int kChannels = 8 * kPerWarp;
+};
+constexpr int kSStageBytes = 2 * 16384;  // gate + up rows of one block
+
+// ------------------------------------------------------------------ screen
+// Unit = (active expert, block of ScreenGeom::kChannels channels).  The
+// block's gate and up sketch rows are contiguous: one thread copies them into
+// shared memory with two bulk copies, the next unit's copies in flight while
+// this one is computed (two stages).  A warp takes the expert's tokens kSTG
+// at a time, their activations at its lanes' sketch vectors in registers,
+// and its channels one pass at a time; the lanes of one channel (LG =
+// min(32, d / 64) of them) reduce its dots with shuffles.  Scores follow the
+// one-cluster reader: ghat = ((float)G alpha_g) c_x, uhat likewise,
+// ahat = silu_r(ghat) uhat, sigma = |ahat|, with G, U the exact integer dots
+// less the code offset sum(q).
+template <int NVL>
+__device__ __forceinline__ void screen_issue(const ExpertArgs& a, int u, int nblk, char* dst, uint64_t* bar) {
+  using Geo = ScreenGeom<NVL>;
+  const int ea = u / nblk, blk = u - ea * nblk;
+  const int e = __ldcg(a.ws.act_e + ea);
+  const int i0 = blk * Geo::kChannels, ncw = min(Geo::kChannels, a.I - i0);
+  const size_t row = (size_t)a.d / 4;  // bytes of one sketch row
+  const uint32_t bytes = (uint32_t)(ncw * row);
+  mbar_expect_tx(bar, 2 * bytes);
+  bulk_g2s(dst, reinterpret_cast<const char*>(a.sk_gate) + ((size_t)e * a.I + i0) * row, bytes, bar);
+  bulk_g2s(dst + kSStageBytes / 2, reinterpret_cast<const char*>(a.sk_up) + ((size_t)e * a.I + i0) * row, bytes, bar);
+}
+
+template <int NVL>
+__global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  using Geo = ScreenGeom<NVL>;
+  extern __shared__ __align__(128) char sk_stage[];  // [2][gate 16 KB | up 16 KB]
+  __shared__ float sah[kSTG][Geo::kChannels];
+  __shared__ float salg[Geo::kChannels], salu[Geo::kChannels];
+  __shared__ __align__(8) uint64_t bars[2];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tid = threadIdx.x;
+  const int I = a.I, d = a.d, r = a.r;
+  const int nv = d >> 6;                          // sketch vectors per row
+  // a pass covers SUB channels (LG lanes each); small d can leave lanes idle
+  const int LG = nv < 32 ? nv : 32, SUB = 32 / LG, PP = (Geo::kPerWarp + SUB - 1) / SUB;
+  const int lv = lane & (LG - 1), sub = lane / LG;
+  const int nblk = (I + Geo::kChannels - 1) / Geo::kChannels;
+  const int zstride = (I + 15) / 16;              // zpart blocks per pair (the finest geometry)
+  const int n_act = __ldcg(a.ws.n_act);
+  const int units = n_act * nblk;
+  uint32_t* err = a.ws.err;
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0 && (int)blockIdx.x < units) screen_issue<NVL>(a, blockIdx.x, nblk, sk_stage, &bars[0]);
+  int it = 0;
+#pragma unroll 1
+  for (int u = blockIdx.x; u < units; u += gridDim.x, it++) {
+    const int st = it & 1;
+    if (tid == 0 && u + (int)gridDim.x < units)
+      screen_issue<NVL>(a, u + gridDim.x, nblk, sk_stage + (st ^ 1) * kSStageBytes, &bars[st ^ 1]);
+    const int ea = u / nblk, blk = u - ea * nblk;
+    const int e = __ldcg(a.ws.act_e + ea), p0 = __ldcg(a.ws.act_off + ea);
+    const int m = __ldcg(a.ws.act_off + ea + 1) - p0;
+    const int i0 = blk * Geo::kChannels, ncw = min(Geo::kChannels, I - i0);
+    if (tid < ncw) {
+      salg[tid] = __ldg(a.alpha_gate + (size_t)e * I + i0 + tid);
+      salu[tid] = __ldg(a.alpha_up + (size_t)e * I + i0 + tid);
+    }
+    __syncthreads();
+    const uint4* skg = reinterpret_cast<const uint4*>(sk_stage + st * kSStageBytes);
+    const uint4* sku = skg + kSStageBytes / 32;
+    mbar_wait_bounded(&bars[st], (it >> 1) & 1, err);
+#pragma unroll 1
+    for (int tg = 0; tg < m; tg += kSTG) {
+      const int ng = min(kSTG, m - tg);
+      int tk[kSTG], qs[kSTG];
+      float cx[kSTG];
+#pragma unroll
+      for (int t = 0; t < kSTG; t++) {
+        tk[t] = __ldcg(a.ws.pair_tok + p0 + tg + min(t, ng - 1));
+        qs[t] = __ldcg(a.ws.qsum + tk[t]);
+        cx[t] = __ldcg(a.ws.cx + tk[t]);
+      }
+      // the tokens' activations at this lane's sketch vectors
+      uint4 qv[kSTG][NVL][4];
+#pragma unroll
+      for (int t = 0; t < kSTG; t++)
+#pragma unroll
+        for (int k = 0; k < NVL; k++) {
+          const uint4* qp = reinterpret_cast<const uint4*>(a.ws.q + (size_t)tk[t] * d) + 4 * (lv + LG * k);
+#pragma unroll
+          for (int w = 0; w < 4; w++) qv[t][k][w] = ld_cg4(qp + w);
+        }
+#pragma unroll 1
+      for (int pp = 0; pp < PP; pp++) {
+        const int lc = warp * Geo::kPerWarp + pp * SUB + sub;
+        const bool ok = pp * SUB + sub < Geo::kPerWarp && lc < ncw;
+        int ga[kSTG][4], ua[kSTG][4];
+#pragma unroll
+        for (int t = 0; t < kSTG; t++)
+#pragma unroll
+          for (int w = 0; w < 4; w++) ga[t][w] = ua[t][w] = 0;
+#pragma unroll
+        for (int k = 0; k < NVL; k++) {
+          const int o = lc * nv + lv + LG * k;
+          const uint4 g4 = ok ? skg[o] : make_uint4(0u, 0u, 0u, 0u);
+          const uint4 u4 = ok ? sku[o] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int t = 0; t < kSTG; t++) {
+            if (t >= ng) break;
+            code_dot16(g4.x, qv[t][k][0], ga[t]);
+            code_dot16(g4.y, qv[t][k][1], ga[t]);
+            code_dot16(g4.z, qv[t][k][2], ga[t]);
+            code_dot16(g4.w, qv[t][k][3], ga[t]);
+            code_dot16(u4.x, qv[t][k][0], ua[t]);
+            code_dot16(u4.y, qv[t][k][1], ua[t]);
+            code_dot16(u4.z, qv[t][k][2], ua[t]);
+            code_dot16(u4.w, qv[t][k][3], ua[t]);
+          }
+        }
+        // channel sums; the finishing lane of token t holds (g, u)
+        int g, uu, t;
+        if (LG == 32) {
+          // reduce-scatter of (G0, U0, G1, U1) over the warp: lane 16 t
+          // ends with G_t, lane 16 t + 8 with U_t
+          const int v0 = code_dot_total(ga[0]), v1 = code_dot_total(ua[0]);
+          const int v2 = code_dot_total(ga[1]), v3 = code_dot_total(ua[1]);
+          const bool h16 = lane & 16, h8 = lane & 8;
+          const int a0 = (h16 ? v2 : v0) + __shfl_xor_sync(kFullMask, h16 ? v0 : v2, 16);
+          const int a1 = (h16 ? v3 : v1) + __shfl_xor_sync(kFullMask, h16 ? v1 : v3, 16);
+          int b0 = (h8 ? a1 : a0) + __shfl_xor_sync(kFullMask, h8 ? a0 : a1, 8);
+          b0 += __shfl_xor_sync(kFullMask, b0, 4);
+          b0 += __shfl_xor_sync(kFullMask, b0, 2);
+          b0 += __shfl_xor_sync(kFullMask, b0, 1);
+          g = b0;
+          uu = __shfl_xor_sync(kFullMask, b0, 8);
+          t = (lane & 15) == 0 ? lane >> 4 : kSTG;
+        } else {
+          int G[kSTG], U[kSTG];
+#pragma unroll
+          for (int tt = 0; tt < kSTG; tt++) {
+            G[tt] = code_dot_total(ga[tt]);
+            U[tt] = code_dot_total(ua[tt]);
+          }
+          for (int o = LG >> 1; o > 0; o >>= 1)
+#pragma unroll
+            for (int tt = 0; tt < kSTG; tt++) {
+              G[tt] += __shfl_xor_sync(kFullMask, G[tt], o);
+              U[tt] += __shfl_xor_sync(kFullMask, U[tt], o);
+            }
+          g = G[0];
+          uu = U[0];
+#pragma unroll
+          for (int tt = 1; tt < kSTG; tt++)
+            if (lv == tt) {
+              g = G[tt];
+              uu = U[tt];
+            }
+          t = lv;
+        }
+        if (ok && t < ng) {
+          int tok = tk[0], qst = qs[0];
+          float cxt = cx[0];
+#pragma unroll
+          for (int tt = 1; tt < kSTG; tt++)
+            if (t == tt) {
+              tok = tk[tt];
+              qst = qs[tt];
+              cxt = cx[tt];
+            }
+          const int i = i0 + lc, pr = p0 + tg + t;
+          const int g2 = g - qst, u2 = uu - qst;
+          const float gh = __fmul_rn(__fmul_rn((float)g2, salg[lc]), cxt);
+          const float uh = __fmul_rn(__fmul_rn((float)u2, salu[lc]), cxt);
+          const float ah = __fmul_rn(silu_r(gh), uh);
+          a.ws.sa[(size_t)pr * I + i] = make_float2(fabsf(ah), ah);
+          sah[t][lc] = ah;
+          if (a.dbg_G || a.dbg_U || a.dbg_sigma) {
+            const size_t off = ((size_t)tok * a.top_e + __ldcg(a.ws.pair_slot + pr)) * I + i;
+            if (a.dbg_G) a.dbg_G[off] = g2;
+            if (a.dbg_U) a.dbg_U[off] = u2;
+            if (a.dbg_sigma) a.dbg_sigma[off] = fabsf(ah);
+          }
+        }
+      }
+      // recovery-input partial of the block: sum over its channels of ahat_i Ubar_i
+      if (r > 0) {
+        __syncthreads();
+        for (int o = tid; o < ng * r; o += kSThreads) {
+          const int t = o / r, p = o - t * r;
+          const uint16_t* ub = a.u_sigma + ((size_t)e * I + i0) * r + p;
+          float z0 = 0.0f, z1 = 0.0f;
+          int lc = 0;
+          for (; lc + 2 <= ncw; lc += 2) {
+            z0 = fmaf(sah[t][lc], bf16f(ub[(size_t)lc * r]), z0);
+            z1 = fmaf(sah[t][lc + 1], bf16f(ub[(size_t)(lc + 1) * r]), z1);
+          }
+          if (lc < ncw) z0 = fmaf(sah[t][lc], bf16f(ub[(size_t)lc * r]), z0);
+          a.ws.zpart[((size_t)(p0 + tg + t) * zstride + blk) * r + p] = z0 + z1;
+        }
+      }
+      __syncthreads();
+    }
+    // every warp is done with this stage before the copy two units on reuses it
+    __syncthreads();
+    if (tid == 0) fence_proxy_async();
+  }
+}
+
+// Shared memory of the selection kernels (one pair per CTA, 512 threads).
+struct SelSmem {
+  __align__(16) int hist[2 * 2048];
+  __align__(16) uint32_t keys[kMaxI];
+  __align__(16) int list[kMaxI];
+  __align__(16) int misc[128];
+  __align__(16) int scratch[128];
+  __align__(16) uint32_t mk[64];
+  __align__(16) uint32_t kw[64];
+  __align__(16) float zr[kSelT];
+};
+
+// -------------------------------------------------------------- top-c
+// One pair per CTA: the c channels with the largest sigma (ties to the lower
+// channel).  The last pair of an expert to finish ORs its expert's candidate
+// masks into the union list the exact stage reads.
+__global__ void __launch_bounds__(kSelT) select_c_kernel(ExpertArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ SelSmem sm;
+  const int tid = threadIdx.x;
+  const int I = a.I, W = (I + 31) >> 5, P = a.B * a.top_e;
+#pragma unroll 1
+  for (int p = blockIdx.x; p < P; p += gridDim.x) {
+    const float* sp = reinterpret_cast<const float*>(a.ws.sa + (size_t)p * I);
+    for (int i = tid; i < I; i += kSelT) sm.keys[i] = __float_as_uint(__ldcg(sp + 2 * i));  // sigma >= 0
+    __syncthreads();
+    sel::block_select_top(sm.keys, 1, I, a.c, sm.hist, sm.misc, sm.mk);
+    for (int w = tid; w < W; w += kSelT) a.ws.candm[(size_t)p * W + w] = sm.mk[w];
+    if (a.dbg_cand) {
+      const int tok = __ldcg(a.ws.pair_tok + p), slot = __ldcg(a.ws.pair_slot + p);
+      sel::block_mask_to_list(sm.mk, nullptr, I, a.dbg_cand + ((size_t)tok * a.top_e + slot) * a.c, &sm.misc[1],
+                              sm.scratch);
+    }
+    const int ea = __ldcg(a.ws.pair_ea + p);
+    const int p0 = __ldcg(a.ws.act_off + ea), m = __ldcg(a.ws.act_off + ea + 1) - p0;
+    __syncthreads();  // the CTA's mask stores precede the release below
+    if (tid == 0) sm.misc[0] = arrive_last(a.ws.arrive + ea, (unsigned)m);
+    __syncthreads();
+    if (sm.misc[0]) {
+      for (int w = tid; w < W; w += kSelT) {
+        uint32_t o = 0u;
+        for (int q = 0; q < m; q++) o |= __ldcg(a.ws.candm + (size_t)(p0 + q) * W + w);
+        sm.mk[w] = o;
+      }
+      __syncthreads();
+      sel::block_mask_to_list(sm.mk, nullptr, I, a.ws.ulist + (size_t)ea * I, a.ws.n_u + ea, sm.scratch);
+    }
+    __syncthreads();
+  }
+}
+
+// -------------------------------------------------------------- top-k
+// One pair per CTA: the k candidates with the largest |a| (ties to the lower
+// channel), then the recovery input z = sum over the block partials of
+// ahat Ubar minus the part of the channels the down rows cover: -ahat_i Ubar_i
+// for kept channels and, with the exact recovery input, -(ahat_i - a_i) Ubar_i
+// for dropped candidates.  The last pair of an expert forms the kept union
+// and the coefficient of every pair on each of its rows.
+__global__ void __launch_bounds__(kSelT) select_k_kernel(ExpertArgs a, int nblk) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ SelSmem sm;
+  const int tid = threadIdx.x;
+  const int I = a.I, W = (I + 31) >> 5, P = a.B * a.top_e, r = a.r;
+  const int zstride = (I + 15) / 16;
+  const bool rec_exact = a.recovery_input == 1;
+#pragma unroll 1
+  for (int p = blockIdx.x; p < P; p += gridDim.x) {
+    const int ea = __ldcg(a.ws.pair_ea + p);
+    const int e = __ldcg(a.ws.act_e + ea);
+    for (int w = tid; w < W; w += kSelT) {
+      sm.mk[w] = __ldcg(a.ws.candm + (size_t)p * W + w);
+      sm.kw[w] = 0u;
+    }
+    __syncthreads();
+    // candidate channels, ascending, and their keys |a|
+    sel::block_mask_to_list(sm.mk, nullptr, I, sm.list, &sm.misc[1], sm.scratch);
+    const int nc = sm.misc[1];
+    const float* ap = a.ws.apos + (size_t)p * I;
+    for (int j = tid; j < nc; j += kSelT) sm.keys[j] = __float_as_uint(fabsf(__ldcg(ap + sm.list[j])));
+    __syncthreads();
+    sel::block_select_top(sm.keys, 1, nc, a.k, sm.hist, sm.misc, sm.mk);  // mk: kept positions
+    for (int j = tid; j < nc; j += kSelT)
+      if ((sm.mk[j >> 5] >> (j & 31)) & 1u) atomicOr(&sm.kw[sm.list[j] >> 5], 1u << (sm.list[j] & 31));
+    __syncthreads();
+    for (int w = tid; w < W; w += kSelT) a.ws.keptm[(size_t)p * W + w] = sm.kw[w];
+    if (a.dbg_kept) {
+      // kept channels ascending: the kept positions in order
+      int* klist = reinterpret_cast<int*>(sm.keys);
+      sel::block_mask_to_list(sm.mk, nullptr, nc, klist, &sm.misc[2], sm.scratch);
+      const int tok = __ldcg(a.ws.pair_tok + p), slot = __ldcg(a.ws.pair_slot + p);
+      const size_t off = ((size_t)tok * a.top_e + slot) * a.k;
+      for (int t = tid; t < a.k && t < sm.misc[2]; t += kSelT) {
+        const int i = sm.list[klist[t]];
+        a.dbg_kept[off + t] = i;
+        if (a.dbg_a_kept) a.dbg_a_kept[off + t] = __ldcg(ap + i);
+      }
+      __syncthreads();
+    }
+    if (r > 0) {
+      // thread (part, p): candidate positions part, part + parts, ...
+      const int parts = kSelT / r, part = tid / r, pz = tid - part * r;
+      float acc = 0.0f;
+      if (part < parts) {
+        const float* sap = reinterpret_cast<const float*>(a.ws.sa + (size_t)p * I);
+        for (int j = part; j < nc; j += parts) {
+          const bool kept = (sm.mk[j >> 5] >> (j & 31)) & 1u;
+          if (!kept && !rec_exact) continue;
+          const int i = sm.list[j];
+          const float ah = __ldcg(sap + 2 * i + 1);
+          const float co = kept ? ah : __fsub_rn(ah, __ldcg(ap + i));
+          acc = fmaf(co, bf16f(a.u_sigma[((size_t)e * I + i) * r + pz]), acc);
+        }
+      }
+      sm.zr[tid] = acc;
+      __syncthreads();
+      if (tid < r) {
+        float s0 = 0.0f, s1 = 0.0f;
+        for (int q = 0; q < parts; q++) s0 += sm.zr[q * r + tid];
+        const float* zp = a.ws.zpart + (size_t)p * zstride * r + tid;
+        for (int b = 0; b < nblk; b++) s1 += __ldcg(zp + (size_t)b * r);
+        a.ws.z[(size_t)p * r + tid] = s1 - s0;
+      }
+    }
+    // the expert's last pair: kept union and row coefficients
+    const int p0 = __ldcg(a.ws.act_off + ea), m = __ldcg(a.ws.act_off + ea + 1) - p0;
+    __syncthreads();
+    if (tid == 0) sm.misc[0] = arrive_last(a.ws.arrive + a.E + ea, (unsigned)m);
+    __syncthreads();
+    if (sm.misc[0]) {
+      for (int w = tid; w < W; w += kSelT) {
+        uint32_t o = 0u;
+        for (int q = 0; q < m; q++) o |= __ldcg(a.ws.keptm + (size_t)(p0 + q) * W + w);
+        sm.kw[w] = o;
+      }
+      __syncthreads();
+      int* dl = a.ws.dlist + (size_t)ea * I;
+      sel::block_mask_to_list(sm.kw, nullptr, I, sm.list, &sm.misc[3], sm.scratch);
+      const int nd = sm.misc[3];
+      for (int u = tid; u < nd; u += kSelT) dl[u] = sm.list[u];
+      if (tid == 0) a.ws.n_d[ea] = nd;
+      for (int o = tid; o < m * nd; o += kSelT) {
+        const int q = o / nd, u = o - q * nd, i = sm.list[u];
+        const bool kept = (__ldcg(a.ws.keptm + (size_t)(p0 + q) * W + (i >> 5)) >> (i & 31)) & 1u;
+        a.ws.coef[(size_t)(p0 + q) * I + u] = kept ? __ldcg(a.ws.apos + (size_t)(p0 + q) * I + i) : 0.0f;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// Butterfly reduce-scatter of 8 per-lane values over the warp (9 shuffles):
+// afterwards lane L holds the warp sum of value 4 b4 + 2 b3 + b2, where bN is
+// bit N of L.
+__device__ __forceinline__ float reduce_scatter8(float (&v)[8]) {
+  const int lane = threadIdx.x & 31;
+  const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
+#pragma unroll
+  for (int j = 0; j < 4; j++) {
+    const float send = h16 ? v[j] : v[j + 4], keep = h16 ? v[j + 4] : v[j];
+    v[j] = keep + __shfl_xor_sync(kFullMask, send, 16);
+  }
+#pragma unroll
+  for (int j = 0; j < 2; j++) {
+    const float send = h8 ? v[j] : v[j + 2], keep = h8 ? v[j + 2] : v[j];
+    v[j] = keep + __shfl_xor_sync(kFullMask, send, 8);
+  }
+  {
+    const float send = h4 ? v[0] : v[1], keep = h4 ? v[1] : v[0];
+    v[0] = keep + __shfl_xor_sync(kFullMask, send, 4);
+  }
+  float s = v[0];
+  s += __shfl_xor_sync(kFullMask, s, 2);
+  s += __shfl_xor_sync(kFullMask, s, 1);
+  return s;
+}
+
+// bf16 m16n8k16 tensor-core product, fp32 accumulate: c += A B.
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Expert of unit u: cu holds the exclusive prefix of units per active expert.
+__device__ __forceinline__ int unit_expert(const int* cu, int n_act, int u) {
+  int lo = 0, hi = n_act;  // cu[lo] <= u < cu[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (cu[mid] <= u) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// ------------------------------------------------------- exact candidates
+// g = W_gate[e] x and u = W_up[e] x for kXRows rows of the expert's
+// candidate union and up to 16 of its tokens per pass, on the tensor cores:
+// D[token][row] += X[token][k] W[row][k] with tokens as M (16, zero-padded),
+// rows as N (one 8-row tile per warp) and d as K, bf16 products summed in
+// fp32.  The order of the K sum is free, so each thread loads 16 contiguous
+// bytes of its row (and of its token from shared memory) and uses them as the
+// fragments of two k-steps (both operands permuted alike).  Warp w takes tile
+// w % 2 and the K slice w / 2 (one eighth of d); the slices' partial sums meet
+// in shared memory.  Each CTA takes a contiguous range of units and prefetches
+// the next unit's rows into L2 while it computes.
+constexpr int kXThreads = 512, kXWarps = kXThreads / 32, kXRows = 16, kXTok = 16;
+
+__global__ void __launch_bounds__(kXThreads, 1) exact_kernel(ExpertArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ __align__(16) char xsm[];  // [kXTok][2 d + 64] bf16 tokens (padded rows)
+  __shared__ int cu[kMaxAct + 1];
+  __shared__ int srow[kXRows];
+  __shared__ __align__(16) float red[2][kXWarps / 2][32][8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tid = threadIdx.x;
+  const int tile = warp & 1, kq = warp >> 1;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int I = a.I, d = a.d, W = (I + 31) >> 5;
+  const int xstride = 2 * d + 64;                // bytes; rows land 16 banks apart
+  const int kslice = d / 8, nkb = kslice / 32;   // elements and 32-element blocks per warp
+  const int n_act = __ldcg(a.ws.n_act);
+  if (warp == 0) {
+    int run = 0;
+    for (int b0 = 0; b0 < n_act; b0 += 32) {
+      const int ea = b0 + lane;
+      const int c = ea < n_act ? (__ldcg(a.ws.n_u + ea) + kXRows - 1) / kXRows : 0;
+      int inc = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFullMask, inc, o);
+        if (lane >= o) inc += v;
+      }
+      if (ea < n_act) cu[ea] = run + inc - c;
+      run += __shfl_sync(kFullMask, inc, 31);
+    }
+    if (lane == 0) cu[n_act] = run;
+  }
+  __syncthreads();
+  const int total = cu[n_act];
+  const int ub = (int)((long long)total * blockIdx.x / gridDim.x);
+  const int ue = (int)((long long)total * (blockIdx.x + 1) / gridDim.x);
+  int staged_ea = -1, staged_mt = -1;
+#pragma unroll 1
+  for (int u = ub; u < ue; u++) {
+    const int ea = unit_expert(cu, n_act, u);
+    const int e = __ldcg(a.ws.act_e + ea), p0 = __ldcg(a.ws.act_off + ea);
+    const int m = __ldcg(a.ws.act_off + ea + 1) - p0;
+    const int j0 = (u - cu[ea]) * kXRows;
+    const int nrows = min(kXRows, __ldcg(a.ws.n_u + ea) - j0);
+    __syncthreads();  // the previous unit is done with srow, xsm and red
+    if (tid < kXRows) srow[tid] = tid < nrows ? __ldcg(a.ws.ulist + (size_t)ea * I + j0 + tid) : -1;
+    if (warp == kXWarps - 1 && lane < kXRows && u + 1 < ue) {
+      // the next unit's rows start moving into L2
+      const int un = u + 1, ean = unit_expert(cu, n_act, un);
+      const int jn = (un - cu[ean]) * kXRows + lane;
+      if (jn < __ldcg(a.ws.n_u + ean)) {
+        const size_t row = (size_t)__ldcg(a.ws.act_e + ean) * I + __ldcg(a.ws.ulist + (size_t)ean * I + jn);
+        bulk_prefetch_l2(a.w_gate + row * d, 2 * d);
+        bulk_prefetch_l2(a.w_up + row * d, 2 * d);
+      }
+    }
+#pragma unroll 1
+    for (int mt = 0; mt < m; mt += kXTok) {
+      const int nt = min(kXTok, m - mt);
+      if (mt > 0) __syncthreads();  // the previous pass's epilogue is done with red
+      if (ea != staged_ea || mt != staged_mt) {
+        const int d8 = d >> 3;
+        for (int o = tid; o < nt * d8; o += kXThreads) {
+          const int t = o / d8, j8 = o - t * d8;
+          const int tok = __ldcg(a.ws.pair_tok + p0 + mt + t);
+          *reinterpret_cast<uint4*>(xsm + (size_t)t * xstride + 16 * j8) =
+              __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)tok * d) + j8);
+        }
+        staged_ea = ea;
+        staged_mt = mt;
+      }
+      __syncthreads();
+      const int rowi = srow[tile * 8 + gid];
+      const uint4* gr = reinterpret_cast<const uint4*>(a.w_gate + ((size_t)e * I + max(rowi, 0)) * d);
+      const uint4* ur = reinterpret_cast<const uint4*>(a.w_up + ((size_t)e * I + max(rowi, 0)) * d);
+      const char* xa_p = xsm + (size_t)gid * xstride;
+      const char* xb_p = xsm + (size_t)(gid + 8) * xstride;
+      float cg[4] = {0.0f, 0.0f, 0.0f, 0.0f}, cv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 1
+      for (int kb0 = 0; kb0 < nkb; kb0 += 8) {
+        uint4 wg[8], wu[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+          const int kel = kq * kslice + (kb0 + j) * 32 + tig * 8;
+          const bool ok = kb0 + j < nkb && rowi >= 0;
+          wg[j] = ok ? ld_stream(gr + kel / 8) : make_uint4(0u, 0u, 0u, 0u);
+          wu[j] = ok ? ld_stream(ur + kel / 8) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+          if (kb0 + j >= nkb) break;
+          const int kel = kq * kslice + (kb0 + j) * 32 + tig * 8;
+          const uint4 xa = gid < nt ? *reinterpret_cast<const uint4*>(xa_p + 2 * kel) : make_uint4(0u, 0u, 0u, 0u);
+          const uint4 xb =
+              gid + 8 < nt ? *reinterpret_cast<const uint4*>(xb_p + 2 * kel) : make_uint4(0u, 0u, 0u, 0u);
+          mma16816(cg, xa.x, xb.x, xa.y, xb.y, wg[j].x, wg[j].y);
+          mma16816(cv, xa.x, xb.x, xa.y, xb.y, wu[j].x, wu[j].y);
+          mma16816(cg, xa.z, xb.z, xa.w, xb.w, wg[j].z, wg[j].w);
+          mma16816(cv, xa.z, xb.z, xa.w, xb.w, wu[j].z, wu[j].w);
+        }
+      }
+      float4* rp = reinterpret_cast<float4*>(&red[tile][kq][lane][0]);
+      rp[0] = make_float4(cg[0], cg[1], cg[2], cg[3]);
+      rp[1] = make_float4(cv[0], cv[1], cv[2], cv[3]);
+      __syncthreads();
+      if (kq == 0) {
+        float sg[4] = {0.0f, 0.0f, 0.0f, 0.0f}, su[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int q = 0; q < kXWarps / 2; q++) {
+          const float4 pg = *reinterpret_cast<const float4*>(&red[tile][q][lane][0]);
+          const float4 pu = *reinterpret_cast<const float4*>(&red[tile][q][lane][4]);
+          sg[0] += pg.x;
+          sg[1] += pg.y;
+          sg[2] += pg.z;
+          sg[3] += pg.w;
+          su[0] += pu.x;
+          su[1] += pu.y;
+          su[2] += pu.z;
+          su[3] += pu.w;
+        }
+        // element h: token gid (+ 8 for h >= 2), tile row tig * 2 + (h & 1)
+#pragma unroll
+        for (int h = 0; h < 4; h++) {
+          const int tl = gid + (h >= 2 ? 8 : 0), rl = tile * 8 + tig * 2 + (h & 1);
+          if (tl < nt && rl < nrows) {
+            const int i = srow[rl], pr = p0 + mt + tl;
+            if ((__ldcg(a.ws.candm + (size_t)pr * W + (i >> 5)) >> (i & 31)) & 1u)
+              a.ws.apos[(size_t)pr * I + i] = __fmul_rn(silu_r(sg[h]), su[h]);
+          }
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------ down rows + combine
+// Unit = (active expert, column slice of SW columns).  Thread (g, q) takes
+// the 16-byte chunk q of the slice in kept-union rows g, g + G, ...; each
+// row enters every token of the expert with its coefficient (a if the token
+// kept the channel, else 0).  Then y_e = (row sum) + V z per (token, column),
+// written to the step's per-slot outputs; the last of a token's top-e slots
+// to arrive for a slice combines them in slot order (fp32 FMAs, plus the
+// residual) into bf16.
+template <int SW>
+__global__ void __launch_bounds__(kDThreads) down_kernel(ExpertArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  constexpr int QW = SW / 8, G = kDThreads / QW;
+  __shared__ __align__(16) float red[G][kDTG][SW];
+  __shared__ int sidx[kDRows];
+  __shared__ float scoef[kDTG][kDRows];
+  __shared__ int lastf[kDTG];
+  const int tid = threadIdx.x;
+  const int I = a.I, d = a.d, r = a.r, ns = d / SW, d8 = d >> 3;
+  const int g = tid / QW, q = tid - g * QW;
+  const int n_act = __ldcg(a.ws.n_act);
+  const int units = n_act * ns;
+#pragma unroll 1
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const int ea = u / ns, sl = u - ea * ns, j0 = sl * SW;
+    const int e = __ldcg(a.ws.act_e + ea), p0 = __ldcg(a.ws.act_off + ea);
+    const int m = __ldcg(a.ws.act_off + ea + 1) - p0;
+    const int nd = __ldcg(a.ws.n_d + ea);
+    const int* dl = a.ws.dlist + (size_t)ea * I;
+    const uint4* wd = reinterpret_cast<const uint4*>(a.w_down + (size_t)e * I * d + j0) + q;
+#pragma unroll 1
+    for (int tg = 0; tg < m; tg += kDTG) {
+      const int ng = min(kDTG, m - tg);
+      float acc[kDTG][8];
+#pragma unroll
+      for (int t = 0; t < kDTG; t++)
+#pragma unroll
+        for (int c = 0; c < 8; c++) acc[t][c] = 0.0f;
+      const float* cf = a.ws.coef + (size_t)(p0 + tg) * I;
+#pragma unroll 1
+      for (int r0 = 0; r0 < nd; r0 += kDRows) {
+        // the chunk's row indices and coefficients, staged once for all threads
+        const int nr = min(kDRows, nd - r0);
+        __syncthreads();
+        for (int o = tid; o < nr; o += kDThreads) sidx[o] = __ldcg(dl + r0 + o);
+        for (int o = tid; o < kDTG * nr; o += kDThreads) {
+          const int t = o / nr, rr = o - t * nr;
+          scoef[t][rr] = t < ng ? __ldcg(cf + (size_t)t * I + r0 + rr) : 0.0f;
+        }
+        __syncthreads();
+        int mr = g;
+#pragma unroll 1
+        for (; mr + 7 * G < nr; mr += 8 * G) {
+          uint4 w[8];
+#pragma unroll
+          for (int k = 0; k < 8; k++) w[k] = ld_stream(wd + (size_t)sidx[mr + k * G] * d8);
+#pragma unroll
+          for (int k = 0; k < 8; k++) {
+            float f[8];
+            bf16x8_to_f32(w[k], f);
+#pragma unroll
+            for (int t = 0; t < kDTG; t++) {
+              const float co = scoef[t][mr + k * G];
+#pragma unroll
+              for (int c = 0; c < 8; c++) acc[t][c] = fmaf(co, f[c], acc[t][c]);
+            }
+          }
+        }
+#pragma unroll 1
+        for (; mr < nr; mr += G) {
+          float f[8];
+          bf16x8_to_f32(ld_stream(wd + (size_t)sidx[mr] * d8), f);
+#pragma unroll
+          for (int t = 0; t < kDTG; t++) {
+            const float co = scoef[t][mr];
+#pragma unroll
+            for (int c = 0; c < 8; c++) acc[t][c] = fmaf(co, f[c], acc[t][c]);
+          }
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < kDTG; t++) {
+        float4* dst = reinterpret_cast<float4*>(&red[g][t][8 * q]);
+        dst[0] = make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
+        dst[1] = make_float4(acc[t][4], acc[t][5], acc[t][6], acc[t][7]);
+      }
+      __syncthreads();
+      for (int o = tid; o < ng * SW; o += kDThreads) {
+        const int t = o / SW, col = o - t * SW;
+        float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+        for (int gg = 0; gg < G; gg += 2) {
+          s0 += red[gg][t][col];
+          s1 += red[gg + 1][t][col];
+        }
+        float y = s0 + s1;
+        const int pr = p0 + tg + t;
+        if (r > 0) {
+          const uint16_t* vr = a.v + ((size_t)e * d + j0 + col) * r;
+          const float* zp = a.ws.z + (size_t)pr * r;
+          float r0 = 0.0f, r1 = 0.0f;
+          for (int k = 0; k < r; k += 8) {
+            const uint4 v8 = __ldg(reinterpret_cast<const uint4*>(vr + k));
+            const float4 za = __ldcg(reinterpret_cast<const float4*>(zp + k));
+            const float4 zb = __ldcg(reinterpret_cast<const float4*>(zp + k + 4));
+            r0 = fmaf(bf16lo(v8.x), za.x, r0);
+            r1 = fmaf(bf16hi(v8.x), za.y, r1);
+            r0 = fmaf(bf16lo(v8.y), za.z, r0);
+            r1 = fmaf(bf16hi(v8.y), za.w, r1);
+            r0 = fmaf(bf16lo(v8.z), zb.x, r0);
+            r1 = fmaf(bf16hi(v8.z), zb.y, r1);
+            r0 = fmaf(bf16lo(v8.w), zb.z, r0);
+            r1 = fmaf(bf16hi(v8.w), zb.w, r1);
+          }
+          y += r0 + r1;
+        }
+        const int tok = __ldcg(a.ws.pair_tok + pr), slot = __ldcg(a.ws.pair_slot + pr);
+        const size_t off = ((size_t)tok * a.top_e + slot) * d + j0 + col;
+        a.ws.ye[off] = y;
+        if (a.dbg_y_expert) a.dbg_y_expert[off] = y;
+      }
+      __syncthreads();  // the CTA's outputs precede the releases below
+      if (tid < ng) {
+        const int tok = __ldcg(a.ws.pair_tok + p0 + tg + tid);
+        lastf[tid] = arrive_last(a.ws.counters + tok * kMaxCluster + sl, (unsigned)a.top_e);
+      }
+      __syncthreads();
+#pragma unroll 1
+      for (int t = 0; t < ng; t++) {
+        if (!lastf[t]) continue;
+        const int tok = __ldcg(a.ws.pair_tok + p0 + tg + t);
+        for (int col = tid; col < SW; col += kDThreads) {
+          const int j = j0 + col;
+          float acc2 = 0.0f;
+          for (int s = 0; s < a.top_e; s++)
+            acc2 = fmaf(__ldcg(a.ws.wts + tok * a.top_e + s), __ldcg(a.ws.ye + ((size_t)tok * a.top_e + s) * d + j),
+                        acc2);
+          if (a.residual) acc2 += bf16f(a.residual[(size_t)tok * d + j]);
+          a.y[(size_t)tok * d + j] = f2bf16(acc2);
+        }
+        if (tid == 0) a.ws.counters[tok * kMaxCluster + sl] = 0u;
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Resident CTAs per SM of each kernel, per device (queried once).
+struct Occupancy {
+  int dev = -1, sms = 0;
+  int screen1 = 0, screen2 = 0, selc = 0, selk = 0, exact = 0, down128 = 0, down256 = 0;
+};
+Occupancy g_occ;
+
+// Also raises the kernel's dynamic shared-memory limit to `smem`.
+template <class K>
+int occ(K kernel, int threads, size_t smem) {
+  int n = 0;
+  if (smem > 48 * 1024) cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess) n = 1;
+  return n > 0 ? n : 1;
+}
+
+template <class K, class... Args>
+cudaError_t launch_pdl(K kernel, int grid, int threads, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid > 0 ? grid : 1);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+size_t exact_smem(int d) { return (size_t)kXTok * (2 * d + 64); }
+
+}  // namespace
+
+void set_path(int path) { g_path = path; }
+bool use_streamed(int B) { return g_path == 2 || (g_path == 0 && B > 2); }
+
+cudaError_t launch_stream(const ExpertArgs& a, cudaStream_t s) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (g_occ.dev != dev) {
+    Occupancy o;
+    o.dev = dev;
+    err = cudaDeviceGetAttribute(&o.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    o.exact = occ(exact_kernel, kXThreads, exact_smem(4096));  // the largest staging; sets the limit
+    o.screen1 = occ(screen_kernel<1>, kSThreads, 2 * kSStageBytes);
+    o.screen2 = occ(screen_kernel<2>, kSThreads, 2 * kSStageBytes);
+    o.selc = occ(select_c_kernel, kSelT, 0);
+    o.selk = occ(select_k_kernel, kSelT, 0);
+    o.down128 = occ(down_kernel<128>, kDThreads, 0);
+    o.down256 = occ(down_kernel<256>, kDThreads, 0);
+    g_occ = o;
+  }
+  const int P = a.B * a.top_e, nact = a.E < P ? a.E : P;
+  const int sms = g_occ.sms;
+  // screen
+  const int nvl = a.d <= 2048 ? 1 : 2;
+  const int chans = nvl == 1 ? ScreenGeom<1>::kChannels : ScreenGeom<2>::kChannels;
+  const int nblk = (a.I + chans - 1) / chans;
+  const int gs = nact * nblk < sms * (nvl == 1 ? g_occ.screen1 : g_occ.screen2) ? nact * nblk
+                                                                                   : sms * (nvl == 1 ? g_occ.screen1 : g_occ.screen2);
+  err = nvl == 1 ? launch_pdl(screen_kernel<1>, gs, kSThreads, 2 * kSStageBytes, s, a)
+                 : launch_pdl(screen_kernel<2>, gs, kSThreads, 2 * kSStageBytes, s, a);
+  if (err != cudaSuccess) return err;
+  // top-c
+  err = launch_pdl(select_c_kernel, P < sms * g_occ.selc ? P : sms * g_occ.selc, kSelT, 0, s, a);
+  if (err != cudaSuccess) return err;
+  // exact candidates
+  err = launch_pdl(exact_kernel, sms * g_occ.exact, kXThreads, exact_smem(a.d), s, a);
+  if (err != cudaSuccess) return err;
+  // top-k
+  err = launch_pdl(select_k_kernel, P < sms * g_occ.selk ? P : sms * g_occ.selk, kSelT, 0, s, a, nblk);
+  if (err != cudaSuccess) return err;
+  // down rows + combine
+  if (a.d <= 2048) {
+    const int ns = a.d / 128, gd = nact * ns < sms * g_occ.down128 ? nact * ns : sms * g_occ.down128;
+    return launch_pdl(down_kernel<128>, gd, kDThreads, 0, s, a);
+  }
+  const int ns = a.d / 256, gd = nact * ns < sms * g_occ.down256 ? nact * ns : sms * g_occ.down256;
+  return launch_pdl(down_kernel<256>, gd, kDThreads, 0, s, a);
+}
+
+}  // namespace moe

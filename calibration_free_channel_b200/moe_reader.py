@@ -20,7 +20,7 @@ _STATUS = {0: "MOE_OK", 1: "MOE_EINVAL", 2: "MOE_EUNSUPPORTED", 3: "MOE_ECUDA", 
 EXPORTS = ["moe_reader_workspace_bytes", "moe_reader_build_sketch", "moe_reader_lowrank_workspace_bytes",
            "moe_reader_build_lowrank", "moe_reader_forward", "moe_reader_forward_dense",
            "moe_reader_forward_host", "moe_reader_rmsnorm", "moe_reader_set_expert_events",
-           "moe_reader_check_error", "moe_reader_set_cluster_size", "moe_reader_launch_plan",
+           "moe_reader_check_error", "moe_reader_set_cluster_size", "moe_reader_set_path", "moe_reader_launch_plan",
            "moe_reader_forward_noalloc", "moe_reader_last_error"]
 
 
@@ -69,6 +69,7 @@ def lib():
         L.moe_reader_set_expert_events.argtypes = [P, P]
         L.moe_reader_check_error.argtypes = [P, P]
         L.moe_reader_set_cluster_size.argtypes = [i32]
+        L.moe_reader_set_path.argtypes = [i32]
         L.moe_reader_launch_plan.argtypes = [i32] * 7 + [P]
         L.moe_reader_forward_noalloc.argtypes = [C.POINTER(MoeReaderLayer), i32, i32, i32, P, P, P, P]
         L.moe_reader_last_error.restype = C.c_char_p
@@ -160,6 +161,12 @@ def moe_reader_check_error(workspace, stream=None):
 
 def moe_reader_set_cluster_size(cs: int):
     _check(lib().moe_reader_set_cluster_size(cs))
+
+
+def moe_reader_set_path(path: int):
+    """0: automatic (one cluster per expert for B <= 2, streamed above), 1: the
+    one-cluster reader, 2: the streamed reader (process-wide)."""
+    _check(lib().moe_reader_set_path(path))
 
 
 def moe_reader_launch_plan(dense: bool, B, E, top_e, I, d, r) -> dict:

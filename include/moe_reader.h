@@ -212,6 +212,18 @@ moe_status moe_reader_set_expert_events(void* ev_before, void* ev_after);
  * automatically (the size that keeps the most SMs busy for the launch). */
 moe_status moe_reader_set_cluster_size(int cs);
 
+/* Which reader runs a sparse step (process-wide; both compute the same sets
+ * and outputs within the tolerances above):
+ *   0  automatic: one cluster per expert for B <= 2, streamed for B > 2;
+ *   1  one thread-block cluster per (expert, token group), all stages in one
+ *      kernel (latency-bound chain; best at one or two tokens);
+ *   2  streamed: five kernels after routing (screen, top-c, exact
+ *      candidates, top-k, down rows + combine), each over every
+ *      (token, expert) pair of the step on all SMs, chained with
+ *      programmatic dependent launch.
+ * MOE_EINVAL for any other value. */
+moe_status moe_reader_set_path(int path);
+
 /* The launch the expert kernel would use for this shape on the current
  * device (dense != 0: the dense block): out4 = {cluster size, copy-ring rows
  * per warp, dynamic shared memory bytes per CTA, co-resident clusters}. */

@@ -122,7 +122,9 @@ def run_pair(layer: M.Layer, oc: OracleCache, x, k, c, top_e, use_oracle_factors
     W = oc.W
     logits, ids, _ = O.route(x, W["w_router"], W.get("router_bias"), top_e)
     lr = oc.lowrank_for(ids)
-    if use_oracle_factors and lr is not None:
+    if oc.r == 0:
+        layer.set_lowrank(None, None)  # no recovery on either side
+    elif use_oracle_factors:
         layer.set_lowrank(torch.from_numpy(lr[0].view(np.int16)).view(torch.bfloat16),
                           torch.from_numpy(lr[1].view(np.int16)).view(torch.bfloat16))
     y, dbg = layer.forward(x.cuda(), k=k, c=c, debug=True, recovery_input=recovery_input)
