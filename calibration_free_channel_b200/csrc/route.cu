@@ -14,7 +14,7 @@ namespace moe {
 
 namespace {
 
-constexpr int kRouteExpertsPerCta = 8;  // one warp per expert row
+constexpr int kRouteExpertsPerCta = 2;  // four warps per expert row
 constexpr int kRouteTokensPerCta = 8;
 
 __device__ __forceinline__ void dfma8(uint4 w, uint4 x, double& acc) {
@@ -29,48 +29,57 @@ __device__ __forceinline__ void dfma8(uint4 w, uint4 x, double& acc) {
 }
 
 // Blocks [0, n_logit_blocks) compute logits; the next B blocks (sparse path)
-// rotate and quantise one token each.
+// rotate and quantise one token each.  A logits block takes 2 experts and up
+// to 8 tokens: 4 warps per expert, each a quarter of d (two 16-byte chunks
+// per lane at a time, the chunks of every token in flight together); the
+// quarters' fp64 sums meet in shared memory.
 __global__ void __launch_bounds__(256) route_kernel(RouteArgs a, int n_logit_blocks, int n_eblk) {
   pdl_trigger();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if ((int)blockIdx.x < n_logit_blocks) {
-    const int e = (blockIdx.x % n_eblk) * kRouteExpertsPerCta + warp;
+    __shared__ double part[kRouteExpertsPerCta][4][kRouteTokensPerCta];
+    const int el = warp >> 2, wq = warp & 3;
+    const int e = (blockIdx.x % n_eblk) * kRouteExpertsPerCta + el;
     const int t0 = (blockIdx.x / n_eblk) * kRouteTokensPerCta;
     const int nt = min(kRouteTokensPerCta, a.B - t0);
-    if (e >= a.E) return;
     double acc[kRouteTokensPerCta];
 #pragma unroll
     for (int t = 0; t < kRouteTokensPerCta; t++) acc[t] = 0.0;
-    const uint4* wrow = reinterpret_cast<const uint4*>(a.w_router + (size_t)e * a.d);
     const int d8 = a.d / 8;
-    // the lane's router chunks 8 at a time, all loads in flight together
+    if (e < a.E) {
+      const uint4* wrow = reinterpret_cast<const uint4*>(a.w_router + (size_t)e * a.d);
+      // chunk j = 32 wq + lane + 128 u of the row
 #pragma unroll 1
-    for (int j0 = 0; j0 < d8; j0 += 256) {
-      uint4 w[8];
+      for (int u0 = 0; 128 * u0 < d8; u0 += 2) {
+        uint4 w[2], xv[kRouteTokensPerCta][2];
 #pragma unroll
-      for (int u = 0; u < 8; u++) {
-        const int j = j0 + 32 * u + lane;
-        w[u] = j < d8 ? __ldg(wrow + j) : make_uint4(0u, 0u, 0u, 0u);
-      }
+        for (int u = 0; u < 2; u++) {
+          const int j = 32 * wq + lane + 128 * (u0 + u);
+          w[u] = j < d8 ? __ldg(wrow + j) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-      for (int t = 0; t < kRouteTokensPerCta; t++) {
-        if (t >= nt) break;
-        const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)(t0 + t) * a.d);
-        uint4 xv[8];
-#pragma unroll
-        for (int u = 0; u < 8; u++) {
-          const int j = j0 + 32 * u + lane;
-          xv[u] = j < d8 ? __ldg(xr + j) : make_uint4(0u, 0u, 0u, 0u);
+          for (int t = 0; t < kRouteTokensPerCta; t++)
+            xv[t][u] = j < d8 && t < nt ? __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)(t0 + t) * a.d) + j)
+                                        : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < 8; u++) dfma8(w[u], xv[u], acc[t]);
+        for (int t = 0; t < kRouteTokensPerCta; t++) {
+          dfma8(w[0], xv[t][0], acc[t]);
+          dfma8(w[1], xv[t][1], acc[t]);
+        }
       }
     }
 #pragma unroll
     for (int t = 0; t < kRouteTokensPerCta; t++) {
-      if (t < nt) {
-        const double s = warp_sum(acc[t]);
-        if (lane == 0) a.ws.logits[(size_t)(t0 + t) * a.E + e] = s + (a.bias ? (double)a.bias[e] : 0.0);
+      const double s = warp_sum(acc[t]);
+      if (lane == 0) part[el][wq][t] = s;
+    }
+    __syncthreads();
+    if (threadIdx.x < kRouteExpertsPerCta * kRouteTokensPerCta) {
+      const int ee = threadIdx.x / kRouteTokensPerCta, t = threadIdx.x % kRouteTokensPerCta;
+      const int eg = (blockIdx.x % n_eblk) * kRouteExpertsPerCta + ee;
+      if (eg < a.E && t < nt) {
+        const double s = (part[ee][0][t] + part[ee][1][t]) + (part[ee][2][t] + part[ee][3][t]);
+        a.ws.logits[(size_t)(t0 + t) * a.E + eg] = s + (a.bias ? (double)a.bias[eg] : 0.0);
       }
     }
     return;

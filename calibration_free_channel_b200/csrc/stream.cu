@@ -33,7 +33,7 @@ namespace {
 
 constexpr unsigned kFullMask = 0xffffffffu;
 
-constexpr int kSThreads = 256;  // screen: 8 warps, 4 / NVL channels per warp
+constexpr int kSThreads = 128;  // screen: 4 warps, 8 / NVL channels per warp
 constexpr int kSTG = 2;         // screen: tokens per register group
 constexpr int kSelT = sel::kSelThreads;
 constexpr int kDThreads = 256;  // down rows
@@ -76,27 +76,31 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 w, float (&f)[8]) {
   f[7] = bf16hi(w.w);
 }
 
-// Screen-block geometry: channels per warp and per block for NVL 16-byte
-// sketch vectors per lane and row (NVL = 1 for d <= 2048, 2 for d = 4096);
+// Screen-block geometry for NVL = 1 (d <= 2048) and NVL = 2 (d = 4096): a
+// warp takes kPerWarp channels, each split over kParts lanes (parts of d);
 // a block's sketch rows are 16 KB per matrix either way.
 template <int NVL>
 struct ScreenGeom {
-  static constexpr int kPerWarp = 4 / NVL;
-  static constexpr int kChannels = 8 * kPerWarp;
+  static constexpr int kPerWarp = 8 / NVL;
+  static constexpr int kParts = 32 / kPerWarp;
+  static constexpr int kChannels = 4 * kPerWarp;  // 4 warps
 };
-constexpr int kSStageBytes = 2 * 16384;  // gate + up rows of one block
+constexpr int kSkBytes = 16384;                      // sketch rows of one block, per matrix
+constexpr int kSStageBytes = 2 * kSkBytes + 8192;   // + the block's Ubar rows (<= 32 x 128 bf16)
+constexpr int kQChunk = 80;                          // staged activations: 64 bytes per chunk, padded
 
 // ------------------------------------------------------------------ screen
 // Unit = (active expert, block of ScreenGeom::kChannels channels).  The
-// block's gate and up sketch rows are contiguous: one thread copies them into
-// shared memory with two bulk copies, the next unit's copies in flight while
-// this one is computed (two stages).  A warp takes the expert's tokens kSTG
-// at a time, their activations at its lanes' sketch vectors in registers,
-// and its channels one pass at a time; the lanes of one channel (LG =
-// min(32, d / 64) of them) reduce its dots with shuffles.  Scores follow the
-// one-cluster reader: ghat = ((float)G alpha_g) c_x, uhat likewise,
-// ahat = silu_r(ghat) uhat, sigma = |ahat|, with G, U the exact integer dots
-// less the code offset sum(q).
+// block's gate and up sketch rows (and its Ubar rows) are contiguous: one
+// thread copies them into shared memory with bulk copies, the next unit's
+// copies in flight while this one is computed (two stages).  Lane (c, p) of a
+// warp takes channel c and part p of d: it walks its 64-trit chunks of both
+// rows (in an order rotated by lane, so the eight lanes of a shared-memory
+// wavefront read distinct banks) against the tokens' activations, staged kSTG
+// tokens at a time; two shuffles sum the parts, and lane p = t of the channel
+// finishes token t.  Scores follow the one-cluster reader: ghat =
+// ((float)G alpha_g) c_x, uhat likewise, ahat = silu_r(ghat) uhat,
+// sigma = |ahat|, with G, U the exact integer dots less the code offset sum(q).
 template <int NVL>
 __device__ __forceinline__ void screen_issue(const ExpertArgs& a, int u, int nblk, char* dst, uint64_t* bar) {
   using Geo = ScreenGeom<NVL>;
@@ -104,10 +108,11 @@ __device__ __forceinline__ void screen_issue(const ExpertArgs& a, int u, int nbl
   const int e = __ldcg(a.ws.act_e + ea);
   const int i0 = blk * Geo::kChannels, ncw = min(Geo::kChannels, a.I - i0);
   const size_t row = (size_t)a.d / 4;  // bytes of one sketch row
-  const uint32_t bytes = (uint32_t)(ncw * row);
-  mbar_expect_tx(bar, 2 * bytes);
+  const uint32_t bytes = (uint32_t)(ncw * row), ubytes = (uint32_t)(ncw * a.r * 2);
+  mbar_expect_tx(bar, 2 * bytes + ubytes);
   bulk_g2s(dst, reinterpret_cast<const char*>(a.sk_gate) + ((size_t)e * a.I + i0) * row, bytes, bar);
-  bulk_g2s(dst + kSStageBytes / 2, reinterpret_cast<const char*>(a.sk_up) + ((size_t)e * a.I + i0) * row, bytes, bar);
+  bulk_g2s(dst + kSkBytes, reinterpret_cast<const char*>(a.sk_up) + ((size_t)e * a.I + i0) * row, bytes, bar);
+  if (ubytes) bulk_g2s(dst + 2 * kSkBytes, a.u_sigma + ((size_t)e * a.I + i0) * a.r, ubytes, bar);
 }
 
 template <int NVL>
@@ -115,18 +120,22 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
   pdl_trigger();
   pdl_wait();
   using Geo = ScreenGeom<NVL>;
-  extern __shared__ __align__(128) char sk_stage[];  // [2][gate 16 KB | up 16 KB]
+  extern __shared__ __align__(128) char sk_stage[];  // [2][gate 16 KB | up 16 KB | Ubar 8 KB]
+  __shared__ __align__(16) char qst[kSTG * 64 * kQChunk];  // staged activations (d <= 4096)
   __shared__ float sah[kSTG][Geo::kChannels];
   __shared__ float salg[Geo::kChannels], salu[Geo::kChannels];
+  __shared__ int stok[kSTG], sqs[kSTG];
+  __shared__ float scx[kSTG];
   __shared__ __align__(8) uint64_t bars[2];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tid = threadIdx.x;
   const int I = a.I, d = a.d, r = a.r;
-  const int nv = d >> 6;                          // sketch vectors per row
-  // a pass covers SUB channels (LG lanes each); small d can leave lanes idle
-  const int LG = nv < 32 ? nv : 32, SUB = 32 / LG, PP = (Geo::kPerWarp + SUB - 1) / SUB;
-  const int lv = lane & (LG - 1), sub = lane / LG;
+  const int nv = d >> 6;                     // 64-trit chunks (16 bytes) per row
+  const int nch = nv / Geo::kParts;          // chunks per lane
+  const int c = lane / Geo::kParts, part = lane - c * Geo::kParts;
+  const int lc = warp * Geo::kPerWarp + c;   // the lane's channel in the block
+  const int rot = lane & 7;
   const int nblk = (I + Geo::kChannels - 1) / Geo::kChannels;
-  const int zstride = (I + 15) / 16;              // zpart blocks per pair (the finest geometry)
+  const int zstride = (I + 15) / 16;         // zpart blocks per pair (the finest geometry)
   const int n_act = __ldcg(a.ws.n_act);
   const int units = n_act * nblk;
   uint32_t* err = a.ws.err;
@@ -137,7 +146,7 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
   }
   __syncthreads();
   if (tid == 0 && (int)blockIdx.x < units) screen_issue<NVL>(a, blockIdx.x, nblk, sk_stage, &bars[0]);
-  int it = 0;
+  int it = 0, staged_p0 = -1, staged_tg = -1;
 #pragma unroll 1
   for (int u = blockIdx.x; u < units; u += gridDim.x, it++) {
     const int st = it & 1;
@@ -147,125 +156,97 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
     const int e = __ldcg(a.ws.act_e + ea), p0 = __ldcg(a.ws.act_off + ea);
     const int m = __ldcg(a.ws.act_off + ea + 1) - p0;
     const int i0 = blk * Geo::kChannels, ncw = min(Geo::kChannels, I - i0);
+    const bool ok = lc < ncw;
     if (tid < ncw) {
       salg[tid] = __ldg(a.alpha_gate + (size_t)e * I + i0 + tid);
       salu[tid] = __ldg(a.alpha_up + (size_t)e * I + i0 + tid);
     }
-    __syncthreads();
-    const uint4* skg = reinterpret_cast<const uint4*>(sk_stage + st * kSStageBytes);
-    const uint4* sku = skg + kSStageBytes / 32;
+    const char* stage = sk_stage + st * kSStageBytes;
+    const uint4* grow = reinterpret_cast<const uint4*>(stage) + (size_t)lc * nv + part * nch;
+    const uint4* urow = reinterpret_cast<const uint4*>(stage + kSkBytes) + (size_t)lc * nv + part * nch;
+    const uint16_t* ubs = reinterpret_cast<const uint16_t*>(stage + 2 * kSkBytes);
     mbar_wait_bounded(&bars[st], (it >> 1) & 1, err);
 #pragma unroll 1
     for (int tg = 0; tg < m; tg += kSTG) {
       const int ng = min(kSTG, m - tg);
-      int tk[kSTG], qs[kSTG];
-      float cx[kSTG];
-#pragma unroll
-      for (int t = 0; t < kSTG; t++) {
-        tk[t] = __ldcg(a.ws.pair_tok + p0 + tg + min(t, ng - 1));
-        qs[t] = __ldcg(a.ws.qsum + tk[t]);
-        cx[t] = __ldcg(a.ws.cx + tk[t]);
+      __syncthreads();  // the previous group is done with qst (and the alpha stores are visible)
+      if (p0 != staged_p0 || tg != staged_tg) {
+        if (tid < kSTG) {
+          const int tk = __ldcg(a.ws.pair_tok + p0 + tg + min(tid, ng - 1));
+          stok[tid] = tk;
+          sqs[tid] = __ldcg(a.ws.qsum + tk);
+          scx[tid] = __ldcg(a.ws.cx + tk);
+        }
+        for (int o = tid; o < ng * nv * 4; o += kSThreads) {
+          const int t = o / (nv * 4), w = o - t * nv * 4;
+          const int tk = __ldcg(a.ws.pair_tok + p0 + tg + t);
+          *reinterpret_cast<uint4*>(qst + (t * nv + (w >> 2)) * kQChunk + (w & 3) * 16) =
+              ld_cg4(reinterpret_cast<const uint4*>(a.ws.q + (size_t)tk * d) + w);
+        }
+        staged_p0 = p0;
+        staged_tg = tg;
+        __syncthreads();
       }
-      // the tokens' activations at this lane's sketch vectors
-      uint4 qv[kSTG][NVL][4];
+      int ga[kSTG][4], ua[kSTG][4];
 #pragma unroll
       for (int t = 0; t < kSTG; t++)
 #pragma unroll
-        for (int k = 0; k < NVL; k++) {
-          const uint4* qp = reinterpret_cast<const uint4*>(a.ws.q + (size_t)tk[t] * d) + 4 * (lv + LG * k);
-#pragma unroll
-          for (int w = 0; w < 4; w++) qv[t][k][w] = ld_cg4(qp + w);
-        }
-#pragma unroll 1
-      for (int pp = 0; pp < PP; pp++) {
-        const int lc = warp * Geo::kPerWarp + pp * SUB + sub;
-        const bool ok = pp * SUB + sub < Geo::kPerWarp && lc < ncw;
-        int ga[kSTG][4], ua[kSTG][4];
-#pragma unroll
-        for (int t = 0; t < kSTG; t++)
-#pragma unroll
-          for (int w = 0; w < 4; w++) ga[t][w] = ua[t][w] = 0;
-#pragma unroll
-        for (int k = 0; k < NVL; k++) {
-          const int o = lc * nv + lv + LG * k;
-          const uint4 g4 = ok ? skg[o] : make_uint4(0u, 0u, 0u, 0u);
-          const uint4 u4 = ok ? sku[o] : make_uint4(0u, 0u, 0u, 0u);
+        for (int w = 0; w < 4; w++) ga[t][w] = ua[t][w] = 0;
+      if (ok) {
+#pragma unroll 2
+        for (int j = 0; j < nch; j++) {
+          const int jr = (j + rot) & (nch - 1);
+          const uint4 g4 = grow[jr], u4 = urow[jr];
+          const char* qc = qst + (part * nch + jr) * kQChunk;
 #pragma unroll
           for (int t = 0; t < kSTG; t++) {
             if (t >= ng) break;
-            code_dot16(g4.x, qv[t][k][0], ga[t]);
-            code_dot16(g4.y, qv[t][k][1], ga[t]);
-            code_dot16(g4.z, qv[t][k][2], ga[t]);
-            code_dot16(g4.w, qv[t][k][3], ga[t]);
-            code_dot16(u4.x, qv[t][k][0], ua[t]);
-            code_dot16(u4.y, qv[t][k][1], ua[t]);
-            code_dot16(u4.z, qv[t][k][2], ua[t]);
-            code_dot16(u4.w, qv[t][k][3], ua[t]);
+            const uint4* qv = reinterpret_cast<const uint4*>(qc + t * nv * kQChunk);
+            const uint4 q0 = qv[0], q1 = qv[1], q2 = qv[2], q3 = qv[3];
+            code_dot16(g4.x, q0, ga[t]);
+            code_dot16(g4.y, q1, ga[t]);
+            code_dot16(g4.z, q2, ga[t]);
+            code_dot16(g4.w, q3, ga[t]);
+            code_dot16(u4.x, q0, ua[t]);
+            code_dot16(u4.y, q1, ua[t]);
+            code_dot16(u4.z, q2, ua[t]);
+            code_dot16(u4.w, q3, ua[t]);
           }
         }
-        // channel sums; the finishing lane of token t holds (g, u)
-        int g, uu, t;
-        if (LG == 32) {
-          // reduce-scatter of (G0, U0, G1, U1) over the warp: lane 16 t
-          // ends with G_t, lane 16 t + 8 with U_t
-          const int v0 = code_dot_total(ga[0]), v1 = code_dot_total(ua[0]);
-          const int v2 = code_dot_total(ga[1]), v3 = code_dot_total(ua[1]);
-          const bool h16 = lane & 16, h8 = lane & 8;
-          const int a0 = (h16 ? v2 : v0) + __shfl_xor_sync(kFullMask, h16 ? v0 : v2, 16);
-          const int a1 = (h16 ? v3 : v1) + __shfl_xor_sync(kFullMask, h16 ? v1 : v3, 16);
-          int b0 = (h8 ? a1 : a0) + __shfl_xor_sync(kFullMask, h8 ? a0 : a1, 8);
-          b0 += __shfl_xor_sync(kFullMask, b0, 4);
-          b0 += __shfl_xor_sync(kFullMask, b0, 2);
-          b0 += __shfl_xor_sync(kFullMask, b0, 1);
-          g = b0;
-          uu = __shfl_xor_sync(kFullMask, b0, 8);
-          t = (lane & 15) == 0 ? lane >> 4 : kSTG;
-        } else {
-          int G[kSTG], U[kSTG];
+      }
+      // sum over the channel's parts (adjacent lanes)
+      int G[kSTG], U[kSTG];
 #pragma unroll
-          for (int tt = 0; tt < kSTG; tt++) {
-            G[tt] = code_dot_total(ga[tt]);
-            U[tt] = code_dot_total(ua[tt]);
-          }
-          for (int o = LG >> 1; o > 0; o >>= 1)
+      for (int t = 0; t < kSTG; t++) {
+        G[t] = code_dot_total(ga[t]);
+        U[t] = code_dot_total(ua[t]);
 #pragma unroll
-            for (int tt = 0; tt < kSTG; tt++) {
-              G[tt] += __shfl_xor_sync(kFullMask, G[tt], o);
-              U[tt] += __shfl_xor_sync(kFullMask, U[tt], o);
-            }
-          g = G[0];
-          uu = U[0];
-#pragma unroll
-          for (int tt = 1; tt < kSTG; tt++)
-            if (lv == tt) {
-              g = G[tt];
-              uu = U[tt];
-            }
-          t = lv;
+        for (int o = 1; o < Geo::kParts; o <<= 1) {
+          G[t] += __shfl_xor_sync(kFullMask, G[t], o);
+          U[t] += __shfl_xor_sync(kFullMask, U[t], o);
         }
-        if (ok && t < ng) {
-          int tok = tk[0], qst = qs[0];
-          float cxt = cx[0];
+      }
+      if (ok && part < ng) {
+        const int t = part;
+        int g = G[0], uu = U[0];
 #pragma unroll
-          for (int tt = 1; tt < kSTG; tt++)
-            if (t == tt) {
-              tok = tk[tt];
-              qst = qs[tt];
-              cxt = cx[tt];
-            }
-          const int i = i0 + lc, pr = p0 + tg + t;
-          const int g2 = g - qst, u2 = uu - qst;
-          const float gh = __fmul_rn(__fmul_rn((float)g2, salg[lc]), cxt);
-          const float uh = __fmul_rn(__fmul_rn((float)u2, salu[lc]), cxt);
-          const float ah = __fmul_rn(silu_r(gh), uh);
-          a.ws.sa[(size_t)pr * I + i] = make_float2(fabsf(ah), ah);
-          sah[t][lc] = ah;
-          if (a.dbg_G || a.dbg_U || a.dbg_sigma) {
-            const size_t off = ((size_t)tok * a.top_e + __ldcg(a.ws.pair_slot + pr)) * I + i;
-            if (a.dbg_G) a.dbg_G[off] = g2;
-            if (a.dbg_U) a.dbg_U[off] = u2;
-            if (a.dbg_sigma) a.dbg_sigma[off] = fabsf(ah);
+        for (int tt = 1; tt < kSTG; tt++)
+          if (t == tt) {
+            g = G[tt];
+            uu = U[tt];
           }
+        const int i = i0 + lc, pr = p0 + tg + t;
+        const int g2 = g - sqs[t], u2 = uu - sqs[t];
+        const float gh = __fmul_rn(__fmul_rn((float)g2, salg[lc]), scx[t]);
+        const float uh = __fmul_rn(__fmul_rn((float)u2, salu[lc]), scx[t]);
+        const float ah = __fmul_rn(silu_r(gh), uh);
+        a.ws.sa[(size_t)pr * I + i] = make_float2(fabsf(ah), ah);
+        sah[t][lc] = ah;
+        if (a.dbg_G || a.dbg_U || a.dbg_sigma) {
+          const size_t off = ((size_t)stok[t] * a.top_e + __ldcg(a.ws.pair_slot + pr)) * I + i;
+          if (a.dbg_G) a.dbg_G[off] = g2;
+          if (a.dbg_U) a.dbg_U[off] = u2;
+          if (a.dbg_sigma) a.dbg_sigma[off] = fabsf(ah);
         }
       }
       // recovery-input partial of the block: sum over its channels of ahat_i Ubar_i
@@ -273,18 +254,17 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
         __syncthreads();
         for (int o = tid; o < ng * r; o += kSThreads) {
           const int t = o / r, p = o - t * r;
-          const uint16_t* ub = a.u_sigma + ((size_t)e * I + i0) * r + p;
+          const uint16_t* ub = ubs + p;
           float z0 = 0.0f, z1 = 0.0f;
-          int lc = 0;
-          for (; lc + 2 <= ncw; lc += 2) {
-            z0 = fmaf(sah[t][lc], bf16f(ub[(size_t)lc * r]), z0);
-            z1 = fmaf(sah[t][lc + 1], bf16f(ub[(size_t)(lc + 1) * r]), z1);
+          int l = 0;
+          for (; l + 2 <= ncw; l += 2) {
+            z0 = fmaf(sah[t][l], bf16f(ub[(size_t)l * r]), z0);
+            z1 = fmaf(sah[t][l + 1], bf16f(ub[(size_t)(l + 1) * r]), z1);
           }
-          if (lc < ncw) z0 = fmaf(sah[t][lc], bf16f(ub[(size_t)lc * r]), z0);
+          if (l < ncw) z0 = fmaf(sah[t][l], bf16f(ub[(size_t)l * r]), z0);
           a.ws.zpart[((size_t)(p0 + tg + t) * zstride + blk) * r + p] = z0 + z1;
         }
       }
-      __syncthreads();
     }
     // every warp is done with this stage before the copy two units on reuses it
     __syncthreads();
@@ -301,7 +281,6 @@ struct SelSmem {
   __align__(16) int scratch[128];
   __align__(16) uint32_t mk[64];
   __align__(16) uint32_t kw[64];
-  __align__(16) float zr[kSelT];
 };
 
 // -------------------------------------------------------------- top-c
@@ -393,25 +372,48 @@ __global__ void __launch_bounds__(kSelT) select_k_kernel(ExpertArgs a, int nblk)
       __syncthreads();
     }
     if (r > 0) {
-      // thread (part, p): candidate positions part, part + parts, ...
-      const int parts = kSelT / r, part = tid / r, pz = tid - part * r;
-      float acc = 0.0f;
-      if (part < parts) {
-        const float* sap = reinterpret_cast<const float*>(a.ws.sa + (size_t)p * I);
-        for (int j = part; j < nc; j += parts) {
-          const bool kept = (sm.mk[j >> 5] >> (j & 31)) & 1u;
-          if (!kept && !rec_exact) continue;
-          const int i = sm.list[j];
+      // coefficient of each candidate position (0 where its Ubar row does not
+      // enter), then thread (jl, c) sums coefficient x Ubar chunk c (8 entries)
+      // over positions jl, jl + nj, ...; the partials meet in the (free)
+      // selection histogram in a fixed order
+      float* co = reinterpret_cast<float*>(sm.keys);
+      const float* sap = reinterpret_cast<const float*>(a.ws.sa + (size_t)p * I);
+      for (int j = tid; j < nc; j += kSelT) {
+        const bool kept = (sm.mk[j >> 5] >> (j & 31)) & 1u;
+        const int i = sm.list[j];
+        float v = 0.0f;
+        if (kept || rec_exact) {
           const float ah = __ldcg(sap + 2 * i + 1);
-          const float co = kept ? ah : __fsub_rn(ah, __ldcg(ap + i));
-          acc = fmaf(co, bf16f(a.u_sigma[((size_t)e * I + i) * r + pz]), acc);
+          v = kept ? ah : __fsub_rn(ah, __ldcg(ap + i));
+        }
+        co[j] = v;
+      }
+      __syncthreads();
+      const int nchk = r / 8, nj = kSelT / nchk;
+      const int c = tid % nchk, jl = tid / nchk;
+      float acc[8];
+#pragma unroll
+      for (int h = 0; h < 8; h++) acc[h] = 0.0f;
+      if (jl < nj) {
+        const uint16_t* ub = a.u_sigma + (size_t)e * I * r + 8 * c;
+#pragma unroll 4
+        for (int j = jl; j < nc; j += nj) {
+          const float cj = co[j];
+          if (cj == 0.0f) continue;
+          float f[8];
+          bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(ub + (size_t)sm.list[j] * r)), f);
+#pragma unroll
+          for (int h = 0; h < 8; h++) acc[h] = fmaf(cj, f[h], acc[h]);
         }
       }
-      sm.zr[tid] = acc;
+      float* zs = reinterpret_cast<float*>(sm.hist);  // [nj][r]
+      if (jl < nj)
+#pragma unroll
+        for (int h = 0; h < 8; h++) zs[jl * r + 8 * c + h] = acc[h];
       __syncthreads();
       if (tid < r) {
         float s0 = 0.0f, s1 = 0.0f;
-        for (int q = 0; q < parts; q++) s0 += sm.zr[q * r + tid];
+        for (int q = 0; q < nj; q++) s0 += zs[q * r + tid];
         const float* zp = a.ws.zpart + (size_t)p * zstride * r + tid;
         for (int b = 0; b < nblk; b++) s1 += __ldcg(zp + (size_t)b * r);
         a.ws.z[(size_t)p * r + tid] = s1 - s0;
@@ -442,32 +444,6 @@ __global__ void __launch_bounds__(kSelT) select_k_kernel(ExpertArgs a, int nblk)
     }
     __syncthreads();
   }
-}
-
-// Butterfly reduce-scatter of 8 per-lane values over the warp (9 shuffles):
-// afterwards lane L holds the warp sum of value 4 b4 + 2 b3 + b2, where bN is
-// bit N of L.
-__device__ __forceinline__ float reduce_scatter8(float (&v)[8]) {
-  const int lane = threadIdx.x & 31;
-  const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
-#pragma unroll
-  for (int j = 0; j < 4; j++) {
-    const float send = h16 ? v[j] : v[j + 4], keep = h16 ? v[j + 4] : v[j];
-    v[j] = keep + __shfl_xor_sync(kFullMask, send, 16);
-  }
-#pragma unroll
-  for (int j = 0; j < 2; j++) {
-    const float send = h8 ? v[j] : v[j + 2], keep = h8 ? v[j + 2] : v[j];
-    v[j] = keep + __shfl_xor_sync(kFullMask, send, 8);
-  }
-  {
-    const float send = h4 ? v[0] : v[1], keep = h4 ? v[1] : v[0];
-    v[0] = keep + __shfl_xor_sync(kFullMask, send, 4);
-  }
-  float s = v[0];
-  s += __shfl_xor_sync(kFullMask, s, 2);
-  s += __shfl_xor_sync(kFullMask, s, 1);
-  return s;
 }
 
 // bf16 m16n8k16 tensor-core product, fp32 accumulate: c += A B.
@@ -649,7 +625,8 @@ template <int SW>
 __global__ void __launch_bounds__(kDThreads) down_kernel(ExpertArgs a) {
   pdl_trigger();
   pdl_wait();
-  constexpr int QW = SW / 8, G = kDThreads / QW;
+  constexpr int QW = SW / 8, G = kDThreads / QW, CR = 16 * G;  // CR: rows staged per chunk (16 per thread)
+  static_assert(CR <= kDRows, "row chunk exceeds the staging arrays");
   __shared__ __align__(16) float red[G][kDTG][SW];
   __shared__ int sidx[kDRows];
   __shared__ float scoef[kDTG][kDRows];
@@ -659,6 +636,7 @@ __global__ void __launch_bounds__(kDThreads) down_kernel(ExpertArgs a) {
   const int g = tid / QW, q = tid - g * QW;
   const int n_act = __ldcg(a.ws.n_act);
   const int units = n_act * ns;
+  int staged_ea = -1, staged_tg = -1, staged_r0 = -1;
 #pragma unroll 1
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
     const int ea = u / ns, sl = u - ea * ns, j0 = sl * SW;
@@ -677,38 +655,34 @@ __global__ void __launch_bounds__(kDThreads) down_kernel(ExpertArgs a) {
         for (int c = 0; c < 8; c++) acc[t][c] = 0.0f;
       const float* cf = a.ws.coef + (size_t)(p0 + tg) * I;
 #pragma unroll 1
-      for (int r0 = 0; r0 < nd; r0 += kDRows) {
+      for (int r0 = 0; r0 < nd; r0 += CR) {
         // the chunk's row indices and coefficients, staged once for all threads
-        const int nr = min(kDRows, nd - r0);
-        __syncthreads();
-        for (int o = tid; o < nr; o += kDThreads) sidx[o] = __ldcg(dl + r0 + o);
-        for (int o = tid; o < kDTG * nr; o += kDThreads) {
-          const int t = o / nr, rr = o - t * nr;
-          scoef[t][rr] = t < ng ? __ldcg(cf + (size_t)t * I + r0 + rr) : 0.0f;
-        }
-        __syncthreads();
-        int mr = g;
-#pragma unroll 1
-        for (; mr + 7 * G < nr; mr += 8 * G) {
-          uint4 w[8];
-#pragma unroll
-          for (int k = 0; k < 8; k++) w[k] = ld_stream(wd + (size_t)sidx[mr + k * G] * d8);
-#pragma unroll
-          for (int k = 0; k < 8; k++) {
-            float f[8];
-            bf16x8_to_f32(w[k], f);
-#pragma unroll
-            for (int t = 0; t < kDTG; t++) {
-              const float co = scoef[t][mr + k * G];
-#pragma unroll
-              for (int c = 0; c < 8; c++) acc[t][c] = fmaf(co, f[c], acc[t][c]);
-            }
+        const int nr = min(CR, nd - r0);
+        if (ea != staged_ea || tg != staged_tg || r0 != staged_r0) {
+          __syncthreads();
+          for (int o = tid; o < nr; o += kDThreads) sidx[o] = __ldcg(dl + r0 + o);
+          for (int o = tid; o < kDTG * nr; o += kDThreads) {
+            const int t = o / nr, rr = o - t * nr;
+            scoef[t][rr] = t < ng ? __ldcg(cf + (size_t)t * I + r0 + rr) : 0.0f;
           }
+          staged_ea = ea;
+          staged_tg = tg;
+          staged_r0 = r0;
+          __syncthreads();
         }
-#pragma unroll 1
-        for (; mr < nr; mr += G) {
+        // every row of the chunk this thread takes, all loads in flight together
+        uint4 w[16];
+#pragma unroll
+        for (int k = 0; k < 16; k++) {
+          const int mr = g + k * G;
+          w[k] = mr < nr ? ld_stream(wd + (size_t)sidx[mr] * d8) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < 16; k++) {
+          const int mr = g + k * G;
+          if (mr >= nr) break;
           float f[8];
-          bf16x8_to_f32(ld_stream(wd + (size_t)sidx[mr] * d8), f);
+          bf16x8_to_f32(w[k], f);
 #pragma unroll
           for (int t = 0; t < kDTG; t++) {
             const float co = scoef[t][mr];
@@ -738,6 +712,7 @@ __global__ void __launch_bounds__(kDThreads) down_kernel(ExpertArgs a) {
           const uint16_t* vr = a.v + ((size_t)e * d + j0 + col) * r;
           const float* zp = a.ws.z + (size_t)pr * r;
           float r0 = 0.0f, r1 = 0.0f;
+#pragma unroll 4
           for (int k = 0; k < r; k += 8) {
             const uint4 v8 = __ldg(reinterpret_cast<const uint4*>(vr + k));
             const float4 za = __ldcg(reinterpret_cast<const float4*>(zp + k));
