@@ -79,9 +79,11 @@ moe_status check_layer(const moe_reader_layer* L, bool sparse) {
   return MOE_OK;
 }
 
+// ep_size > 0: expert-parallel step of rank ep_rank; writes y_partial (fp32)
+// instead of y.
 moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uint16_t* x, const uint16_t* residual,
                        uint16_t* y, const moe_reader_debug* dbg, void* workspace, size_t ws_bytes, void* stream,
-                       bool dense) {
+                       bool dense, int ep_rank = 0, int ep_size = 0, float* y_partial = nullptr) {
   moe_status st = check_layer(L, !dense);
   if (st != MOE_OK) return st;
   st = check_shape(B, L->E, L->top_e, L->I, L->d);
@@ -91,7 +93,13 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
     REQUIRE(c >= k && c <= L->I, "c = %d outside [k = %d, I = %d]", c, k, L->I);
   }
   REQUIRE_PTR(x);
-  REQUIRE_PTR(y);
+  if (ep_size > 0) {
+    REQUIRE(ep_size <= L->E && ep_rank >= 0 && ep_rank < ep_size, "ep_rank = %d, ep_size = %d: need 0 <= rank < size <= E",
+            ep_rank, ep_size);
+    REQUIRE_PTR(y_partial);
+  } else {
+    REQUIRE_PTR(y);
+  }
   OPT_PTR(residual);
   REQUIRE_PTR(workspace);
   const int sI = dense ? 0 : L->I, sr = dense ? 0 : L->r;
@@ -115,7 +123,9 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   ra.dbg_w = dbg ? dbg->weights : nullptr;
   ra.quantize = !dense;
   cudaError_t e = cudaSuccess;
-  const bool streamed = !dense && moe::use_streamed(B);
+  const bool streamed = !dense && (ep_size > 0 || moe::use_streamed(B));
+  ra.ep_rank = ep_rank;
+  ra.ep_size = ep_size;
   if (!moe::fused_routing(B) || streamed) {
     e = moe::launch_route(ra, s);
     if (e != cudaSuccess) return cuda_fail(e, "route launch");
@@ -131,6 +141,7 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   a.c = c;
   a.r = dense ? 0 : L->r;
   a.recovery_input = dense ? 0 : L->recovery_input;
+  a.ep_partial = ep_size > 0 ? 1 : 0;
   a.cs = 0;  // chosen at launch (16 when schedulable, else 8)
   a.nmax = B < moe::kMaxGroup ? B : moe::kMaxGroup;
   a.x = x;
@@ -164,6 +175,10 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   if (g_ev_before) cudaEventRecord(g_ev_before, s);
   e = dense ? moe::launch_dense(a, s) : streamed ? moe::launch_stream(a, s) : moe::launch_reader(a, s);
   if (e != cudaSuccess) return cuda_fail(e, dense ? "dense expert launch" : "reader launch");
+  if (ep_size > 0) {
+    e = moe::launch_ep_combine(B, L->top_e, L->d, ep_rank, ep_size, ws, y_partial, s);
+    if (e != cudaSuccess) return cuda_fail(e, "expert-parallel combine launch");
+  }
   if (g_ev_after) cudaEventRecord(g_ev_after, s);
   return MOE_OK;
 }
@@ -232,6 +247,25 @@ moe_status moe_reader_forward(const moe_reader_layer* layer, int B, int k, int c
                               const uint16_t* residual, uint16_t* y, const moe_reader_debug* dbg, void* workspace,
                               size_t ws_bytes, void* stream) {
   return run_forward(layer, B, k, c, x, residual, y, dbg, workspace, ws_bytes, stream, false);
+}
+
+moe_status moe_reader_forward_ep(const moe_reader_layer* layer, int B, int k, int c, const uint16_t* x, int ep_rank,
+                                 int ep_size, float* y_partial, const moe_reader_debug* dbg, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  REQUIRE(ep_size >= 1, "ep_size = %d must be >= 1", ep_size);
+  return run_forward(layer, B, k, c, x, nullptr, nullptr, dbg, workspace, ws_bytes, stream, false, ep_rank, ep_size,
+                     y_partial);
+}
+
+moe_status moe_reader_ep_finish(int B, int d, const float* y_sum, const uint16_t* residual, uint16_t* y,
+                                void* stream) {
+  REQUIRE(B >= 1 && B <= 256, "B = %d outside [1, 256]", B);
+  REQUIRE(d >= 1 && d <= 4096, "d = %d outside [1, 4096]", d);
+  REQUIRE_PTR(y_sum);
+  REQUIRE_PTR(y);
+  OPT_PTR(residual);
+  cudaError_t e = moe::launch_ep_finish(B, d, y_sum, residual, y, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "expert-parallel finish launch");
 }
 
 moe_status moe_reader_forward_dense(const moe_reader_layer* layer, int B, const uint16_t* x, const uint16_t* residual,

@@ -64,6 +64,7 @@ struct RouteArgs {
   int32_t* dbg_ids;
   float* dbg_w;
   bool quantize;  // also rotate + quantize the tokens (sparse path)
+  int ep_rank, ep_size;  // expert parallelism: pairs of experts e % ep_size == ep_rank only (ep_size 0/1: all)
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 
@@ -73,6 +74,7 @@ struct ExpertArgs {
   int nmax;          // max tokens per work item this launch
   int ring_rows;     // copy-ring row slots per warp (sparse) / rows (dense)
   int recovery_input;  // 0: ahat of every skipped channel; 1: exact a of dropped candidates
+  int ep_partial;      // 1: write the per-slot outputs only (no combine); expert-parallel steps
   const uint16_t* x;
   const uint16_t* w_router;  // routing inside the expert kernel (small B)
   const float* bias;
@@ -113,6 +115,12 @@ cudaError_t launch_stream(const ExpertArgs& a, cudaStream_t s);
 // cluster, 2: streamed; 0: automatic, streamed above two tokens).
 bool use_streamed(int B);
 void set_path(int path);
+// Expert parallelism: y_partial[b] = sum over the slots of b whose expert this
+// rank owns of w * y_e (fp32, slot order); y = bf16(y_sum + residual).
+cudaError_t launch_ep_combine(int B, int top_e, int d, int ep_rank, int ep_size, const Workspace& ws,
+                              float* y_partial, cudaStream_t s);
+cudaError_t launch_ep_finish(int B, int d, const float* y_sum, const uint16_t* residual, uint16_t* y,
+                             cudaStream_t s);
 cudaError_t launch_dense(const ExpertArgs& a, cudaStream_t s);
 void set_forced_cluster_size(int cs);
 cudaError_t query_plan(const ExpertArgs& a, bool dense, int out[4]);

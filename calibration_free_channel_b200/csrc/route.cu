@@ -218,12 +218,15 @@ __global__ void __launch_bounds__(512) select_kernel(RouteArgs a) {
     if (lane == 0) cnt[e] = c;
   }
   __syncthreads();
+  // experts this rank owns (expert parallelism); the pair table holds only theirs
+  auto owned = [&](int e) { return a.ep_size <= 1 || e % a.ep_size == a.ep_rank; };
   // exclusive prefixes over the experts: pairs, work items, active experts
   if (warp == 0) {
     int rp = 0, ri = 0, ra = 0;
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
-      const int c = e < E ? cnt[e] : 0, it = (c + kMaxGroup - 1) / kMaxGroup, ac = c > 0;
+      const int ca = e < E ? cnt[e] : 0, it = (ca + kMaxGroup - 1) / kMaxGroup;
+      const int c = e < E && owned(e) ? ca : 0, ac = c > 0;
       int ip = c, ii = it, ia = ac;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -258,6 +261,7 @@ __global__ void __launch_bounds__(512) select_kernel(RouteArgs a) {
   // each expert's pairs and work items, tokens ascending
   for (int e = warp; e < E; e += nwarp) {
     if (cnt[e] == 0) continue;
+    const bool own = owned(e);
     int run = 0;
     for (int t0 = 0; t0 < B; t0 += 32) {
       const int t = t0 + lane;
@@ -268,10 +272,12 @@ __global__ void __launch_bounds__(512) select_kernel(RouteArgs a) {
       const unsigned bal = __ballot_sync(0xffffffffu, slot >= 0);
       if (slot >= 0) {
         const int pos = run + __popc(bal & ((1u << lane) - 1u));
-        const int pr = pbase[e] + pos;
-        a.ws.pair_tok[pr] = t;
-        a.ws.pair_slot[pr] = slot;
-        a.ws.pair_ea[pr] = aidx[e];
+        if (own) {
+          const int pr = pbase[e] + pos;
+          a.ws.pair_tok[pr] = t;
+          a.ws.pair_slot[pr] = slot;
+          a.ws.pair_ea[pr] = aidx[e];
+        }
         const int item = ibase[e] + pos / kMaxGroup, g = pos % kMaxGroup;
         if (item < a.ws.max_items) {
           a.ws.item_tok[item * kMaxGroup + g] = t;

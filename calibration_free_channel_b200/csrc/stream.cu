@@ -292,7 +292,8 @@ __global__ void __launch_bounds__(kSelT) select_c_kernel(ExpertArgs a) {
   pdl_wait();
   __shared__ SelSmem sm;
   const int tid = threadIdx.x;
-  const int I = a.I, W = (I + 31) >> 5, P = a.B * a.top_e;
+  const int I = a.I, W = (I + 31) >> 5;
+  const int P = __ldcg(a.ws.act_off + __ldcg(a.ws.n_act));  // pairs of this step (this rank's, under EP)
 #pragma unroll 1
   for (int p = blockIdx.x; p < P; p += gridDim.x) {
     const float* sp = reinterpret_cast<const float*>(a.ws.sa + (size_t)p * I);
@@ -335,7 +336,8 @@ __global__ void __launch_bounds__(kSelT) select_k_kernel(ExpertArgs a, int nblk)
   pdl_wait();
   __shared__ SelSmem sm;
   const int tid = threadIdx.x;
-  const int I = a.I, W = (I + 31) >> 5, P = a.B * a.top_e, r = a.r;
+  const int I = a.I, W = (I + 31) >> 5, r = a.r;
+  const int P = __ldcg(a.ws.act_off + __ldcg(a.ws.n_act));  // pairs of this step (this rank's, under EP)
   const int zstride = (I + 15) / 16;
   const bool rec_exact = a.recovery_input == 1;
 #pragma unroll 1
@@ -734,6 +736,7 @@ __global__ void __launch_bounds__(kDThreads) down_kernel(ExpertArgs a) {
         if (a.dbg_y_expert) a.dbg_y_expert[off] = y;
       }
       __syncthreads();  // the CTA's outputs precede the releases below
+      if (a.ep_partial) continue;  // expert-parallel step: the per-slot outputs are the result
       if (tid < ng) {
         const int tok = __ldcg(a.ws.pair_tok + p0 + tg + tid);
         lastf[tid] = arrive_last(a.ws.counters + tok * kMaxCluster + sl, (unsigned)a.top_e);
@@ -792,7 +795,56 @@ cudaError_t launch_pdl(K kernel, int grid, int threads, size_t smem, cudaStream_
 
 size_t exact_smem(int d) { return (size_t)kXTok * (2 * d + 64); }
 
+// ------------------------------------------------- expert parallelism
+// y_partial[b][j] = sum over b's slots s whose expert this rank owns of
+// w[b][s] y_e[b][s][j], fp32 FMAs in slot order.
+__global__ void __launch_bounds__(256) ep_combine_kernel(int B, int top_e, int d, int ep_rank, int ep_size,
+                                                         Workspace ws, float* y_partial) {
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.y, j = blockIdx.x * 256 + threadIdx.x;
+  if (j >= d) return;
+  float acc = 0.0f;
+  for (int s = 0; s < top_e; s++) {
+    const int e = __ldcg(ws.ids + b * top_e + s);
+    if (e % ep_size != ep_rank) continue;
+    acc = fmaf(__ldcg(ws.wts + b * top_e + s), __ldcg(ws.ye + ((size_t)b * top_e + s) * d + j), acc);
+  }
+  y_partial[(size_t)b * d + j] = acc;
+}
+
+// y = bf16(y_sum + residual) after the ranks' partials are summed.
+__global__ void __launch_bounds__(256) ep_finish_kernel(int B, int d, const float* y_sum, const uint16_t* residual,
+                                                        uint16_t* y) {
+  const size_t o = (size_t)blockIdx.x * 256 + threadIdx.x;
+  if (o >= (size_t)B * d) return;
+  float v = y_sum[o];
+  if (residual) v += bf16f(residual[o]);
+  y[o] = f2bf16(v);
+}
+
 }  // namespace
+
+cudaError_t launch_ep_combine(int B, int top_e, int d, int ep_rank, int ep_size, const Workspace& ws,
+                              float* y_partial, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((d + 255) / 256, B);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, ep_combine_kernel, B, top_e, d, ep_rank, ep_size, ws, y_partial);
+}
+
+cudaError_t launch_ep_finish(int B, int d, const float* y_sum, const uint16_t* residual, uint16_t* y,
+                             cudaStream_t s) {
+  const size_t n = (size_t)B * d;
+  ep_finish_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(B, d, y_sum, residual, y);
+  return cudaGetLastError();
+}
 
 void set_path(int path) { g_path = path; }
 bool use_streamed(int B) { return g_path == 2 || (g_path == 0 && B > 2); }

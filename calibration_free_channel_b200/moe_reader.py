@@ -21,7 +21,7 @@ EXPORTS = ["moe_reader_workspace_bytes", "moe_reader_build_sketch", "moe_reader_
            "moe_reader_build_lowrank", "moe_reader_forward", "moe_reader_forward_dense",
            "moe_reader_forward_host", "moe_reader_rmsnorm", "moe_reader_set_expert_events",
            "moe_reader_check_error", "moe_reader_set_cluster_size", "moe_reader_set_path", "moe_reader_launch_plan",
-           "moe_reader_forward_noalloc", "moe_reader_last_error"]
+           "moe_reader_forward_noalloc", "moe_reader_forward_ep", "moe_reader_ep_finish", "moe_reader_last_error"]
 
 
 class MoeReaderLayer(C.Structure):
@@ -64,6 +64,9 @@ def lib():
         L.moe_reader_forward.argtypes = [C.POINTER(MoeReaderLayer), i32, i32, i32, P, P, P,
                                          C.POINTER(MoeReaderDebug), P, sz, P]
         L.moe_reader_forward_dense.argtypes = [C.POINTER(MoeReaderLayer), i32, P, P, P, P, sz, P]
+        L.moe_reader_forward_ep.argtypes = [C.POINTER(MoeReaderLayer), i32, i32, i32, P, i32, i32, P,
+                                            C.POINTER(MoeReaderDebug), P, sz, P]
+        L.moe_reader_ep_finish.argtypes = [i32, i32, P, P, P, P]
         L.moe_reader_forward_host.argtypes = [C.POINTER(MoeReaderLayer), i32, i32, i32, P, P, P, P, P, sz, P]
         L.moe_reader_rmsnorm.argtypes = [i32, i32, C.c_float, P, P, P]
         L.moe_reader_set_expert_events.argtypes = [P, P]
@@ -120,6 +123,17 @@ def moe_reader_build_sketch(E, I, d, w_gate, w_up, rot_seed, rot_sign, sk_gate, 
 def moe_reader_build_lowrank(E, I, d, r, w_down, u_sigma, v, workspace, ws_bytes, stream=None):
     _check(lib().moe_reader_build_lowrank(E, I, d, r, _ptr(w_down), _ptr(u_sigma), _ptr(v), _ptr(workspace),
                                           ws_bytes, _stream(stream)))
+
+
+def moe_reader_forward_ep(layer: MoeReaderLayer, B, k, c, x, ep_rank, ep_size, y_partial, dbg, workspace, ws_bytes,
+                          stream=None):
+    _check(lib().moe_reader_forward_ep(C.byref(layer), B, k, c, _ptr(x), ep_rank, ep_size, _ptr(y_partial),
+                                       C.byref(dbg) if dbg is not None else None, _ptr(workspace), ws_bytes,
+                                       _stream(stream)))
+
+
+def moe_reader_ep_finish(B, d, y_sum, residual, y, stream=None):
+    _check(lib().moe_reader_ep_finish(B, d, _ptr(y_sum), _ptr(residual), _ptr(y), _stream(stream)))
 
 
 def moe_reader_forward(layer: MoeReaderLayer, B, k, c, x, residual, y, dbg, workspace, ws_bytes, stream=None):
@@ -237,27 +251,38 @@ class Layer:
             self._ws = torch.zeros(nb, dtype=torch.uint8, device=self.w["w_gate"].device)
         return self._ws
 
+    def _debug(self, B, k, c, dev):
+        P = (B, self.top_e)
+        dbg_t = dict(ids=torch.empty(P, dtype=torch.int32, device=dev),
+                     weights=torch.empty(P, dtype=torch.float32, device=dev),
+                     dot_gate=torch.empty(P + (self.I,), dtype=torch.int32, device=dev),
+                     dot_up=torch.empty(P + (self.I,), dtype=torch.int32, device=dev),
+                     score=torch.empty(P + (self.I,), dtype=torch.float32, device=dev),
+                     cand=torch.empty(P + (c,), dtype=torch.int32, device=dev),
+                     kept=torch.empty(P + (k,), dtype=torch.int32, device=dev),
+                     a_kept=torch.empty(P + (k,), dtype=torch.float32, device=dev),
+                     y_expert=torch.empty(P + (self.d,), dtype=torch.float32, device=dev),
+                     phase_ns=torch.zeros((B * self.top_e, 16), dtype=torch.int64, device=dev))
+        return dbg_t, MoeReaderDebug(*[_ptr(dbg_t[n]) for n, _ in MoeReaderDebug._fields_])
+
+    def forward_ep(self, x, k: int, c: int, ep_rank: int, ep_size: int, debug: bool = False, r: int | None = None,
+                   stream=None, out=None, recovery_input: int = 0):
+        """This rank's fp32 partial of the block ([B, d]) over the experts
+        e % ep_size == ep_rank; sum it over the ranks, then ep_finish."""
+        B = x.shape[0]
+        ws = self.workspace(B)
+        yp = out if out is not None else torch.empty((B, self.d), dtype=torch.float32, device=x.device)
+        dbg_t, dbg = self._debug(B, k, c, x.device) if debug else (None, None)
+        moe_reader_forward_ep(self.struct(r, recovery_input), B, k, c, x, ep_rank, ep_size, yp, dbg, ws, ws.numel(),
+                              stream)
+        return (yp, dbg_t) if debug else yp
+
     def forward(self, x, k: int, c: int, residual=None, debug: bool = False, r: int | None = None, stream=None,
                 out=None, recovery_input: int = 0):
         B = x.shape[0]
         ws = self.workspace(B)
         y = out if out is not None else torch.empty_like(x)
-        dbg = None
-        dbg_t = None
-        if debug:
-            dev = x.device
-            P = (B, self.top_e)
-            dbg_t = dict(ids=torch.empty(P, dtype=torch.int32, device=dev),
-                         weights=torch.empty(P, dtype=torch.float32, device=dev),
-                         dot_gate=torch.empty(P + (self.I,), dtype=torch.int32, device=dev),
-                         dot_up=torch.empty(P + (self.I,), dtype=torch.int32, device=dev),
-                         score=torch.empty(P + (self.I,), dtype=torch.float32, device=dev),
-                         cand=torch.empty(P + (c,), dtype=torch.int32, device=dev),
-                         kept=torch.empty(P + (k,), dtype=torch.int32, device=dev),
-                         a_kept=torch.empty(P + (k,), dtype=torch.float32, device=dev),
-                         y_expert=torch.empty(P + (self.d,), dtype=torch.float32, device=dev),
-                         phase_ns=torch.zeros((B * self.top_e, 16), dtype=torch.int64, device=dev))
-            dbg = MoeReaderDebug(*[_ptr(dbg_t[n]) for n, _ in MoeReaderDebug._fields_])
+        dbg_t, dbg = self._debug(B, k, c, x.device) if debug else (None, None)
         moe_reader_forward(self.struct(r, recovery_input), B, k, c, x, residual, y, dbg, ws, ws.numel(), stream)
         return (y, dbg_t) if debug else y
 

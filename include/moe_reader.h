@@ -172,6 +172,28 @@ moe_status moe_reader_forward_dense(const moe_reader_layer* layer, int B, const 
                                     const uint16_t* residual, uint16_t* y, void* workspace,
                                     size_t ws_bytes, void* stream);
 
+/* Expert parallelism (one process per GPU, experts split by e % ep_size):
+ * the step of rank ep_rank over the experts it owns.  Routing is computed in
+ * full on every rank (the router is replicated); only the (token, slot)
+ * pairs whose expert this rank owns are read and computed, with the
+ * streamed kernels.  Writes y_partial[b] = sum over b's owned slots, in slot
+ * order, of w_slot * y_e (DEVICE, [B, d] fp32, 16-byte aligned; no residual,
+ * no rounding).  The caller sums y_partial over the ranks (e.g. one NCCL
+ * all-reduce) and calls moe_reader_ep_finish.  The per-pair debug outputs
+ * are written for owned pairs only.  Needs the layer's own weights for the
+ * owned experts at least (other experts' rows are never read).
+ * MOE_EINVAL unless 1 <= ep_size <= E and 0 <= ep_rank < ep_size. */
+moe_status moe_reader_forward_ep(const moe_reader_layer* layer, int B, int k, int c,
+                                 const uint16_t* x, int ep_rank, int ep_size, float* y_partial,
+                                 const moe_reader_debug* dbg, void* workspace, size_t ws_bytes,
+                                 void* stream);
+
+/* y = bf16(y_sum + residual) (round to nearest even), [B, d]: the last step
+ * of an expert-parallel block after the partials are summed.  residual may
+ * be NULL; DEVICE pointers. */
+moe_status moe_reader_ep_finish(int B, int d, const float* y_sum, const uint16_t* residual,
+                                uint16_t* y, void* stream);
+
 /* moe_reader_forward with HOST input and output: copies x_host (pinned,
  * [B, d] bf16) into x_dev, runs the step, copies y_dev back into y_host
  * (pinned), all enqueued on `stream`.  The caller synchronizes. */
