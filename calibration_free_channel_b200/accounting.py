@@ -29,6 +29,22 @@ def expert_bytes(I: int, d: int, r: int, n_cand_rows: int, n_kept_rows: int) -> 
                 total=sketch + cand + down + lowrank)
 
 
+def sketch_row_bytes(d: int, packing: str = "2bit") -> int:
+    """Bytes of one resident sketch row: 2-bit codes (d / 4), or base 3 with
+    five trits per byte, ceil(d / 5) bytes rounded up to whole sectors."""
+    if packing == "2bit":
+        return d // 4
+    if packing == "base3":
+        return -(-((d + 4) // 5) // SECTOR) * SECTOR
+    raise ValueError(packing)
+
+
+def sketch_footprint(I: int, d: int, packing: str = "2bit") -> float:
+    """Resident sketch of one expert (gate and up rows plus alpha) as a
+    fraction of its BF16 gate, up and down weights."""
+    return (2 * I * sketch_row_bytes(d, packing) + 2 * I * 4) / dense_expert_bytes(I, d)
+
+
 def dense_expert_bytes(I: int, d: int) -> int:
     return 3 * I * d * 2
 

@@ -11,13 +11,17 @@
 //   select_c_kernel   one pair per CTA: top-c by sigma; the expert's last pair
 //                     forms the candidate union (rows of the next stage)
 //   exact_kernel      16 union rows of one expert per unit: g, u of every
-//                     token of the expert, a = silu(g) u for its candidates
+//                     token of the expert on the tensor cores (mma.sync bf16),
+//                     a = silu(g) u for its candidates
 //   select_k_kernel   one pair per CTA: top-k by |a| over its candidates, the
 //                     recovery input z; the expert's last pair forms the kept
 //                     union and the per-pair row coefficients
 //   down_kernel       one (expert, column slice) per unit: kept down rows,
 //                     V z, and the combine over the top-e slots by the last
 //                     arriving slot of each (token, slice)
+// Expert-parallel steps (one rank's experts) skip that combine; then
+// ep_combine_kernel sums the rank's slots per token into an fp32 partial and,
+// after the caller's all-reduce, ep_finish_kernel adds the residual and rounds.
 // Each kernel is launched with programmatic dependent launch and waits on
 // its predecessor before reading its outputs; weights are read with
 // non-allocating loads, data written by earlier kernels of the chain through

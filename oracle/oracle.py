@@ -56,6 +56,8 @@ def lib():
         L.orc_rotate_quantize.argtypes = [i32, P, P, P, P, P]
         L.orc_twn_row.argtypes = [i32, P, P, P, P, P]
         L.orc_pack_trits.argtypes = [i32, P, P]
+        L.orc_pack_trits_base3.argtypes = [i32, P, P]
+        L.orc_unpack_trits_base3.argtypes = [i32, P, P]
         L.orc_unpack_trit.restype = i32
         L.orc_unpack_trit.argtypes = [P, i32]
         L.orc_build_sketch.argtypes = [i32, i32, i32, P, P, u64, P, P, P, P, P]
@@ -144,6 +146,21 @@ def pack_trits(trits: np.ndarray) -> np.ndarray:
     trits = np.ascontiguousarray(trits, np.int8)
     out = np.empty(trits.size // 16, np.uint32)
     lib().orc_pack_trits(trits.size, _p(trits), _p(out))
+    return out
+
+
+def pack_trits_base3(trits: np.ndarray) -> np.ndarray:
+    """Five trits per byte (ceil(d / 5) bytes per row)."""
+    trits = np.ascontiguousarray(trits, np.int8)
+    out = np.empty((trits.size + 4) // 5, np.uint8)
+    lib().orc_pack_trits_base3(trits.size, _p(trits), _p(out))
+    return out
+
+
+def unpack_trits_base3(packed: np.ndarray, d: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, np.uint8)
+    out = np.empty(d, np.int8)
+    lib().orc_unpack_trits_base3(d, _p(packed), _p(out))
     return out
 
 
