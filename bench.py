@@ -37,6 +37,17 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-block µs/step & achieved HBM GB/s (vs ~8 TB/s) at k/I≈18%, batch 1–16"
 
 
+def launches_per_step(B: int, path: int) -> int:
+    """Kernel launches of one sparse step: the one-cluster reader routes inside
+    its kernel at B <= 2 (one launch) and after the route and select kernels
+    above (three); the streamed reader is route, select and five stage
+    kernels."""
+    streamed = path == 2 or (path == 0 and B > 2)
+    if streamed:
+        return 7
+    return 1 if B <= 2 else 3
+
+
 def workload_name(B: int) -> str:
     return f"qwen3_30b_a3b_layer_b{B}"
 
@@ -345,7 +356,7 @@ def run_native(args, rank, world, local_rank):
         "step_roofline_frac": round(value / world / peak, 4),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": B * shape.d * 2,
                 "d2h_bytes_per_step": B * shape.d * 2, "us_per_step": float(t[0]) * 1e3},
-        "gpu_launches": (1 if B <= 2 else 3) * nsteps,  # in-kernel routing at B <= 2
+        "gpu_launches": launches_per_step(B, args.path) * nsteps,
         "clocks": clocks,
         "dense": dense,
         "recovery_exact_input": variant,
