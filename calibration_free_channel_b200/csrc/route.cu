@@ -1,5 +1,8 @@
 // route.cu -- router logits, rotation + int8 quantisation, top-e selection
-// and the per-step work table.
+// and the per-step tables: work items of up to two tokens (one-cluster and
+// dense kernels) and the active experts with their (token, slot) pairs in
+// expert order (streamed kernels; under expert parallelism only the experts
+// e % ep_size == ep_rank).
 //
 // Routing follows the pages' "routed experts" (abstract of "Channel Selection
 // for Mixture-of-Experts Decoding Needs No Calibration Data"): softmax routing
