@@ -30,6 +30,23 @@ def test_header_declares_the_binding_names():
     assert declared_functions() == sorted(M.EXPORTS)
 
 
+def declared_arity():
+    """Parameter count of every moe_reader_* prototype in the header."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(moe_reader_\w+)\s*\(([^)]*)\)\s*;", src):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argtypes_match_the_prototypes(lib):
+    arity = declared_arity()
+    assert sorted(arity) == declared_functions()
+    for name, n in arity.items():
+        assert len(getattr(lib, name).argtypes or []) == n, name
+
+
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
