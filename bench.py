@@ -37,15 +37,12 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-block µs/step & achieved HBM GB/s (vs ~8 TB/s) at k/I≈18%, batch 1–16"
 
 
-def launches_per_step(B: int, path: int) -> int:
-    """Kernel launches of one sparse step: the one-cluster reader routes inside
-    its kernel at B <= 2 (one launch) and after the route and select kernels
-    above (three); the streamed reader is route, select and five stage
-    kernels."""
-    streamed = path == 2 or (path == 0 and B > 2)
-    if streamed:
-        return 7
-    return 1 if B <= 2 else 3
+def launches_per_step(B: int, path: int, d: int = 2048) -> int:
+    """Kernel launches of one sparse step: the one-cluster reader (B <= 2,
+    d <= 2048) routes inside its one kernel; the streamed reader is the route
+    and select kernels and five stage kernels."""
+    cluster = path == 1 or (path == 0 and B <= 2 and d <= 2048)
+    return 1 if cluster else 7
 
 
 def workload_name(B: int) -> str:
@@ -62,6 +59,7 @@ def parse():
     p.add_argument("--k", type=int, default=136)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense", action="store_true")
+    p.add_argument("--no-sweep", action="store_true", help="skip the batch and skewed-routing sweeps")
     p.add_argument("--layers", type=int, default=32, help="distinct device copies of the layer the steps cycle through")
     p.add_argument("--path", type=int, default=0, choices=[0, 1, 2],
                    help="sparse reader: 0 automatic, 1 one cluster per expert, 2 streamed kernels")
@@ -146,7 +144,6 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ native
 def run_native(args, rank, world, local_rank):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -155,11 +152,11 @@ def run_native(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    M.moe_reader_set_path(args.path)
     shape = synth.QWEN3_30B_A3B
     B, k, c, r = args.batch, args.k, 2 * args.k, 32
     W = synth.layer_weights(shape, seed=0, device=str(dev))
     layer = M.Layer(W, top_e=shape.top_e, device=dev).build_sketch(synth.rot_seed(0)).build_lowrank(r)
+    layer.path = args.path
     # distinct device copies of the layer (same values, separate memory): the
     # timed steps cycle through them so the working set is far above the L2
     layers = [layer] + [replicate(layer) for _ in range(max(1, args.layers) - 1)]
@@ -167,17 +164,29 @@ def run_native(args, rank, world, local_rank):
     ntok = 20
     toks = [synth.tokens(shape.d, B, seed=1000 * rank + s) for s in range(ntok)]
     xs = [t.to(dev) for t in toks]
-    y = torch.empty_like(xs[0])
+    y_bufs = {}
 
-    # algorithmic bytes of each token's step (exact sector accounting of the
-    # rows the reader reads, from its own debug outputs; untimed)
-    step_bytes = []
-    for x in xs:
-        _, dbg = layer.forward(x, k=k, c=c, debug=True)
-        ids, cand, kept = (dbg[n].cpu().numpy() for n in ("ids", "cand", "kept"))
-        step_bytes.append(accounting.step_bytes(shape.E, shape.I, shape.d, r, ids, cand, kept)["total"])
-    layer.check()
-    expert_bytes = [b - accounting.router_bytes(shape.E, shape.d, False) for b in step_bytes]
+    def out_buf(Bq):
+        if Bq not in y_bufs:
+            y_bufs[Bq] = torch.empty((Bq, shape.d), dtype=torch.bfloat16, device=dev)
+        return y_bufs[Bq]
+
+    def step_accounting(lays, xq, kq, cq):
+        """Algorithmic bytes of each token set's sparse step and of the dense
+        block on the same routing (exact sector accounting of the rows the
+        reader reads, from its own debug outputs; untimed)."""
+        sb, db = [], []
+        bias = lays[0].w.get("router_bias") is not None
+        for x in xq:
+            _, dbg = lays[0].forward(x, k=kq, c=cq, debug=True)
+            ids, cand, kept = (dbg[n].cpu().numpy() for n in ("ids", "cand", "kept"))
+            acc = accounting.step_bytes(shape.E, shape.I, shape.d, r, ids, cand, kept, bias=bias)
+            sb.append(acc["total"])
+            db.append(acc["dense"])
+        lays[0].check()
+        return sb, db
+
+    step_bytes, dense_bytes = step_accounting(layers, xs, k, c)
 
     # L2 flush between timed steps: READ a buffer of twice the L2 size, so the
     # L2 holds only clean lines afterwards (a write-flush would leave ~L2-size
@@ -186,12 +195,8 @@ def run_native(args, rank, world, local_rank):
     flush_buf = torch.ones(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
     flush_out = torch.empty((), dtype=torch.float32, device=dev)
 
-    class _Flush:
-        @staticmethod
-        def zero_():
-            torch.sum(flush_buf, dim=0, out=flush_out)
-
-    flush = _Flush()
+    def flush():
+        torch.sum(flush_buf, dim=0, out=flush_out)
 
     def barrier():
         if world > 1:
@@ -202,10 +207,12 @@ def run_native(args, rank, world, local_rank):
     spin_cycles = int(2.0e9 * chunk * 150e-6)  # ~150 us of host time per step, at up to 2 GHz
 
     def time_loop(fn, steps, warmup, kernel_events=False, flushed=False):
+        """One event pair around every step (and, with kernel_events, one
+        around the step's expert kernels inside the library)."""
         for i in range(warmup):
             if flushed:
-                flush.zero_()
-            fn(i)
+                flush()
+            fn(i, None)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)] \
             if kernel_events else None
@@ -214,68 +221,72 @@ def run_native(args, rank, world, local_rank):
                 a_.record()
                 b_.record()
         barrier()
-        with ClockSampler(local_rank) as cs:
-            for i in range(steps):
-                if i % chunk == 0:
-                    # a device-side spin ahead of each chunk of steps: the host
-                    # queues the whole chunk before the GPU reaches it, so the
-                    # per-step events time the device, not the Python launch path
-                    torch.cuda._sleep(spin_cycles)
-                if flushed:
-                    flush.zero_()
-                if kev:
-                    M.moe_reader_set_expert_events(kev[i][0], kev[i][1])
-                ev[i][0].record()
-                fn(i)
-                ev[i][1].record()
-            barrier()
-        M.moe_reader_set_expert_events(None, None)
+        for i in range(steps):
+            if i % chunk == 0:
+                # a device-side spin ahead of each chunk of steps: the host
+                # queues the whole chunk before the GPU reaches it, so the
+                # per-step events time the device, not the Python launch path
+                torch.cuda._sleep(spin_cycles)
+            if flushed:
+                flush()
+            ev[i][0].record()
+            fn(i, kev[i] if kev else None)
+            ev[i][1].record()
+        barrier()
         per = [a.elapsed_time(b) for a, b in ev]
         kper = [a.elapsed_time(b) for a, b in kev] if kev else None
-        return per, kper, cs.summary()
+        return per, kper
 
-    def chunk_loop(fn, steps, warmup):
-        """Back-to-back steps timed per chunk of `chunk` steps (one event pair
-        per chunk, a device spin ahead of it so the host has queued the whole
-        chunk): nothing but the steps' own kernels runs between the events, so
-        consecutive launches overlap as they do in a decode loop.  Returns the
-        mean time per step of each chunk (ms)."""
+    def chunk_loop(fn, steps, warmup, sample_clocks=False):
+        """Exactly `steps` back-to-back steps, timed per chunk of at most
+        `chunk` steps (one event pair per chunk, a device spin ahead of it so
+        the host has queued the whole chunk): nothing but the steps' own
+        kernels runs between the events, so consecutive launches overlap as
+        they do in a decode loop.  Returns the mean time per step (ms) and the
+        clocks sampled during the timed region."""
         for i in range(warmup):
             fn(i)
-        nch = max(1, steps // chunk)
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nch)]
+        sizes = [chunk] * (steps // chunk) + ([steps % chunk] if steps % chunk else [])
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in sizes]
         barrier()
-        with ClockSampler(local_rank) as cs:
-            for q in range(nch):
-                torch.cuda._sleep(spin_cycles)
-                ev[q][0].record()
-                for i in range(q * chunk, (q + 1) * chunk):
-                    fn(i)
-                ev[q][1].record()
-            barrier()
-        return [a.elapsed_time(b) / chunk for a, b in ev], nch * chunk, cs.summary()
+        cs = ClockSampler(local_rank) if sample_clocks else None
+        if cs:
+            cs.__enter__()
+        i = 0
+        for q, n in enumerate(sizes):
+            torch.cuda._sleep(spin_cycles)
+            ev[q][0].record()
+            for _ in range(n):
+                fn(i)
+                i += 1
+            ev[q][1].record()
+        barrier()
+        if cs:
+            cs.__exit__(None, None, None)
+        total = sum(a.elapsed_time(b) for a, b in ev)
+        return total / steps, (cs.summary() if cs else None)
 
-    def sparse_step(j):
-        layers[j % nlay].forward(xs[j % ntok], k=k, c=c, out=y)
+    def max_over_ranks(*vals):
+        t = torch.tensor(vals, dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return [float(v) for v in t]
 
-    def sparse_step_one_layer(j):
-        layer.forward(xs[j % ntok], k=k, c=c, out=y)
+    # ---------------------------------------------------- the headline step
+    def sparse_step(j, ev=None):
+        layers[j % nlay].forward(xs[j % ntok], k=k, c=c, out=out_buf(B), events=ev)
 
-    per, nsteps, clocks = chunk_loop(sparse_step, args.steps, args.warmup)
-    # the expert launch alone (events right around it inside the library): it
-    # separates the kernel from the step, at the cost of the launch overlap
-    _, kper, _ = time_loop(sparse_step, max(64, args.steps // 8), args.warmup, kernel_events=True)
-    fper, fkper, _ = time_loop(sparse_step_one_layer, max(50, args.steps // 4), args.warmup, kernel_events=True,
-                               flushed=True)
-    ms = statistics.mean(per)
-    kms = statistics.mean(kper)
-    mean_bytes = statistics.mean(step_bytes[i % ntok] for i in range(nsteps))
-    mean_ebytes = statistics.mean(expert_bytes[i % ntok] for i in range(nsteps))
-    # max over ranks
-    t = torch.tensor([ms, kms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max, kms_max = float(t[0]), float(t[1])
+    def sparse_step_one_layer(j, ev=None):
+        layer.forward(xs[j % ntok], k=k, c=c, out=out_buf(B), events=ev)
+
+    K = args.steps
+    ms, clocks = chunk_loop(sparse_step, K, args.warmup, sample_clocks=True)
+    # the expert kernels alone (events right around them inside the library):
+    # they separate the kernels from the step, at the cost of the launch overlap
+    _, kper = time_loop(sparse_step, max(64, K // 8), args.warmup, kernel_events=True)
+    fper, fkper = time_loop(sparse_step_one_layer, max(64, K // 8), args.warmup, kernel_events=True, flushed=True)
+    mean_bytes = statistics.mean(step_bytes[i % ntok] for i in range(K))
+    ms_max, kms_max = max_over_ranks(ms, statistics.mean(kper))
     value = world * mean_bytes / (ms_max * 1e-3) / 1e9
 
     # end to end through the host-buffer C-ABI call: H2D x, step, D2H y
@@ -286,45 +297,86 @@ def run_native(args, rank, world, local_rank):
     ws = layer.workspace(B)
     sts = [lay.struct() for lay in layers]
 
-    def e2e_step(j):
+    def e2e_step(j, ev=None):
         M.moe_reader_forward_host(sts[j % nlay], B, k, c, xh[j % ntok], xd, yd, yh, ws, ws.numel())
 
-    e2e_steps = max(50, args.steps // 4)
-    eper, _, _ = time_loop(e2e_step, e2e_steps, args.warmup)
-    ems = statistics.mean(eper)
-    t = torch.tensor([ems], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_value = world * mean_bytes / (float(t[0]) * 1e-3) / 1e9
+    eper, _ = time_loop(e2e_step, max(64, K // 4), args.warmup)
+    (ems,) = max_over_ranks(statistics.mean(eper))
+    e2e_value = world * mean_bytes / (ems * 1e-3) / 1e9
 
+    peak, peak_kind = measured_peaks()
     dense = None
     if not args.no_dense:
         def dense_step(j):
-            layers[j % nlay].forward_dense(xs[j % ntok], out=y)
-        dper, _, _ = chunk_loop(dense_step, max(64, args.steps // 4), args.warmup)
-        dms = statistics.mean(dper)
-        dbytes = accounting.router_bytes(shape.E, shape.d, False) + \
-            shape.top_e * B * accounting.dense_expert_bytes(shape.I, shape.d) if B == 1 else None
-        dense = {"us_per_step": dms * 1e3, "speedup_of_sparse": dms / ms,
-                 "achieved_gbs": (dbytes / (dms * 1e-3) / 1e9) if dbytes else None}
+            layers[j % nlay].forward_dense(xs[j % ntok], out=out_buf(B))
+        dms, _ = chunk_loop(dense_step, max(64, K), args.warmup)
+        (dms,) = max_over_ranks(dms)
+        dmean = statistics.mean(dense_bytes)
+        dense = {"us_per_step": dms * 1e3, "speedup_of_sparse": dms / ms_max,
+                 "achieved_gbs": dmean / (dms * 1e-3) / 1e9, "bytes_per_step": dmean,
+                 "hbm_bound_us": dmean / (peak * 1e9) * 1e6,
+                 "note": "this build's all-channel block on the same weights and routing"}
     # the exact-input recovery (dropped candidates enter V z with their exact
-    # a): same bytes, the down stage walks every candidate
+    # a): same bytes
     variant = None
     if r > 0:
         def variant_step(j):
-            layers[j % nlay].forward(xs[j % ntok], k=k, c=c, out=y, recovery_input=1)
-        vper, _, _ = chunk_loop(variant_step, max(64, args.steps // 4), args.warmup)
-        variant = {"us_per_step": statistics.mean(vper) * 1e3}
+            layers[j % nlay].forward(xs[j % ntok], k=k, c=c, out=out_buf(B), recovery_input=1)
+        vms, _ = chunk_loop(variant_step, max(64, K), args.warmup)
+        variant = {"us_per_step": vms * 1e3}
     layer.check()
 
-    peak, peak_kind = measured_peaks()
-    # At B <= 2 the expert kernel routes in-kernel: it is the step's only
-    # kernel and reads the router too, so a launch's bytes are the step's and
-    # its average duration in the back-to-back chunks is the step time.  At
-    # larger B the route/select kernels run first; the expert kernel's share
-    # is timed with events right around its launch.
+    # ------------------------------------------------ batch sweeps (extra keys)
+    def sweep(lays, batches, kq, seed0, with_dense=True):
+        res = {}
+        for Bq in batches:
+            xq = [synth.tokens(shape.d, Bq, seed=seed0 + 100 * Bq + s).to(dev) for s in range(8)]
+            sb, db = step_accounting(lays, xq, kq, 2 * kq)
+            yq = out_buf(Bq)
+
+            def sp(j, xq=xq, yq=yq):
+                lays[j % len(lays)].forward(xq[j % len(xq)], k=kq, c=2 * kq, out=yq)
+
+            sms, _ = chunk_loop(sp, 64, 4)
+            (sms,) = max_over_ranks(sms)
+            ent = {"sparse_us": sms * 1e3, "sparse_gbs": statistics.mean(sb) / (sms * 1e-3) / 1e9,
+                   "sparse_bytes": statistics.mean(sb), "sparse_hbm_bound_us": statistics.mean(sb) / (peak * 1e9) * 1e6}
+            if with_dense:
+                def dn(j, xq=xq, yq=yq):
+                    lays[j % len(lays)].forward_dense(xq[j % len(xq)], out=yq)
+                dms_, _ = chunk_loop(dn, 64, 4)
+                (dms_,) = max_over_ranks(dms_)
+                ent.update(dense_us=dms_ * 1e3, dense_bytes=statistics.mean(db),
+                           dense_hbm_bound_us=statistics.mean(db) / (peak * 1e9) * 1e6,
+                           speedup_vs_dense=dms_ / sms)
+            res[f"B{Bq}"] = ent
+            lays[0].check()
+        return res
+
+    batch_sweep = skewed_sweep = None
+    if not args.no_sweep:
+        batch_sweep = {"k": k, "c": c, "note": "budget/batch sweep of the same layer (8 token sets per batch, "
+                                                 "64 back-to-back steps, steps cycle through the layer copies)"}
+        batch_sweep.update(sweep(layers, (4, 16), k, 5000 + 1000 * rank))
+        if args.k == 136:
+            batch_sweep["k100"] = sweep(layers, (1, 4, 8, 16), 100, 7000 + 1000 * rank, with_dense=False)
+        # skewed routing prior: the same weights with a per-expert logit bias ~ N(0, 1)
+        bias = synth.router_bias(shape, seed=1).to(dev)
+        skewed = []
+        for lay in layers:
+            sl = replicate_view(lay)
+            sl.w["router_bias"] = bias
+            skewed.append(sl)
+        skewed_sweep = {"k": k, "c": c, "note": "router logit bias ~ N(0,1) per expert; sparse vs this build's "
+                                                  "dense block on the same weights"}
+        skewed_sweep.update(sweep(skewed, (1, 8, 16, 32, 64), k, 9000 + 1000 * rank))
+
     fused = B <= 2 and args.path != 2
-    launch_bytes = mean_bytes if fused else mean_ebytes
+    # At B <= 2 the reader routes in-kernel: it is the step's only kernel and
+    # reads the router too, so a launch's bytes are the step's and its average
+    # duration in the back-to-back chunks is the step time.  Above, the
+    # streamed kernels' share is timed with events right around them.
+    launch_bytes = mean_bytes if fused else mean_bytes - accounting.router_bytes(shape.E, shape.d, False)
     launch_ms = ms_max if fused else kms_max
     achieved = launch_bytes / (launch_ms * 1e-3) / 1e9
     out = {
@@ -332,7 +384,7 @@ def run_native(args, rank, world, local_rank):
         "value": round(value, 2),
         "unit": "GB/s",
         "n_gpus": world,
-        "steps": nsteps,
+        "steps": K,
         "warmup": args.warmup,
         "ms_per_step": ms_max,
         "us_per_step": ms_max * 1e3,
@@ -349,23 +401,34 @@ def run_native(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "kernel": "reader_kernel" if fused else "streamed kernels (screen .. down)",
                      "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
+                     "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json), burst copy",
                      "bytes_per_launch": launch_bytes, "launch_us": launch_ms * 1e3,
                      "isolated_launch_us": kms_max * 1e3,
                      "traffic": profiled_traffic("reader_kernel", workload_name(B)) if fused else None},
         "step_roofline_frac": round(value / world / peak, 4),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": B * shape.d * 2,
-                "d2h_bytes_per_step": B * shape.d * 2, "us_per_step": float(t[0]) * 1e3},
-        "gpu_launches": launches_per_step(B, args.path) * nsteps,
+                "d2h_bytes_per_step": B * shape.d * 2, "us_per_step": ems * 1e3},
+        "gpu_launches": launches_per_step(B, args.path) * K,
         "clocks": clocks,
         "dense": dense,
         "recovery_exact_input": variant,
         "l2_flush": {"us_per_step": statistics.mean(fper) * 1e3, "kernel_us": statistics.mean(fkper) * 1e3,
                      "note": "one layer, L2 flushed before every step (also evicts the kernel code)"},
+        "batch_sweep": batch_sweep,
+        "skewed_sweep": skewed_sweep,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(W, toks[:4], k, c, r, shape, budget_s=15.0)
+        out["cpu_baseline"] = cpu_baseline(W, toks[:4], k, c, r, shape, budget_s=12.0)
     return out
+
+
+def replicate_view(layer):
+    """A second descriptor of the same device tensors (its own weight dict)."""
+    import copy
+    L = copy.copy(layer)
+    L.w = dict(layer.w)
+    L._ws = None
+    return L
 
 
 def replicate(layer):
@@ -400,7 +463,7 @@ def _oracle_setup(W_host, shape, r, toks, rot_seed):
     return sk, lr
 
 
-def _oracle_time(W_host, sk, lr, toks, k, c, r, shape, budget_s):
+def _oracle_time(W_host, sk, lr, toks, k, c, r, shape, budget_s, threads=1, max_steps=200):
     from calibration_free_channel_b200 import accounting
     from oracle import oracle as O
     n = 0
@@ -408,23 +471,37 @@ def _oracle_time(W_host, sk, lr, toks, k, c, r, shape, budget_s):
     t0 = time.perf_counter()
     while True:
         x = toks[n % len(toks)]
-        _, _, dbg = O.forward(x, W_host, sk, lr, k=k, c=c, r=r, top_e=shape.top_e, debug=True)
-        nbytes += accounting.step_bytes(shape.E, shape.I, shape.d, r, dbg["ids"], dbg["cand"], dbg["kept"])["total"]
+        _, _, dbg = O.forward(x, W_host, sk, lr, k=k, c=c, r=r, top_e=shape.top_e, debug=True, threads=threads)
+        nbytes += accounting.step_bytes(shape.E, shape.I, shape.d, r, dbg["ids"], dbg["cand"], dbg["kept"],
+                                        bias=W_host.get("router_bias") is not None)["total"]
         n += 1
         el = time.perf_counter() - t0
-        if el >= budget_s or n >= 200:
+        if el >= budget_s or n >= max_steps:
             return n, nbytes, el
 
 
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def cpu_baseline(W, toks, k, c, r, shape, budget_s):
+    """The oracle on the host cores: its OpenMP variant over (token, slot)
+    pairs on every core (the reported value), and single-threaded."""
     W_host = {n: (v.cpu() if v is not None else None) for n, v in W.items()}
     from calibration_free_channel_b200 import synth
     sk, lr = _oracle_setup(W_host, shape, r, toks, synth.rot_seed(0))
-    n, nbytes, el = _oracle_time(W_host, sk, lr, toks, k, c, r, shape, budget_s)
-    return {"value": round(nbytes / el / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+    cores = host_cores()
+    n, nbytes, el = _oracle_time(W_host, sk, lr, toks, k, c, r, shape, budget_s, threads=cores)
+    n1, nb1, el1 = _oracle_time(W_host, sk, lr, toks, k, c, r, shape, budget_s / 2, threads=1)
+    return {"value": round(nbytes / el / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
             "us_per_step": el / n * 1e6,
-            "sample": f"{n} decode steps of the same layer and tokens, single-threaded plain C oracle "
-                      f"(fp64 exact stage; sketch/SVD build excluded), {el:.1f} s"}
+            "sample": f"{n} decode steps of the same layer and tokens, plain C oracle with its (token, slot) "
+                      f"readers on {cores} OpenMP threads (fp64 exact stage; sketch/SVD build excluded), {el:.1f} s",
+            "single_thread": {"value": round(nb1 / el1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                              "us_per_step": el1 / n1 * 1e6, "sample": f"{n1} decode steps, {el1:.1f} s"}}
 
 
 def run_reference(args, rank, world):
@@ -437,21 +514,23 @@ def run_reference(args, rank, world):
     W = synth.layer_weights(shape, seed=0)
     toks = [synth.tokens(shape.d, B, seed=s) for s in range(4)]
     sk, lr = _oracle_setup(W, shape, r, toks, synth.rot_seed(0))
-    # each step: one whole decode step of the oracle; the run stops after K
-    # steps or a 120 s budget, whichever comes first (a bounded sample)
+    cores = host_cores()
+    # each step: one whole decode step of the oracle on every core; the run
+    # stops after K steps or a 120 s budget, whichever comes first (a bounded
+    # sample)
     for w in range(min(args.warmup, 2)):
-        _oracle_time(W, sk, lr, toks[w % 4:w % 4 + 1], k, c, r, shape, 0.0)
+        _oracle_time(W, sk, lr, toks[w % 4:w % 4 + 1], k, c, r, shape, 0.0, threads=cores)
     tot_n = tot_b = 0
     tot_t = 0.0
     while tot_n < args.steps and tot_t < 120.0:
-        n, nb, el = _oracle_time(W, sk, lr, toks[tot_n % 4:tot_n % 4 + 1], k, c, r, shape, 0.0)
+        n, nb, el = _oracle_time(W, sk, lr, toks[tot_n % 4:tot_n % 4 + 1], k, c, r, shape, 0.0, threads=cores)
         tot_n, tot_b, tot_t = tot_n + n, tot_b + nb, tot_t + el
     value = tot_b / tot_t / 1e9
-    cb = {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-          "sample": f"{tot_n} decode steps (of {args.steps} asked, 120 s cap), single-threaded plain C oracle, "
-                    f"tokens 0-3; sketch/SVD build excluded"}
+    cb = {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+          "sample": f"{tot_n} decode steps (of {args.steps} asked, 120 s cap), plain C oracle on {cores} OpenMP "
+                    f"threads, tokens 0-3; sketch/SVD build excluded"}
     return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / tot_n * 1e3,
+            "steps": tot_n, "warmup": args.warmup, "ms_per_step": tot_t / tot_n * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64/f32 (oracle)",
             "data": "synthetic", "config": {"workload": workload_name(B), "batch": B, "k": k, "c": c, "r": r},
             "cpu_baseline": cb,

@@ -13,7 +13,6 @@
 namespace {
 
 thread_local std::string g_err;
-thread_local cudaEvent_t g_ev_before = nullptr, g_ev_after = nullptr;
 
 moe_status fail(moe_status st, const char* fmt, ...) {
   char buf[512];
@@ -57,6 +56,8 @@ moe_status check_shape(int B, int E, int top_e, int I, int d) {
 
 moe_status check_layer(const moe_reader_layer* L, bool sparse) {
   REQUIRE(L != nullptr, "layer is NULL");
+  REQUIRE(L->cluster_size == 0 || (L->cluster_size >= 2 && L->cluster_size <= 16),
+          "cluster_size = %d: use 0 (automatic) or 2 .. 16", L->cluster_size);
   REQUIRE_PTR(L->w_router);
   OPT_PTR(L->router_bias);
   REQUIRE_PTR(L->w_gate);
@@ -69,6 +70,8 @@ moe_status check_layer(const moe_reader_layer* L, bool sparse) {
     REQUIRE_PTR(L->alpha_gate);
     REQUIRE_PTR(L->alpha_up);
     REQUIRE(L->recovery_input == 0 || L->recovery_input == 1, "recovery_input = %d: use 0 or 1", L->recovery_input);
+    REQUIRE(L->path >= 0 && L->path <= 2, "path = %d: use 0 (automatic), 1 (one cluster per expert) or 2 (streamed)",
+            L->path);
     REQUIRE(L->r >= 0 && L->r <= 128 && L->r % 8 == 0 && L->r <= L->I, "r = %d: need r in {0, 8, ..., 128}, r <= I",
             L->r);
     if (L->r > 0) {
@@ -80,10 +83,12 @@ moe_status check_layer(const moe_reader_layer* L, bool sparse) {
 }
 
 // ep_size > 0: expert-parallel step of rank ep_rank; writes y_partial (fp32)
-// instead of y.
+// instead of y.  clear_counters: after validation, before any launch, zero
+// the workspace's combine counters (the noalloc entry's shared scratch).
 moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uint16_t* x, const uint16_t* residual,
                        uint16_t* y, const moe_reader_debug* dbg, void* workspace, size_t ws_bytes, void* stream,
-                       bool dense, int ep_rank = 0, int ep_size = 0, float* y_partial = nullptr) {
+                       bool dense, int ep_rank = 0, int ep_size = 0, float* y_partial = nullptr,
+                       bool clear_counters = false) {
   moe_status st = check_layer(L, !dense);
   if (st != MOE_OK) return st;
   st = check_shape(B, L->E, L->top_e, L->I, L->d);
@@ -105,9 +110,17 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   const int sI = dense ? 0 : L->I, sr = dense ? 0 : L->r;
   const size_t need = moe::workspace_layout(B, L->E, L->top_e, L->d, sI, sr, nullptr, nullptr);
   REQUIRE(ws_bytes >= need, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  const bool streamed = !dense && (ep_size > 0 || L->path == 2 || (L->path == 0 && !moe::reader_supports(B, L->d)));
+  if (!dense && !streamed && !moe::reader_supports(B, L->d))
+    return fail(MOE_EUNSUPPORTED, "path 1 (one cluster per expert) runs B <= 2 and d <= 2048 (B = %d, d = %d)", B,
+                L->d);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   moe::Workspace ws;
   moe::workspace_layout(B, L->E, L->top_e, L->d, sI, sr, workspace, &ws);
+  if (clear_counters) {
+    const cudaError_t ce = cudaMemsetAsync(ws.counters, 0, sizeof(unsigned) * moe::kMaxTokens * moe::kMaxCluster, s);
+    if (ce != cudaSuccess) return cuda_fail(ce, "clearing the combine counters");
+  }
 
   moe::RouteArgs ra = {};
   ra.B = B;
@@ -123,7 +136,6 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   ra.dbg_w = dbg ? dbg->weights : nullptr;
   ra.quantize = !dense;
   cudaError_t e = cudaSuccess;
-  const bool streamed = !dense && (ep_size > 0 || moe::use_streamed(B));
   ra.ep_rank = ep_rank;
   ra.ep_size = ep_size;
   if (!moe::fused_routing(B) || streamed) {
@@ -142,7 +154,8 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   a.r = dense ? 0 : L->r;
   a.recovery_input = dense ? 0 : L->recovery_input;
   a.ep_partial = ep_size > 0 ? 1 : 0;
-  a.cs = 0;  // chosen at launch (16 when schedulable, else 8)
+  a.cs = 0;  // chosen at launch
+  a.force_cs = L->cluster_size;
   a.nmax = B < moe::kMaxGroup ? B : moe::kMaxGroup;
   a.x = x;
   a.w_router = L->w_router;
@@ -172,14 +185,16 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
     a.dbg_y_expert = dbg->y_expert;
     a.dbg_phase = reinterpret_cast<unsigned long long*>(dbg->phase_ns);
   }
-  if (g_ev_before) cudaEventRecord(g_ev_before, s);
+  cudaEvent_t ev_before = dbg ? static_cast<cudaEvent_t>(dbg->ev_before) : nullptr;
+  cudaEvent_t ev_after = dbg ? static_cast<cudaEvent_t>(dbg->ev_after) : nullptr;
+  if (ev_before) cudaEventRecord(ev_before, s);
   e = dense ? moe::launch_dense(a, s) : streamed ? moe::launch_stream(a, s) : moe::launch_reader(a, s);
   if (e != cudaSuccess) return cuda_fail(e, dense ? "dense expert launch" : "reader launch");
   if (ep_size > 0) {
     e = moe::launch_ep_combine(B, L->top_e, L->d, ep_rank, ep_size, ws, y_partial, s);
     if (e != cudaSuccess) return cuda_fail(e, "expert-parallel combine launch");
   }
-  if (g_ev_after) cudaEventRecord(g_ev_after, s);
+  if (ev_after) cudaEventRecord(ev_after, s);
   return MOE_OK;
 }
 
@@ -188,6 +203,11 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
 moe_status moe::set_last_error(moe_status st, const char* msg) {
   g_err = msg;
   return st;
+}
+
+moe_status moe::forward_scratch(const moe_reader_layer* layer, int B, int k, int c, const uint16_t* x,
+                                const uint16_t* residual, uint16_t* y, void* scratch, size_t bytes, void* stream) {
+  return run_forward(layer, B, k, c, x, residual, y, nullptr, scratch, bytes, stream, false, 0, 0, nullptr, true);
 }
 
 extern "C" {
@@ -301,13 +321,13 @@ moe_status moe_reader_rmsnorm(int B, int d, float eps, const uint16_t* x, uint16
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "rmsnorm launch");
 }
 
-moe_status moe_reader_set_expert_events(void* ev_before, void* ev_after) {
-  g_ev_before = static_cast<cudaEvent_t>(ev_before);
-  g_ev_after = static_cast<cudaEvent_t>(ev_after);
-  return MOE_OK;
-}
-
 moe_status moe_reader_check_error(void* workspace, void* stream) {
+  if (!workspace) {
+    // the noalloc entry's scratch on the current device
+    cudaError_t se = cudaSuccess;
+    workspace = moe::noalloc_scratch(&se);
+    if (!workspace) return cuda_fail(se, "scratch set-up (cudaGetSymbolAddress)");
+  }
   REQUIRE_PTR(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(s);
@@ -321,18 +341,6 @@ moe_status moe_reader_check_error(void* workspace, void* stream) {
   const uint32_t zero = 0;
   cudaMemcpy(ws.err, &zero, sizeof zero, cudaMemcpyHostToDevice);
   return fail(MOE_ETIMEOUT, "device error word 0x%x (1: a bounded copy wait ran out; 2: bad work item)", word);
-}
-
-moe_status moe_reader_set_cluster_size(int cs) {
-  REQUIRE(cs == 0 || cs == 4 || cs == 8 || cs == 16, "cluster size %d: use 0 (automatic), 4, 8 or 16", cs);
-  moe::set_forced_cluster_size(cs);
-  return MOE_OK;
-}
-
-moe_status moe_reader_set_path(int path) {
-  REQUIRE(path >= 0 && path <= 2, "path %d: use 0 (automatic), 1 (one cluster per expert) or 2 (streamed)", path);
-  moe::set_path(path);
-  return MOE_OK;
 }
 
 moe_status moe_reader_launch_plan(int dense, int B, int E, int top_e, int I, int d, int r, int32_t* out4) {

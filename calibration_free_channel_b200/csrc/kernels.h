@@ -10,6 +10,13 @@ namespace moe {
 
 // Records the message returned by moe_reader_last_error and returns st.
 moe_status set_last_error(moe_status st, const char* msg);
+// moe_reader_forward on a given scratch buffer whose combine counters are
+// cleared after validation, before any launch (the noalloc entry).
+moe_status forward_scratch(const moe_reader_layer* layer, int B, int k, int c, const uint16_t* x,
+                           const uint16_t* residual, uint16_t* y, void* scratch, size_t bytes, void* stream);
+// Device address of the noalloc entry's scratch array on the current device
+// (looked up on the first call on each device); nullptr and *err on failure.
+void* noalloc_scratch(cudaError_t* err);
 
 // Workspace carved out of the caller's buffer (see workspace_layout).
 struct Workspace {
@@ -71,6 +78,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 struct ExpertArgs {
   int B, E, top_e, I, d, k, c, r;
   int cs;            // CTAs per cluster (one cluster per work item)
+  int force_cs;      // 0: cluster size chosen per launch; else this size
   int nmax;          // max tokens per work item this launch
   int ring_rows;     // copy-ring row slots per warp (sparse) / rows (dense)
   int recovery_input;  // 0: ahat of every skipped channel; 1: exact a of dropped candidates
@@ -106,15 +114,13 @@ struct ExpertArgs {
 // Steps of at most this many tokens route inside the expert kernel (one
 // launch per step); larger steps use the route and select kernels first.
 bool fused_routing(int B);
+// The one-cluster reader (reader.cu) runs steps of at most two tokens with
+// d <= 2048.
+bool reader_supports(int B, int d);
 cudaError_t launch_reader(const ExpertArgs& a, cudaStream_t s);
 // The streamed reader: screen, top-c, exact candidates, top-k, down rows +
 // combine, each one kernel over every pair of the step (after launch_route).
 cudaError_t launch_stream(const ExpertArgs& a, cudaStream_t s);
-// Which reader runs a sparse step of B tokens: the one-cluster-per-expert
-// kernel (false) or the streamed kernels (true).  set_path forces one (1:
-// cluster, 2: streamed; 0: automatic, streamed above two tokens).
-bool use_streamed(int B);
-void set_path(int path);
 // Expert parallelism: y_partial[b] = sum over the slots of b whose expert this
 // rank owns of w * y_e (fp32, slot order); y = bf16(y_sum + residual).
 cudaError_t launch_ep_combine(int B, int top_e, int d, int ep_rank, int ep_size, const Workspace& ws,
@@ -122,7 +128,6 @@ cudaError_t launch_ep_combine(int B, int top_e, int d, int ep_rank, int ep_size,
 cudaError_t launch_ep_finish(int B, int d, const float* y_sum, const uint16_t* residual, uint16_t* y,
                              cudaStream_t s);
 cudaError_t launch_dense(const ExpertArgs& a, cudaStream_t s);
-void set_forced_cluster_size(int cs);
 cudaError_t query_plan(const ExpertArgs& a, bool dense, int out[4]);
 
 cudaError_t launch_build_sketch(int E, int I, int d, const uint16_t* w_gate, const uint16_t* w_up,

@@ -1,13 +1,14 @@
 // noalloc.cu -- moe_reader_forward_noalloc: the sparse step with its scratch
 // in a fixed device array, for callers that cannot allocate device memory.
 //
-// Some callers cannot call cudaMalloc or an allocating library: code that
-// runs while a stream is being captured into a CUDA graph (allocation is not
-// a capturable operation), serving loops that forbid any allocation after
-// start-up so their memory footprint stays fixed, and hosts whose device
-// allocator belongs to another runtime.  For them this entry point keeps the
-// step's workspace in a file-scope __device__ array of a fixed size, which
-// every GPU that loads the library holds until the process exits.
+// Some callers cannot call cudaMalloc or an allocating library: serving
+// loops that forbid any allocation after start-up so that their memory
+// footprint stays fixed, and hosts whose device memory belongs to another
+// runtime's allocator, which this library cannot call.  For them this entry
+// point keeps the step's workspace in a file-scope __device__ array of a
+// fixed size, which every GPU that loads the library holds until the
+// process exits.  Its device error word (offset 0, set by a bounded wait
+// that ran out) is read and cleared by moe_reader_check_error(NULL, stream).
 #include <cstdio>
 #include <mutex>
 
@@ -28,9 +29,11 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
 
+}  // namespace
+
 // Device address of the scratch array on the current device (set up on the
 // first call on each device).  Returns nullptr and fills *err on failure.
-void* scratch_address(cudaError_t* err) {
+void* moe::noalloc_scratch(cudaError_t* err) {
   int dev = 0;
   *err = cudaGetDevice(&dev);
   if (*err != cudaSuccess) return nullptr;
@@ -48,28 +51,17 @@ void* scratch_address(cudaError_t* err) {
   return g_scratch_ptr[dev];
 }
 
-}  // namespace
-
 extern "C" moe_status moe_reader_forward_noalloc(const moe_reader_layer* layer, int B, int k, int c,
                                                  const uint16_t* x, const uint16_t* residual, uint16_t* y,
                                                  void* stream) {
-  if (!layer) return moe::set_last_error(MOE_EINVAL, "layer is NULL");
-  // Shapes whose workspace exceeds the fixed array are rejected by the
-  // forward's own validation below ("workspace has N bytes, needs M"),
-  // before anything is enqueued.
-  const size_t need = moe_reader_workspace_bytes(B, layer->E, layer->top_e, layer->I, layer->d, k, c, layer->r);
   cudaError_t err = cudaSuccess;
-  void* scratch = scratch_address(&err);
+  void* scratch = moe::noalloc_scratch(&err);
   if (!scratch) return moe::set_last_error(MOE_ECUDA, "scratch set-up (cudaGetSymbolAddress) failed");
-  if (need > 0 && need <= kScratchBytes) {
-    // The combine counters at the start of the workspace must be zero when a
-    // step begins.  The kernels leave them zero, but the array keeps whatever
-    // an earlier (possibly interrupted) call left, so clear them here.
-    moe::Workspace ws;
-    moe::workspace_layout(1, 1, 1, 16, 0, 0, scratch, &ws);
-    err = cudaMemsetAsync(ws.counters, 0, sizeof(unsigned) * moe::kMaxTokens * moe::kMaxCluster,
-                          static_cast<cudaStream_t>(stream));
-    if (err != cudaSuccess) return moe::set_last_error(MOE_ECUDA, "clearing the scratch counters failed");
-  }
-  return moe_reader_forward(layer, B, k, c, x, residual, y, nullptr, scratch, kScratchBytes, stream);
+  // The combine counters in the scratch must be zero when a step begins.  The
+  // kernels leave them zero, but the array keeps whatever an earlier
+  // (possibly interrupted) call left, so the forward clears them once the
+  // arguments have been validated, before its first launch.  Shapes whose
+  // workspace exceeds the array are rejected by the same validation
+  // ("workspace has N bytes, needs M") with nothing enqueued.
+  return moe::forward_scratch(layer, B, k, c, x, residual, y, scratch, kScratchBytes, stream);
 }

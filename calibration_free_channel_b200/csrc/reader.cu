@@ -139,7 +139,7 @@ __host__ inline Layout make_layout(int NT, int ntok, bool fused, int E, int I, i
 
 // misc ints
 enum {
-  MI_E = 0, MI_N, MI_NU, MI_ND, MI_DIG, MI_REM, MI_CNT, MI_DONE,
+  MI_E = 0, MI_N, MI_NU, MI_ND, MI_DIG, MI_REM, MI_CNT, MI_DONE = 12,
   MI_TOK = 16, MI_SLOT = 32, MI_LAST = 48, MI_TIX = 64, MI_CX = 80, MI_RED = 96, MI_WT = 112,
   MI_RIDS = 128,  // in-kernel routing: ids [B <= 2][top_e <= 16]
   MI_RW = 192,    // in-kernel routing: weights
@@ -309,13 +309,14 @@ __device__ void load_tokens(const ExpertArgs& a, const Layout& L, char* smem, co
 // runs alone when the count is odd.  Every element sees the reference
 // butterflies (a + b, a - b) of every stage in the reference stage order, so
 // the bits equal the reference transform's.  d >= 256.  sv_pre holds the
-// signs of elements 4T .. 4T+3, loaded early by the caller.
-__device__ void rotate_quantize(const ExpertArgs& a, const Layout& L, char* smem, int t, float* v, float* cx_out,
+// signs of elements 4T .. 4T+3, loaded early by the caller.  xt: the token
+// (bf16, shared memory), qt: its int8 codes (shared memory).
+__device__ void rotate_quantize(const ExpertArgs& a, const uint16_t* xt, int8_t* qt, float* v, float* cx_out,
                                 float* red, char4 sv_pre) {
-  const int d = a.d;
+  const int d = a.d, d8 = d >> 3;
   const int T = threadIdx.x, lane = T & 31, warp = T >> 5;
-  for (int c = T; c < 2 * L.d8; c += NTHR) {  // d / 4 is a multiple of 32: whole warps
-    const uint2 xv = reinterpret_cast<const uint2*>(smem + L.x + (size_t)t * d * 2)[c];
+  for (int c = T; c < 2 * d8; c += NTHR) {  // d / 4 is a multiple of 32: whole warps
+    const uint2 xv = reinterpret_cast<const uint2*>(xt)[c];
     const char4 sv = c == T ? sv_pre : reinterpret_cast<const char4*>(a.rot_sign)[c];
     float r0 = (float)sv.x * bf16lo(xv.x), r1 = (float)sv.y * bf16hi(xv.x);
     float r2 = (float)sv.z * bf16lo(xv.y), r3 = (float)sv.w * bf16hi(xv.y);
@@ -342,7 +343,7 @@ __device__ void rotate_quantize(const ExpertArgs& a, const Layout& L, char* smem
     __syncthreads();
     m = 0.0f;
     if (2 * h < d) {
-      for (int p = T; p < 2 * L.d8; p += NTHR) {
+      for (int p = T; p < 2 * d8; p += NTHR) {
         const int b = ((p >> lh) << (lh + 2)) | (p & (h - 1));
         const float a0 = v[b], a1 = v[b + h], a2 = v[b + 2 * h], a3 = v[b + 3 * h];
         const float s0 = __fadd_rn(a0, a1), s1 = __fsub_rn(a0, a1);  // stage h
@@ -358,7 +359,7 @@ __device__ void rotate_quantize(const ExpertArgs& a, const Layout& L, char* smem
       h <<= 2;
       lh += 2;
     } else {  // the last stage, h = d / 2
-      for (int p = T; p < 4 * L.d8; p += NTHR) {
+      for (int p = T; p < 4 * d8; p += NTHR) {
         const float x0 = v[p], x1 = v[p + h];
         const float o0 = __fadd_rn(x0, x1), o1 = __fsub_rn(x0, x1);
         v[p] = o0;
@@ -379,7 +380,7 @@ __device__ void rotate_quantize(const ExpertArgs& a, const Layout& L, char* smem
     const float4 r4 = reinterpret_cast<const float4*>(red)[w >> 2];
     amax = fmaxf(amax, fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w)));
   }
-  int8_t* q = reinterpret_cast<int8_t*>(smem + L.q) + (size_t)t * d;
+  int8_t* q = qt;
   for (int j = T; j < d; j += NTHR) {
     int n = 0;
     if (amax > 0.0f) n = max(-127, min(127, __float2int_rn(__fdiv_rn(__fmul_rn(v[j], 127.0f), amax))));
@@ -408,11 +409,12 @@ __device__ __forceinline__ void load_row8(const uint4* row, int j0, int d8, int 
 // read straight into registers, overlapping the token loads) and pushes them
 // to all CTAs; after the cluster barrier every CTA takes the same top-e and
 // one warp derives the softmax weights and this cluster's work item (one
-// item per routed expert, experts ascending).  Returns false if this cluster
-// has no item.
-template <int NT>
-__device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, int* misc, int cs, int rank,
-                            int cid, cg::cluster_group& cluster) {
+// item per routed expert, experts ascending).  `mid()` runs once the tokens
+// are in shared memory, while the router rows are still in flight.  Returns
+// false if this cluster has no item.
+template <int NT, class LT, class Mid>
+__device__ bool fused_route(const ExpertArgs& a, const LT& L, char* smem, int* misc, int cs, int rank, int cid,
+                            cg::cluster_group& cluster, Mid mid) {
   const int B = a.B, E = a.E, top = a.top_e;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int e0 = L.ex0[rank], ne = L.ex0[rank + 1] - e0;
@@ -428,6 +430,7 @@ __device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, in
       xs[t * L.d8 + j] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d) + j);
   if (threadIdx.x < B) misc[MI_TOK + threadIdx.x] = threadIdx.x;
   __syncthreads();
+  mid();
   // logit_e = sum_j W_r[e, j] x_j (+ b_e): bf16 products are exact in fp32
   // (8-bit significands; products below 2^-126 in magnitude excepted) and are
   // summed in fp64
@@ -468,9 +471,9 @@ __device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, in
       if (t < B && lane < cs) st_cluster(&lg[t * E + e], lane, s);
     }
   }
-  stamp(a, cid, rank, 1);
-  cluster.sync();
   stamp(a, cid, rank, 2);
+  cluster.sync();
+  stamp(a, cid, rank, 3);
   // top-e per token by rank: 4 threads per expert count the logits that beat
   // it (larger, or equal with a lower id); rank < top_e is chosen
   int* rids = misc + MI_RIDS;
@@ -535,7 +538,8 @@ __device__ bool fused_route(const ExpertArgs& a, const Layout& L, char* smem, in
 // Routing weights of the in-kernel router (one warp, off the critical path):
 // softmax over the chosen logits, summed in slot order (fp32 exponentials of
 // the fp64 logit differences; the weights only scale outputs).
-__device__ void route_weights(const ExpertArgs& a, const Layout& L, char* smem, int* misc, int cid, int rank) {
+template <class LT>
+__device__ void route_weights(const ExpertArgs& a, const LT& L, char* smem, int* misc, int cid, int rank) {
   const int lane = threadIdx.x & 31;
   const int top = a.top_e, nent = a.B * top;
   const double* lg = reinterpret_cast<const double*>(smem + L.logit);
@@ -695,123 +699,321 @@ __device__ __forceinline__ void reduce_gu(const int (&G)[NT], const int (&U)[NT]
   u = lo ? o : v;
 }
 
+
+// ================================================================ sparse
+// The one-cluster reader for steps of one or two tokens: one cluster of cs
+// CTAs per routed expert (work item), every stage in one launch.  CTA `rank`
+// owns the channels [ch0[rank], ch0[rank+1]) of the expert for the screen,
+// the exact stage and the down rows, and the output columns
+// [col0[rank], col0[rank+1]) for the final sum.
+//
+// Selections without a block-wide histogram.  A channel is a candidate if
+// fewer than c channels of the expert beat its screening score (larger, or
+// equal with a lower index), and kept if fewer than k candidates beat its
+// |a|; that count is all a CTA needs, and only for its own channels.  Each
+// CTA sorts its own values (counting ranks among its own channels), pushes
+// the sorted list to every other CTA of the cluster, and after the cluster
+// barrier adds, for each own channel, how many entries of every other CTA's
+// list beat it (a binary search per list).  Four exchanges over distributed
+// shared memory, each a push into the receivers' shared memory followed by a
+// cluster barrier: the router logits, the sorted score lists, the sorted
+// |a| lists of the candidates, and the partial outputs (each CTA sums its
+// column slice).  Loads the selections will most likely ask for start before
+// the selections are known: after its screen, a CTA starts copying the
+// gate/up rows of its own highest-scoring channels; after its exact stage,
+// the down rows of all its own candidates.  Rows a selection then leaves out
+// are read and not used (measured traffic, not algorithmic bytes).
+constexpr int kMaxOwn = 256;        // channels per CTA
+constexpr int kRSlots = 4;          // exact-stage row slots per warp (at most)
+constexpr int kMaxDSlots = 64;      // down-row slots
+
+struct RLayout {
+  int mbar, misc, x, q, logit, alpha, ubar, vown, ahat, aown, vloc, rloc, listc, listk, flags, rows, drows, kslot,
+      kco, dcnt, gu, zred, zparts, ztot, ybuf, ring, total;
+  int P, Pext;  // exact-stage slots (gate + up rows of one channel, 4d bytes each): P per warp, one more
+                // for warps 0 .. Pext - 1
+  int W;        // warps that own slots (all when P >= 1)
+  int ndslot;   // down-row slots (2d bytes each)
+  int nskbuf;   // 16-channel sketch chunks resident at once
+  int own_max, om4, cols_max, d8, skc, rr, nsteps;
+  int ch0[17], col0[17], ex0[17];
+};
+
+__host__ inline RLayout make_rlayout(int NT, int B, int E, int I, int d, int r, int cs, int smem_max) {
+  RLayout L = {};
+  for (int o = 0; o <= cs && o < 17; o++) {
+    const int c4 = 4 * cdiv(o * cdiv(I, 4), cs);
+    L.ch0[o] = c4 < I ? c4 : I;
+    L.col0[o] = 8 * cdiv(o * (d / 8), cs);
+    L.ex0[o] = cdiv(o * E, cs);
+  }
+  for (int o = 0; o < cs && o < 16; o++)
+    if (L.ch0[o + 1] - L.ch0[o] > L.own_max) L.own_max = L.ch0[o + 1] - L.ch0[o];
+  L.om4 = rup(L.own_max, 4);
+  L.nsteps = 0;
+  while ((1 << L.nsteps) <= L.om4) L.nsteps++;  // binary-search steps over om4 entries
+  L.cols_max = 8 * cdiv(d / 8, cs);
+  L.d8 = d / 8;
+  L.skc = 16 * (d / 4);
+  L.rr = r > 0 ? r : 1;
+  int o = 0;
+  auto take = [&](int bytes) {
+    const int at = o;
+    o = rup(o + bytes, 128);
+    return at;
+  };
+  L.mbar = take((kSkBars + 1 + NWARP * kRSlots + kMaxDSlots) * 8);
+  L.misc = take(256 * 4);
+  L.x = take(B * d * 2);
+  L.q = take(B * d);
+  L.logit = take(B * E * 8);
+  L.alpha = take(2 * L.om4 * 4);
+  L.ubar = take(L.om4 * L.rr * 2);
+  L.vown = take(L.cols_max * L.rr * 2);
+  L.ahat = take(NT * L.om4 * 4);
+  L.aown = take(NT * L.om4 * 4);
+  L.vloc = take(NT * L.om4 * 8);
+  L.rloc = take(NT * L.om4 * 4);
+  // the partial outputs arrive (last exchange) long after every CTA is done
+  // with the score lists (first exchange): one region serves both
+  const int lc_bytes = NT * cs * L.om4 * 8, yb_bytes = cs * NT * L.cols_max * 4;
+  L.listc = take(lc_bytes > yb_bytes ? lc_bytes : yb_bytes);
+  L.ybuf = L.listc;
+  L.listk = take(NT * cs * L.om4 * 8);
+  L.flags = take(L.om4);
+  L.rows = take(L.om4 * 4);
+  L.drows = take(L.om4 * 4);
+  L.kslot = take(L.om4 * 4);
+  L.kco = take(NT * L.om4 * 4);
+  L.dcnt = take(2 * NT * 16 * 4);
+  L.gu = take(NWARP * 4 * NT * 2 * 4);
+  L.zred = take(NWARP * NT * L.rr * 4);
+  L.zparts = take(cs * NT * L.rr * 4);
+  L.ztot = take(NT * L.rr * 4);
+  L.ring = o;
+  const int avail = smem_max - o;
+  const int ring = avail > 0 ? avail / (8 * d) * (8 * d) : 0;
+  int ns = ring / (4 * d);
+  if (ns > NWARP * kRSlots) ns = NWARP * kRSlots;
+  L.P = ns / NWARP;
+  L.Pext = ns % NWARP;
+  L.W = L.P > 0 ? NWARP : L.Pext;
+  L.ndslot = ring / (2 * d) < kMaxDSlots ? ring / (2 * d) : kMaxDSlots;
+  L.nskbuf = ring / (8 * d) < kSkBars ? ring / (8 * d) : kSkBars;
+  L.total = o + ring;
+  return L;
+}
+
+// misc ints of the sparse kernel (beyond the shared positions above)
+enum { MI_NSPEC = 8, MI_NROWS = 9, MI_NDC = 10, MI_NK = 11 };
+static_assert((int)MI_NK < (int)MI_DONE, "misc positions");
+// flags of an own channel: candidate of token t (bit t), kept by token t
+// (bit 2 + t), started before the candidates were known (bit 4)
+constexpr unsigned char kFlagSpec = 16;
+
 // Bulk copies of sketch chunk ch (rows i0 + 16 ch .. of both matrices) into
-// buffer slot `slot`, completing on bars[slot].
-__device__ __forceinline__ void issue_sketch(const ExpertArgs& a, const Layout& L, char* buf, uint64_t* bars, int e,
+// chunk buffer `slot` of the ring, completing on bars[slot].
+__device__ __forceinline__ void issue_sketch(const ExpertArgs& a, const RLayout& L, char* ring, uint64_t* bars, int e,
                                              int i0, int i1, int ch, int slot) {
   const int c0 = i0 + 16 * ch, cnt = min(16, i1 - c0);
   const uint32_t bytes = cnt * (a.d / 4);
-  char* dst = buf + (size_t)slot * 2 * L.skc;
+  char* dst = ring + (size_t)slot * 2 * L.skc;
   mbar_expect_tx(&bars[slot], 2 * bytes);
   bulk_g2s(dst, a.sk_gate + ((size_t)e * a.I + c0) * (a.d / 16), bytes, &bars[slot]);
   bulk_g2s(dst + L.skc, a.sk_up + ((size_t)e * a.I + c0) * (a.d / 16), bytes, &bars[slot]);
 }
 
-// ================================================================ sparse
-template <int NT, bool FUSED, bool DBG>
-__global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L) {
+// Gate and up rows of channel i into a 4d-byte slot.
+__device__ __forceinline__ void issue_gate_up(const ExpertArgs& a, int e, int i, char* dst, uint64_t* bar) {
+  const uint32_t rowb = (uint32_t)a.d * 2;
+  mbar_expect_tx(bar, 2 * rowb);
+  bulk_g2s(dst, a.w_gate + ((size_t)e * a.I + i) * a.d, rowb, bar);
+  bulk_g2s(dst + rowb, a.w_up + ((size_t)e * a.I + i) * a.d, rowb, bar);
+}
+
+__device__ __forceinline__ void issue_down(const ExpertArgs& a, int e, int i, char* dst, uint64_t* bar) {
+  const uint32_t rowb = (uint32_t)a.d * 2;
+  mbar_expect_tx(bar, rowb);
+  bulk_g2s(dst, a.w_down + ((size_t)e * a.I + i) * a.d, rowb, bar);
+}
+
+// Sort key of a channel: its value's bits above, the complement of its index
+// below, so that a larger key means a larger value or an equal value at a
+// lower channel (the tie rule of both selections); values are non-negative
+// floats, so their bit patterns order like the values.
+__device__ __forceinline__ uint64_t sort_key(float v, int i) {
+  return ((uint64_t)__float_as_uint(v) << 32) | (uint32_t)(0xffffffffu - (uint32_t)i);
+}
+
+// rank[li] = #{lj < n : v[lj] > v[li]} for li < n (keys distinct), n <=
+// kMaxOwn: thread (li, part) compares against lj = part, part + 4, ...
+__device__ void local_ranks(const uint64_t* v, int n, int* rank) {
+#pragma unroll 1
+  for (int base = 0; base < n; base += NTHR / 4) {
+    const int li = base + (threadIdx.x >> 2), part = threadIdx.x & 3;
+    const uint64_t vi = li < n ? v[li] : 0ull;
+    int cnt = 0;
+    if (li < n)
+#pragma unroll 4
+      for (int lj = part; lj < n; lj += 4) cnt += v[lj] > vi;
+    cnt += __shfl_xor_sync(kFull, cnt, 1);
+    cnt += __shfl_xor_sync(kFull, cnt, 2);
+    if (li < n && part == 0) rank[li] = cnt;
+  }
+}
+
+// Entries above v in the sorted lists (descending, zero padded, om4 entries
+// each) of CTAs q, q + 4, q + 8, q + 12 other than `self`: binary searches in
+// lockstep.
+__device__ __forceinline__ int count_above(uint64_t v, const uint64_t* lists, int om4, int nsteps, int cs, int self,
+                                           int q) {
+  int lo[4], hi[4];
+#pragma unroll
+  for (int j = 0; j < 4; j++) {
+    const int o = q + 4 * j;
+    lo[j] = 0;
+    hi[j] = o < cs && o != self ? om4 : 0;
+  }
+#pragma unroll 1
+  for (int s = 0; s < nsteps; s++) {
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      if (lo[j] < hi[j]) {
+        const int mid = (lo[j] + hi[j]) >> 1;
+        if (lists[(q + 4 * j) * om4 + mid] > v) lo[j] = mid + 1;
+        else hi[j] = mid;
+      }
+    }
+  }
+  return lo[0] + lo[1] + lo[2] + lo[3];
+}
+
+// The sorted list of the nonzero keys among n own keys (local ranks given;
+// zero keys, which tie, are left out) into this CTA's slot of a list array,
+// whose entries were zeroed at the start.
+__device__ __forceinline__ void write_sorted(const uint64_t* v, const int* rank, int n, uint64_t* mine) {
+  for (int li = threadIdx.x; li < n; li += NTHR)
+    if (v[li]) mine[rank[li]] = v[li];
+}
+
+template <int NT, bool DBG>
+__global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L) {
   extern __shared__ __align__(128) char smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int cs = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
   const int cid = cluster_id();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.mbar);
-  uint64_t* wbars = bars + warp * kMaxSlots;
-  uint64_t* skbars = bars + NWARP * kMaxSlots;
+  uint64_t* skbars = reinterpret_cast<uint64_t*>(smem + L.mbar);
   uint64_t* uvbar = skbars + kSkBars;
+  const int sbase = warp * L.P + min(warp, L.Pext), Pw = L.P + (warp < L.Pext ? 1 : 0);
+  const int W = L.W;  // rows go to warps 0 .. W - 1 (those that own slots)
+  uint64_t* wbars = uvbar + 1 + sbase;                // this warp's exact-stage slots
+  uint64_t* dbars = uvbar + 1 + NWARP * kRSlots;      // down-row slots
   int* misc = reinterpret_cast<int*>(smem + L.misc);
-  int* hist = reinterpret_cast<int*>(smem + L.hist);
-  if (tid < NWARP * kMaxSlots + kSkBars + 2) mbar_init(&bars[tid], 1);
+  unsigned char* flags = reinterpret_cast<unsigned char*>(smem + L.flags);
+  if (tid < kSkBars + 1 + NWARP * kRSlots + kMaxDSlots) mbar_init(&skbars[tid], 1);
+  for (int i = tid; i < L.om4; i += NTHR) flags[i] = 0;
+  {
+    // this CTA's slots of both list arrays start zeroed (the peers write only theirs)
+    uint64_t* lc = reinterpret_cast<uint64_t*>(smem + L.listc);
+    uint64_t* lk = reinterpret_cast<uint64_t*>(smem + L.listk);
+    const int rk = (int)cg::this_cluster().block_rank(), ncs = (int)cg::this_cluster().num_blocks();
+    for (int i = tid; i < NT * L.om4; i += NTHR) {
+      const int t = i / L.om4, j = i - t * L.om4;
+      lc[((size_t)t * ncs + rk) * L.om4 + j] = 0ull;
+      lk[((size_t)t * ncs + rk) * L.om4 + j] = 0ull;
+    }
+  }
   if (tid == 0) misc[MI_DONE] = 0;
   fence_mbar_init();
   __syncthreads();
   if (DBG) stamp(a, cid, rank, 0);
 
   // Programmatic dependent launch: the next kernel in the stream may be
-  // scheduled now (onto free SMs); this one reads nothing in global memory
-  // before the previous kernel has completed and its writes are visible.
+  // scheduled now; nothing in global memory is read before the previous
+  // kernel has completed and its writes are visible.
   pdl_trigger();
   pdl_wait();
-  char4 sv_pre = make_char4(0, 0, 0, 0);  // rotation signs of elements 4 tid .. 4 tid + 3 (in-kernel routing)
-  if (FUSED) {
-    if (tid < a.d / 4) sv_pre = __ldg(reinterpret_cast<const char4*>(a.rot_sign) + tid);
-    if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, cluster)) return;  // uniform per cluster
-  } else {
-    if (!load_item_table(a, cid, misc, NT)) return;
-  }
-  if (DBG) stamp(a, cid, rank, 3);
+  const int d = a.d, I = a.I, r = a.r, om = L.om4;
+  char* ring = smem + L.ring;
+  const uint16_t* xs = reinterpret_cast<const uint16_t*>(smem + L.x);
+  int8_t* qs = reinterpret_cast<int8_t*>(smem + L.q);
+  float* cxs = reinterpret_cast<float*>(misc + MI_CX);
+  char4 sv_pre = make_char4(0, 0, 0, 0);  // rotation signs of elements 4 tid .. 4 tid + 3
+  if (tid < d / 4) sv_pre = __ldg(reinterpret_cast<const char4*>(a.rot_sign) + tid);
+
+  // ------------------------------------------------ R: routing + rotation
+  // every token is rotated and quantised while the router rows are in flight
+  // (the fp32 scratch of the transform is the start of the ring)
+  const bool has_item = fused_route<NT>(a, L, smem, misc, cs, rank, cid, cluster, [&] {
+#pragma unroll 1
+    for (int t = 0; t < a.B; t++)
+      rotate_quantize(a, xs + (size_t)t * d, qs + (size_t)t * d, reinterpret_cast<float*>(ring), cxs + t,
+                      reinterpret_cast<float*>(misc + MI_RED), sv_pre);
+    if (DBG) stamp(a, cid, rank, 1);
+  });
+  if (!has_item) return;  // uniform per cluster; no exchange follows
+  if (DBG) stamp(a, cid, rank, 4);
   const int e = misc[MI_E], n = misc[MI_N];
-  const int I = a.I, d = a.d, r = a.r;
   const int i0 = L.ch0[rank], i1 = L.ch0[rank + 1], nown = i1 - i0;
   const int j0 = L.col0[rank], ncols = L.col0[rank + 1] - j0;
   uint32_t* err = a.ws.err;
-  char* skbuf = smem + L.ring;
   const int nchunk = cdiv(nown, 16);
 
-  // factor rows of the own channels, V rows of the own columns, and the
-  // first round of sketch chunks: all in flight before the token work
-  if (tid == 0) {
-    if (r > 0) {
+  // the sketch chunks (warp w copies chunk w), the sketch scales (on chunk
+  // 0's barrier, which every warp waits for first), the factor rows of the
+  // own channels and the V rows of the own columns: all in flight at once
+  if (lane == 0) {
+    fence_proxy_async();  // the ring held the transform scratch (generic stores)
+    if (warp == 0 && I % 4 == 0 && nown > 0) {
+      mbar_expect_tx_only(&skbars[0], 2 * nown * 4);
+      bulk_g2s(smem + L.alpha, a.alpha_gate + (size_t)e * I + i0, nown * 4, &skbars[0]);
+      bulk_g2s(smem + L.alpha + om * 4, a.alpha_up + (size_t)e * I + i0, nown * 4, &skbars[0]);
+    }
+    if (warp < min(nchunk, L.nskbuf)) issue_sketch(a, L, ring, skbars, e, i0, i1, warp, warp);
+    if (warp == NWARP - 1 && r > 0) {
       const uint32_t bu = nown * r * 2, bv = ncols * r * 2;
       mbar_expect_tx(uvbar, bu + bv);
       bulk_g2s(smem + L.ubar, a.u_sigma + ((size_t)e * I + i0) * r, bu, uvbar);
       bulk_g2s(smem + L.vown, a.v + ((size_t)e * d + j0) * r, bv, uvbar);
     }
-    // the sketch scales of the own channels complete on chunk 0's barrier
-    // (every warp waits for chunk 0 before its first channel)
-    if (I % 4 == 0 && nown > 0) {
-      mbar_expect_tx_only(&skbars[0], 2 * nown * 4);  // chunk 0's copies arrive on it below
-      bulk_g2s(smem + L.alpha, a.alpha_gate + (size_t)e * I + i0, nown * 4, &skbars[0]);
-      bulk_g2s(smem + L.alpha + L.own_max * 4, a.alpha_up + (size_t)e * I + i0, nown * 4, &skbars[0]);
-    }
-    const int c1 = min(nchunk, L.sk_round);
-    for (int ch = 0; ch < c1; ch++) issue_sketch(a, L, skbuf, skbars, e, i0, i1, ch, ch);
   }
   float* alg = reinterpret_cast<float*>(smem + L.alpha);
-  float* alu = alg + L.own_max;
-  if (I % 4 != 0) {  // unaligned scale slices: plain loads, made visible by the barrier below
+  float* alu = alg + om;
+  if (I % 4 != 0) {  // unaligned scale slices: plain loads
     for (int li = tid; li < nown; li += NTHR) {
       alg[li] = __ldg(a.alpha_gate + (size_t)e * I + i0 + li);
       alu[li] = __ldg(a.alpha_up + (size_t)e * I + i0 + li);
     }
   }
   int tix[NT];
-  if (FUSED) {
-    // rotate + quantise every token while the sketch is in flight (the fp32
-    // scratch sits past the sketch buffers); its barriers also publish the
-    // scales loaded above
-    float* scratch = reinterpret_cast<float*>(smem + L.ring + NWARP * L.ring_bytes - d * 4);
-#pragma unroll 1
-    for (int t = 0; t < a.B; t++)
-      rotate_quantize(a, L, smem, t, scratch, reinterpret_cast<float*>(misc + MI_CX) + t,
-                      reinterpret_cast<float*>(misc + MI_RED), sv_pre);
-  } else {
-    load_tokens(a, L, smem, misc, n, true);
-    __syncthreads();
-  }
 #pragma unroll
   for (int t = 0; t < NT; t++) tix[t] = misc[MI_TIX + (t < n ? t : 0)];
-  if (DBG) stamp(a, cid, rank, 4);
+  __syncthreads();
 
-  float* sa = reinterpret_cast<float*>(smem + L.sa);          // [I, NT] (sigma, ahat) pairs, slices from the owners
-  float* zparts = reinterpret_cast<float*>(smem + L.zparts);  // [cs, NT, r]
-  float* z = reinterpret_cast<float*>(smem + L.z);            // [NT, r]
-  float* apos = reinterpret_cast<float*>(smem + L.apos);      // [NT, I] by union position
-  uint32_t* candm = reinterpret_cast<uint32_t*>(smem + L.candm);
-  uint32_t* keptm = reinterpret_cast<uint32_t*>(smem + L.keptm);  // over union positions
-  int* ulist = reinterpret_cast<int*>(smem + L.ulist);
-  int* dlist = reinterpret_cast<int*>(smem + L.dlist);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.keys);
-  const float* cxs = reinterpret_cast<const float*>(misc + MI_CX);
+  float* ahat = reinterpret_cast<float*>(smem + L.ahat);        // [NT, om] sketch estimates, own channels
+  float* aown = reinterpret_cast<float*>(smem + L.aown);        // [NT, om] exact a, own candidates
+  uint64_t* vloc = reinterpret_cast<uint64_t*>(smem + L.vloc);  // [NT, om] sort keys, own channels
+  int* rloc = reinterpret_cast<int*>(smem + L.rloc);            // [NT, om] local ranks
+  uint64_t* listc = reinterpret_cast<uint64_t*>(smem + L.listc);  // [NT, cs, om] sorted score keys
+  uint64_t* listk = reinterpret_cast<uint64_t*>(smem + L.listk);  // [NT, cs, om] sorted |a| keys
+  float* zparts = reinterpret_cast<float*>(smem + L.zparts);    // [cs, NT, rr]
+  int* rows = reinterpret_cast<int*>(smem + L.rows);
+  int* drows = reinterpret_cast<int*>(smem + L.drows);
+  int* dcnt = reinterpret_cast<int*>(smem + L.dcnt);            // [2, NT, 16] debug list counts
+  const uint16_t* ub = reinterpret_cast<const uint16_t*>(smem + L.ubar);
 
   // ---------------------------------------------------------- S: screen
+  // warp w takes channel 16 j + w of every sketch chunk j.  Each channel's
+  // dots are reduced over the warp and parked; every 4 chunks (and at the
+  // end) one pass over the lanes turns the parked sums into sigma and ahat.
   {
-    const int nv = L.d64;  // 16-byte sketch vectors per row
+    const int nv = d >> 6;  // 16-byte sketch vectors per row
     int sq[NT];
 #pragma unroll
     for (int t = 0; t < NT; t++) {
-      const uint4* qv = reinterpret_cast<const uint4*>(smem + L.q + (size_t)tix[t] * d);
+      const uint4* qv = reinterpret_cast<const uint4*>(qs + (size_t)tix[t] * d);
       int s = 0;
       for (int j = lane; j < L.d8 / 2; j += 32) {
         const uint4 q4 = qv[j];
@@ -822,40 +1024,33 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
       }
       sq[t] = warp_sum(s);  // sum of the token's activations: the code offset
     }
-    const uint16_t* ub = reinterpret_cast<const uint16_t*>(smem + L.ubar);
     float zacc[NT][4];
 #pragma unroll
     for (int t = 0; t < NT; t++)
 #pragma unroll
       for (int kk = 0; kk < 4; kk++) zacc[t][kk] = 0.0f;
     bool uv_ready = r == 0;
-    // this lane's activations for sketch vector lane (the row's first 32
-    // vectors), kept in registers across the channels
-    uint4 qr[NT][4];
+    uint4 qr[NT][4];  // activations of sketch vector `lane` (the row's first 32 vectors)
 #pragma unroll
     for (int t = 0; t < NT; t++) {
-      const uint4* qv = reinterpret_cast<const uint4*>(smem + L.q + (size_t)tix[t] * d);
+      const uint4* qv = reinterpret_cast<const uint4*>(qs + (size_t)tix[t] * d);
 #pragma unroll
       for (int kk = 0; kk < 4; kk++) qr[t][kk] = lane < nv ? qv[4 * lane + kk] : make_uint4(0u, 0u, 0u, 0u);
     }
-    // warp w takes channel 16 j + w of every sketch chunk j (one channel per
-    // warp and chunk).  Each channel's dots are reduced over the warp and
-    // parked in the warp's slot of gu; every 4 chunks (and at the end) one
-    // pass over the lanes turns the parked sums into sigma and ahat.
-    int* gu = hist + warp * 4 * NT * 2;  // [4 channels][NT tokens][g, u]; hist is free during the screen
+    int* gu = reinterpret_cast<int*>(smem + L.gu) + warp * 4 * NT * 2;  // parked sums
     int rb = 0, par = 0;  // first chunk of the resident round, parity of its barriers
 #pragma unroll 1
     for (int j = 0; j < nchunk; j++) {
       const int li = 16 * j + warp;
-      if (j == rb + L.sk_round) {
+      if (j == rb + L.nskbuf) {
         // the next round of chunks reuses the buffers: every warp is done with them
         __syncthreads();
         rb = j;
         par ^= 1;
         if (tid == 0) {
           fence_proxy_async();
-          const int c1 = min(nchunk, j + L.sk_round);
-          for (int ch = j; ch < c1; ch++) issue_sketch(a, L, skbuf, skbars, e, i0, i1, ch, ch - j);
+          const int c1 = min(nchunk, j + L.nskbuf);
+          for (int ch = j; ch < c1; ch++) issue_sketch(a, L, ring, skbars, e, i0, i1, ch, ch - j);
         }
       }
       int G[NT], U[NT];
@@ -864,8 +1059,8 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
       if (li < nown) {
         const int slot = j - rb;
         if (!mbar_wait_bounded(&skbars[slot], par, err)) misc[MI_DONE] = 1;
-        const uint4* gw = reinterpret_cast<const uint4*>(skbuf + (size_t)slot * 2 * L.skc + warp * (d / 4));
-        const uint4* uw = reinterpret_cast<const uint4*>(skbuf + (size_t)slot * 2 * L.skc + L.skc + warp * (d / 4));
+        const uint4* gw = reinterpret_cast<const uint4*>(ring + (size_t)slot * 2 * L.skc + warp * (d / 4));
+        const uint4* uw = reinterpret_cast<const uint4*>(ring + (size_t)slot * 2 * L.skc + L.skc + warp * (d / 4));
         int ga[NT][4], ua[NT][4];
 #pragma unroll
         for (int t = 0; t < NT; t++)
@@ -878,7 +1073,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
           for (int t = 0; t < NT; t++) {
             uint4 q0 = qr[t][0], q1 = qr[t][1], q2 = qr[t][2], q3 = qr[t][3];
             if (vv != lane) {
-              const uint4* qv = reinterpret_cast<const uint4*>(smem + L.q + (size_t)tix[t] * d) + 4 * vv;
+              const uint4* qv = reinterpret_cast<const uint4*>(qs + (size_t)tix[t] * d) + 4 * vv;
               q0 = qv[0];
               q1 = qv[1];
               q2 = qv[2];
@@ -924,7 +1119,8 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
         const float uh = __fmul_rn(__fmul_rn((float)u2, valid ? alu[lc] : 0.0f), cx);
         const float ah = __fmul_rn(silu_r(gh), uh);
         if (valid) {
-          reinterpret_cast<float2*>(sa)[(i0 + lc) * NT + t] = make_float2(fabsf(ah), ah);
+          vloc[t * om + lc] = sort_key(fabsf(ah), i0 + lc);
+          ahat[t * om + lc] = ah;
           if (DBG) {
             const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * I + i0 + lc;
             if (a.dbg_G) a.dbg_G[off] = g2;
@@ -932,7 +1128,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
             if (a.dbg_sigma) a.dbg_sigma[off] = fabsf(ah);
           }
         }
-        // partial recovery input z_w = sum over this warp's channels of ahat_i Ubar_i
+        // partial recovery input: sum over this warp's channels of ahat_i Ubar_i
         if (r > 0) {
           if (!uv_ready) {
             if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
@@ -957,9 +1153,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
         __syncwarp();
       }
     }
-    if (FUSED && warp == NWARP - 1) route_weights(a, L, smem, misc, cid, rank);
-    if (DBG) stamp(a, cid, rank, 5);
-    // z partials of the CTA, pushed to every CTA: zparts[rank][t]
+    if (warp == NWARP - 1) route_weights(a, L, smem, misc, cid, rank);
     if (r > 0) {
       float* zr = reinterpret_cast<float*>(smem + L.zred);  // [NWARP, NT, r]
 #pragma unroll
@@ -969,248 +1163,452 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, Layout L)
           const int p = lane + 32 * kk;
           if (p < r) zr[(warp * NT + t) * r + p] = zacc[t][kk];
         }
-      __syncthreads();
-      for (int tp = tid; tp < NT * r; tp += NTHR) {
-        float zz = 0.0f;
+    }
+  }
+  __syncthreads();  // sort keys and estimates of the own channels are in place; the sketch buffers are free
+  if (DBG) stamp(a, cid, rank, 5);
+
+  // ------------------------------------------- c: candidates (top-c by sigma)
+  // own sorted score lists to every CTA, the own channels most likely to be
+  // candidates started, then each own channel's rank over the expert
+#pragma unroll 1
+  for (int t = 0; t < n; t++) local_ranks(vloc + t * om, nown, rloc + t * om);
+  __syncthreads();
+#pragma unroll 1
+  for (int t = 0; t < n; t++) write_sorted(vloc + t * om, rloc + t * om, nown, listc + ((size_t)t * cs + rank) * om);
+  __syncthreads();
+  {
+    const int per = om / 2;  // 16-byte pieces of one list
+    const int tot = n * per;
+#pragma unroll 1
+    for (int w = tid; w < (cs - 1) * tot; w += NTHR) {
+      const int pi = idiv(w, tot), j = w - pi * tot;
+      const int o = pi + (pi >= rank);
+      const int t = j >= per ? 1 : 0, qq = j - t * per;
+      const float4* src = reinterpret_cast<const float4*>(listc + ((size_t)t * cs + rank) * om) + qq;
+      st_cluster(src, o, *src);
+    }
+  }
+  cluster_arrive();
+  if (r > 0) {
+    // the own partial of z_all = sum over the own channels of ahat_i Ubar_i
+    const float* zr = reinterpret_cast<const float*>(smem + L.zred);
+    for (int tp = tid; tp < n * r; tp += NTHR) {
+      const int t = tp / r, p = tp - t * r;
+      float zz = 0.0f;
+#pragma unroll 4
+      for (int w = 0; w < NWARP; w++) zz += zr[(w * NT + t) * r + p];
+      zparts[(rank * NT + t) * r + p] = zz;
+    }
+  }
+  {
+    // started early: each token's highest own scores, as many as the exact
+    // stage's slots hold at once
+    const int take = (NWARP * L.P + L.Pext) / n;
+    if (warp == 0) {
+      int base = 0;
+      for (int w0 = 0; w0 < nown; w0 += 32) {
+        const int li = w0 + lane;
+        bool on = false;
 #pragma unroll
-        for (int w = 0; w < NWARP; w++) zz += zr[w * NT * r + tp];
-        zparts[rank * NT * r + tp] = zz;
+        for (int t = 0; t < NT; t++) on |= t < n && li < nown && rloc[t * om + li] < take;
+        const unsigned bal = __ballot_sync(kFull, on);
+        if (on) {
+          rows[base + __popc(bal & ((1u << lane) - 1u))] = li;
+          flags[li] = kFlagSpec;
+        }
+        base += __popc(bal);
       }
+      if (lane == 0) misc[MI_NSPEC] = base;
     }
     __syncthreads();
-    // push the own (sigma, ahat) slice and z partial to every other CTA: one
-    // 16-byte store per thread and peer, all in flight together
-    {
-      const int nsa4 = cdiv((i1 - i0) * NT * 2, 4), nz4 = r > 0 ? NT * r / 4 : 0, per = nsa4 + nz4;
-      const float4* sa4 = reinterpret_cast<const float4*>(sa + i0 * NT * 2);
-      const float4* z4 = reinterpret_cast<const float4*>(zparts + rank * NT * r);
-#pragma unroll 1
-      for (int w = tid; w < (cs - 1) * per; w += NTHR) {
-        const int pi = idiv(w, per), j = w - pi * per;
-        const int o = pi + (pi >= rank);
-        if (j < nsa4) st_cluster(&sa4[j], o, sa4[j]);
-        else st_cluster(&z4[j - nsa4], o, z4[j - nsa4]);
+    const int nspec = misc[MI_NSPEC];
+    if (lane == 0) {
+      fence_proxy_async();  // the ring held the sketch
+      for (int m = 0; m < Pw; m++) {
+        const int j = warp + W * m;
+        if (j < nspec) issue_gate_up(a, e, i0 + rows[j], ring + (size_t)(sbase + m) * 4 * d, &wbars[m]);
       }
     }
   }
   if (DBG) stamp(a, cid, rank, 6);
-  cluster.sync();
+  cluster_wait();
   if (DBG) stamp(a, cid, rank, 7);
-
-  // ---------------------------------------------------------- c: top-c
-#pragma unroll 1
-  for (int t = 0; t < n; t++)
-    block_select_top(reinterpret_cast<const uint32_t*>(sa) + 2 * t, 2 * NT, I, a.c, hist, misc, candm + t * L.words);
-  // union of the candidates, ascending
-  block_mask_to_list(candm, n > 1 ? candm + L.words : nullptr, I, ulist, &misc[MI_NU], hist);
-  const int nU = misc[MI_NU];
-  if (DBG && a.dbg_cand && rank == 0 && warp < n) {
-    const int t = warp;
-    int base = 0;
-    int* out = a.dbg_cand + ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.c;
-    for (int w0 = 0; w0 < I; w0 += 32) {
-      const int p = w0 + lane;
-      const bool on = p < I && ((candm[t * L.words + (w0 >> 5)] >> lane) & 1u);
-      const unsigned bal = __ballot_sync(kFull, on);
-      if (on) out[base + __popc(bal & ((1u << lane) - 1u))] = p;
-      base += __popc(bal);
-    }
-  }
-  if (DBG) stamp(a, cid, rank, 8);
-
-  // -------------------------------------------- C: exact candidate stage
-  {
-    const int u0 = idiv(rank * nU + cs - 1, cs), u1 = idiv((rank + 1) * nU + cs - 1, cs), nsl = u1 - u0;
-    const int m0 = (warp * nsl) / NWARP, m1 = ((warp + 1) * nsl) / NWARP;
-    const int rowb = d * 2;
-    const int P = max(1, min(kMaxSlots, L.c_slots));
-    const uint4* xs = reinterpret_cast<const uint4*>(smem + L.x);
-    const int vx = L.d8;
-    char* ring = smem + L.ring + warp * L.ring_bytes;
-    uint32_t par = 0;
-    warp_stream(
-        m1 - m0, P, wbars, par, err,
-        [&](int j, int s, uint64_t* bar) {
-          const int i = ulist[u0 + m0 + j];
-          char* dst = ring + s * 2 * rowb;
-          mbar_expect_tx(bar, 2 * rowb);
-          bulk_g2s(dst, a.w_gate + ((size_t)e * I + i) * d, rowb, bar);
-          bulk_g2s(dst + rowb, a.w_up + ((size_t)e * I + i) * d, rowb, bar);
-          if (j + P < m1 - m0) {
-            // the row this slot takes next starts moving into L2 now
-            const int i2 = ulist[u0 + m0 + j + P];
-            bulk_prefetch_l2(a.w_gate + ((size_t)e * I + i2) * d, rowb);
-            bulk_prefetch_l2(a.w_up + ((size_t)e * I + i2) * d, rowb);
-          }
-        },
-        [&](int j, int s) {
-          const int u = u0 + m0 + j, i = ulist[u];
-          const uint4* gr = reinterpret_cast<const uint4*>(ring + s * 2 * rowb);
-          const uint4* ur = gr + vx;
-          float g0[NT], g1[NT], v0[NT], v1[NT];
-#pragma unroll
-          for (int t = 0; t < NT; t++) g0[t] = g1[t] = v0[t] = v1[t] = 0.0f;
-#pragma unroll 2
-          for (int vv = lane; vv < vx; vv += 32) {
-            const uint4 gv = gr[vv], uv = ur[vv];
-#pragma unroll
-            for (int t = 0; t < NT; t++) {
-              const uint4 xv = xs[tix[t] * vx + vv];
-              dot8_mixed(gv, xv, g0[t], g1[t]);
-              dot8_mixed(uv, xv, v0[t], v1[t]);
-            }
-          }
-#pragma unroll
-          for (int t = 0; t < NT; t++) {
-            if (t < n) {
-              const float gs = warp_sum(g0[t] + g1[t]), us = warp_sum(v0[t] + v1[t]);
-              const bool is_c = (candm[t * L.words + (i >> 5)] >> (i & 31)) & 1u;
-              const float av = is_c ? __fmul_rn(silu_r(gs), us) : 0.0f;
-              if (lane == 0) apos[t * I + u] = av;
-            }
-          }
-        });
-    // push the own a values to every other CTA, one store per thread and peer
-    __syncthreads();
-    const int per = n * nsl;
-#pragma unroll 1
-    for (int w = tid; w < (cs - 1) * per; w += NTHR) {
-      const int pi = idiv(w, per), j = w - pi * per;
-      const int o = pi + (pi >= rank);
-      const int t = j >= nsl ? 1 : 0, u = u0 + j - t * nsl;
-      st_cluster(&apos[t * I + u], o, apos[t * I + u]);
-    }
-  }
-  if (DBG) stamp(a, cid, rank, 9);
-  cluster.sync();  // the last exchange: no CTA touches another's smem after this
-  if (DBG) stamp(a, cid, rank, 10);
-
-  // ------------------------------------------------------------ k: top-k
-  // over union positions; a token's non-candidates get key 0, its candidates
-  // |a| + 1 (same order, ties still to the lower channel)
+  // candidate of token t: fewer than c channels of the expert beat it
 #pragma unroll 1
   for (int t = 0; t < n; t++) {
-    for (int u = tid; u < nU; u += NTHR) {
-      const int i = ulist[u];
-      const bool c = (candm[t * L.words + (i >> 5)] >> (i & 31)) & 1u;
-      keys[u] = c ? __float_as_uint(fabsf(apos[t * I + u])) + 1u : 0u;
+#pragma unroll 1
+    for (int base = 0; base < nown; base += NTHR / 4) {
+      const int li = base + (tid >> 2), q = tid & 3;
+      const uint64_t v = li < nown ? vloc[t * om + li] : ~0ull;
+      int cnt = count_above(v, listc + (size_t)t * cs * om, om, L.nsteps, cs, rank, q);
+      cnt += __shfl_xor_sync(kFull, cnt, 1);
+      cnt += __shfl_xor_sync(kFull, cnt, 2);
+      if (li < nown && q == 0 && rloc[t * om + li] + cnt < a.c) atomicOr(reinterpret_cast<unsigned*>(flags) + (li >> 2),
+                                                                         (1u << t) << (8 * (li & 3)));
     }
-    __syncthreads();
-    block_select_top(keys, 1, nU, a.k, hist, misc, keptm + t * L.words);
-    if (DBG && a.dbg_kept && rank == 0 && warp == 0) {
-      const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.k;
-      int base = 0;
-      for (int w0 = 0; w0 < nU; w0 += 32) {
-        const int u = w0 + lane;
-        const bool on = u < nU && ((keptm[t * L.words + (w0 >> 5)] >> lane) & 1u);
-        const unsigned bal = __ballot_sync(kFull, on);
-        const int at = base + __popc(bal & ((1u << lane) - 1u));
-        if (on && at < a.k) {
-          a.dbg_kept[off + at] = ulist[u];
-          if (a.dbg_a_kept) a.dbg_a_kept[off + at] = apos[t * I + u];
+  }
+  __syncthreads();
+  if (DBG) stamp(a, cid, rank, 8);
+  // rows of the exact stage: the started ones, then the own candidates not
+  // started yet; drows: every own candidate, ascending
+  const int nspec = misc[MI_NSPEC];
+  if (warp == 0) {
+    int base = nspec, dbase = 0;
+    for (int w0 = 0; w0 < nown; w0 += 32) {
+      const int li = w0 + lane;
+      const unsigned f = li < nown ? flags[li] : 0u;
+      const bool cand = (f & 3u) != 0, miss = cand && !(f & kFlagSpec);
+      const unsigned bm = __ballot_sync(kFull, miss), bc = __ballot_sync(kFull, cand);
+      if (miss) rows[base + __popc(bm & ((1u << lane) - 1u))] = li;
+      if (cand) drows[dbase + __popc(bc & ((1u << lane) - 1u))] = li;
+      base += __popc(bm);
+      dbase += __popc(bc);
+    }
+    if (lane == 0) {
+      misc[MI_NROWS] = base;
+      misc[MI_NDC] = dbase;
+    }
+  }
+  __syncthreads();
+  const int nrows = misc[MI_NROWS], ndc = misc[MI_NDC];
+
+  // -------------------------------------------- C: exact candidate stage
+  // warp w < W takes rows w, w + W, ...: position m of the warp in its slot m % Pw
+  {
+    const int nmine = warp < W && nrows > warp ? cdiv(nrows - warp, W) : 0;
+    char* wring = ring + (size_t)sbase * 4 * d;
+    if (lane == 0) {
+      fence_proxy_async();
+      for (int m = 0; m < Pw && m < nmine; m++) {
+        const int j = warp + W * m;
+        if (j >= nspec) issue_gate_up(a, e, i0 + rows[j], wring + (size_t)m * 4 * d, &wbars[m]);
+      }
+    }
+    __syncwarp();
+    const uint4* xv4 = reinterpret_cast<const uint4*>(xs);
+    uint32_t par = 0;
+#pragma unroll 1
+    for (int m = 0; m < nmine; m++) {
+      const int s = m % Pw;
+      if (!mbar_wait_bounded(&wbars[s], (par >> s) & 1u, err)) misc[MI_DONE] = 1;
+      par ^= 1u << s;
+      const int j = warp + W * m, li = rows[j];
+      const unsigned f = flags[li];
+      if (f & 3u) {
+        const uint4* gr = reinterpret_cast<const uint4*>(wring + (size_t)s * 4 * d);
+        const uint4* ur = gr + L.d8;
+        float g0[NT], g1[NT], v0[NT], v1[NT];
+#pragma unroll
+        for (int t = 0; t < NT; t++) g0[t] = g1[t] = v0[t] = v1[t] = 0.0f;
+#pragma unroll 2
+        for (int vv = lane; vv < L.d8; vv += 32) {
+          const uint4 gv = gr[vv], uv = ur[vv];
+#pragma unroll
+          for (int t = 0; t < NT; t++) {
+            const uint4 xq = xv4[tix[t] * L.d8 + vv];
+            dot8_mixed(gv, xq, g0[t], g1[t]);
+            dot8_mixed(uv, xq, v0[t], v1[t]);
+          }
         }
-        base += __popc(bal);
+#pragma unroll
+        for (int t = 0; t < NT; t++) {
+          if (t < n) {
+            const float gs = warp_sum(g0[t] + g1[t]), us = warp_sum(v0[t] + v1[t]);
+            if (lane == 0 && ((f >> t) & 1u)) aown[t * om + li] = __fmul_rn(silu_r(gs), us);
+          }
+        }
+      }
+      __syncwarp();
+      if (m + Pw < nmine && lane == 0) {
+        fence_proxy_async();
+        issue_gate_up(a, e, i0 + rows[j + W * Pw], wring + (size_t)s * 4 * d, &wbars[s]);
       }
     }
   }
-  // rows of the down stage: union positions kept by any token
-  block_mask_to_list(keptm, n > 1 ? keptm + L.words : nullptr, nU, dlist, &misc[MI_ND], hist);
-  const int nD = misc[MI_ND];
+  __syncthreads();  // every issued row was consumed: the ring is free
+  if (DBG) stamp(a, cid, rank, 9);
+  // the down rows of every own candidate start now (warp m % 16 copies row
+  // m); the top-k keeps about k / c of them.  If they do not fit, the kept
+  // ones follow the selection.
+  const bool dspec = ndc <= L.ndslot;
+  if (dspec && lane == 0) {
+    fence_proxy_async();
+    for (int m = warp; m < ndc; m += NWARP) issue_down(a, e, i0 + drows[m], ring + (size_t)m * 2 * d, &dbars[m]);
+  }
+
+  // ------------------------------------------------ k: kept (top-k by |a|)
+  // each token's own candidates: sort keys of |a|, local ranks, sorted lists
+  // to every CTA
+#pragma unroll 1
+  for (int t = 0; t < n; t++)
+    for (int m = tid; m < ndc; m += NTHR) {
+      const int li = drows[m];
+      vloc[t * om + m] = ((flags[li] >> t) & 1u) ? sort_key(fabsf(aown[t * om + li]), i0 + li) : 0ull;
+    }
+  __syncthreads();
+#pragma unroll 1
+  for (int t = 0; t < n; t++) local_ranks(vloc + t * om, ndc, rloc + t * om);
+  __syncthreads();
+#pragma unroll 1
+  for (int t = 0; t < n; t++) write_sorted(vloc + t * om, rloc + t * om, ndc, listk + ((size_t)t * cs + rank) * om);
+  if (DBG && tid < n) {
+    int cnt = 0;
+    for (int m = 0; m < ndc; m++) cnt += (flags[drows[m]] >> tid) & 1u;
+    dcnt[tid * 16 + rank] = cnt;  // own candidates of token tid (debug list offsets)
+  }
+  __syncthreads();
+  {
+    const int per = om / 2;
+    const int tot = n * per;
+#pragma unroll 1
+    for (int w = tid; w < (cs - 1) * tot; w += NTHR) {
+      const int pi = idiv(w, tot), j = w - pi * tot;
+      const int o = pi + (pi >= rank);
+      const int t = j >= per ? 1 : 0, qq = j - t * per;
+      const float4* src = reinterpret_cast<const float4*>(listk + ((size_t)t * cs + rank) * om) + qq;
+      st_cluster(src, o, *src);
+    }
+    if (DBG && tid < n)
+      for (int o = 0; o < cs; o++)
+        if (o != rank) asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr(&dcnt[tid * 16 + rank], o)),
+                                    "r"(dcnt[tid * 16 + rank])
+                                    : "memory");
+  }
+  cluster_arrive();
+  cluster_wait();
+  if (DBG) stamp(a, cid, rank, 10);
+#pragma unroll 1
+  for (int t = 0; t < n; t++) {
+#pragma unroll 1
+    for (int base = 0; base < ndc; base += NTHR / 4) {
+      const int m = base + (tid >> 2), q = tid & 3;
+      const bool cand = m < ndc && ((flags[drows[m < ndc ? m : 0]] >> t) & 1u);
+      const uint64_t v = cand ? vloc[t * om + m] : ~0ull;
+      int cnt = count_above(v, listk + (size_t)t * cs * om, om, L.nsteps, cs, rank, q);
+      cnt += __shfl_xor_sync(kFull, cnt, 1);
+      cnt += __shfl_xor_sync(kFull, cnt, 2);
+      if (cand && q == 0 && rloc[t * om + m] + cnt < a.k) {
+        const int li = drows[m];
+        atomicOr(reinterpret_cast<unsigned*>(flags) + (li >> 2), (4u << t) << (8 * (li & 3)));
+      }
+    }
+  }
+  __syncthreads();
+  if (DBG && warp < n && (a.dbg_cand || a.dbg_kept || a.dbg_a_kept)) {
+    // this CTA's part of the ascending candidate list (offset: the candidates
+    // of the lower CTAs); the kept list follows after the last exchange
+    const int t = warp;
+    int off = 0;
+    for (int o = 0; o < rank; o++) off += dcnt[t * 16 + o];
+    int* out = a.dbg_cand ? a.dbg_cand + ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.c : nullptr;
+    int base = off, kc = 0;
+    for (int m0 = 0; m0 < ndc; m0 += 32) {
+      const int m = m0 + lane;
+      const unsigned f = m < ndc ? flags[drows[m]] : 0u;
+      const bool on = (f >> t) & 1u;
+      const unsigned bal = __ballot_sync(kFull, on);
+      if (on && out && base + __popc(bal & ((1u << lane) - 1u)) < a.c)
+        out[base + __popc(bal & ((1u << lane) - 1u))] = i0 + drows[m];
+      base += __popc(bal);
+      kc += __popc(__ballot_sync(kFull, (f >> (2 + t)) & 1u));
+    }
+    if (lane == 0) dcnt[(NT + t) * 16 + rank] = kc;  // own kept channels of token t
+  }
   if (DBG) stamp(a, cid, rank, 11);
 
   // ---------------------------------------------- D: down rows + recovery
-  float* red = reinterpret_cast<float*>(smem + L.ring);
-  const int ncq = ncols >> 3, nr8 = r >> 3, nch = ncq + nr8;
-  // Rows: the kept union (recovery from the sketch estimates of every skipped
-  // channel: the factor rows of the kept channels enter with -ahat), or, with
-  // the exact recovery input, the whole candidate union (factor rows of the
-  // candidates enter with -(ahat - a) when dropped, -ahat when kept; down
-  // rows are read for the kept ones only).
-  const bool rec_exact = a.recovery_input == 1;
-  const int rg = down_rows<NT>(
-      a, e, j0, ncq, nr8, rec_exact ? nU : nD, r, [&](int m) { return ulist[rec_exact ? m : dlist[m]]; },
-      [&](int m, int i, bool is_w, float (&co)[NT]) {
-        const int u = rec_exact ? m : dlist[m];
-        bool need = false;
+  // kept rows, compacted with each token's coefficient; warp 0 waits for
+  // their copies, then thread tid adds columns 4 tid .. 4 tid + 3 of every row
+  int* kslot = reinterpret_cast<int*>(smem + L.kslot);
+  float* kco = reinterpret_cast<float*>(smem + L.kco);  // [NT, om]
+  if (warp == 0) {
+    int base = 0;
+    for (int m0 = 0; m0 < ndc; m0 += 32) {
+      const int m = m0 + lane;
+      const int li = m < ndc ? drows[m] : 0;
+      const unsigned f = m < ndc ? flags[li] : 0u;
+      const bool kept = (f & 12u) != 0;
+      const unsigned bal = __ballot_sync(kFull, kept);
+      if (kept) {
+        const int at = base + __popc(bal & ((1u << lane) - 1u));
+        kslot[at] = dspec ? m : li;  // dspec: the slot of the row; else the channel
+#pragma unroll
+        for (int t = 0; t < NT; t++) kco[t * om + at] = t < n && ((f >> (2 + t)) & 1u) ? aown[t * om + li] : 0.0f;
+      }
+      base += __popc(bal);
+    }
+    if (lane == 0) misc[MI_NK] = base;
+  }
+  __syncthreads();
+  const int nk = misc[MI_NK];
+  float acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; t++)
+#pragma unroll
+    for (int c = 0; c < 4; c++) acc[t][c] = 0.0f;
+  const bool colt = 4 * tid < d;
+  const int rnd = dspec ? (nk > 0 ? nk : 1) : L.ndslot;
+#pragma unroll 1
+  for (int base = 0; base < nk; base += rnd) {
+    const int cnt = min(rnd, nk - base);
+    if (!dspec) {
+      __syncthreads();  // every thread is done with the previous round's slots
+      if (lane == 0) {
+        fence_proxy_async();
+        for (int m = warp; m < cnt; m += NWARP)
+          issue_down(a, e, i0 + kslot[base + m], ring + (size_t)m * 2 * d, &dbars[m]);
+      }
+    }
+    if (warp == 0) {
+      const uint32_t par = dspec ? 0u : (uint32_t)(base / rnd) & 1u;
+      for (int m = lane; m < cnt; m += 32) {
+        const int s = dspec ? kslot[base + m] : m;
+        if (!mbar_wait_bounded(&dbars[s], par, err)) misc[MI_DONE] = 1;
+      }
+    }
+    __syncthreads();
+    if (colt) {
+#pragma unroll 2
+      for (int m = 0; m < cnt; m++) {
+        const int s = dspec ? kslot[base + m] : m;
+        const uint2 w2 = reinterpret_cast<const uint2*>(ring + (size_t)s * 2 * d)[tid];
+        const float f0 = bf16lo(w2.x), f1 = bf16hi(w2.x), f2 = bf16lo(w2.y), f3 = bf16hi(w2.y);
 #pragma unroll
         for (int t = 0; t < NT; t++) {
-          const bool kept = t < n && ((keptm[t * L.words + (u >> 5)] >> (u & 31)) & 1u);
-          const bool cand = t < n && ((candm[t * L.words + (i >> 5)] >> (i & 31)) & 1u);
-          const float ah = sa[(i * NT + t) * 2 + 1];
-          if (is_w) co[t] = kept ? apos[t * I + u] : 0.0f;
-          else if (kept) co[t] = ah;
-          else co[t] = rec_exact && cand ? __fsub_rn(ah, apos[t * I + u]) : 0.0f;
-          need |= kept || (!is_w && rec_exact && cand);
+          const float co = kco[t * om + base + m];
+          acc[t][0] = fmaf(co, f0, acc[t][0]);
+          acc[t][1] = fmaf(co, f1, acc[t][1]);
+          acc[t][2] = fmaf(co, f2, acc[t][2]);
+          acc[t][3] = fmaf(co, f3, acc[t][3]);
         }
-        return need;
-      },
-      red);
-  float* yfin = reinterpret_cast<float*>(smem + L.x);  // [n, cols_max]; x is no longer needed
-#pragma unroll 1
-  for (int o = tid; o < n * nch * 8; o += NTHR) {
-    const int t = o >= nch * 8 ? 1 : 0;
-    const int oc = o - t * nch * 8;
-    const float* rp = red + (size_t)t * nch * 8 + oc;
-    const int gstride = NT * nch * 8;
-    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
-    int gg = 0;
-#pragma unroll 1
-    for (; gg + 4 <= rg; gg += 4) {
-      s0 += rp[(gg + 0) * gstride];
-      s1 += rp[(gg + 1) * gstride];
-      s2 += rp[(gg + 2) * gstride];
-      s3 += rp[(gg + 3) * gstride];
-    }
-    for (; gg < rg; gg++) s0 += rp[gg * gstride];
-    const float s = (s0 + s1) + (s2 + s3);
-    if (oc < ncols) {
-      yfin[t * L.cols_max + oc] = s;
-    } else {
-      // z = (sum over the CTAs' partials of all channels) - (the kept part)
-      const int p = oc - ncols;
-      float z0 = 0.0f, z1 = 0.0f;
-      int o = 0;
-#pragma unroll 1
-      for (; o + 2 <= cs; o += 2) {
-        z0 += zparts[(o * NT + t) * r + p];
-        z1 += zparts[((o + 1) * NT + t) * r + p];
       }
-      if (o < cs) z0 += zparts[(o * NT + t) * r + p];
-      z[t * r + p] = (z0 + z1) - s;
     }
   }
+  if (dspec && nk < ndc && warp == 1) {
+    // copies of rows the top-k left out must land before the CTA ends
+    for (int m = lane; m < ndc; m += 32) {
+      const unsigned f = flags[drows[m]];
+      if (!(f & 12u) && !mbar_wait_bounded(&dbars[m], 0, err)) misc[MI_DONE] = 1;
+    }
+  }
+  // the own partial of z: z_all less the kept channels' ahat (and, with the
+  // exact recovery input, less ahat - a of the dropped candidates)
   if (r > 0) {
     if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
-    __syncthreads();
-    const uint16_t* vo = reinterpret_cast<const uint16_t*>(smem + L.vown);
+    const bool rec_exact = a.recovery_input == 1;
+    for (int tp = tid; tp < n * r; tp += NTHR) {
+      const int t = tp / r, p = tp - t * r;
+      float zz = zparts[(rank * NT + t) * r + p];
 #pragma unroll 1
-    for (int t = 0; t < n; t++)
-      for (int col = tid; col < ncols; col += NTHR) {
-        float rec0 = 0.0f, rec1 = 0.0f;
-#pragma unroll 4
-        for (int p = 0; p < r; p += 8) {
-          const uint4 v8 = *reinterpret_cast<const uint4*>(vo + col * r + p);
-          const float4 za = *reinterpret_cast<const float4*>(z + t * r + p);
-          const float4 zb = *reinterpret_cast<const float4*>(z + t * r + p + 4);
-          rec0 = fmaf(bf16lo(v8.x), za.x, rec0);
-          rec1 = fmaf(bf16hi(v8.x), za.y, rec1);
-          rec0 = fmaf(bf16lo(v8.y), za.z, rec0);
-          rec1 = fmaf(bf16hi(v8.y), za.w, rec1);
-          rec0 = fmaf(bf16lo(v8.z), zb.x, rec0);
-          rec1 = fmaf(bf16hi(v8.z), zb.y, rec1);
-          rec0 = fmaf(bf16lo(v8.w), zb.z, rec0);
-          rec1 = fmaf(bf16hi(v8.w), zb.w, rec1);
-        }
-        yfin[t * L.cols_max + col] += rec0 + rec1;
+      for (int m = 0; m < ndc; m++) {
+        const int li = drows[m];
+        const unsigned f = flags[li];
+        if (!((f >> t) & 1u)) continue;
+        const float u = bf16f(ub[li * r + p]), ah = ahat[t * om + li];
+        if ((f >> (2 + t)) & 1u) zz = fmaf(-ah, u, zz);
+        else if (rec_exact) zz = fmaf(-__fsub_rn(ah, aown[t * om + li]), u, zz);
       }
+      zparts[(rank * NT + t) * r + p] = zz;
+    }
   }
   __syncthreads();
   if (DBG) stamp(a, cid, rank, 12);
-  write_and_combine(a, rank, j0, ncols, L.cols_max, yfin, misc,
-                    FUSED ? reinterpret_cast<const float*>(misc + MI_RW) : a.ws.wts);
+  // push: the partial outputs to the owners of their columns, z to everyone
+  float* ybuf = reinterpret_cast<float*>(smem + L.ybuf);  // [cs, NT, cols_max] from every sender
+  if (colt) {
+    const int c0 = 4 * tid;
+    int o = 0;
+    while (o + 1 < cs && L.col0[o + 1] <= c0) o++;
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+      if (t < n)
+        st_cluster(&ybuf[((size_t)rank * NT + t) * L.cols_max + c0 - L.col0[o]], o,
+                   make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]));
+  }
+  if (r > 0) {
+    const int nq = n * r / 4;
+    for (int w = tid; w < (cs - 1) * nq; w += NTHR) {
+      const int pi = idiv(w, nq), j = w - pi * nq;
+      const int o = pi + (pi >= rank);
+      const float4* src = reinterpret_cast<const float4*>(zparts + (size_t)rank * NT * r) + j;
+      st_cluster(src, o, *src);
+    }
+  }
+  if (DBG && tid < n)
+    for (int o = 0; o < cs; o++)
+      if (o != rank) asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr(&dcnt[(NT + tid) * 16 + rank], o)),
+                                  "r"(dcnt[(NT + tid) * 16 + rank])
+                                  : "memory");
+  cluster.sync();  // the last exchange: no CTA touches another's shared memory after this
+  if (DBG) stamp(a, cid, rank, 13);
+  if (DBG && warp < n && (a.dbg_kept || a.dbg_a_kept)) {
+    const int t = warp;
+    int off = 0;
+    for (int o = 0; o < rank; o++) off += dcnt[(NT + t) * 16 + o];
+    const size_t obase = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.k;
+    int base = off;
+    for (int m0 = 0; m0 < ndc; m0 += 32) {
+      const int m = m0 + lane;
+      const int li = m < ndc ? drows[m] : 0;
+      const bool on = m < ndc && ((flags[li] >> (2 + t)) & 1u);
+      const unsigned bal = __ballot_sync(kFull, on);
+      const int at = base + __popc(bal & ((1u << lane) - 1u));
+      if (on && at < a.k) {
+        if (a.dbg_kept) a.dbg_kept[obase + at] = i0 + li;
+        if (a.dbg_a_kept) a.dbg_a_kept[obase + at] = aown[t * om + li];
+      }
+      base += __popc(bal);
+    }
+  }
+
+  // ------------------------------------ the own columns: sum, V z, combine
+  float* ztot = reinterpret_cast<float*>(smem + L.ztot);
+  if (r > 0)
+    for (int tp = tid; tp < n * r; tp += NTHR) {
+      const int t = tp / r, p = tp - t * r;
+      float zz = 0.0f;
+#pragma unroll 1
+      for (int o = 0; o < cs; o++) zz += zparts[(o * NT + t) * r + p];
+      ztot[t * r + p] = zz;
+    }
+  __syncthreads();
+  float* yfin = reinterpret_cast<float*>(smem + L.x);  // [n, cols_max]; x is no longer needed
+  const uint16_t* vo = reinterpret_cast<const uint16_t*>(smem + L.vown);
+#pragma unroll 1
+  for (int tc = tid; tc < n * ncols; tc += NTHR) {
+    const int t = tc >= ncols ? 1 : 0, col = tc - t * ncols;
+    float s0 = 0.0f, s1 = 0.0f;
+    int o = 0;
+#pragma unroll 1
+    for (; o + 2 <= cs; o += 2) {
+      s0 += ybuf[((size_t)o * NT + t) * L.cols_max + col];
+      s1 += ybuf[((size_t)(o + 1) * NT + t) * L.cols_max + col];
+    }
+    if (o < cs) s0 += ybuf[((size_t)o * NT + t) * L.cols_max + col];
+    float rec0 = 0.0f, rec1 = 0.0f;
+#pragma unroll 1
+    for (int p = 0; p < r; p += 8) {
+      const uint4 v8 = *reinterpret_cast<const uint4*>(vo + col * r + p);
+      const float4 za = *reinterpret_cast<const float4*>(ztot + t * r + p);
+      const float4 zb = *reinterpret_cast<const float4*>(ztot + t * r + p + 4);
+      rec0 = fmaf(bf16lo(v8.x), za.x, rec0);
+      rec1 = fmaf(bf16hi(v8.x), za.y, rec1);
+      rec0 = fmaf(bf16lo(v8.y), za.z, rec0);
+      rec1 = fmaf(bf16hi(v8.y), za.w, rec1);
+      rec0 = fmaf(bf16lo(v8.z), zb.x, rec0);
+      rec1 = fmaf(bf16hi(v8.z), zb.y, rec1);
+      rec0 = fmaf(bf16lo(v8.w), zb.z, rec0);
+      rec1 = fmaf(bf16hi(v8.w), zb.w, rec1);
+    }
+    yfin[t * L.cols_max + col] = (s0 + s1) + (rec0 + rec1);
+  }
+  __syncthreads();
+  if (DBG) stamp(a, cid, rank, 14);
+  write_and_combine(a, rank, j0, ncols, L.cols_max, yfin, misc, reinterpret_cast<const float*>(misc + MI_RW));
   if (DBG) {
     __syncthreads();
-    stamp(a, cid, rank, 13);
+    stamp(a, cid, rank, 15);
   }
 }
 
@@ -1233,7 +1631,7 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
   pdl_trigger();
   pdl_wait();
   if (FUSED) {
-    if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, cluster)) return;
+    if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, cluster, [] {})) return;
     if (warp == NWARP - 1) route_weights(a, L, smem, misc, cid, rank);
   } else {
     if (!load_item_table(a, cid, misc, NT)) return;
@@ -1332,34 +1730,52 @@ __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) 
 }
 
 // ---------------------------------------------------------- launch plans
-struct LaunchPlan {
-  int dev, dense, NT, fused, B, E, I, d, r, items, forced;
+// Cluster size: among the sizes that fit the shape, the one with the least
+// estimated time, waves * (1 + 8 / cs) with waves = ceil(items / co-resident
+// clusters): a wave costs a fixed latency plus work that shrinks with the
+// cluster's width.  `force_cs` (ExpertArgs::force_cs) pins it.
+
+int occupancy_clusters(const void* f, int cs, int smem) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs);
+  cfg.blockDim = dim3(NTHR);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int nc = 0;
+  if (cudaOccupancyMaxActiveClusters(&nc, f, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    nc = 0;
+  }
+  return nc;
+}
+
+// ----- dense block
+struct DensePlan {
+  int dev, NT, fused, B, E, I, d, items, forced;
   int cs, ring_rows, smem, max_clusters;
   Layout L;
 };
 
-int g_forced_cs = 0;  // 0: automatic
-
 template <int NT, bool FUSED>
-const void* kernel_ptr(bool dense, bool dbg) {
-  if (dense) return reinterpret_cast<const void*>(&dense_kernel<NT, FUSED>);
-  return dbg ? reinterpret_cast<const void*>(&reader_kernel<NT, FUSED, true>)
-             : reinterpret_cast<const void*>(&reader_kernel<NT, FUSED, false>);
+const void* dense_ptr() {
+  return reinterpret_cast<const void*>(&dense_kernel<NT, FUSED>);
 }
 static_assert(kMaxGroup == 2, "kernels are instantiated for 1 and 2 tokens per item");
-const void* pick_kernel(bool dense, int NT, bool fused, bool dbg) {
-  if (NT == 1) return fused ? kernel_ptr<1, true>(dense, dbg) : kernel_ptr<1, false>(dense, dbg);
-  return fused ? kernel_ptr<2, true>(dense, dbg) : kernel_ptr<2, false>(dense, dbg);
+const void* pick_dense(int NT, bool fused) {
+  if (NT == 1) return fused ? dense_ptr<1, true>() : dense_ptr<1, false>();
+  return fused ? dense_ptr<2, true>() : dense_ptr<2, false>();
 }
 
-// Cluster size: among 8..16 (those that fit this shape), the one with the
-// least estimated time, waves * (1 + 8 / cs) with waves = ceil(items /
-// co-resident clusters): a wave costs a fixed latency plus work that shrinks
-// with the cluster's width.  Ring: the deepest that fits, with room for the
-// down stage's partial sums (NT x 16 KB), the rotation scratch and at least
-// one sketch chunk.
-cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
-  thread_local LaunchPlan cache[16];
+// Ring: the deepest that fits, with room for the down stage's partial sums
+// (NT x 16 KB).
+cudaError_t plan_dense(const ExpertArgs& a, DensePlan* out) {
+  thread_local DensePlan cache[8];
   thread_local int ncache = 0, next = 0;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -1368,9 +1784,9 @@ cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
   const bool fused = fused_routing(a.B);
   const int items = fused ? (a.B * a.top_e < a.E ? a.B * a.top_e : a.E) : a.ws.max_items;
   for (int i = 0; i < ncache; i++) {
-    const LaunchPlan& c = cache[i];
-    if (c.dev == dev && c.dense == (int)dense && c.NT == NT && c.fused == (int)fused && c.B == a.B && c.E == a.E &&
-        c.I == a.I && c.d == a.d && c.r == a.r && c.items == items && c.forced == g_forced_cs) {
+    const DensePlan& c = cache[i];
+    if (c.dev == dev && c.NT == NT && c.fused == (int)fused && c.B == a.B && c.E == a.E && c.I == a.I &&
+        c.d == a.d && c.items == items && c.forced == a.force_cs) {
       *out = c;
       return cudaSuccess;
     }
@@ -1378,51 +1794,28 @@ cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
   int smem_max = 0;
   err = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (err != cudaSuccess) return err;
-  const void* fns[2] = {pick_kernel(dense, NT, fused, false), pick_kernel(dense, NT, fused, true)};
-  for (const void* f : fns) {
-    err = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (err != cudaSuccess) return err;
-  }
-  LaunchPlan p = {dev, (int)dense, NT, (int)fused, a.B, a.E, a.I, a.d, a.r, items, g_forced_cs, 0, 0, 0, 0, {}};
+  const void* f = pick_dense(NT, fused);
+  err = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (err != cudaSuccess) return err;
+  DensePlan p = {dev, NT, (int)fused, a.B, a.E, a.I, a.d, items, a.force_cs, 0, 0, 0, 0, {}};
   double best = 1e30;
   const int ntok = fused ? a.B : NT;
   for (int cs = 16; cs >= 8; cs--) {
-    if (g_forced_cs && cs != g_forced_cs) continue;
+    if (a.force_cs && cs != a.force_cs) continue;
     const int cols_max = 8 * cdiv(a.d / 8, cs);
     if (cols_max > kMaxCols || a.I < cs || (fused && a.E < cs)) continue;
     const int red_need = NT * NTHR * 8 * 4;
     int rr = 0;
     for (int t = 2; t <= 64; t++) {
-      const Layout L = make_layout(NT, ntok, fused, a.E, a.I, a.d, a.r, cs, t, dense);
+      const Layout L = make_layout(NT, ntok, fused, a.E, a.I, a.d, 0, cs, t, true);
       if (L.total > smem_max) break;
-      const int region = NWARP * L.ring_bytes;
-      if (L.c_slots >= 1 && region >= red_need && (dense || L.sk_round >= 1)) rr = t;
+      if (L.c_slots >= 1 && NWARP * L.ring_bytes >= red_need) rr = t;
     }
     if (rr < 2) continue;
-    const Layout L = make_layout(NT, ntok, fused, a.E, a.I, a.d, a.r, cs, rr, dense);
-    int nclusters = 1 << 30;
-    for (const void* f : fns) {
-      err = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
-      if (err != cudaSuccess) return err;
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(cs);
-      cfg.blockDim = dim3(NTHR);
-      cfg.dynamicSmemBytes = L.total;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = cs;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int nc = 0;
-      err = cudaOccupancyMaxActiveClusters(&nc, f, &cfg);
-      if (err != cudaSuccess) {
-        cudaGetLastError();
-        nc = 0;
-      }
-      nclusters = nc < nclusters ? nc : nclusters;
-    }
+    const Layout L = make_layout(NT, ntok, fused, a.E, a.I, a.d, 0, cs, rr, true);
+    err = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+    if (err != cudaSuccess) return err;
+    const int nclusters = occupancy_clusters(f, cs, L.total);
     if (nclusters < 1) continue;
     const double cost = (double)cdiv(items, nclusters) * (1.0 + 8.0 / cs);
     if (cost < best - 1e-12) {
@@ -1435,54 +1828,155 @@ cudaError_t plan_launch(const ExpertArgs& a, bool dense, LaunchPlan* out) {
     }
   }
   if (p.cs == 0) return cudaErrorInvalidConfiguration;
-  if (ncache < 16) cache[ncache++] = p;
-  else cache[next++ % 16] = p;
+  if (ncache < 8) cache[ncache++] = p;
+  else cache[next++ % 8] = p;
   *out = p;
   return cudaSuccess;
 }
 
-cudaError_t launch_expert(const ExpertArgs& a0, cudaStream_t s, bool dense) {
-  ExpertArgs a = a0;
-  LaunchPlan plan;
-  cudaError_t err = plan_launch(a, dense, &plan);
+// ----- sparse reader (one or two tokens)
+struct ReaderPlan {
+  int dev, B, E, I, d, r, forced;
+  int cs, smem, max_clusters, items;
+  RLayout L;
+};
+
+template <int NT>
+const void* reader_ptr(bool dbg) {
+  return dbg ? reinterpret_cast<const void*>(&reader_kernel<NT, true>)
+             : reinterpret_cast<const void*>(&reader_kernel<NT, false>);
+}
+
+cudaError_t plan_reader(const ExpertArgs& a, ReaderPlan* out) {
+  thread_local ReaderPlan cache[8];
+  thread_local int ncache = 0, next = 0;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  a.cs = plan.cs;
-  a.ring_rows = plan.ring_rows;
-  const bool dbg = a.dbg_ids || a.dbg_w || a.dbg_G || a.dbg_U || a.dbg_sigma || a.dbg_cand || a.dbg_kept ||
-                   a.dbg_a_kept || a.dbg_y_expert || a.dbg_phase;
-  const void* fn = pick_kernel(dense, plan.NT, plan.fused, dbg);
-  err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem);
+  if (a.B > kMaxGroup) return cudaErrorInvalidConfiguration;
+  for (int i = 0; i < ncache; i++) {
+    const ReaderPlan& c = cache[i];
+    if (c.dev == dev && c.B == a.B && c.E == a.E && c.I == a.I && c.d == a.d && c.r == a.r &&
+        c.forced == a.force_cs) {
+      *out = c;
+      return cudaSuccess;
+    }
+  }
+  int smem_max = 0;
+  err = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (err != cudaSuccess) return err;
+  const int NT = a.B;
+  const void* fns[2] = {NT == 1 ? reader_ptr<1>(false) : reader_ptr<2>(false),
+                        NT == 1 ? reader_ptr<1>(true) : reader_ptr<2>(true)};
+  for (const void* f : fns) {
+    err = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (err != cudaSuccess) return err;
+  }
+  const int items = a.B * a.top_e < a.E ? a.B * a.top_e : a.E;
+  ReaderPlan p = {dev, a.B, a.E, a.I, a.d, a.r, a.force_cs, 0, 0, 0, items, {}};
+  double best = 1e30;
+  for (int cs = 16; cs >= 2; cs--) {
+    if (a.force_cs && cs != a.force_cs) continue;
+    if (a.I < 4 * cs || a.E < cs || 8 * cdiv(a.d / 8, cs) > a.d) continue;
+    const RLayout L = make_rlayout(NT, a.B, a.E, a.I, a.d, a.r, cs, smem_max);
+    if (L.own_max > kMaxOwn || L.W < 4 || L.nskbuf < 1 || L.ndslot < 1 || L.total > smem_max) continue;
+    int nclusters = 1 << 30;
+    for (const void* f : fns) {
+      err = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+      if (err != cudaSuccess) return err;
+      const int nc = occupancy_clusters(f, cs, L.total);
+      nclusters = nc < nclusters ? nc : nclusters;
+    }
+    if (nclusters < 1) continue;
+    const double cost = (double)cdiv(items, nclusters) * (1.0 + 8.0 / cs);
+    if (cost < best - 1e-12) {
+      best = cost;
+      p.cs = cs;
+      p.smem = L.total;
+      p.max_clusters = nclusters;
+      p.L = L;
+    }
+  }
+  if (p.cs == 0) return cudaErrorInvalidConfiguration;
+  if (ncache < 8) cache[ncache++] = p;
+  else cache[next++ % 8] = p;
+  *out = p;
+  return cudaSuccess;
+}
+
+cudaLaunchConfig_t cluster_config(int grid, int cs, int smem, cudaStream_t s, cudaLaunchAttribute (&attr)[2]) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(plan.items * a.cs);
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(NTHR);
-  cfg.dynamicSmemBytes = plan.smem;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = a.cs;
+  attr[0].val.clusterDim.x = cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;  // programmatic dependent launch: overlaps this launch with the previous kernel's tail
-  void* args[] = {&a, &plan.L};
-  return cudaLaunchKernelExC(&cfg, fn, args);
+  return cfg;
 }
 
 }  // namespace
 
 bool fused_routing(int B) { return B <= kMaxGroup; }
-cudaError_t launch_reader(const ExpertArgs& a, cudaStream_t s) { return launch_expert(a, s, false); }
-cudaError_t launch_dense(const ExpertArgs& a, cudaStream_t s) { return launch_expert(a, s, true); }
-void set_forced_cluster_size(int cs) { g_forced_cs = cs; }
+
+bool reader_supports(int B, int d) { return B <= kMaxGroup && d <= 2048; }
+
+cudaError_t launch_reader(const ExpertArgs& a0, cudaStream_t s) {
+  ExpertArgs a = a0;
+  ReaderPlan plan;
+  cudaError_t err = plan_reader(a, &plan);
+  if (err != cudaSuccess) return err;
+  a.cs = plan.cs;
+  const bool dbg = a.dbg_ids || a.dbg_w || a.dbg_G || a.dbg_U || a.dbg_sigma || a.dbg_cand || a.dbg_kept ||
+                   a.dbg_a_kept || a.dbg_y_expert || a.dbg_phase;
+  const void* fn = a.B == 1 ? reader_ptr<1>(dbg) : reader_ptr<2>(dbg);
+  err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = cluster_config(plan.items * a.cs, a.cs, plan.smem, s, attr);
+  void* args[] = {&a, &plan.L};
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+cudaError_t launch_dense(const ExpertArgs& a0, cudaStream_t s) {
+  ExpertArgs a = a0;
+  DensePlan plan;
+  cudaError_t err = plan_dense(a, &plan);
+  if (err != cudaSuccess) return err;
+  a.cs = plan.cs;
+  a.ring_rows = plan.ring_rows;
+  const void* fn = pick_dense(plan.NT, plan.fused);
+  err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem);
+  if (err != cudaSuccess) return err;
+  const int items = plan.fused ? plan.items : a.ws.max_items;
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = cluster_config(items * a.cs, a.cs, plan.smem, s, attr);
+  void* args[] = {&a, &plan.L};
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
 cudaError_t query_plan(const ExpertArgs& a, bool dense, int out[4]) {
-  LaunchPlan p;
-  cudaError_t e = plan_launch(a, dense, &p);
+  if (dense) {
+    DensePlan p;
+    cudaError_t e = plan_dense(a, &p);
+    if (e != cudaSuccess) return e;
+    out[0] = p.cs;
+    out[1] = p.ring_rows;
+    out[2] = p.smem;
+    out[3] = p.max_clusters;
+    return cudaSuccess;
+  }
+  ReaderPlan p;
+  cudaError_t e = plan_reader(a, &p);
   if (e != cudaSuccess) return e;
   out[0] = p.cs;
-  out[1] = p.ring_rows;
+  out[1] = p.L.P * NWARP + p.L.Pext;
   out[2] = p.smem;
   out[3] = p.max_clusters;
   return cudaSuccess;

@@ -46,8 +46,6 @@ constexpr int kDRows = 256;     // down: kept-union rows staged per chunk
 constexpr int kMaxI = 2048;
 constexpr int kMaxAct = 1024;   // active experts (E <= 1024)
 
-int g_path = 0;
-
 // 16-byte load of weights that are read once per step: no L1 allocation.
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 v;
@@ -850,8 +848,6 @@ cudaError_t launch_ep_finish(int B, int d, const float* y_sum, const uint16_t* r
   return cudaGetLastError();
 }
 
-void set_path(int path) { g_path = path; }
-bool use_streamed(int B) { return g_path == 2 || (g_path == 0 && B > 2); }
 
 cudaError_t launch_stream(const ExpertArgs& a, cudaStream_t s) {
   int dev = 0;

@@ -19,8 +19,7 @@ _STATUS = {0: "MOE_OK", 1: "MOE_EINVAL", 2: "MOE_EUNSUPPORTED", 3: "MOE_ECUDA", 
 
 EXPORTS = ["moe_reader_workspace_bytes", "moe_reader_build_sketch", "moe_reader_lowrank_workspace_bytes",
            "moe_reader_build_lowrank", "moe_reader_forward", "moe_reader_forward_dense",
-           "moe_reader_forward_host", "moe_reader_rmsnorm", "moe_reader_set_expert_events",
-           "moe_reader_check_error", "moe_reader_set_cluster_size", "moe_reader_set_path", "moe_reader_launch_plan",
+           "moe_reader_forward_host", "moe_reader_rmsnorm", "moe_reader_check_error", "moe_reader_launch_plan",
            "moe_reader_forward_noalloc", "moe_reader_forward_ep", "moe_reader_ep_finish", "moe_reader_last_error"]
 
 
@@ -30,12 +29,12 @@ class MoeReaderLayer(C.Structure):
                 ("w_up", C.c_void_p), ("w_down", C.c_void_p), ("rot_sign", C.c_void_p),
                 ("sk_gate", C.c_void_p), ("sk_up", C.c_void_p), ("alpha_gate", C.c_void_p),
                 ("alpha_up", C.c_void_p), ("u_sigma", C.c_void_p), ("v", C.c_void_p),
-                ("recovery_input", C.c_int32)]
+                ("recovery_input", C.c_int32), ("path", C.c_int32), ("cluster_size", C.c_int32)]
 
 
 class MoeReaderDebug(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("ids", "weights", "dot_gate", "dot_up", "score", "cand", "kept",
-                                          "a_kept", "y_expert", "phase_ns")]
+                                          "a_kept", "y_expert", "phase_ns", "ev_before", "ev_after")]
 
 
 class MoeError(RuntimeError):
@@ -69,10 +68,7 @@ def lib():
         L.moe_reader_ep_finish.argtypes = [i32, i32, P, P, P, P]
         L.moe_reader_forward_host.argtypes = [C.POINTER(MoeReaderLayer), i32, i32, i32, P, P, P, P, P, sz, P]
         L.moe_reader_rmsnorm.argtypes = [i32, i32, C.c_float, P, P, P]
-        L.moe_reader_set_expert_events.argtypes = [P, P]
         L.moe_reader_check_error.argtypes = [P, P]
-        L.moe_reader_set_cluster_size.argtypes = [i32]
-        L.moe_reader_set_path.argtypes = [i32]
         L.moe_reader_launch_plan.argtypes = [i32] * 7 + [P]
         L.moe_reader_forward_noalloc.argtypes = [C.POINTER(MoeReaderLayer), i32, i32, i32, P, P, P, P]
         L.moe_reader_last_error.restype = C.c_char_p
@@ -164,23 +160,18 @@ def moe_reader_rmsnorm(B, d, eps, x, h, stream=None):
     _check(lib().moe_reader_rmsnorm(B, d, eps, _ptr(x), _ptr(h), _stream(stream)))
 
 
-def moe_reader_set_expert_events(ev_before, ev_after):
-    h = lambda ev: None if ev is None else ev.cuda_event  # noqa: E731
-    _check(lib().moe_reader_set_expert_events(h(ev_before), h(ev_after)))
-
-
 def moe_reader_check_error(workspace, stream=None):
+    """workspace None: the error word of moe_reader_forward_noalloc's scratch."""
     _check(lib().moe_reader_check_error(_ptr(workspace), _stream(stream)))
 
 
-def moe_reader_set_cluster_size(cs: int):
-    _check(lib().moe_reader_set_cluster_size(cs))
-
-
-def moe_reader_set_path(path: int):
-    """0: automatic (one cluster per expert for B <= 2, streamed above), 1: the
-    one-cluster reader, 2: the streamed reader (process-wide)."""
-    _check(lib().moe_reader_set_path(path))
+def timing_debug(ev_before, ev_after) -> MoeReaderDebug:
+    """A debug block that only records two torch.cuda.Event around the expert
+    kernels of one call (no per-stage outputs)."""
+    d = MoeReaderDebug()
+    d.ev_before = ev_before.cuda_event
+    d.ev_after = ev_after.cuda_event
+    return d
 
 
 def moe_reader_launch_plan(dense: bool, B, E, top_e, I, d, r) -> dict:
@@ -207,6 +198,8 @@ class Layer:
         self.u_sigma = None
         self.v = None
         self._ws = None
+        self.path = 0          # which reader runs a sparse step (see struct)
+        self.cluster_size = 0  # CTAs per cluster of the cluster kernels (0: automatic)
 
     def build_sketch(self, rot_seed: int, stream=None):
         moe_reader_build_sketch(self.E, self.I, self.d, self.w["w_gate"], self.w["w_up"], rot_seed,
@@ -237,13 +230,19 @@ class Layer:
             self.r = int(u_sigma.shape[-1])
         return self
 
-    def struct(self, r: int | None = None, recovery_input: int = 0) -> MoeReaderLayer:
+    def struct(self, r: int | None = None, recovery_input: int = 0, path: int | None = None,
+               cluster_size: int | None = None) -> MoeReaderLayer:
+        """The C description of the layer.  path: 0 automatic, 1 one-cluster
+        reader, 2 streamed reader (default: this layer's `path`);
+        cluster_size: 0 automatic (default: this layer's `cluster_size`)."""
         rr = self.r if r is None else r
         return MoeReaderLayer(self.E, self.I, self.d, self.top_e, rr, _ptr(self.w["w_router"]),
                               _ptr(self.w.get("router_bias")), _ptr(self.w["w_gate"]), _ptr(self.w["w_up"]),
                               _ptr(self.w["w_down"]), _ptr(self.rot_sign), _ptr(self.sk_gate), _ptr(self.sk_up),
                               _ptr(self.alpha_gate), _ptr(self.alpha_up),
-                              _ptr(self.u_sigma) if rr else None, _ptr(self.v) if rr else None, recovery_input)
+                              _ptr(self.u_sigma) if rr else None, _ptr(self.v) if rr else None, recovery_input,
+                              self.path if path is None else path,
+                              self.cluster_size if cluster_size is None else cluster_size)
 
     def workspace(self, B: int):
         nb = moe_reader_workspace_bytes(B, self.E, self.top_e, self.I, self.d, 1, 1, self.r)
@@ -263,7 +262,7 @@ class Layer:
                      a_kept=torch.empty(P + (k,), dtype=torch.float32, device=dev),
                      y_expert=torch.empty(P + (self.d,), dtype=torch.float32, device=dev),
                      phase_ns=torch.zeros((B * self.top_e, 16), dtype=torch.int64, device=dev))
-        return dbg_t, MoeReaderDebug(*[_ptr(dbg_t[n]) for n, _ in MoeReaderDebug._fields_])
+        return dbg_t, MoeReaderDebug(*[_ptr(dbg_t[n]) if n in dbg_t else None for n, _ in MoeReaderDebug._fields_])
 
     def forward_ep(self, x, k: int, c: int, ep_rank: int, ep_size: int, debug: bool = False, r: int | None = None,
                    stream=None, out=None, recovery_input: int = 0):
@@ -278,12 +277,17 @@ class Layer:
         return (yp, dbg_t) if debug else yp
 
     def forward(self, x, k: int, c: int, residual=None, debug: bool = False, r: int | None = None, stream=None,
-                out=None, recovery_input: int = 0):
+                out=None, recovery_input: int = 0, path: int | None = None, events=None):
+        """events: (ev_before, ev_after) torch.cuda.Event recorded around the
+        expert kernels (timing only; not with debug)."""
         B = x.shape[0]
         ws = self.workspace(B)
         y = out if out is not None else torch.empty_like(x)
         dbg_t, dbg = self._debug(B, k, c, x.device) if debug else (None, None)
-        moe_reader_forward(self.struct(r, recovery_input), B, k, c, x, residual, y, dbg, ws, ws.numel(), stream)
+        if events is not None:
+            dbg = timing_debug(*events)
+        moe_reader_forward(self.struct(r, recovery_input, path), B, k, c, x, residual, y, dbg, ws, ws.numel(),
+                           stream)
         return (y, dbg_t) if debug else y
 
     def forward_dense(self, x, residual=None, stream=None, out=None):

@@ -107,6 +107,12 @@ def _layer_weights_device(shape: BlockShape, seed: int, layer: int, bias: bool, 
     return out
 
 
+def router_bias(shape: BlockShape, seed: int = 0, layer: int = 0) -> torch.Tensor:
+    """The skewed routing prior alone: fp32 [E] ~ N(0, 1), the same values as
+    layer_weights(..., bias=True) on the CPU draws for this seed and layer."""
+    return torch.from_numpy(_gen(seed, layer, T_BIAS, 0).standard_normal(shape.E).astype(np.float32))
+
+
 def tokens(d: int, B: int, seed: int = 0, layer: int = 0) -> torch.Tensor:
     """B tokens x = RMSNorm(t), t_j ~ Student-t(4), bf16 [B, d]."""
     g = _gen(seed, layer, T_TOKENS, 0)

@@ -81,6 +81,24 @@ typedef struct {
    * stage computed them) and ahat_i only outside the candidate set; it reads
    * no extra weight rows.  Any other value is MOE_EINVAL. */
   int32_t recovery_input;
+  /* Which reader runs a sparse step.  Both compute the same routing, dots,
+   * scores and candidate sets bit for bit, and outputs within the stated
+   * tolerances.
+   *   0  automatic: the one-cluster reader when B <= 2 and d <= 2048, the
+   *      streamed reader otherwise;
+   *   1  the one-cluster reader: one thread-block cluster per routed expert,
+   *      every stage in one kernel (B <= 2 and d <= 2048, else
+   *      MOE_EUNSUPPORTED);
+   *   2  the streamed reader: after routing, five kernels (screen, top-c,
+   *      exact candidates, top-k, down rows + combine), each over every
+   *      (token, expert) pair of the step on all SMs.
+   * Any other value is MOE_EINVAL.  The dense block ignores it. */
+  int32_t path;
+  /* CTAs per thread-block cluster of the cluster kernels (the one-cluster
+   * reader, the dense block): 0 chooses per launch; 2 .. 16 pins the size
+   * (MOE_ECUDA "invalid configuration" if that size does not fit the shape
+   * on this device).  Other values are MOE_EINVAL. */
+  int32_t cluster_size;
 } moe_reader_layer;
 
 /* Optional per-stage outputs of moe_reader_forward (each pointer may be
@@ -96,14 +114,20 @@ typedef struct {
   float* a_kept;     /* [B, top_e, k] exact silu(g)*u of the kept channels        */
   float* y_expert;   /* [B, top_e, d] fp32 expert output before the combine      */
   uint64_t* phase_ns; /* [B * top_e, 16] device clock (ns) at the stage
-                         boundaries of the sparse expert kernel, one row per work
-                         item (its first CTA): 0 start, 1 token rotated, 2 router
-                         logits done, 3 logits exchanged, 4 item known, 5 screen
-                         dots done, 6 screen pushed, 7 screen exchanged,
-                         8 candidates chosen, 9 union listed, 10 exact stage done,
-                         11 exact exchanged, 12 kept chosen, 13 kept listed,
-                         14 down + recovery done, 15 combined; 0 where a stage
-                         does not run (routing stamps need B <= 2)            */
+                         boundaries of the one-cluster reader, one row per work
+                         item (its first CTA): 0 start, 1 tokens rotated,
+                         2 router logits done, 3 logits exchanged, 4 item known,
+                         5 screen done, 6 first exact rows started, 7 scores
+                         exchanged, 8 candidates chosen, 9 exact stage done,
+                         10 exact values exchanged, 11 kept chosen, 12 down
+                         rows done, 13 partial outputs exchanged, 14 own
+                         columns summed, 15 combined; 0 where a stage does not
+                         run (the streamed reader writes none)               */
+  /* Timing hooks (cudaEvent_t, or NULL): recorded on `stream` right before
+   * and right after the expert kernels of this call.  They do not switch on
+   * the per-stage outputs above. */
+  void* ev_before;
+  void* ev_after;
 } moe_reader_debug;
 
 /* Bytes of device workspace moe_reader_forward / moe_reader_forward_dense
@@ -202,10 +226,11 @@ moe_status moe_reader_forward_host(const moe_reader_layer* layer, int B, int k, 
                                    uint16_t* y_host, void* workspace, size_t ws_bytes, void* stream);
 
 /* moe_reader_forward with no caller-provided workspace, for callers that
- * cannot allocate device memory: code that runs while a stream is captured
- * into a CUDA graph, serving loops that forbid allocation after start-up,
- * hosts whose device allocator belongs to another runtime.  (The paper has no
- * counterpart; this is an interface convenience.)
+ * cannot allocate device memory: serving loops that forbid any allocation
+ * after start-up so that their memory footprint stays fixed, and hosts whose
+ * device memory is owned by another runtime's allocator, which this library
+ * cannot call.  (The paper has no counterpart; this is an interface
+ * convenience.)
  *  - The scratch is a fixed 8 MiB __device__ array inside the library; every
  *    GPU that loads the library holds it until the process exits.  Shapes
  *    whose workspace (moe_reader_workspace_bytes) exceeds 8 MiB return
@@ -215,8 +240,11 @@ moe_status moe_reader_forward_host(const moe_reader_layer* layer, int B, int k, 
  *  - Every call shares the one array per device: calls that may overlap on
  *    the GPU (different streams, no ordering) race and must not be issued.
  *    Each call first clears the array's combine counters (cudaMemsetAsync on
- *    `stream`); nothing is allocated or freed.
- *  - No debug outputs; errors as for moe_reader_forward. */
+ *    `stream`, after the arguments were validated); nothing is allocated or
+ *    freed.
+ *  - No debug outputs.  Argument errors as for moe_reader_forward; a bounded
+ *    device wait that ran out sets the array's error word, which
+ *    moe_reader_check_error(NULL, stream) reads and clears. */
 moe_status moe_reader_forward_noalloc(const moe_reader_layer* layer, int B, int k, int c,
                                       const uint16_t* x, const uint16_t* residual, uint16_t* y, void* stream);
 
@@ -224,36 +252,17 @@ moe_status moe_reader_forward_noalloc(const moe_reader_layer* layer, int B, int 
  * no learned gain (fp32). */
 moe_status moe_reader_rmsnorm(int B, int d, float eps, const uint16_t* x, uint16_t* h, void* stream);
 
-/* Optional timing hooks: when set (non-NULL cudaEvent_t handles), the
- * forward calls of this thread record events[0] before the expert kernel and
- * events[1] after it on `stream`.  Pass NULL to clear. */
-moe_status moe_reader_set_expert_events(void* ev_before, void* ev_after);
-
-/* Tuning: force the thread-block cluster size of the expert kernels (one
- * cluster per (expert, token group)): 4, 8 or 16 CTAs, or 0 to choose
- * automatically (the size that keeps the most SMs busy for the launch). */
-moe_status moe_reader_set_cluster_size(int cs);
-
-/* Which reader runs a sparse step (process-wide; both compute the same sets
- * and outputs within the tolerances above):
- *   0  automatic: one cluster per expert for B <= 2, streamed for B > 2;
- *   1  one thread-block cluster per (expert, token group), all stages in one
- *      kernel (latency-bound chain; best at one or two tokens);
- *   2  streamed: five kernels after routing (screen, top-c, exact
- *      candidates, top-k, down rows + combine), each over every
- *      (token, expert) pair of the step on all SMs, chained with
- *      programmatic dependent launch.
- * MOE_EINVAL for any other value. */
-moe_status moe_reader_set_path(int path);
-
-/* The launch the expert kernel would use for this shape on the current
- * device (dense != 0: the dense block): out4 = {cluster size, copy-ring rows
- * per warp, dynamic shared memory bytes per CTA, co-resident clusters}. */
+/* The launch the cluster kernel would use for this shape on the current
+ * device with an automatic cluster size (dense != 0: the dense block; else
+ * the one-cluster reader, B <= 2): out4 = {cluster size, copy-ring rows (dense:
+ * per warp; reader: exact-stage row slots per CTA), dynamic shared memory
+ * bytes per CTA, co-resident clusters}. */
 moe_status moe_reader_launch_plan(int dense, int B, int E, int top_e, int I, int d, int r, int32_t* out4);
 
-/* Synchronizes `stream`, reads and clears the workspace's device error word.
- * Returns MOE_OK, or MOE_ETIMEOUT if a bounded wait ran out since the last
- * check. */
+/* Synchronizes `stream`, reads and clears the workspace's device error word
+ * (workspace NULL: the error word of moe_reader_forward_noalloc's scratch on
+ * the current device).  Returns MOE_OK, or MOE_ETIMEOUT if a bounded wait ran
+ * out since the last check. */
 moe_status moe_reader_check_error(void* workspace, void* stream);
 
 /* Message for the last non-OK status returned on this thread. */

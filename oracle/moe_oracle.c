@@ -267,7 +267,7 @@ void orc_build_sketch(int E, int I, int d, const uint16_t* w_gate, const uint16_
  * largest.  Weights: softmax over the chosen logits (fp64), stored fp32.
  * Reading: "top-8 softmax-renormalised" = softmax over all experts, keep the
  * top 8, renormalise -- identical to a softmax over the 8 chosen logits. */
-static const double* g_sort_logits;
+static _Thread_local const double* g_sort_logits; /* qsort context, per thread */
 static int cmp_logit_desc(const void* a, const void* b) {
     int ia = *(const int*)a, ib = *(const int*)b;
     double la = g_sort_logits[ia], lb = g_sort_logits[ib];
@@ -306,7 +306,7 @@ void orc_route(int B, int E, int d, int top_e, const uint16_t* x, const uint16_t
  * Keep the n indices with the largest key; ties go to the lower index, i.e.
  * sort by (key descending, index ascending) and take the first n.  The result
  * is returned in ascending index order. */
-static const float* g_sort_keys;
+static _Thread_local const float* g_sort_keys;    /* qsort context, per thread */
 static int cmp_key_desc(const void* a, const void* b) {
     int ia = *(const int*)a, ib = *(const int*)b;
     float ka = g_sort_keys[ia], kb = g_sort_keys[ib];
@@ -450,7 +450,10 @@ void orc_expert_reader(int I, int d, int k, int c, int r, int exact_mode, int re
  * One MoE block over B tokens: route, rotate+quantize, reader per (token,
  * slot), then y_b = sum over slots (routing order) of w * y_e, fp64, rounded
  * once to bf16.  If `residual` is given, it is added before the rounding.
- * Debug arrays (any may be NULL) are laid out [B, top_e, ...]. */
+ * Debug arrays (any may be NULL) are laid out [B, top_e, ...].  `threads` > 1
+ * runs the (token, slot) readers on that many OpenMP threads; every pair is
+ * independent and the combine stays serial, so the result is the same bits
+ * for any thread count. */
 void orc_forward(int B, int E, int top_e, int I, int d, int k, int c, int r, int exact_mode, int recovery_input,
                  const uint16_t* x, const uint16_t* w_router, const float* bias,
                  const uint16_t* w_gate, const uint16_t* w_up, const uint16_t* w_down,
@@ -460,36 +463,43 @@ void orc_forward(int B, int E, int top_e, int I, int d, int k, int c, int r, int
                  uint16_t* y, double* y_f64,
                  int32_t* dbg_ids, float* dbg_w, int32_t* dbg_G, int32_t* dbg_U,
                  float* dbg_sigma, int32_t* dbg_cand, int32_t* dbg_kept,
-                 float* dbg_a_kept, double* dbg_y_expert) {
+                 float* dbg_a_kept, double* dbg_y_expert, int threads) {
     double* logits = (double*)malloc(sizeof(double) * (size_t)B * E);
     int32_t* ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)B * top_e);
     float* w = (float*)malloc(sizeof(float) * (size_t)B * top_e);
     float* v = (float*)malloc(sizeof(float) * (size_t)d);
-    int8_t* q = (int8_t*)malloc((size_t)d);
-    double* ye = (double*)malloc(sizeof(double) * (size_t)d);
+    int8_t* q = (int8_t*)malloc((size_t)B * d);
+    float* cx = (float*)malloc(sizeof(float) * (size_t)B);
+    double* ye = (double*)malloc(sizeof(double) * (size_t)B * top_e * d);
     double* acc = (double*)malloc(sizeof(double) * (size_t)d);
     orc_route(B, E, d, top_e, x, w_router, bias, logits, ids, w);
     const long rowsz = (long)I * d, skrow = (long)I * (d / 16);
+    for (int b = 0; b < B; b++) orc_rotate_quantize(d, x + (long)b * d, rot_sign, v, q + (long)b * d, &cx[b]);
+    /* the reader of every (token, slot) pair */
+    const long npairs = (long)B * top_e;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(threads > 1 ? threads : 1) if (threads > 1)
+    for (long ps = 0; ps < npairs; ps++) {
+        const int b = (int)(ps / top_e);
+        const int e = ids[ps];
+        orc_expert_reader(I, d, k, c, r, exact_mode, recovery_input, x + (long)b * d, q + (long)b * d, cx[b],
+                          sk_gate + e * skrow, sk_up + e * skrow,
+                          alpha_gate + (long)e * I, alpha_up + (long)e * I,
+                          w_gate + e * rowsz, w_up + e * rowsz, w_down + e * rowsz,
+                          ubar ? ubar + (long)e * I * r : NULL,
+                          vmap ? vmap + (long)e * d * r : NULL, ye + ps * d,
+                          dbg_G ? dbg_G + ps * I : NULL, dbg_U ? dbg_U + ps * I : NULL,
+                          dbg_sigma ? dbg_sigma + ps * I : NULL,
+                          dbg_cand ? dbg_cand + ps * c : NULL,
+                          dbg_kept ? dbg_kept + ps * k : NULL,
+                          dbg_a_kept ? dbg_a_kept + ps * k : NULL);
+    }
+    /* combine, slots in routing order */
     for (int b = 0; b < B; b++) {
-        float cx;
-        orc_rotate_quantize(d, x + (long)b * d, rot_sign, v, q, &cx);
         for (int j = 0; j < d; j++) acc[j] = 0.0;
         for (int s = 0; s < top_e; s++) {
-            int e = ids[b * top_e + s];
-            long ps = (long)b * top_e + s;
-            orc_expert_reader(I, d, k, c, r, exact_mode, recovery_input, x + (long)b * d, q, cx,
-                              sk_gate + e * skrow, sk_up + e * skrow,
-                              alpha_gate + (long)e * I, alpha_up + (long)e * I,
-                              w_gate + e * rowsz, w_up + e * rowsz, w_down + e * rowsz,
-                              ubar ? ubar + (long)e * I * r : NULL,
-                              vmap ? vmap + (long)e * d * r : NULL, ye,
-                              dbg_G ? dbg_G + ps * I : NULL, dbg_U ? dbg_U + ps * I : NULL,
-                              dbg_sigma ? dbg_sigma + ps * I : NULL,
-                              dbg_cand ? dbg_cand + ps * c : NULL,
-                              dbg_kept ? dbg_kept + ps * k : NULL,
-                              dbg_a_kept ? dbg_a_kept + ps * k : NULL);
-            if (dbg_y_expert) memcpy(dbg_y_expert + ps * d, ye, sizeof(double) * (size_t)d);
-            for (int j = 0; j < d; j++) acc[j] += (double)w[b * top_e + s] * ye[j];
+            const long ps = (long)b * top_e + s;
+            if (dbg_y_expert) memcpy(dbg_y_expert + ps * d, ye + ps * d, sizeof(double) * (size_t)d);
+            for (int j = 0; j < d; j++) acc[j] += (double)w[ps] * ye[ps * d + j];
         }
         for (int j = 0; j < d; j++) {
             double o = acc[j] + (residual ? (double)bf16_to_f32(residual[(long)b * d + j]) : 0.0);
@@ -499,7 +509,7 @@ void orc_forward(int B, int E, int top_e, int I, int d, int k, int c, int r, int
     }
     if (dbg_ids) memcpy(dbg_ids, ids, sizeof(int32_t) * (size_t)B * top_e);
     if (dbg_w) memcpy(dbg_w, w, sizeof(float) * (size_t)B * top_e);
-    free(logits); free(ids); free(w); free(v); free(q); free(ye); free(acc);
+    free(logits); free(ids); free(w); free(v); free(q); free(cx); free(ye); free(acc);
 }
 
 /* ------------------------------------------------------------ dense expert

@@ -27,7 +27,7 @@ SRC_PATH = os.path.join(HERE, "moe_oracle.c")
 def build(force: bool = False) -> str:
     """Compile the C oracle with strict IEEE semantics (no contraction)."""
     if force or not os.path.exists(LIB_PATH) or os.path.getmtime(LIB_PATH) < os.path.getmtime(SRC_PATH):
-        subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=gnu11",
+        subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=gnu11", "-fopenmp",
                                "-Wall", "-fPIC", "-shared", "-o", LIB_PATH, SRC_PATH, "-lm"])
     return LIB_PATH
 
@@ -65,7 +65,7 @@ def lib():
         L.orc_top_n.argtypes = [i32, P, P, i32, P]
         L.orc_expert_reader.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, f32, P, P, P, P,
                                         P, P, P, P, P, P, P, P, P, P, P, P]
-        L.orc_forward.argtypes = [i32] * 10 + [P] * 25
+        L.orc_forward.argtypes = [i32] * 10 + [P] * 25 + [i32]
         L.orc_forward_dense.argtypes = [i32] * 5 + [P] * 9
         L.orc_rmsnorm.argtypes = [i32, i32, f64, P, P]
         _lib = L
@@ -235,7 +235,8 @@ def build_lowrank(w_down, r: int, experts=None):
 
 # ---------------------------------------------------------------- forward
 def forward(x, W: dict, sketch, lowrank, k: int, c: int, r: int, top_e: int,
-            exact_mode: bool = False, residual=None, debug: bool = False, recovery_input: int = 0):
+            exact_mode: bool = False, residual=None, debug: bool = False, recovery_input: int = 0,
+            threads: int = 1):
     """The sparse reader over B tokens.  Returns y (uint16 bf16 [B,d]), the
     fp64 output before rounding and (if debug) the per-stage values.
     recovery_input 1 feeds the low-rank map the exact a of dropped candidates
@@ -265,7 +266,7 @@ def forward(x, W: dict, sketch, lowrank, k: int, c: int, r: int, top_e: int,
                       _p(x), _p(wr), _p(bias), _p(wg), _p(wu), _p(wd), _p(s), _p(skg), _p(sku),
                       _p(ag), _p(au), _p(us), _p(vv), _p(res), _p(y), _p(y64),
                       g("ids"), g("weights"), g("dot_gate"), g("dot_up"), g("score"), g("cand"),
-                      g("kept"), g("a_kept"), g("y_expert"))
+                      g("kept"), g("a_kept"), g("y_expert"), int(threads))
     return y, y64, dbg
 
 

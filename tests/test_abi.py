@@ -87,6 +87,28 @@ def test_forward_rejects_bad_arguments(lib, kw, args):
     assert lib.moe_reader_last_error()
 
 
+@pytest.mark.parametrize("kw", [dict(path=3), dict(path=-1), dict(cluster_size=1), dict(cluster_size=17),
+                                dict(recovery_input=2)])
+def test_forward_rejects_bad_options(lib, kw):
+    assert _fwd(lib, _layer(**kw)) == M.MOE_EINVAL
+    assert lib.moe_reader_last_error()
+
+
+def test_one_cluster_reader_limits(lib):
+    # the one-cluster reader runs one or two tokens with d <= 2048; asking for
+    # it above that is refused before anything is enqueued
+    assert _fwd(lib, _layer(path=1), B=3) == M.MOE_EUNSUPPORTED
+    assert b"B <= 2" in lib.moe_reader_last_error()
+    assert _fwd(lib, _layer(path=1, d=4096), B=1) == M.MOE_EUNSUPPORTED
+
+
+def test_layer_struct_layout():
+    # the binding's structs match the header's field order and sizes
+    assert [n for n, _ in M.MoeReaderLayer._fields_][-3:] == ["recovery_input", "path", "cluster_size"]
+    assert [n for n, _ in M.MoeReaderDebug._fields_][-2:] == ["ev_before", "ev_after"]
+    assert C.sizeof(M.MoeReaderDebug) == 12 * C.sizeof(C.c_void_p)
+
+
 def test_forward_without_recovery_needs_no_factors(lib):
     # r = 0: the factor pointers may be NULL; validation passes up to the
     # workspace-size check, which fails here on purpose (nothing launches).

@@ -20,9 +20,9 @@ def bench():
 def test_launches_per_step(bench):
     assert bench.launches_per_step(1, 0) == 1   # in-kernel routing
     assert bench.launches_per_step(2, 1) == 1
-    assert bench.launches_per_step(4, 1) == 3   # route, select, one-cluster reader
     assert bench.launches_per_step(3, 0) == 7   # route, select, five streamed stages
     assert bench.launches_per_step(1, 2) == 7
+    assert bench.launches_per_step(1, 0, d=4096) == 7  # the one-cluster reader runs d <= 2048
 
 
 def test_workload_names(bench):

@@ -1,6 +1,10 @@
-"""GPU parity of both readers at batch sizes where the automatic choice does
-not take them: the streamed kernels at one and two tokens, the one-cluster
-kernel above two tokens, and the two paths against each other."""
+"""GPU parity of both readers where the automatic choice does not take
+them: the streamed kernels at one and two tokens, the one-cluster reader at
+pinned cluster sizes, and the two paths against each other.  The reader is
+chosen per call (the layer's `path` field), so two threads that ask for
+different readers at the same time each get their own."""
+import threading
+
 import numpy as np
 import pytest
 import torch
@@ -12,7 +16,7 @@ from tests.gpu_helpers import OracleCache, bf16_ulp, check_pair
 pytestmark = pytest.mark.gpu
 
 QWEN = synth.QWEN3_30B_A3B
-CLUSTER, STREAMED = 1, 2
+AUTO, CLUSTER, STREAMED = 0, 1, 2
 
 
 @pytest.fixture(scope="module")
@@ -29,50 +33,67 @@ def qwen():
     return W, M.Layer(W, top_e=8).build_sketch(seed), OracleCache(W, seed, 32)
 
 
-@pytest.fixture
-def path(request):
-    M.moe_reader_set_path(request.param)
-    try:
-        yield request.param
-    finally:
-        M.moe_reader_set_path(0)
+class using:
+    """Sets a layer's reader path and cluster size for the block."""
+
+    def __init__(self, layer, path=AUTO, cluster_size=0):
+        self.layer, self.path, self.cs = layer, path, cluster_size
+
+    def __enter__(self):
+        self.layer.path, self.layer.cluster_size = self.path, self.cs
+        return self.layer
+
+    def __exit__(self, *exc):
+        self.layer.path, self.layer.cluster_size = AUTO, 0
 
 
-@pytest.mark.parametrize("path", [STREAMED], indirect=True)
 @pytest.mark.parametrize("B", [1, 2])
 @pytest.mark.parametrize("recovery_input", [0, 1])
-def test_streamed_tiny_small_batch(tiny, path, B, recovery_input):
+def test_streamed_tiny_small_batch(tiny, B, recovery_input):
     _, layer, oc = tiny
-    for seed in range(3):
-        check_pair(layer, oc, synth.tokens(256, B, seed=seed), k=24, c=48, top_e=2, recovery_input=recovery_input)
+    with using(layer, STREAMED):
+        for seed in range(3):
+            check_pair(layer, oc, synth.tokens(256, B, seed=seed), k=24, c=48, top_e=2, recovery_input=recovery_input)
 
 
-@pytest.mark.parametrize("path", [STREAMED], indirect=True)
 @pytest.mark.parametrize("k,c,r", [(1, 1, 8), (128, 128, 0), (5, 17, 0), (64, 100, 8)])
-def test_streamed_tiny_budgets_batch1(tiny, path, k, c, r):
+def test_streamed_tiny_budgets_batch1(tiny, k, c, r):
     W, layer, _ = tiny
     oc = OracleCache(W, synth.rot_seed(0), r)
-    check_pair(layer, oc, synth.tokens(256, 1, seed=12), k=k, c=c, top_e=2)
+    with using(layer, STREAMED):
+        check_pair(layer, oc, synth.tokens(256, 1, seed=12), k=k, c=c, top_e=2)
 
 
-@pytest.mark.parametrize("path", [STREAMED], indirect=True)
 @pytest.mark.parametrize("recovery_input", [0, 1])
-def test_streamed_qwen_batch1(qwen, path, recovery_input):
+def test_streamed_qwen_batch1(qwen, recovery_input):
     _, layer, oc = qwen
-    for seed in (0, 7):
-        check_pair(layer, oc, synth.tokens(2048, 1, seed=seed), k=136, c=272, top_e=8, recovery_input=recovery_input)
+    with using(layer, STREAMED):
+        for seed in (0, 7):
+            check_pair(layer, oc, synth.tokens(2048, 1, seed=seed), k=136, c=272, top_e=8,
+                       recovery_input=recovery_input)
 
 
-@pytest.mark.parametrize("path", [CLUSTER], indirect=True)
-@pytest.mark.parametrize("B", [3, 4])
-def test_cluster_path_above_two_tokens(tiny, qwen, path, B):
-    _, lt, ot = tiny
-    check_pair(lt, ot, synth.tokens(256, B, seed=40 + B), k=24, c=48, top_e=2)
-    _, lq, oq = qwen
-    check_pair(lq, oq, synth.tokens(2048, B, seed=50 + B), k=136, c=272, top_e=8)
+@pytest.mark.parametrize("cs", [2, 4, 6, 8])
+@pytest.mark.parametrize("B", [1, 2])
+def test_cluster_reader_pinned_sizes_tiny(tiny, cs, B):
+    """Other channel and column partitions of the one-cluster reader (the
+    automatic size differs), with every exact-stage slot count they give."""
+    _, layer, oc = tiny
+    with using(layer, CLUSTER, cs):
+        check_pair(layer, oc, synth.tokens(256, B, seed=60 + cs), k=24, c=48, top_e=2)
 
 
-@pytest.mark.parametrize("B", [1, 3, 16])
+@pytest.mark.parametrize("cs", [6, 8, 16])
+def test_cluster_reader_pinned_sizes_qwen(qwen, cs):
+    """Six CTAs own 128 channels each (exact rows in several rounds per
+    warp), sixteen own 48: both ends of the partition at the layer shape."""
+    _, layer, oc = qwen
+    with using(layer, CLUSTER, cs):
+        check_pair(layer, oc, synth.tokens(2048, 1, seed=80 + cs), k=136, c=272, top_e=8)
+        check_pair(layer, oc, synth.tokens(2048, 2, seed=90 + cs), k=136, c=272, top_e=8)
+
+
+@pytest.mark.parametrize("B", [1, 2])
 def test_paths_agree(qwen, B):
     """Routing, sketch dots, scores and candidate sets agree bit for bit
     between the two readers; kept sets agree; outputs agree to the rounding
@@ -83,11 +104,9 @@ def test_paths_agree(qwen, B):
     out = {}
     try:
         for p in (CLUSTER, STREAMED):
-            M.moe_reader_set_path(p)
-            out[p] = layer.forward(x, k=136, c=272, debug=True)
+            out[p] = layer.forward(x, k=136, c=272, debug=True, path=p)
             layer.check()
     finally:
-        M.moe_reader_set_path(0)
         layer.set_lowrank(None, None)
     (y1, d1), (y2, d2) = out[CLUSTER], out[STREAMED]
     for n in ("ids", "dot_gate", "dot_up", "cand"):
@@ -97,3 +116,31 @@ def test_paths_agree(qwen, B):
     assert (k1 == k2).mean() > 0.99  # near-tie swaps of |a| only
     a, b = y1.float().cpu().numpy(), y2.float().cpu().numpy()
     assert np.all(np.abs(a - b) <= 2 * bf16_ulp(np.maximum(np.abs(a), np.abs(b))) + 1e-3)
+
+
+def test_two_threads_get_their_own_reader(qwen):
+    """Two host threads run steps at the same time, one asking for the
+    one-cluster reader and one for the streamed reader (separate layers'
+    descriptors, workspaces and streams).  Each gets the reader it asked for:
+    only the one-cluster reader writes stage time stamps."""
+    _, layer, _ = qwen
+    x = synth.tokens(2048, 1, seed=5).cuda()
+    lay2 = M.Layer.__new__(M.Layer)
+    lay2.__dict__.update(layer.__dict__)
+    lay2._ws = None  # its own workspace
+    res = {}
+
+    def run(lay, p):
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            for _ in range(20):
+                _, dbg = lay.forward(x, k=136, c=272, debug=True, path=p, stream=s)
+            s.synchronize()
+        res[p] = int((dbg["phase_ns"].cpu() != 0).sum())
+
+    th = [threading.Thread(target=run, args=(layer, CLUSTER)), threading.Thread(target=run, args=(lay2, STREAMED))]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    assert res[CLUSTER] > 0 and res[STREAMED] == 0, res

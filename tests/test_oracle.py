@@ -515,3 +515,17 @@ def test_oracle_tiny_forward_regression():
         assert dbg["cand"][0, s].tolist() == [int(v) for v in rec[f"cand{s}"]]
         assert dbg["kept"][0, s].tolist() == [int(v) for v in rec[f"kept{s}"]]
     assert y.ravel().tolist() == [int(v, 16) for v in rec["y"]]
+
+
+def test_openmp_pairs_give_the_same_bits(tiny):
+    """The oracle's OpenMP variant runs the (token, slot) readers in
+    parallel and combines serially: every output and stage value equals the
+    single-threaded run bit for bit, whatever the thread count."""
+    W, sk, lr = tiny
+    x = synth.tokens(256, 7, seed=21)
+    ref = O.forward(x, W, sk, lr, k=24, c=48, r=8, top_e=2, debug=True)
+    for threads in (2, 5, 16):
+        got = O.forward(x, W, sk, lr, k=24, c=48, r=8, top_e=2, debug=True, threads=threads)
+        assert np.array_equal(ref[0], got[0]) and np.array_equal(ref[1], got[1])
+        for n in ref[2]:
+            assert np.array_equal(ref[2][n], got[2][n]), n
