@@ -138,6 +138,7 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   cudaError_t e = cudaSuccess;
   ra.ep_rank = ep_rank;
   ra.ep_size = ep_size;
+  // steps of at most two tokens route inside the cluster kernels
   if (!moe::fused_routing(B) || streamed) {
     e = moe::launch_route(ra, s);
     if (e != cudaSuccess) return cuda_fail(e, "route launch");

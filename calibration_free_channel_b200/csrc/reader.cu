@@ -41,6 +41,7 @@
 // byte-wise dots on pre-masked code words.
 #include "common.cuh"
 #include "kernels.h"
+#include "rotate.cuh"
 #include "select.cuh"
 
 namespace moe {
@@ -246,12 +247,13 @@ __device__ bool load_item_table(const ExpertArgs& a, int cid, int* misc, int NT)
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     const bool ok_cid = cid < a.ws.max_items;
+    // written by the previous kernel of the step: read through L2
     int v = 0;
-    if (lane == 0) v = *a.ws.n_items;
-    else if (lane == 1 && ok_cid) v = a.ws.item_e[cid];
-    else if (lane == 2 && ok_cid) v = a.ws.item_n[cid];
-    else if (lane >= 4 && lane < 4 + kMaxGroup && ok_cid) v = a.ws.item_tok[cid * kMaxGroup + lane - 4];
-    else if (lane >= 8 && lane < 8 + kMaxGroup && ok_cid) v = a.ws.item_slot[cid * kMaxGroup + lane - 8];
+    if (lane == 0) v = __ldcg(a.ws.n_items);
+    else if (lane == 1 && ok_cid) v = __ldcg(a.ws.item_e + cid);
+    else if (lane == 2 && ok_cid) v = __ldcg(a.ws.item_n + cid);
+    else if (lane >= 4 && lane < 4 + kMaxGroup && ok_cid) v = __ldcg(a.ws.item_tok + cid * kMaxGroup + lane - 4);
+    else if (lane >= 8 && lane < 8 + kMaxGroup && ok_cid) v = __ldcg(a.ws.item_slot + cid * kMaxGroup + lane - 8);
     const int n_items = __shfl_sync(kFull, v, 0);
     int e = __shfl_sync(kFull, v, 1), n = __shfl_sync(kFull, v, 2);
     if (!(cid < n_items && ok_cid)) {
@@ -273,7 +275,7 @@ __device__ bool load_item_table(const ExpertArgs& a, int cid, int* misc, int NT)
       misc[MI_TOK + t] = tok;
       misc[MI_SLOT + t] = sl;
       misc[MI_TIX + t] = t;  // tokens are loaded in item order
-      reinterpret_cast<float*>(misc + MI_CX)[t] = a.ws.cx[tok];
+      reinterpret_cast<float*>(misc + MI_CX)[t] = __ldcg(a.ws.cx + tok);
     }
     if (lane == 0) {
       misc[MI_E] = e;
@@ -298,96 +300,6 @@ __device__ void load_tokens(const ExpertArgs& a, const Layout& L, char* smem, co
       for (int j = threadIdx.x; j < L.d8 / 2; j += NTHR)
         qs[t * (L.d8 / 2) + j] = __ldcg(reinterpret_cast<const uint4*>(a.ws.q + (size_t)tok * a.d) + j);
   }
-}
-
-// Rotation + int8 quantisation of smem token t: v = FWHT(s . x) in the fp32
-// scratch (d floats), q = rint(127 v / amax), c_x = amax / (127 d).  Stages
-// h = 1, 2 run in registers (thread c holds elements 4c .. 4c+3) and
-// h = 4 .. 64 across the lanes of a warp (a warp holds 128 consecutive
-// elements); from h = 128 on, each pass over shared memory applies two stages
-// (h and 2h) to four elements held in registers, and a last single stage
-// runs alone when the count is odd.  Every element sees the reference
-// butterflies (a + b, a - b) of every stage in the reference stage order, so
-// the bits equal the reference transform's.  d >= 256.  sv_pre holds the
-// signs of elements 4T .. 4T+3, loaded early by the caller.  xt: the token
-// (bf16, shared memory), qt: its int8 codes (shared memory).
-__device__ void rotate_quantize(const ExpertArgs& a, const uint16_t* xt, int8_t* qt, float* v, float* cx_out,
-                                float* red, char4 sv_pre) {
-  const int d = a.d, d8 = d >> 3;
-  const int T = threadIdx.x, lane = T & 31, warp = T >> 5;
-  for (int c = T; c < 2 * d8; c += NTHR) {  // d / 4 is a multiple of 32: whole warps
-    const uint2 xv = reinterpret_cast<const uint2*>(xt)[c];
-    const char4 sv = c == T ? sv_pre : reinterpret_cast<const char4*>(a.rot_sign)[c];
-    float r0 = (float)sv.x * bf16lo(xv.x), r1 = (float)sv.y * bf16hi(xv.x);
-    float r2 = (float)sv.z * bf16lo(xv.y), r3 = (float)sv.w * bf16hi(xv.y);
-    float b0 = __fadd_rn(r0, r1), b1 = __fsub_rn(r0, r1), b2 = __fadd_rn(r2, r3), b3 = __fsub_rn(r2, r3);  // h = 1
-    r0 = __fadd_rn(b0, b2);  // h = 2
-    r2 = __fsub_rn(b0, b2);
-    r1 = __fadd_rn(b1, b3);
-    r3 = __fsub_rn(b1, b3);
-#pragma unroll 1
-    for (int m = 1; m < 32; m <<= 1) {  // h = 4m: partner lane ^ m
-      const bool up = lane & m;
-      const float p0 = __shfl_xor_sync(kFull, r0, m), p1 = __shfl_xor_sync(kFull, r1, m);
-      const float p2 = __shfl_xor_sync(kFull, r2, m), p3 = __shfl_xor_sync(kFull, r3, m);
-      r0 = up ? __fsub_rn(p0, r0) : __fadd_rn(r0, p0);
-      r1 = up ? __fsub_rn(p1, r1) : __fadd_rn(r1, p1);
-      r2 = up ? __fsub_rn(p2, r2) : __fadd_rn(r2, p2);
-      r3 = up ? __fsub_rn(p3, r3) : __fadd_rn(r3, p3);
-    }
-    reinterpret_cast<float4*>(v)[c] = make_float4(r0, r1, r2, r3);
-  }
-  float m = 0.0f;  // max |v| over this thread's outputs of the last pass
-#pragma unroll 1
-  for (int h = 128, lh = 7; h < d;) {
-    __syncthreads();
-    m = 0.0f;
-    if (2 * h < d) {
-      for (int p = T; p < 2 * d8; p += NTHR) {
-        const int b = ((p >> lh) << (lh + 2)) | (p & (h - 1));
-        const float a0 = v[b], a1 = v[b + h], a2 = v[b + 2 * h], a3 = v[b + 3 * h];
-        const float s0 = __fadd_rn(a0, a1), s1 = __fsub_rn(a0, a1);  // stage h
-        const float s2 = __fadd_rn(a2, a3), s3 = __fsub_rn(a2, a3);
-        const float o0 = __fadd_rn(s0, s2), o2 = __fsub_rn(s0, s2);  // stage 2h
-        const float o1 = __fadd_rn(s1, s3), o3 = __fsub_rn(s1, s3);
-        v[b] = o0;
-        v[b + h] = o1;
-        v[b + 2 * h] = o2;
-        v[b + 3 * h] = o3;
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(o0), fabsf(o1)), fmaxf(fabsf(o2), fabsf(o3))));
-      }
-      h <<= 2;
-      lh += 2;
-    } else {  // the last stage, h = d / 2
-      for (int p = T; p < 4 * d8; p += NTHR) {
-        const float x0 = v[p], x1 = v[p + h];
-        const float o0 = __fadd_rn(x0, x1), o1 = __fsub_rn(x0, x1);
-        v[p] = o0;
-        v[p + h] = o1;
-        m = fmaxf(m, fmaxf(fabsf(o0), fabsf(o1)));
-      }
-      h <<= 1;
-      lh += 1;
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-  if (lane == 0) red[warp] = m;
-  __syncthreads();
-  float amax = 0.0f;
-#pragma unroll
-  for (int w = 0; w < NWARP; w += 4) {
-    const float4 r4 = reinterpret_cast<const float4*>(red)[w >> 2];
-    amax = fmaxf(amax, fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w)));
-  }
-  int8_t* q = qt;
-  for (int j = T; j < d; j += NTHR) {
-    int n = 0;
-    if (amax > 0.0f) n = max(-127, min(127, __float2int_rn(__fdiv_rn(__fmul_rn(v[j], 127.0f), amax))));
-    q[j] = (int8_t)n;
-  }
-  if (T == 0) *cx_out = amax > 0.0f ? __fdiv_rn(amax, __fmul_rn(127.0f, (float)d)) : 0.0f;
-  __syncthreads();
 }
 
 // Stage time stamps (globaltimer, ns) of the first CTA of each cluster.
@@ -419,15 +331,29 @@ __device__ bool fused_route(const ExpertArgs& a, const LT& L, char* smem, int* m
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int e0 = L.ex0[rank], ne = L.ex0[rank + 1] - e0;
   uint4* xs = reinterpret_cast<uint4*>(smem + L.x);
+  // the tokens first (every later step needs them), then the router rows
+  uint4 xv[NT][2];
+#pragma unroll
+  for (int t = 0; t < NT; t++)
+#pragma unroll
+    for (int k = 0; k < 2; k++) {
+      const int j = threadIdx.x + k * NTHR;
+      xv[t][k] = t < B && j < L.d8 ? __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d) + j)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+    }
   uint4 w[8];
   double bias_w = 0.0;
   if (warp < ne) {
     load_row8(reinterpret_cast<const uint4*>(a.w_router + (size_t)(e0 + warp) * a.d), 0, L.d8, lane, w);
     if (a.bias) bias_w = (double)__ldg(a.bias + e0 + warp);
   }
-  for (int t = 0; t < B; t++)
-    for (int j = threadIdx.x; j < L.d8; j += NTHR)
-      xs[t * L.d8 + j] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d) + j);
+#pragma unroll
+  for (int t = 0; t < NT; t++)
+#pragma unroll
+    for (int k = 0; k < 2; k++) {
+      const int j = threadIdx.x + k * NTHR;
+      if (t < B && j < L.d8) xs[t * L.d8 + j] = xv[t][k];
+    }
   if (threadIdx.x < B) misc[MI_TOK + threadIdx.x] = threadIdx.x;
   __syncthreads();
   mid();
@@ -599,14 +525,11 @@ __device__ void write_and_combine(const ExpertArgs& a, int rank, int j0, int nco
     const int tok = misc[MI_TOK + t];
     for (int col = threadIdx.x; col < ncols; col += NTHR) {
       const int j = j0 + col;
-      float v[16];
-#pragma unroll
-      for (int s = 0; s < 16; s++)
-        v[s] = s < a.top_e ? __ldcg(&a.ws.ye[((size_t)tok * a.top_e + s) * a.d + j]) : 0.0f;
+      // slot order; four loads in flight at a time
       float acc = 0.0f;
-#pragma unroll
-      for (int s = 0; s < 16; s++)
-        if (s < a.top_e) acc = fmaf(wts[tok * a.top_e + s], v[s], acc);
+#pragma unroll 4
+      for (int s = 0; s < a.top_e; s++)
+        acc = fmaf(wts[tok * a.top_e + s], __ldcg(&a.ws.ye[((size_t)tok * a.top_e + s) * a.d + j]), acc);
       if (a.residual) acc += bf16f(a.residual[(size_t)tok * a.d + j]);
       a.y[(size_t)tok * a.d + j] = f2bf16(acc);
     }
@@ -729,10 +652,11 @@ constexpr int kMaxDSlots = 64;      // down-row slots
 
 struct RLayout {
   int mbar, misc, x, q, logit, alpha, ubar, vown, ahat, aown, vloc, rloc, listc, listk, flags, rows, drows, kslot,
-      kco, dcnt, gu, zred, zparts, ztot, ybuf, ring, total;
+      kco, dcnt, gu, zred, zparts, ztot, ybuf, cntb, ring, total;
   int P, Pext;  // exact-stage slots (gate + up rows of one channel, 4d bytes each): P per warp, one more
                 // for warps 0 .. Pext - 1
   int W;        // warps that own slots (all when P >= 1)
+  int ringb;    // ring bytes
   int ndslot;   // down-row slots (2d bytes each)
   int nskbuf;   // 16-channel sketch chunks resident at once
   int own_max, om4, cols_max, d8, skc, rr, nsteps;
@@ -786,7 +710,8 @@ __host__ inline RLayout make_rlayout(int NT, int B, int E, int I, int d, int r, 
   L.kslot = take(L.om4 * 4);
   L.kco = take(NT * L.om4 * 4);
   L.dcnt = take(2 * NT * 16 * 4);
-  L.gu = take(NWARP * 4 * NT * 2 * 4);
+  L.gu = take(L.om4 * NT * 2 * 4);
+  L.cntb = take(cs * L.om4 * 4);
   L.zred = take(NWARP * NT * L.rr * 4);
   L.zparts = take(cs * NT * L.rr * 4);
   L.ztot = take(NT * L.rr * 4);
@@ -799,14 +724,17 @@ __host__ inline RLayout make_rlayout(int NT, int B, int E, int I, int d, int r, 
   L.Pext = ns % NWARP;
   L.W = L.P > 0 ? NWARP : L.Pext;
   L.ndslot = ring / (2 * d) < kMaxDSlots ? ring / (2 * d) : kMaxDSlots;
-  L.nskbuf = ring / (8 * d) < kSkBars ? ring / (8 * d) : kSkBars;
+  // sketch chunks stay clear of the transform's fp32 scratch at the ring's end
+  L.nskbuf = (ring - 4 * d) / (8 * d) < kSkBars ? (ring - 4 * d) / (8 * d) : kSkBars;
+  L.ringb = ring;
   L.total = o + ring;
   return L;
 }
 
 // misc ints of the sparse kernel (beyond the shared positions above)
-enum { MI_NSPEC = 8, MI_NROWS = 9, MI_NDC = 10, MI_NK = 11 };
-static_assert((int)MI_NK < (int)MI_DONE, "misc positions");
+enum { MI_NSPEC = 8, MI_NROWS = 9, MI_NDC = 10, MI_NK = 11, MI_SQ = 13 };  // MI_SQ: B <= 2 ints
+static_assert((int)MI_NK < (int)MI_DONE && (int)MI_SQ > (int)MI_DONE && (int)MI_SQ + 2 <= (int)MI_TOK,
+              "misc positions");
 // flags of an own channel: candidate of token t (bit t), kept by token t
 // (bit 2 + t), started before the candidates were known (bit 4)
 constexpr unsigned char kFlagSpec = 16;
@@ -862,30 +790,36 @@ __device__ void local_ranks(const uint64_t* v, int n, int* rank) {
   }
 }
 
-// Entries above v in the sorted lists (descending, zero padded, om4 entries
-// each) of CTAs q, q + 4, q + 8, q + 12 other than `self`: binary searches in
-// lockstep.
-__device__ __forceinline__ int count_above(uint64_t v, const uint64_t* lists, int om4, int nsteps, int cs, int self,
-                                           int q) {
-  int lo[4], hi[4];
-#pragma unroll
-  for (int j = 0; j < 4; j++) {
-    const int o = q + 4 * j;
-    lo[j] = 0;
-    hi[j] = o < cs && o != self ? om4 : 0;
-  }
+// For the n entries of this CTA's sorted list `mine` (descending), how many
+// entries of the sorted list of CTA o beat each one: warp o (o < cs, o !=
+// self) merges the two lists, lane l taking a run of consecutive own entries
+// (one binary search for its first, then steps forward).  cnt[o * om4 + r]
+// gets the count for own entry r.  Lists are zero padded to om4 entries;
+// zero entries never beat anything.
+__device__ __forceinline__ void merge_counts(const uint64_t* lists, const uint64_t* mine, int n, int om4, int nsteps,
+                                             int cs, int self, int* cnt) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp >= cs || warp == self || n <= 0) return;
+  const uint64_t* L = lists + (size_t)warp * om4;
+  const int run = (n + 31) >> 5, r0 = lane * run, r1 = min(n, r0 + run);
+  if (r0 >= r1) return;
+  // first own entry of the run: entries of L above it
+  const uint64_t v0 = mine[r0];
+  int lo = 0, hi = om4;
 #pragma unroll 1
-  for (int s = 0; s < nsteps; s++) {
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-      if (lo[j] < hi[j]) {
-        const int mid = (lo[j] + hi[j]) >> 1;
-        if (lists[(q + 4 * j) * om4 + mid] > v) lo[j] = mid + 1;
-        else hi[j] = mid;
-      }
-    }
+  for (int s = 0; s < nsteps && lo < hi; s++) {
+    const int mid = (lo + hi) >> 1;
+    if (L[mid] > v0) lo = mid + 1;
+    else hi = mid;
   }
-  return lo[0] + lo[1] + lo[2] + lo[3];
+  cnt[warp * om4 + r0] = lo;
+  // the rest of the run: own entries fall, so the count only grows
+#pragma unroll 1
+  for (int r = r0 + 1; r < r1; r++) {
+    const uint64_t v = mine[r];
+    while (lo < om4 && L[lo] > v) lo++;
+    cnt[warp * om4 + r] = lo;
+  }
 }
 
 // The sorted list of the nonzero keys among n own keys (local ranks given;
@@ -940,19 +874,14 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
   const uint16_t* xs = reinterpret_cast<const uint16_t*>(smem + L.x);
   int8_t* qs = reinterpret_cast<int8_t*>(smem + L.q);
   float* cxs = reinterpret_cast<float*>(misc + MI_CX);
+
   char4 sv_pre = make_char4(0, 0, 0, 0);  // rotation signs of elements 4 tid .. 4 tid + 3
   if (tid < d / 4) sv_pre = __ldg(reinterpret_cast<const char4*>(a.rot_sign) + tid);
 
-  // ------------------------------------------------ R: routing + rotation
-  // every token is rotated and quantised while the router rows are in flight
-  // (the fp32 scratch of the transform is the start of the ring)
-  const bool has_item = fused_route<NT>(a, L, smem, misc, cs, rank, cid, cluster, [&] {
-#pragma unroll 1
-    for (int t = 0; t < a.B; t++)
-      rotate_quantize(a, xs + (size_t)t * d, qs + (size_t)t * d, reinterpret_cast<float*>(ring), cxs + t,
-                      reinterpret_cast<float*>(misc + MI_RED), sv_pre);
-    if (DBG) stamp(a, cid, rank, 1);
-  });
+  // ---------------------------------------------------------- R: routing
+  // (every CTA of every cluster takes the same top-e from the exchanged
+  // logits; a cluster past the last work item has nothing to do)
+  const bool has_item = fused_route<NT>(a, L, smem, misc, cs, rank, cid, cluster, [] {});
   if (!has_item) return;  // uniform per cluster; no exchange follows
   if (DBG) stamp(a, cid, rank, 4);
   const int e = misc[MI_E], n = misc[MI_N];
@@ -965,7 +894,6 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
   // 0's barrier, which every warp waits for first), the factor rows of the
   // own channels and the V rows of the own columns: all in flight at once
   if (lane == 0) {
-    fence_proxy_async();  // the ring held the transform scratch (generic stores)
     if (warp == 0 && I % 4 == 0 && nown > 0) {
       mbar_expect_tx_only(&skbars[0], 2 * nown * 4);
       bulk_g2s(smem + L.alpha, a.alpha_gate + (size_t)e * I + i0, nown * 4, &skbars[0]);
@@ -987,10 +915,17 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
       alu[li] = __ldg(a.alpha_up + (size_t)e * I + i0 + li);
     }
   }
+  // every token is rotated and quantised while the copies are in flight (the
+  // fp32 scratch of the transform sits past the sketch buffers); its block
+  // barriers also publish the scale loads above
+#pragma unroll 1
+  for (int t = 0; t < a.B; t++)
+    rotate_quantize(a, xs + (size_t)t * d, qs + (size_t)t * d, reinterpret_cast<float*>(ring + L.ringb - 4 * d),
+                    cxs + t, reinterpret_cast<float*>(misc + MI_RED), sv_pre, misc + MI_SQ + t);
+  if (DBG) stamp(a, cid, rank, 1);
   int tix[NT];
 #pragma unroll
   for (int t = 0; t < NT; t++) tix[t] = misc[MI_TIX + (t < n ? t : 0)];
-  __syncthreads();
 
   float* ahat = reinterpret_cast<float*>(smem + L.ahat);        // [NT, om] sketch estimates, own channels
   float* aown = reinterpret_cast<float*>(smem + L.aown);        // [NT, om] exact a, own candidates
@@ -1005,39 +940,33 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
   const uint16_t* ub = reinterpret_cast<const uint16_t*>(smem + L.ubar);
 
   // ---------------------------------------------------------- S: screen
-  // warp w takes channel 16 j + w of every sketch chunk j.  Each channel's
-  // dots are reduced over the warp and parked; every 4 chunks (and at the
-  // end) one pass over the lanes turns the parked sums into sigma and ahat.
+  // warp w takes channel 16 j + w of every sketch chunk j: per chunk the
+  // lanes' partial dots, then the warp reduction of the previous chunk (its
+  // shuffles overlap these dots); the sums are parked per channel and one
+  // pass over (channel, token) afterwards turns them into scores.
+  int* gsum = reinterpret_cast<int*>(smem + L.gu);  // [om, NT, 2] exact G, U (code offset not yet removed)
   {
     const int nv = d >> 6;  // 16-byte sketch vectors per row
-    int sq[NT];
-#pragma unroll
-    for (int t = 0; t < NT; t++) {
-      const uint4* qv = reinterpret_cast<const uint4*>(qs + (size_t)tix[t] * d);
-      int s = 0;
-      for (int j = lane; j < L.d8 / 2; j += 32) {
-        const uint4 q4 = qv[j];
-        s = __dp4a((int)q4.x, 0x01010101, s);
-        s = __dp4a((int)q4.y, 0x01010101, s);
-        s = __dp4a((int)q4.z, 0x01010101, s);
-        s = __dp4a((int)q4.w, 0x01010101, s);
-      }
-      sq[t] = warp_sum(s);  // sum of the token's activations: the code offset
-    }
-    float zacc[NT][4];
-#pragma unroll
-    for (int t = 0; t < NT; t++)
-#pragma unroll
-      for (int kk = 0; kk < 4; kk++) zacc[t][kk] = 0.0f;
-    bool uv_ready = r == 0;
-    uint4 qr[NT][4];  // activations of sketch vector `lane` (the row's first 32 vectors)
+    uint4 qr[NT][4];        // activations of sketch vector `lane` (the row's first 32 vectors)
 #pragma unroll
     for (int t = 0; t < NT; t++) {
       const uint4* qv = reinterpret_cast<const uint4*>(qs + (size_t)tix[t] * d);
 #pragma unroll
       for (int kk = 0; kk < 4; kk++) qr[t][kk] = lane < nv ? qv[4 * lane + kk] : make_uint4(0u, 0u, 0u, 0u);
     }
-    int* gu = reinterpret_cast<int*>(smem + L.gu) + warp * 4 * NT * 2;  // parked sums
+    int pG[NT], pU[NT];  // the previous chunk's lane partials
+#pragma unroll
+    for (int t = 0; t < NT; t++) pG[t] = pU[t] = 0;
+    auto park = [&](int jc) {  // reduce chunk jc's partials over the warp and park them
+      int gs, us;
+      reduce_gu<NT>(pG, pU, gs, us);
+      const int lc = 16 * jc + warp;
+      if (lane < 16 && (lane & 7) == 0 && lc < nown) {
+        const int t = NT == 2 ? lane >> 3 : 0;
+        gsum[(lc * NT + t) * 2] = gs;
+        gsum[(lc * NT + t) * 2 + 1] = us;
+      }
+    };
     int rb = 0, par = 0;  // first chunk of the resident round, parity of its barriers
 #pragma unroll 1
     for (int j = 0; j < nchunk; j++) {
@@ -1048,7 +977,6 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
         rb = j;
         par ^= 1;
         if (tid == 0) {
-          fence_proxy_async();
           const int c1 = min(nchunk, j + L.nskbuf);
           for (int ch = j; ch < c1; ch++) issue_sketch(a, L, ring, skbars, e, i0, i1, ch, ch - j);
         }
@@ -1095,74 +1023,36 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
           U[t] = code_dot_total(ua[t]);
         }
       }
-      int gs, us;
-      reduce_gu<NT>(G, U, gs, us);
-      if (lane < 16 && (lane & 7) == 0) {
-        const int t = NT == 2 ? lane >> 3 : 0;
-        gu[((j & 3) * NT + t) * 2] = gs;
-        gu[((j & 3) * NT + t) * 2 + 1] = us;
-      }
-      if ((j & 3) == 3 || j == nchunk - 1) {
-        // the batch's epilogue: lane (channel c, token t), c < 4, t < NT
-        __syncwarp();
-        const int jb = j & ~3;
-        const int c = lane / NT, t = lane - c * NT;
-        const int lc = 16 * (jb + c) + warp;
-        const bool valid = lane < 4 * NT && jb + c <= j && lc < nown && t < n;
-        int g2 = 0, u2 = 0;
-        if (lane < 4 * NT) {
-          g2 = gu[lane * 2] - (NT == 2 && t ? sq[NT - 1] : sq[0]);
-          u2 = gu[lane * 2 + 1] - (NT == 2 && t ? sq[NT - 1] : sq[0]);
-        }
-        const float cx = cxs[tix[NT == 2 && t ? NT - 1 : 0]];
-        const float gh = __fmul_rn(__fmul_rn((float)g2, valid ? alg[lc] : 0.0f), cx);
-        const float uh = __fmul_rn(__fmul_rn((float)u2, valid ? alu[lc] : 0.0f), cx);
-        const float ah = __fmul_rn(silu_r(gh), uh);
-        if (valid) {
-          vloc[t * om + lc] = sort_key(fabsf(ah), i0 + lc);
-          ahat[t * om + lc] = ah;
-          if (DBG) {
-            const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * I + i0 + lc;
-            if (a.dbg_G) a.dbg_G[off] = g2;
-            if (a.dbg_U) a.dbg_U[off] = u2;
-            if (a.dbg_sigma) a.dbg_sigma[off] = fabsf(ah);
-          }
-        }
-        // partial recovery input: sum over this warp's channels of ahat_i Ubar_i
-        if (r > 0) {
-          if (!uv_ready) {
-            if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
-            uv_ready = true;
-          }
+      if (j > 0) park(j - 1);
 #pragma unroll
-          for (int cc = 0; cc < 4; cc++) {
-            const int lcc = 16 * (jb + cc) + warp;
-            if (jb + cc <= j && lcc < nown) {
-#pragma unroll
-              for (int tt = 0; tt < NT; tt++) {
-                const float aht = __shfl_sync(kFull, ah, cc * NT + tt);
-#pragma unroll
-                for (int kk = 0; kk < 4; kk++) {
-                  const int p = lane + 32 * kk;
-                  if (p < r && tt < n) zacc[tt][kk] = fmaf(aht, bf16f(ub[lcc * r + p]), zacc[tt][kk]);
-                }
-              }
-            }
-          }
-        }
-        __syncwarp();
+      for (int t = 0; t < NT; t++) {
+        pG[t] = G[t];
+        pU[t] = U[t];
       }
     }
+    if (nchunk > 0) park(nchunk - 1);
     if (warp == NWARP - 1) route_weights(a, L, smem, misc, cid, rank);
-    if (r > 0) {
-      float* zr = reinterpret_cast<float*>(smem + L.zred);  // [NWARP, NT, r]
-#pragma unroll
-      for (int t = 0; t < NT; t++)
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++) {
-          const int p = lane + 32 * kk;
-          if (p < r) zr[(warp * NT + t) * r + p] = zacc[t][kk];
-        }
+  }
+  __syncthreads();
+  // scores of (own channel, token): ghat = ((float)G alpha_g) c_x, uhat
+  // likewise, ahat = silu_r(ghat) uhat, sigma = |ahat|; G, U the exact dots
+  // less the code offset sum(q)
+#pragma unroll 1
+  for (int k = tid; k < nown * n; k += NTHR) {
+    const int lc = n == 2 ? k >> 1 : k, t = k - lc * n;
+    const int g2 = gsum[(lc * NT + t) * 2] - misc[MI_SQ + tix[NT == 2 && t ? NT - 1 : 0]];
+    const int u2 = gsum[(lc * NT + t) * 2 + 1] - misc[MI_SQ + tix[NT == 2 && t ? NT - 1 : 0]];
+    const float cx = cxs[tix[NT == 2 && t ? NT - 1 : 0]];
+    const float gh = __fmul_rn(__fmul_rn((float)g2, alg[lc]), cx);
+    const float uh = __fmul_rn(__fmul_rn((float)u2, alu[lc]), cx);
+    const float ah = __fmul_rn(silu_r(gh), uh);
+    vloc[t * om + lc] = sort_key(fabsf(ah), i0 + lc);
+    ahat[t * om + lc] = ah;
+    if (DBG) {
+      const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * I + i0 + lc;
+      if (a.dbg_G) a.dbg_G[off] = g2;
+      if (a.dbg_U) a.dbg_U[off] = u2;
+      if (a.dbg_sigma) a.dbg_sigma[off] = fabsf(ah);
     }
   }
   __syncthreads();  // sort keys and estimates of the own channels are in place; the sketch buffers are free
@@ -1189,18 +1079,6 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
       st_cluster(src, o, *src);
     }
   }
-  cluster_arrive();
-  if (r > 0) {
-    // the own partial of z_all = sum over the own channels of ahat_i Ubar_i
-    const float* zr = reinterpret_cast<const float*>(smem + L.zred);
-    for (int tp = tid; tp < n * r; tp += NTHR) {
-      const int t = tp / r, p = tp - t * r;
-      float zz = 0.0f;
-#pragma unroll 4
-      for (int w = 0; w < NWARP; w++) zz += zr[(w * NT + t) * r + p];
-      zparts[(rank * NT + t) * r + p] = zz;
-    }
-  }
   {
     // started early: each token's highest own scores, as many as the exact
     // stage's slots hold at once
@@ -1224,7 +1102,11 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
     __syncthreads();
     const int nspec = misc[MI_NSPEC];
     if (lane == 0) {
-      fence_proxy_async();  // the ring held the sketch
+      // the ring held the transform's scratch (generic stores of every
+      // thread, ordered by the block barriers since): order them before the
+      // copies.  Later copies into the ring only follow generic reads, whose
+      // values were consumed before the issuing warp's barrier.
+      fence_proxy_async();
       for (int m = 0; m < Pw; m++) {
         const int j = warp + W * m;
         if (j < nspec) issue_gate_up(a, e, i0 + rows[j], ring + (size_t)(sbase + m) * 4 * d, &wbars[m]);
@@ -1232,23 +1114,25 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
     }
   }
   if (DBG) stamp(a, cid, rank, 6);
+  // the pushes above had the selection's time to land: arrive (release) now
+  cluster_arrive();
   cluster_wait();
   if (DBG) stamp(a, cid, rank, 7);
   // candidate of token t: fewer than c channels of the expert beat it
+  int* cntb = reinterpret_cast<int*>(smem + L.cntb);  // [cs, om] entries of each peer's list above each own entry
 #pragma unroll 1
   for (int t = 0; t < n; t++) {
-#pragma unroll 1
-    for (int base = 0; base < nown; base += NTHR / 4) {
-      const int li = base + (tid >> 2), q = tid & 3;
-      const uint64_t v = li < nown ? vloc[t * om + li] : ~0ull;
-      int cnt = count_above(v, listc + (size_t)t * cs * om, om, L.nsteps, cs, rank, q);
-      cnt += __shfl_xor_sync(kFull, cnt, 1);
-      cnt += __shfl_xor_sync(kFull, cnt, 2);
-      if (li < nown && q == 0 && rloc[t * om + li] + cnt < a.c) atomicOr(reinterpret_cast<unsigned*>(flags) + (li >> 2),
-                                                                         (1u << t) << (8 * (li & 3)));
+    merge_counts(listc + (size_t)t * cs * om, listc + ((size_t)t * cs + rank) * om, nown, om, L.nsteps, cs, rank, cntb);
+    __syncthreads();
+    for (int li = tid; li < nown; li += NTHR) {
+      const int r0 = rloc[t * om + li];
+      int tot = r0;
+      for (int o = 0; o < cs; o++)
+        if (o != rank) tot += cntb[o * om + r0];
+      if (tot < a.c) atomicOr(reinterpret_cast<unsigned*>(flags) + (li >> 2), (1u << t) << (8 * (li & 3)));
     }
+    __syncthreads();
   }
-  __syncthreads();
   if (DBG) stamp(a, cid, rank, 8);
   // rows of the exact stage: the started ones, then the own candidates not
   // started yet; drows: every own candidate, ascending
@@ -1279,7 +1163,6 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
     const int nmine = warp < W && nrows > warp ? cdiv(nrows - warp, W) : 0;
     char* wring = ring + (size_t)sbase * 4 * d;
     if (lane == 0) {
-      fence_proxy_async();
       for (int m = 0; m < Pw && m < nmine; m++) {
         const int j = warp + W * m;
         if (j >= nspec) issue_gate_up(a, e, i0 + rows[j], wring + (size_t)m * 4 * d, &wbars[m]);
@@ -1321,21 +1204,13 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
       }
       __syncwarp();
       if (m + Pw < nmine && lane == 0) {
-        fence_proxy_async();
         issue_gate_up(a, e, i0 + rows[j + W * Pw], wring + (size_t)s * 4 * d, &wbars[s]);
       }
     }
   }
   __syncthreads();  // every issued row was consumed: the ring is free
   if (DBG) stamp(a, cid, rank, 9);
-  // the down rows of every own candidate start now (warp m % 16 copies row
-  // m); the top-k keeps about k / c of them.  If they do not fit, the kept
-  // ones follow the selection.
   const bool dspec = ndc <= L.ndslot;
-  if (dspec && lane == 0) {
-    fence_proxy_async();
-    for (int m = warp; m < ndc; m += NWARP) issue_down(a, e, i0 + drows[m], ring + (size_t)m * 2 * d, &dbars[m]);
-  }
 
   // ------------------------------------------------ k: kept (top-k by |a|)
   // each token's own candidates: sort keys of |a|, local ranks, sorted lists
@@ -1375,26 +1250,32 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
                                     "r"(dcnt[tid * 16 + rank])
                                     : "memory");
   }
+  // while the pushes land: the down rows of every own candidate start now
+  // (warp m % 16 copies row m; the top-k keeps about k / c of them; if they
+  // do not fit, the kept ones follow the selection)
+  if (dspec && lane == 0) {
+    for (int m = warp; m < ndc; m += NWARP) issue_down(a, e, i0 + drows[m], ring + (size_t)m * 2 * d, &dbars[m]);
+  }
   cluster_arrive();
   cluster_wait();
   if (DBG) stamp(a, cid, rank, 10);
 #pragma unroll 1
   for (int t = 0; t < n; t++) {
-#pragma unroll 1
-    for (int base = 0; base < ndc; base += NTHR / 4) {
-      const int m = base + (tid >> 2), q = tid & 3;
-      const bool cand = m < ndc && ((flags[drows[m < ndc ? m : 0]] >> t) & 1u);
-      const uint64_t v = cand ? vloc[t * om + m] : ~0ull;
-      int cnt = count_above(v, listk + (size_t)t * cs * om, om, L.nsteps, cs, rank, q);
-      cnt += __shfl_xor_sync(kFull, cnt, 1);
-      cnt += __shfl_xor_sync(kFull, cnt, 2);
-      if (cand && q == 0 && rloc[t * om + m] + cnt < a.k) {
-        const int li = drows[m];
-        atomicOr(reinterpret_cast<unsigned*>(flags) + (li >> 2), (4u << t) << (8 * (li & 3)));
-      }
+    int nct = 0;  // own candidates of token t (the nonzero entries of the own list)
+    for (int m = 0; m < ndc; m++) nct += (flags[drows[m]] >> t) & 1u;
+    merge_counts(listk + (size_t)t * cs * om, listk + ((size_t)t * cs + rank) * om, nct, om, L.nsteps, cs, rank, cntb);
+    __syncthreads();
+    for (int m = tid; m < ndc; m += NTHR) {
+      const int li = drows[m];
+      if (!((flags[li] >> t) & 1u)) continue;
+      const int r0 = rloc[t * om + m];
+      int tot = r0;
+      for (int o = 0; o < cs; o++)
+        if (o != rank) tot += cntb[o * om + r0];
+      if (tot < a.k) atomicOr(reinterpret_cast<unsigned*>(flags) + (li >> 2), (4u << t) << (8 * (li & 3)));
     }
+    __syncthreads();
   }
-  __syncthreads();
   if (DBG && warp < n && (a.dbg_cand || a.dbg_kept || a.dbg_a_kept)) {
     // this CTA's part of the ascending candidate list (offset: the candidates
     // of the lower CTAs); the kept list follows after the last exchange
@@ -1416,6 +1297,49 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
     if (lane == 0) dcnt[(NT + t) * 16 + rank] = kc;  // own kept channels of token t
   }
   if (DBG) stamp(a, cid, rank, 11);
+
+  // ------------------------------------------ recovery input z (own part)
+  // z_t = sum over the own channels not kept by token t of their recovery
+  // input times Ubar_i: the sketch estimate ahat_i, or with the exact input
+  // the exact a_i of a dropped candidate.  Warp w takes channels w, w + 16,
+  // ..., lane p the entries p, p + 32, ...; the warps' sums meet in shared
+  // memory.
+  if (r > 0) {
+    if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
+    const bool rec_exact = a.recovery_input == 1;
+    float zacc[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) zacc[t][kk] = 0.0f;
+#pragma unroll 1
+    for (int li = warp; li < nown; li += NWARP) {
+      const unsigned f = flags[li];
+      float co[NT];
+#pragma unroll
+      for (int t = 0; t < NT; t++) {
+        const bool kept = (f >> (2 + t)) & 1u, cand = (f >> t) & 1u;
+        co[t] = t >= n || kept ? 0.0f : cand && rec_exact ? aown[t * om + li] : ahat[t * om + li];
+      }
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) {
+        const int p = lane + 32 * kk;
+        if (p < r) {
+          const float u = bf16f(ub[li * r + p]);
+#pragma unroll
+          for (int t = 0; t < NT; t++) zacc[t][kk] = fmaf(co[t], u, zacc[t][kk]);
+        }
+      }
+    }
+    float* zr = reinterpret_cast<float*>(smem + L.zred);  // [NWARP, NT, r]
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) {
+        const int p = lane + 32 * kk;
+        if (p < r) zr[(warp * NT + t) * r + p] = zacc[t][kk];
+      }
+  }
 
   // ---------------------------------------------- D: down rows + recovery
   // kept rows, compacted with each token's coefficient; warp 0 waits for
@@ -1455,7 +1379,6 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
     if (!dspec) {
       __syncthreads();  // every thread is done with the previous round's slots
       if (lane == 0) {
-        fence_proxy_async();
         for (int m = warp; m < cnt; m += NWARP)
           issue_down(a, e, i0 + kslot[base + m], ring + (size_t)m * 2 * d, &dbars[m]);
       }
@@ -1492,24 +1415,19 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
       if (!(f & 12u) && !mbar_wait_bounded(&dbars[m], 0, err)) misc[MI_DONE] = 1;
     }
   }
-  // the own partial of z: z_all less the kept channels' ahat (and, with the
-  // exact recovery input, less ahat - a of the dropped candidates)
+  // the own part of z: the warps' sums (their writes ordered by the block
+  // barriers of the down stage)
   if (r > 0) {
-    if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
-    const bool rec_exact = a.recovery_input == 1;
+    const float* zr = reinterpret_cast<const float*>(smem + L.zred);
     for (int tp = tid; tp < n * r; tp += NTHR) {
-      const int t = tp / r, p = tp - t * r;
-      float zz = zparts[(rank * NT + t) * r + p];
-#pragma unroll 1
-      for (int m = 0; m < ndc; m++) {
-        const int li = drows[m];
-        const unsigned f = flags[li];
-        if (!((f >> t) & 1u)) continue;
-        const float u = bf16f(ub[li * r + p]), ah = ahat[t * om + li];
-        if ((f >> (2 + t)) & 1u) zz = fmaf(-ah, u, zz);
-        else if (rec_exact) zz = fmaf(-__fsub_rn(ah, aown[t * om + li]), u, zz);
+      const int t = tp >= r ? 1 : 0, p = tp - t * r;
+      float z0 = 0.0f, z1 = 0.0f;
+#pragma unroll 4
+      for (int w = 0; w < NWARP; w += 2) {
+        z0 += zr[(w * NT + t) * r + p];
+        z1 += zr[((w + 1) * NT + t) * r + p];
       }
-      zparts[(rank * NT + t) * r + p] = zz;
+      zparts[(rank * NT + t) * r + p] = z0 + z1;
     }
   }
   __syncthreads();
@@ -1836,7 +1754,7 @@ cudaError_t plan_dense(const ExpertArgs& a, DensePlan* out) {
 
 // ----- sparse reader (one or two tokens)
 struct ReaderPlan {
-  int dev, B, E, I, d, r, forced;
+  int dev, B, E, I, d, r, top_e, forced;
   int cs, smem, max_clusters, items;
   RLayout L;
 };
@@ -1857,7 +1775,7 @@ cudaError_t plan_reader(const ExpertArgs& a, ReaderPlan* out) {
   for (int i = 0; i < ncache; i++) {
     const ReaderPlan& c = cache[i];
     if (c.dev == dev && c.B == a.B && c.E == a.E && c.I == a.I && c.d == a.d && c.r == a.r &&
-        c.forced == a.force_cs) {
+        c.top_e == a.top_e && c.forced == a.force_cs) {
       *out = c;
       return cudaSuccess;
     }
@@ -1873,7 +1791,7 @@ cudaError_t plan_reader(const ExpertArgs& a, ReaderPlan* out) {
     if (err != cudaSuccess) return err;
   }
   const int items = a.B * a.top_e < a.E ? a.B * a.top_e : a.E;
-  ReaderPlan p = {dev, a.B, a.E, a.I, a.d, a.r, a.force_cs, 0, 0, 0, items, {}};
+  ReaderPlan p = {dev, a.B, a.E, a.I, a.d, a.r, a.top_e, a.force_cs, 0, 0, 0, items, {}};
   double best = 1e30;
   for (int cs = 16; cs >= 2; cs--) {
     if (a.force_cs && cs != a.force_cs) continue;

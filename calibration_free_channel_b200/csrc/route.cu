@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a, int n_logit_blo
   }
 }
 
+
 // One CTA: top-e per token (ties to the lower id) and softmax weights, one
 // warp per token; then, one warp per expert, the token-ordered tables of the
 // step from ballots over the tokens: the work items of up to kMaxGroup tokens
