@@ -3,8 +3,9 @@ C ABI and the CPU oracle on the same seeded inputs, then compare.
 
 The parity bar: routing ids, integer sketch dots, screening scores and
 candidate sets bit-exact; kept sets equal except for swaps inside an oracle
-boundary gap below 1e-3 relative; outputs within max-abs 2e-2 and rel-L2
-1e-2 (fp32 accumulation, bf16 in and out)."""
+boundary gap below 1e-3 relative; fp32 per-expert outputs within max-abs
+2e-2; bf16 outputs within 2e-2 beyond half a bf16 ulp of the exact value and
+rel-L2 1e-2 (fp32 accumulation, bf16 in and out)."""
 from __future__ import annotations
 
 import numpy as np
@@ -101,9 +102,10 @@ def compare_step(W, x, gpu_y, gdbg, ora_y64, odbg, k, ora_logits=None, check_kep
     diff = np.abs(yg - yo)
     err = float(diff.max())
     rel = float(np.linalg.norm(yg - yo) / max(np.linalg.norm(yo), 1e-30))
-    # bf16 output: 2e-2 beyond one bf16 ulp of the exact value
+    # bf16 output: within 2e-2 beyond half a bf16 ulp of the exact value (half
+    # an ulp is the error of rounding the exact value once to bf16)
     ulp = bf16_ulp(yo)
-    excess = float((diff - ulp).max())
+    excess = float((diff - 0.5 * ulp).max())
     assert excess <= MAX_ABS and rel <= REL_L2, dict(max_abs=err, excess=excess, rel=rel, ye_err=ye_err,
                                                      swaps=swaps, ymax=float(np.abs(yo).max()))
     return dict(max_abs=err, excess_over_ulp=excess, rel_l2=rel, y_expert_max_abs=ye_err, swaps=swaps)

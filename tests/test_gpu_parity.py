@@ -79,29 +79,34 @@ def test_forward_tiny_budgets(tiny, k, c, r):
 
 
 def test_forward_qwen_layer_batch1_steps(qwen):
-    """The Qwen3-30B-A3B-shaped layer at batch 1 over decode steps with
-    tokens from seeds 0..7 (k = 136, c = 272, r = 32)."""
+    """The Qwen3-30B-A3B-shaped layer at batch 1 over all 20 decode steps
+    (tokens from seeds 0..19; k = 136, c = 272, r = 32)."""
     W, layer, oc = qwen
-    for s in range(8):
+    for s in range(20):
         x = synth.tokens(2048, 1, seed=s)
         check_pair(layer, oc, x, k=136, c=272, top_e=8)
 
 
-@pytest.mark.parametrize("B,k", [(4, 100), (16, 136), (8, 100)])
+@pytest.mark.parametrize("B", [1, 4, 8, 16])
+@pytest.mark.parametrize("k", [100, 136])
 def test_forward_qwen_budget_sweep(qwen, B, k):
+    """The budget sweep: k = 100 (13%) and k = 136 (18%), c = 2k, r = 32, at
+    batch 1, 4, 8 and 16 (tokens drawn independently)."""
     W, layer, oc = qwen
-    x = synth.tokens(2048, B, seed=100 + B)
+    x = synth.tokens(2048, B, seed=100 + B + k)
     check_pair(layer, oc, x, k=k, c=2 * k, top_e=8)
 
 
-@pytest.mark.parametrize("B", [32, 64])
+@pytest.mark.parametrize("B", [1, 8, 16, 32, 64])
 def test_forward_qwen_skewed_batch(qwen_skewed, B):
-    """Skewed router prior: many tokens share experts, so one expert's
-    tokens span several work items of up to 8 tokens."""
+    """Skewed router prior (logit bias ~ N(0, 1) per expert), the batch sweep
+    at 1, 8, 16, 32 and 64 tokens: at the larger batches many tokens share
+    experts, so one expert's tokens span several work items."""
     W, layer, oc = qwen_skewed
     x = synth.tokens(2048, B, seed=200 + B)
     _, ids, _ = O.route(x, W["w_router"], W["router_bias"], 8)
-    assert np.bincount(ids.ravel()).max() > 8
+    if B >= 32:
+        assert np.bincount(ids.ravel()).max() > 8
     check_pair(layer, oc, x, k=136, c=272, top_e=8)
 
 
@@ -138,7 +143,7 @@ def test_forward_host_matches_forward(qwen):
 # ------------------------------------------------------------------ dense
 def _check_out(y, y64):
     yg = y.float().cpu().numpy().astype(np.float64)
-    assert (np.abs(yg - y64) - bf16_ulp(y64)).max() <= MAX_ABS
+    assert (np.abs(yg - y64) - 0.5 * bf16_ulp(y64)).max() <= MAX_ABS
     assert np.linalg.norm(yg - y64) / np.linalg.norm(y64) <= REL_L2
 
 

@@ -1,9 +1,10 @@
 """moe_reader_forward_noalloc: the step with the library's fixed device
 scratch instead of a caller-allocated workspace, for callers that cannot
-allocate device memory (code running under stream capture, serving loops that
-forbid allocation after start-up, hosts whose allocator belongs to another
-runtime).  Its outputs must match moe_reader_forward's on the same inputs, on
-two calls in a row (the scratch persists between calls).
+allocate device memory (serving loops that forbid any allocation after
+start-up so their footprint stays fixed, hosts whose device memory belongs to
+another runtime's allocator).  Its outputs must match moe_reader_forward's on
+the same inputs, on two calls in a row (the scratch persists between calls),
+and the scratch's device error word must read clear afterwards.
 
 This file is collected last on purpose, so a stop-at-first-failure run has
 already run every other test; it also passes on its own in a fresh process.
@@ -20,6 +21,8 @@ pytestmark = pytest.mark.gpu
 
 
 def _close(y, ref):
+    # both outputs are bf16 roundings of fp32 sums in different orders: they
+    # may sit one bf16 ulp apart at a rounding boundary
     yg = y.float().cpu().numpy().astype(np.float64)
     yr = ref.float().cpu().numpy().astype(np.float64)
     assert (np.abs(yg - yr) - bf16_ulp(yr)).max() <= MAX_ABS
@@ -38,6 +41,7 @@ def test_noalloc_matches_forward_twice(B):
         M.moe_reader_forward_noalloc(st, B, 24, 48, x, None, y)
         torch.cuda.synchronize()
         _close(y, ref)
+    M.moe_reader_check_error(None)  # the scratch's error word: no bounded wait ran out
 
 
 def test_noalloc_qwen_layer_batch1_twice():
@@ -51,6 +55,7 @@ def test_noalloc_qwen_layer_batch1_twice():
         M.moe_reader_forward_noalloc(st, 1, 136, 272, x, None, y)
         torch.cuda.synchronize()
         _close(y, ref)
+    M.moe_reader_check_error(None)
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
