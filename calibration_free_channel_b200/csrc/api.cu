@@ -98,6 +98,8 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
     REQUIRE(c >= k && c <= L->I, "c = %d outside [k = %d, I = %d]", c, k, L->I);
   }
   REQUIRE_PTR(x);
+  if (dbg) REQUIRE(dbg->withhold_copy == 0 || dbg->withhold_copy == 1, "withhold_copy = %d: use 0 or 1",
+                   dbg->withhold_copy);
   if (ep_size > 0) {
     REQUIRE(ep_size <= L->E && ep_rank >= 0 && ep_rank < ep_size, "ep_rank = %d, ep_size = %d: need 0 <= rank < size <= E",
             ep_rank, ep_size);
@@ -157,6 +159,8 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   a.ep_partial = ep_size > 0 ? 1 : 0;
   a.cs = 0;  // chosen at launch
   a.force_cs = L->cluster_size;
+  a.wait_ns = dbg && dbg->wait_limit_us ? 1000ull * dbg->wait_limit_us : moe::kWaitLimitNs;
+  a.withhold_copy = dbg ? dbg->withhold_copy : 0;
   a.nmax = B < moe::kMaxGroup ? B : moe::kMaxGroup;
   a.x = x;
   a.w_router = L->w_router;

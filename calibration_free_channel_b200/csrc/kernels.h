@@ -82,6 +82,8 @@ struct ExpertArgs {
   int nmax;          // max tokens per work item this launch
   int ring_rows;     // copy-ring row slots per warp (sparse) / rows (dense)
   int recovery_input;  // 0: ahat of every skipped channel; 1: exact a of dropped candidates
+  unsigned long long wait_ns;  // limit of every bounded copy wait (test hook; kWaitLimitNs normally)
+  int withhold_copy;           // test hook: 1 = the one-cluster reader never issues one sketch copy
   int ep_partial;      // 1: write the per-slot outputs only (no combine); expert-parallel steps
   const uint16_t* x;
   const uint16_t* w_router;  // routing inside the expert kernel (small B)

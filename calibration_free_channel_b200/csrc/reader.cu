@@ -748,6 +748,9 @@ __device__ __forceinline__ void issue_sketch(const ExpertArgs& a, const RLayout&
   char* dst = ring + (size_t)slot * 2 * L.skc;
   mbar_expect_tx(&bars[slot], 2 * bytes);
   bulk_g2s(dst, a.sk_gate + ((size_t)e * a.I + c0) * (a.d / 16), bytes, &bars[slot]);
+  // test hook: chunk 0's up rows are expected but never copied, so every
+  // wait for that chunk runs out (nothing is left in flight)
+  if (a.withhold_copy && ch == 0) return;
   bulk_g2s(dst + L.skc, a.sk_up + ((size_t)e * a.I + c0) * (a.d / 16), bytes, &bars[slot]);
 }
 
@@ -986,7 +989,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
       for (int t = 0; t < NT; t++) G[t] = U[t] = 0;
       if (li < nown) {
         const int slot = j - rb;
-        if (!mbar_wait_bounded(&skbars[slot], par, err)) misc[MI_DONE] = 1;
+        if (!mbar_wait_bounded(&skbars[slot], par, err, a.wait_ns)) misc[MI_DONE] = 1;
         const uint4* gw = reinterpret_cast<const uint4*>(ring + (size_t)slot * 2 * L.skc + warp * (d / 4));
         const uint4* uw = reinterpret_cast<const uint4*>(ring + (size_t)slot * 2 * L.skc + L.skc + warp * (d / 4));
         int ga[NT][4], ua[NT][4];
@@ -1174,7 +1177,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
 #pragma unroll 1
     for (int m = 0; m < nmine; m++) {
       const int s = m % Pw;
-      if (!mbar_wait_bounded(&wbars[s], (par >> s) & 1u, err)) misc[MI_DONE] = 1;
+      if (!mbar_wait_bounded(&wbars[s], (par >> s) & 1u, err, a.wait_ns)) misc[MI_DONE] = 1;
       par ^= 1u << s;
       const int j = warp + W * m, li = rows[j];
       const unsigned f = flags[li];
@@ -1305,7 +1308,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
   // ..., lane p the entries p, p + 32, ...; the warps' sums meet in shared
   // memory.
   if (r > 0) {
-    if (!mbar_wait_bounded(uvbar, 0, err)) misc[MI_DONE] = 1;
+    if (!mbar_wait_bounded(uvbar, 0, err, a.wait_ns)) misc[MI_DONE] = 1;
     const bool rec_exact = a.recovery_input == 1;
     float zacc[NT][4];
 #pragma unroll
@@ -1387,7 +1390,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
       const uint32_t par = dspec ? 0u : (uint32_t)(base / rnd) & 1u;
       for (int m = lane; m < cnt; m += 32) {
         const int s = dspec ? kslot[base + m] : m;
-        if (!mbar_wait_bounded(&dbars[s], par, err)) misc[MI_DONE] = 1;
+        if (!mbar_wait_bounded(&dbars[s], par, err, a.wait_ns)) misc[MI_DONE] = 1;
       }
     }
     __syncthreads();
@@ -1412,7 +1415,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
     // copies of rows the top-k left out must land before the CTA ends
     for (int m = lane; m < ndc; m += 32) {
       const unsigned f = flags[drows[m]];
-      if (!(f & 12u) && !mbar_wait_bounded(&dbars[m], 0, err)) misc[MI_DONE] = 1;
+      if (!(f & 12u) && !mbar_wait_bounded(&dbars[m], 0, err, a.wait_ns)) misc[MI_DONE] = 1;
     }
   }
   // the own part of z: the warps' sums (their writes ordered by the block

@@ -167,7 +167,9 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
     const uint4* grow = reinterpret_cast<const uint4*>(stage) + (size_t)lc * nv + part * nch;
     const uint4* urow = reinterpret_cast<const uint4*>(stage + kSkBytes) + (size_t)lc * nv + part * nch;
     const uint16_t* ubs = reinterpret_cast<const uint16_t*>(stage + 2 * kSkBytes);
-    mbar_wait_bounded(&bars[st], (it >> 1) & 1, err);
+    // a stage whose copy did not land in time is not read (the error word
+    // records it; the unit's scores stay zero)
+    const bool landed = mbar_wait_bounded(&bars[st], (it >> 1) & 1, err, a.wait_ns);
 #pragma unroll 1
     for (int tg = 0; tg < m; tg += kSTG) {
       const int ng = min(kSTG, m - tg);
@@ -194,7 +196,7 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
       for (int t = 0; t < kSTG; t++)
 #pragma unroll
         for (int w = 0; w < 4; w++) ga[t][w] = ua[t][w] = 0;
-      if (ok) {
+      if (ok && landed) {
 #pragma unroll 2
         for (int j = 0; j < nch; j++) {
           const int jr = (j + rot) & (nch - 1);
@@ -258,12 +260,12 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
           const int t = o / r, p = o - t * r;
           const uint16_t* ub = ubs + p;
           float z0 = 0.0f, z1 = 0.0f;
-          int l = 0;
+          int l = landed ? 0 : ncw;
           for (; l + 2 <= ncw; l += 2) {
             z0 = fmaf(sah[t][l], bf16f(ub[(size_t)l * r]), z0);
             z1 = fmaf(sah[t][l + 1], bf16f(ub[(size_t)(l + 1) * r]), z1);
           }
-          if (l < ncw) z0 = fmaf(sah[t][l], bf16f(ub[(size_t)l * r]), z0);
+          if (landed && l < ncw) z0 = fmaf(sah[t][l], bf16f(ub[(size_t)l * r]), z0);
           a.ws.zpart[((size_t)(p0 + tg + t) * zstride + blk) * r + p] = z0 + z1;
         }
       }

@@ -34,7 +34,8 @@ class MoeReaderLayer(C.Structure):
 
 class MoeReaderDebug(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("ids", "weights", "dot_gate", "dot_up", "score", "cand", "kept",
-                                          "a_kept", "y_expert", "phase_ns", "ev_before", "ev_after")]
+                                          "a_kept", "y_expert", "phase_ns", "ev_before", "ev_after")] + \
+               [("wait_limit_us", C.c_uint32), ("withhold_copy", C.c_int32)]
 
 
 class MoeError(RuntimeError):
@@ -262,7 +263,10 @@ class Layer:
                      a_kept=torch.empty(P + (k,), dtype=torch.float32, device=dev),
                      y_expert=torch.empty(P + (self.d,), dtype=torch.float32, device=dev),
                      phase_ns=torch.zeros((B * self.top_e, 16), dtype=torch.int64, device=dev))
-        return dbg_t, MoeReaderDebug(*[_ptr(dbg_t[n]) if n in dbg_t else None for n, _ in MoeReaderDebug._fields_])
+        dbg = MoeReaderDebug()
+        for n, v in dbg_t.items():
+            setattr(dbg, n, _ptr(v))
+        return dbg_t, dbg
 
     def forward_ep(self, x, k: int, c: int, ep_rank: int, ep_size: int, debug: bool = False, r: int | None = None,
                    stream=None, out=None, recovery_input: int = 0):

@@ -128,6 +128,14 @@ typedef struct {
    * the per-stage outputs above. */
   void* ev_before;
   void* ev_after;
+  /* Failure-detection hooks for tests (0 = off).  wait_limit_us: limit of
+   * every bounded device wait of this call, in microseconds (default 2 s).
+   * withhold_copy = 1: the one-cluster reader sets up, but never issues, one
+   * of the sketch copies of each work item, so its bounded wait runs out;
+   * the kernel still completes (with unusable outputs) and the error word
+   * reads MOE_ETIMEOUT.  Any other value is MOE_EINVAL. */
+  uint32_t wait_limit_us;
+  int32_t withhold_copy;
 } moe_reader_debug;
 
 /* Bytes of device workspace moe_reader_forward / moe_reader_forward_dense

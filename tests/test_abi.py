@@ -94,6 +94,14 @@ def test_forward_rejects_bad_options(lib, kw):
     assert lib.moe_reader_last_error()
 
 
+def test_forward_rejects_bad_test_hook(lib):
+    dbg = M.MoeReaderDebug()
+    dbg.withhold_copy = 2
+    st = lib.moe_reader_forward(C.byref(_layer()), 1, 24, 48, 0x10000, None, 0x10000, C.byref(dbg), 0x10000,
+                                1 << 30, None)
+    assert st == M.MOE_EINVAL and b"withhold_copy" in lib.moe_reader_last_error()
+
+
 def test_one_cluster_reader_limits(lib):
     # the one-cluster reader runs one or two tokens with d <= 2048; asking for
     # it above that is refused before anything is enqueued
@@ -105,8 +113,9 @@ def test_one_cluster_reader_limits(lib):
 def test_layer_struct_layout():
     # the binding's structs match the header's field order and sizes
     assert [n for n, _ in M.MoeReaderLayer._fields_][-3:] == ["recovery_input", "path", "cluster_size"]
-    assert [n for n, _ in M.MoeReaderDebug._fields_][-2:] == ["ev_before", "ev_after"]
-    assert C.sizeof(M.MoeReaderDebug) == 12 * C.sizeof(C.c_void_p)
+    assert [n for n, _ in M.MoeReaderDebug._fields_][-4:] == ["ev_before", "ev_after", "wait_limit_us",
+                                                            "withhold_copy"]
+    assert C.sizeof(M.MoeReaderDebug) == 12 * C.sizeof(C.c_void_p) + 8
 
 
 def test_forward_without_recovery_needs_no_factors(lib):
