@@ -61,6 +61,8 @@ def parse():
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-sweep", action="store_true", help="skip the batch and skewed-routing sweeps")
     p.add_argument("--layers", type=int, default=32, help="distinct device copies of the layer the steps cycle through")
+    p.add_argument("--sketch", default="2bit", choices=["2bit", "base3"],
+                   help="sketch rows of the headline steps: 2-bit codes or base 3 (five trits per byte)")
     p.add_argument("--path", type=int, default=0, choices=[0, 1, 2],
                    help="sparse reader: 0 automatic, 1 one cluster per expert, 2 streamed kernels")
     return p.parse_args()
@@ -77,7 +79,7 @@ def measured_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("reader.cu", "common.cuh", "kernels.h"):
+    for name in ("reader.cu", "common.cuh", "kernels.h", "rotate.cuh", "select.cuh"):
         with open(os.path.join(ROOT, "calibration_free_channel_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -177,14 +179,31 @@ def run_native(args, rank, world, local_rank):
         reader reads, from its own debug outputs; untimed)."""
         sb, db = [], []
         bias = lays[0].w.get("router_bias") is not None
+        packing = "base3" if lays[0].sketch_format == 1 else "2bit"
         for x in xq:
             _, dbg = lays[0].forward(x, k=kq, c=cq, debug=True)
             ids, cand, kept = (dbg[n].cpu().numpy() for n in ("ids", "cand", "kept"))
-            acc = accounting.step_bytes(shape.E, shape.I, shape.d, r, ids, cand, kept, bias=bias)
+            acc = accounting.step_bytes(shape.E, shape.I, shape.d, r, ids, cand, kept, bias=bias, packing=packing)
             sb.append(acc["total"])
             db.append(acc["dense"])
         lays[0].check()
         return sb, db
+
+    def to_base3(lay):
+        """A descriptor of the same layer whose sketch rows are base 3 (five
+        trits per byte), repacked from its 2-bit codes in new device memory."""
+        l3 = replicate_view(lay)
+        rb = M.moe_reader_sketch_row_bytes(shape.d, 1)
+        l3.sk_gate = torch.empty((shape.E, shape.I, rb), dtype=torch.uint8, device=dev)
+        l3.sk_up = torch.empty_like(l3.sk_gate)
+        M.moe_reader_sketch_to_base3(shape.E, shape.I, shape.d, lay.sk_gate, l3.sk_gate)
+        M.moe_reader_sketch_to_base3(shape.E, shape.I, shape.d, lay.sk_up, l3.sk_up)
+        l3.sketch_format = 1
+        return l3
+
+    if args.sketch == "base3":
+        layers = [to_base3(lay) for lay in layers]
+        layer = layers[0]
 
     step_bytes, dense_bytes = step_accounting(layers, xs, k, c)
 
@@ -371,6 +390,33 @@ def run_native(args, rank, world, local_rank):
                                                   "dense block on the same weights"}
         skewed_sweep.update(sweep(skewed, (1, 8, 16, 32, 64), k, 9000 + 1000 * rank))
 
+    # the same steps with base-3 sketch rows (five trits per byte) against the
+    # 2-bit codes, on the same token sets and layer copies
+    base3 = None
+    if not args.no_sweep and args.sketch == "2bit":
+        l3s = [to_base3(lay) for lay in layers]
+        base3 = {"note": "sketch rows 1.6 bits per trit (base 3) against 2-bit codes; same weights, tokens and "
+                         "layer copies, 64 back-to-back steps each"}
+        for Bq in (1, 16):
+            xq = [synth.tokens(shape.d, Bq, seed=11000 + 100 * Bq + s).to(dev) for s in range(8)]
+            yq = out_buf(Bq)
+            ent = {}
+            for name, lays in (("2bit", layers), ("base3", l3s)):
+                sb, _ = step_accounting(lays, xq, k, c)
+
+                def sp(j, lays=lays, xq=xq, yq=yq):
+                    lays[j % len(lays)].forward(xq[j % len(xq)], k=k, c=c, out=yq)
+
+                tms, _ = chunk_loop(sp, 64, 4)
+                (tms,) = max_over_ranks(tms)
+                ent[name] = {"us_per_step": tms * 1e3, "bytes_per_step": statistics.mean(sb)}
+            ent["sketch_bytes_per_expert"] = {
+                "2bit": 2 * shape.I * accounting.sketch_row_bytes(shape.d, "2bit") + 8 * shape.I,
+                "base3": 2 * shape.I * accounting.sketch_row_bytes(shape.d, "base3") + 8 * shape.I}
+            base3[f"B{Bq}"] = ent
+            l3s[0].check()
+        del l3s
+
     fused = B <= 2 and args.path != 2
     # At B <= 2 the reader routes in-kernel: it is the step's only kernel and
     # reads the router too, so a launch's bytes are the step's and its average
@@ -391,13 +437,14 @@ def run_native(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16 (int8 x 2-bit sketch dots, fp32 accumulate)",
+        "dtype": "bf16 (int8 x %s sketch dots, fp32 accumulate)" % ("base-3" if args.sketch == "base3" else "2-bit"),
         "data": "synthetic (seeded; Qwen3-30B-A3B layer shape, lognormal channel scales, Student-t tokens)",
         "config": {"workload": workload_name(B), "d": shape.d, "I": shape.I, "E": shape.E, "top_e": shape.top_e,
                    "batch": B, "k": k, "c": c, "r": r, "decode_steps_cycled": ntok,
                    "l2": f"inputs larger than L2: steps cycle through {nlay} distinct device copies of the layer "
                          f"({nlay * layer_bytes(layer) / 1e9:.1f} GB)",
-                   "parallelism": f"replicas x{world}", "algorithmic_bytes_per_step": mean_bytes},
+                   "parallelism": f"replicas x{world}", "algorithmic_bytes_per_step": mean_bytes,
+                   "sketch": args.sketch},
         "roofline": {"bound": "hbm", "kernel": "reader_kernel" if fused else "streamed kernels (screen .. down)",
                      "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
@@ -416,6 +463,7 @@ def run_native(args, rank, world, local_rank):
                      "note": "one layer, L2 flushed before every step (also evicts the kernel code)"},
         "batch_sweep": batch_sweep,
         "skewed_sweep": skewed_sweep,
+        "base3_sketch": base3,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(W, toks[:4], k, c, r, shape, budget_s=12.0)

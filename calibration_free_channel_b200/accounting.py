@@ -10,7 +10,8 @@ low-rank map), plus the router.
 Every row the reader touches starts on a 32-byte boundary and is a multiple
 of 32 bytes long (gate/up/down rows are 2d bytes, sketch rows d/4 bytes,
 alpha blocks 4I bytes, low-rank rows 2r bytes with r % 16 == 0 or whole
-blocks), so the sector count times 32 equals the byte count.
+blocks; base-3 sketch rows are padded to whole sectors), so the sector count
+times 32 equals the byte count.
 """
 from __future__ import annotations
 
@@ -19,9 +20,9 @@ import numpy as np
 SECTOR = 32
 
 
-def expert_bytes(I: int, d: int, r: int, n_cand_rows: int, n_kept_rows: int) -> dict:
+def expert_bytes(I: int, d: int, r: int, n_cand_rows: int, n_kept_rows: int, packing: str = "2bit") -> dict:
     """Algorithmic bytes of one active expert in one step."""
-    sketch = 2 * I * (d // 4) + 2 * I * 4
+    sketch = 2 * I * sketch_row_bytes(d, packing) + 2 * I * 4
     cand = 2 * n_cand_rows * d * 2
     down = n_kept_rows * d * 2
     lowrank = (I + d) * r * 2 if r > 0 else 0
@@ -54,7 +55,7 @@ def router_bytes(E: int, d: int, bias: bool) -> int:
 
 
 def step_bytes(E: int, I: int, d: int, r: int, ids: np.ndarray, cand: np.ndarray, kept: np.ndarray,
-               bias: bool = False) -> dict:
+               bias: bool = False, packing: str = "2bit") -> dict:
     """Bytes of one sparse step over B tokens.
 
     ids [B, top_e] routed experts; cand [B, top_e, c] and kept [B, top_e, k]
@@ -66,7 +67,7 @@ def step_bytes(E: int, I: int, d: int, r: int, ids: np.ndarray, cand: np.ndarray
         bs, ss = np.nonzero(ids == e)
         cu = np.unique(np.concatenate([np.asarray(cand)[b, s] for b, s in zip(bs, ss)]))
         ku = np.unique(np.concatenate([np.asarray(kept)[b, s] for b, s in zip(bs, ss)]))
-        per[int(e)] = expert_bytes(I, d, r, cu.size, ku.size)
+        per[int(e)] = expert_bytes(I, d, r, cu.size, ku.size, packing)
     total = router_bytes(E, d, bias) + sum(v["total"] for v in per.values())
     return dict(per_expert=per, router=router_bytes(E, d, bias), total=total,
                 dense=router_bytes(E, d, bias) + len(per) * dense_expert_bytes(I, d))

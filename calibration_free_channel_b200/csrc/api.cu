@@ -63,10 +63,13 @@ moe_status check_layer(const moe_reader_layer* L, bool sparse) {
   REQUIRE_PTR(L->w_gate);
   REQUIRE_PTR(L->w_up);
   REQUIRE_PTR(L->w_down);
+  OPT_PTR(L->expert_slot);
   if (sparse) {
     REQUIRE_PTR(L->rot_sign);
     REQUIRE_PTR(L->sk_gate);
     REQUIRE_PTR(L->sk_up);
+    REQUIRE(L->sketch_format == 0 || L->sketch_format == 1,
+            "sketch_format = %d: use 0 (2-bit codes) or 1 (base 3, five trits per byte)", L->sketch_format);
     REQUIRE_PTR(L->alpha_gate);
     REQUIRE_PTR(L->alpha_up);
     REQUIRE(L->recovery_input == 0 || L->recovery_input == 1, "recovery_input = %d: use 0 or 1", L->recovery_input);
@@ -112,7 +115,10 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   const int sI = dense ? 0 : L->I, sr = dense ? 0 : L->r;
   const size_t need = moe::workspace_layout(B, L->E, L->top_e, L->d, sI, sr, nullptr, nullptr);
   REQUIRE(ws_bytes >= need, "workspace has %zu bytes, needs %zu", ws_bytes, need);
-  const bool streamed = !dense && (ep_size > 0 || L->path == 2 || (L->path == 0 && !moe::reader_supports(B, L->d)));
+  if (L->expert_slot && (dense || L->path == 1))
+    return fail(MOE_EUNSUPPORTED, "expert_slot (held experts only) is read by the streamed reader (path 0 or 2)");
+  const bool streamed = !dense && (ep_size > 0 || L->path == 2 || L->expert_slot ||
+                                   (L->path == 0 && !moe::reader_supports(B, L->d)));
   if (!dense && !streamed && !moe::reader_supports(B, L->d))
     return fail(MOE_EUNSUPPORTED, "path 1 (one cluster per expert) runs B <= 2 and d <= 2048 (B = %d, d = %d)", B,
                 L->d);
@@ -140,6 +146,7 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   cudaError_t e = cudaSuccess;
   ra.ep_rank = ep_rank;
   ra.ep_size = ep_size;
+  ra.expert_slot = L->expert_slot;
   // steps of at most two tokens route inside the cluster kernels
   if (!moe::fused_routing(B) || streamed) {
     e = moe::launch_route(ra, s);
@@ -169,8 +176,9 @@ moe_status run_forward(const moe_reader_layer* L, int B, int k, int c, const uin
   a.w_gate = L->w_gate;
   a.w_up = L->w_up;
   a.w_down = L->w_down;
-  a.sk_gate = L->sk_gate;
-  a.sk_up = L->sk_up;
+  a.sk_gate = static_cast<const uint32_t*>(L->sk_gate);
+  a.sk_up = static_cast<const uint32_t*>(L->sk_up);
+  a.sk3 = dense ? 0 : L->sketch_format;
   a.alpha_gate = L->alpha_gate;
   a.alpha_up = L->alpha_up;
   a.u_sigma = L->u_sigma;
@@ -239,6 +247,23 @@ moe_status moe_reader_build_sketch(int E, int I, int d, const uint16_t* w_gate, 
   cudaError_t e = moe::launch_build_sketch(E, I, d, w_gate, w_up, rot_seed, rot_sign, sk_gate, sk_up, alpha_gate,
                                            alpha_up, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "build_sketch launch");
+}
+
+size_t moe_reader_sketch_row_bytes(int d, int format) {
+  if (d < 16 || d % 16 != 0) return 0;
+  if (format == 0) return (size_t)d / 4;
+  if (format == 1) return (size_t)moe::sk3_row_bytes(d);
+  return 0;
+}
+
+moe_status moe_reader_sketch_to_base3(int E, int I, int d, const uint32_t* sk_codes, uint8_t* sk_base3,
+                                      void* stream) {
+  moe_status st = check_shape(1, E, 1, I, d);
+  if (st != MOE_OK) return st;
+  REQUIRE_PTR(sk_codes);
+  REQUIRE_PTR(sk_base3);
+  cudaError_t e = moe::launch_sketch_to_base3((long)E * I, d, sk_codes, sk_base3, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "sketch_to_base3 launch");
 }
 
 size_t moe_reader_lowrank_workspace_bytes(int E, int I, int d, int r) {
@@ -345,7 +370,10 @@ moe_status moe_reader_check_error(void* workspace, void* stream) {
   if (word == 0) return MOE_OK;
   const uint32_t zero = 0;
   cudaMemcpy(ws.err, &zero, sizeof zero, cudaMemcpyHostToDevice);
-  return fail(MOE_ETIMEOUT, "device error word 0x%x (1: a bounded copy wait ran out; 2: bad work item)", word);
+  return fail((word & moe::kErrCopyTimeout) ? MOE_ETIMEOUT : MOE_EDEVICE,
+              "device error word 0x%x (1: a bounded copy wait ran out; 2: bad work item; 4: a routed expert has no "
+              "weight slot)",
+              word);
 }
 
 moe_status moe_reader_launch_plan(int dense, int B, int E, int top_e, int I, int d, int r, int32_t* out4) {

@@ -98,6 +98,31 @@ __global__ void __launch_bounds__(256) sketch_kernel(int E, int I, int d, const 
   }
 }
 
+// Base-3 repacking: output byte g of a row = sum_i code(5g + i) 3^i with
+// code = t + 1 read from the 2-bit words (code 1, a zero trit, past d); the
+// bytes past ceil(d / 5) that pad the row to whole sectors hold five zero
+// trits (121).
+__global__ void sketch_base3_kernel(long rows, int d, const uint32_t* __restrict__ codes, uint8_t* __restrict__ out) {
+  const int rb = sk3_row_bytes(d), words = d / 16;
+  const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * rb) return;
+  const long row = idx / rb;
+  const int g = (int)(idx - row * rb);
+  const uint32_t* w = codes + row * words;
+  uint32_t v = 0, pw = 1;
+  for (int i = 0; i < 5; i++) {
+    const int j = 5 * g + i;
+    uint32_t code = 1u;
+    if (j < d) {
+      const int p = j & 15;
+      code = (w[j >> 4] >> (8 * (p & 3) + 2 * (p >> 2))) & 3u;
+    }
+    v += code * pw;
+    pw *= 3u;
+  }
+  out[idx] = (uint8_t)v;
+}
+
 __global__ void rmsnorm_kernel(int d, float eps, const uint16_t* __restrict__ x, uint16_t* __restrict__ h) {
   __shared__ float red[32];
   const uint16_t* xb = x + (size_t)blockIdx.x * d;
@@ -130,6 +155,13 @@ cudaError_t launch_build_sketch(int E, int I, int d, const uint16_t* w_gate, con
   const long grid = (rows + kRowsPerCta - 1) / kRowsPerCta;
   sketch_kernel<<<(unsigned)grid, 256, smem, s>>>(E, I, d, w_gate, w_up, rot_sign, sk_gate, sk_up, alpha_gate,
                                                    alpha_up);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sketch_to_base3(long rows, int d, const uint32_t* codes, uint8_t* out, cudaStream_t s) {
+  const long n = rows * sk3_row_bytes(d);
+  if (n == 0) return cudaSuccess;
+  sketch_base3_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(rows, d, codes, out);
   return cudaGetLastError();
 }
 

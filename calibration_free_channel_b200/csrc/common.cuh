@@ -18,6 +18,7 @@ constexpr int kMaxTokens = 256;        // tokens per step (B)
 // Error word bits (workspace), set by bounded waits that ran out.
 constexpr uint32_t kErrCopyTimeout = 1u;
 constexpr uint32_t kErrBadWorkItem = 2u;
+constexpr uint32_t kErrNoWeights = 4u;     // an active expert has no weight slot (expert_slot[e] < 0)
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 // ------------------------------------------------------------------ bf16
@@ -178,5 +179,66 @@ __device__ __forceinline__ void code_dot16(uint32_t w, uint4 q, int (&acc)[4]) {
 __device__ __forceinline__ int code_dot_total(const int (&acc)[4]) {
   return acc[0] + (acc[1] >> 2) + (acc[2] >> 4) + (acc[3] >> 6);
 }
+
+// ------------------------------------------------- base-3 sketch rows
+// Five trits per byte: byte g of a row holds trits 5g .. 5g+4 as
+// sum_i (t_{5g+i} + 1) 3^i (at most 242).  A row of d trits takes
+// ceil(d / 5) bytes; it is padded to whole 32-byte sectors with bytes of
+// five zero trits (121), so rows stay 16-byte aligned for bulk copies.
+//
+// Decoding is plain integer arithmetic on four bytes at once: the bytes sit
+// in two registers as 16-bit lanes (bytes 0 and 2, bytes 1 and 3), and
+// floor(b / 3^k) comes from one multiply and shift per lane pair
+// (b * 171 >> 9, b * 57 >> 9, b * 19 >> 9, b * 203 >> 14 are exact for
+// b <= 242 and stay inside 16 bits), so digit k = floor(b / 3^k) -
+// 3 floor(b / 3^(k+1)).  The digits come out digit-major: word k holds
+// digit k (the code t + 1 of trit 5g + k) of the four bytes, one per byte,
+// ready for dp4a against the activations staged the same way:
+// qd[5w + k] = (q[5(4w + b) + k], b = 0..3) for the bytes 4w .. 4w+3 of a
+// 16-byte chunk (w = 0..3; 80 bytes per chunk).
+__host__ __device__ inline int sk3_row_bytes(int d) { return ((d + 4) / 5 + 31) / 32 * 32; }
+__device__ __forceinline__ void b3_digits2(uint32_t R, uint32_t (&dg)[5]) {
+  const uint32_t f1 = ((R * 171u) >> 9) & 0x007f007fu;   // floor(b / 3)
+  const uint32_t f2 = ((R * 57u) >> 9) & 0x001f001fu;    // floor(b / 9)
+  const uint32_t f3 = ((R * 19u) >> 9) & 0x000f000fu;    // floor(b / 27)
+  const uint32_t f4 = ((R * 203u) >> 14) & 0x00030003u;  // floor(b / 81)
+  dg[0] = R - 3u * f1;
+  dg[1] = f1 - 3u * f2;
+  dg[2] = f2 - 3u * f3;
+  dg[3] = f3 - 3u * f4;
+  dg[4] = f4;
+}
+// The codes of one 16-byte chunk (80 trits), digit-major: o[5w + k].
+__device__ __forceinline__ void b3_decode16(uint4 s, uint32_t (&o)[20]) {
+  const uint32_t sw[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+  for (int w = 0; w < 4; w++) {
+    uint32_t dx[5], dy[5];
+    b3_digits2(sw[w] & 0x00ff00ffu, dx);
+    b3_digits2((sw[w] >> 8) & 0x00ff00ffu, dy);
+#pragma unroll
+    for (int k = 0; k < 5; k++) o[5 * w + k] = dx[k] | (dy[k] << 8);
+  }
+}
+__device__ __forceinline__ int b3_dot16(const uint32_t (&o)[20], const uint32_t* qd, int acc) {
+#pragma unroll
+  for (int i = 0; i < 20; i++) acc = dp4a_us(o[i], qd[i], acc);
+  return acc;
+}
+// The 20 staged activation words of one chunk (16-byte aligned).
+__device__ __forceinline__ void b3_load_q(const void* p, uint32_t (&qd)[20]) {
+  const uint4* q4 = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int v = 0; v < 5; v++) {
+    const uint4 w4 = q4[v];
+    qd[4 * v] = w4.x;
+    qd[4 * v + 1] = w4.y;
+    qd[4 * v + 2] = w4.z;
+    qd[4 * v + 3] = w4.w;
+  }
+}
+// Staging position (byte offset in an 80-byte chunk) of activation q[5g + k]
+// for group g of the chunk (0..15).
+__host__ __device__ inline int b3_qpos(int g, int k) { return 4 * (5 * (g >> 2) + k) + (g & 3); }
 
 }  // namespace moe

@@ -39,6 +39,7 @@ struct Workspace {
   int* qsum;            // [B] sum of each token's int8 activations (the code offset)
   int* n_act;           // [1] experts chosen by at least one token this step
   int* act_e;           // [E] those experts, ascending
+  int* act_w;           // [E] their weight slots (index into the per-expert arrays)
   int* act_off;         // [E + 1] first pair of each (act_off[n_act] = B * top_e)
   int* pair_tok;        // [P] token of each pair
   int* pair_slot;       // [P] routing slot of each pair
@@ -72,6 +73,7 @@ struct RouteArgs {
   float* dbg_w;
   bool quantize;  // also rotate + quantize the tokens (sparse path)
   int ep_rank, ep_size;  // expert parallelism: pairs of experts e % ep_size == ep_rank only (ep_size 0/1: all)
+  const int32_t* expert_slot;  // [E] weight slot of each expert (< 0: none held), or null (slot = e)
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 
@@ -85,6 +87,7 @@ struct ExpertArgs {
   unsigned long long wait_ns;  // limit of every bounded copy wait (test hook; kWaitLimitNs normally)
   int withhold_copy;           // test hook: 1 = the one-cluster reader never issues one sketch copy
   int ep_partial;      // 1: write the per-slot outputs only (no combine); expert-parallel steps
+  int sk3;             // sketch rows: 0 2-bit codes (d / 4 bytes), 1 base 3 (sk3_row_bytes(d) bytes)
   const uint16_t* x;
   const uint16_t* w_router;  // routing inside the expert kernel (small B)
   const float* bias;
@@ -135,6 +138,9 @@ cudaError_t query_plan(const ExpertArgs& a, bool dense, int out[4]);
 cudaError_t launch_build_sketch(int E, int I, int d, const uint16_t* w_gate, const uint16_t* w_up,
                                 uint64_t seed, int8_t* rot_sign, uint32_t* sk_gate, uint32_t* sk_up,
                                 float* alpha_gate, float* alpha_up, cudaStream_t s);
+// Repacks rows of 2-bit codes ([rows, d / 16] words) as base-3 rows
+// ([rows, sk3_row_bytes(d)] bytes).
+cudaError_t launch_sketch_to_base3(long rows, int d, const uint32_t* codes, uint8_t* out, cudaStream_t s);
 size_t lowrank_ws_bytes(int E, int I, int d, int r);
 cudaError_t launch_build_lowrank(int E, int I, int d, int r, const uint16_t* w_down, uint16_t* u_sigma,
                                  uint16_t* v, void* ws, cudaStream_t s);

@@ -652,7 +652,9 @@ constexpr int kMaxDSlots = 64;      // down-row slots
 
 struct RLayout {
   int mbar, misc, x, q, logit, alpha, ubar, vown, ahat, aown, vloc, rloc, listc, listk, flags, rows, drows, kslot,
-      kco, dcnt, gu, zred, zparts, ztot, ybuf, cntb, ring, total;
+      kco, dcnt, gu, zred, zparts, ztot, ybuf, cntb, q5, ring, total;
+  int skrow;    // bytes of one sketch row (2-bit codes: d / 4; base 3: sk3_row_bytes(d))
+  int nv3;      // 16-byte chunks of a base-3 row (0 for 2-bit codes)
   int P, Pext;  // exact-stage slots (gate + up rows of one channel, 4d bytes each): P per warp, one more
                 // for warps 0 .. Pext - 1
   int W;        // warps that own slots (all when P >= 1)
@@ -663,7 +665,7 @@ struct RLayout {
   int ch0[17], col0[17], ex0[17];
 };
 
-__host__ inline RLayout make_rlayout(int NT, int B, int E, int I, int d, int r, int cs, int smem_max) {
+__host__ inline RLayout make_rlayout(int NT, int B, int E, int I, int d, int r, int cs, int smem_max, bool sk3) {
   RLayout L = {};
   for (int o = 0; o <= cs && o < 17; o++) {
     const int c4 = 4 * cdiv(o * cdiv(I, 4), cs);
@@ -679,6 +681,8 @@ __host__ inline RLayout make_rlayout(int NT, int B, int E, int I, int d, int r, 
   L.cols_max = 8 * cdiv(d / 8, cs);
   L.d8 = d / 8;
   L.skc = 16 * (d / 4);
+  L.skrow = sk3 ? sk3_row_bytes(d) : d / 4;
+  L.nv3 = sk3 ? L.skrow / 16 : 0;
   L.rr = r > 0 ? r : 1;
   int o = 0;
   auto take = [&](int bytes) {
@@ -715,6 +719,8 @@ __host__ inline RLayout make_rlayout(int NT, int B, int E, int I, int d, int r, 
   L.zred = take(NWARP * NT * L.rr * 4);
   L.zparts = take(cs * NT * L.rr * 4);
   L.ztot = take(NT * L.rr * 4);
+  // base-3 sketch: the tokens' activations staged per 16-byte chunk, digit-major
+  L.q5 = sk3 ? take(B * L.nv3 * 80) : 0;
   L.ring = o;
   const int avail = smem_max - o;
   const int ring = avail > 0 ? avail / (8 * d) * (8 * d) : 0;
@@ -732,7 +738,7 @@ __host__ inline RLayout make_rlayout(int NT, int B, int E, int I, int d, int r, 
 }
 
 // misc ints of the sparse kernel (beyond the shared positions above)
-enum { MI_NSPEC = 8, MI_NROWS = 9, MI_NDC = 10, MI_NK = 11, MI_SQ = 13 };  // MI_SQ: B <= 2 ints
+enum { MI_NCT = 2, MI_NSPEC = 8, MI_NROWS = 9, MI_NDC = 10, MI_NK = 11, MI_SQ = 13 };  // MI_NCT, MI_SQ: B <= 2 ints
 static_assert((int)MI_NK < (int)MI_DONE && (int)MI_SQ > (int)MI_DONE && (int)MI_SQ + 2 <= (int)MI_TOK,
               "misc positions");
 // flags of an own channel: candidate of token t (bit t), kept by token t
@@ -744,14 +750,15 @@ constexpr unsigned char kFlagSpec = 16;
 __device__ __forceinline__ void issue_sketch(const ExpertArgs& a, const RLayout& L, char* ring, uint64_t* bars, int e,
                                              int i0, int i1, int ch, int slot) {
   const int c0 = i0 + 16 * ch, cnt = min(16, i1 - c0);
-  const uint32_t bytes = cnt * (a.d / 4);
+  const uint32_t bytes = cnt * L.skrow;
   char* dst = ring + (size_t)slot * 2 * L.skc;
   mbar_expect_tx(&bars[slot], 2 * bytes);
-  bulk_g2s(dst, a.sk_gate + ((size_t)e * a.I + c0) * (a.d / 16), bytes, &bars[slot]);
+  bulk_g2s(dst, reinterpret_cast<const char*>(a.sk_gate) + ((size_t)e * a.I + c0) * L.skrow, bytes, &bars[slot]);
   // test hook: chunk 0's up rows are expected but never copied, so every
   // wait for that chunk runs out (nothing is left in flight)
   if (a.withhold_copy && ch == 0) return;
-  bulk_g2s(dst + L.skc, a.sk_up + ((size_t)e * a.I + c0) * (a.d / 16), bytes, &bars[slot]);
+  bulk_g2s(dst + L.skc, reinterpret_cast<const char*>(a.sk_up) + ((size_t)e * a.I + c0) * L.skrow, bytes,
+           &bars[slot]);
 }
 
 // Gate and up rows of channel i into a 4d-byte slot.
@@ -833,7 +840,7 @@ __device__ __forceinline__ void write_sorted(const uint64_t* v, const int* rank,
     if (v[li]) mine[rank[li]] = v[li];
 }
 
-template <int NT, bool DBG>
+template <int NT, bool DBG, bool SK3>
 __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L) {
   extern __shared__ __align__(128) char smem[];
   cg::cluster_group cluster = cg::this_cluster();
@@ -925,6 +932,18 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
   for (int t = 0; t < a.B; t++)
     rotate_quantize(a, xs + (size_t)t * d, qs + (size_t)t * d, reinterpret_cast<float*>(ring + L.ringb - 4 * d),
                     cxs + t, reinterpret_cast<float*>(misc + MI_RED), sv_pre, misc + MI_SQ + t);
+  if (SK3) {
+    // activations staged per 16-byte chunk of the base-3 rows, digit-major
+    // (b3_qpos); zero past d
+    for (int o = tid; o < a.B * L.nv3 * 16; o += NTHR) {
+      const int t = o / (L.nv3 * 16), g = o - t * (L.nv3 * 16);
+      const int8_t* qt = qs + (size_t)t * d;
+      char* c5 = smem + L.q5 + ((size_t)t * L.nv3 + (g >> 4)) * 80;
+#pragma unroll
+      for (int k = 0; k < 5; k++) c5[b3_qpos(g & 15, k)] = 5 * g + k < d ? (char)qt[5 * g + k] : (char)0;
+    }
+    __syncthreads();
+  }
   if (DBG) stamp(a, cid, rank, 1);
   int tix[NT];
 #pragma unroll
@@ -987,7 +1006,24 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
       int G[NT], U[NT];
 #pragma unroll
       for (int t = 0; t < NT; t++) G[t] = U[t] = 0;
-      if (li < nown) {
+      if (SK3 && li < nown) {
+        const int slot = j - rb;
+        if (!mbar_wait_bounded(&skbars[slot], par, err, a.wait_ns)) misc[MI_DONE] = 1;
+        if (lane < L.nv3) {  // lane = the row's 16-byte chunk (80 trits)
+          const uint4 g4 = reinterpret_cast<const uint4*>(ring + (size_t)slot * 2 * L.skc + warp * L.skrow)[lane];
+          const uint4 u4 =
+              reinterpret_cast<const uint4*>(ring + (size_t)slot * 2 * L.skc + L.skc + warp * L.skrow)[lane];
+          uint32_t go[20], uo[20], qd[20];
+          b3_decode16(g4, go);
+          b3_decode16(u4, uo);
+#pragma unroll
+          for (int t = 0; t < NT; t++) {
+            b3_load_q(smem + L.q5 + ((size_t)tix[t] * L.nv3 + lane) * 80, qd);
+            G[t] = b3_dot16(go, qd, 0);
+            U[t] = b3_dot16(uo, qd, 0);
+          }
+        }
+      } else if (!SK3 && li < nown) {
         const int slot = j - rb;
         if (!mbar_wait_bounded(&skbars[slot], par, err, a.wait_ns)) misc[MI_DONE] = 1;
         const uint4* gw = reinterpret_cast<const uint4*>(ring + (size_t)slot * 2 * L.skc + warp * (d / 4));
@@ -1130,6 +1166,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
     for (int li = tid; li < nown; li += NTHR) {
       const int r0 = rloc[t * om + li];
       int tot = r0;
+#pragma unroll 4
       for (int o = 0; o < cs; o++)
         if (o != rank) tot += cntb[o * om + r0];
       if (tot < a.c) atomicOr(reinterpret_cast<unsigned*>(flags) + (li >> 2), (1u << t) << (8 * (li & 3)));
@@ -1141,7 +1178,9 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
   // started yet; drows: every own candidate, ascending
   const int nspec = misc[MI_NSPEC];
   if (warp == 0) {
-    int base = nspec, dbase = 0;
+    int base = nspec, dbase = 0, nct[NT];
+#pragma unroll
+    for (int t = 0; t < NT; t++) nct[t] = 0;
     for (int w0 = 0; w0 < nown; w0 += 32) {
       const int li = w0 + lane;
       const unsigned f = li < nown ? flags[li] : 0u;
@@ -1151,10 +1190,14 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
       if (cand) drows[dbase + __popc(bc & ((1u << lane) - 1u))] = li;
       base += __popc(bm);
       dbase += __popc(bc);
+#pragma unroll
+      for (int t = 0; t < NT; t++) nct[t] += __popc(__ballot_sync(kFull, (f >> t) & 1u));
     }
     if (lane == 0) {
       misc[MI_NROWS] = base;
       misc[MI_NDC] = dbase;
+#pragma unroll
+      for (int t = 0; t < NT; t++) misc[MI_NCT + t] = nct[t];  // own candidates of each token
     }
   }
   __syncthreads();
@@ -1264,8 +1307,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
   if (DBG) stamp(a, cid, rank, 10);
 #pragma unroll 1
   for (int t = 0; t < n; t++) {
-    int nct = 0;  // own candidates of token t (the nonzero entries of the own list)
-    for (int m = 0; m < ndc; m++) nct += (flags[drows[m]] >> t) & 1u;
+    const int nct = misc[MI_NCT + t];  // own candidates of token t (the nonzero entries of the own list)
     merge_counts(listk + (size_t)t * cs * om, listk + ((size_t)t * cs + rank) * om, nct, om, L.nsteps, cs, rank, cntb);
     __syncthreads();
     for (int m = tid; m < ndc; m += NTHR) {
@@ -1273,6 +1315,7 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
       if (!((flags[li] >> t) & 1u)) continue;
       const int r0 = rloc[t * om + m];
       int tot = r0;
+#pragma unroll 4
       for (int o = 0; o < cs; o++)
         if (o != rank) tot += cntb[o * om + r0];
       if (tot < a.k) atomicOr(reinterpret_cast<unsigned*>(flags) + (li >> 2), (4u << t) << (8 * (li & 3)));
@@ -1757,15 +1800,19 @@ cudaError_t plan_dense(const ExpertArgs& a, DensePlan* out) {
 
 // ----- sparse reader (one or two tokens)
 struct ReaderPlan {
-  int dev, B, E, I, d, r, top_e, forced;
+  int dev, B, E, I, d, r, top_e, forced, sk3;
   int cs, smem, max_clusters, items;
   RLayout L;
 };
 
-template <int NT>
-const void* reader_ptr(bool dbg) {
-  return dbg ? reinterpret_cast<const void*>(&reader_kernel<NT, true>)
-             : reinterpret_cast<const void*>(&reader_kernel<NT, false>);
+template <int NT, bool SK3>
+const void* reader_ptr_f(bool dbg) {
+  return dbg ? reinterpret_cast<const void*>(&reader_kernel<NT, true, SK3>)
+             : reinterpret_cast<const void*>(&reader_kernel<NT, false, SK3>);
+}
+const void* reader_ptr(int NT, bool sk3, bool dbg) {
+  if (NT == 1) return sk3 ? reader_ptr_f<1, true>(dbg) : reader_ptr_f<1, false>(dbg);
+  return sk3 ? reader_ptr_f<2, true>(dbg) : reader_ptr_f<2, false>(dbg);
 }
 
 cudaError_t plan_reader(const ExpertArgs& a, ReaderPlan* out) {
@@ -1778,7 +1825,7 @@ cudaError_t plan_reader(const ExpertArgs& a, ReaderPlan* out) {
   for (int i = 0; i < ncache; i++) {
     const ReaderPlan& c = cache[i];
     if (c.dev == dev && c.B == a.B && c.E == a.E && c.I == a.I && c.d == a.d && c.r == a.r &&
-        c.top_e == a.top_e && c.forced == a.force_cs) {
+        c.top_e == a.top_e && c.forced == a.force_cs && c.sk3 == a.sk3) {
       *out = c;
       return cudaSuccess;
     }
@@ -1787,19 +1834,19 @@ cudaError_t plan_reader(const ExpertArgs& a, ReaderPlan* out) {
   err = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (err != cudaSuccess) return err;
   const int NT = a.B;
-  const void* fns[2] = {NT == 1 ? reader_ptr<1>(false) : reader_ptr<2>(false),
-                        NT == 1 ? reader_ptr<1>(true) : reader_ptr<2>(true)};
+  const bool sk3 = a.sk3 != 0;
+  const void* fns[2] = {reader_ptr(NT, sk3, false), reader_ptr(NT, sk3, true)};
   for (const void* f : fns) {
     err = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (err != cudaSuccess) return err;
   }
   const int items = a.B * a.top_e < a.E ? a.B * a.top_e : a.E;
-  ReaderPlan p = {dev, a.B, a.E, a.I, a.d, a.r, a.top_e, a.force_cs, 0, 0, 0, items, {}};
+  ReaderPlan p = {dev, a.B, a.E, a.I, a.d, a.r, a.top_e, a.force_cs, a.sk3, 0, 0, 0, items, {}};
   double best = 1e30;
   for (int cs = 16; cs >= 2; cs--) {
     if (a.force_cs && cs != a.force_cs) continue;
     if (a.I < 4 * cs || a.E < cs || 8 * cdiv(a.d / 8, cs) > a.d) continue;
-    const RLayout L = make_rlayout(NT, a.B, a.E, a.I, a.d, a.r, cs, smem_max);
+    const RLayout L = make_rlayout(NT, a.B, a.E, a.I, a.d, a.r, cs, smem_max, sk3);
     if (L.own_max > kMaxOwn || L.W < 4 || L.nskbuf < 1 || L.ndslot < 1 || L.total > smem_max) continue;
     int nclusters = 1 << 30;
     for (const void* f : fns) {
@@ -1856,7 +1903,7 @@ cudaError_t launch_reader(const ExpertArgs& a0, cudaStream_t s) {
   a.cs = plan.cs;
   const bool dbg = a.dbg_ids || a.dbg_w || a.dbg_G || a.dbg_U || a.dbg_sigma || a.dbg_cand || a.dbg_kept ||
                    a.dbg_a_kept || a.dbg_y_expert || a.dbg_phase;
-  const void* fn = a.B == 1 ? reader_ptr<1>(dbg) : reader_ptr<2>(dbg);
+  const void* fn = reader_ptr(a.B, a.sk3 != 0, dbg);
   err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem);
   if (err != cudaSuccess) return err;
   cudaLaunchAttribute attr[2];

@@ -248,6 +248,12 @@ __global__ void __launch_bounds__(512) select_kernel(RouteArgs a) {
         aidx[e] = ra + ia - ac;
         if (ac) {
           a.ws.act_e[ra + ia - 1] = e;
+          int w = a.expert_slot ? __ldg(a.expert_slot + e) : e;
+          if (w < 0) {  // routed to an expert whose weights this caller does not hold
+            atomicOr(a.ws.err, kErrNoWeights);
+            w = 0;
+          }
+          a.ws.act_w[ra + ia - 1] = w;
           a.ws.act_off[ra + ia - 1] = rp + ip - c;
         }
       }
@@ -327,7 +333,7 @@ size_t workspace_layout(int B, int E, int top_e, int d, int I, int r, void* base
   // the streamed path
   const size_t P = (size_t)B * top_e, W = (size_t)(I + 31) / 32, nbs = (size_t)(I + 15) / 16;
   const bool st = I > 0;
-  const size_t o_qs = take(sizeof(int) * B), o_na = take(16), o_ae = take(sizeof(int) * E),
+  const size_t o_qs = take(sizeof(int) * B), o_na = take(16), o_ae = take(sizeof(int) * E), o_aw = take(sizeof(int) * E),
                o_ao = take(sizeof(int) * (E + 1)), o_pt = take(sizeof(int) * P), o_ps = take(sizeof(int) * P),
                o_pe = take(sizeof(int) * P), o_ar = take(sizeof(unsigned) * 2 * E);
   const size_t o_sa = st ? take(sizeof(float2) * P * I) : 0, o_zp = st ? take(sizeof(float) * P * nbs * r) : 0,
@@ -355,6 +361,7 @@ size_t workspace_layout(int B, int E, int top_e, int d, int I, int r, void* base
     ws->qsum = reinterpret_cast<int*>(p + o_qs);
     ws->n_act = reinterpret_cast<int*>(p + o_na);
     ws->act_e = reinterpret_cast<int*>(p + o_ae);
+    ws->act_w = reinterpret_cast<int*>(p + o_aw);
     ws->act_off = reinterpret_cast<int*>(p + o_ao);
     ws->pair_tok = reinterpret_cast<int*>(p + o_pt);
     ws->pair_slot = reinterpret_cast<int*>(p + o_ps);

@@ -103,13 +103,13 @@ constexpr int kQChunk = 80;                          // staged activations: 64 b
 // finishes token t.  Scores follow the one-cluster reader: ghat =
 // ((float)G alpha_g) c_x, uhat likewise, ahat = silu_r(ghat) uhat,
 // sigma = |ahat|, with G, U the exact integer dots less the code offset sum(q).
-template <int NVL>
+template <int NVL, bool SK3>
 __device__ __forceinline__ void screen_issue(const ExpertArgs& a, int u, int nblk, char* dst, uint64_t* bar) {
   using Geo = ScreenGeom<NVL>;
   const int ea = u / nblk, blk = u - ea * nblk;
-  const int e = __ldcg(a.ws.act_e + ea);
+  const int e = __ldcg(a.ws.act_w + ea);  // weight slot of the active expert
   const int i0 = blk * Geo::kChannels, ncw = min(Geo::kChannels, a.I - i0);
-  const size_t row = (size_t)a.d / 4;  // bytes of one sketch row
+  const size_t row = SK3 ? (size_t)sk3_row_bytes(a.d) : (size_t)a.d / 4;  // bytes of one sketch row
   const uint32_t bytes = (uint32_t)(ncw * row), ubytes = (uint32_t)(ncw * a.r * 2);
   mbar_expect_tx(bar, 2 * bytes + ubytes);
   bulk_g2s(dst, reinterpret_cast<const char*>(a.sk_gate) + ((size_t)e * a.I + i0) * row, bytes, bar);
@@ -117,7 +117,7 @@ __device__ __forceinline__ void screen_issue(const ExpertArgs& a, int u, int nbl
   if (ubytes) bulk_g2s(dst + 2 * kSkBytes, a.u_sigma + ((size_t)e * a.I + i0) * a.r, ubytes, bar);
 }
 
-template <int NVL>
+template <int NVL, bool SK3>
 __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
   pdl_trigger();
   pdl_wait();
@@ -141,21 +141,24 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
   const int n_act = __ldcg(a.ws.n_act);
   const int units = n_act * nblk;
   uint32_t* err = a.ws.err;
+  // base 3: rows of skrow bytes, nv3 16-byte chunks (80 trits each); lane
+  // part p takes chunks p, p + kParts, ...
+  const int skrow = SK3 ? sk3_row_bytes(d) : d / 4, nv3 = skrow / 16;
   if (tid == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
     fence_mbar_init();
   }
   __syncthreads();
-  if (tid == 0 && (int)blockIdx.x < units) screen_issue<NVL>(a, blockIdx.x, nblk, sk_stage, &bars[0]);
+  if (tid == 0 && (int)blockIdx.x < units) screen_issue<NVL, SK3>(a, blockIdx.x, nblk, sk_stage, &bars[0]);
   int it = 0, staged_p0 = -1, staged_tg = -1;
 #pragma unroll 1
   for (int u = blockIdx.x; u < units; u += gridDim.x, it++) {
     const int st = it & 1;
     if (tid == 0 && u + (int)gridDim.x < units)
-      screen_issue<NVL>(a, u + gridDim.x, nblk, sk_stage + (st ^ 1) * kSStageBytes, &bars[st ^ 1]);
+      screen_issue<NVL, SK3>(a, u + gridDim.x, nblk, sk_stage + (st ^ 1) * kSStageBytes, &bars[st ^ 1]);
     const int ea = u / nblk, blk = u - ea * nblk;
-    const int e = __ldcg(a.ws.act_e + ea), p0 = __ldcg(a.ws.act_off + ea);
+    const int e = __ldcg(a.ws.act_w + ea), p0 = __ldcg(a.ws.act_off + ea);  // e: weight slot
     const int m = __ldcg(a.ws.act_off + ea + 1) - p0;
     const int i0 = blk * Geo::kChannels, ncw = min(Geo::kChannels, I - i0);
     const bool ok = lc < ncw;
@@ -181,11 +184,23 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
           sqs[tid] = __ldcg(a.ws.qsum + tk);
           scx[tid] = __ldcg(a.ws.cx + tk);
         }
-        for (int o = tid; o < ng * nv * 4; o += kSThreads) {
-          const int t = o / (nv * 4), w = o - t * nv * 4;
-          const int tk = __ldcg(a.ws.pair_tok + p0 + tg + t);
-          *reinterpret_cast<uint4*>(qst + (t * nv + (w >> 2)) * kQChunk + (w & 3) * 16) =
-              ld_cg4(reinterpret_cast<const uint4*>(a.ws.q + (size_t)tk * d) + w);
+        if (SK3) {
+          // per 16-byte chunk of a base-3 row (16 groups of 5 trits), digit-major (b3_qpos)
+          for (int o = tid; o < ng * nv3 * 16; o += kSThreads) {
+            const int t = o / (nv3 * 16), g = o - t * nv3 * 16;
+            const int tk = __ldcg(a.ws.pair_tok + p0 + tg + t);
+            const signed char* qt = reinterpret_cast<const signed char*>(a.ws.q) + (size_t)tk * d;
+            char* c5 = qst + (t * nv3 + (g >> 4)) * kQChunk;
+#pragma unroll
+            for (int k = 0; k < 5; k++) c5[b3_qpos(g & 15, k)] = 5 * g + k < d ? (char)__ldcg(qt + 5 * g + k) : (char)0;
+          }
+        } else {
+          for (int o = tid; o < ng * nv * 4; o += kSThreads) {
+            const int t = o / (nv * 4), w = o - t * nv * 4;
+            const int tk = __ldcg(a.ws.pair_tok + p0 + tg + t);
+            *reinterpret_cast<uint4*>(qst + (t * nv + (w >> 2)) * kQChunk + (w & 3) * 16) =
+                ld_cg4(reinterpret_cast<const uint4*>(a.ws.q + (size_t)tk * d) + w);
+          }
         }
         staged_p0 = p0;
         staged_tg = tg;
@@ -196,7 +211,24 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
       for (int t = 0; t < kSTG; t++)
 #pragma unroll
         for (int w = 0; w < 4; w++) ga[t][w] = ua[t][w] = 0;
-      if (ok && landed) {
+      if (SK3 && ok && landed) {
+        const uint4* g3 = reinterpret_cast<const uint4*>(stage + (size_t)lc * skrow);
+        const uint4* u3 = reinterpret_cast<const uint4*>(stage + kSkBytes + (size_t)lc * skrow);
+#pragma unroll 1
+        for (int j = part; j < nv3; j += Geo::kParts) {
+          uint32_t go[20], uo[20];
+          b3_decode16(g3[j], go);
+          b3_decode16(u3[j], uo);
+#pragma unroll
+          for (int t = 0; t < kSTG; t++) {
+            if (t >= ng) break;
+            uint32_t qd[20];
+            b3_load_q(qst + (t * nv3 + j) * kQChunk, qd);
+            ga[t][0] = b3_dot16(go, qd, ga[t][0]);
+            ua[t][0] = b3_dot16(uo, qd, ua[t][0]);
+          }
+        }
+      } else if (!SK3 && ok && landed) {
 #pragma unroll 2
         for (int j = 0; j < nch; j++) {
           const int jr = (j + rot) & (nch - 1);
@@ -222,8 +254,8 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
       int G[kSTG], U[kSTG];
 #pragma unroll
       for (int t = 0; t < kSTG; t++) {
-        G[t] = code_dot_total(ga[t]);
-        U[t] = code_dot_total(ua[t]);
+        G[t] = SK3 ? ga[t][0] : code_dot_total(ga[t]);
+        U[t] = SK3 ? ua[t][0] : code_dot_total(ua[t]);
 #pragma unroll
         for (int o = 1; o < Geo::kParts; o <<= 1) {
           G[t] += __shfl_xor_sync(kFullMask, G[t], o);
@@ -347,7 +379,7 @@ __global__ void __launch_bounds__(kSelT) select_k_kernel(ExpertArgs a, int nblk)
 #pragma unroll 1
   for (int p = blockIdx.x; p < P; p += gridDim.x) {
     const int ea = __ldcg(a.ws.pair_ea + p);
-    const int e = __ldcg(a.ws.act_e + ea);
+    const int e = __ldcg(a.ws.act_w + ea);  // weight slot of the pair's expert
     for (int w = tid; w < W; w += kSelT) {
       sm.mk[w] = __ldcg(a.ws.candm + (size_t)p * W + w);
       sm.kw[w] = 0u;
@@ -524,7 +556,7 @@ __global__ void __launch_bounds__(kXThreads, 1) exact_kernel(ExpertArgs a) {
 #pragma unroll 1
   for (int u = ub; u < ue; u++) {
     const int ea = unit_expert(cu, n_act, u);
-    const int e = __ldcg(a.ws.act_e + ea), p0 = __ldcg(a.ws.act_off + ea);
+    const int e = __ldcg(a.ws.act_w + ea), p0 = __ldcg(a.ws.act_off + ea);  // e: weight slot
     const int m = __ldcg(a.ws.act_off + ea + 1) - p0;
     const int j0 = (u - cu[ea]) * kXRows;
     const int nrows = min(kXRows, __ldcg(a.ws.n_u + ea) - j0);
@@ -535,7 +567,7 @@ __global__ void __launch_bounds__(kXThreads, 1) exact_kernel(ExpertArgs a) {
       const int un = u + 1, ean = unit_expert(cu, n_act, un);
       const int jn = (un - cu[ean]) * kXRows + lane;
       if (jn < __ldcg(a.ws.n_u + ean)) {
-        const size_t row = (size_t)__ldcg(a.ws.act_e + ean) * I + __ldcg(a.ws.ulist + (size_t)ean * I + jn);
+        const size_t row = (size_t)__ldcg(a.ws.act_w + ean) * I + __ldcg(a.ws.ulist + (size_t)ean * I + jn);
         bulk_prefetch_l2(a.w_gate + row * d, 2 * d);
         bulk_prefetch_l2(a.w_up + row * d, 2 * d);
       }
@@ -646,7 +678,7 @@ __global__ void __launch_bounds__(kDThreads) down_kernel(ExpertArgs a) {
 #pragma unroll 1
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
     const int ea = u / ns, sl = u - ea * ns, j0 = sl * SW;
-    const int e = __ldcg(a.ws.act_e + ea), p0 = __ldcg(a.ws.act_off + ea);
+    const int e = __ldcg(a.ws.act_w + ea), p0 = __ldcg(a.ws.act_off + ea);  // e: weight slot
     const int m = __ldcg(a.ws.act_off + ea + 1) - p0;
     const int nd = __ldcg(a.ws.n_d + ea);
     const int* dl = a.ws.dlist + (size_t)ea * I;
@@ -769,9 +801,10 @@ __global__ void __launch_bounds__(kDThreads) down_kernel(ExpertArgs a) {
 // Resident CTAs per SM of each kernel, per device (queried once).
 struct Occupancy {
   int dev = -1, sms = 0;
-  int screen1 = 0, screen2 = 0, selc = 0, selk = 0, exact = 0, down128 = 0, down256 = 0;
+  int screen1 = 0, screen2 = 0, screen1b3 = 0, screen2b3 = 0, selc = 0, selk = 0, exact = 0, down128 = 0,
+      down256 = 0;
 };
-Occupancy g_occ;
+thread_local Occupancy g_occ;  // per calling thread: occupancies on its current device
 
 // Also raises the kernel's dynamic shared-memory limit to `smem`.
 template <class K>
@@ -861,8 +894,10 @@ cudaError_t launch_stream(const ExpertArgs& a, cudaStream_t s) {
     err = cudaDeviceGetAttribute(&o.sms, cudaDevAttrMultiProcessorCount, dev);
     if (err != cudaSuccess) return err;
     o.exact = occ(exact_kernel, kXThreads, exact_smem(4096));  // the largest staging; sets the limit
-    o.screen1 = occ(screen_kernel<1>, kSThreads, 2 * kSStageBytes);
-    o.screen2 = occ(screen_kernel<2>, kSThreads, 2 * kSStageBytes);
+    o.screen1 = occ(screen_kernel<1, false>, kSThreads, 2 * kSStageBytes);
+    o.screen2 = occ(screen_kernel<2, false>, kSThreads, 2 * kSStageBytes);
+    o.screen1b3 = occ(screen_kernel<1, true>, kSThreads, 2 * kSStageBytes);
+    o.screen2b3 = occ(screen_kernel<2, true>, kSThreads, 2 * kSStageBytes);
     o.selc = occ(select_c_kernel, kSelT, 0);
     o.selk = occ(select_k_kernel, kSelT, 0);
     o.down128 = occ(down_kernel<128>, kDThreads, 0);
@@ -875,10 +910,14 @@ cudaError_t launch_stream(const ExpertArgs& a, cudaStream_t s) {
   const int nvl = a.d <= 2048 ? 1 : 2;
   const int chans = nvl == 1 ? ScreenGeom<1>::kChannels : ScreenGeom<2>::kChannels;
   const int nblk = (a.I + chans - 1) / chans;
-  const int gs = nact * nblk < sms * (nvl == 1 ? g_occ.screen1 : g_occ.screen2) ? nact * nblk
-                                                                                   : sms * (nvl == 1 ? g_occ.screen1 : g_occ.screen2);
-  err = nvl == 1 ? launch_pdl(screen_kernel<1>, gs, kSThreads, 2 * kSStageBytes, s, a)
-                 : launch_pdl(screen_kernel<2>, gs, kSThreads, 2 * kSStageBytes, s, a);
+  const int socc = a.sk3 ? (nvl == 1 ? g_occ.screen1b3 : g_occ.screen2b3) : (nvl == 1 ? g_occ.screen1 : g_occ.screen2);
+  const int gs = nact * nblk < sms * socc ? nact * nblk : sms * socc;
+  if (a.sk3)
+    err = nvl == 1 ? launch_pdl(screen_kernel<1, true>, gs, kSThreads, 2 * kSStageBytes, s, a)
+                   : launch_pdl(screen_kernel<2, true>, gs, kSThreads, 2 * kSStageBytes, s, a);
+  else
+    err = nvl == 1 ? launch_pdl(screen_kernel<1, false>, gs, kSThreads, 2 * kSStageBytes, s, a)
+                   : launch_pdl(screen_kernel<2, false>, gs, kSThreads, 2 * kSStageBytes, s, a);
   if (err != cudaSuccess) return err;
   // top-c
   err = launch_pdl(select_c_kernel, P < sms * g_occ.selc ? P : sms * g_occ.selc, kSelT, 0, s, a);

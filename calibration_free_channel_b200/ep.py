@@ -19,6 +19,21 @@ def owned_experts(E: int, rank: int, world: int) -> list[int]:
     return [e for e in range(E) if e % world == rank]
 
 
+def shard_weights(W: dict, rank: int, world: int):
+    """The weights rank `rank` holds: the router whole, w_gate / w_up /
+    w_down of the experts e % world == rank stacked in that order, and the
+    [E] int32 slot map (e // world for them, -1 elsewhere) that
+    moe_reader_layer.expert_slot takes."""
+    E = W["w_router"].shape[0]
+    own = list(range(rank, E, world))
+    idx = torch.tensor(own, dtype=torch.long)
+    out = {n: (v if v is None or n in ("w_router", "router_bias") else v.index_select(0, idx.to(v.device)))
+           for n, v in W.items()}
+    slot = torch.full((E,), -1, dtype=torch.int32)
+    slot[idx] = torch.arange(len(own), dtype=torch.int32)
+    return out, slot
+
+
 def ep_step(partial: torch.Tensor, finish, group=None):
     """Sums this rank's fp32 partial [B, d] over the group in place (one
     all-reduce) and returns finish(sum)."""

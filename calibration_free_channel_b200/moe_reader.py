@@ -14,13 +14,15 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmoe_reader.so")
 
-MOE_OK, MOE_EINVAL, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT = range(5)
-_STATUS = {0: "MOE_OK", 1: "MOE_EINVAL", 2: "MOE_EUNSUPPORTED", 3: "MOE_ECUDA", 4: "MOE_ETIMEOUT"}
+MOE_OK, MOE_EINVAL, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT, MOE_EDEVICE = range(6)
+_STATUS = {0: "MOE_OK", 1: "MOE_EINVAL", 2: "MOE_EUNSUPPORTED", 3: "MOE_ECUDA", 4: "MOE_ETIMEOUT",
+           5: "MOE_EDEVICE"}
 
 EXPORTS = ["moe_reader_workspace_bytes", "moe_reader_build_sketch", "moe_reader_lowrank_workspace_bytes",
            "moe_reader_build_lowrank", "moe_reader_forward", "moe_reader_forward_dense",
            "moe_reader_forward_host", "moe_reader_rmsnorm", "moe_reader_check_error", "moe_reader_launch_plan",
-           "moe_reader_forward_noalloc", "moe_reader_forward_ep", "moe_reader_ep_finish", "moe_reader_last_error"]
+           "moe_reader_forward_noalloc", "moe_reader_forward_ep", "moe_reader_ep_finish", "moe_reader_last_error",
+           "moe_reader_sketch_row_bytes", "moe_reader_sketch_to_base3"]
 
 
 class MoeReaderLayer(C.Structure):
@@ -29,7 +31,8 @@ class MoeReaderLayer(C.Structure):
                 ("w_up", C.c_void_p), ("w_down", C.c_void_p), ("rot_sign", C.c_void_p),
                 ("sk_gate", C.c_void_p), ("sk_up", C.c_void_p), ("alpha_gate", C.c_void_p),
                 ("alpha_up", C.c_void_p), ("u_sigma", C.c_void_p), ("v", C.c_void_p),
-                ("recovery_input", C.c_int32), ("path", C.c_int32), ("cluster_size", C.c_int32)]
+                ("recovery_input", C.c_int32), ("path", C.c_int32), ("cluster_size", C.c_int32),
+                ("sketch_format", C.c_int32), ("expert_slot", C.c_void_p)]
 
 
 class MoeReaderDebug(C.Structure):
@@ -74,9 +77,12 @@ def lib():
         L.moe_reader_forward_noalloc.argtypes = [C.POINTER(MoeReaderLayer), i32, i32, i32, P, P, P, P]
         L.moe_reader_last_error.restype = C.c_char_p
         L.moe_reader_last_error.argtypes = []
+        L.moe_reader_sketch_row_bytes.restype = sz
+        L.moe_reader_sketch_row_bytes.argtypes = [i32, i32]
+        L.moe_reader_sketch_to_base3.argtypes = [i32, i32, i32, P, P, P]
         for f in EXPORTS:
-            if f != "moe_reader_workspace_bytes" and f != "moe_reader_lowrank_workspace_bytes" \
-                    and f != "moe_reader_last_error":
+            if f not in ("moe_reader_workspace_bytes", "moe_reader_lowrank_workspace_bytes", "moe_reader_last_error",
+                         "moe_reader_sketch_row_bytes"):
                 getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -115,6 +121,14 @@ def moe_reader_build_sketch(E, I, d, w_gate, w_up, rot_seed, rot_sign, sk_gate, 
     _check(lib().moe_reader_build_sketch(E, I, d, _ptr(w_gate), _ptr(w_up), rot_seed & ((1 << 64) - 1),
                                          _ptr(rot_sign), _ptr(sk_gate), _ptr(sk_up), _ptr(alpha_gate),
                                          _ptr(alpha_up), _stream(stream)))
+
+
+def moe_reader_sketch_row_bytes(d, fmt) -> int:
+    return int(lib().moe_reader_sketch_row_bytes(d, fmt))
+
+
+def moe_reader_sketch_to_base3(E, I, d, sk_codes, sk_base3, stream=None):
+    _check(lib().moe_reader_sketch_to_base3(E, I, d, _ptr(sk_codes), _ptr(sk_base3), _stream(stream)))
 
 
 def moe_reader_build_lowrank(E, I, d, r, w_down, u_sigma, v, workspace, ws_bytes, stream=None):
@@ -186,34 +200,65 @@ class Layer:
     """A resident MoE layer on the GPU: bf16 weights, the sketch and the
     low-rank map, with the C struct that describes them."""
 
-    def __init__(self, weights: dict, top_e: int, device="cuda"):
+    def __init__(self, weights: dict, top_e: int, device="cuda", expert_slot=None):
+        """weights: w_router [E, d] (and router_bias [E]) for every expert;
+        w_gate, w_up, w_down for all E experts, or (with expert_slot, [E]
+        int32: the index of each expert in those arrays, -1 if not held) for
+        the held experts only, compacted."""
         dev = torch.device(device)
         self.w = {k: (v.to(dev).contiguous() if v is not None else None) for k, v in weights.items()}
-        E, I, d = self.w["w_gate"].shape
-        self.E, self.I, self.d, self.top_e, self.r = E, I, d, top_e, 0
+        Eh, I, d = self.w["w_gate"].shape
+        E = self.w["w_router"].shape[0]
+        if expert_slot is None and Eh != E:
+            raise ValueError(f"{Eh} experts of weights for a router of {E}: pass expert_slot")
+        self.E, self.E_held, self.I, self.d, self.top_e, self.r = E, Eh, I, d, top_e, 0
         self.rot_sign = torch.empty(d, dtype=torch.int8, device=dev)
-        self.sk_gate = torch.empty((E, I, d // 16), dtype=torch.int32, device=dev)
+        self.sk_gate = torch.empty((Eh, I, d // 16), dtype=torch.int32, device=dev)
         self.sk_up = torch.empty_like(self.sk_gate)
-        self.alpha_gate = torch.empty((E, I), dtype=torch.float32, device=dev)
+        self.alpha_gate = torch.empty((Eh, I), dtype=torch.float32, device=dev)
         self.alpha_up = torch.empty_like(self.alpha_gate)
         self.u_sigma = None
         self.v = None
         self._ws = None
         self.path = 0          # which reader runs a sparse step (see struct)
+        self.sketch_format = 0  # 0: 2-bit codes, 1: base 3 (build_sketch(packing=...))
+        # [E] int32 weight slot of each expert (held experts only, compacted), or None
+        self.expert_slot = None if expert_slot is None else \
+            torch.as_tensor(expert_slot, dtype=torch.int32).to(dev).contiguous()
         self.cluster_size = 0  # CTAs per cluster of the cluster kernels (0: automatic)
 
-    def build_sketch(self, rot_seed: int, stream=None):
-        moe_reader_build_sketch(self.E, self.I, self.d, self.w["w_gate"], self.w["w_up"], rot_seed,
+    def build_sketch(self, rot_seed: int, stream=None, packing: str = "2bit"):
+        """packing "2bit": [E, I, d/16] words of 2-bit codes; "base3": [E, I,
+        sketch_row_bytes] bytes, five trits per byte (the codes are built,
+        repacked and dropped)."""
+        if packing not in ("2bit", "base3"):
+            raise ValueError(f"packing {packing!r}: use '2bit' or 'base3'")
+        dev = self.w["w_gate"].device
+        Eh = self.E_held
+        if self.sk_gate.dtype != torch.int32:  # rebuilt after a base-3 packing
+            self.sk_gate = torch.empty((Eh, self.I, self.d // 16), dtype=torch.int32, device=dev)
+            self.sk_up = torch.empty_like(self.sk_gate)
+        moe_reader_build_sketch(Eh, self.I, self.d, self.w["w_gate"], self.w["w_up"], rot_seed,
                                 self.rot_sign, self.sk_gate, self.sk_up, self.alpha_gate, self.alpha_up, stream)
+        self.sketch_format = 0
+        if packing == "base3":
+            rb = moe_reader_sketch_row_bytes(self.d, 1)
+            g3 = torch.empty((Eh, self.I, rb), dtype=torch.uint8, device=dev)
+            u3 = torch.empty_like(g3)
+            moe_reader_sketch_to_base3(Eh, self.I, self.d, self.sk_gate, g3, stream)
+            moe_reader_sketch_to_base3(Eh, self.I, self.d, self.sk_up, u3, stream)
+            torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+            self.sk_gate, self.sk_up, self.sketch_format = g3, u3, 1
         return self
 
     def build_lowrank(self, r: int, stream=None):
         dev = self.w["w_down"].device
-        self.u_sigma = torch.empty((self.E, self.I, r), dtype=torch.bfloat16, device=dev)
-        self.v = torch.empty((self.E, self.d, r), dtype=torch.bfloat16, device=dev)
-        nb = moe_reader_lowrank_workspace_bytes(self.E, self.I, self.d, r)
+        Eh = self.E_held
+        self.u_sigma = torch.empty((Eh, self.I, r), dtype=torch.bfloat16, device=dev)
+        self.v = torch.empty((Eh, self.d, r), dtype=torch.bfloat16, device=dev)
+        nb = moe_reader_lowrank_workspace_bytes(Eh, self.I, self.d, r)
         ws = torch.empty(nb, dtype=torch.uint8, device=dev)
-        moe_reader_build_lowrank(self.E, self.I, self.d, r, self.w["w_down"], self.u_sigma, self.v, ws, nb, stream)
+        moe_reader_build_lowrank(Eh, self.I, self.d, r, self.w["w_down"], self.u_sigma, self.v, ws, nb, stream)
         torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
         del ws
         self.r = r
@@ -243,7 +288,29 @@ class Layer:
                               _ptr(self.alpha_gate), _ptr(self.alpha_up),
                               _ptr(self.u_sigma) if rr else None, _ptr(self.v) if rr else None, recovery_input,
                               self.path if path is None else path,
-                              self.cluster_size if cluster_size is None else cluster_size)
+                              self.cluster_size if cluster_size is None else cluster_size, self.sketch_format,
+                              _ptr(self.expert_slot))
+
+    def shard(self, rank: int, world: int) -> "Layer":
+        """What rank `rank` of a `world`-way expert-parallel step holds: the
+        experts e % world == rank of this layer (weights, sketch, low-rank
+        map) copied into new compacted arrays, the router whole, and
+        expert_slot[e] = e // world for them, -1 elsewhere."""
+        import copy
+        dev = self.w["w_gate"].device
+        own = torch.arange(rank, self.E, world, device=dev)
+        S = copy.copy(self)
+        S.w = {n: (v if v is None or n in ("w_router", "router_bias") else v.index_select(0, own).contiguous())
+               for n, v in self.w.items()}
+        for n in ("sk_gate", "sk_up", "alpha_gate", "alpha_up", "u_sigma", "v"):
+            t = getattr(self, n)
+            setattr(S, n, t.index_select(0, own).contiguous() if t is not None else None)
+        slot = torch.full((self.E,), -1, dtype=torch.int32)
+        slot[rank::world] = torch.arange(own.numel(), dtype=torch.int32)
+        S.expert_slot = slot.to(dev)
+        S.E_held = int(own.numel())
+        S._ws = None
+        return S
 
     def workspace(self, B: int):
         nb = moe_reader_workspace_bytes(B, self.E, self.top_e, self.I, self.d, 1, 1, self.r)

@@ -113,10 +113,11 @@ def router_bias(shape: BlockShape, seed: int = 0, layer: int = 0) -> torch.Tenso
     return torch.from_numpy(_gen(seed, layer, T_BIAS, 0).standard_normal(shape.E).astype(np.float32))
 
 
-def tokens(d: int, B: int, seed: int = 0, layer: int = 0) -> torch.Tensor:
-    """B tokens x = RMSNorm(t), t_j ~ Student-t(4), bf16 [B, d]."""
+def tokens(d: int, B: int, seed: int = 0, layer: int = 0, dof: float | None = 4.0) -> torch.Tensor:
+    """B tokens x = RMSNorm(t), t_j ~ Student-t(dof) (standard normal for
+    dof=None), bf16 [B, d]."""
     g = _gen(seed, layer, T_TOKENS, 0)
-    t = g.standard_t(4.0, size=(B, d))
+    t = g.standard_t(dof, size=(B, d)) if dof is not None else g.standard_normal(size=(B, d))
     t = t / np.sqrt(np.mean(t * t, axis=1, keepdims=True) + 1e-6)
     return _to_bf16(t)
 

@@ -52,7 +52,8 @@ typedef enum {
   MOE_EINVAL = 1,       /* bad argument (null, misaligned, out of range)      */
   MOE_EUNSUPPORTED = 2, /* valid shape outside this build's compiled limits   */
   MOE_ECUDA = 3,        /* a CUDA launch or query failed                      */
-  MOE_ETIMEOUT = 4      /* a bounded device wait ran out (moe_reader_check_error) */
+  MOE_ETIMEOUT = 4,     /* a bounded device wait ran out (moe_reader_check_error) */
+  MOE_EDEVICE = 5       /* a device-side check failed (moe_reader_check_error)  */
 } moe_status;
 
 /* One resident MoE layer: the weights and what the offline builders made
@@ -68,8 +69,9 @@ typedef struct {
   const uint16_t* w_up;        /* [E, I, d] bf16                                 */
   const uint16_t* w_down;      /* [E, I, d] bf16, channel-major                  */
   const int8_t* rot_sign;      /* [d] +-1: the random signs of the rotation      */
-  const uint32_t* sk_gate;     /* [E, I, d/16] 2-bit ternary sketch of W_gate     */
-  const uint32_t* sk_up;       /* [E, I, d/16] 2-bit ternary sketch of W_up       */
+  const void* sk_gate;         /* ternary sketch of W_gate, [E, I] rows in the
+                                  layout sketch_format names (below)             */
+  const void* sk_up;           /* ternary sketch of W_up, same layout             */
   const float* alpha_gate;     /* [E, I] per-row sketch scale                    */
   const float* alpha_up;       /* [E, I]                                         */
   const uint16_t* u_sigma;     /* [E, I, r] bf16 = U_r Sigma_r of W_down, or NULL */
@@ -99,6 +101,31 @@ typedef struct {
    * (MOE_ECUDA "invalid configuration" if that size does not fit the shape
    * on this device).  Other values are MOE_EINVAL. */
   int32_t cluster_size;
+  /* Layout of the sketch rows sk_gate / sk_up point to (both readers decode
+   * either; the trits, and so every dot, score and set, are the same).
+   *   0  2-bit codes: [E, I, d/16] uint32 words as moe_reader_build_sketch
+   *      writes them (d/4 bytes per row, 8.3% of the bf16 gate/up bytes);
+   *   1  base 3: [E, I, moe_reader_sketch_row_bytes(d, 1)] bytes as
+   *      moe_reader_sketch_to_base3 writes them, five trits per byte (416
+   *      bytes per row at d = 2048, 6.8%; "A reader that needs no data at
+   *      all" puts the resident sketch at about 7% of the BF16 checkpoint).
+   * Other values are MOE_EINVAL; the dense block ignores the sketch. */
+  int32_t sketch_format;
+  /* Which experts' weights the per-expert arrays hold (expert parallelism
+   * with a compacted layout): DEVICE [E] int32, expert_slot[e] = the index
+   * of expert e in w_gate, w_up, w_down, sk_gate, sk_up, alpha_gate,
+   * alpha_up, u_sigma and v, or -1 for an expert whose weights are not held;
+   * those arrays then have max(slot) + 1 entries instead of E (the router
+   * stays [E, d]).  A rank of an N-way expert-parallel step holding experts
+   * e % N == rank passes slot[e] = e / N for those and -1 elsewhere, and
+   * holds about E / N of the experts.  NULL: every array holds all E experts
+   * (slot = e).  Read by the streamed reader only: with expert_slot set,
+   * path 0 runs the streamed reader, path 1 and moe_reader_forward_dense
+   * return MOE_EUNSUPPORTED.  A step that routes a token to an expert with
+   * slot -1 reads slot 0 in its place and records device error bit 4
+   * (moe_reader_check_error: MOE_EDEVICE); under moe_reader_forward_ep only
+   * owned experts are read, so -1 is safe for every other expert. */
+  const int32_t* expert_slot;
 } moe_reader_layer;
 
 /* Optional per-stage outputs of moe_reader_forward (each pointer may be
@@ -163,6 +190,24 @@ moe_status moe_reader_build_sketch(int E, int I, int d, const uint16_t* w_gate, 
                                    uint64_t rot_seed, int8_t* rot_sign, uint32_t* sk_gate,
                                    uint32_t* sk_up, float* alpha_gate, float* alpha_up, void* stream);
 
+/* Bytes of one sketch row of d trits in a sketch_format (0: d/4; 1: ceil(d/5)
+ * rounded up to a multiple of 32); 0 for a d that is not a positive multiple
+ * of 16 or an unknown format. */
+size_t moe_reader_sketch_row_bytes(int d, int format);
+
+/* Offline: repacks one sketch matrix from the 2-bit codes of
+ * moe_reader_build_sketch ([E, I, d/16] words) to base 3 ([E, I,
+ * moe_reader_sketch_row_bytes(d, 1)] bytes; sketch_format 1).  Byte g of a
+ * row holds trits 5g .. 5g+4 as sum_i (T_{5g+i} + 1) 3^i (at most 242); the
+ * last group's positions past d hold zero trits, and the bytes past
+ * ceil(d/5) that pad the row to whole 32-byte sectors hold five zero trits
+ * (121).  Five trits per byte is 1.6 bits per trit, against 2 for the codes:
+ * the sketch's share of the bf16 gate/up bytes drops from 8.3% to 6.8% at
+ * d = 2048 ("A reader that needs no data at all": about 7%).  Call it once
+ * per matrix (gate, up); the input may be freed afterwards. */
+moe_status moe_reader_sketch_to_base3(int E, int I, int d, const uint32_t* sk_codes, uint8_t* sk_base3,
+                                      void* stream);
+
 /* Offline: the low-rank map of the down projections ("A reader that needs
  * no data at all": skipped channels are recovered through a low-rank map of
  * the down projections).  Per expert, the rank-r truncated SVD
@@ -213,7 +258,8 @@ moe_status moe_reader_forward_dense(const moe_reader_layer* layer, int B, const 
  * no rounding).  The caller sums y_partial over the ranks (e.g. one NCCL
  * all-reduce) and calls moe_reader_ep_finish.  The per-pair debug outputs
  * are written for owned pairs only.  Needs the layer's own weights for the
- * owned experts at least (other experts' rows are never read).
+ * owned experts at least (other experts' rows are never read): with
+ * layer->expert_slot, only the owned experts' weights, compacted.
  * MOE_EINVAL unless 1 <= ep_size <= E and 0 <= ep_rank < ep_size. */
 moe_status moe_reader_forward_ep(const moe_reader_layer* layer, int B, int k, int c,
                                  const uint16_t* x, int ep_rank, int ep_size, float* y_partial,
@@ -244,7 +290,7 @@ moe_status moe_reader_forward_host(const moe_reader_layer* layer, int B, int k, 
  *    whose workspace (moe_reader_workspace_bytes) exceeds 8 MiB return
  *    MOE_EINVAL ("workspace has ... bytes, needs ...") and launch nothing.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *    (cudaGetSymbolAddress) once and keeps it for later calls.
  *  - Every call shares the one array per device: calls that may overlap on
  *    the GPU (different streams, no ordering) race and must not be issued.
  *    Each call first clears the array's combine counters (cudaMemsetAsync on
@@ -269,8 +315,11 @@ moe_status moe_reader_launch_plan(int dense, int B, int E, int top_e, int I, int
 
 /* Synchronizes `stream`, reads and clears the workspace's device error word
  * (workspace NULL: the error word of moe_reader_forward_noalloc's scratch on
- * the current device).  Returns MOE_OK, or MOE_ETIMEOUT if a bounded wait ran
- * out since the last check. */
+ * the current device).  Returns MOE_OK; MOE_ETIMEOUT if a bounded wait ran
+ * out since the last check (bit 1); otherwise MOE_EDEVICE for the other
+ * device-side checks (bit 2: a work item out of range; bit 4: a routed
+ * expert without a weight slot, see moe_reader_layer.expert_slot).  The
+ * message names the bits. */
 moe_status moe_reader_check_error(void* workspace, void* stream);
 
 /* Message for the last non-OK status returned on this thread. */

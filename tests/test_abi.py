@@ -112,7 +112,9 @@ def test_one_cluster_reader_limits(lib):
 
 def test_layer_struct_layout():
     # the binding's structs match the header's field order and sizes
-    assert [n for n, _ in M.MoeReaderLayer._fields_][-3:] == ["recovery_input", "path", "cluster_size"]
+    assert [n for n, _ in M.MoeReaderLayer._fields_][-5:] == ["recovery_input", "path", "cluster_size",
+                                                             "sketch_format", "expert_slot"]
+    assert C.sizeof(M.MoeReaderLayer) == 5 * 4 + 4 + 12 * C.sizeof(C.c_void_p) + 4 * 4 + C.sizeof(C.c_void_p)
     assert [n for n, _ in M.MoeReaderDebug._fields_][-4:] == ["ev_before", "ev_after", "wait_limit_us",
                                                             "withhold_copy"]
     assert C.sizeof(M.MoeReaderDebug) == 12 * C.sizeof(C.c_void_p) + 8
@@ -125,6 +127,21 @@ def test_forward_without_recovery_needs_no_factors(lib):
     assert st == M.MOE_EINVAL and b"workspace" in lib.moe_reader_last_error()
 
 
+def test_sketch_format_is_validated(lib):
+    assert _fwd(lib, _layer(sketch_format=2)) == M.MOE_EINVAL
+    assert b"sketch_format" in lib.moe_reader_last_error()
+
+
+def test_sketch_row_bytes(lib):
+    # 2-bit codes: d / 4; base 3: ceil(d / 5) rounded up to whole 32-byte sectors
+    assert M.moe_reader_sketch_row_bytes(2048, 0) == 512
+    assert M.moe_reader_sketch_row_bytes(2048, 1) == 416
+    assert M.moe_reader_sketch_row_bytes(256, 1) == 64
+    assert M.moe_reader_sketch_row_bytes(4096, 1) == 832
+    assert M.moe_reader_sketch_row_bytes(2048, 2) == 0
+    assert M.moe_reader_sketch_row_bytes(100, 1) == 0
+
+
 def test_build_calls_validate(lib):
     f = 0x10000
     assert lib.moe_reader_build_sketch(8, 128, 100, f, f, 1, f, f, f, f, f, None) == M.MOE_EINVAL
@@ -133,9 +150,22 @@ def test_build_calls_validate(lib):
     assert lib.moe_reader_build_lowrank(8, 128, 256, 96, f, f, f, f, 1 << 40, None) == M.MOE_EUNSUPPORTED
     assert lib.moe_reader_build_lowrank(8, 128, 256, 8, f, f, f, f, 16, None) == M.MOE_EINVAL
     assert lib.moe_reader_rmsnorm(1, 256, -1.0, f, f, None) == M.MOE_EINVAL
+    assert lib.moe_reader_sketch_to_base3(8, 128, 100, f, f, None) == M.MOE_EINVAL
+    assert lib.moe_reader_sketch_to_base3(8, 128, 256, None, f, None) == M.MOE_EINVAL
     assert lib.moe_reader_forward_dense(C.byref(_layer(w_up=None)), 1, f, None, f, f, 1 << 30, None) == M.MOE_EINVAL
 
 
 def test_binding_raises_with_the_message(lib):
     with pytest.raises(M.MoeError, match="MOE_EINVAL.*d = 200"):
         M.moe_reader_forward(_layer(d=200), 1, 24, 48, 0x10000, None, 0x10000, None, 0x10000, 1 << 30)
+
+
+def test_expert_slot_rules(lib):
+    # the slot map is read by the streamed reader only: path 1 and the dense
+    # block refuse it before anything is enqueued; it must be 16-byte aligned
+    assert _fwd(lib, _layer(expert_slot=0x10000, path=1)) == M.MOE_EUNSUPPORTED
+    assert b"expert_slot" in lib.moe_reader_last_error()
+    st = lib.moe_reader_forward_dense(C.byref(_layer(expert_slot=0x10000)), 1, 0x10000, None, 0x10000, 0x10000,
+                                      1 << 30, None)
+    assert st == M.MOE_EUNSUPPORTED
+    assert _fwd(lib, _layer(expert_slot=0x10004)) == M.MOE_EINVAL

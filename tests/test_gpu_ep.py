@@ -100,3 +100,62 @@ def test_ep_rejects_bad_rank(tiny):
     x = synth.tokens(256, 1, seed=0).cuda()
     with pytest.raises(M.MoeError):
         layer.forward_ep(x, 24, 48, 2, 2)
+
+
+@pytest.mark.parametrize("world", [2, 8])
+def test_compacted_shards_match_the_full_layer(qwen, world):
+    """A rank that holds only its experts (compacted [E/N, ...] arrays and
+    expert_slot) computes the same partial, bit for bit, as a rank that
+    holds the whole layer, and holds 1/N of the expert bytes."""
+    W, layer, oc, top_e = qwen
+    x = synth.tokens(QWEN.d, 4, seed=43).cuda()
+    full_bytes = sum(t.numel() * t.element_size() for t in (layer.w["w_gate"], layer.w["w_up"], layer.w["w_down"],
+                                                          layer.sk_gate, layer.sk_up))
+    for rank in range(world):
+        S = layer.shard(rank, world)
+        held = sum(t.numel() * t.element_size() for t in (S.w["w_gate"], S.w["w_up"], S.w["w_down"], S.sk_gate,
+                                                        S.sk_up))
+        assert S.w["w_gate"].shape[0] == len(range(rank, QWEN.E, world))
+        assert held * world == full_bytes
+        want = layer.forward_ep(x, 136, 272, rank, world)
+        got = S.forward_ep(x, 136, 272, rank, world)
+        layer.check()
+        S.check()
+        assert torch.equal(got, want)
+
+
+def test_compacted_shard_base3_sketch(tiny):
+    """The slot indirection also covers base-3 sketch rows."""
+    W, _, _, _ = tiny
+    full = M.Layer(W, top_e=2).build_sketch(synth.rot_seed(0), packing="base3").build_lowrank(8)
+    x = synth.tokens(256, 5, seed=44).cuda()
+    for rank in range(2):
+        want = full.forward_ep(x, 24, 48, rank, 2)
+        got = full.shard(rank, 2).forward_ep(x, 24, 48, rank, 2)
+        assert torch.equal(got, want)
+
+
+def test_forward_with_a_missing_expert_reports_edevice(tiny):
+    """A plain step whose routing reaches an expert with no weight slot reads
+    slot 0 in its place (in bounds) and reports MOE_EDEVICE; the next check
+    is clean."""
+    W, layer, _, _ = tiny
+    S = layer.shard(0, 2)  # holds experts 0, 2, 4, 6 only
+    x = synth.tokens(256, 8, seed=45).cuda()  # 8 tokens x 2 slots reach odd experts too
+    S.forward(x, k=24, c=48)
+    with pytest.raises(M.MoeError, match="MOE_EDEVICE"):
+        S.check()
+    S.check()
+
+
+def test_shard_weights_builds_the_same_rank(tiny):
+    """A rank built from only its experts' weights (ep.shard_weights, never
+    holding the others) equals the slice of the full layer."""
+    from calibration_free_channel_b200 import ep
+    W, layer, _, _ = tiny
+    Wr, slot = ep.shard_weights(W, 1, 2)
+    R = M.Layer(Wr, top_e=2, expert_slot=slot).build_sketch(synth.rot_seed(0)).build_lowrank(8)
+    S = M.Layer(W, top_e=2).build_sketch(synth.rot_seed(0)).build_lowrank(8).shard(1, 2)
+    assert torch.equal(R.sk_gate, S.sk_gate) and torch.equal(R.u_sigma, S.u_sigma)
+    x = synth.tokens(256, 3, seed=46).cuda()
+    assert torch.equal(R.forward_ep(x, 24, 48, 1, 2), S.forward_ep(x, 24, 48, 1, 2))
