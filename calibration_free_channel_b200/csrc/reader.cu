@@ -1151,6 +1151,19 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
         if (j < nspec) issue_gate_up(a, e, i0 + rows[j], ring + (size_t)(sbase + m) * 4 * d, &wbars[m]);
       }
     }
+    // the next most likely candidates (own ranks up to 1.15 times the CTA's
+    // expected share of c) start moving into L2, so that their copies after
+    // the selection hit L2; those the selection leaves out are read unused
+    const int pf = min(nown, (int)(1.15f * (float)a.c * (float)nown / (float)I) + 1);
+    for (int li = tid; li < nown; li += NTHR) {
+      bool on = false;
+#pragma unroll
+      for (int t = 0; t < NT; t++) on |= t < n && rloc[t * om + li] < pf;
+      if (on && flags[li] != kFlagSpec) {
+        bulk_prefetch_l2(a.w_gate + ((size_t)e * I + i0 + li) * d, 2 * d);
+        bulk_prefetch_l2(a.w_up + ((size_t)e * I + i0 + li) * d, 2 * d);
+      }
+    }
   }
   if (DBG) stamp(a, cid, rank, 6);
   // the pushes above had the selection's time to land: arrive (release) now
@@ -1174,6 +1187,10 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
     __syncthreads();
   }
   if (DBG) stamp(a, cid, rank, 8);
+  // the down rows of every own candidate start moving into L2 now (the
+  // top-k keeps about k / c of them; their copies follow the exact stage)
+  for (int li = tid; li < nown; li += NTHR)
+    if (flags[li] & 3u) bulk_prefetch_l2(a.w_down + ((size_t)e * I + i0 + li) * d, 2 * d);
   // rows of the exact stage: the started ones, then the own candidates not
   // started yet; drows: every own candidate, ascending
   const int nspec = misc[MI_NSPEC];
