@@ -127,17 +127,38 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 __device__ __forceinline__ void mbar_expect_tx_only(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
+// L2 policy of the streamed weights: evict first.  A decode step reads each
+// weight byte once, and far more of them than the L2 holds; marking them
+// first to go keeps the lines that are reused from launch to launch (the
+// kernels' code, the per-step tables) resident instead.
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// 16-byte load of streamed weights: read-only, not kept in L1, evict-first
+// in L2.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p), "l"(evict_first_policy()));
+  return v;
+}
 // Bulk prefetch of [src, src + bytes) into L2 (16-byte aligned, multiple of 16).
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(src), "r"(bytes),
+               "l"(evict_first_policy())
+               : "memory");
 }
-// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
-// dst, src 16-byte aligned; bytes a multiple of 16.
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`
+// (weights: evict-first in L2).  dst, src 16-byte aligned; bytes a multiple
+// of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
           smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(evict_first_policy())
       : "memory");
 }
 __device__ __forceinline__ void cluster_arrive() {

@@ -312,7 +312,7 @@ __device__ __forceinline__ void load_row8(const uint4* row, int j0, int d8, int 
 #pragma unroll
   for (int u = 0; u < 8; u++) {
     const int j = j0 + 32 * u + lane;
-    w[u] = j < d8 ? __ldg(row + j) : make_uint4(0u, 0u, 0u, 0u);
+    w[u] = j < d8 ? ld_stream(row + j) : make_uint4(0u, 0u, 0u, 0u);
   }
 }
 

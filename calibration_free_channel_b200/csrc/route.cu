@@ -158,9 +158,15 @@ __global__ void __launch_bounds__(512) select_kernel(RouteArgs a) {
   for (int b = warp; b < B; b += nwarp) {
     const double* L = a.ws.logits + (size_t)b * E;
     uint32_t taken = 0;
-    double lv[32];  // this lane's logits (E <= 1024), read once
+    // this lane's logits (E <= 1024), read once; the unrolled loops stop at
+    // the first m past E (m < ceil(E / 32))
+    const int nm = (E + 31) >> 5;
+    double lv[32];
 #pragma unroll
-    for (int m = 0; m < 32; m++) lv[m] = lane + 32 * m < E ? L[lane + 32 * m] : -INFINITY;
+    for (int m = 0; m < 32; m++) {
+      if (m >= nm) break;
+      lv[m] = lane + 32 * m < E ? L[lane + 32 * m] : -INFINITY;
+    }
     double l0 = 0.0, my_l = 0.0;
     int my_id = 0;
     for (int s = 0; s < top; s++) {
@@ -168,6 +174,7 @@ __global__ void __launch_bounds__(512) select_kernel(RouteArgs a) {
       int bi = 0x7fffffff;
 #pragma unroll
       for (int m = 0; m < 32; m++) {
+        if (m >= nm) break;
         const int e = lane + 32 * m;
         if (e >= E || (taken & (1u << m))) continue;
         if (bi == 0x7fffffff || lv[m] > bv) {

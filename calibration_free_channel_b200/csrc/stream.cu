@@ -47,13 +47,6 @@ constexpr int kMaxI = 2048;
 constexpr int kMaxAct = 1024;   // active experts (E <= 1024)
 
 // 16-byte load of weights that are read once per step: no L1 allocation.
-__device__ __forceinline__ uint4 ld_stream(const void* p) {
-  uint4 v;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-      : "l"(p));
-  return v;
-}
 __device__ __forceinline__ uint4 ld_cg4(const void* p) { return __ldcg(reinterpret_cast<const uint4*>(p)); }
 
 // Counts one arrival at ctr (release of everything this thread ordered
@@ -88,7 +81,7 @@ struct ScreenGeom {
   static constexpr int kChannels = 4 * kPerWarp;  // 4 warps
 };
 constexpr int kSkBytes = 16384;                      // sketch rows of one block, per matrix
-constexpr int kSStageBytes = 2 * kSkBytes + 8192;   // + the block's Ubar rows (<= 32 x 128 bf16)
+constexpr int kSStageBytes = 2 * kSkBytes + 8192 + 256;  // + the block's Ubar rows (<= 32 x 128 bf16), alpha_g, alpha_u
 constexpr int kQChunk = 80;                          // staged activations: 64 bytes per chunk, padded
 
 // ------------------------------------------------------------------ screen
@@ -111,10 +104,15 @@ __device__ __forceinline__ void screen_issue(const ExpertArgs& a, int u, int nbl
   const int i0 = blk * Geo::kChannels, ncw = min(Geo::kChannels, a.I - i0);
   const size_t row = SK3 ? (size_t)sk3_row_bytes(a.d) : (size_t)a.d / 4;  // bytes of one sketch row
   const uint32_t bytes = (uint32_t)(ncw * row), ubytes = (uint32_t)(ncw * a.r * 2);
-  mbar_expect_tx(bar, 2 * bytes + ubytes);
+  const bool acopy = a.I % 4 == 0;  // the scales' slices are 16-byte aligned (else plain loads)
+  mbar_expect_tx(bar, 2 * bytes + ubytes + (acopy ? 8 * ncw : 0));
   bulk_g2s(dst, reinterpret_cast<const char*>(a.sk_gate) + ((size_t)e * a.I + i0) * row, bytes, bar);
   bulk_g2s(dst + kSkBytes, reinterpret_cast<const char*>(a.sk_up) + ((size_t)e * a.I + i0) * row, bytes, bar);
   if (ubytes) bulk_g2s(dst + 2 * kSkBytes, a.u_sigma + ((size_t)e * a.I + i0) * a.r, ubytes, bar);
+  if (acopy) {
+    bulk_g2s(dst + 2 * kSkBytes + 8192, a.alpha_gate + (size_t)e * a.I + i0, 4 * ncw, bar);
+    bulk_g2s(dst + 2 * kSkBytes + 8192 + 128, a.alpha_up + (size_t)e * a.I + i0, 4 * ncw, bar);
+  }
 }
 
 template <int NVL, bool SK3>
@@ -150,6 +148,10 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
     fence_mbar_init();
   }
   __syncthreads();
+  // units are dealt round-robin: the CTAs in flight together read one
+  // contiguous stretch of the sketch arrays, which spreads the reads evenly
+  // over the DRAM channels (contiguous ranges per CTA measured slower)
+  const bool acopy = I % 4 == 0;  // the scales arrive with the stage's bulk copies
   if (tid == 0 && (int)blockIdx.x < units) screen_issue<NVL, SK3>(a, blockIdx.x, nblk, sk_stage, &bars[0]);
   int it = 0, staged_p0 = -1, staged_tg = -1;
 #pragma unroll 1
@@ -162,11 +164,13 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
     const int m = __ldcg(a.ws.act_off + ea + 1) - p0;
     const int i0 = blk * Geo::kChannels, ncw = min(Geo::kChannels, I - i0);
     const bool ok = lc < ncw;
-    if (tid < ncw) {
+    const char* stage = sk_stage + st * kSStageBytes;
+    if (!acopy && tid < ncw) {
       salg[tid] = __ldg(a.alpha_gate + (size_t)e * I + i0 + tid);
       salu[tid] = __ldg(a.alpha_up + (size_t)e * I + i0 + tid);
     }
-    const char* stage = sk_stage + st * kSStageBytes;
+    const float* alg = acopy ? reinterpret_cast<const float*>(stage + 2 * kSkBytes + 8192) : salg;
+    const float* alu = acopy ? reinterpret_cast<const float*>(stage + 2 * kSkBytes + 8192 + 128) : salu;
     const uint4* grow = reinterpret_cast<const uint4*>(stage) + (size_t)lc * nv + part * nch;
     const uint4* urow = reinterpret_cast<const uint4*>(stage + kSkBytes) + (size_t)lc * nv + part * nch;
     const uint16_t* ubs = reinterpret_cast<const uint16_t*>(stage + 2 * kSkBytes);
@@ -273,8 +277,8 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
           }
         const int i = i0 + lc, pr = p0 + tg + t;
         const int g2 = g - sqs[t], u2 = uu - sqs[t];
-        const float gh = __fmul_rn(__fmul_rn((float)g2, salg[lc]), scx[t]);
-        const float uh = __fmul_rn(__fmul_rn((float)u2, salu[lc]), scx[t]);
+        const float gh = __fmul_rn(__fmul_rn((float)g2, alg[lc]), scx[t]);
+        const float uh = __fmul_rn(__fmul_rn((float)u2, alu[lc]), scx[t]);
         const float ah = __fmul_rn(silu_r(gh), uh);
         a.ws.sa[(size_t)pr * I + i] = make_float2(fabsf(ah), ah);
         sah[t][lc] = ah;
@@ -285,20 +289,23 @@ __global__ void __launch_bounds__(kSThreads) screen_kernel(ExpertArgs a) {
           if (a.dbg_sigma) a.dbg_sigma[off] = fabsf(ah);
         }
       }
-      // recovery-input partial of the block: sum over its channels of ahat_i Ubar_i
+      // recovery-input partial of the block: sum over its channels of
+      // ahat_i Ubar_i; four adjacent lanes split the channels of one
+      // (token, column) and meet in two shuffles
       if (r > 0) {
         __syncthreads();
-        for (int o = tid; o < ng * r; o += kSThreads) {
-          const int t = o / r, p = o - t * r;
-          const uint16_t* ub = ubs + p;
-          float z0 = 0.0f, z1 = 0.0f;
-          int l = landed ? 0 : ncw;
-          for (; l + 2 <= ncw; l += 2) {
-            z0 = fmaf(sah[t][l], bf16f(ub[(size_t)l * r]), z0);
-            z1 = fmaf(sah[t][l + 1], bf16f(ub[(size_t)(l + 1) * r]), z1);
+        const int nq = ng * r * 4, per = Geo::kChannels / 4;
+        for (int o0 = 0; o0 < nq; o0 += kSThreads) {
+          const int o = o0 + tid, tp = o >> 2, q4 = o & 3;
+          const int t = tp / r, p = tp - t * r;
+          float z = 0.0f;
+          if (o < nq && landed) {
+            const int l1 = min(ncw, q4 * per + per);
+            for (int l = q4 * per; l < l1; l++) z = fmaf(sah[t][l], bf16f(ubs[(size_t)l * r + p]), z);
           }
-          if (landed && l < ncw) z0 = fmaf(sah[t][l], bf16f(ub[(size_t)l * r]), z0);
-          a.ws.zpart[((size_t)(p0 + tg + t) * zstride + blk) * r + p] = z0 + z1;
+          z += __shfl_xor_sync(kFullMask, z, 1);
+          z += __shfl_xor_sync(kFullMask, z, 2);
+          if (o < nq && q4 == 0) a.ws.zpart[((size_t)(p0 + tg + t) * zstride + blk) * r + p] = z;
         }
       }
     }
@@ -380,6 +387,8 @@ __global__ void __launch_bounds__(kSelT) select_k_kernel(ExpertArgs a, int nblk)
   for (int p = blockIdx.x; p < P; p += gridDim.x) {
     const int ea = __ldcg(a.ws.pair_ea + p);
     const int e = __ldcg(a.ws.act_w + ea);  // weight slot of the pair's expert
+    // the expert's Ubar block starts moving into L2 for the gather below
+    if (tid == 0 && r > 0) bulk_prefetch_l2(a.u_sigma + (size_t)e * I * r, (uint32_t)(I * r * 2));
     for (int w = tid; w < W; w += kSelT) {
       sm.mk[w] = __ldcg(a.ws.candm + (size_t)p * W + w);
       sm.kw[w] = 0u;
@@ -452,8 +461,17 @@ __global__ void __launch_bounds__(kSelT) select_k_kernel(ExpertArgs a, int nblk)
       if (tid < r) {
         float s0 = 0.0f, s1 = 0.0f;
         for (int q = 0; q < nj; q++) s0 += zs[q * r + tid];
+        // the screen blocks' partials: independent loads, eight in flight
         const float* zp = a.ws.zpart + (size_t)p * zstride * r + tid;
-        for (int b = 0; b < nblk; b++) s1 += __ldcg(zp + (size_t)b * r);
+        float zb[8];
+#pragma unroll
+        for (int h = 0; h < 8; h++) zb[h] = 0.0f;
+        int b = 0;
+        for (; b + 8 <= nblk; b += 8)
+#pragma unroll
+          for (int h = 0; h < 8; h++) zb[h] += __ldcg(zp + (size_t)(b + h) * r);
+        for (; b < nblk; b++) zb[0] += __ldcg(zp + (size_t)b * r);
+        s1 = ((zb[0] + zb[1]) + (zb[2] + zb[3])) + ((zb[4] + zb[5]) + (zb[6] + zb[7]));
         a.ws.z[(size_t)p * r + tid] = s1 - s0;
       }
     }
@@ -523,7 +541,8 @@ __global__ void __launch_bounds__(kXThreads, 1) exact_kernel(ExpertArgs a) {
   pdl_wait();
   extern __shared__ __align__(16) char xsm[];  // [kXTok][2 d + 64] bf16 tokens (padded rows)
   __shared__ int cu[kMaxAct + 1];
-  __shared__ int srow[kXRows];
+  __shared__ int tw[kMaxAct], toff[kMaxAct + 1], tnu[kMaxAct];
+  __shared__ int srow3[3][kXRows];
   __shared__ __align__(16) float red[2][kXWarps / 2][32][8];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tid = threadIdx.x;
   const int tile = warp & 1, kq = warp >> 1;
@@ -548,30 +567,50 @@ __global__ void __launch_bounds__(kXThreads, 1) exact_kernel(ExpertArgs a) {
     }
     if (lane == 0) cu[n_act] = run;
   }
+  // per active expert, read once: weight slot, first pair, candidate-union size
+  for (int ea = tid; ea < n_act; ea += kXThreads) {
+    tw[ea] = __ldcg(a.ws.act_w + ea);
+    toff[ea] = __ldcg(a.ws.act_off + ea);
+    tnu[ea] = __ldcg(a.ws.n_u + ea);
+  }
+  if (tid == 0) toff[n_act] = __ldcg(a.ws.act_off + n_act);
   __syncthreads();
   const int total = cu[n_act];
   const int ub = (int)((long long)total * blockIdx.x / gridDim.x);
   const int ue = (int)((long long)total * (blockIdx.x + 1) / gridDim.x);
+  // row `lane16` of unit un (-1 past the expert's union) and its L2 prefetch
+  auto unit_row = [&](int un, int l16) {
+    const int ean = unit_expert(cu, n_act, un);
+    const int jn = (un - cu[ean]) * kXRows + l16;
+    return jn < tnu[ean] ? __ldcg(a.ws.ulist + (size_t)ean * I + jn) : -1;
+  };
+  auto prefetch_row = [&](int un, int row) {
+    if (row < 0) return;
+    const size_t g = (size_t)tw[unit_expert(cu, n_act, un)] * I + row;
+    bulk_prefetch_l2(a.w_gate + g * d, 2 * d);
+    bulk_prefetch_l2(a.w_up + g * d, 2 * d);
+  };
+  // the rows of units u .. u + 2 sit in a ring of three; the first two now
+  if (tid < kXRows)
+    for (int un = ub; un < ub + 2 && un < ue; un++) {
+      const int rw = unit_row(un, tid);
+      srow3[un % 3][tid] = rw;
+      prefetch_row(un, rw);
+    }
   int staged_ea = -1, staged_mt = -1;
 #pragma unroll 1
   for (int u = ub; u < ue; u++) {
     const int ea = unit_expert(cu, n_act, u);
-    const int e = __ldcg(a.ws.act_w + ea), p0 = __ldcg(a.ws.act_off + ea);  // e: weight slot
-    const int m = __ldcg(a.ws.act_off + ea + 1) - p0;
+    const int e = tw[ea], p0 = toff[ea];  // e: weight slot
+    const int m = toff[ea + 1] - p0;
     const int j0 = (u - cu[ea]) * kXRows;
-    const int nrows = min(kXRows, __ldcg(a.ws.n_u + ea) - j0);
-    __syncthreads();  // the previous unit is done with srow, xsm and red
-    if (tid < kXRows) srow[tid] = tid < nrows ? __ldcg(a.ws.ulist + (size_t)ea * I + j0 + tid) : -1;
-    if (warp == kXWarps - 1 && lane < kXRows && u + 1 < ue) {
-      // the next unit's rows start moving into L2
-      const int un = u + 1, ean = unit_expert(cu, n_act, un);
-      const int jn = (un - cu[ean]) * kXRows + lane;
-      if (jn < __ldcg(a.ws.n_u + ean)) {
-        const size_t row = (size_t)__ldcg(a.ws.act_w + ean) * I + __ldcg(a.ws.ulist + (size_t)ean * I + jn);
-        bulk_prefetch_l2(a.w_gate + row * d, 2 * d);
-        bulk_prefetch_l2(a.w_up + row * d, 2 * d);
-      }
-    }
+    const int nrows = min(kXRows, tnu[ea] - j0);
+    const int* srow = srow3[u % 3];
+    // the rows of the unit two on: loaded while this one is computed, then
+    // stored into the ring and started into L2
+    int row2 = -1;
+    if (tid < kXRows && u + 2 < ue) row2 = unit_row(u + 2, tid);
+    __syncthreads();  // the previous unit is done with xsm and red (and the ring slots are written)
 #pragma unroll 1
     for (int mt = 0; mt < m; mt += kXTok) {
       const int nt = min(kXTok, m - mt);
@@ -588,6 +627,15 @@ __global__ void __launch_bounds__(kXThreads, 1) exact_kernel(ExpertArgs a) {
         staged_mt = mt;
       }
       __syncthreads();
+      // the epilogue's candidate-mask words, in flight during the products
+      uint32_t cmw[4] = {0u, 0u, 0u, 0u};
+      if (kq == 0)
+#pragma unroll
+        for (int h = 0; h < 4; h++) {
+          const int tl = gid + (h >= 2 ? 8 : 0), rl = tile * 8 + tig * 2 + (h & 1);
+          if (tl < nt && rl < nrows)
+            cmw[h] = __ldcg(a.ws.candm + (size_t)(p0 + mt + tl) * W + (srow[rl] >> 5));
+        }
       const int rowi = srow[tile * 8 + gid];
       const uint4* gr = reinterpret_cast<const uint4*>(a.w_gate + ((size_t)e * I + max(rowi, 0)) * d);
       const uint4* ur = reinterpret_cast<const uint4*>(a.w_up + ((size_t)e * I + max(rowi, 0)) * d);
@@ -642,11 +690,14 @@ __global__ void __launch_bounds__(kXThreads, 1) exact_kernel(ExpertArgs a) {
           const int tl = gid + (h >= 2 ? 8 : 0), rl = tile * 8 + tig * 2 + (h & 1);
           if (tl < nt && rl < nrows) {
             const int i = srow[rl], pr = p0 + mt + tl;
-            if ((__ldcg(a.ws.candm + (size_t)pr * W + (i >> 5)) >> (i & 31)) & 1u)
-              a.ws.apos[(size_t)pr * I + i] = __fmul_rn(silu_r(sg[h]), su[h]);
+            if ((cmw[h] >> (i & 31)) & 1u) a.ws.apos[(size_t)pr * I + i] = __fmul_rn(silu_r(sg[h]), su[h]);
           }
         }
       }
+    }
+    if (tid < kXRows && u + 2 < ue) {
+      srow3[(u + 2) % 3][tid] = row2;
+      prefetch_row(u + 2, row2);
     }
   }
 }
@@ -674,14 +725,32 @@ __global__ void __launch_bounds__(kDThreads) down_kernel(ExpertArgs a) {
   const int g = tid / QW, q = tid - g * QW;
   const int n_act = __ldcg(a.ws.n_act);
   const int units = n_act * ns;
-  int staged_ea = -1, staged_tg = -1, staged_r0 = -1;
+  // units are dealt round-robin: the column slices of one expert's rows are
+  // read by different CTAs at about the same time, whole rows at once (one
+  // CTA taking a contiguous range of slices measured slower)
+  int staged_ea = -1, staged_tg = -1, staged_r0 = -1, cur_ea = -1;
+  __shared__ int se[4];  // the current expert: weight slot, first pair, last pair + 1, kept-union size
 #pragma unroll 1
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
     const int ea = u / ns, sl = u - ea * ns, j0 = sl * SW;
-    const int e = __ldcg(a.ws.act_w + ea), p0 = __ldcg(a.ws.act_off + ea);  // e: weight slot
-    const int m = __ldcg(a.ws.act_off + ea + 1) - p0;
-    const int nd = __ldcg(a.ws.n_d + ea);
+    if (ea != cur_ea) {
+      __syncthreads();  // every thread is done with the previous expert's scalars
+      if (tid == 0) {
+        const int w = __ldcg(a.ws.act_w + ea), o0 = __ldcg(a.ws.act_off + ea), o1 = __ldcg(a.ws.act_off + ea + 1),
+                  n = __ldcg(a.ws.n_d + ea);
+        se[0] = w;
+        se[1] = o0;
+        se[2] = o1;
+        se[3] = n;
+      }
+      __syncthreads();
+      cur_ea = ea;
+    }
+    const int e = se[0], p0 = se[1];  // e: weight slot
+    const int m = se[2] - p0, nd = se[3];
     const int* dl = a.ws.dlist + (size_t)ea * I;
+    // this slice's V rows start moving into L2 for the epilogue below
+    if (tid == 0 && r > 0) bulk_prefetch_l2(a.v + ((size_t)e * d + j0) * r, (uint32_t)(SW * r * 2));
     const uint4* wd = reinterpret_cast<const uint4*>(a.w_down + (size_t)e * I * d + j0) + q;
 #pragma unroll 1
     for (int tg = 0; tg < m; tg += kDTG) {
