@@ -199,7 +199,8 @@ __device__ __forceinline__ void dot8_mixed(uint4 a, uint4 b, float& acc0, float&
 // stops issuing and drains what is in flight).
 template <class Issue, class Consume>
 __device__ __forceinline__ bool warp_stream(int cnt, int P, uint64_t* bars, uint32_t& par, uint32_t* err,
-                                            Issue issue, Consume consume) {
+                                            Issue issue, Consume consume,
+                                            unsigned long long limit_ns = kWaitLimitNs) {
   const int lane = threadIdx.x & 31;
   if (cnt <= 0) return true;
   P = min(P, cnt);
@@ -215,7 +216,7 @@ __device__ __forceinline__ bool warp_stream(int cnt, int P, uint64_t* bars, uint
   int s = 0;
 #pragma unroll 1
   for (int j = 0; j < cnt; j++) {
-    ok = mbar_wait_bounded(&bars[s], (par >> s) & 1u, err);
+    ok = mbar_wait_bounded(&bars[s], (par >> s) & 1u, err, limit_ns);
     if (!ok) break;
     par ^= 1u << s;
     pend &= ~(1u << s);
@@ -235,7 +236,7 @@ __device__ __forceinline__ bool warp_stream(int cnt, int P, uint64_t* bars, uint
 #pragma unroll 1
     for (int q = 0; q < P; q++)
       if ((pend >> q) & 1u)
-        if (mbar_wait_bounded(&bars[q], (par >> q) & 1u, err)) par ^= 1u << q;
+        if (mbar_wait_bounded(&bars[q], (par >> q) & 1u, err, limit_ns)) par ^= 1u << q;
   }
   return ok;
 }
@@ -573,7 +574,7 @@ __device__ int down_rows(const ExpertArgs& a, int e, int j0, int ncq, int nr8, i
         for (int t = 0; t < NT; t++) co[u][t] = 0.0f;
         if (m < nrows) {
           const int i = chan(m);
-          if (coef(m, i, is_w, co[u])) w[u] = __ldg(reinterpret_cast<const uint4*>(base + (size_t)i * stride));
+          if (coef(m, i, is_w, co[u])) w[u] = ld_stream(base + (size_t)i * stride);
         }
       }
 #pragma unroll
@@ -1593,6 +1594,542 @@ __global__ void __launch_bounds__(NTHR, 1) reader_kernel(ExpertArgs a, RLayout L
   }
 }
 
+// ========================================================= batch-1 sparse
+// The one-token reader: one cluster per routed expert.  Each CTA screens a
+// slice of the expert's channels and pushes its (sigma, ahat) slice and its
+// part of the recovery input to every CTA, so that after one exchange every
+// CTA holds all I scores and selects the same top-c itself; the candidate
+// union is split evenly over the CTAs for the exact stage, whose a values
+// are exchanged once more; every CTA then selects the same top-k, reads its
+// column slice of the kept down rows (and the recovery rows) and combines.
+// Two exchanges in all, and an exact stage balanced over the cluster: at one
+// token this is faster than the channel-owning kernel above (30.8 against
+// 34.5 us per step on the Qwen layer shape), which wins from two tokens on
+// (56.7 against 78.4 us at two).  Prefetching likely rows into L2 ahead of
+// the selections, which helps the channel-owning kernel, made this one
+// slower (32.4 us) and is left out.
+__device__ __forceinline__ void issue_sketch1(const ExpertArgs& a, const Layout& L, char* buf, uint64_t* bars, int e,
+                                              int i0, int i1, int ch, int slot) {
+  const int c0 = i0 + 16 * ch, cnt = min(16, i1 - c0);
+  const uint32_t bytes = cnt * (a.d / 4);
+  char* dst = buf + (size_t)slot * 2 * L.skc;
+  mbar_expect_tx(&bars[slot], 2 * bytes);
+  bulk_g2s(dst, a.sk_gate + ((size_t)e * a.I + c0) * (a.d / 16), bytes, &bars[slot]);
+  // test hook: chunk 0's up rows are expected but never copied, so every
+  // wait for that chunk runs out (nothing is left in flight)
+  if (a.withhold_copy && ch == 0) return;
+  bulk_g2s(dst + L.skc, a.sk_up + ((size_t)e * a.I + c0) * (a.d / 16), bytes, &bars[slot]);
+}
+
+template <bool DBG>
+__global__ void __launch_bounds__(NTHR, 1) reader1_kernel(ExpertArgs a, Layout L) {
+  constexpr int NT = 1;         // one token per work item
+  constexpr bool FUSED = true;  // routing inside the kernel
+  extern __shared__ __align__(128) char smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int cs = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int cid = cluster_id();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.mbar);
+  uint64_t* wbars = bars + warp * kMaxSlots;
+  uint64_t* skbars = bars + NWARP * kMaxSlots;
+  uint64_t* uvbar = skbars + kSkBars;
+  int* misc = reinterpret_cast<int*>(smem + L.misc);
+  int* hist = reinterpret_cast<int*>(smem + L.hist);
+  if (tid < NWARP * kMaxSlots + kSkBars + 2) mbar_init(&bars[tid], 1);
+  if (tid == 0) misc[MI_DONE] = 0;
+  fence_mbar_init();
+  __syncthreads();
+  if (DBG) stamp(a, cid, rank, 0);
+
+  // Programmatic dependent launch: the next kernel in the stream may be
+  // scheduled now (onto free SMs); this one reads nothing in global memory
+  // before the previous kernel has completed and its writes are visible.
+  pdl_trigger();
+  pdl_wait();
+  char4 sv_pre = make_char4(0, 0, 0, 0);  // rotation signs of elements 4 tid .. 4 tid + 3 (in-kernel routing)
+  if (FUSED) {
+    if (tid < a.d / 4) sv_pre = __ldg(reinterpret_cast<const char4*>(a.rot_sign) + tid);
+    if (!fused_route<NT>(a, L, smem, misc, cs, rank, cid, cluster, [] {})) return;  // uniform per cluster
+  } else {
+    if (!load_item_table(a, cid, misc, NT)) return;
+  }
+  if (DBG) stamp(a, cid, rank, 4);
+  const int e = misc[MI_E], n = misc[MI_N];
+  const int I = a.I, d = a.d, r = a.r;
+  const int i0 = L.ch0[rank], i1 = L.ch0[rank + 1], nown = i1 - i0;
+  const int j0 = L.col0[rank], ncols = L.col0[rank + 1] - j0;
+  uint32_t* err = a.ws.err;
+  char* skbuf = smem + L.ring;
+  const int nchunk = cdiv(nown, 16);
+
+  // factor rows of the own channels, V rows of the own columns, and the
+  // first round of sketch chunks: all in flight before the token work
+  if (tid == 0) {
+    if (r > 0) {
+      const uint32_t bu = nown * r * 2, bv = ncols * r * 2;
+      mbar_expect_tx(uvbar, bu + bv);
+      bulk_g2s(smem + L.ubar, a.u_sigma + ((size_t)e * I + i0) * r, bu, uvbar);
+      bulk_g2s(smem + L.vown, a.v + ((size_t)e * d + j0) * r, bv, uvbar);
+    }
+    // the sketch scales of the own channels complete on chunk 0's barrier
+    // (every warp waits for chunk 0 before its first channel)
+    if (I % 4 == 0 && nown > 0) {
+      mbar_expect_tx_only(&skbars[0], 2 * nown * 4);  // chunk 0's copies arrive on it below
+      bulk_g2s(smem + L.alpha, a.alpha_gate + (size_t)e * I + i0, nown * 4, &skbars[0]);
+      bulk_g2s(smem + L.alpha + L.own_max * 4, a.alpha_up + (size_t)e * I + i0, nown * 4, &skbars[0]);
+    }
+    const int c1 = min(nchunk, L.sk_round);
+    for (int ch = 0; ch < c1; ch++) issue_sketch1(a, L, skbuf, skbars, e, i0, i1, ch, ch);
+  }
+  float* alg = reinterpret_cast<float*>(smem + L.alpha);
+  float* alu = alg + L.own_max;
+  if (I % 4 != 0) {  // unaligned scale slices: plain loads, made visible by the barrier below
+    for (int li = tid; li < nown; li += NTHR) {
+      alg[li] = __ldg(a.alpha_gate + (size_t)e * I + i0 + li);
+      alu[li] = __ldg(a.alpha_up + (size_t)e * I + i0 + li);
+    }
+  }
+  int tix[NT];
+  if (FUSED) {
+    // rotate + quantise every token while the sketch is in flight (the fp32
+    // scratch sits past the sketch buffers); its barriers also publish the
+    // scales loaded above
+    float* scratch = reinterpret_cast<float*>(smem + L.ring + NWARP * L.ring_bytes - d * 4);
+#pragma unroll 1
+    for (int t = 0; t < a.B; t++)
+      rotate_quantize(a, reinterpret_cast<const uint16_t*>(smem + L.x) + (size_t)t * d,
+                      reinterpret_cast<int8_t*>(smem + L.q) + (size_t)t * d, scratch,
+                      reinterpret_cast<float*>(misc + MI_CX) + t, reinterpret_cast<float*>(misc + MI_RED), sv_pre);
+  } else {
+    load_tokens(a, L, smem, misc, n, true);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int t = 0; t < NT; t++) tix[t] = misc[MI_TIX + (t < n ? t : 0)];
+  if (DBG) stamp(a, cid, rank, 1);
+
+  float* sa = reinterpret_cast<float*>(smem + L.sa);          // [I, NT] (sigma, ahat) pairs, slices from the owners
+  float* zparts = reinterpret_cast<float*>(smem + L.zparts);  // [cs, NT, r]
+  float* z = reinterpret_cast<float*>(smem + L.z);            // [NT, r]
+  float* apos = reinterpret_cast<float*>(smem + L.apos);      // [NT, I] by union position
+  uint32_t* candm = reinterpret_cast<uint32_t*>(smem + L.candm);
+  uint32_t* keptm = reinterpret_cast<uint32_t*>(smem + L.keptm);  // over union positions
+  int* ulist = reinterpret_cast<int*>(smem + L.ulist);
+  int* dlist = reinterpret_cast<int*>(smem + L.dlist);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.keys);
+  const float* cxs = reinterpret_cast<const float*>(misc + MI_CX);
+
+  // ---------------------------------------------------------- S: screen
+  {
+    const int nv = L.d64;  // 16-byte sketch vectors per row
+    int sq[NT];
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+      const uint4* qv = reinterpret_cast<const uint4*>(smem + L.q + (size_t)tix[t] * d);
+      int s = 0;
+      for (int j = lane; j < L.d8 / 2; j += 32) {
+        const uint4 q4 = qv[j];
+        s = __dp4a((int)q4.x, 0x01010101, s);
+        s = __dp4a((int)q4.y, 0x01010101, s);
+        s = __dp4a((int)q4.z, 0x01010101, s);
+        s = __dp4a((int)q4.w, 0x01010101, s);
+      }
+      sq[t] = warp_sum(s);  // sum of the token's activations: the code offset
+    }
+    const uint16_t* ub = reinterpret_cast<const uint16_t*>(smem + L.ubar);
+    float zacc[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; t++)
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) zacc[t][kk] = 0.0f;
+    bool uv_ready = r == 0;
+    // this lane's activations for sketch vector lane (the row's first 32
+    // vectors), kept in registers across the channels
+    uint4 qr[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; t++) {
+      const uint4* qv = reinterpret_cast<const uint4*>(smem + L.q + (size_t)tix[t] * d);
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) qr[t][kk] = lane < nv ? qv[4 * lane + kk] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // warp w takes channel 16 j + w of every sketch chunk j (one channel per
+    // warp and chunk).  Each channel's dots are reduced over the warp and
+    // parked in the warp's slot of gu; every 4 chunks (and at the end) one
+    // pass over the lanes turns the parked sums into sigma and ahat.
+    int* gu = hist + warp * 4 * NT * 2;  // [4 channels][NT tokens][g, u]; hist is free during the screen
+    int rb = 0, par = 0;  // first chunk of the resident round, parity of its barriers
+#pragma unroll 1
+    for (int j = 0; j < nchunk; j++) {
+      const int li = 16 * j + warp;
+      if (j == rb + L.sk_round) {
+        // the next round of chunks reuses the buffers: every warp is done with them
+        __syncthreads();
+        rb = j;
+        par ^= 1;
+        if (tid == 0) {
+          fence_proxy_async();
+          const int c1 = min(nchunk, j + L.sk_round);
+          for (int ch = j; ch < c1; ch++) issue_sketch1(a, L, skbuf, skbars, e, i0, i1, ch, ch - j);
+        }
+      }
+      int G[NT], U[NT];
+#pragma unroll
+      for (int t = 0; t < NT; t++) G[t] = U[t] = 0;
+      if (li < nown) {
+        const int slot = j - rb;
+        if (!mbar_wait_bounded(&skbars[slot], par, err, a.wait_ns)) misc[MI_DONE] = 1;
+        const uint4* gw = reinterpret_cast<const uint4*>(skbuf + (size_t)slot * 2 * L.skc + warp * (d / 4));
+        const uint4* uw = reinterpret_cast<const uint4*>(skbuf + (size_t)slot * 2 * L.skc + L.skc + warp * (d / 4));
+        int ga[NT][4], ua[NT][4];
+#pragma unroll
+        for (int t = 0; t < NT; t++)
+#pragma unroll
+          for (int kk = 0; kk < 4; kk++) ga[t][kk] = ua[t][kk] = 0;
+#pragma unroll 1
+        for (int vv = lane; vv < nv; vv += 32) {
+          const uint4 g4 = gw[vv], u4 = uw[vv];
+#pragma unroll
+          for (int t = 0; t < NT; t++) {
+            uint4 q0 = qr[t][0], q1 = qr[t][1], q2 = qr[t][2], q3 = qr[t][3];
+            if (vv != lane) {
+              const uint4* qv = reinterpret_cast<const uint4*>(smem + L.q + (size_t)tix[t] * d) + 4 * vv;
+              q0 = qv[0];
+              q1 = qv[1];
+              q2 = qv[2];
+              q3 = qv[3];
+            }
+            code_dot16(g4.x, q0, ga[t]);
+            code_dot16(g4.y, q1, ga[t]);
+            code_dot16(g4.z, q2, ga[t]);
+            code_dot16(g4.w, q3, ga[t]);
+            code_dot16(u4.x, q0, ua[t]);
+            code_dot16(u4.y, q1, ua[t]);
+            code_dot16(u4.z, q2, ua[t]);
+            code_dot16(u4.w, q3, ua[t]);
+          }
+        }
+#pragma unroll
+        for (int t = 0; t < NT; t++) {
+          G[t] = code_dot_total(ga[t]);
+          U[t] = code_dot_total(ua[t]);
+        }
+      }
+      int gs, us;
+      reduce_gu<NT>(G, U, gs, us);
+      if (lane < 16 && (lane & 7) == 0) {
+        const int t = NT == 2 ? lane >> 3 : 0;
+        gu[((j & 3) * NT + t) * 2] = gs;
+        gu[((j & 3) * NT + t) * 2 + 1] = us;
+      }
+      if ((j & 3) == 3 || j == nchunk - 1) {
+        // the batch's epilogue: lane (channel c, token t), c < 4, t < NT
+        __syncwarp();
+        const int jb = j & ~3;
+        const int c = lane / NT, t = lane - c * NT;
+        const int lc = 16 * (jb + c) + warp;
+        const bool valid = lane < 4 * NT && jb + c <= j && lc < nown && t < n;
+        int g2 = 0, u2 = 0;
+        if (lane < 4 * NT) {
+          g2 = gu[lane * 2] - (NT == 2 && t ? sq[NT - 1] : sq[0]);
+          u2 = gu[lane * 2 + 1] - (NT == 2 && t ? sq[NT - 1] : sq[0]);
+        }
+        const float cx = cxs[tix[NT == 2 && t ? NT - 1 : 0]];
+        const float gh = __fmul_rn(__fmul_rn((float)g2, valid ? alg[lc] : 0.0f), cx);
+        const float uh = __fmul_rn(__fmul_rn((float)u2, valid ? alu[lc] : 0.0f), cx);
+        const float ah = __fmul_rn(silu_r(gh), uh);
+        if (valid) {
+          reinterpret_cast<float2*>(sa)[(i0 + lc) * NT + t] = make_float2(fabsf(ah), ah);
+          if (DBG) {
+            const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * I + i0 + lc;
+            if (a.dbg_G) a.dbg_G[off] = g2;
+            if (a.dbg_U) a.dbg_U[off] = u2;
+            if (a.dbg_sigma) a.dbg_sigma[off] = fabsf(ah);
+          }
+        }
+        // partial recovery input z_w = sum over this warp's channels of ahat_i Ubar_i
+        if (r > 0) {
+          if (!uv_ready) {
+            if (!mbar_wait_bounded(uvbar, 0, err, a.wait_ns)) misc[MI_DONE] = 1;
+            uv_ready = true;
+          }
+#pragma unroll
+          for (int cc = 0; cc < 4; cc++) {
+            const int lcc = 16 * (jb + cc) + warp;
+            if (jb + cc <= j && lcc < nown) {
+#pragma unroll
+              for (int tt = 0; tt < NT; tt++) {
+                const float aht = __shfl_sync(kFull, ah, cc * NT + tt);
+#pragma unroll
+                for (int kk = 0; kk < 4; kk++) {
+                  const int p = lane + 32 * kk;
+                  if (p < r && tt < n) zacc[tt][kk] = fmaf(aht, bf16f(ub[lcc * r + p]), zacc[tt][kk]);
+                }
+              }
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+    if (FUSED && warp == NWARP - 1) route_weights(a, L, smem, misc, cid, rank);
+    if (DBG) stamp(a, cid, rank, 5);
+    // z partials of the CTA, pushed to every CTA: zparts[rank][t]
+    if (r > 0) {
+      float* zr = reinterpret_cast<float*>(smem + L.zred);  // [NWARP, NT, r]
+#pragma unroll
+      for (int t = 0; t < NT; t++)
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++) {
+          const int p = lane + 32 * kk;
+          if (p < r) zr[(warp * NT + t) * r + p] = zacc[t][kk];
+        }
+      __syncthreads();
+      for (int tp = tid; tp < NT * r; tp += NTHR) {
+        float zz = 0.0f;
+#pragma unroll
+        for (int w = 0; w < NWARP; w++) zz += zr[w * NT * r + tp];
+        zparts[rank * NT * r + tp] = zz;
+      }
+    }
+    __syncthreads();
+    // push the own (sigma, ahat) slice and z partial to every other CTA: one
+    // 16-byte store per thread and peer, all in flight together
+    {
+      const int nsa4 = cdiv((i1 - i0) * NT * 2, 4), nz4 = r > 0 ? NT * r / 4 : 0, per = nsa4 + nz4;
+      const float4* sa4 = reinterpret_cast<const float4*>(sa + i0 * NT * 2);
+      const float4* z4 = reinterpret_cast<const float4*>(zparts + rank * NT * r);
+#pragma unroll 1
+      for (int w = tid; w < (cs - 1) * per; w += NTHR) {
+        const int pi = idiv(w, per), j = w - pi * per;
+        const int o = pi + (pi >= rank);
+        if (j < nsa4) st_cluster(&sa4[j], o, sa4[j]);
+        else st_cluster(&z4[j - nsa4], o, z4[j - nsa4]);
+      }
+    }
+  }
+  if (DBG) stamp(a, cid, rank, 6);
+  cluster.sync();
+  if (DBG) stamp(a, cid, rank, 7);
+
+  // ---------------------------------------------------------- c: top-c
+#pragma unroll 1
+  for (int t = 0; t < n; t++)
+    block_select_top(reinterpret_cast<const uint32_t*>(sa) + 2 * t, 2 * NT, I, a.c, hist, misc, candm + t * L.words);
+  // union of the candidates, ascending
+  block_mask_to_list(candm, n > 1 ? candm + L.words : nullptr, I, ulist, &misc[MI_NU], hist);
+  const int nU = misc[MI_NU];
+  if (DBG && a.dbg_cand && rank == 0 && warp < n) {
+    const int t = warp;
+    int base = 0;
+    int* out = a.dbg_cand + ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.c;
+    for (int w0 = 0; w0 < I; w0 += 32) {
+      const int p = w0 + lane;
+      const bool on = p < I && ((candm[t * L.words + (w0 >> 5)] >> lane) & 1u);
+      const unsigned bal = __ballot_sync(kFull, on);
+      if (on) out[base + __popc(bal & ((1u << lane) - 1u))] = p;
+      base += __popc(bal);
+    }
+  }
+  if (DBG) stamp(a, cid, rank, 8);
+  // -------------------------------------------- C: exact candidate stage
+  {
+    const int u0 = idiv(rank * nU + cs - 1, cs), u1 = idiv((rank + 1) * nU + cs - 1, cs), nsl = u1 - u0;
+    const int m0 = (warp * nsl) / NWARP, m1 = ((warp + 1) * nsl) / NWARP;
+    const int rowb = d * 2;
+    const int P = max(1, min(kMaxSlots, L.c_slots));
+    const uint4* xs = reinterpret_cast<const uint4*>(smem + L.x);
+    const int vx = L.d8;
+    char* ring = smem + L.ring + warp * L.ring_bytes;
+    uint32_t par = 0;
+    warp_stream(
+        m1 - m0, P, wbars, par, err,
+        [&](int j, int s, uint64_t* bar) {
+          const int i = ulist[u0 + m0 + j];
+          char* dst = ring + s * 2 * rowb;
+          mbar_expect_tx(bar, 2 * rowb);
+          bulk_g2s(dst, a.w_gate + ((size_t)e * I + i) * d, rowb, bar);
+          bulk_g2s(dst + rowb, a.w_up + ((size_t)e * I + i) * d, rowb, bar);
+          if (j + P < m1 - m0) {
+            // the row this slot takes next starts moving into L2 now
+            const int i2 = ulist[u0 + m0 + j + P];
+            bulk_prefetch_l2(a.w_gate + ((size_t)e * I + i2) * d, rowb);
+            bulk_prefetch_l2(a.w_up + ((size_t)e * I + i2) * d, rowb);
+          }
+        },
+        [&](int j, int s) {
+          const int u = u0 + m0 + j, i = ulist[u];
+          const uint4* gr = reinterpret_cast<const uint4*>(ring + s * 2 * rowb);
+          const uint4* ur = gr + vx;
+          float g0[NT], g1[NT], v0[NT], v1[NT];
+#pragma unroll
+          for (int t = 0; t < NT; t++) g0[t] = g1[t] = v0[t] = v1[t] = 0.0f;
+#pragma unroll 2
+          for (int vv = lane; vv < vx; vv += 32) {
+            const uint4 gv = gr[vv], uv = ur[vv];
+#pragma unroll
+            for (int t = 0; t < NT; t++) {
+              const uint4 xv = xs[tix[t] * vx + vv];
+              dot8_mixed(gv, xv, g0[t], g1[t]);
+              dot8_mixed(uv, xv, v0[t], v1[t]);
+            }
+          }
+#pragma unroll
+          for (int t = 0; t < NT; t++) {
+            if (t < n) {
+              const float gs = warp_sum(g0[t] + g1[t]), us = warp_sum(v0[t] + v1[t]);
+              const bool is_c = (candm[t * L.words + (i >> 5)] >> (i & 31)) & 1u;
+              const float av = is_c ? __fmul_rn(silu_r(gs), us) : 0.0f;
+              if (lane == 0) apos[t * I + u] = av;
+            }
+          }
+        },
+        a.wait_ns);
+    // push the own a values to every other CTA, one store per thread and peer
+    __syncthreads();
+    const int per = n * nsl;
+#pragma unroll 1
+    for (int w = tid; w < (cs - 1) * per; w += NTHR) {
+      const int pi = idiv(w, per), j = w - pi * per;
+      const int o = pi + (pi >= rank);
+      const int t = j >= nsl ? 1 : 0, u = u0 + j - t * nsl;
+      st_cluster(&apos[t * I + u], o, apos[t * I + u]);
+    }
+  }
+  if (DBG) stamp(a, cid, rank, 9);
+  cluster.sync();  // the last exchange: no CTA touches another's smem after this
+  if (DBG) stamp(a, cid, rank, 10);
+
+  // ------------------------------------------------------------ k: top-k
+  // over union positions; a token's non-candidates get key 0, its candidates
+  // |a| + 1 (same order, ties still to the lower channel)
+#pragma unroll 1
+  for (int t = 0; t < n; t++) {
+    for (int u = tid; u < nU; u += NTHR) {
+      const int i = ulist[u];
+      const bool c = (candm[t * L.words + (i >> 5)] >> (i & 31)) & 1u;
+      keys[u] = c ? __float_as_uint(fabsf(apos[t * I + u])) + 1u : 0u;
+    }
+    __syncthreads();
+    block_select_top(keys, 1, nU, a.k, hist, misc, keptm + t * L.words);
+    if (DBG && a.dbg_kept && rank == 0 && warp == 0) {
+      const size_t off = ((size_t)misc[MI_TOK + t] * a.top_e + misc[MI_SLOT + t]) * a.k;
+      int base = 0;
+      for (int w0 = 0; w0 < nU; w0 += 32) {
+        const int u = w0 + lane;
+        const bool on = u < nU && ((keptm[t * L.words + (w0 >> 5)] >> lane) & 1u);
+        const unsigned bal = __ballot_sync(kFull, on);
+        const int at = base + __popc(bal & ((1u << lane) - 1u));
+        if (on && at < a.k) {
+          a.dbg_kept[off + at] = ulist[u];
+          if (a.dbg_a_kept) a.dbg_a_kept[off + at] = apos[t * I + u];
+        }
+        base += __popc(bal);
+      }
+    }
+  }
+  // rows of the down stage: union positions kept by any token
+  block_mask_to_list(keptm, n > 1 ? keptm + L.words : nullptr, nU, dlist, &misc[MI_ND], hist);
+  const int nD = misc[MI_ND];
+  if (DBG) stamp(a, cid, rank, 11);
+
+  // ---------------------------------------------- D: down rows + recovery
+  float* red = reinterpret_cast<float*>(smem + L.ring);
+  const int ncq = ncols >> 3, nr8 = r >> 3, nch = ncq + nr8;
+  // Rows: the kept union (recovery from the sketch estimates of every skipped
+  // channel: the factor rows of the kept channels enter with -ahat), or, with
+  // the exact recovery input, the whole candidate union (factor rows of the
+  // candidates enter with -(ahat - a) when dropped, -ahat when kept; down
+  // rows are read for the kept ones only).
+  const bool rec_exact = a.recovery_input == 1;
+  const int rg = down_rows<NT>(
+      a, e, j0, ncq, nr8, rec_exact ? nU : nD, r, [&](int m) { return ulist[rec_exact ? m : dlist[m]]; },
+      [&](int m, int i, bool is_w, float (&co)[NT]) {
+        const int u = rec_exact ? m : dlist[m];
+        bool need = false;
+#pragma unroll
+        for (int t = 0; t < NT; t++) {
+          const bool kept = t < n && ((keptm[t * L.words + (u >> 5)] >> (u & 31)) & 1u);
+          const bool cand = t < n && ((candm[t * L.words + (i >> 5)] >> (i & 31)) & 1u);
+          const float ah = sa[(i * NT + t) * 2 + 1];
+          if (is_w) co[t] = kept ? apos[t * I + u] : 0.0f;
+          else if (kept) co[t] = ah;
+          else co[t] = rec_exact && cand ? __fsub_rn(ah, apos[t * I + u]) : 0.0f;
+          need |= kept || (!is_w && rec_exact && cand);
+        }
+        return need;
+      },
+      red);
+  float* yfin = reinterpret_cast<float*>(smem + L.x);  // [n, cols_max]; x is no longer needed
+#pragma unroll 1
+  for (int o = tid; o < n * nch * 8; o += NTHR) {
+    const int t = o >= nch * 8 ? 1 : 0;
+    const int oc = o - t * nch * 8;
+    const float* rp = red + (size_t)t * nch * 8 + oc;
+    const int gstride = NT * nch * 8;
+    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+    int gg = 0;
+#pragma unroll 1
+    for (; gg + 4 <= rg; gg += 4) {
+      s0 += rp[(gg + 0) * gstride];
+      s1 += rp[(gg + 1) * gstride];
+      s2 += rp[(gg + 2) * gstride];
+      s3 += rp[(gg + 3) * gstride];
+    }
+    for (; gg < rg; gg++) s0 += rp[gg * gstride];
+    const float s = (s0 + s1) + (s2 + s3);
+    if (oc < ncols) {
+      yfin[t * L.cols_max + oc] = s;
+    } else {
+      // z = (sum over the CTAs' partials of all channels) - (the kept part)
+      const int p = oc - ncols;
+      float z0 = 0.0f, z1 = 0.0f;
+      int o = 0;
+#pragma unroll 1
+      for (; o + 2 <= cs; o += 2) {
+        z0 += zparts[(o * NT + t) * r + p];
+        z1 += zparts[((o + 1) * NT + t) * r + p];
+      }
+      if (o < cs) z0 += zparts[(o * NT + t) * r + p];
+      z[t * r + p] = (z0 + z1) - s;
+    }
+  }
+  if (r > 0) {
+    if (!mbar_wait_bounded(uvbar, 0, err, a.wait_ns)) misc[MI_DONE] = 1;
+    __syncthreads();
+    const uint16_t* vo = reinterpret_cast<const uint16_t*>(smem + L.vown);
+#pragma unroll 1
+    for (int t = 0; t < n; t++)
+      for (int col = tid; col < ncols; col += NTHR) {
+        float rec0 = 0.0f, rec1 = 0.0f;
+#pragma unroll 4
+        for (int p = 0; p < r; p += 8) {
+          const uint4 v8 = *reinterpret_cast<const uint4*>(vo + col * r + p);
+          const float4 za = *reinterpret_cast<const float4*>(z + t * r + p);
+          const float4 zb = *reinterpret_cast<const float4*>(z + t * r + p + 4);
+          rec0 = fmaf(bf16lo(v8.x), za.x, rec0);
+          rec1 = fmaf(bf16hi(v8.x), za.y, rec1);
+          rec0 = fmaf(bf16lo(v8.y), za.z, rec0);
+          rec1 = fmaf(bf16hi(v8.y), za.w, rec1);
+          rec0 = fmaf(bf16lo(v8.z), zb.x, rec0);
+          rec1 = fmaf(bf16hi(v8.z), zb.y, rec1);
+          rec0 = fmaf(bf16lo(v8.w), zb.z, rec0);
+          rec1 = fmaf(bf16hi(v8.w), zb.w, rec1);
+        }
+        yfin[t * L.cols_max + col] += rec0 + rec1;
+      }
+  }
+  __syncthreads();
+  if (DBG) stamp(a, cid, rank, 12);
+  write_and_combine(a, rank, j0, ncols, L.cols_max, yfin, misc,
+                    FUSED ? reinterpret_cast<const float*>(misc + MI_RW) : a.ws.wts);
+  if (DBG) {
+    __syncthreads();
+    stamp(a, cid, rank, 15);
+  }
+}
+
 // ================================================================= dense
 template <int NT, bool FUSED>
 __global__ void __launch_bounds__(NTHR, 1) dense_kernel(ExpertArgs a, Layout L) {
@@ -1889,6 +2426,89 @@ cudaError_t plan_reader(const ExpertArgs& a, ReaderPlan* out) {
   return cudaSuccess;
 }
 
+// ----- batch-1 sparse reader (reader1_kernel)
+struct Reader1Plan {
+  int dev, E, I, d, r, top_e, forced;
+  int cs, ring_rows, smem, max_clusters, items;
+  Layout L;
+};
+
+const void* reader1_ptr(bool dbg) {
+  return dbg ? reinterpret_cast<const void*>(&reader1_kernel<true>)
+             : reinterpret_cast<const void*>(&reader1_kernel<false>);
+}
+
+// Cluster size 8..16 by the same estimate as the dense block; ring: the
+// deepest that fits with room for the down stage's partial sums, the
+// rotation scratch and at least one sketch chunk.
+cudaError_t plan_reader1(const ExpertArgs& a, Reader1Plan* out) {
+  thread_local Reader1Plan cache[8];
+  thread_local int ncache = 0, next = 0;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  for (int i = 0; i < ncache; i++) {
+    const Reader1Plan& c = cache[i];
+    if (c.dev == dev && c.E == a.E && c.I == a.I && c.d == a.d && c.r == a.r && c.top_e == a.top_e &&
+        c.forced == a.force_cs) {
+      *out = c;
+      return cudaSuccess;
+    }
+  }
+  int smem_max = 0;
+  err = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (err != cudaSuccess) return err;
+  const void* fns[2] = {reader1_ptr(false), reader1_ptr(true)};
+  for (const void* f : fns) {
+    err = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (err != cudaSuccess) return err;
+  }
+  const int items = a.top_e < a.E ? a.top_e : a.E;
+  Reader1Plan p = {dev, a.E, a.I, a.d, a.r, a.top_e, a.force_cs, 0, 0, 0, 0, items, {}};
+  double best = 1e30;
+  for (int cs = 16; cs >= 8; cs--) {
+    if (a.force_cs && cs != a.force_cs) continue;
+    const int cols_max = 8 * cdiv(a.d / 8, cs);
+    if (cols_max > kMaxCols || a.I < cs || a.E < cs) continue;
+    const int red_need = NTHR * 8 * 4;
+    int rr = 0;
+    for (int t = 2; t <= 64; t++) {
+      const Layout L = make_layout(1, 1, true, a.E, a.I, a.d, a.r, cs, t, false);
+      if (L.total > smem_max) break;
+      if (L.c_slots >= 1 && NWARP * L.ring_bytes >= red_need && L.sk_round >= 1) rr = t;
+    }
+    if (rr < 2) continue;
+    const Layout L = make_layout(1, 1, true, a.E, a.I, a.d, a.r, cs, rr, false);
+    int nclusters = 1 << 30;
+    for (const void* f : fns) {
+      err = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+      if (err != cudaSuccess) return err;
+      const int nc = occupancy_clusters(f, cs, L.total);
+      nclusters = nc < nclusters ? nc : nclusters;
+    }
+    if (nclusters < 1) continue;
+    const double cost = (double)cdiv(items, nclusters) * (1.0 + 8.0 / cs);
+    if (cost < best - 1e-12) {
+      best = cost;
+      p.cs = cs;
+      p.ring_rows = rr;
+      p.smem = L.total;
+      p.max_clusters = nclusters;
+      p.L = L;
+    }
+  }
+  if (p.cs == 0) return cudaErrorInvalidConfiguration;
+  if (ncache < 8) cache[ncache++] = p;
+  else cache[next++ % 8] = p;
+  *out = p;
+  return cudaSuccess;
+}
+
+// The batch-1 kernel takes one-token steps on 2-bit sketch rows, with
+// clusters of 8 to 16 CTAs (a pinned size below 8 runs the channel-owning
+// kernel).
+bool use_reader1(const ExpertArgs& a) { return a.B == 1 && a.sk3 == 0 && (a.force_cs == 0 || a.force_cs >= 8); }
+
 cudaLaunchConfig_t cluster_config(int grid, int cs, int smem, cudaStream_t s, cudaLaunchAttribute (&attr)[2]) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -1914,12 +2534,26 @@ bool reader_supports(int B, int d) { return B <= kMaxGroup && d <= 2048; }
 
 cudaError_t launch_reader(const ExpertArgs& a0, cudaStream_t s) {
   ExpertArgs a = a0;
+  const bool dbg = a.dbg_ids || a.dbg_w || a.dbg_G || a.dbg_U || a.dbg_sigma || a.dbg_cand || a.dbg_kept ||
+                   a.dbg_a_kept || a.dbg_y_expert || a.dbg_phase;
+  if (use_reader1(a)) {
+    Reader1Plan p1;
+    cudaError_t e1 = plan_reader1(a, &p1);
+    if (e1 != cudaSuccess) return e1;
+    a.cs = p1.cs;
+    a.ring_rows = p1.ring_rows;
+    const void* f1 = reader1_ptr(dbg);
+    e1 = cudaFuncSetAttribute(f1, cudaFuncAttributeMaxDynamicSharedMemorySize, p1.smem);
+    if (e1 != cudaSuccess) return e1;
+    cudaLaunchAttribute at1[2];
+    cudaLaunchConfig_t c1 = cluster_config(p1.items * a.cs, a.cs, p1.smem, s, at1);
+    void* args1[] = {&a, &p1.L};
+    return cudaLaunchKernelExC(&c1, f1, args1);
+  }
   ReaderPlan plan;
   cudaError_t err = plan_reader(a, &plan);
   if (err != cudaSuccess) return err;
   a.cs = plan.cs;
-  const bool dbg = a.dbg_ids || a.dbg_w || a.dbg_G || a.dbg_U || a.dbg_sigma || a.dbg_cand || a.dbg_kept ||
-                   a.dbg_a_kept || a.dbg_y_expert || a.dbg_phase;
   const void* fn = reader_ptr(a.B, a.sk3 != 0, dbg);
   err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem);
   if (err != cudaSuccess) return err;
@@ -1955,6 +2589,16 @@ cudaError_t query_plan(const ExpertArgs& a, bool dense, int out[4]) {
     out[1] = p.ring_rows;
     out[2] = p.smem;
     out[3] = p.max_clusters;
+    return cudaSuccess;
+  }
+  if (use_reader1(a)) {
+    Reader1Plan p1;
+    cudaError_t e1 = plan_reader1(a, &p1);
+    if (e1 != cudaSuccess) return e1;
+    out[0] = p1.cs;
+    out[1] = p1.ring_rows;
+    out[2] = p1.smem;
+    out[3] = p1.max_clusters;
     return cudaSuccess;
   }
   ReaderPlan p;
