@@ -421,6 +421,9 @@ def run_native(args, rank, world, local_rank):
         del l3s
 
     fused = B <= 2 and args.path != 2
+    # the one-cluster kernel of the step: the two-exchange kernel at one token
+    # on 2-bit rows, the channel-owning kernel otherwise
+    kname = "reader1_kernel" if B == 1 and args.sketch == "2bit" and args.path != 2 else "reader_kernel"
     # At B <= 2 the reader routes in-kernel: it is the step's only kernel and
     # reads the router too, so a launch's bytes are the step's and its average
     # duration in the back-to-back chunks is the step time.  Above, the
@@ -448,13 +451,13 @@ def run_native(args, rank, world, local_rank):
                          f"({nlay * layer_bytes(layer) / 1e9:.1f} GB)",
                    "parallelism": f"replicas x{world}", "algorithmic_bytes_per_step": mean_bytes,
                    "sketch": args.sketch},
-        "roofline": {"bound": "hbm", "kernel": "reader_kernel" if fused else "streamed kernels (screen .. down)",
+        "roofline": {"bound": "hbm", "kernel": kname if fused else "streamed kernels (screen .. down)",
                      "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json), burst copy",
                      "bytes_per_launch": launch_bytes, "launch_us": launch_ms * 1e3,
                      "isolated_launch_us": kms_max * 1e3,
-                     "traffic": profiled_traffic("reader_kernel", workload_name(B)) if fused else None},
+                     "traffic": profiled_traffic(kname, workload_name(B)) if fused else None},
         "step_roofline_frac": round(value / world / peak, 4),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": B * shape.d * 2,
                 "d2h_bytes_per_step": B * shape.d * 2, "us_per_step": ems * 1e3},
