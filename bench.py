@@ -166,6 +166,10 @@ def run_native(args, rank, world, local_rank):
     # timed steps cycle through them so the working set is far above the L2
     layers = [layer] + [replicate(layer) for _ in range(max(1, args.layers) - 1)]
     nlay = len(layers)
+    # every layer copy's workspace exists before any timing (sized for the
+    # largest batch this run steps), so no allocation lands in a timed region
+    for lay in layers:
+        lay.workspace(max(B, 64))
     ntok = 20
     toks = [synth.tokens(shape.d, B, seed=1000 * rank + s) for s in range(ntok)]
     xs = [t.to(dev) for t in toks]
@@ -499,6 +503,8 @@ def run_ep(args, rank, world, local_rank):
     layer = layer.build_lowrank(r)
     layers = [layer] + [replicate(layer) for _ in range(max(1, args.layers) - 1)]
     nlay = len(layers)
+    for lay in layers:  # no allocation inside the timed region
+        lay.workspace(B)
     toks = [synth.tokens(shape.d, B, seed=s).to(dev) for s in range(20)]
     # bytes of the whole step (all ranks together): the full reader's sets,
     # from this rank's debug outputs of the owned pairs summed over the ranks
@@ -551,11 +557,12 @@ def run_ep(args, rank, world, local_rank):
 
 
 def replicate_view(layer):
-    """A second descriptor of the same device tensors (its own weight dict)."""
+    """A second descriptor of the same device tensors (its own weight dict);
+    it shares the layer's workspace (the two are stepped one after the other
+    on one stream, never concurrently)."""
     import copy
     L = copy.copy(layer)
     L.w = dict(layer.w)
-    L._ws = None
     return L
 
 

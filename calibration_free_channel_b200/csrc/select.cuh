@@ -51,13 +51,19 @@ static __device__ __noinline__ void block_select_top(const uint32_t* keys, int k
     const int shift = pass == 0 ? 21 : pass == 1 ? 10 : 0;
     const int nb = pass == 2 ? 1024 : 2048;
     int* h = hist + (pass & 1) * 2048;
+    // lanes that fall into the same bin add their count once (keys of
+    // similar magnitude share the top bits, and same-address shared atomics
+    // serialise)
 #pragma unroll 1
     for (int base = 0; base < N; base += kSelThreads) {
       const int p = base + tid;
+      int bin = -1;
       if (p < N) {
         const uint32_t k = keys[p * kstride];
-        if ((k & mask) == prefix) atomicAdd(&h[(k >> shift) & (nb - 1)], 1);
+        if ((k & mask) == prefix) bin = (int)((k >> shift) & (uint32_t)(nb - 1));
       }
+      const unsigned grp = __match_any_sync(kSelFull, bin);
+      if (bin >= 0 && lane == __ffs(grp) - 1) atomicAdd(&h[bin], __popc(grp));
     }
     // the other half is zeroed for the next pass (its counts were read before the last barrier)
     if (pass < 2) reinterpret_cast<int4*>(hist + ((pass + 1) & 1) * 2048)[tid] = make_int4(0, 0, 0, 0);

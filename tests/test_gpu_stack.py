@@ -99,11 +99,11 @@ def test_stack_qwen_layer_shape_two_layers_batch1():
 
 
 # ------------------------------------------------------ 48-layer stack (config 4)
-def _oracle_parts(Wh, experts, rot_seed, r):
+def _oracle_parts(Wh, experts, rot_seed, r, lowrank=True):
     """The oracle's sketch and low-rank factors of one layer, built from its
     weights for the given experts only (the rest stay zero and are never
-    read): the sketch rows of those experts, and their rank-r SVD maps,
-    several SVDs at a time."""
+    read): the sketch rows of those experts, and (lowrank) their rank-r SVD
+    maps, several SVDs at a time."""
     from concurrent.futures import ThreadPoolExecutor
     E, I, d = Wh["w_gate"].shape
     experts = sorted(set(int(e) for e in np.ravel(experts)))
@@ -115,6 +115,8 @@ def _oracle_parts(Wh, experts, rot_seed, r):
     sub = O.build_sketch(Wh["w_gate"][experts], Wh["w_up"][experts], rot_seed)
     s[:] = sub[0]
     skg[experts], sku[experts], ag[experts], au[experts] = sub[1], sub[2], sub[3], sub[4]
+    if not lowrank:
+        return (s, skg, sku, ag, au), None
     wd = synth.bf16_bits(Wh["w_down"])
     us = np.zeros((E, I, r), np.uint16)
     vv = np.zeros((E, d, r), np.uint16)
@@ -133,8 +135,12 @@ def test_stack_48_layers_cold_decode():
     the GPU's own sketches and low-rank maps.
       - At batch 1 and batch 16 the first, a middle and the last layer are
         checked against the oracle on the GPU's own layer input (teacher
-        forcing; the oracle builds its sketch and SVD maps from the weights,
-        for the experts it routes to).
+        forcing; the oracle builds its sketch from the weights for the
+        experts it routes to, and reads the layer's low-rank factors as every
+        parity test gives both sides the same factors: two bf16-rounded
+        rank-32 maps from different SVD methods differ enough to move a
+        per-expert output by 2e-2, and the builders have tests of their
+        own).
       - At batch 1 the oracle also runs the first four layers on its own
         activations: the GPU's output stays within 5e-2 relative L2 of it.
         Further on, the two free runs decorrelate on these random weights: a
@@ -163,7 +169,9 @@ def test_stack_48_layers_cold_decode():
             if l in checked:
                 hb = h.cpu()
                 logits, ids, _ = O.route(hb, Wh["w_router"], None, top)
-                sk, lr = _oracle_parts(Wh, ids, synth.rot_seed(0, l), r)
+                sk, _ = _oracle_parts(Wh, ids, synth.rot_seed(0, l), r, lowrank=False)
+                lr = (lay.u_sigma.view(torch.int16).cpu().numpy().view(np.uint16),
+                      lay.v.view(torch.int16).cpu().numpy().view(np.uint16))
                 _, y64, odbg = O.forward(hb, Wh, sk, lr, k=k, c=c, r=r, top_e=top,
                                          residual=synth.bf16_bits(x.cpu()), debug=True)
                 compare_step(Wh, hb, y, dbg, y64, odbg, k, ora_logits=logits)
