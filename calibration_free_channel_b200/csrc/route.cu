@@ -215,18 +215,17 @@ __global__ void __launch_bounds__(512) select_kernel(RouteArgs a) {
   }
   for (int i = threadIdx.x; i < B * kMaxCluster; i += blockDim.x) a.ws.counters[i] = 0u;
   for (int i = threadIdx.x; i < 2 * E; i += blockDim.x) a.ws.arrive[i] = 0u;
+  // tokens per expert, and each expert's token set as a bit mask (emask[e]
+  // holds nwb words): one pass over the (token, slot) entries
+  const int nwb = (B + 31) >> 5;
+  uint32_t* emask = reinterpret_cast<uint32_t*>(aidx + E);  // [E, nwb]
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  for (int i = threadIdx.x; i < E * nwb; i += blockDim.x) emask[i] = 0u;
   __syncthreads();
-  // tokens per expert
-  for (int e = warp; e < E; e += nwarp) {
-    int c = 0;
-    for (int t0 = 0; t0 < B; t0 += 32) {
-      const int t = t0 + lane;
-      bool on = false;
-      if (t < B)
-        for (int s = 0; s < top; s++) on |= sids[t * top + s] == e;
-      c += __popc(__ballot_sync(0xffffffffu, on));
-    }
-    if (lane == 0) cnt[e] = c;
+  for (int i = threadIdx.x; i < B * top; i += blockDim.x) {
+    const int e = sids[i], t = i / top;
+    atomicAdd(&cnt[e], 1);
+    atomicOr(&emask[e * nwb + (t >> 5)], 1u << (t & 31));
   }
   __syncthreads();
   // experts this rank owns (expert parallelism); the pair table holds only theirs
@@ -275,37 +274,27 @@ __global__ void __launch_bounds__(512) select_kernel(RouteArgs a) {
     }
   }
   __syncthreads();
-  // each expert's pairs and work items, tokens ascending
-  for (int e = warp; e < E; e += nwarp) {
-    if (cnt[e] == 0) continue;
-    const bool own = owned(e);
-    int run = 0;
-    for (int t0 = 0; t0 < B; t0 += 32) {
-      const int t = t0 + lane;
-      int slot = -1;
-      if (t < B)
-        for (int s = 0; s < top; s++)
-          if (sids[t * top + s] == e) slot = s;
-      const unsigned bal = __ballot_sync(0xffffffffu, slot >= 0);
-      if (slot >= 0) {
-        const int pos = run + __popc(bal & ((1u << lane) - 1u));
-        if (own) {
-          const int pr = pbase[e] + pos;
-          a.ws.pair_tok[pr] = t;
-          a.ws.pair_slot[pr] = slot;
-          a.ws.pair_ea[pr] = aidx[e];
-        }
-        const int item = ibase[e] + pos / kMaxGroup, g = pos % kMaxGroup;
-        if (item < a.ws.max_items) {
-          a.ws.item_tok[item * kMaxGroup + g] = t;
-          a.ws.item_slot[item * kMaxGroup + g] = slot;
-          if (g == 0) {
-            a.ws.item_e[item] = e;
-            a.ws.item_n[item] = min(kMaxGroup, cnt[e] - pos);
-          }
-        }
+  // each expert's pairs and work items, tokens ascending: entry (t, s) of
+  // expert e sits at the count of e's tokens below t
+  for (int i = threadIdx.x; i < B * top; i += blockDim.x) {
+    const int e = sids[i], t = i / top, slot = i - t * top;
+    const uint32_t* em = emask + e * nwb;
+    int pos = __popc(em[t >> 5] & ((1u << (t & 31)) - 1u));
+    for (int w = 0; w < (t >> 5); w++) pos += __popc(em[w]);
+    if (owned(e)) {
+      const int pr = pbase[e] + pos;
+      a.ws.pair_tok[pr] = t;
+      a.ws.pair_slot[pr] = slot;
+      a.ws.pair_ea[pr] = aidx[e];
+    }
+    const int item = ibase[e] + pos / kMaxGroup, g = pos % kMaxGroup;
+    if (item < a.ws.max_items) {
+      a.ws.item_tok[item * kMaxGroup + g] = t;
+      a.ws.item_slot[item * kMaxGroup + g] = slot;
+      if (g == 0) {
+        a.ws.item_e[item] = e;
+        a.ws.item_n[item] = min(kMaxGroup, cnt[e] - pos);
       }
-      run += __popc(bal);
     }
   }
 }
@@ -402,7 +391,11 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1);
   cfg.blockDim = dim3(512);
-  cfg.dynamicSmemBytes = sizeof(int) * (4 * a.E + a.B * a.top_e);
+  cfg.dynamicSmemBytes = sizeof(int) * (4 * a.E + a.B * a.top_e + a.E * ((a.B + 31) / 32));
+  if (cfg.dynamicSmemBytes > 48 * 1024) {
+    err = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.dynamicSmemBytes);
+    if (err != cudaSuccess) return err;
+  }
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
