@@ -165,6 +165,33 @@ cudaError_t launch_sketch_to_base3(long rows, int d, const uint32_t* codes, uint
   return cudaGetLastError();
 }
 
+namespace {
+__global__ void __launch_bounds__(256) copy16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                     size_t n16) {
+  pdl_trigger();
+  pdl_wait();  // the previous kernel's writes (and reads of dst) are complete
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = src[i];
+}
+}  // namespace
+
+cudaError_t launch_copy16(const void* src, void* dst, size_t bytes, cudaStream_t s) {
+  const size_t n16 = bytes / 16;
+  if (n16 == 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  const size_t blocks = (n16 + 255) / 256;
+  cfg.gridDim = dim3((unsigned)(blocks < 148 ? blocks : 148));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, copy16_kernel, reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst),
+                            n16);
+}
+
 cudaError_t launch_rmsnorm(int B, int d, float eps, const uint16_t* x, uint16_t* h, cudaStream_t s) {
   rmsnorm_kernel<<<B, 256, 0, s>>>(d, eps, x, h);
   return cudaGetLastError();

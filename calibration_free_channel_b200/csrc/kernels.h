@@ -145,5 +145,9 @@ size_t lowrank_ws_bytes(int E, int I, int d, int r);
 cudaError_t launch_build_lowrank(int E, int I, int d, int r, const uint16_t* w_down, uint16_t* u_sigma,
                                  uint16_t* v, void* ws, cudaStream_t s);
 cudaError_t launch_rmsnorm(int B, int d, float eps, const uint16_t* x, uint16_t* h, cudaStream_t s);
+// bytes (a multiple of 16) from src to dst with 16-byte loads and stores on the
+// SMs (either side may be device-addressable host memory); chained to the
+// previous kernel by programmatic dependent launch.
+cudaError_t launch_copy16(const void* src, void* dst, size_t bytes, cudaStream_t s);
 
 }  // namespace moe

@@ -126,16 +126,19 @@ def test_identical_tokens_share_work_items(tiny):
     check_pair(layer, oc, x, k=24, c=48, top_e=2)
 
 
-def test_forward_host_matches_forward(qwen):
+@pytest.mark.parametrize("B,pinned", [(1, True), (1, False), (16, True)])
+def test_forward_host_matches_forward(qwen, B, pinned):
+    """The host-buffer entry equals the device one bit for bit: pinned buffers
+    go through the copy kernels, pageable ones through cudaMemcpyAsync."""
     W, layer, oc = qwen
-    x = synth.tokens(2048, 1, seed=7)
+    x = synth.tokens(2048, B, seed=7)
     y_dev = layer.forward(x.cuda(), k=136, c=272)
-    xh = x.pin_memory()
-    yh = torch.empty_like(xh).pin_memory()
+    xh = x.pin_memory() if pinned else x.clone()
+    yh = torch.empty_like(xh).pin_memory() if pinned else torch.empty_like(xh)
     xd = torch.empty_like(x, device="cuda")
     yd = torch.empty_like(x, device="cuda")
-    ws = layer.workspace(1)
-    M.moe_reader_forward_host(layer.struct(), 1, 136, 272, xh, xd, yd, yh, ws, ws.numel())
+    ws = layer.workspace(B)
+    M.moe_reader_forward_host(layer.struct(), B, 136, 272, xh, xd, yd, yh, ws, ws.numel())
     torch.cuda.synchronize()
     assert torch.equal(yh, y_dev.cpu())
 
