@@ -39,6 +39,14 @@
 // are written for latency: few block barriers per stage, no serial loops over
 // warps, the rotation placed under the sketch's DRAM latency, the screen's
 // byte-wise dots on pre-masked code words.
+//
+// Two kernels implement these steps.  reader1_kernel (one-token steps on
+// 2-bit sketch rows) follows the stages above as written.  reader_kernel
+// (two-token steps, base-3 rows, pinned clusters below 8 CTAs) keeps each
+// CTA's channel slice through the whole step: the selections count ranks
+// over sorted lists the CTAs exchange, and the exact and down rows of the
+// likely channels start before the selections end; it is faster at two
+// tokens and slower at one (see the note above reader1_kernel).
 #include "common.cuh"
 #include "kernels.h"
 #include "rotate.cuh"
