@@ -65,3 +65,20 @@ def test_footprints_of_the_qwen3_layer():
     f3 = accounting.sketch_footprint(768, 2048, "base3")
     assert abs(f2 - 0.0840) < 1e-4 and abs(f3 - 0.0684) < 1e-4
     assert abs(f3 - 0.07) < abs(f2 - 0.07)  # closer to the pages' about 7%
+
+
+def test_multiply_shift_divisions_are_exact():
+    """The GPU decode of a base-3 byte takes floor(b / 3^k) for k = 1..4 as one
+    multiply and shift each on two bytes packed in 16-bit lanes (b * 171 >> 9,
+    b * 57 >> 9, b * 19 >> 9, b * 203 >> 14).  For every byte value a packing
+    can hold (0..242) they are exact, and no product leaves its 16-bit lane."""
+    for b in range(243):
+        assert (b * 171) >> 9 == b // 3
+        assert (b * 57) >> 9 == b // 9
+        assert (b * 19) >> 9 == b // 27
+        assert (b * 203) >> 14 == b // 81
+        assert max(b * 171, b * 57, b * 19, b * 203) < 1 << 16
+        # the digits the decode forms from them are the base-3 digits
+        f = [b, (b * 171) >> 9, (b * 57) >> 9, (b * 19) >> 9, (b * 203) >> 14]
+        digits = [f[k] - 3 * f[k + 1] for k in range(4)] + [f[4]]
+        assert digits == [(b // 3 ** k) % 3 for k in range(5)]

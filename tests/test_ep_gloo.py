@@ -60,3 +60,24 @@ def test_owned_experts_partition():
         flat = sorted(e for p in parts for e in p)
         assert flat == list(range(E))
         assert all(len(p) in (E // world, E // world + 1) for p in parts)
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 8])
+def test_shard_weights_holds_only_owned_experts(world):
+    """ep.shard_weights: the router whole, the experts e % world == rank
+    stacked in order, and the slot map the C layer's expert_slot takes."""
+    W = synth.layer_weights(synth.TINY, seed=0, bias=True)
+    E = W["w_router"].shape[0]
+    seen = []
+    for rank in range(world):
+        Wr, slot = ep.shard_weights(W, rank, world)
+        own = ep.owned_experts(E, rank, world)
+        assert torch.equal(Wr["w_router"], W["w_router"]) and torch.equal(Wr["router_bias"], W["router_bias"])
+        for n in ("w_gate", "w_up", "w_down"):
+            assert Wr[n].shape[0] == len(own)
+            assert torch.equal(Wr[n], W[n][own])
+        assert slot.dtype == torch.int32 and slot.shape == (E,)
+        assert slot[own].tolist() == list(range(len(own)))
+        assert all(int(slot[e]) == -1 for e in range(E) if e not in own)
+        seen += own
+    assert sorted(seen) == list(range(E))
