@@ -77,3 +77,13 @@ def test_top_k_read_budget_is_input_independent():
         _, _, dbg = O.forward(x, W, sk, None, k=24, c=48, r=0, top_e=2, debug=True)
         totals.add(accounting.step_bytes(8, 128, 256, 0, dbg["ids"], dbg["cand"], dbg["kept"])["total"])
     assert len(totals) == 1
+
+
+def test_expert_bytes_with_base3_sketch_rows():
+    # the Qwen layer shape: sketch rows of 416 bytes instead of 512, the rest unchanged
+    two = accounting.expert_bytes(768, 2048, 32, 272, 136)
+    three = accounting.expert_bytes(768, 2048, 32, 272, 136, packing="base3")
+    assert two["sketch"] == 2 * 768 * 512 + 2 * 768 * 4 == 792576
+    assert three["sketch"] == 2 * 768 * 416 + 2 * 768 * 4 == 645120
+    assert two["total"] - three["total"] == two["sketch"] - three["sketch"]
+    assert three["total"] % accounting.SECTOR == 0
